@@ -1,0 +1,139 @@
+"""fp64 CPU oracle for the RTPurbo decode step -- TEST INFRASTRUCTURE.
+
+Only the tests, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline
+leg may import this package.  The product path (the CUDA library and its
+binding) never loads it and shares no code with it.
+
+The arithmetic lives in ``rtp_oracle.c`` (plain C, fp64), which states what
+it computes and which passage of the RTPurbo pages each step follows.  This
+module compiles it with gcc and marshals numpy arrays.
+
+Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
+(brute force, closed forms, invariants and hand-derived fixtures under
+``tests/golden/``); none is "parity unpinned".
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Dict, Optional
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "rtp_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+D, R, BLK = 128, 16, 64
+
+
+def build(force: bool = False) -> str:
+    """Compile rtp_oracle.c into liboracle.so (gcc -O2, OpenMP)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".{os.getpid()}.tmp"
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", _SRC, "-o", tmp, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+_lib = None
+
+
+def _L():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        i32, i64, dbl, vp = ctypes.c_int, ctypes.c_int64, ctypes.c_double, ctypes.c_void_p
+        lib.oracle_rope.argtypes = [vp, i64, dbl, vp]
+        lib.oracle_topp.argtypes = [vp, i64, dbl, vp, vp, vp, vp, vp, vp]
+        lib.oracle_topp.restype = i32
+        lib.oracle_index_scores.argtypes = [i32, i32, i32, i64, vp, i32, vp, vp, vp, i32, i32, i64, vp]
+        lib.oracle_attend.argtypes = [i32, i32, i32, i64, vp, i32, vp, vp, vp, i32, i32, vp, i64, vp]
+        lib.oracle_decode_step.argtypes = [i32, i32, i32, i64, vp, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32,
+                                           i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, i64]
+        lib.oracle_decode_step.restype = i32
+        _lib = lib
+    return _lib
+
+
+def _p(a: Optional[np.ndarray]):
+    if a is None:
+        return None
+    assert a.flags["C_CONTIGUOUS"]
+    return ctypes.c_void_p(a.ctypes.data)
+
+
+def rope(x: np.ndarray, pos: int, theta: float = 1.0e6) -> np.ndarray:
+    x = np.ascontiguousarray(x, dtype=np.float64).reshape(D)
+    y = np.empty(D, dtype=np.float64)
+    _L().oracle_rope(_p(x), int(pos), float(theta), _p(y))
+    return y
+
+
+def topp(s: np.ndarray, p: float) -> Dict[str, object]:
+    """Dynamic Top-P on raw index scores s (temperature 4 = sqrt(16))."""
+    s = np.ascontiguousarray(s, dtype=np.float64)
+    L = s.size
+    order = np.empty(L, dtype=np.int64)
+    k = ctypes.c_int64()
+    zm, Z, cb, ca = (ctypes.c_double() for _ in range(4))
+    rc = _L().oracle_topp(_p(s), L, float(p), _p(order), ctypes.byref(k), ctypes.byref(zm), ctypes.byref(Z),
+                          ctypes.byref(cb), ctypes.byref(ca))
+    if rc != 0:
+        raise ValueError(f"oracle_topp rc={rc}")
+    return {"order": order, "kstar": int(k.value), "kept": np.sort(order[:k.value]), "zmax": zm.value, "Z": Z.value,
+            "cum_before": cb.value, "cum_at": ca.value}
+
+
+def _geom(case):
+    bt = None if case.block_table is None else np.ascontiguousarray(case.block_table, dtype=np.int32)
+    return (case.B, case.Hq, case.Hkv, int(case.Ncap), bt, case.max_blocks_per_seq)
+
+
+def index_scores(case, b: int, h: int) -> np.ndarray:
+    B, Hq, Hkv, Ncap, bt, mbps = _geom(case)
+    L = int(case.seq_lens[b])
+    s = np.empty(L, dtype=np.float64)
+    _L().oracle_index_scores(B, Hq, Hkv, Ncap, _p(bt), mbps, _p(case.q_pre), _p(case.Wq_idx), _p(case.k_idx),
+                             b, h, L, _p(s))
+    return s
+
+
+def attend(case, b: int, h: int, positions: np.ndarray) -> np.ndarray:
+    """Exact softmax attention of (b, h) over an arbitrary position set."""
+    B, Hq, Hkv, Ncap, bt, mbps = _geom(case)
+    pos = np.ascontiguousarray(np.sort(np.asarray(positions, dtype=np.int64)))
+    out = np.empty(D, dtype=np.float64)
+    _L().oracle_attend(B, Hq, Hkv, Ncap, _p(bt), mbps, _p(case.q_rope), _p(case.k_cache), _p(case.v_cache), b, h,
+                       _p(pos), pos.size, _p(out))
+    return out
+
+
+def decode_step(case, nthreads: int = 0) -> Dict[str, np.ndarray]:
+    """The whole decode step in fp64.  Returns out [B,Hq,128] and, per (b,h),
+    kstar, tau, zmax, Z, cum_before, cum_at, next_s and kept_blocks
+    [B,Hq,nblk_cap] (uint8)."""
+    B, Hq, Hkv, Ncap, bt, mbps = _geom(case)
+    BH = B * Hq
+    nblk = (Ncap + BLK - 1) // BLK
+    res = {
+        "out": np.zeros((B, Hq, D), dtype=np.float64),
+        "kstar": np.zeros((B, Hq), dtype=np.int64),
+        "tau": np.full((B, Hq), np.nan),
+        "zmax": np.full((B, Hq), np.nan),
+        "Z": np.full((B, Hq), np.nan),
+        "cum_before": np.full((B, Hq), np.nan),
+        "cum_at": np.full((B, Hq), np.nan),
+        "next_s": np.full((B, Hq), np.nan),
+        "kept_blocks": np.zeros((B, Hq, nblk), dtype=np.uint8),
+    }
+    hk = np.ascontiguousarray(case.head_kind, dtype=np.uint8)
+    rc = _L().oracle_decode_step(B, Hq, Hkv, Ncap, _p(bt), mbps, _p(case.q_pre), _p(case.q_rope), _p(case.k_idx),
+                                 _p(case.k_cache), _p(case.v_cache), _p(case.Wq_idx),
+                                 _p(np.ascontiguousarray(case.seq_lens, dtype=np.int32)), _p(hk),
+                                 _p(np.ascontiguousarray(case.p, dtype=np.float32)), int(case.window), int(case.sink),
+                                 int(nthreads), _p(res["out"]), _p(res["kstar"]), _p(res["tau"]), _p(res["zmax"]),
+                                 _p(res["Z"]), _p(res["cum_before"]), _p(res["cum_at"]), _p(res["next_s"]),
+                                 _p(res["kept_blocks"]), nblk)
+    res["rc"] = rc
+    return res

@@ -1,0 +1,285 @@
+/*
+ * fp64 CPU oracle for the RTPurbo decode step.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path loads this file: it
+ * is called by the tests, by __graft_entry__.smoke() and by the benchmark's
+ * CPU-baseline leg, to check and to time the CUDA path.  It shares no code,
+ * header, table or constant with the CUDA sources.
+ *
+ * What it computes, per sequence b and query head h (sources: "Full
+ * Attention Strikes Back" / RTPurbo -- the paper review on
+ * dongryeollee1.github.io, section Method: "Adaptive sparse attention"
+ * (its equation for s_h(m,n) and S_h(m) = Top-P(s_h(m,.), p)) and
+ * "Hardware-aware top-p decoding kernel" (block mask, cumulative mass
+ * reaching p_top); and the aitrends.kr summary, items 2 "Low-rank Retrieval
+ * Routing" (O_h(m) as a softmax over S_h(m)) and 5 (block-sparse attention)):
+ *
+ *   local head     : attend over P = [0, min(sink,L)) U [max(0,L-window), L)
+ *   retrieval head : q_idx = W^Q_h q^pre                      (16-vector)
+ *                    s_n   = q_idx . k_idx_n,  n < L           (index score)
+ *                    z_n   = s_n / sqrt(16)                    (top-p temperature)
+ *                    pi    = softmax(z)
+ *                    order tokens by (s desc, n asc); k* = smallest k whose
+ *                    prefix mass reaches p (>= p); p >= 1 keeps every token
+ *                    T = first k* tokens; blocks K = { floor(n/64) : n in T }
+ *                    P = union of [64j, min(64j+64, L)) over j in K
+ *   both           : a_n = q_rope . k_n / sqrt(128), w = softmax(a over P),
+ *                    out = sum_n w_n v_n
+ *
+ * Everything is fp64, from the exact upcast of the bf16 inputs, with no
+ * blocking or reordering beyond the definitions above.  A sequence's p is
+ * meant to lie in (0, 1]; p >= 1 keeps every token, p <= 0 or NaN is an
+ * input error.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORC_D 128
+#define ORC_R 16
+#define ORC_BLK 64
+
+static double bf(uint16_t b) {
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return (double)f;
+}
+
+/* cache geometry: contiguous [B,Hkv,Ncap,dim] or paged [pages,Hkv,64,dim] */
+typedef struct {
+    int B, Hq, Hkv;
+    int64_t Ncap;
+    const int32_t* block_table; /* NULL = contiguous */
+    int mbps;                   /* max blocks per sequence (paged) */
+} geom;
+
+static const uint16_t* row(const geom* g, const uint16_t* base, int dim, int b, int kv, int64_t n) {
+    if (!g->block_table) return base + (((int64_t)b * g->Hkv + kv) * g->Ncap + n) * dim;
+    int64_t page = g->block_table[(int64_t)b * g->mbps + n / ORC_BLK];
+    return base + ((page * g->Hkv + kv) * ORC_BLK + n % ORC_BLK) * dim;
+}
+
+/* RoPE, rotate-half pairing (i, i+64), angle pos * theta^(-2i/128): the
+ * relative-position form of the review's "RoPE ... low-dim subspace" insight
+ * (score = sum_i a_i cos(theta_i D) + b_i sin(theta_i D), D = m - n). */
+void oracle_rope(const double* x, int64_t pos, double theta, double* y) {
+    double t[ORC_D];
+    for (int i = 0; i < 64; ++i) {
+        double a = (double)pos * pow(theta, -2.0 * (double)i / 128.0);
+        double c = cos(a), s = sin(a);
+        t[i] = x[i] * c - x[i + 64] * s;
+        t[i + 64] = x[i + 64] * c + x[i] * s;
+    }
+    memcpy(y, t, sizeof t);
+}
+
+typedef struct {
+    double s;
+    int64_t n;
+} scored;
+
+/* (s descending, n ascending): the selection order, ties toward the lower index */
+static int by_score_then_index(const void* a, const void* b) {
+    const scored* x = (const scored*)a;
+    const scored* y = (const scored*)b;
+    if (x->s > y->s) return -1;
+    if (x->s < y->s) return 1;
+    return (x->n < y->n) ? -1 : (x->n > y->n);
+}
+
+/*
+ * Dynamic Top-P over raw index scores s[0..L) (the review's S_h(m) =
+ * Top-P(s_h(m,.), p), temperature sqrt(16)).
+ * Outputs: order[0..L) (selection order), *kstar, and for checks the max of
+ * z = s/4, Z = sum exp(z - zmax), and the cumulative mass of the first k*-1
+ * and first k* tokens.
+ */
+int oracle_topp(const double* s, int64_t L, double p, int64_t* order, int64_t* kstar_out, double* zmax_out,
+                double* Z_out, double* cum_before_out, double* cum_at_out) {
+    if (L <= 0) return 2;
+    if (!(p > 0.0)) return 6;                 /* p <= 0 or NaN */
+    double zmax = -INFINITY;
+    for (int64_t n = 0; n < L; ++n) zmax = fmax(zmax, s[n] / 4.0);
+    double Z = 0.0;
+    for (int64_t n = 0; n < L; ++n) Z += exp(s[n] / 4.0 - zmax);
+    scored* v = (scored*)malloc(sizeof(scored) * (size_t)L);
+    for (int64_t n = 0; n < L; ++n) {
+        v[n].s = s[n];
+        v[n].n = n;
+    }
+    qsort(v, (size_t)L, sizeof(scored), by_score_then_index);
+    int64_t k = L;
+    double cum = 0.0, before = 0.0;
+    if (p < 1.0) {
+        for (int64_t i = 0; i < L; ++i) {
+            before = cum;
+            cum += exp(v[i].s / 4.0 - zmax) / Z;
+            if (cum >= p) {
+                k = i + 1;
+                break;
+            }
+        }
+    } else {
+        for (int64_t i = 0; i < L; ++i) {
+            before = cum;
+            cum += exp(v[i].s / 4.0 - zmax) / Z;
+        }
+    }
+    if (order)
+        for (int64_t i = 0; i < L; ++i) order[i] = v[i].n;
+    free(v);
+    if (kstar_out) *kstar_out = k;
+    if (zmax_out) *zmax_out = zmax;
+    if (Z_out) *Z_out = Z;
+    if (cum_before_out) *cum_before_out = before;
+    if (cum_at_out) *cum_at_out = cum;
+    return 0;
+}
+
+/* index scores s_n = (W^Q_h q^pre) . k_idx_n for n < L (fp64) */
+static void index_scores(const geom* g, const uint16_t* q_pre, const uint16_t* Wq, const uint16_t* k_idx, int b,
+                         int h, int64_t L, double* s) {
+    int G = g->Hq / g->Hkv, kv = h / G;
+    double qi[ORC_R];
+    const uint16_t* q = q_pre + ((int64_t)b * g->Hq + h) * ORC_D;
+    const uint16_t* W = Wq + (int64_t)h * ORC_R * ORC_D;
+    for (int r = 0; r < ORC_R; ++r) {
+        double a = 0.0;
+        for (int d = 0; d < ORC_D; ++d) a += bf(W[r * ORC_D + d]) * bf(q[d]);
+        qi[r] = a;
+    }
+    for (int64_t n = 0; n < L; ++n) {
+        const uint16_t* k = row(g, k_idx, ORC_R, b, kv, n);
+        double a = 0.0;
+        for (int r = 0; r < ORC_R; ++r) a += qi[r] * bf(k[r]);
+        s[n] = a;
+    }
+}
+
+void oracle_index_scores(int B, int Hq, int Hkv, int64_t Ncap, const int32_t* block_table, int mbps,
+                         const uint16_t* q_pre, const uint16_t* Wq, const uint16_t* k_idx, int b, int h, int64_t L,
+                         double* s) {
+    geom g = {B, Hq, Hkv, Ncap, block_table, mbps};
+    index_scores(&g, q_pre, Wq, k_idx, b, h, L, s);
+}
+
+/* exact softmax attention of head h of sequence b over the positions pos[0..npos) */
+static void attend(const geom* g, const uint16_t* q_rope, const uint16_t* k_cache, const uint16_t* v_cache, int b,
+                   int h, const int64_t* pos, int64_t npos, double* out) {
+    int G = g->Hq / g->Hkv, kv = h / G;
+    const uint16_t* q = q_rope + ((int64_t)b * g->Hq + h) * ORC_D;
+    double qd[ORC_D];
+    for (int d = 0; d < ORC_D; ++d) qd[d] = bf(q[d]);
+    double* a = (double*)malloc(sizeof(double) * (size_t)(npos > 0 ? npos : 1));
+    double amax = -INFINITY;
+    for (int64_t i = 0; i < npos; ++i) {
+        const uint16_t* k = row(g, k_cache, ORC_D, b, kv, pos[i]);
+        double t = 0.0;
+        for (int d = 0; d < ORC_D; ++d) t += qd[d] * bf(k[d]);
+        a[i] = t / sqrt((double)ORC_D);
+        amax = fmax(amax, a[i]);
+    }
+    double den = 0.0;
+    for (int64_t i = 0; i < npos; ++i) den += exp(a[i] - amax);
+    for (int d = 0; d < ORC_D; ++d) out[d] = 0.0;
+    for (int64_t i = 0; i < npos; ++i) {
+        double w = exp(a[i] - amax) / den;
+        const uint16_t* v = row(g, v_cache, ORC_D, b, kv, pos[i]);
+        for (int d = 0; d < ORC_D; ++d) out[d] += w * bf(v[d]);
+    }
+    free(a);
+}
+
+void oracle_attend(int B, int Hq, int Hkv, int64_t Ncap, const int32_t* block_table, int mbps,
+                   const uint16_t* q_rope, const uint16_t* k_cache, const uint16_t* v_cache, int b, int h,
+                   const int64_t* pos, int64_t npos, double* out) {
+    geom g = {B, Hq, Hkv, Ncap, block_table, mbps};
+    attend(&g, q_rope, k_cache, v_cache, b, h, pos, npos, out);
+}
+
+/* local head positions: [0, min(sink,L)) U [max(0,L-window), L), each once, ascending */
+static int64_t local_positions(int64_t L, int window, int sink, int64_t* pos) {
+    int64_t k = 0;
+    int64_t s_end = sink < L ? sink : L;
+    int64_t w_lo = L - window > 0 ? L - window : 0;
+    for (int64_t n = 0; n < L; ++n)
+        if (n < s_end || n >= w_lo) pos[k++] = n;
+    return k;
+}
+
+/*
+ * One decode step for every (b, h).  Returns 0, or 6 if some sequence has an
+ * invalid p (its heads are then left untouched).
+ * Optional per-(b,h) outputs (NULL to skip; retrieval heads only, local heads
+ * get kstar = number of attended positions):
+ *   kstar, tau (the k*-th score s), zmax (max z), Z (sum exp(z - zmax)),
+ *   cum_before / cum_at (prefix mass of the first k*-1 / k* tokens),
+ *   next_s (score of token k*+1 in the order, NaN when k* = L),
+ *   kept_blocks [B,Hq,nblk_cap] (1 = block kept).
+ */
+int oracle_decode_step(int B, int Hq, int Hkv, int64_t Ncap, const int32_t* block_table, int mbps,
+                       const uint16_t* q_pre, const uint16_t* q_rope, const uint16_t* k_idx, const uint16_t* k_cache,
+                       const uint16_t* v_cache, const uint16_t* Wq_idx, const int32_t* seq_lens,
+                       const uint8_t* head_kind, const float* p, int window, int sink, int nthreads, double* out,
+                       int64_t* kstar, double* tau, double* zmax, double* Z, double* cum_before, double* cum_at,
+                       double* next_s, uint8_t* kept_blocks, int64_t nblk_cap) {
+    geom g = {B, Hq, Hkv, Ncap, block_table, mbps};
+    int bad = 0;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+    for (int64_t bh = 0; bh < (int64_t)B * Hq; ++bh) {
+        int b = (int)(bh / Hq), h = (int)(bh % Hq);
+        int64_t L = seq_lens[b];
+        double* o = out + bh * ORC_D;
+        int64_t* pos = (int64_t*)malloc(sizeof(int64_t) * (size_t)L);
+        int64_t np = 0;
+        if (!head_kind[h]) {
+            np = local_positions(L, window, sink, pos);
+            if (kstar) kstar[bh] = np;
+        } else {
+            double pb = (double)p[b];
+            if (!(pb > 0.0)) {
+                bad = 1;
+                free(pos);
+                continue;
+            }
+            double* s = (double*)malloc(sizeof(double) * (size_t)L);
+            int64_t* order = (int64_t*)malloc(sizeof(int64_t) * (size_t)L);
+            index_scores(&g, q_pre, Wq_idx, k_idx, b, h, L, s);
+            int64_t k;
+            double zm, Zs, cb, ca;
+            oracle_topp(s, L, pb, order, &k, &zm, &Zs, &cb, &ca);
+            uint8_t* keep = (uint8_t*)calloc((size_t)((L + ORC_BLK - 1) / ORC_BLK), 1);
+            for (int64_t i = 0; i < k; ++i) keep[order[i] / ORC_BLK] = 1;
+            for (int64_t n = 0; n < L; ++n)
+                if (keep[n / ORC_BLK]) pos[np++] = n;
+            if (kstar) kstar[bh] = k;
+            if (tau) tau[bh] = s[order[k - 1]];
+            if (zmax) zmax[bh] = zm;
+            if (Z) Z[bh] = Zs;
+            if (cum_before) cum_before[bh] = cb;
+            if (cum_at) cum_at[bh] = ca;
+            if (next_s) next_s[bh] = (k < L) ? s[order[k]] : NAN;
+            if (kept_blocks) {
+                uint8_t* kb = kept_blocks + bh * nblk_cap;
+                memset(kb, 0, (size_t)nblk_cap);
+                for (int64_t j = 0; j < (L + ORC_BLK - 1) / ORC_BLK && j < nblk_cap; ++j) kb[j] = keep[j];
+            }
+            free(keep);
+            free(order);
+            free(s);
+        }
+        attend(&g, q_rope, k_cache, v_cache, b, h, pos, np, o);
+        free(pos);
+    }
+    return bad ? 6 : 0;
+}

@@ -1,0 +1,379 @@
+"""Pins for the fp64 oracle: brute force, closed forms, invariants and
+hand-derived fixtures (tests/golden/).  CPU only."""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def load(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+# ----------------------------------------------------------------------------
+# a hand-built case: explicit q/k/v, contiguous layout
+# ----------------------------------------------------------------------------
+def hand_case(L, *, Hkv=1, G=1, head_kind=None, p=0.9, window=4, sink=1, seed=0, q_rope=None, k_cache=None,
+              v_cache=None, k_idx=None, q_pre=None, Wq=None):
+    Hq = Hkv * G
+    ncap = ((L + 63) // 64) * 64
+    rng = np.random.default_rng(seed)
+    hk = np.ones(Hq, np.uint8) if head_kind is None else np.asarray(head_kind, np.uint8)
+
+    def bf(x):
+        return synth.to_bf16(np.asarray(x, np.float64))
+
+    kc = synth.nan_fill((1, Hkv, ncap, 128))
+    vc = synth.nan_fill((1, Hkv, ncap, 128))
+    ki = synth.nan_fill((1, Hkv, ncap, 16))
+    kc[:, :, :L] = bf(rng.standard_normal((1, Hkv, L, 128)) if k_cache is None else k_cache)
+    vc[:, :, :L] = bf(rng.standard_normal((1, Hkv, L, 128)) if v_cache is None else v_cache)
+    ki[:, :, :L] = bf(rng.standard_normal((1, Hkv, L, 16)) if k_idx is None else k_idx)
+    qp = bf(rng.standard_normal((1, Hq, 128)) if q_pre is None else q_pre)
+    qr = bf(rng.standard_normal((1, Hq, 128)) if q_rope is None else q_rope)
+    W = bf(rng.standard_normal((Hq, 16, 128)) / math.sqrt(128) if Wq is None else Wq)
+    return synth.Case(name="hand", B=1, Hq=Hq, Hkv=Hkv, Ncap=ncap, seq_lens=np.array([L], np.int32), head_kind=hk,
+                      p=np.array([p], np.float32), window=window, sink=sink, q_pre=qp, q_rope=qr, Wq_idx=W, k_idx=ki,
+                      k_cache=kc, v_cache=vc)
+
+
+# ----------------------------------------------------------------------------
+# Top-P
+# ----------------------------------------------------------------------------
+def brute_force_topp(s, p):
+    """Smallest cardinality of a token set whose softmax(s/4) mass reaches p,
+    and among those sets the one of largest mass, ties to the lexicographically
+    smallest sorted index list -- by enumerating every subset."""
+    n = len(s)
+    w = np.exp(np.asarray(s) / 4.0 - np.max(s) / 4.0)
+    w = w / w.sum()
+    for k in range(1, n + 1):
+        best = None
+        for sub in itertools.combinations(range(n), k):
+            m = sum(w[i] for i in sub)
+            if m >= p - 1e-12:
+                key = (-round(m, 12), sub)
+                if best is None or key < best[0]:
+                    best = (key, sub)
+        if best is not None:
+            return k, list(best[1])
+    return n, list(range(n))
+
+
+@pytest.mark.parametrize("trial", range(60))
+def test_topp_matches_brute_force(trial):
+    rng = np.random.default_rng(1000 + trial)
+    n = int(rng.integers(1, 11))
+    if trial % 3 == 0:
+        s = rng.integers(-3, 4, n).astype(np.float64) * 2.0          # many ties
+    else:
+        s = rng.standard_normal(n) * rng.uniform(0.5, 8.0)
+    w = np.exp(s / 4 - s.max() / 4)
+    w /= w.sum()
+    cums = np.cumsum(np.sort(w)[::-1])
+    while True:
+        p = float(rng.uniform(0.05, 0.999))
+        if np.min(np.abs(cums - p)) > 1e-6:
+            break
+    r = oracle.topp(s, p)
+    k_bf, set_bf = brute_force_topp(s, p)
+    assert r["kstar"] == k_bf
+    assert sorted(r["kept"].tolist()) == set_bf
+
+
+def test_topp_golden():
+    for case in load("topp_hand.json")["cases"]:
+        for chk in case["checks"]:
+            r = oracle.topp(np.array(case["s"]), chk["p"])
+            assert r["kstar"] == chk["kstar"], (case["scores"], chk)
+            assert r["kept"].tolist() == chk["kept"], (case["scores"], chk)
+
+
+@pytest.mark.parametrize("L,p", [(1000, 0.3337), (1000, 0.9001), (777, 0.5555), (64, 0.01)])
+def test_topp_all_equal_closed_form(L, p):
+    r = oracle.topp(np.full(L, 2.5), p)
+    k = math.ceil(p * L)
+    assert r["kstar"] == k
+    assert r["kept"].tolist() == list(range(k))          # ties toward the lower index
+
+
+@pytest.mark.parametrize("a,b,L,p", [(40.0, 0.0, 5000, 0.9), (20.0, 1.0, 3000, 0.8), (30.0, -2.0, 100000, 0.95),
+                                     (8.0, 0.0, 100, 0.5)])
+def test_topp_one_peak_closed_form(a, b, L, p):
+    s = np.full(L, b)
+    pos = L // 3
+    s[pos] = a
+    m1 = math.exp(a / 4) / (math.exp(a / 4) + (L - 1) * math.exp(b / 4))
+    m0 = math.exp(b / 4) / (math.exp(a / 4) + (L - 1) * math.exp(b / 4))
+    k = 1 if m1 >= p else 1 + math.ceil((p - m1) / m0)
+    r = oracle.topp(s, p)
+    assert r["kstar"] == k
+    expect = sorted({pos} | set([i for i in range(L) if i != pos][:k - 1]))
+    assert r["kept"].tolist() == expect
+
+
+def test_topp_p_one_and_invalid():
+    s = np.random.default_rng(3).standard_normal(500)
+    r = oracle.topp(s, 1.0)
+    assert r["kstar"] == 500
+    assert abs(r["cum_at"] - 1.0) < 1e-12                 # softmax mass sums to 1
+    r = oracle.topp(s, 1.5)
+    assert r["kstar"] == 500
+    for bad in (0.0, -0.1, float("nan")):
+        with pytest.raises(ValueError):
+            oracle.topp(s, bad)
+
+
+def test_softmax_normaliser():
+    rng = np.random.default_rng(5)
+    s = rng.standard_normal(10000) * 9
+    r = oracle.topp(s, 1.0)
+    z = s / 4
+    assert abs(r["zmax"] - z.max()) == 0
+    # Z = sum exp(z - zmax): compare against a log-sum-exp computed in sorted order
+    zs = np.sort(z - z.max())
+    assert abs(r["Z"] - math.fsum(np.exp(zs))) < 1e-12 * r["Z"]
+    assert abs(r["cum_at"] - 1.0) < 1e-12
+
+
+# ----------------------------------------------------------------------------
+# RoPE
+# ----------------------------------------------------------------------------
+def test_rope_golden():
+    for c in load("rope_hand.json")["cases"]:
+        x = np.zeros(128)
+        x[c["i"]] = 1.0
+        y = oracle.rope(x, c["pos"])
+        assert abs(y[c["i"]] - c["y_i"]) < 1e-12
+        assert abs(y[c["i"] + 64] - c["y_i64"]) < 1e-12
+        rest = np.delete(y, [c["i"], c["i"] + 64])
+        assert np.all(rest == 0)
+
+
+def test_rope_relative_position_identity():
+    rng = np.random.default_rng(7)
+    for _ in range(20):
+        q, k = rng.standard_normal(128), rng.standard_normal(128)
+        m, n, c = (int(x) for x in rng.integers(0, 1 << 20, 3))
+        lhs = oracle.rope(q, m + c) @ oracle.rope(k, n + c)
+        rhs = oracle.rope(q, m) @ oracle.rope(k, n)
+        assert abs(lhs - rhs) < 1e-9 * (np.abs(q).sum() * np.abs(k).sum() / 10)
+
+
+def test_rope_complex_form_and_norm():
+    rng = np.random.default_rng(8)
+    x = rng.standard_normal(128)
+    pos = 12345
+    theta = 1e6 ** (-np.arange(64) * 2 / 128)
+    zc = (x[:64] + 1j * x[64:]) * np.exp(1j * pos * theta)
+    y = oracle.rope(x, pos)
+    assert np.allclose(y[:64], zc.real, atol=1e-12) and np.allclose(y[64:], zc.imag, atol=1e-12)
+    assert abs(np.linalg.norm(y) - np.linalg.norm(x)) < 1e-12
+    assert np.array_equal(oracle.rope(x, 0), x)
+
+
+def test_generator_rope_matches_oracle_rope():
+    """The workloads' RoPE'd keys and queries are bf16(RoPE(pre-RoPE vector))."""
+    c = synth.workload(1)
+    seed = c.seed
+    pos = np.array([0, 1, 77, 4095])
+    _, _, kpre = synth.keys_for(seed, synth.stream_id("k", 0, 0), pos, None, False, want_kpre=True)
+    for i, n in enumerate(pos):
+        if n in c.needles.get((0, 0), []):
+            continue
+        want = synth.to_bf16(oracle.rope(synth.from_bf16(kpre[i]), int(n)))
+        assert np.array_equal(c.k_cache[0, 0, n], want)
+    for h in range(c.Hq):
+        want = synth.to_bf16(oracle.rope(synth.from_bf16(c.q_pre[0, h]), int(c.seq_lens[0])))
+        assert np.array_equal(c.q_rope[0, h], want)
+
+
+# ----------------------------------------------------------------------------
+# index scores
+# ----------------------------------------------------------------------------
+def test_index_scores_hand():
+    """W^Q picks the odd dims of q^pre (W[r, 2r+1] = 1), q^pre[d] = d, and
+    k_idx row n is the unit vector e_(n mod 16): s_n = 2 (n mod 16) + 1.
+    A transposed W or a swapped q/k index gives different numbers."""
+    L = 40
+    W = np.zeros((1, 16, 128))
+    for r in range(16):
+        W[0, r, 2 * r + 1] = 1.0
+    q = np.arange(128, dtype=np.float64)[None, None, :]
+    ki = np.zeros((1, 1, L, 16))
+    ki[0, 0, np.arange(L), np.arange(L) % 16] = 1.0
+    c = hand_case(L, Wq=W, q_pre=q, k_idx=ki)
+    s = oracle.index_scores(c, 0, 0)
+    assert s.tolist() == [2.0 * (n % 16) + 1.0 for n in range(L)]
+
+
+def test_index_scores_linear_in_query():
+    c = hand_case(300, seed=4)
+    s1 = oracle.index_scores(c, 0, 0)
+    c.q_pre = synth.to_bf16(2.0 * synth.from_bf16(c.q_pre))    # exact doubling in bf16
+    s2 = oracle.index_scores(c, 0, 0)
+    assert np.array_equal(s2, 2.0 * s1)
+
+
+# ----------------------------------------------------------------------------
+# attention
+# ----------------------------------------------------------------------------
+def test_attention_uniform_when_keys_equal():
+    L = 100
+    rng = np.random.default_rng(9)
+    kc = np.repeat(rng.standard_normal((1, 1, 1, 128)), L, axis=2)
+    c = hand_case(L, k_cache=kc, seed=9)
+    pos = np.array([3, 10, 50, 99])
+    out = oracle.attend(c, 0, 0, pos)
+    v = synth.from_bf16(c.v_cache[0, 0, pos])
+    assert np.allclose(out, v.mean(0), atol=1e-12)
+
+
+def test_attention_one_dominant_key():
+    L = 64
+    q = np.zeros((1, 1, 128))
+    q[0, 0, 5] = 8.0
+    kc = np.zeros((1, 1, L, 128))
+    kc[0, 0, 17, 5] = 64.0          # logit 8*64/sqrt(128) = 45.25 vs 0 elsewhere
+    c = hand_case(L, q_rope=q, k_cache=kc, seed=10)
+    out = oracle.attend(c, 0, 0, np.arange(L))
+    v = synth.from_bf16(c.v_cache[0, 0])
+    w17 = 1.0 / (1.0 + (L - 1) * math.exp(-8 * 64 / math.sqrt(128)))
+    want = w17 * v[17] + (1 - w17) / (L - 1) * (v.sum(0) - v[17])
+    assert np.allclose(out, want, atol=1e-12)
+
+
+def test_attention_permutation_invariant_and_weights_sum_to_one():
+    c = hand_case(200, seed=11)
+    pos = np.random.default_rng(11).choice(200, 50, replace=False)
+    a = oracle.attend(c, 0, 0, pos)
+    b = oracle.attend(c, 0, 0, pos[::-1])
+    assert np.allclose(a, b, atol=1e-13)
+    c.v_cache[:] = synth.to_bf16(np.ones(1))                     # every value vector = 1
+    assert np.allclose(oracle.attend(c, 0, 0, pos), 1.0, atol=1e-13)
+
+
+# ----------------------------------------------------------------------------
+# the whole step
+# ----------------------------------------------------------------------------
+def test_local_positions_golden():
+    for cs in load("local_positions_hand.json")["cases"]:
+        L = cs["L"]
+        c = hand_case(L, head_kind=[0], window=cs["window"], sink=cs["sink"], seed=L)
+        r = oracle.decode_step(c)
+        want = oracle.attend(c, 0, 0, np.array(cs["positions"]))
+        assert np.array_equal(r["out"][0, 0], want), cs
+        assert r["kstar"][0, 0] == len(cs["positions"])
+        assert synth.local_positions(L, cs["window"], cs["sink"]).tolist() == cs["positions"]
+
+
+def test_local_head_special_cases():
+    L = 300
+    c = hand_case(L, head_kind=[0], window=1, sink=0, seed=12)
+    r = oracle.decode_step(c)
+    assert np.array_equal(r["out"][0, 0], synth.from_bf16(c.v_cache[0, 0, L - 1]))
+    c = hand_case(L, head_kind=[0], window=L + 5, sink=4, seed=13)
+    r = oracle.decode_step(c)
+    assert np.array_equal(r["out"][0, 0], oracle.attend(c, 0, 0, np.arange(L)))
+
+
+def test_widening_golden():
+    """Hand fixture: kept tokens -> whole blocks.  Realised with integer scores
+    so that exactly the listed tokens are kept (their score 80, all others 0,
+    p chosen below their joint mass)."""
+    for cs in load("widening_hand.json")["cases"]:
+        L = cs["L"]
+        W = np.zeros((1, 16, 128))
+        W[0, 0, 0] = 1.0
+        q = np.zeros((1, 1, 128))
+        q[0, 0, 0] = 8.0
+        ki = np.zeros((1, 1, L, 16))
+        ki[0, 0, cs["kept_tokens"], 0] = 10.0                  # s = 80 vs 0
+        c = hand_case(L, Wq=W, q_pre=q, k_idx=ki, p=0.99, seed=L)
+        r = oracle.decode_step(c)
+        assert r["kstar"][0, 0] == len(cs["kept_tokens"])
+        kept = np.nonzero(r["kept_blocks"][0, 0])[0].tolist()
+        assert kept == cs["blocks"]
+        pos = np.concatenate([np.arange(64 * j, min(64 * j + 64, L)) for j in kept])
+        assert pos.size == cs["positions_count"]
+        assert np.array_equal(r["out"][0, 0], oracle.attend(c, 0, 0, pos))
+
+
+def test_p_one_equals_dense():
+    c = synth.workload(2, scale=16)
+    c.p[:] = 1.0
+    r = oracle.decode_step(c)
+    for h in np.nonzero(c.head_kind)[0]:
+        L = int(c.seq_lens[0])
+        assert r["kstar"][0, h] == L
+        assert np.array_equal(r["out"][0, h], oracle.attend(c, 0, h, np.arange(L)))
+
+
+def test_kept_blocks_are_topp_widened():
+    c = synth.workload(3, scale=32)
+    r = oracle.decode_step(c)
+    for b in range(c.B):
+        for h in np.nonzero(c.head_kind)[0][:3]:
+            t = oracle.topp(oracle.index_scores(c, b, h), float(c.p[b]))
+            blocks = np.unique(t["kept"] // 64)
+            assert np.nonzero(r["kept_blocks"][b, h])[0].tolist() == blocks.tolist()
+            assert r["kstar"][b, h] == t["kstar"]
+
+
+@pytest.mark.parametrize("w", [1, 2])
+def test_needles_always_selected(w):
+    c = synth.workload(w, scale=1 if w == 1 else 4)
+    for (b, h), plist in c.needles.items():
+        t = oracle.topp(oracle.index_scores(c, b, h), float(c.p[b]))
+        assert set(plist) <= set(t["kept"].tolist())
+
+
+def test_needle_regime_keeps_one_token():
+    c = synth.workload(4, scale=64)
+    r = oracle.decode_step(c)
+    for h in np.nonzero(c.head_kind)[0]:
+        assert r["kstar"][0, h] == 1
+        assert r["cum_at"][0, h] >= 0.99
+
+
+def test_paged_layout_equals_contiguous():
+    base = synth.make_case("pg", B=3, Hkv=2, G=2, seq_lens=[700, 64, 1000], ret_groups=[1], p=[0.9, 0.5, 0.95],
+                           window=100, sink=4, seed=21, regimes=["gaussian", "needle", "diffuse"], paged=False)
+    paged = synth.make_case("pg", B=3, Hkv=2, G=2, seq_lens=[700, 64, 1000], ret_groups=[1], p=[0.9, 0.5, 0.95],
+                            window=100, sink=4, seed=21, regimes=["gaussian", "needle", "diffuse"], paged=True)
+    ra, rb = oracle.decode_step(base), oracle.decode_step(paged)
+    assert np.array_equal(ra["out"], rb["out"])
+    assert np.array_equal(ra["kstar"], rb["kstar"])
+
+
+def test_gqa_head_to_group_mapping():
+    """Heads 2..3 read KV head 1: giving KV head 1 the contents of KV head 0
+    makes them equal to heads 0..1 run on the same queries."""
+    c = synth.make_case("gqa", B=1, Hkv=2, G=2, seq_lens=[500], ret_groups=[0, 1], p=[0.9], window=64, sink=4,
+                        seed=22, regimes=["gaussian"])
+    for arr in (c.k_cache, c.v_cache, c.k_idx):
+        arr[:, 1] = arr[:, 0]
+    c.q_pre[:, 2:4] = c.q_pre[:, 0:2]
+    c.q_rope[:, 2:4] = c.q_rope[:, 0:2]
+    c.Wq_idx[2:4] = c.Wq_idx[0:2]
+    r = oracle.decode_step(c)
+    assert np.array_equal(r["out"][0, 2:4], r["out"][0, 0:2])
+    c.v_cache[:, 1] = synth.to_bf16(synth.from_bf16(c.v_cache[:, 1]) + 1.0)
+    r2 = oracle.decode_step(c)
+    assert np.array_equal(r2["out"][0, 0:2], r["out"][0, 0:2])
+    assert not np.allclose(r2["out"][0, 2:4], r["out"][0, 2:4])
+
+
+def test_invalid_p_is_an_error():
+    c = synth.workload(1, scale=4)
+    c.p[:] = 0.0
+    assert oracle.decode_step(c)["rc"] == 6

@@ -1,0 +1,334 @@
+#!/usr/bin/env python
+"""Decode-step benchmark of the RTPurbo sparse attention library on B200.
+
+One step = one rtp_decode_step call over one batch of a synthetic workload
+(index scoring, top-p selection, block lists, retrieval and local attention,
+combine).  Default workload: 1M context (B=1, 8 KV heads x GQA 4, one
+retrieval KV group, 28 local heads, window 4096, sink 4, p=0.9,
+needle-peaked), inputs resident in HBM, L2 flushed (256 MB write) before
+every timed step.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 1..5] [--impl ours|reference]
+
+Multi-GPU: replicas (the step has no cross-GPU exchange); launched by
+torch.distributed.run, one process per GPU; time = max over ranks.
+Prints ONE JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode context-tokens/s (RTPurbo sparse decode step)"
+UNIT = "tokens/s"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", type=int, default=4)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--dense", action="store_true", help="p = 1 for every sequence (dense comparator)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def hbm_peak():
+    try:
+        with open(PEAKS_FILE) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def workload_config(case, wl):
+    import synth
+
+    return {"workload": synth.WORKLOADS[wl], "name": case.name, "batch": int(case.B),
+            "context": [int(x) for x in case.seq_lens][:16], "context_total": int(case.seq_lens.sum()),
+            "q_heads": case.Hq, "kv_heads": case.Hkv, "retrieval_heads": int(case.head_kind.sum()),
+            "window": case.window, "sink": case.sink, "p": sorted(set(float(x) for x in case.p)),
+            "layout": "paged" if case.paged else "contiguous", "l2": "flushed (256 MB write) before every timed step"}
+
+
+def algorithmic_bytes(case, kept):
+    """North-star byte count of one step: index cache of every retrieval KV
+    group + the union of kept K/V blocks per retrieval group (rows < L) +
+    sink/window rows of every local KV group.  512 B per K+V row, 32 B per
+    index row."""
+    import synth
+
+    G = case.G
+    idx = kv = loc = 0
+    for b in range(case.B):
+        L = int(case.seq_lens[b])
+        nblk = (L + 63) // 64
+        rows = np.minimum(64, L - 64 * np.arange(nblk))
+        for g in range(case.Hkv):
+            heads = range(g * G, (g + 1) * G)
+            if any(case.head_kind[h] for h in heads):
+                idx += L * 32
+                uni = np.zeros(nblk, dtype=bool)
+                for h in heads:
+                    if case.head_kind[h]:
+                        uni |= kept[b, h, :nblk].astype(bool)
+                kv += int(rows[uni].sum()) * 512
+            if any(not case.head_kind[h] for h in heads):
+                loc += synth.local_positions(L, case.window, case.sink).size * 512
+    return {"index": idx, "kept_kv": kv, "local": loc, "total": idx + kv + loc}
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = max(mx, float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def run_reference(args, rank):
+    """The oracle (fp64 C, OpenMP over heads) on the host cores, same workload."""
+    if rank != 0:
+        return
+    import oracle
+    import synth
+
+    case = synth.workload(args.workload)
+    if args.dense:
+        case.p[:] = 1.0
+    cores = os.cpu_count() or 1
+    for _ in range(args.warmup):
+        oracle.decode_step(case, nthreads=cores)
+    ts = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle.decode_step(case, nthreads=cores)
+        ts.append(time.perf_counter() - t0)
+    t = statistics.mean(ts)
+    tokens = float(case.seq_lens.sum())
+    v = tokens / t
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(case, args.workload),
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": f"whole decode step of the workload per timed step ({args.steps} steps)"},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    import sparse_attention_decode_rtpurbo_b200 as rtp
+    import synth
+    from synth.torch_io import DeviceCase
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        from datetime import timedelta
+
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    case = synth.workload(args.workload)
+    if args.dense:
+        case.p[:] = 1.0
+    dc = DeviceCase(case, device=dev, debug=True)
+    stream = torch.cuda.current_stream(dev)
+
+    # one debug step: kept blocks for the algorithmic byte count
+    dc.run(stream)
+    res = dc.results()
+    if res["status"] != 0:
+        raise SystemExit(f"device status {res['status']}")
+    nbytes = algorithmic_bytes(case, res["kept"])
+    ret = np.nonzero(case.head_kind)[0]
+    kept_tokens = float(np.mean([res["kstar"][b, h] / case.seq_lens[b] for b in range(case.B) for h in ret])) \
+        if ret.size else 0.0
+    kept_blocks = float(np.mean([res["kept_blocks"][b, h] / ((case.seq_lens[b] + 63) // 64)
+                                 for b in range(case.B) for h in ret])) if ret.size else 0.0
+    import ctypes
+
+    dc.step.dims.debug = ctypes.POINTER(rtp.RtpDebug)()   # timed steps run without diagnostics
+
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    NE = rtp.TIMING_EVENTS
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(NE)] for _ in range(args.steps)]
+    for e in (x for row in evs for x in row):
+        e.record(stream)
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        dc.run(stream)
+    torch.cuda.synchronize(dev)
+
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize(dev)
+    for i in range(args.steps):
+        flush.zero_()
+        dc.step.set_timing_events(evs[i])
+        dc.run(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clocks = sampler.stop()
+    dc.step.set_timing_events(None)
+    step_ms = [evs[i][0].elapsed_time(evs[i][NE - 1]) for i in range(args.steps)]
+    phase_ms = {name: statistics.mean(evs[i][k].elapsed_time(evs[i][k + 1]) for i in range(args.steps))
+                for k, name in enumerate(rtp.PHASES)}
+    t_ms = statistics.mean(step_ms)
+
+    # ---- end to end: host query/len/p -> device, step, output -> host ----
+    hq_pre = torch.from_numpy(case.q_pre.view(np.int16)).view(torch.bfloat16).pin_memory()
+    hq_rope = torch.from_numpy(case.q_rope.view(np.int16)).view(torch.bfloat16).pin_memory()
+    hlens = torch.from_numpy(case.seq_lens.astype(np.int32)).pin_memory()
+    hp = torch.from_numpy(case.p.astype(np.float32)).pin_memory()
+    hout = torch.empty(dc.out.shape, dtype=torch.bfloat16).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (hq_pre, hq_rope, hlens, hp))
+    d2h = hout.numel() * hout.element_size()
+    e2e_ms = []
+    for i in range(max(3, args.warmup) + args.steps):
+        flush.zero_()
+        a = torch.cuda.Event(enable_timing=True)
+        z = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        dc.q_pre.copy_(hq_pre, non_blocking=True)
+        dc.q_rope.copy_(hq_rope, non_blocking=True)
+        dc.seq_lens.copy_(hlens, non_blocking=True)
+        dc.p.copy_(hp, non_blocking=True)
+        dc.run(stream)
+        hout.copy_(dc.out, non_blocking=True)
+        z.record(stream)
+        z.synchronize()
+        if i >= max(3, args.warmup):
+            e2e_ms.append(a.elapsed_time(z))
+    e2e_t = statistics.mean(e2e_ms)
+
+    # ---- max over ranks ----
+    vals = torch.tensor([t_ms, e2e_t] + [phase_ms[n] for n in rtp.PHASES], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+    t_ms, e2e_t = float(vals[0]), float(vals[1])
+    phase_ms = {n: float(vals[2 + k]) for k, n in enumerate(rtp.PHASES)}
+
+    tokens = float(case.seq_lens.sum())
+    value = world * tokens / (t_ms * 1e-3)
+    peak, peak_kind = hbm_peak()
+    phase_bytes = {"local": nbytes["local"], "score": nbytes["index"], "retrieval": nbytes["kept_kv"]}
+    dom = max(phase_bytes, key=lambda n: phase_ms[n])
+    ach = phase_bytes[dom] / (phase_ms[dom] * 1e-3) / 1e9
+    step_gbs = nbytes["total"] / (t_ms * 1e-3) / 1e9
+    launches_per_step = (1 if any(not h for h in case.head_kind) else 0) + (8 if ret.size else 0)
+
+    line = None
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            import oracle
+
+            cores = os.cpu_count() or 1
+            oracle.decode_step(case, nthreads=cores)
+            reps, t0 = 0, time.perf_counter()
+            while time.perf_counter() - t0 < 10.0 and reps < 50:
+                oracle.decode_step(case, nthreads=cores)
+                reps += 1
+            tc = (time.perf_counter() - t0) / reps
+            cpu = {"value": tokens / tc, "unit": UNIT, "cores": cores, "kind": "oracle",
+                   "sample": f"{reps} whole decode steps of this workload (fp64 C oracle, OpenMP over heads)"}
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": t_ms, "us_per_step": t_ms * 1e3,
+            "us_per_step_p10_p90": [float(np.percentile(step_ms, 10)) * 1e3, float(np.percentile(step_ms, 90)) * 1e3],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16 in, fp32 accumulate",
+            "data": "synthetic (seeded; see DESIGN.md input recipe)",
+            "config": dict(workload_config(case, args.workload), parallelism=f"replicas x{world}",
+                           dense_p1=bool(args.dense)),
+            "roofline": {"bound": "hbm", "kernel": dom, "achieved": ach, "peak": peak, "unit": "GB/s",
+                         "frac": ach / peak, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)",
+                         "traffic": None, "algorithmic_bytes_per_launch": phase_bytes[dom]},
+            "step_roofline": {"algorithmic_bytes": nbytes, "achieved": step_gbs, "peak": peak, "unit": "GB/s",
+                              "frac": step_gbs / peak},
+            "phases_us": {n: phase_ms[n] * 1e3 for n in rtp.PHASES},
+            "sparsity": {"kept_token_frac": kept_tokens, "kept_block_frac": kept_blocks},
+            "e2e": {"value": world * tokens / (e2e_t * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "us_per_step": e2e_t * 1e3},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clocks,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,165 @@
+/*
+ * rtp_decode.h -- C ABI of the RTPurbo decode-step sparse attention library
+ * (librtp.so, CUDA, sm_100a).
+ *
+ * The operation (sources: "Full Attention Strikes Back" / RTPurbo -- the
+ * paper review on dongryeollee1.github.io, section Method: "Adaptive sparse
+ * attention" (s_h(m,n) = (W^Q_h q^pre_m)^T (W^K_h k^pre_n),
+ * S_h(m) = Top-P(s_h(m,.), p)) and "Hardware-aware top-p decoding kernel"
+ * (histogram threshold where the cumulative mass reaches p_top, block mask,
+ * block-sparse decode); the aitrends.kr summary, items 2 and 5 (softmax
+ * attention over S_h(m); block-sparse attention with a cross-split reduce)):
+ *
+ * For every sequence b and query head h of one decode step:
+ *   local head (head_kind[h] == 0): exact softmax attention of q_rope[b,h]
+ *     over cache positions [0, min(sink,L)) U [max(0, L-window), L);
+ *   retrieval head (head_kind[h] == 1):
+ *     q_idx = Wq_idx[h] . q_pre[b,h] (16 values, fp32),
+ *     s_n   = q_idx . k_idx[b, kv(h), n] for every cached n < L,
+ *     keep the smallest set of tokens whose softmax(s/4) mass reaches p[b],
+ *     taking tokens in order of decreasing s, equal scores toward the lower
+ *     index; p[b] >= 1 keeps every token;
+ *     widen the kept tokens to whole 64-token blocks [64j, 64j+64) n [0, L);
+ *     exact softmax attention of q_rope[b,h] over those positions.
+ *   Attention logits are q.k / sqrt(128); kv(h) = h / (Hq / Hkv) (GQA).
+ *
+ * Conventions
+ *   - Every tensor pointer is DEVICE memory owned by the caller unless marked
+ *     host.  bf16 tensors are passed as uint16_t bit patterns.  Strides are
+ *     the dense row-major strides of the stated shapes.
+ *   - The library allocates no memory.  Scratch lives in a caller-allocated
+ *     device workspace of rtp_workspace_size() bytes.  Zero-fill it once
+ *     after allocation (cudaMemset); every call leaves it ready for the next.
+ *   - Work is enqueued on `stream` (a cudaStream_t); nothing synchronises the
+ *     host.  Calls that share a workspace must be ordered on the GPU.
+ *   - Errors the host can see (null pointers, unsupported sizes, a small
+ *     workspace) return a status and enqueue nothing.  Errors only the device
+ *     can see (a seq_len outside [1, capacity], p <= 0 or NaN, a page id
+ *     outside [0, num_pages), a wait that timed out) set a status word in the
+ *     workspace, the affected sequence's outputs are not written (bad seq_len,
+ *     bad p) or unspecified (bad page id, timeout), and rtp_get_status()
+ *     reports it.
+ *   - No C++ exception crosses this interface.
+ */
+#ifndef RTP_DECODE_H
+#define RTP_DECODE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum rtp_status {
+    RTP_OK = 0,
+    RTP_ERR_NULL = 1,          /* a required pointer is NULL */
+    RTP_ERR_SHAPE = 2,         /* inconsistent sizes (e.g. Hq % Hkv != 0, capacity not a multiple of 64) */
+    RTP_ERR_UNSUPPORTED = 3,   /* head_dim != 128, idx_dim != 16, block_size != 64, GQA group > 8, ... */
+    RTP_ERR_WORKSPACE = 4,     /* workspace missing or smaller than rtp_workspace_size() */
+    RTP_ERR_CUDA = 5,          /* a CUDA launch or query failed */
+    RTP_ERR_DEVICE_INPUT = 6,  /* device-side: bad seq_len, p or page id (see rtp_get_status) */
+    RTP_ERR_TIMEOUT = 7        /* device-side: a bounded wait inside a kernel gave up */
+} rtp_status;
+
+/*
+ * Optional diagnostic outputs (device pointers; any may be NULL).  Entries are
+ * indexed by b * num_q_heads + h and written for retrieval heads only.
+ */
+typedef struct rtp_debug {
+    float* tau;              /* [B*Hq] the k*-th kept score s (fp32) */
+    int32_t* kstar;          /* [B*Hq] number of kept tokens k* */
+    int32_t* kept_blocks;    /* [B*Hq] number of kept 64-token blocks */
+    float* smax;             /* [B*Hq] largest index score s */
+    double* Z;               /* [B*Hq] sum over n < L of exp((s_n - smax)/4) */
+    uint32_t* block_bitmap;  /* [B*Hq*words], words = ceil(ceil(capacity/64)/32); bit j%32 of word j/32 = block j kept */
+} rtp_debug;
+
+/*
+ * Sizes and layout of one call.
+ *   batch, num_q_heads (Hq), num_kv_heads (Hkv): Hq % Hkv == 0, Hq/Hkv <= 8.
+ *   head_dim must be 128, idx_dim 16, block_size 64.
+ *   max_seq_len: per-sequence capacity in tokens, a multiple of 64.
+ *     Contiguous layout: caches are [batch, Hkv, max_seq_len, dim].
+ *     Paged layout (block_table != NULL): caches are [num_pages, Hkv, 64, dim]
+ *     and max_seq_len must equal max_blocks_per_seq * 64.
+ *   block_table: device int32 [batch, max_blocks_per_seq], page id of each
+ *     64-token block of each sequence, or NULL for the contiguous layout.
+ *   workspace / workspace_bytes: caller-allocated device scratch.
+ *   debug: host pointer to an rtp_debug of device pointers, or NULL.
+ *   timing_events / n_timing_events: optional host array of cudaEvent_t
+ *     handles (created by the caller).  When n_timing_events >=
+ *     RTP_TIMING_EVENTS the call records event i on `stream` at boundary i of
+ *     the kernel sequence (see RTP_PHASE_*), so phase i lasts from event i to
+ *     event i+1.  Phases with nothing to do still record their events.
+ */
+enum {
+    RTP_PHASE_LOCAL = 0,      /* local heads: sink + window attention and combine */
+    RTP_PHASE_SCORE = 1,      /* index scores + per-group selection decision */
+    RTP_PHASE_SELECT = 2,     /* exact top-p radix passes (heads that need them) */
+    RTP_PHASE_MARK = 3,       /* block masks */
+    RTP_PHASE_BLOCKLIST = 4,  /* per-KV-group union block lists */
+    RTP_PHASE_RETRIEVAL = 5,  /* retrieval heads: block-sparse attention and combine */
+    RTP_TIMING_EVENTS = 7
+};
+
+typedef struct rtp_dims {
+    int32_t batch, num_q_heads, num_kv_heads;
+    int32_t head_dim, idx_dim, block_size;
+    int32_t max_seq_len;
+    const int32_t* block_table;
+    int32_t max_blocks_per_seq, num_pages;
+    void* workspace;
+    size_t workspace_bytes;
+    const rtp_debug* debug;
+    void* const* timing_events;
+    int32_t n_timing_events;
+} rtp_dims;
+
+/*
+ * Bytes of device workspace rtp_decode_step needs for these sizes and this
+ * head split (head_kind is a HOST array of num_q_heads bytes, 1 = retrieval,
+ * 0 = local).  Returns 0 if the sizes are invalid or unsupported.
+ */
+size_t rtp_workspace_size(const rtp_dims* dims, const uint8_t* head_kind);
+
+/*
+ * One decode step (see the top of this file).
+ *   q_pre     [B, Hq, 128]  bf16  pre-RoPE query (indexer input)
+ *   q_rope    [B, Hq, 128]  bf16  RoPE'd query (attention input)
+ *   k_idx     [B, Hkv, cap, 16] or paged [pages, Hkv, 64, 16]   bf16 index keys W^K k^pre
+ *   k_cache   [B, Hkv, cap, 128] or paged [pages, Hkv, 64, 128] bf16 RoPE'd keys
+ *   v_cache   same layout as k_cache, bf16 values
+ *   Wq_idx    [Hq, 16, 128] bf16 indexer query projections (rows of local heads unused)
+ *   seq_lens  [B] int32, 1 <= L <= cap (device)
+ *   head_kind [Hq] uint8, HOST memory: 1 = retrieval head, 0 = local head
+ *   p         [B] fp32 top-p mass per sequence, in (0, 1]; >= 1 keeps all tokens (device)
+ *   window, sink: local heads' sliding window and sink sizes, >= 0, window + sink >= 1
+ *   out       [B, Hq, 128] bf16 (round to nearest even)
+ *   stream    cudaStream_t to enqueue on (NULL = legacy default stream)
+ * Rows no head may read (rows >= L; for KV heads without retrieval heads,
+ * rows outside the sink and window) never enter the arithmetic, whatever they
+ * hold (NaN included).  They may still be copied into shared memory as part
+ * of a 64-row tile that also holds readable rows, so the whole capacity
+ * (contiguous) or whole pages (paged) must be allocated.
+ */
+rtp_status rtp_decode_step(const rtp_dims* dims, const uint16_t* q_pre, const uint16_t* q_rope,
+                           const uint16_t* k_idx, const uint16_t* k_cache, const uint16_t* v_cache,
+                           const uint16_t* Wq_idx, const int32_t* seq_lens, const uint8_t* head_kind,
+                           const float* p, int32_t window, int32_t sink, uint16_t* out, void* stream);
+
+/*
+ * Synchronises `stream`, returns the first device-side error recorded in the
+ * workspace since the last call to this function (RTP_OK if none) and clears
+ * it.  For tests and debugging; it blocks the host.
+ */
+rtp_status rtp_get_status(const rtp_dims* dims, void* stream);
+
+/* Static string naming a status code. */
+const char* rtp_status_string(rtp_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RTP_DECODE_H */

@@ -1,0 +1,162 @@
+"""RTPurbo decode-step sparse attention on B200 (sm_100a).
+
+Thin ctypes binding of ``librtp.so`` (C ABI declared in
+``include/rtp_decode.h``).  This module only marshals arguments: every step of
+the decode path runs in the library's CUDA kernels.  PyTorch supplies device
+memory and streams.  There is no CPU fallback: if the library cannot be
+loaded, importing this package raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+from .build import LIB as _LIB_PATH
+
+__all__ = ["RTP_OK", "RtpError", "RtpDims", "RtpDebug", "lib", "status_string", "workspace_size", "decode_step",
+           "get_status", "Step", "PHASES", "TIMING_EVENTS"]
+
+RTP_OK = 0
+_STATUS_NAMES = {0: "RTP_OK", 1: "RTP_ERR_NULL", 2: "RTP_ERR_SHAPE", 3: "RTP_ERR_UNSUPPORTED", 4: "RTP_ERR_WORKSPACE",
+                 5: "RTP_ERR_CUDA", 6: "RTP_ERR_DEVICE_INPUT", 7: "RTP_ERR_TIMEOUT"}
+
+
+class RtpError(RuntimeError):
+    def __init__(self, code: int, what: str = ""):
+        self.code = code
+        super().__init__(f"{_STATUS_NAMES.get(code, code)}: {status_string(code)}{' (' + what + ')' if what else ''}")
+
+
+class RtpDebug(ctypes.Structure):
+    _fields_ = [("tau", ctypes.c_void_p), ("kstar", ctypes.c_void_p), ("kept_blocks", ctypes.c_void_p),
+                ("smax", ctypes.c_void_p), ("Z", ctypes.c_void_p), ("block_bitmap", ctypes.c_void_p)]
+
+
+class RtpDims(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("num_q_heads", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("idx_dim", ctypes.c_int32), ("block_size", ctypes.c_int32),
+                ("max_seq_len", ctypes.c_int32), ("block_table", ctypes.c_void_p),
+                ("max_blocks_per_seq", ctypes.c_int32), ("num_pages", ctypes.c_int32),
+                ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+                ("debug", ctypes.POINTER(RtpDebug)), ("timing_events", ctypes.c_void_p),
+                ("n_timing_events", ctypes.c_int32)]
+
+
+PHASES = ["local", "score", "select", "mark", "blocklist", "retrieval"]
+TIMING_EVENTS = len(PHASES) + 1
+
+
+def _load():
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(f"librtp.so not built ({_LIB_PATH}); run `python -m sparse_attention_decode_rtpurbo_b200.build`")
+    L = ctypes.CDLL(_LIB_PATH)
+    vp, i32 = ctypes.c_void_p, ctypes.c_int32
+    L.rtp_workspace_size.argtypes = [ctypes.POINTER(RtpDims), vp]
+    L.rtp_workspace_size.restype = ctypes.c_size_t
+    L.rtp_decode_step.argtypes = [ctypes.POINTER(RtpDims), vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, vp, vp]
+    L.rtp_decode_step.restype = ctypes.c_int
+    L.rtp_get_status.argtypes = [ctypes.POINTER(RtpDims), vp]
+    L.rtp_get_status.restype = ctypes.c_int
+    L.rtp_status_string.argtypes = [ctypes.c_int]
+    L.rtp_status_string.restype = ctypes.c_char_p
+    return L
+
+
+lib = _load()
+
+
+def status_string(code: int) -> str:
+    return lib.rtp_status_string(int(code)).decode()
+
+
+def _ptr(x) -> Optional[int]:
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def make_dims(batch: int, num_q_heads: int, num_kv_heads: int, max_seq_len: int, *, block_table=None,
+              max_blocks_per_seq: int = 0, num_pages: int = 0, workspace=None, workspace_bytes: int = 0,
+              debug: Optional[RtpDebug] = None) -> RtpDims:
+    d = RtpDims(batch, num_q_heads, num_kv_heads, 128, 16, 64, max_seq_len, _ptr(block_table), max_blocks_per_seq,
+                num_pages, _ptr(workspace), workspace_bytes, None)
+    if debug is not None:
+        d.debug = ctypes.pointer(debug)
+    return d
+
+
+def _head_kind_buf(head_kind) -> ctypes.Array:
+    hk = bytes(int(x) for x in head_kind)
+    return (ctypes.c_uint8 * len(hk)).from_buffer_copy(hk)
+
+
+def workspace_size(dims: RtpDims, head_kind) -> int:
+    return int(lib.rtp_workspace_size(ctypes.byref(dims), _head_kind_buf(head_kind)))
+
+
+def decode_step(dims: RtpDims, q_pre, q_rope, k_idx, k_cache, v_cache, Wq_idx, seq_lens, head_kind, p,
+                window: int, sink: int, out, stream=None) -> None:
+    """rtp_decode_step: tensors are device tensors (bf16 / int32 / fp32), or
+    raw device pointers as ints; head_kind is a host sequence of 0/1."""
+    st = 0 if stream is None else (stream if isinstance(stream, int) else stream.cuda_stream)
+    rc = lib.rtp_decode_step(ctypes.byref(dims), _ptr(q_pre), _ptr(q_rope), _ptr(k_idx), _ptr(k_cache),
+                             _ptr(v_cache), _ptr(Wq_idx), _ptr(seq_lens), _head_kind_buf(head_kind), _ptr(p),
+                             int(window), int(sink), _ptr(out), st)
+    if rc != RTP_OK:
+        raise RtpError(rc, "rtp_decode_step")
+
+
+def get_status(dims: RtpDims, stream=None) -> int:
+    st = 0 if stream is None else (stream if isinstance(stream, int) else stream.cuda_stream)
+    return int(lib.rtp_get_status(ctypes.byref(dims), st))
+
+
+class Step:
+    """Convenience holder for one layer's decode-step configuration: owns the
+    workspace (a torch uint8 device tensor, zero-filled once) and the dims."""
+
+    def __init__(self, batch: int, num_q_heads: int, num_kv_heads: int, max_seq_len: int, head_kind, *,
+                 block_table=None, num_pages: int = 0, device="cuda", debug: Optional[RtpDebug] = None):
+        import torch
+
+        self.head_kind = [int(x) for x in head_kind]
+        mbps = 0 if block_table is None else int(block_table.shape[1])
+        self.block_table = block_table
+        probe = make_dims(batch, num_q_heads, num_kv_heads, max_seq_len, block_table=block_table,
+                          max_blocks_per_seq=mbps, num_pages=num_pages)
+        nbytes = workspace_size(probe, self.head_kind)
+        if nbytes == 0:
+            raise RtpError(2, "rtp_workspace_size returned 0 (invalid or unsupported sizes)")
+        self.workspace = torch.zeros(nbytes, dtype=torch.uint8, device=device)
+        self.debug = debug
+        self.dims = make_dims(batch, num_q_heads, num_kv_heads, max_seq_len, block_table=block_table,
+                              max_blocks_per_seq=mbps, num_pages=num_pages, workspace=self.workspace,
+                              workspace_bytes=nbytes, debug=debug)
+
+    def __call__(self, q_pre, q_rope, k_idx, k_cache, v_cache, Wq_idx, seq_lens, p, window, sink, out, stream=None):
+        decode_step(self.dims, q_pre, q_rope, k_idx, k_cache, v_cache, Wq_idx, seq_lens, self.head_kind, p, window,
+                    sink, out, stream)
+
+    def status(self, stream=None) -> int:
+        return get_status(self.dims, stream)
+
+    def set_timing_events(self, events) -> None:
+        """Record the given torch.cuda.Event objects (TIMING_EVENTS of them,
+        created with enable_timing=True) at the phase boundaries of every
+        following call; None switches it off."""
+        if events is None:
+            self._ev_arr = None
+            self.dims.timing_events = None
+            self.dims.n_timing_events = 0
+            return
+        assert len(events) >= TIMING_EVENTS
+        for e in events:
+            if not e.cuda_event:
+                e.record()      # materialise the underlying cudaEvent_t
+        torch_handles = [e.cuda_event for e in events]
+        self._ev_arr = (ctypes.c_void_p * len(torch_handles))(*torch_handles)
+        self.dims.timing_events = ctypes.cast(self._ev_arr, ctypes.c_void_p)
+        self.dims.n_timing_events = len(torch_handles)

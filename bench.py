@@ -41,6 +41,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", type=int, default=4)
+    ap.add_argument("--scale", type=int, default=1, help="divide the workload's context lengths (profiling runs)")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--dense", action="store_true", help="p = 1 for every sequence (dense comparator)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -146,7 +147,7 @@ def run_reference(args, rank):
     import oracle
     import synth
 
-    case = synth.workload(args.workload)
+    case = synth.workload(args.workload, scale=args.scale)
     if args.dense:
         case.p[:] = 1.0
     cores = os.cpu_count() or 1
@@ -197,7 +198,7 @@ def main():
         if world > 1:
             dist.barrier()
 
-    case = synth.workload(args.workload)
+    case = synth.workload(args.workload, scale=args.scale)
     if args.dense:
         case.p[:] = 1.0
     dc = DeviceCase(case, device=dev, debug=True)
@@ -218,14 +219,30 @@ def main():
 
     dc.step.dims.debug = ctypes.POINTER(rtp.RtpDebug)()   # timed steps run without diagnostics
 
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    # L2 flush between timed steps: write 256 MB, then read another 256 MB so
+    # the dirty lines of the write are evicted before the step, not during it
+    flush_w = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush_r = torch.ones(256 << 20, dtype=torch.uint8, device=dev)
+
+    def flush():
+        flush_w.zero_()
+        flush_r.sum(dtype=torch.int64)
+
+    # one step = one replay of a CUDA graph holding the rtp_decode_step launches
     NE = rtp.TIMING_EVENTS
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(NE)] for _ in range(args.steps)]
-    for e in (x for row in evs for x in row):
+    inner = [torch.cuda.Event(enable_timing=True) for _ in range(NE)]
+    for e in inner:
         e.record(stream)
+    dc.run(stream)                               # eager warm-up (sets kernel attributes)
+    torch.cuda.synchronize(dev)
+    dc.step.set_timing_events(inner)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        dc.run(torch.cuda.current_stream(dev))
+    dc.step.set_timing_events(None)
     for _ in range(max(3, args.warmup)):
-        flush.zero_()
-        dc.run(stream)
+        flush()
+        graph.replay()
     torch.cuda.synchronize(dev)
 
     sampler = ClockSampler(local_rank)
@@ -233,17 +250,24 @@ def main():
     time.sleep(0.3)
     barrier()
     torch.cuda.synchronize(dev)
+    step_ms, phase_acc = [], [0.0] * len(rtp.PHASES)
+    t_begin = time.perf_counter()
     for i in range(args.steps):
-        flush.zero_()
-        dc.step.set_timing_events(evs[i])
-        dc.run(stream)
+        flush()
+        a = torch.cuda.Event(enable_timing=True)
+        z = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        graph.replay()
+        z.record(stream)
+        z.synchronize()
+        step_ms.append(a.elapsed_time(z))
+        for k in range(len(rtp.PHASES)):
+            phase_acc[k] += inner[k].elapsed_time(inner[k + 1])
     torch.cuda.synchronize(dev)
     barrier()
+    wall = time.perf_counter() - t_begin
     clocks = sampler.stop()
-    dc.step.set_timing_events(None)
-    step_ms = [evs[i][0].elapsed_time(evs[i][NE - 1]) for i in range(args.steps)]
-    phase_ms = {name: statistics.mean(evs[i][k].elapsed_time(evs[i][k + 1]) for i in range(args.steps))
-                for k, name in enumerate(rtp.PHASES)}
+    phase_ms = {n: phase_acc[k] / args.steps for k, n in enumerate(rtp.PHASES)}
     t_ms = statistics.mean(step_ms)
 
     # ---- end to end: host query/len/p -> device, step, output -> host ----
@@ -256,7 +280,7 @@ def main():
     d2h = hout.numel() * hout.element_size()
     e2e_ms = []
     for i in range(max(3, args.warmup) + args.steps):
-        flush.zero_()
+        flush()
         a = torch.cuda.Event(enable_timing=True)
         z = torch.cuda.Event(enable_timing=True)
         a.record(stream)
@@ -264,13 +288,15 @@ def main():
         dc.q_rope.copy_(hq_rope, non_blocking=True)
         dc.seq_lens.copy_(hlens, non_blocking=True)
         dc.p.copy_(hp, non_blocking=True)
-        dc.run(stream)
+        graph.replay()
         hout.copy_(dc.out, non_blocking=True)
         z.record(stream)
         z.synchronize()
         if i >= max(3, args.warmup):
             e2e_ms.append(a.elapsed_time(z))
     e2e_t = statistics.mean(e2e_ms)
+    if dc.step.status() != 0:
+        raise SystemExit("device status set during the timed steps")
 
     # ---- max over ranks ----
     vals = torch.tensor([t_ms, e2e_t] + [phase_ms[n] for n in rtp.PHASES], dtype=torch.float64, device=dev)
@@ -310,7 +336,9 @@ def main():
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16 in, fp32 accumulate",
             "data": "synthetic (seeded; see DESIGN.md input recipe)",
             "config": dict(workload_config(case, args.workload), parallelism=f"replicas x{world}",
-                           dense_p1=bool(args.dense)),
+                           dense_p1=bool(args.dense), timing="CUDA-graph replay of one rtp_decode_step per step; "
+                           "CUDA events on the launching stream"),
+            "wall_s_timed_loop": wall,
             "roofline": {"bound": "hbm", "kernel": dom, "achieved": ach, "peak": peak, "unit": "GB/s",
                          "frac": ach / peak, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)",
                          "traffic": None, "algorithmic_bytes_per_launch": phase_bytes[dom]},

@@ -224,41 +224,81 @@ struct AttnCore {
 };
 
 // Combine the partials of `nparts` splits (stride G*PSTRIDE floats) for the
-// heads in `heads` and write out[b, g*G + h] as bf16.
+// heads in `heads` and write out[b, g*G + h] as bf16.  `scratch` is free
+// shared memory of at least G*nparts floats (the tile ring).  Pass 1 finds
+// each head's max and the split weights 2^(m_i - m*) (threads over
+// (head, split) pairs); pass 2 has each thread own 4 dims of one head and
+// stream the splits' float4 partials with independent loads.
 template <int G>
-__device__ void combine_parts(const Params& P, const float* parts, int nparts, uint32_t heads, int b, int g, int tid) {
-    __shared__ float s_red[ATT_THREADS / 32];
-    for (int h = 0; h < G; ++h) {
-        if (!((heads >> h) & 1u)) continue;
+__device__ void combine_parts(const Params& P, const float* parts, int nparts, uint32_t heads, int b, int g, int tid,
+                              float* scratch) {
+    __shared__ float s_den[G];
+    for (int x = tid; x < G * nparts; x += ATT_THREADS) {
+        const int h = x % G, i = x / G;
+        const float* pp = parts + ((int64_t)i * G + h) * PSTRIDE;
+        const float l = __ldcg(pp + 1), m = __ldcg(pp);
+        scratch[h * nparts + i] = (l > 0.f) ? m : -INFINITY;
+    }
+    __syncthreads();
+    // per-head max over the splits (one warp per head)
+    const int warp = tid >> 5, lane = tid & 31;
+    for (int h = warp; h < G; h += ATT_THREADS / 32) {
         float m = -INFINITY;
-        for (int i = tid; i < nparts; i += ATT_THREADS) {
-            const float* pp = parts + ((int64_t)i * G + h) * PSTRIDE;
-            if (__ldcg(pp + 1) > 0.f) m = fmaxf(m, __ldcg(pp));
-        }
+        for (int i = lane; i < nparts; i += 32) m = fmaxf(m, scratch[h * nparts + i]);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        if ((tid & 31) == 0) s_red[tid >> 5] = m;
-        __syncthreads();
-        m = s_red[0];
-        for (int w = 1; w < ATT_THREADS / 32; ++w) m = fmaxf(m, s_red[w]);
-        __syncthreads();
-        float num = 0.f, den = 0.f;
-        if (m != -INFINITY) {
-            for (int i = 0; i < nparts; ++i) {
-                const float* pp = parts + ((int64_t)i * G + h) * PSTRIDE;
-                const float l = __ldcg(pp + 1);
-                if (l > 0.f) {
-                    const float w = exp2f(__ldcg(pp) - m);
-                    den += w * l;
-                    num += w * __ldcg(pp + 4 + tid);
-                }
-            }
+        float den = 0.f;
+        for (int i = lane; i < nparts; i += 32) {
+            const float mi = scratch[h * nparts + i];
+            const float w = (mi == -INFINITY) ? 0.f : exp2f(mi - m);
+            scratch[h * nparts + i] = w;
+            if (w > 0.f) den += w * __ldcg(parts + ((int64_t)i * G + h) * PSTRIDE + 1);
         }
-        const float o = den > 0.f ? num / den : 0.f;
-        if (den > 0.f) {
-            P.out[((int64_t)b * P.Hq + g * G + h) * D + tid] = __bfloat16_as_ushort(__float2bfloat16_rn(o));
-        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+        if (lane == 0) s_den[h] = den;
     }
+    __syncthreads();
+    for (int x = tid; x < G * 32; x += ATT_THREADS) {
+        const int h = x / 32, q = x % 32;
+        if (!((heads >> h) & 1u)) continue;
+        const float den = s_den[h];
+        if (!(den > 0.f)) continue;
+        float4 acc0 = make_float4(0.f, 0.f, 0.f, 0.f), acc1 = acc0;
+        int i = 0;
+        for (; i + 1 < nparts; i += 2) {
+            const float w0 = scratch[h * nparts + i], w1 = scratch[h * nparts + i + 1];
+            const float4 a0 = __ldcg(reinterpret_cast<const float4*>(parts + ((int64_t)i * G + h) * PSTRIDE + 4) + q);
+            const float4 a1 =
+                __ldcg(reinterpret_cast<const float4*>(parts + ((int64_t)(i + 1) * G + h) * PSTRIDE + 4) + q);
+            acc0.x = fmaf(w0, a0.x, acc0.x);
+            acc0.y = fmaf(w0, a0.y, acc0.y);
+            acc0.z = fmaf(w0, a0.z, acc0.z);
+            acc0.w = fmaf(w0, a0.w, acc0.w);
+            acc1.x = fmaf(w1, a1.x, acc1.x);
+            acc1.y = fmaf(w1, a1.y, acc1.y);
+            acc1.z = fmaf(w1, a1.z, acc1.z);
+            acc1.w = fmaf(w1, a1.w, acc1.w);
+        }
+        if (i < nparts) {
+            const float w0 = scratch[h * nparts + i];
+            const float4 a0 = __ldcg(reinterpret_cast<const float4*>(parts + ((int64_t)i * G + h) * PSTRIDE + 4) + q);
+            acc0.x = fmaf(w0, a0.x, acc0.x);
+            acc0.y = fmaf(w0, a0.y, acc0.y);
+            acc0.z = fmaf(w0, a0.z, acc0.z);
+            acc0.w = fmaf(w0, a0.w, acc0.w);
+        }
+        const float inv = 1.f / den;
+        const float o0 = (acc0.x + acc1.x) * inv, o1 = (acc0.y + acc1.y) * inv, o2 = (acc0.z + acc1.z) * inv,
+                    o3 = (acc0.w + acc1.w) * inv;
+        uint16_t* dst = P.out + ((int64_t)b * P.Hq + g * G + h) * D + q * 4;
+        const uint32_t lo = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(o0)) |
+                            ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(o1)) << 16);
+        const uint32_t hi = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(o2)) |
+                            ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(o3)) << 16);
+        *reinterpret_cast<uint2*>(dst) = make_uint2(lo, hi);
+    }
+    __syncthreads();
 }
 
 // ---------------------------------------------------------------------------
@@ -393,7 +433,7 @@ __global__ void __launch_bounds__(ATT_THREADS) local_attn_kernel(const __grid_co
     __syncthreads();
     if (!last_arrival(P.tick_local + b * P.n_lg + lgi, nitems, &S.flag)) return;
     __threadfence();
-    combine_parts<G>(P, parts, nitems, heads, b, g, tid);
+    combine_parts<G>(P, parts, nitems, heads, b, g, tid, reinterpret_cast<float*>(&S.stage[0][0]));
 }
 
 // ---------------------------------------------------------------------------
@@ -452,7 +492,7 @@ __global__ void __launch_bounds__(ATT_THREADS) ret_attn_kernel(const __grid_cons
             __syncthreads();
             if (last_arrival(P.tick_ret + bg, nitems, &S.flag)) {
                 __threadfence();
-                combine_parts<G>(P, parts, nitems, heads, b, g, tid);
+                combine_parts<G>(P, parts, nitems, heads, b, g, tid, reinterpret_cast<float*>(&S.stage[0][0]));
                 __syncthreads();
             }
         }

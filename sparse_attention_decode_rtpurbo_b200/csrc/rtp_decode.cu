@@ -127,8 +127,12 @@ static rtp_status make_plan(const rtp_dims* d, const uint8_t* head_kind, int win
 
 template <int G>
 static cudaError_t launch_all(const Params& P, const Plan& pl, cudaStream_t s, void* const* ev) {
+    // under stream capture the records must become event nodes of the graph
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (ev) cudaStreamIsCapturing(s, &cap);
+    const unsigned ev_flags = (cap == cudaStreamCaptureStatusActive) ? cudaEventRecordExternal : cudaEventRecordDefault;
     auto mark = [&](int i) {
-        if (ev) cudaEventRecord((cudaEvent_t)ev[i], s);
+        if (ev) cudaEventRecordWithFlags((cudaEvent_t)ev[i], s, ev_flags);
     };
     const size_t smem = sizeof(AttnSmem<G>);
     static std::atomic<int> attr_done{0};

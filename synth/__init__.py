@@ -283,7 +283,8 @@ def make_case(name: str, *, B: int, Hkv: int, G: int, seq_lens: Sequence[int], r
     regimes[b] in {"gaussian", "needle", "diffuse", "needles4x"}:
       gaussian  - plain N(0,1) q/k/v; scores s/4 ~ N(0, ~1)
       needle    - one token per retrieval group whose index key sits along the
-                  group's mean projected-query direction, sized so that its
+                  direction equally aligned with all the group's projected
+                  queries (min-norm solution of qhat_h . u = const), sized so that its
                   score beats the Cauchy-Schwarz bound of every other token's
                   score by 4 ln(99 L): it alone carries >= 0.99 of each head's
                   softmax(s/4) mass
@@ -383,7 +384,10 @@ def make_case(name: str, *, B: int, Hkv: int, G: int, seq_lens: Sequence[int], r
             rms_comp = rms_norm / math.sqrt(R)
             qidx = {h: _q_idx(Wq[h], q_pre[b, h]) for h in heads}
             qhat = {h: qidx[h] / np.linalg.norm(qidx[h]) for h in heads}
-            u = sum(qhat[h] for h in heads)
+            # direction equally aligned with every head's projected query:
+            # min-norm solution of qhat_h . u' = 1 for all heads, normalised
+            Qh = np.stack([qhat[h] for h in heads])
+            u = np.linalg.lstsq(Qh, np.ones(len(heads)), rcond=None)[0]
             u = u / np.linalg.norm(u)
             ms = stream_id("pos", b, g)
             if reg == "needle":

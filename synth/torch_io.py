@@ -60,6 +60,8 @@ class DeviceCase:
 
     def run(self, stream=None):
         c = self.case
+        if stream is None:
+            stream = torch.cuda.current_stream(self.out.device)
         self.step(self.q_pre, self.q_rope, self.k_idx, self.k_cache, self.v_cache, self.Wq, self.seq_lens, self.p,
                   c.window, c.sink, self.out, stream)
 

@@ -24,7 +24,8 @@ def blocks_to_positions(kept: np.ndarray, L: int) -> np.ndarray:
     return np.concatenate([np.arange(64 * j, min(64 * j + 64, L)) for j in js]).astype(np.int64)
 
 
-def compare(case, gpu, ref, *, exact_sets: bool = False, check_kstar: bool = False, heads=None):
+def compare(case, gpu, ref, *, exact_sets: bool = False, check_kstar: bool = False, check_tau: bool = False,
+            heads=None):
     """Returns a list of failure strings (empty = pass) and a stats dict."""
     fails = []
     stats = {"set_diffs": 0, "heads": 0, "max_err": 0.0}
@@ -60,10 +61,10 @@ def compare(case, gpu, ref, *, exact_sets: bool = False, check_kstar: bool = Fal
                                          f"{band:.3g} of tau={tau:.6g}; nearest {np.min(np.abs(blk - tau)):.3g}")
                             break
                     r_out = oracle.attend(case, b, h, blocks_to_positions(gk, L))
-                elif check_kstar:
-                    if int(gpu["kstar"][b, h]) != int(ref["kstar"][b, h]):
+                else:
+                    if check_kstar and int(gpu["kstar"][b, h]) != int(ref["kstar"][b, h]):
                         fails.append(f"b{b} h{h}: kstar {gpu['kstar'][b, h]} != {ref['kstar'][b, h]}")
-                    if float(gpu["tau"][b, h]) != float(ref["tau"][b, h]):
+                    if check_tau and float(gpu["tau"][b, h]) != float(ref["tau"][b, h]):
                         fails.append(f"b{b} h{h}: tau {gpu['tau'][b, h]} != {ref['tau'][b, h]}")
                 if int(gpu["kept_blocks"][b, h]) != int(gk.sum()):
                     fails.append(f"b{b} h{h}: kept_blocks {gpu['kept_blocks'][b, h]} != bitmap popcount {gk.sum()}")

@@ -15,13 +15,13 @@ from synth.torch_io import DeviceCase  # noqa: E402
 from tests.parity import compare  # noqa: E402
 
 
-def run_both(case, exact=False, check_kstar=False):
+def run_both(case, exact=False, check_kstar=False, check_tau=False):
     dc = DeviceCase(case)
     dc.run()
     gpu = dc.results()
     ref = oracle.decode_step(case)
     assert ref["rc"] == 0
-    fails, stats = compare(case, gpu, ref, exact_sets=exact, check_kstar=check_kstar)
+    fails, stats = compare(case, gpu, ref, exact_sets=exact, check_kstar=check_kstar, check_tau=check_tau)
     return fails, stats, gpu, ref
 
 
@@ -50,7 +50,7 @@ def test_integer_scores_exact_block_sets():
             dc = DeviceCase(case)
             dc.run()
             gpu = dc.results()
-            fails, _ = compare(case, gpu, ref, exact_sets=True, check_kstar=True)
+            fails, _ = compare(case, gpu, ref, exact_sets=True, check_kstar=True, check_tau=True)
             assert not fails, f"seed {seed} G{G} paged{paged}:\n" + "\n".join(fails[:10])
             done += 1
     assert done >= 60

@@ -89,19 +89,11 @@ typedef struct rtp_debug {
  *   debug: host pointer to an rtp_debug of device pointers, or NULL.
  *   timing_events / n_timing_events: optional host array of cudaEvent_t
  *     handles (created by the caller).  When n_timing_events >=
- *     RTP_TIMING_EVENTS the call records event i on `stream` at boundary i of
- *     the kernel sequence (see RTP_PHASE_*), so phase i lasts from event i to
- *     event i+1.  Phases with nothing to do still record their events.
+ *     RTP_TIMING_EVENTS the call records event 0 on `stream` just before its
+ *     kernel and event 1 just after it (external event nodes when the stream
+ *     is being captured into a CUDA graph).
  */
-enum {
-    RTP_PHASE_LOCAL = 0,      /* local heads: sink + window attention and combine */
-    RTP_PHASE_SCORE = 1,      /* index scores + per-group selection decision */
-    RTP_PHASE_SELECT = 2,     /* exact top-p radix passes (heads that need them) */
-    RTP_PHASE_MARK = 3,       /* block masks */
-    RTP_PHASE_BLOCKLIST = 4,  /* per-KV-group union block lists */
-    RTP_PHASE_RETRIEVAL = 5,  /* retrieval heads: block-sparse attention and combine */
-    RTP_TIMING_EVENTS = 7
-};
+enum { RTP_TIMING_EVENTS = 2 };
 
 typedef struct rtp_dims {
     int32_t batch, num_q_heads, num_kv_heads;

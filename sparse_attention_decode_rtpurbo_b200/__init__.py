@@ -43,7 +43,7 @@ class RtpDims(ctypes.Structure):
                 ("n_timing_events", ctypes.c_int32)]
 
 
-PHASES = ["local", "score", "select", "mark", "blocklist", "retrieval"]
+PHASES = ["step"]
 TIMING_EVENTS = len(PHASES) + 1
 
 

@@ -1,5 +1,5 @@
 // C ABI of the RTPurbo decode step: argument checks, workspace layout and the
-// launch sequence of the sm_100a kernels (rtp_select.cuh, rtp_attn.cuh).
+// launch of the persistent sm_100a decode-step kernel (rtp_step.cuh, rtp_step_kernel.cuh).
 #include <cuda_runtime.h>
 #include <stdint.h>
 #include <string.h>
@@ -8,13 +8,12 @@
 #include <atomic>
 
 #include "../../include/rtp_decode.h"
-#include "rtp_attn.cuh"
-#include "rtp_select.cuh"
+#include "rtp_step_kernel.cuh"
 
 namespace rtp {
 
-constexpr int NSM_PLAN = 148;      // SMs of a B200: sizes the persistent grids and the split counts
-constexpr int RET_CTAS_PER_SM = 2; // two attention CTAs (about 99 KB shared memory each) per SM
+constexpr int NSM_PLAN = 148;       // SMs of a B200: sizes the split counts
+constexpr int MAX_GRID = 148 * 4;   // upper bound of the persistent grid (partials are sized for it)
 
 struct Plan {
     int B, Hq, Hkv, G, Ncap, nblk_cap, words_cap, nchunks;
@@ -24,8 +23,8 @@ struct Plan {
     uint8_t lg_group[MAX_HKV], lg_mask[MAX_HKV];
     uint8_t slot_head[MAX_HQ], slot_rg[MAX_HQ];
     // workspace byte offsets
-    size_t o_status, o_tick_score, o_tick_radix, o_tick_local, o_tick_ret, o_keys, o_cstat, o_hs, o_hist_cnt,
-        o_hist_mass, o_chunk_cnt, o_tie_off, o_bitmap, o_blist, o_bcount, o_lpart, o_rpart, total;
+    size_t o_status, o_sync, o_rlist, o_rglist, o_tick_score, o_tick_radix, o_tick_local, o_tick_ret, o_keys, o_cstat,
+        o_hs, o_hist_cnt, o_hist_mass, o_chunk_cnt, o_tie_off, o_bitmap, o_blist, o_bcount, o_lpart, o_rpart, total;
 };
 
 static size_t align_up(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -92,9 +91,11 @@ static rtp_status make_plan(const rtp_dims* d, const uint8_t* head_kind, int win
         const int64_t nv_max = std::min<int64_t>(pl->nblk_cap, (sink + BLK - 1) / BLK + (window + BLK - 1) / BLK + 1);
         const int64_t total = (int64_t)pl->B * pl->n_lg * nv_max;
         pl->local_kb = (int)std::max<int64_t>(1, (total + 2 * NSM_PLAN - 1) / (2 * NSM_PLAN));
+        // the split combine keeps one weight per (head, split) in 512*G floats
+        pl->local_kb = (int)std::max<int64_t>(pl->local_kb, (nv_max + 511) / 512);
         pl->local_items = (int)((nv_max + pl->local_kb - 1) / pl->local_kb);
     }
-    pl->ret_grid = NSM_PLAN * RET_CTAS_PER_SM;
+    pl->ret_grid = MAX_GRID;
     // workspace layout
     const size_t BR = (size_t)pl->B * pl->n_ret, BG = (size_t)pl->B * pl->n_rg, BL = (size_t)pl->B * pl->n_lg;
     size_t o = 0;
@@ -104,6 +105,9 @@ static rtp_status make_plan(const rtp_dims* d, const uint8_t* head_kind, int win
         return at;
     };
     pl->o_status = take(64);
+    pl->o_sync = take(sizeof(Sync));
+    pl->o_rlist = take(BR * 4);
+    pl->o_rglist = take(BG * 4);
     pl->o_tick_score = take(BG * 4);
     pl->o_tick_radix = take(BR * 4);
     pl->o_tick_local = take(BL * 4);
@@ -126,38 +130,36 @@ static rtp_status make_plan(const rtp_dims* d, const uint8_t* head_kind, int win
 }
 
 template <int G>
-static cudaError_t launch_all(const Params& P, const Plan& pl, cudaStream_t s, void* const* ev) {
+static cudaError_t launch_step(const Params& P, const Plan& pl, uint8_t* ws, cudaStream_t s, void* const* ev) {
+    const size_t smem = sizeof(StepSmem<G>);
+    static std::atomic<int> ctas_per_sm{0};
+    static std::atomic<int> num_sms{0};
+    if (!ctas_per_sm.load()) {
+        cudaError_t e = cudaFuncSetAttribute(step_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        int n = 0, dev = 0, sms = 0;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, step_kernel<G>, STEP_THREADS, smem);
+        if (e != cudaSuccess) return e;
+        if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+        if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+        num_sms.store(sms);
+        ctas_per_sm.store(std::max(1, n));
+    }
     // under stream capture the records must become event nodes of the graph
     cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
     if (ev) cudaStreamIsCapturing(s, &cap);
     const unsigned ev_flags = (cap == cudaStreamCaptureStatusActive) ? cudaEventRecordExternal : cudaEventRecordDefault;
-    auto mark = [&](int i) {
-        if (ev) cudaEventRecordWithFlags((cudaEvent_t)ev[i], s, ev_flags);
-    };
-    const size_t smem = sizeof(AttnSmem<G>);
-    static std::atomic<int> attr_done{0};
-    if (!attr_done.load()) {
-        cudaError_t e = cudaFuncSetAttribute(local_attn_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(ret_attn_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        attr_done.store(1);
-    }
-    mark(RTP_PHASE_LOCAL);
-    if (pl.n_lg) local_attn_kernel<G><<<dim3(pl.local_items, pl.n_lg, pl.B), ATT_THREADS, smem, s>>>(P);
-    mark(RTP_PHASE_SCORE);
-    if (pl.n_ret) score_kernel<G><<<dim3(pl.nchunks, pl.n_rg, pl.B), SEL_THREADS, 0, s>>>(P);
-    mark(RTP_PHASE_SELECT);
-    if (pl.n_ret)
-        for (int pass = 0; pass < 4; ++pass)
-            radix_kernel<<<dim3(pl.nchunks, pl.n_ret, pl.B), SEL_THREADS, 0, s>>>(P, pass);
-    mark(RTP_PHASE_MARK);
-    if (pl.n_ret) mark_kernel<<<dim3(pl.nchunks, pl.n_ret, pl.B), SEL_THREADS, 0, s>>>(P);
-    mark(RTP_PHASE_BLOCKLIST);
-    if (pl.n_ret) blocklist_kernel<<<dim3(pl.n_rg, pl.B), BL_THREADS, 0, s>>>(P);
-    mark(RTP_PHASE_RETRIEVAL);
-    if (pl.n_ret) ret_attn_kernel<G><<<pl.ret_grid, ATT_THREADS, smem, s>>>(P);
-    mark(RTP_PHASE_RETRIEVAL + 1);
+    StepParams SP;
+    SP.P = P;
+    SP.sync = reinterpret_cast<Sync*>(ws + pl.o_sync);
+    SP.rlist = reinterpret_cast<uint32_t*>(ws + pl.o_rlist);
+    SP.rglist = reinterpret_cast<uint32_t*>(ws + pl.o_rglist);
+    SP.n_score_items = pl.B * pl.n_rg * pl.nchunks;
+    SP.n_local_items = pl.B * pl.n_lg * pl.local_items;
+    const int grid = std::min(MAX_GRID, ctas_per_sm.load() * num_sms.load());
+    if (ev) cudaEventRecordWithFlags((cudaEvent_t)ev[0], s, ev_flags);
+    step_kernel<G><<<grid, STEP_THREADS, smem, s>>>(SP);
+    if (ev) cudaEventRecordWithFlags((cudaEvent_t)ev[1], s, ev_flags);
     return cudaGetLastError();
 }
 
@@ -253,10 +255,10 @@ extern "C" rtp_status rtp_decode_step(const rtp_dims* dims, const uint16_t* q_pr
     void* const* ev = (dims->timing_events && dims->n_timing_events >= RTP_TIMING_EVENTS) ? dims->timing_events : nullptr;
     cudaError_t e;
     switch (pl.G) {
-        case 1: e = launch_all<1>(P, pl, s, ev); break;
-        case 2: e = launch_all<2>(P, pl, s, ev); break;
-        case 4: e = launch_all<4>(P, pl, s, ev); break;
-        default: e = launch_all<8>(P, pl, s, ev); break;
+        case 1: e = launch_step<1>(P, pl, ws, s, ev); break;
+        case 2: e = launch_step<2>(P, pl, ws, s, ev); break;
+        case 4: e = launch_step<4>(P, pl, ws, s, ev); break;
+        default: e = launch_step<8>(P, pl, ws, s, ev); break;
     }
     return e == cudaSuccess ? RTP_OK : RTP_ERR_CUDA;
 }

@@ -1,0 +1,931 @@
+// Item handlers and the persistent kernel of the decode step (see rtp_step.cuh).
+#pragma once
+#include "rtp_step.cuh"
+
+namespace rtp {
+
+struct StepParams {
+    Params P;
+    Sync* sync;
+    uint32_t* rlist;    // [B*n_ret] (b << 16 | slot) of heads needing the radix select
+    uint32_t* rglist;   // [B*n_rg]  (b << 16 | rg) of groups holding such heads
+    int n_score_items, n_local_items;
+};
+
+// ===========================================================================
+// index scores (consumers)
+// ===========================================================================
+template <int G>
+struct ScoreState {
+    uint32_t mk[G], am[G], nk[G];
+    float ms[G], sm[G];
+};
+
+template <int G>
+__device__ void score_begin(const Params& P, StepSmem<G>& S, ScoreState<G>& st, int b, int rgi, int tid) {
+    const int nh = P.rg_nh[rgi], slot0 = P.rg_slot0[rgi];
+    const int warp = tid >> 5, lane = tid & 31;
+    // q_idx = Wq_idx[h] . q_pre[b,h] (fp32), one warp per (head, row)
+    for (int pr = warp; pr < nh * R; pr += CONSUMERS / 32) {
+        const int hh = pr / R, r = pr % R;
+        const int h = P.slot_head[slot0 + hh];
+        const uint2 w = *reinterpret_cast<const uint2*>(P.Wq + ((int64_t)h * R + r) * D + lane * 4);
+        const uint2 q = *reinterpret_cast<const uint2*>(P.q_pre + ((int64_t)b * P.Hq + h) * D + lane * 4);
+        float a = bf_lo(w.x) * bf_lo(q.x);
+        a = fmaf(bf_hi(w.x), bf_hi(q.x), a);
+        a = fmaf(bf_lo(w.y), bf_lo(q.y), a);
+        a = fmaf(bf_hi(w.y), bf_hi(q.y), a);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+        if (lane == 0) S.qi[hh][r] = a;
+    }
+#pragma unroll
+    for (int hh = 0; hh < G; ++hh) {
+        st.mk[hh] = 0u;
+        st.am[hh] = 0xFFFFFFFFu;
+        st.nk[hh] = 0xFFFFFFFFu;
+        st.ms[hh] = -INFINITY;
+        st.sm[hh] = 0.f;
+    }
+    consumer_sync();
+}
+
+// rows [0, nvalid) of the staged k_idx tile are tokens n0 + row
+template <int G>
+__device__ void score_tile(const Params& P, StepSmem<G>& S, ScoreState<G>& st, const uint8_t* data, int b, int rgi,
+                           int n0, int nvalid, int tid) {
+    const int nh = P.rg_nh[rgi], slot0 = P.rg_slot0[rgi];
+    const uint4* rows = reinterpret_cast<const uint4*>(data);
+    for (int r = tid; r < nvalid; r += CONSUMERS) {
+        const uint4 u0 = rows[2 * r], u1 = rows[2 * r + 1];
+        float k[R];
+        k[0] = bf_lo(u0.x); k[1] = bf_hi(u0.x); k[2] = bf_lo(u0.y); k[3] = bf_hi(u0.y);
+        k[4] = bf_lo(u0.z); k[5] = bf_hi(u0.z); k[6] = bf_lo(u0.w); k[7] = bf_hi(u0.w);
+        k[8] = bf_lo(u1.x); k[9] = bf_hi(u1.x); k[10] = bf_lo(u1.y); k[11] = bf_hi(u1.y);
+        k[12] = bf_lo(u1.z); k[13] = bf_hi(u1.z); k[14] = bf_lo(u1.w); k[15] = bf_hi(u1.w);
+        const int n = n0 + r;
+#pragma unroll
+        for (int hh = 0; hh < G; ++hh) {
+            if (hh >= nh) break;
+            float s = 0.f;
+#pragma unroll
+            for (int i = 0; i < R; ++i) s = fmaf(S.qi[hh][i], k[i], s);
+            const uint32_t key = f2key(s);
+            P.keys[((int64_t)b * P.n_ret + slot0 + hh) * P.Ncap + n] = key;
+            if (key > st.mk[hh]) {
+                st.mk[hh] = key;
+                st.am[hh] = (uint32_t)n;
+            }
+            st.nk[hh] = min(st.nk[hh], key);
+            if (s > st.ms[hh]) {
+                st.sm[hh] = st.sm[hh] * expf((st.ms[hh] - s) * 0.25f) + 1.f;
+                st.ms[hh] = s;
+            } else {
+                st.sm[hh] += expf((s - st.ms[hh]) * 0.25f);
+            }
+        }
+    }
+}
+
+// Selection of the heads of group (b, rgi) from its chunk partials.  Heads
+// whose best token alone reaches p, or whose p >= 1, are final; if all heads
+// of the group are final its block list is written here.
+template <int G>
+__device__ void score_decide(const StepParams& SP, StepSmem<G>& S, int b, int rgi, int L, int nch, int tid) {
+    const Params& P = SP.P;
+    const int nh = P.rg_nh[rgi], slot0 = P.rg_slot0[rgi], g = P.rg_group[rgi];
+    const int warp = tid >> 5, lane = tid & 31;
+    const int nblk = (L + BLK - 1) / BLK;
+    const int nwords = (nblk + 31) / 32;
+    __shared__ int s_mode[MAX_G];
+    __shared__ uint32_t s_arg[MAX_G];
+    for (int hh = 0; hh < nh; ++hh) {
+        const int slot = slot0 + hh;
+        const ChunkStat* cs = P.cstat + ((int64_t)b * P.n_ret + slot) * P.nchunks;
+        uint32_t k = 0, a = 0xFFFFFFFFu, mn = 0xFFFFFFFFu;
+        for (int c = tid; c < nch; c += CONSUMERS) {
+            const ChunkStat x = cs[c];
+            if (x.maxkey > k || (x.maxkey == k && x.argmax < a)) {
+                k = x.maxkey;
+                a = x.argmax;
+            }
+            mn = min(mn, x.minkey);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const uint32_t k2 = __shfl_xor_sync(0xffffffffu, k, o);
+            const uint32_t a2 = __shfl_xor_sync(0xffffffffu, a, o);
+            mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+            if (k2 > k || (k2 == k && a2 < a)) {
+                k = k2;
+                a = a2;
+            }
+        }
+        if (lane == 0) {
+            S.w_key[0][warp] = k;
+            S.w_arg[0][warp] = a;
+            S.w_min[0][warp] = mn;
+        }
+        consumer_sync();
+        k = S.w_key[0][0];
+        a = S.w_arg[0][0];
+        mn = S.w_min[0][0];
+        for (int w = 1; w < 4; ++w) {
+            if (S.w_key[0][w] > k || (S.w_key[0][w] == k && S.w_arg[0][w] < a)) {
+                k = S.w_key[0][w];
+                a = S.w_arg[0][w];
+            }
+            mn = min(mn, S.w_min[0][w]);
+        }
+        const float smax = key2f(k);
+        double su = 0.0;
+        for (int c = tid; c < nch; c += CONSUMERS) {
+            const ChunkStat x = cs[c];
+            su += x.sum * exp(((double)key2f(x.maxkey) - (double)smax) * 0.25);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) su += __shfl_xor_sync(0xffffffffu, su, o);
+        consumer_sync();
+        if (lane == 0) S.w_sum[0][warp] = su;
+        consumer_sync();
+        if (tid == 0) {
+            const double z = S.w_sum[0][0] + S.w_sum[0][1] + S.w_sum[0][2] + S.w_sum[0][3];
+            const float pb = __ldg(P.p + b);
+            HeadState h;
+            h.smax = smax;
+            h.maxkey = k;
+            h.argmax = a;
+            h.minkey = mn;
+            h.pad0 = 0;
+            h.zrel = z;
+            h.target = 0;
+            h.mass_above = 0;
+            h.prefix = 0;
+            h.count_above = 0;
+            h.n_eq = 0;
+            h.n_tie = 0;
+            h.all_ties = 1;
+            h.tau_key = 0;
+            h.pad1 = 0;
+            if (!(pb > 0.f)) {
+                h.mode = MODE_SKIP;
+                h.kstar = 0;
+                set_status(P, ST_DEVICE_INPUT);
+            } else if (pb >= 1.f) {
+                h.mode = MODE_ALL;
+                h.kstar = (uint32_t)L;
+                h.tau_key = mn;
+            } else if (1.0 >= (double)pb * z * (1.0 + 1e-6)) {
+                h.mode = MODE_TOP1;   // the best token alone reaches p
+                h.kstar = 1;
+                h.tau_key = k;
+            } else {
+                h.mode = MODE_RADIX;
+                h.kstar = 0;
+            }
+            P.hs[(int64_t)b * P.n_ret + slot] = h;
+            const int bh = b * P.Hq + P.slot_head[slot];
+            if (P.dbg_smax) P.dbg_smax[bh] = smax;
+            if (P.dbg_Z) P.dbg_Z[bh] = z;
+            if (h.mode != MODE_RADIX) {
+                if (P.dbg_tau) P.dbg_tau[bh] = key2f(h.tau_key);
+                if (P.dbg_kstar) P.dbg_kstar[bh] = (int32_t)h.kstar;
+                if (P.dbg_kept)
+                    P.dbg_kept[bh] = h.mode == MODE_TOP1 ? 1 : (h.mode == MODE_ALL ? nblk : 0);
+            }
+            s_mode[hh] = h.mode;
+            s_arg[hh] = a;
+        }
+        // the radix histogram of this head starts at zero
+        for (int d = tid; d < 256; d += CONSUMERS) {
+            P.hist_cnt[((int64_t)b * P.n_ret + slot) * 256 + d] = 0;
+            P.hist_mass[((int64_t)b * P.n_ret + slot) * 256 + d] = 0ull;
+        }
+        consumer_sync();
+    }
+
+    bool any_radix = false, any_all = false;
+    uint32_t all_mask = 0;
+    for (int hh = 0; hh < nh; ++hh) {
+        any_radix |= s_mode[hh] == MODE_RADIX;
+        if (s_mode[hh] == MODE_ALL) {
+            any_all = true;
+            all_mask |= 1u << (P.slot_head[slot0 + hh] - g * P.G);
+        }
+    }
+    // bitmap words of the heads that are final (read by the block-list
+    // builder of a group that also has radix heads, and by the debug sink)
+    const bool want_words = any_radix || P.dbg_bitmap != nullptr;
+    if (want_words) {
+        for (int hh = 0; hh < nh; ++hh) {
+            const int mode = s_mode[hh];
+            if (mode == MODE_RADIX) continue;
+            const int slot = slot0 + hh;
+            for (int w = tid; w < nwords; w += CONSUMERS) {
+                uint32_t word = 0;
+                if (mode == MODE_ALL) {
+                    const int nb = min(32, nblk - w * 32);
+                    word = nb >= 32 ? 0xFFFFFFFFu : ((1u << nb) - 1u);
+                } else if (mode == MODE_TOP1) {
+                    const int j = (int)(s_arg[hh] / BLK) - w * 32;
+                    if (j >= 0 && j < 32) word = 1u << j;
+                }
+                if (any_radix) P.bitmap[((int64_t)b * P.n_ret + slot) * P.words_cap + w] = word;
+                if (P.dbg_bitmap) P.dbg_bitmap[((int64_t)b * P.Hq + P.slot_head[slot]) * P.words_cap + w] = word;
+            }
+        }
+    }
+    const int bg = b * P.n_rg + rgi;
+    if (any_radix) {
+        consumer_sync();
+        if (tid == 0) {
+            for (int hh = 0; hh < nh; ++hh)
+                if (s_mode[hh] == MODE_RADIX) {
+                    const uint32_t k = atomicAdd(&SP.sync->n_radix_heads, 1u);
+                    SP.rlist[k] = ((uint32_t)b << 16) | (uint32_t)(slot0 + hh);
+                }
+            const uint32_t gi = atomicAdd(&SP.sync->n_radix_groups, 1u);
+            SP.rglist[gi] = ((uint32_t)b << 16) | (uint32_t)rgi;
+            __threadfence();
+            atomicAdd(&SP.sync->groups_decided, 1u);
+        }
+        return;
+    }
+    // every head final: write the group's block list now
+    uint32_t* list = P.blist + (int64_t)bg * P.nblk_cap;
+    if (any_all) {
+        for (int j = tid; j < nblk; j += CONSUMERS) {
+            uint32_t hm = all_mask;
+            for (int hh = 0; hh < nh; ++hh)
+                if (s_mode[hh] == MODE_TOP1 && (int)(s_arg[hh] / BLK) == j) hm |= 1u << (P.slot_head[slot0 + hh] - g * P.G);
+            list[j] = ((uint32_t)j << 8) | hm;
+        }
+        if (tid == 0) P.bcount[bg] = (uint32_t)nblk;
+    } else if (tid == 0) {
+        // distinct argmax blocks of the TOP1 heads, ascending
+        uint32_t cnt = 0;
+        int last = -1;
+        while (true) {
+            int best = INT_MAX;
+            for (int hh = 0; hh < nh; ++hh)
+                if (s_mode[hh] == MODE_TOP1) {
+                    const int j = (int)(s_arg[hh] / BLK);
+                    if (j > last && j < best) best = j;
+                }
+            if (best == INT_MAX) break;
+            uint32_t hm = 0;
+            for (int hh = 0; hh < nh; ++hh)
+                if (s_mode[hh] == MODE_TOP1 && (int)(s_arg[hh] / BLK) == best)
+                    hm |= 1u << (P.slot_head[slot0 + hh] - g * P.G);
+            list[cnt++] = ((uint32_t)best << 8) | hm;
+            last = best;
+        }
+        P.bcount[bg] = cnt;
+    }
+    consumer_sync();
+    if (tid == 0) {
+        __threadfence();
+        atomicAdd(&SP.sync->groups_decided, 1u);
+        atomicAdd(&SP.sync->groups_ready, 1u);
+    }
+}
+
+template <int G>
+__device__ void score_end(const StepParams& SP, StepSmem<G>& S, ScoreState<G>& st, int b, int rgi, int chunk, int L,
+                          int nch, int tid) {
+    const Params& P = SP.P;
+    const int nh = P.rg_nh[rgi], slot0 = P.rg_slot0[rgi];
+    const int warp = tid >> 5, lane = tid & 31;
+#pragma unroll
+    for (int hh = 0; hh < G; ++hh) {
+        if (hh >= nh) break;
+        uint32_t k = st.mk[hh], a = st.am[hh], mn = st.nk[hh];
+        float m = st.ms[hh];
+        double su = (double)st.sm[hh];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const uint32_t k2 = __shfl_xor_sync(0xffffffffu, k, o);
+            const uint32_t a2 = __shfl_xor_sync(0xffffffffu, a, o);
+            const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
+            const double s2 = __shfl_xor_sync(0xffffffffu, su, o);
+            mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+            if (k2 > k || (k2 == k && a2 < a)) {
+                k = k2;
+                a = a2;
+            }
+            const float mm = fmaxf(m, m2);
+            su = (mm == -INFINITY) ? 0.0 : su * exp((double)(m - mm) * 0.25) + s2 * exp((double)(m2 - mm) * 0.25);
+            m = mm;
+        }
+        if (lane == 0) {
+            S.w_key[hh][warp] = k;
+            S.w_arg[hh][warp] = a;
+            S.w_min[hh][warp] = mn;
+            S.w_m[hh][warp] = m;
+            S.w_sum[hh][warp] = su;
+        }
+    }
+    consumer_sync();
+    if (tid < nh) {
+        const int hh = tid;
+        uint32_t k = 0, a = 0xFFFFFFFFu, mn = 0xFFFFFFFFu;
+        float m = -INFINITY;
+        for (int w = 0; w < 4; ++w) {
+            if (S.w_key[hh][w] > k || (S.w_key[hh][w] == k && S.w_arg[hh][w] < a)) {
+                k = S.w_key[hh][w];
+                a = S.w_arg[hh][w];
+            }
+            mn = min(mn, S.w_min[hh][w]);
+            m = fmaxf(m, S.w_m[hh][w]);
+        }
+        double su = 0.0;
+        for (int w = 0; w < 4; ++w)
+            if (S.w_m[hh][w] != -INFINITY) su += S.w_sum[hh][w] * exp((double)(S.w_m[hh][w] - m) * 0.25);
+        ChunkStat cs;
+        cs.maxkey = k;
+        cs.argmax = a;
+        cs.minkey = mn;
+        cs.pad = 0;
+        cs.sum = su;
+        P.cstat[((int64_t)b * P.n_ret + slot0 + hh) * P.nchunks + chunk] = cs;
+    }
+    if (!consumer_last(P.tick_score + b * P.n_rg + rgi, nch, &S.flag)) return;
+    __threadfence();
+    score_decide<G>(SP, S, b, rgi, L, nch, tid);
+}
+
+// ===========================================================================
+// exact radix select, block marking, block lists (consumers, L2-resident)
+// ===========================================================================
+template <int G>
+__device__ void radix_item(const StepParams& SP, StepSmem<G>& S, int j, int pass, int tid) {
+    const Params& P = SP.P;
+    const int k = j / P.nchunks, chunk = j % P.nchunks;
+    const uint32_t e = __ldcg(SP.rlist + k);
+    const int b = (int)(e >> 16), slot = (int)(e & 0xFFFFu);
+    const int L = __ldg(P.seq_lens + b);
+    const int nch = (L + CHUNK - 1) / CHUNK;
+    if (chunk >= nch) return;
+    const int64_t bs = (int64_t)b * P.n_ret + slot;
+    HeadState* hsp = P.hs + bs;
+    for (int d = tid; d < 256; d += CONSUMERS) {
+        S.hcnt[d] = 0;
+        S.hmass[d] = 0ull;
+    }
+    consumer_sync();
+    const uint32_t prefix = __ldcg(&hsp->prefix);
+    const float smax = __ldcg(&hsp->smax);
+    const int shift = 24 - 8 * pass;
+    const int n_begin = chunk * CHUNK, n_end = min(L, n_begin + CHUNK);
+    const uint32_t* keys = P.keys + bs * P.Ncap;
+    for (int n = n_begin + tid; n < n_end; n += CONSUMERS) {
+        const uint32_t key = __ldcg(keys + n);
+        if (pass > 0 && (key >> (32 - 8 * pass)) != prefix) continue;
+        const int d = (key >> shift) & 255;
+        atomicAdd(&S.hcnt[d], 1u);
+        atomicAdd(&S.hmass[d], fixmass(key, smax));
+    }
+    consumer_sync();
+    uint32_t* gcnt = P.hist_cnt + bs * 256;
+    unsigned long long* gmass = P.hist_mass + bs * 256;
+    for (int d = tid; d < 256; d += CONSUMERS) {
+        if (S.hcnt[d]) {
+            atomicAdd(gcnt + d, S.hcnt[d]);
+            atomicAdd(gmass + d, S.hmass[d]);
+        }
+        if (pass == 3) P.chunk_cnt[(bs * P.nchunks + chunk) * 256 + d] = S.hcnt[d];
+    }
+    if (!consumer_last(P.tick_radix + bs, nch, &S.flag)) return;
+    __threadfence();
+    for (int d = tid; d < 256; d += CONSUMERS) {
+        S.hcnt[d] = __ldcg(gcnt + d);
+        S.hmass[d] = __ldcg(gmass + d);
+        gcnt[d] = 0;
+        gmass[d] = 0ull;
+    }
+    consumer_sync();
+    if (tid == 0) {
+        HeadState st = *hsp;
+        if (pass == 0) {
+            unsigned long long z = 0;
+            for (int d = 0; d < 256; ++d) z += S.hmass[d];
+            const double pb = (double)__ldg(P.p + b);
+            unsigned long long t = (unsigned long long)ceil(pb * (double)z);
+            if (t > z) t = z;
+            if (t == 0) t = 1;
+            st.target = t;
+            st.mass_above = 0;
+            st.count_above = 0;
+            st.prefix = 0;
+        }
+        unsigned long long cum = st.mass_above;
+        uint32_t cabove = st.count_above;
+        int dstar = 0;
+        for (int d = 255; d >= 0; --d) {
+            if (cum + S.hmass[d] >= st.target) {
+                dstar = d;
+                break;
+            }
+            cum += S.hmass[d];
+            cabove += S.hcnt[d];
+        }
+        st.mass_above = cum;
+        st.count_above = cabove;
+        st.prefix = (st.prefix << 8) | (uint32_t)dstar;
+        if (pass == 3) {
+            st.tau_key = st.prefix;
+            st.n_eq = S.hcnt[dstar];
+            const unsigned long long m_tau = st.n_eq ? S.hmass[dstar] / st.n_eq : 0ull;
+            const unsigned long long need = st.target - st.mass_above;
+            uint32_t nt = st.n_eq;
+            if (m_tau > 0) {
+                const unsigned long long q = (need + m_tau - 1) / m_tau;
+                nt = (uint32_t)min((unsigned long long)st.n_eq, max(1ull, q));
+            }
+            st.n_tie = nt;
+            st.all_ties = (nt == st.n_eq) ? 1u : 0u;
+            st.kstar = st.count_above + nt;
+            const int bh = b * P.Hq + P.slot_head[slot];
+            if (P.dbg_tau) P.dbg_tau[bh] = key2f(st.tau_key);
+            if (P.dbg_kstar) P.dbg_kstar[bh] = (int32_t)st.kstar;
+            if (!st.all_ties) {
+                uint32_t run = 0;
+                for (int c = 0; c < nch; ++c) {
+                    P.tie_off[bs * P.nchunks + c] = run;
+                    run += P.chunk_cnt[(bs * P.nchunks + c) * 256 + dstar];
+                }
+            }
+        }
+        *hsp = st;
+        __threadfence();
+        atomicAdd(&SP.sync->pass_done[pass], 1u);
+    }
+}
+
+template <int G>
+__device__ void mark_item(const StepParams& SP, StepSmem<G>& S, int j, int tid) {
+    const Params& P = SP.P;
+    const int k = j / P.nchunks, chunk = j % P.nchunks;
+    const uint32_t e = __ldcg(SP.rlist + k);
+    const int b = (int)(e >> 16), slot = (int)(e & 0xFFFFu);
+    const int L = __ldg(P.seq_lens + b);
+    const int nch = (L + CHUNK - 1) / CHUNK;
+    if (chunk >= nch) return;
+    const int64_t bs = (int64_t)b * P.n_ret + slot;
+    HeadState st;
+    {
+        const HeadState* hsp = P.hs + bs;
+        st.tau_key = __ldcg(&hsp->tau_key);
+        st.all_ties = __ldcg(&hsp->all_ties);
+        st.n_tie = __ldcg(&hsp->n_tie);
+    }
+    const int n_begin = chunk * CHUNK, n_end = min(L, n_begin + CHUNK);
+    const uint32_t* keys = P.keys + bs * P.Ncap;
+    const uint32_t tau = st.tau_key;
+    const uint32_t tie_base = st.all_ties ? 0u : __ldcg(P.tie_off + bs * P.nchunks + chunk);
+    const int warp = tid >> 5, lane = tid & 31;
+    if (tid == 0) S.word = 0;
+    uint32_t carry = 0;
+    uint32_t mine = 0;
+    consumer_sync();
+    for (int base = n_begin; base < n_end; base += CONSUMERS) {
+        const int n = base + tid;
+        const uint32_t key = (n < n_end) ? __ldcg(keys + n) : 0u;
+        bool keep = (n < n_end) && key > tau;
+        const bool tie = (n < n_end) && key == tau;
+        if (st.all_ties) {
+            keep = keep || tie;
+        } else {
+            const uint32_t bal = __ballot_sync(0xffffffffu, tie);
+            if (lane == 0) S.w_key[0][warp] = __popc(bal);
+            consumer_sync();
+            uint32_t before = carry;
+            for (int w = 0; w < warp; ++w) before += S.w_key[0][w];
+            before += __popc(bal & ((1u << lane) - 1u));
+            keep = keep || (tie && tie_base + before < st.n_tie);
+            carry += S.w_key[0][0] + S.w_key[0][1] + S.w_key[0][2] + S.w_key[0][3];
+            consumer_sync();
+        }
+        if (keep) mine |= 1u << ((n - n_begin) / BLK);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mine |= __shfl_xor_sync(0xffffffffu, mine, o);
+    if (lane == 0 && mine) atomicOr(&S.word, mine);
+    consumer_sync();
+    if (tid == 0) P.bitmap[bs * P.words_cap + chunk] = S.word;
+    if (!consumer_last(P.tick_radix + bs, nch, &S.flag)) return;
+    if (tid == 0) {
+        __threadfence();
+        atomicAdd(&SP.sync->mark_done, 1u);
+    }
+}
+
+template <int G>
+__device__ void blist_item(const StepParams& SP, StepSmem<G>& S, int gi, int tid) {
+    const Params& P = SP.P;
+    const uint32_t e = __ldcg(SP.rglist + gi);
+    const int b = (int)(e >> 16), rgi = (int)(e & 0xFFFFu);
+    const int L = __ldg(P.seq_lens + b);
+    const int g = P.rg_group[rgi], nh = P.rg_nh[rgi], slot0 = P.rg_slot0[rgi];
+    const int nblk = (L + BLK - 1) / BLK;
+    const int nwords = (nblk + 31) / 32;
+    const int bg = b * P.n_rg + rgi;
+    uint32_t* list = P.blist + (int64_t)bg * P.nblk_cap;
+    const int warp = tid >> 5, lane = tid & 31;
+    __shared__ int s_kept[MAX_G];
+    __shared__ uint32_t s_base;
+    if (tid < MAX_G) s_kept[tid] = 0;
+    if (tid == 0) s_base = 0;
+    consumer_sync();
+    for (int w0 = 0; w0 < nwords; w0 += CONSUMERS) {
+        const int w = w0 + tid;
+        uint32_t uni = 0;
+        uint32_t wh[MAX_G];
+#pragma unroll
+        for (int hh = 0; hh < MAX_G; ++hh) {
+            wh[hh] = 0;
+            if (hh < nh && w < nwords) {
+                wh[hh] = __ldcg(P.bitmap + ((int64_t)b * P.n_ret + slot0 + hh) * P.words_cap + w);
+                if (w == nwords - 1 && (nblk & 31)) wh[hh] &= (1u << (nblk & 31)) - 1u;
+                uni |= wh[hh];
+                if (wh[hh]) atomicAdd(&s_kept[hh], __popc(wh[hh]));
+                if (P.dbg_bitmap)
+                    P.dbg_bitmap[((int64_t)b * P.Hq + P.slot_head[slot0 + hh]) * P.words_cap + w] = wh[hh];
+            }
+        }
+        const uint32_t c = __popc(uni);
+        uint32_t incl = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += t;
+        }
+        if (lane == 31) S.w_key[0][warp] = incl;
+        consumer_sync();
+        uint32_t off = s_base;
+        for (int ww = 0; ww < warp; ++ww) off += S.w_key[0][ww];
+        uint32_t pos = off + incl - c;
+        while (uni) {
+            const int jb = __ffs(uni) - 1;
+            uni &= uni - 1;
+            uint32_t hm = 0;
+#pragma unroll
+            for (int hh = 0; hh < MAX_G; ++hh)
+                if ((wh[hh] >> jb) & 1u) hm |= 1u << (P.slot_head[slot0 + hh] - g * P.G);
+            list[pos++] = ((uint32_t)(w * 32 + jb) << 8) | hm;
+        }
+        consumer_sync();
+        if (tid == 0) s_base += S.w_key[0][0] + S.w_key[0][1] + S.w_key[0][2] + S.w_key[0][3];
+        consumer_sync();
+    }
+    if (tid < nh && P.dbg_kept) P.dbg_kept[b * P.Hq + P.slot_head[slot0 + tid]] = s_kept[tid];
+    if (tid == 0) {
+        P.bcount[bg] = s_base;
+        __threadfence();
+        atomicAdd(&SP.sync->groups_ready, 1u);
+    }
+    consumer_sync();
+}
+
+// ===========================================================================
+// the persistent kernel
+// ===========================================================================
+template <int G>
+__device__ void producer(const StepParams& SP, StepSmem<G>& S) {
+    constexpr int NST = StepSmem<G>::NST;
+    const Params& P = SP.P;
+    Sync* sy = SP.sync;
+    uint32_t t = 0;   // tiles published so far (same sequence the consumers follow)
+    bool alive = true;
+
+    auto acquire = [&]() -> int {
+        const int st = (int)(t % NST);
+        const uint32_t round = t / NST;
+        if (round > 0 && !mbar_wait_bounded(&S.empty[st], (round - 1) & 1u)) {
+            set_status(P, ST_TIMEOUT);
+            alive = false;
+        }
+        return st;
+    };
+    auto publish_nodata = [&](const Desc& d) {
+        const int st = acquire();
+        if (!alive) return;
+        S.desc[st] = d;
+        mbar_arrive(&S.full[st]);
+        ++t;
+    };
+    auto wait_for = [&](const uint32_t* ctr, uint32_t target) {
+        if (alive && !wait_counter(ctr, target)) {
+            set_status(P, ST_TIMEOUT);
+            alive = false;
+        }
+    };
+
+    const int n_static = SP.n_score_items + SP.n_local_items;
+    uint32_t x = atomicAdd(&sy->queue, 1u);
+    while (alive && (int)x < n_static) {
+        if ((int)x < SP.n_score_items) {
+            // ---- index-score chunk (b, rgi, chunk) ----
+            const int per_b = P.n_rg * P.nchunks;
+            const int b = (int)x / per_b, rgi = ((int)x % per_b) / P.nchunks, chunk = (int)x % P.nchunks;
+            const int L = __ldg(P.seq_lens + b);
+            if (!seq_ok(P, L)) {
+                if (chunk == 0) {   // this sequence's groups: no selection, no blocks
+                    set_status(P, ST_DEVICE_INPUT);
+                    P.bcount[b * P.n_rg + rgi] = 0;
+                    __threadfence();
+                    atomicAdd(&sy->groups_decided, 1u);
+                    atomicAdd(&sy->groups_ready, 1u);
+                }
+            } else {
+                const int nch = (L + CHUNK - 1) / CHUNK;
+                if (chunk < nch) {
+                    const int g = P.rg_group[rgi];
+                    const int n_begin = chunk * CHUNK, n_end = min(L, n_begin + CHUNK);
+                    const int ntiles = (n_end - n_begin + SCORE_ROWS - 1) / SCORE_ROWS;
+                    for (int ti = 0; ti < ntiles && alive; ++ti) {
+                        const int n0 = n_begin + ti * SCORE_ROWS;
+                        const int nvalid = min(SCORE_ROWS, n_end - n0);
+                        const int nblocks = (nvalid + BLK - 1) / BLK;
+                        const int st = acquire();
+                        if (!alive) break;
+                        Desc d;
+                        d.type = IT_SCORE;
+                        d.b = b;
+                        d.grp = rgi;
+                        d.item = chunk;
+                        d.tile = ti;
+                        d.ntiles = ntiles;
+                        d.n0 = n0;
+                        d.nvalid = nvalid;
+                        d.hmask = 0;
+                        d.aux0 = nch;
+                        d.aux1 = L;
+                        d.bad = 0;
+                        S.desc[st] = d;
+                        mbar_expect_tx(&S.full[st], (uint32_t)nblocks * BLK * R * 2);
+                        if (P.block_table == nullptr) {
+                            const uint16_t* src = P.k_idx + (((int64_t)b * P.Hkv + g) * P.Ncap + n0) * R;
+                            bulk_g2s(&S.stage[st][0], src, (uint32_t)nblocks * BLK * R * 2, &S.full[st]);
+                        } else {
+                            for (int q = 0; q < nblocks; ++q) {
+                                int bad = 0;
+                                const int64_t off = tile_off(P, b, g, n0 / BLK + q, R, &bad);
+                                if (bad) set_status(P, ST_DEVICE_INPUT);
+                                bulk_g2s(&S.stage[st][q * BLK * R * 2], P.k_idx + off, BLK * R * 2, &S.full[st]);
+                            }
+                        }
+                        ++t;
+                    }
+                }
+            }
+        } else {
+            // ---- local-head item (b, lgi, item) ----
+            const int y = (int)x - SP.n_score_items;
+            const int per_b = P.n_lg * P.local_items;
+            const int b = y / per_b, lgi = (y % per_b) / P.local_items, item = y % P.local_items;
+            const int L = __ldg(P.seq_lens + b);
+            if (seq_ok(P, L)) {
+                const LocalGeom lg = local_geom(P, L);
+                const int nitems = (lg.nv + P.local_kb - 1) / P.local_kb;
+                if (item < nitems) {
+                    const int g = P.lg_group[lgi];
+                    const int v0 = item * P.local_kb, ntiles = min(P.local_kb, lg.nv - v0);
+                    for (int i = 0; i < ntiles && alive; ++i) {
+                        const int v = v0 + i;
+                        const int j = v < lg.nA ? v : lg.bw0 + (v - lg.nA);
+                        const int st = acquire();
+                        if (!alive) break;
+                        Desc d;
+                        d.type = IT_LOCAL;
+                        d.b = b;
+                        d.grp = lgi;
+                        d.item = item;
+                        d.tile = i;
+                        d.ntiles = ntiles;
+                        d.n0 = j * BLK;
+                        d.nvalid = min(BLK, L - j * BLK);
+                        d.hmask = P.lg_mask[lgi];
+                        d.aux0 = nitems;
+                        d.aux1 = L;
+                        d.bad = 0;
+                        const int64_t off = tile_off(P, b, g, j, D, &d.bad);
+                        S.desc[st] = d;
+                        mbar_expect_tx(&S.full[st], STAGE_BYTES);
+                        bulk_g2s(&S.stage[st][0], P.k_cache + off, TILE_BYTES, &S.full[st]);
+                        bulk_g2s(&S.stage[st][TILE_BYTES], P.v_cache + off, TILE_BYTES, &S.full[st]);
+                        ++t;
+                    }
+                }
+            }
+        }
+        x = atomicAdd(&sy->queue, 1u);
+    }
+
+    // ---- retrieval heads: finish the selection, then their tiles ----
+    if (alive && P.n_rg > 0) {
+        const uint32_t ngroups = (uint32_t)(P.B * P.n_rg);
+        wait_for(&sy->groups_decided, ngroups);
+        const uint32_t nrad = alive ? ld_acquire(&sy->n_radix_heads) : 0u;
+        if (nrad > 0) {
+            const uint32_t nitems = nrad * (uint32_t)P.nchunks;
+            for (int pass = 0; pass < 4 && alive; ++pass) {
+                for (uint32_t j = atomicAdd(&sy->pass_claim[pass], 1u); j < nitems && alive;
+                     j = atomicAdd(&sy->pass_claim[pass], 1u)) {
+                    Desc d{};
+                    d.type = IT_RADIX;
+                    d.item = (int)j;
+                    d.aux0 = pass;
+                    publish_nodata(d);
+                }
+                wait_for(&sy->pass_done[pass], nrad);
+            }
+            for (uint32_t j = atomicAdd(&sy->mark_claim, 1u); j < nitems && alive; j = atomicAdd(&sy->mark_claim, 1u)) {
+                Desc d{};
+                d.type = IT_MARK;
+                d.item = (int)j;
+                publish_nodata(d);
+            }
+            wait_for(&sy->mark_done, nrad);
+            const uint32_t ngr = alive ? ld_acquire(&sy->n_radix_groups) : 0u;
+            for (uint32_t j = atomicAdd(&sy->blist_claim, 1u); j < ngr && alive; j = atomicAdd(&sy->blist_claim, 1u)) {
+                Desc d{};
+                d.type = IT_BLIST;
+                d.item = (int)j;
+                publish_nodata(d);
+            }
+        }
+        wait_for(&sy->groups_ready, ngroups);
+        if (alive) {
+            // blocks per retrieval item, chosen so that the items about fill the grid
+            long long total = 0;
+            for (int bg = 0; bg < (int)ngroups; ++bg)
+                if (seq_ok(P, __ldg(P.seq_lens + bg / P.n_rg))) total += __ldcg(P.bcount + bg);
+            const int KB = (int)max(1ll, (total + gridDim.x - 1) / gridDim.x);
+            int r = (int)x - n_static;
+            // walk the (b, group) segments in order; r only grows
+            int bg = 0, seg_base = 0, seg_items = 0, cnt = 0, L = 0;
+            auto load_seg = [&]() {
+                const int b = bg / P.n_rg;
+                L = __ldg(P.seq_lens + b);
+                cnt = seq_ok(P, L) ? (int)__ldcg(P.bcount + bg) : 0;
+                seg_items = (cnt + KB - 1) / KB;
+            };
+            load_seg();
+            while (alive) {
+                while (bg < (int)ngroups && r >= seg_base + seg_items) {
+                    seg_base += seg_items;
+                    ++bg;
+                    if (bg < (int)ngroups) load_seg();
+                }
+                if (bg >= (int)ngroups) break;
+                const int b = bg / P.n_rg, rgi = bg % P.n_rg, g = P.rg_group[rgi];
+                const int it = r - seg_base;
+                const int k0 = it * KB, ntiles = min(KB, cnt - k0);
+                const uint32_t* list = P.blist + (int64_t)bg * P.nblk_cap;
+                for (int i = 0; i < ntiles && alive; ++i) {
+                    const uint32_t e = __ldcg(list + k0 + i);
+                    const int j = (int)(e >> 8);
+                    const int st = acquire();
+                    if (!alive) break;
+                    Desc d;
+                    d.type = IT_RET;
+                    d.b = b;
+                    d.grp = rgi;
+                    d.item = it;
+                    d.tile = i;
+                    d.ntiles = ntiles;
+                    d.n0 = j * BLK;
+                    d.nvalid = min(BLK, L - j * BLK);
+                    d.hmask = e & 0xFFu;
+                    d.aux0 = seg_base;   // partial slot of the group's first item
+                    d.aux1 = seg_items;
+                    d.bad = 0;
+                    const int64_t off = tile_off(P, b, g, j, D, &d.bad);
+                    S.desc[st] = d;
+                    mbar_expect_tx(&S.full[st], STAGE_BYTES);
+                    bulk_g2s(&S.stage[st][0], P.k_cache + off, TILE_BYTES, &S.full[st]);
+                    bulk_g2s(&S.stage[st][TILE_BYTES], P.v_cache + off, TILE_BYTES, &S.full[st]);
+                    ++t;
+                }
+                r = (int)atomicAdd(&sy->queue, 1u) - n_static;
+            }
+        }
+    }
+    Desc d{};
+    d.type = IT_STOP;
+    publish_nodata(d);
+    // never leave the CTA with copies in flight: wait (bounded) for the last
+    // tile published into each stage to have landed
+    for (uint32_t i = (t > (uint32_t)NST ? t - NST : 0u); i < t; ++i)
+        mbar_wait_bounded(&S.full[i % NST], (i / NST) & 1u);
+}
+
+template <int G>
+__device__ void consumers(const StepParams& SP, StepSmem<G>& S, int tid) {
+    constexpr int NST = StepSmem<G>::NST;
+    const Params& P = SP.P;
+    AttnCore<G> core;
+    ScoreState<G> sc;
+    uint32_t t = 0;
+    const int warp = tid >> 5, lane = tid & 31;
+    while (true) {
+        const int st = (int)(t % NST);
+        const uint32_t par = (t / NST) & 1u;
+        if (!mbar_wait_bounded(&S.full[st], par)) {
+            set_status(P, ST_TIMEOUT);
+            break;
+        }
+        const Desc d = S.desc[st];
+        const uint8_t* data = &S.stage[st][0];
+        ++t;
+        if (d.type == IT_STOP) break;
+        if (d.type == IT_SCORE) {
+            if (d.tile == 0) score_begin<G>(P, S, sc, d.b, d.grp, tid);
+            score_tile<G>(P, S, sc, data, d.b, d.grp, d.n0, d.nvalid, tid);
+            consumer_sync();
+            if (lane == 0) mbar_arrive(&S.empty[st]);
+            if (d.tile == d.ntiles - 1) score_end<G>(SP, S, sc, d.b, d.grp, d.item, d.aux1, d.aux0, tid);
+            continue;
+        }
+        if (d.type == IT_LOCAL || d.type == IT_RET) {
+            const bool local = d.type == IT_LOCAL;
+            const int g = local ? P.lg_group[d.grp] : P.rg_group[d.grp];
+            if (d.tile == 0) core.begin(P, S, d.b, g, tid);
+            if (d.bad) {
+                if (tid == 0) set_status(P, ST_DEVICE_INPUT);
+            } else {
+                int s_end = 0, w_lo = 0;
+                if (local) {
+                    const LocalGeom lg = local_geom(P, d.aux1);
+                    s_end = lg.s_end;
+                    w_lo = lg.w_lo;
+                }
+                core.tile(S, data, d.hmask, d.n0, d.nvalid, local, s_end, w_lo, tid);
+            }
+            if (lane == 0) mbar_arrive(&S.empty[st]);
+            if (d.tile == d.ntiles - 1) {
+                float* parts;
+                uint32_t heads, *ctr;
+                int nitems;
+                if (local) {
+                    parts = P.lpart + (((int64_t)d.b * P.n_lg + d.grp) * P.local_items) * G * PSTRIDE;
+                    heads = P.lg_mask[d.grp];
+                    ctr = P.tick_local + d.b * P.n_lg + d.grp;
+                    nitems = d.aux0;
+                } else {
+                    parts = P.rpart + (int64_t)d.aux0 * G * PSTRIDE;
+                    heads = P.rg_mask[d.grp];
+                    ctr = P.tick_ret + d.b * P.n_rg + d.grp;
+                    nitems = d.aux1;
+                }
+                core.flush(S, parts + (int64_t)d.item * G * PSTRIDE, heads, tid);
+                if (consumer_last(ctr, nitems, &S.flag)) {
+                    __threadfence();
+                    combine_parts<G>(P, S, parts, nitems, heads, d.b, g, tid);
+                }
+            }
+            continue;
+        }
+        // data-less items: release the slot first
+        consumer_sync();
+        if (lane == 0) mbar_arrive(&S.empty[st]);
+        if (d.type == IT_RADIX) radix_item<G>(SP, S, d.item, d.aux0, tid);
+        else if (d.type == IT_MARK) mark_item<G>(SP, S, d.item, tid);
+        else if (d.type == IT_BLIST) blist_item<G>(SP, S, d.item, tid);
+    }
+    (void)warp;
+}
+
+template <int G>
+__global__ void __launch_bounds__(STEP_THREADS) step_kernel(const __grid_constant__ StepParams SP) {
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    StepSmem<G>& S = *reinterpret_cast<StepSmem<G>*>(smem_raw);
+    constexpr int NST = StepSmem<G>::NST;
+    const int tid = threadIdx.x;
+    if (tid == 0) {
+        for (int i = 0; i < NST; ++i) {
+            mbar_init(&S.full[i], 1);
+            mbar_init(&S.empty[i], CONSUMERS / 32);
+        }
+        mbar_fence_init();
+    }
+    __syncthreads();
+    if (tid >= CONSUMERS) {
+        if (tid == CONSUMERS) producer<G>(SP, S);
+        return;
+    }
+    consumers<G>(SP, S, tid);
+    // last CTA out clears the coordination words for the next call
+    consumer_sync();
+    if (tid == 0) {
+        __threadfence();
+        if (atomicAdd(&SP.sync->exit_count, 1u) == gridDim.x - 1) {
+            uint32_t* w = reinterpret_cast<uint32_t*>(SP.sync);
+            for (int i = 0; i < (int)(sizeof(Sync) / 4); ++i) atomicExch(w + i, 0u);
+            __threadfence();
+        }
+    }
+}
+
+}  // namespace rtp

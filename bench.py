@@ -270,6 +270,22 @@ def main():
     phase_ms = {n: phase_acc[k] / args.steps for k, n in enumerate(rtp.PHASES)}
     t_ms = statistics.mean(step_ms)
 
+    # ---- timeline of one step (debug trace, separate untimed replays) ----
+    trace_buf = torch.zeros(16, dtype=torch.int64, device=dev)
+    tdbg = rtp.RtpDebug(trace=trace_buf.data_ptr())
+    dc.step.dims.debug = ctypes.pointer(tdbg)
+    tl = []
+    for _ in range(5):
+        flush()
+        trace_buf.zero_()
+        dc.run(stream)
+        torch.cuda.synchronize(dev)
+        t = trace_buf.cpu().numpy().astype(np.float64)
+        tl.append({n: (t[k] - t[0]) / 1e3 if t[k] > 0 else None for k, n in enumerate(rtp.TRACE_EVENTS) if k})
+    dc.step.dims.debug = ctypes.POINTER(rtp.RtpDebug)()
+    timeline = {n: (statistics.median([x[n] for x in tl]) if tl[0][n] is not None else None)
+                for n in tl[0]}
+
     # ---- end to end: host query/len/p -> device, step, output -> host ----
     hq_pre = torch.from_numpy(case.q_pre.view(np.int16)).view(torch.bfloat16).pin_memory()
     hq_rope = torch.from_numpy(case.q_rope.view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -345,6 +361,7 @@ def main():
             "step_roofline": {"algorithmic_bytes": nbytes, "achieved": step_gbs, "peak": peak, "unit": "GB/s",
                               "frac": step_gbs / peak},
             "phases_us": {n: phase_ms[n] * 1e3 for n in rtp.PHASES},
+            "timeline_us": timeline,
             "sparsity": {"kept_token_frac": kept_tokens, "kept_block_frac": kept_blocks},
             "e2e": {"value": world * tokens / (e2e_t * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "us_per_step": e2e_t * 1e3},

@@ -30,7 +30,12 @@ class RtpError(RuntimeError):
 
 class RtpDebug(ctypes.Structure):
     _fields_ = [("tau", ctypes.c_void_p), ("kstar", ctypes.c_void_p), ("kept_blocks", ctypes.c_void_p),
-                ("smax", ctypes.c_void_p), ("Z", ctypes.c_void_p), ("block_bitmap", ctypes.c_void_p)]
+                ("smax", ctypes.c_void_p), ("Z", ctypes.c_void_p), ("block_bitmap", ctypes.c_void_p),
+                ("trace", ctypes.c_void_p)]
+
+
+TRACE_EVENTS = ["start", "select_done", "local_done", "lists_ready", "retrieval_done", "end", "select_start",
+                "local_combine_start", "radix1", "radix2", "radix3", "radix4", "mark", "t13", "t14", "t15"]
 
 
 class RtpDims(ctypes.Structure):

@@ -25,9 +25,16 @@ enum SelMode : int32_t { MODE_SKIP = 0, MODE_TOP1 = 1, MODE_ALL = 2, MODE_RADIX 
 constexpr uint32_t ST_DEVICE_INPUT = 6;
 constexpr uint32_t ST_TIMEOUT = 7;
 
-struct ChunkStat {
-    uint32_t maxkey, argmax, minkey, pad;
-    double sum;   // sum over the chunk of exp((s - s(maxkey))/4)
+// Per retrieval head and bucket (chunk mod AGG_BUCKETS), folded by score
+// chunks with atomics (all-zero = empty, so a zero-filled workspace is
+// ready): best = (max key << 32) | ~argmax, nmin = ~(min key), ms = (key of
+// the reference score << 32) | fp32 sum of exp((s - ref)/4), the reference
+// being the bucket's max score.  Buckets keep same-address atomics rare.
+constexpr int AGG_BUCKETS = 32;
+struct HeadAgg {
+    unsigned long long best;
+    uint32_t nmin, pad;
+    unsigned long long ms;
 };
 
 struct HeadState {
@@ -56,7 +63,7 @@ struct Params {
     uint32_t* status;
     uint32_t *tick_score, *tick_radix, *tick_local, *tick_ret;
     uint32_t* keys;
-    ChunkStat* cstat;
+    HeadAgg* agg;
     HeadState* hs;
     uint32_t* hist_cnt;
     unsigned long long* hist_mass;
@@ -74,6 +81,7 @@ struct Params {
     float* dbg_smax;
     double* dbg_Z;
     uint32_t* dbg_bitmap;
+    unsigned long long* dbg_trace;
 };
 
 // ---------------------------------------------------------------------------

@@ -23,7 +23,7 @@ struct Plan {
     uint8_t lg_group[MAX_HKV], lg_mask[MAX_HKV];
     uint8_t slot_head[MAX_HQ], slot_rg[MAX_HQ];
     // workspace byte offsets
-    size_t o_status, o_sync, o_rlist, o_rglist, o_tick_score, o_tick_radix, o_tick_local, o_tick_ret, o_keys, o_cstat,
+    size_t o_status, o_sync, o_rlist, o_rglist, o_tick_score, o_tick_radix, o_tick_local, o_tick_ret, o_keys, o_agg,
         o_hs, o_hist_cnt, o_hist_mass, o_chunk_cnt, o_tie_off, o_bitmap, o_blist, o_bcount, o_lpart, o_rpart, total;
 };
 
@@ -113,7 +113,7 @@ static rtp_status make_plan(const rtp_dims* d, const uint8_t* head_kind, int win
     pl->o_tick_local = take(BL * 4);
     pl->o_tick_ret = take(BG * 4);
     pl->o_keys = take(BR * pl->Ncap * 4);
-    pl->o_cstat = take(BR * pl->nchunks * sizeof(ChunkStat));
+    pl->o_agg = take(BR * AGG_BUCKETS * sizeof(HeadAgg));
     pl->o_hs = take(BR * sizeof(HeadState));
     pl->o_hist_cnt = take(BR * 256 * 4);
     pl->o_hist_mass = take(BR * 256 * 8);
@@ -232,7 +232,7 @@ extern "C" rtp_status rtp_decode_step(const rtp_dims* dims, const uint16_t* q_pr
     P.tick_local = (uint32_t*)(ws + pl.o_tick_local);
     P.tick_ret = (uint32_t*)(ws + pl.o_tick_ret);
     P.keys = (uint32_t*)(ws + pl.o_keys);
-    P.cstat = (ChunkStat*)(ws + pl.o_cstat);
+    P.agg = (HeadAgg*)(ws + pl.o_agg);
     P.hs = (HeadState*)(ws + pl.o_hs);
     P.hist_cnt = (uint32_t*)(ws + pl.o_hist_cnt);
     P.hist_mass = (unsigned long long*)(ws + pl.o_hist_mass);
@@ -250,6 +250,7 @@ extern "C" rtp_status rtp_decode_step(const rtp_dims* dims, const uint16_t* q_pr
         P.dbg_smax = dims->debug->smax;
         P.dbg_Z = dims->debug->Z;
         P.dbg_bitmap = dims->debug->block_bitmap;
+        P.dbg_trace = dims->debug->trace;
     }
     cudaStream_t s = (cudaStream_t)stream;
     void* const* ev = (dims->timing_events && dims->n_timing_events >= RTP_TIMING_EVENTS) ? dims->timing_events : nullptr;

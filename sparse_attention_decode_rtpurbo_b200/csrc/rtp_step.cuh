@@ -64,13 +64,15 @@ struct Desc {
 
 template <int G>
 struct StepSmem {
-    static constexpr int NST = (G >= 8) ? 2 : STAGES;
+    // G = 8 runs one CTA per SM (register bound), so it gets a deeper ring
+    static constexpr int NST = (G >= 8) ? 4 : STAGES;
     alignas(128) uint8_t stage[NST][STAGE_BYTES];
     alignas(16) float red[4][G][D];   // per-warp partial sums of the attention accumulators; combine scratch
     alignas(16) float prob[BLK][G];
     float m_run[G], l_run[G], alpha[G];
     alignas(16) float qi[G][R];
     uint32_t hcnt[256];
+    uint32_t hm[3][256];   // 17-bit slices of the per-bin fixed-point mass
     unsigned long long hmass[256];
     Desc desc[NST];
     alignas(8) uint64_t full[NST], empty[NST];
@@ -102,6 +104,11 @@ __device__ __forceinline__ bool wait_counter(const uint32_t* p, uint32_t target)
         if (ld_acquire(p) >= target) return true;
         if (global_ns() - t0 > 2000000000ull) return false;
     }
+}
+
+// optional timeline (debug): latest %globaltimer of event i
+__device__ __forceinline__ void trace_max(const Params& P, int i) {
+    if (P.dbg_trace) atomicMax(P.dbg_trace + i, (unsigned long long)global_ns());
 }
 
 // Ticket among CONSUMER threads: true in exactly one of `count` arrivals.

@@ -77,13 +77,33 @@ __device__ void score_tile(const Params& P, StepSmem<G>& S, ScoreState<G>& st, c
                 st.am[hh] = (uint32_t)n;
             }
             st.nk[hh] = min(st.nk[hh], key);
+            constexpr float C = 0.25f * 1.4426950408889634f;   // (1/4) log2(e)
             if (s > st.ms[hh]) {
-                st.sm[hh] = st.sm[hh] * expf((st.ms[hh] - s) * 0.25f) + 1.f;
+                st.sm[hh] = st.sm[hh] * exp2f((st.ms[hh] - s) * C) + 1.f;
                 st.ms[hh] = s;
             } else {
-                st.sm[hh] += expf((s - st.ms[hh]) * 0.25f);
+                st.sm[hh] += exp2f((s - st.ms[hh]) * C);
             }
         }
+    }
+}
+
+// fold (max key a, running sum sa relative to score key ka) with (b, sb, kb):
+// keys order-preserving; key 0 marks an empty accumulator
+__device__ __forceinline__ void fold_ms(uint32_t& ka, float& sa, uint32_t kb, float sb) {
+    if (kb == 0u) return;
+    if (ka == 0u) {
+        ka = kb;
+        sa = sb;
+        return;
+    }
+    constexpr float C = 0.25f * 1.4426950408889634f;   // (1/4) log2(e)
+    const float ma = key2f(ka), mb = key2f(kb);
+    if (mb > ma) {
+        sa = sa * exp2f((ma - mb) * C) + sb;
+        ka = kb;
+    } else {
+        sa += sb * exp2f((mb - ma) * C);
     }
 }
 
@@ -94,62 +114,54 @@ template <int G>
 __device__ void score_decide(const StepParams& SP, StepSmem<G>& S, int b, int rgi, int L, int nch, int tid) {
     const Params& P = SP.P;
     const int nh = P.rg_nh[rgi], slot0 = P.rg_slot0[rgi], g = P.rg_group[rgi];
-    const int warp = tid >> 5, lane = tid & 31;
     const int nblk = (L + BLK - 1) / BLK;
     const int nwords = (nblk + 31) / 32;
     __shared__ int s_mode[MAX_G];
     __shared__ uint32_t s_arg[MAX_G];
-    for (int hh = 0; hh < nh; ++hh) {
+    // every chunk of the group has folded its partials into its heads'
+    // buckets (score_end): one warp per head reduces the 32 buckets and
+    // re-arms them for the next call
+    __shared__ unsigned long long s_best[MAX_G], s_ms[MAX_G];
+    __shared__ uint32_t s_nmin[MAX_G];
+    {
+        const int warp = tid >> 5, lane = tid & 31;
+        for (int hh = warp; hh < nh; hh += CONSUMERS / 32) {
+            HeadAgg* ag = P.agg + ((int64_t)b * P.n_ret + slot0 + hh) * AGG_BUCKETS + lane;
+            unsigned long long best = __ldcg(&ag->best);
+            uint32_t nmin = __ldcg(&ag->nmin);
+            const unsigned long long ms = __ldcg(&ag->ms);
+            uint32_t km = (uint32_t)(ms >> 32);
+            float su = __uint_as_float((uint32_t)(ms & 0xFFFFFFFFull));
+            ag->best = 0ull;
+            ag->nmin = 0u;
+            ag->ms = 0ull;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                best = max(best, __shfl_xor_sync(0xffffffffu, best, o));
+                nmin = max(nmin, __shfl_xor_sync(0xffffffffu, nmin, o));
+                const uint32_t km2 = __shfl_xor_sync(0xffffffffu, km, o);
+                const float s2 = __shfl_xor_sync(0xffffffffu, su, o);
+                fold_ms(km, su, km2, s2);
+            }
+            if (lane == 0) {
+                s_best[hh] = best;
+                s_nmin[hh] = nmin;
+                s_ms[hh] = ((unsigned long long)km << 32) | __float_as_uint(su);
+            }
+        }
+    }
+    consumer_sync();
+    if (tid < nh) {
+        const int hh = tid;
         const int slot = slot0 + hh;
-        const ChunkStat* cs = P.cstat + ((int64_t)b * P.n_ret + slot) * P.nchunks;
-        uint32_t k = 0, a = 0xFFFFFFFFu, mn = 0xFFFFFFFFu;
-        for (int c = tid; c < nch; c += CONSUMERS) {
-            const ChunkStat x = cs[c];
-            if (x.maxkey > k || (x.maxkey == k && x.argmax < a)) {
-                k = x.maxkey;
-                a = x.argmax;
-            }
-            mn = min(mn, x.minkey);
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const uint32_t k2 = __shfl_xor_sync(0xffffffffu, k, o);
-            const uint32_t a2 = __shfl_xor_sync(0xffffffffu, a, o);
-            mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-            if (k2 > k || (k2 == k && a2 < a)) {
-                k = k2;
-                a = a2;
-            }
-        }
-        if (lane == 0) {
-            S.w_key[0][warp] = k;
-            S.w_arg[0][warp] = a;
-            S.w_min[0][warp] = mn;
-        }
-        consumer_sync();
-        k = S.w_key[0][0];
-        a = S.w_arg[0][0];
-        mn = S.w_min[0][0];
-        for (int w = 1; w < 4; ++w) {
-            if (S.w_key[0][w] > k || (S.w_key[0][w] == k && S.w_arg[0][w] < a)) {
-                k = S.w_key[0][w];
-                a = S.w_arg[0][w];
-            }
-            mn = min(mn, S.w_min[0][w]);
-        }
+        const unsigned long long best = s_best[hh];
+        const uint32_t k = (uint32_t)(best >> 32);
+        const uint32_t a = 0xFFFFFFFFu - (uint32_t)(best & 0xFFFFFFFFull);
+        const uint32_t mn = ~s_nmin[hh];
         const float smax = key2f(k);
-        double su = 0.0;
-        for (int c = tid; c < nch; c += CONSUMERS) {
-            const ChunkStat x = cs[c];
-            su += x.sum * exp(((double)key2f(x.maxkey) - (double)smax) * 0.25);
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) su += __shfl_xor_sync(0xffffffffu, su, o);
-        consumer_sync();
-        if (lane == 0) S.w_sum[0][warp] = su;
-        consumer_sync();
-        if (tid == 0) {
-            const double z = S.w_sum[0][0] + S.w_sum[0][1] + S.w_sum[0][2] + S.w_sum[0][3];
+        // the folded sum's reference is the head's max score, i.e. smax
+        const double z = (double)__uint_as_float((uint32_t)(s_ms[hh] & 0xFFFFFFFFull));
+        {
             const float pb = __ldg(P.p + b);
             HeadState h;
             h.smax = smax;
@@ -175,7 +187,7 @@ __device__ void score_decide(const StepParams& SP, StepSmem<G>& S, int b, int rg
                 h.mode = MODE_ALL;
                 h.kstar = (uint32_t)L;
                 h.tau_key = mn;
-            } else if (1.0 >= (double)pb * z * (1.0 + 1e-6)) {
+            } else if (1.0 >= (double)pb * z * (1.0 + 1e-3)) {
                 h.mode = MODE_TOP1;   // the best token alone reaches p
                 h.kstar = 1;
                 h.tau_key = k;
@@ -196,13 +208,13 @@ __device__ void score_decide(const StepParams& SP, StepSmem<G>& S, int b, int rg
             s_mode[hh] = h.mode;
             s_arg[hh] = a;
         }
-        // the radix histogram of this head starts at zero
-        for (int d = tid; d < 256; d += CONSUMERS) {
-            P.hist_cnt[((int64_t)b * P.n_ret + slot) * 256 + d] = 0;
-            P.hist_mass[((int64_t)b * P.n_ret + slot) * 256 + d] = 0ull;
-        }
-        consumer_sync();
     }
+    // the radix histograms of these heads start at zero
+    for (int x = tid; x < nh * 256; x += CONSUMERS) {
+        P.hist_cnt[((int64_t)b * P.n_ret + slot0) * 256 + x] = 0;
+        P.hist_mass[((int64_t)b * P.n_ret + slot0) * 256 + x] = 0ull;
+    }
+    consumer_sync();
 
     bool any_radix = false, any_all = false;
     uint32_t all_mask = 0;
@@ -287,6 +299,7 @@ __device__ void score_decide(const StepParams& SP, StepSmem<G>& S, int b, int rg
         __threadfence();
         atomicAdd(&SP.sync->groups_decided, 1u);
         atomicAdd(&SP.sync->groups_ready, 1u);
+        trace_max(P, 3);
     }
 }
 
@@ -300,58 +313,61 @@ __device__ void score_end(const StepParams& SP, StepSmem<G>& S, ScoreState<G>& s
     for (int hh = 0; hh < G; ++hh) {
         if (hh >= nh) break;
         uint32_t k = st.mk[hh], a = st.am[hh], mn = st.nk[hh];
-        float m = st.ms[hh];
-        double su = (double)st.sm[hh];
+        uint32_t km = st.mk[hh];   // the running sum is relative to the max score, whose key is mk
+        float su = st.sm[hh];
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
             const uint32_t k2 = __shfl_xor_sync(0xffffffffu, k, o);
             const uint32_t a2 = __shfl_xor_sync(0xffffffffu, a, o);
-            const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
-            const double s2 = __shfl_xor_sync(0xffffffffu, su, o);
+            const uint32_t km2 = __shfl_xor_sync(0xffffffffu, km, o);
+            const float s2 = __shfl_xor_sync(0xffffffffu, su, o);
             mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
             if (k2 > k || (k2 == k && a2 < a)) {
                 k = k2;
                 a = a2;
             }
-            const float mm = fmaxf(m, m2);
-            su = (mm == -INFINITY) ? 0.0 : su * exp((double)(m - mm) * 0.25) + s2 * exp((double)(m2 - mm) * 0.25);
-            m = mm;
+            fold_ms(km, su, km2, s2);
         }
         if (lane == 0) {
             S.w_key[hh][warp] = k;
             S.w_arg[hh][warp] = a;
             S.w_min[hh][warp] = mn;
-            S.w_m[hh][warp] = m;
-            S.w_sum[hh][warp] = su;
+            S.w_m[hh][warp] = __uint_as_float(km);
+            S.w_sum[hh][warp] = (double)su;
         }
     }
     consumer_sync();
     if (tid < nh) {
         const int hh = tid;
-        uint32_t k = 0, a = 0xFFFFFFFFu, mn = 0xFFFFFFFFu;
-        float m = -INFINITY;
+        uint32_t k = 0, a = 0xFFFFFFFFu, mn = 0xFFFFFFFFu, km = 0;
+        float su = 0.f;
         for (int w = 0; w < 4; ++w) {
             if (S.w_key[hh][w] > k || (S.w_key[hh][w] == k && S.w_arg[hh][w] < a)) {
                 k = S.w_key[hh][w];
                 a = S.w_arg[hh][w];
             }
             mn = min(mn, S.w_min[hh][w]);
-            m = fmaxf(m, S.w_m[hh][w]);
+            fold_ms(km, su, __float_as_uint(S.w_m[hh][w]), (float)S.w_sum[hh][w]);
         }
-        double su = 0.0;
-        for (int w = 0; w < 4; ++w)
-            if (S.w_m[hh][w] != -INFINITY) su += S.w_sum[hh][w] * exp((double)(S.w_m[hh][w] - m) * 0.25);
-        ChunkStat cs;
-        cs.maxkey = k;
-        cs.argmax = a;
-        cs.minkey = mn;
-        cs.pad = 0;
-        cs.sum = su;
-        P.cstat[((int64_t)b * P.n_ret + slot0 + hh) * P.nchunks + chunk] = cs;
+        // fold this chunk into its bucket of the head's aggregate
+        HeadAgg* ag = P.agg + ((int64_t)b * P.n_ret + slot0 + hh) * AGG_BUCKETS + (chunk % AGG_BUCKETS);
+        atomicMax(&ag->best, ((unsigned long long)k << 32) | (0xFFFFFFFFu - a));
+        atomicMax(&ag->nmin, ~mn);
+        unsigned long long old = __ldcg(&ag->ms), assumed;
+        do {
+            assumed = old;
+            uint32_t ka = (uint32_t)(assumed >> 32);
+            float sa = __uint_as_float((uint32_t)(assumed & 0xFFFFFFFFull));
+            fold_ms(ka, sa, km, su);
+            const unsigned long long nv = ((unsigned long long)ka << 32) | __float_as_uint(sa);
+            old = atomicCAS(&ag->ms, assumed, nv);
+        } while (old != assumed);
     }
     if (!consumer_last(P.tick_score + b * P.n_rg + rgi, nch, &S.flag)) return;
     __threadfence();
+    if (tid == 0) trace_max(P, 6);
     score_decide<G>(SP, S, b, rgi, L, nch, tid);
+    if (tid == 0) trace_max(P, 1);
 }
 
 // ===========================================================================
@@ -370,7 +386,9 @@ __device__ void radix_item(const StepParams& SP, StepSmem<G>& S, int j, int pass
     HeadState* hsp = P.hs + bs;
     for (int d = tid; d < 256; d += CONSUMERS) {
         S.hcnt[d] = 0;
-        S.hmass[d] = 0ull;
+        S.hm[0][d] = 0;
+        S.hm[1][d] = 0;
+        S.hm[2][d] = 0;
     }
     consumer_sync();
     const uint32_t prefix = __ldcg(&hsp->prefix);
@@ -378,13 +396,42 @@ __device__ void radix_item(const StepParams& SP, StepSmem<G>& S, int j, int pass
     const int shift = 24 - 8 * pass;
     const int n_begin = chunk * CHUNK, n_end = min(L, n_begin + CHUNK);
     const uint32_t* keys = P.keys + bs * P.Ncap;
-    for (int n = n_begin + tid; n < n_end; n += CONSUMERS) {
-        const uint32_t key = __ldcg(keys + n);
-        if (pass > 0 && (key >> (32 - 8 * pass)) != prefix) continue;
-        const int d = (key >> shift) & 255;
-        atomicAdd(&S.hcnt[d], 1u);
-        atomicAdd(&S.hmass[d], fixmass(key, smax));
+    constexpr int PER = CHUNK / CONSUMERS;
+    uint32_t kk[PER];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        const int n = n_begin + tid + i * CONSUMERS;
+        kk[i] = (n < n_end) ? __ldcg(keys + n) : 0u;
     }
+    // Lanes holding the same digit are summed in the warp (match + redux):
+    // the 2^-40 fixed-point mass (< 2^41) is split into 17-bit slices so the
+    // 32-bit warp and shared sums stay exact; one leader per digit updates
+    // the shared histogram.
+    const int lane = tid & 31;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        const int n = n_begin + tid + i * CONSUMERS;
+        const uint32_t key = kk[i];
+        const bool valid = n < n_end && (pass == 0 || (key >> (32 - 8 * pass)) == prefix);
+        const uint32_t d = valid ? ((key >> shift) & 255u) : 0xFFFFFFFFu;
+        const uint32_t peers = __match_any_sync(0xffffffffu, d);
+        if (valid) {
+            const unsigned long long ms = fixmass(key, smax);
+            const uint32_t s0 = __reduce_add_sync(peers, (uint32_t)(ms & 0x1FFFFull));
+            const uint32_t s1 = __reduce_add_sync(peers, (uint32_t)((ms >> 17) & 0x1FFFFull));
+            const uint32_t s2 = __reduce_add_sync(peers, (uint32_t)(ms >> 34));
+            if (lane == __ffs(peers) - 1) {
+                atomicAdd(&S.hcnt[d], (uint32_t)__popc(peers));
+                atomicAdd(&S.hm[0][d], s0);
+                atomicAdd(&S.hm[1][d], s1);
+                atomicAdd(&S.hm[2][d], s2);
+            }
+        }
+    }
+    consumer_sync();
+    for (int d = tid; d < 256; d += CONSUMERS)
+        S.hmass[d] = (unsigned long long)S.hm[0][d] + ((unsigned long long)S.hm[1][d] << 17) +
+                     ((unsigned long long)S.hm[2][d] << 34);
     consumer_sync();
     uint32_t* gcnt = P.hist_cnt + bs * 256;
     unsigned long long* gmass = P.hist_mass + bs * 256;
@@ -459,6 +506,7 @@ __device__ void radix_item(const StepParams& SP, StepSmem<G>& S, int j, int pass
         *hsp = st;
         __threadfence();
         atomicAdd(&SP.sync->pass_done[pass], 1u);
+        trace_max(P, 8 + pass);
     }
 }
 
@@ -487,10 +535,20 @@ __device__ void mark_item(const StepParams& SP, StepSmem<G>& S, int j, int tid) 
     if (tid == 0) S.word = 0;
     uint32_t carry = 0;
     uint32_t mine = 0;
+    constexpr int PER = CHUNK / CONSUMERS;
+    uint32_t kk[PER];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        const int n = n_begin + tid + i * CONSUMERS;
+        kk[i] = (n < n_end) ? __ldcg(keys + n) : 0u;
+    }
     consumer_sync();
-    for (int base = n_begin; base < n_end; base += CONSUMERS) {
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        const int base = n_begin + i * CONSUMERS;
+        if (base >= n_end) break;
         const int n = base + tid;
-        const uint32_t key = (n < n_end) ? __ldcg(keys + n) : 0u;
+        const uint32_t key = kk[i];
         bool keep = (n < n_end) && key > tau;
         const bool tie = (n < n_end) && key == tau;
         if (st.all_ties) {
@@ -517,6 +575,7 @@ __device__ void mark_item(const StepParams& SP, StepSmem<G>& S, int j, int tid) 
     if (tid == 0) {
         __threadfence();
         atomicAdd(&SP.sync->mark_done, 1u);
+        trace_max(P, 12);
     }
 }
 
@@ -583,6 +642,7 @@ __device__ void blist_item(const StepParams& SP, StepSmem<G>& S, int gi, int tid
         P.bcount[bg] = s_base;
         __threadfence();
         atomicAdd(&SP.sync->groups_ready, 1u);
+        trace_max(P, 3);
     }
     consumer_sync();
 }
@@ -882,7 +942,9 @@ __device__ void consumers(const StepParams& SP, StepSmem<G>& S, int tid) {
                 core.flush(S, parts + (int64_t)d.item * G * PSTRIDE, heads, tid);
                 if (consumer_last(ctr, nitems, &S.flag)) {
                     __threadfence();
+                    if (tid == 0 && local) trace_max(P, 7);
                     combine_parts<G>(P, S, parts, nitems, heads, d.b, g, tid);
+                    if (tid == 0) trace_max(P, local ? 2 : 4);
                 }
             }
             continue;
@@ -898,7 +960,7 @@ __device__ void consumers(const StepParams& SP, StepSmem<G>& S, int tid) {
 }
 
 template <int G>
-__global__ void __launch_bounds__(STEP_THREADS) step_kernel(const __grid_constant__ StepParams SP) {
+__global__ void __launch_bounds__(STEP_THREADS, (G >= 8) ? 1 : 2) step_kernel(const __grid_constant__ StepParams SP) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     StepSmem<G>& S = *reinterpret_cast<StepSmem<G>*>(smem_raw);
     constexpr int NST = StepSmem<G>::NST;
@@ -910,6 +972,7 @@ __global__ void __launch_bounds__(STEP_THREADS) step_kernel(const __grid_constan
         }
         mbar_fence_init();
     }
+    if (tid == 0 && SP.P.dbg_trace) atomicCAS(SP.P.dbg_trace, 0ull, (unsigned long long)global_ns());
     __syncthreads();
     if (tid >= CONSUMERS) {
         if (tid == CONSUMERS) producer<G>(SP, S);
@@ -918,6 +981,7 @@ __global__ void __launch_bounds__(STEP_THREADS) step_kernel(const __grid_constan
     consumers<G>(SP, S, tid);
     // last CTA out clears the coordination words for the next call
     consumer_sync();
+    if (tid == 0) trace_max(SP.P, 5);
     if (tid == 0) {
         __threadfence();
         if (atomicAdd(&SP.sync->exit_count, 1u) == gridDim.x - 1) {

@@ -271,7 +271,7 @@ def main():
     t_ms = statistics.mean(step_ms)
 
     # ---- timeline of one step (debug trace, separate untimed replays) ----
-    trace_buf = torch.zeros(16, dtype=torch.int64, device=dev)
+    trace_buf = torch.zeros(32, dtype=torch.int64, device=dev)
     tdbg = rtp.RtpDebug(trace=trace_buf.data_ptr())
     dc.step.dims.debug = ctypes.pointer(tdbg)
     tl = []
@@ -281,7 +281,9 @@ def main():
         dc.run(stream)
         torch.cuda.synchronize(dev)
         t = trace_buf.cpu().numpy().astype(np.float64)
-        tl.append({n: (t[k] - t[0]) / 1e3 if t[k] > 0 else None for k, n in enumerate(rtp.TRACE_EVENTS) if k})
+        ev = {n: (t[k] - t[0]) / 1e3 if t[k] > 0 else None for k, n in enumerate(rtp.TRACE_EVENTS) if k}
+        ev.update({n: t[16 + k] for k, n in enumerate(rtp.TRACE_SUMS)})
+        tl.append(ev)
     dc.step.dims.debug = ctypes.POINTER(rtp.RtpDebug)()
     timeline = {n: (statistics.median([x[n] for x in tl]) if tl[0][n] is not None else None)
                 for n in tl[0]}

@@ -73,10 +73,13 @@ typedef struct rtp_debug {
     float* smax;             /* [B*Hq] largest index score s */
     double* Z;               /* [B*Hq] sum over n < L of exp((s_n - smax)/4) */
     uint32_t* block_bitmap;  /* [B*Hq*words], words = ceil(ceil(capacity/64)/32); bit j%32 of word j/32 = block j kept */
-    /* [16] %globaltimer nanoseconds, zero them before the call: 0 kernel start, 1 last selection
+    /* [32] %globaltimer nanoseconds, zero them before the call: 0 kernel start, 1 last selection
      * decided, 2 last local-head combine done, 3 last block list final, 4 last retrieval combine
      * done, 5 kernel end, 6 last selection started (all index scores of a group done),
-     * 7 last local-head combine started, 8-11 last radix pass 1-4 done, 12 last block mark done */
+     * 7 last local-head combine started, 8-11 last radix pass 1-4 done, 12 last block mark done;
+     * summed over CTAs: 16-24 consumer SM cycles waiting for data, in score begin / tile /
+     * release / epilogue, attention begin / tile / epilogue, other; 25 score tiles; 26-28
+     * producer ns waiting for a free stage, on other CTAs, for queue claims */
     unsigned long long* trace;
 } rtp_debug;
 

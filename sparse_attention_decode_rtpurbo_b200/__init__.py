@@ -35,7 +35,11 @@ class RtpDebug(ctypes.Structure):
 
 
 TRACE_EVENTS = ["start", "select_done", "local_done", "lists_ready", "retrieval_done", "end", "select_start",
-                "local_combine_start", "radix1", "radix2", "radix3", "radix4", "mark", "t13", "t14", "t15"]
+                "local_combine_start", "radix1", "radix2", "radix3", "radix4", "mark"]
+# summed over CTAs (slots 16..28): consumer SM cycles by category, then producer ns
+TRACE_SUMS = ["cyc_wait", "cyc_score_begin", "cyc_score_tile", "cyc_score_release", "cyc_score_epilogue",
+              "cyc_attn_begin", "cyc_attn_tile", "cyc_attn_epilogue", "cyc_other", "n_score_tiles",
+              "ns_prod_slot", "ns_prod_dep", "ns_prod_claim"]
 
 
 class RtpDims(ctypes.Structure):

@@ -9,7 +9,8 @@ namespace rtp {
 constexpr int D = 128;          // head dimension
 constexpr int R = 16;           // indexer rank
 constexpr int BLK = 64;         // KV block (page) size in tokens
-constexpr int CHUNK = 2048;     // tokens per scoring / selection CTA (= 32 blocks = one bitmap word)
+constexpr int CHUNK = 2048;         // tokens per selection item (= 32 blocks = one bitmap word)
+constexpr int SCORE_CHUNK = 2048;   // tokens per index-score item (2 staged tiles)
 constexpr int SEL_THREADS = 256;
 constexpr int ATT_THREADS = 128;
 constexpr int STAGES = 3;                       // K/V tile ring depth of the attention kernels
@@ -26,15 +27,15 @@ constexpr uint32_t ST_DEVICE_INPUT = 6;
 constexpr uint32_t ST_TIMEOUT = 7;
 
 // Per retrieval head and bucket (chunk mod AGG_BUCKETS), folded by score
-// chunks with atomics (all-zero = empty, so a zero-filled workspace is
-// ready): best = (max key << 32) | ~argmax, nmin = ~(min key), ms = (key of
-// the reference score << 32) | fp32 sum of exp((s - ref)/4), the reference
-// being the bucket's max score.  Buckets keep same-address atomics rare.
+// chunks with fire-and-forget atomics (all-zero = empty, so a zero-filled
+// workspace is ready): best = (max key << 32) | ~argmax, nmin = ~(min key),
+// zabs = fp64 sum of exp(s/4), flags bit 0 = a chunk's scores left the range
+// where that sum is safe.  Buckets keep same-address atomics rare.
 constexpr int AGG_BUCKETS = 32;
 struct HeadAgg {
     unsigned long long best;
-    uint32_t nmin, pad;
-    unsigned long long ms;
+    uint32_t nmin, flags;
+    double zabs;
 };
 
 struct HeadState {
@@ -48,7 +49,7 @@ struct HeadState {
 
 struct Params {
     int B, Hq, Hkv, G, Ncap, nblk_cap, words_cap, mbps, num_pages, window, sink;
-    int n_ret, n_rg, n_lg, nchunks;
+    int n_ret, n_rg, n_lg, nchunks, nschunks;
     int local_kb, local_items, ret_grid;
     const uint16_t *q_pre, *q_rope, *k_idx, *k_cache, *v_cache, *Wq;
     const int32_t *seq_lens, *block_table;
@@ -148,6 +149,20 @@ __device__ __forceinline__ bool last_arrival(uint32_t* ctr, uint32_t count, uint
 // mbarrier + bulk copy (TMA engine, non-tensor form)
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+// 2^x on the special-function unit (about 2 ulp; 0 for x = -inf)
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// 16-byte load from a shared-memory address (explicit shared state space)
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+    return v;
+}
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");

@@ -16,7 +16,7 @@ constexpr int NSM_PLAN = 148;       // SMs of a B200: sizes the split counts
 constexpr int MAX_GRID = 148 * 4;   // upper bound of the persistent grid (partials are sized for it)
 
 struct Plan {
-    int B, Hq, Hkv, G, Ncap, nblk_cap, words_cap, nchunks;
+    int B, Hq, Hkv, G, Ncap, nblk_cap, words_cap, nchunks, nschunks;
     int n_ret, n_rg, n_lg;
     int local_kb, local_items, ret_grid;
     uint8_t rg_group[MAX_HKV], rg_mask[MAX_HKV], rg_slot0[MAX_HKV], rg_nh[MAX_HKV];
@@ -59,6 +59,7 @@ static rtp_status make_plan(const rtp_dims* d, const uint8_t* head_kind, int win
     pl->nblk_cap = pl->Ncap / BLK;
     pl->words_cap = (pl->nblk_cap + 31) / 32;
     pl->nchunks = (pl->Ncap + CHUNK - 1) / CHUNK;
+    pl->nschunks = (pl->Ncap + SCORE_CHUNK - 1) / SCORE_CHUNK;
     for (int g = 0; g < pl->Hkv; ++g) {
         uint32_t rm = 0, lm = 0;
         for (int i = 0; i < pl->G; ++i) {
@@ -90,7 +91,7 @@ static rtp_status make_plan(const rtp_dims* d, const uint8_t* head_kind, int win
     if (pl->n_lg) {
         const int64_t nv_max = std::min<int64_t>(pl->nblk_cap, (sink + BLK - 1) / BLK + (window + BLK - 1) / BLK + 1);
         const int64_t total = (int64_t)pl->B * pl->n_lg * nv_max;
-        pl->local_kb = (int)std::max<int64_t>(1, (total + 2 * NSM_PLAN - 1) / (2 * NSM_PLAN));
+        pl->local_kb = (int)std::max<int64_t>(4, (total + 2 * NSM_PLAN - 1) / (2 * NSM_PLAN));
         // the split combine keeps one weight per (head, split) in 512*G floats
         pl->local_kb = (int)std::max<int64_t>(pl->local_kb, (nv_max + 511) / 512);
         pl->local_items = (int)((nv_max + pl->local_kb - 1) / pl->local_kb);
@@ -154,7 +155,7 @@ static cudaError_t launch_step(const Params& P, const Plan& pl, uint8_t* ws, cud
     SP.sync = reinterpret_cast<Sync*>(ws + pl.o_sync);
     SP.rlist = reinterpret_cast<uint32_t*>(ws + pl.o_rlist);
     SP.rglist = reinterpret_cast<uint32_t*>(ws + pl.o_rglist);
-    SP.n_score_items = pl.B * pl.n_rg * pl.nchunks;
+    SP.n_score_items = pl.B * pl.n_rg * pl.nschunks;
     SP.n_local_items = pl.B * pl.n_lg * pl.local_items;
     const int grid = std::min(MAX_GRID, ctas_per_sm.load() * num_sms.load());
     if (ev) cudaEventRecordWithFlags((cudaEvent_t)ev[0], s, ev_flags);
@@ -204,6 +205,7 @@ extern "C" rtp_status rtp_decode_step(const rtp_dims* dims, const uint16_t* q_pr
     P.n_rg = pl.n_rg;
     P.n_lg = pl.n_lg;
     P.nchunks = pl.nchunks;
+    P.nschunks = pl.nschunks;
     P.local_kb = pl.local_kb;
     P.local_items = pl.local_items;
     P.ret_grid = pl.ret_grid;

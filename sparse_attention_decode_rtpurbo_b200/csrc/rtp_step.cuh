@@ -81,6 +81,8 @@ struct StepSmem {
     double w_sum[G][4];
     uint32_t flag, word;
     int dstar;
+    int qi_tag;   // (b, retrieval group) whose q_idx is in qi, + 1; 0 = none
+    unsigned long long acct[10];   // debug cycle accounting (thread 0)
 };
 
 // ---------------------------------------------------------------------------
@@ -194,18 +196,27 @@ template <int G>
 struct AttnCore {
     float acc[G][8];
     float q[G][8];
+    int q_tag = -1;   // (b, KV head) whose queries are in q
 
     __device__ __forceinline__ void begin(const Params& P, StepSmem<G>& S, int b, int g, int tid) {
         const int dc = tid & 15;
+        const int tag = b * P.Hkv + g;
+        if (tag != q_tag) {
+            q_tag = tag;
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                const uint4 u =
+                    *reinterpret_cast<const uint4*>(P.q_rope + ((int64_t)b * P.Hq + g * G + h) * D + dc * 8);
+                const uint32_t* w = reinterpret_cast<const uint32_t*>(&u);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    q[h][2 * j] = bf_lo(w[j]);
+                    q[h][2 * j + 1] = bf_hi(w[j]);
+                }
+            }
+        }
 #pragma unroll
         for (int h = 0; h < G; ++h) {
-            const uint4 u = *reinterpret_cast<const uint4*>(P.q_rope + ((int64_t)b * P.Hq + g * G + h) * D + dc * 8);
-            const uint32_t* w = reinterpret_cast<const uint32_t*>(&u);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                q[h][2 * j] = bf_lo(w[j]);
-                q[h][2 * j + 1] = bf_hi(w[j]);
-            }
 #pragma unroll
             for (int j = 0; j < 8; ++j) acc[h][j] = 0.f;
         }
@@ -222,14 +233,13 @@ struct AttnCore {
     __device__ __forceinline__ void tile(StepSmem<G>& S, const uint8_t* kv, uint32_t hmask, int n0, int nvalid,
                                          bool local, int s_end, int w_lo, int tid) {
         const int lane = tid & 31, tg = tid >> 4, dc = tid & 15;
-        const uint4* K = reinterpret_cast<const uint4*>(kv);
-        const uint4* V = reinterpret_cast<const uint4*>(kv + TILE_BYTES);
+        const uint32_t K = smem_u32(kv), V = K + TILE_BYTES;
         constexpr int CNT = 8 * G;
         constexpr int NV = CNT >= 16 ? CNT / 16 : 1;
         float v[CNT];
 #pragma unroll
         for (int t = 0; t < 8; ++t) {
-            const uint4 u = K[(tg * 8 + t) * 16 + dc];
+            const uint4 u = lds128(K + ((tg * 8 + t) * 16 + dc) * 16);
             const uint32_t* w = reinterpret_cast<const uint32_t*>(&u);
             float k8[8];
 #pragma unroll
@@ -298,7 +308,7 @@ struct AttnCore {
             bool ok = tok < nvalid;
             if (local) ok = ok && (n < s_end || n >= w_lo);
             if (!ok) continue;
-            const uint4 u = V[tok * 16 + dc];
+            const uint4 u = lds128(V + (tok * 16 + dc) * 16);
             const uint32_t* w = reinterpret_cast<const uint32_t*>(&u);
             float v8[8];
 #pragma unroll
@@ -346,7 +356,7 @@ struct AttnCore {
 // Combine the partials of `nparts` splits (stride G*PSTRIDE floats) of the
 // heads in `heads` into out[b, g*G + h] (bf16, round to nearest even).
 template <int G>
-__device__ void combine_parts(const Params& P, StepSmem<G>& S, const float* parts, int nparts, uint32_t heads, int b,
+__device__ __forceinline__ void combine_parts(const Params& P, StepSmem<G>& S, const float* parts, int nparts, uint32_t heads, int b,
                               int g, int tid) {
     float* wts = &S.red[0][0][0];   // G * nparts weights (nparts <= 4*D)
     __shared__ float s_den[G];

@@ -15,75 +15,170 @@ struct StepParams {
 // ===========================================================================
 // index scores (consumers)
 // ===========================================================================
+// Index scoring on the tensor cores: per 16 staged rows, one m16n8k16 bf16
+// MMA against each of three bf16 parts of q_idx (hi + mid + lo = q_idx to
+// fp32 precision; every bf16 x bf16 product is exact and the sums are fp32),
+// N = 8 columns = the group's retrieval heads.  Thread (g = lane/4, t =
+// lane%4) owns heads 2t, 2t+1 of rows g and g+8 of each 16-row group.
 template <int G>
 struct ScoreState {
-    uint32_t mk[G], am[G], nk[G];
-    float ms[G], sm[G];
+    uint32_t b[3][2];                 // B fragments of q_idx hi / mid / lo
+    uint32_t mk[2], am[2], nk[2];     // per owned head: max key, its lowest index, min key
+    float ms[2], sm[2];               // max score, sum of exp((s - ms)/4)
 };
 
 template <int G>
-__device__ void score_begin(const Params& P, StepSmem<G>& S, ScoreState<G>& st, int b, int rgi, int tid) {
+__device__ __forceinline__ void score_begin(const Params& P, StepSmem<G>& S, ScoreState<G>& st, int b, int rgi, int tid) {
     const int nh = P.rg_nh[rgi], slot0 = P.rg_slot0[rgi];
-    const int warp = tid >> 5, lane = tid & 31;
-    // q_idx = Wq_idx[h] . q_pre[b,h] (fp32), one warp per (head, row)
-    for (int pr = warp; pr < nh * R; pr += CONSUMERS / 32) {
-        const int hh = pr / R, r = pr % R;
-        const int h = P.slot_head[slot0 + hh];
-        const uint2 w = *reinterpret_cast<const uint2*>(P.Wq + ((int64_t)h * R + r) * D + lane * 4);
-        const uint2 q = *reinterpret_cast<const uint2*>(P.q_pre + ((int64_t)b * P.Hq + h) * D + lane * 4);
-        float a = bf_lo(w.x) * bf_lo(q.x);
-        a = fmaf(bf_hi(w.x), bf_hi(q.x), a);
-        a = fmaf(bf_lo(w.y), bf_lo(q.y), a);
-        a = fmaf(bf_hi(w.y), bf_hi(q.y), a);
+    const int tag = b * MAX_HKV + rgi + 1;
+    if (S.qi_tag != tag) {
+        // q_idx = Wq_idx[h] . q_pre[b,h] (fp32) for the group's retrieval heads,
+        // all (head, row) dots at once: TPP threads per dot, one round of loads
+        const int npair = nh * R;                    // <= 128
+        const int tpp = CONSUMERS / npair >= 8 ? 8 : (CONSUMERS / npair >= 4 ? 4 : (CONSUMERS / npair >= 2 ? 2 : 1));
+        const int pr = tid / tpp, part = tid % tpp;
+        float a = 0.f;
+        if (pr < npair) {
+            const int hh = pr / R, r = pr % R;
+            const int h = P.slot_head[slot0 + hh];
+            const int span = D / tpp;                // dims per thread: 16..128
+            const uint4* w = reinterpret_cast<const uint4*>(P.Wq + ((int64_t)h * R + r) * D + part * span);
+            const uint4* q = reinterpret_cast<const uint4*>(P.q_pre + ((int64_t)b * P.Hq + h) * D + part * span);
+            for (int i = 0; i < span / 8; ++i) {
+                const uint4 wv = w[i], qv = q[i];
+                a = fmaf(bf_lo(wv.x), bf_lo(qv.x), a);
+                a = fmaf(bf_hi(wv.x), bf_hi(qv.x), a);
+                a = fmaf(bf_lo(wv.y), bf_lo(qv.y), a);
+                a = fmaf(bf_hi(wv.y), bf_hi(qv.y), a);
+                a = fmaf(bf_lo(wv.z), bf_lo(qv.z), a);
+                a = fmaf(bf_hi(wv.z), bf_hi(qv.z), a);
+                a = fmaf(bf_lo(wv.w), bf_lo(qv.w), a);
+                a = fmaf(bf_hi(wv.w), bf_hi(qv.w), a);
+            }
+        }
+        for (int o = 1; o < tpp; o <<= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+        if (pr < npair && part == 0) S.qi[pr / R][pr % R] = a;
+        consumer_sync();
+        if (tid == 0) S.qi_tag = tag;
+    }
+    // B fragment of column g (head g): k = 2t, 2t+1 and 2t+8, 2t+9
+    {
+        const int lane = tid & 31, g = lane >> 2, t = lane & 3;
+        float qv[4] = {0.f, 0.f, 0.f, 0.f};
+        if (g < nh) {
+            qv[0] = S.qi[g][2 * t];
+            qv[1] = S.qi[g][2 * t + 1];
+            qv[2] = S.qi[g][2 * t + 8];
+            qv[3] = S.qi[g][2 * t + 9];
+        }
+        uint16_t part[3][4];
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-        if (lane == 0) S.qi[hh][r] = a;
+        for (int i = 0; i < 4; ++i) {
+            const __nv_bfloat16 hi = __float2bfloat16_rn(qv[i]);
+            const float r1 = qv[i] - __bfloat162float(hi);
+            const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+            const __nv_bfloat16 lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
+            part[0][i] = __bfloat16_as_ushort(hi);
+            part[1][i] = __bfloat16_as_ushort(mid);
+            part[2][i] = __bfloat16_as_ushort(lo);
+        }
+#pragma unroll
+        for (int p = 0; p < 3; ++p) {
+            st.b[p][0] = (uint32_t)part[p][0] | ((uint32_t)part[p][1] << 16);
+            st.b[p][1] = (uint32_t)part[p][2] | ((uint32_t)part[p][3] << 16);
+        }
     }
 #pragma unroll
-    for (int hh = 0; hh < G; ++hh) {
-        st.mk[hh] = 0u;
-        st.am[hh] = 0xFFFFFFFFu;
-        st.nk[hh] = 0xFFFFFFFFu;
-        st.ms[hh] = -INFINITY;
-        st.sm[hh] = 0.f;
+    for (int j = 0; j < 2; ++j) {
+        st.mk[j] = 0u;
+        st.am[j] = 0xFFFFFFFFu;
+        st.nk[j] = 0xFFFFFFFFu;
+        st.ms[j] = -INFINITY;
+        st.sm[j] = 0.f;
     }
     consumer_sync();
 }
 
-// rows [0, nvalid) of the staged k_idx tile are tokens n0 + row
+// rows [0, nvalid) of the staged k_idx tile are tokens n0 + row; warp w
+// takes the 16-row groups w, w+4, ...  Rows past nvalid may hold anything:
+// each MMA row depends only on its own k_idx row and is dropped.
 template <int G>
-__device__ void score_tile(const Params& P, StepSmem<G>& S, ScoreState<G>& st, const uint8_t* data, int b, int rgi,
-                           int n0, int nvalid, int tid) {
+__device__ __forceinline__ void score_tile(const Params& P, StepSmem<G>& S, ScoreState<G>& st, const uint8_t* data, int b,
+                                           int rgi, int n0, int nvalid, int tid) {
     const int nh = P.rg_nh[rgi], slot0 = P.rg_slot0[rgi];
-    const uint4* rows = reinterpret_cast<const uint4*>(data);
-    for (int r = tid; r < nvalid; r += CONSUMERS) {
-        const uint4 u0 = rows[2 * r], u1 = rows[2 * r + 1];
-        float k[R];
-        k[0] = bf_lo(u0.x); k[1] = bf_hi(u0.x); k[2] = bf_lo(u0.y); k[3] = bf_hi(u0.y);
-        k[4] = bf_lo(u0.z); k[5] = bf_hi(u0.z); k[6] = bf_lo(u0.w); k[7] = bf_hi(u0.w);
-        k[8] = bf_lo(u1.x); k[9] = bf_hi(u1.x); k[10] = bf_lo(u1.y); k[11] = bf_hi(u1.y);
-        k[12] = bf_lo(u1.z); k[13] = bf_hi(u1.z); k[14] = bf_lo(u1.w); k[15] = bf_hi(u1.w);
-        const int n = n0 + r;
+    const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
+    const uint32_t rows = smem_u32(data);
+    constexpr float C = 0.25f * 1.4426950408889634f;   // (1/4) log2(e)
+    const int h0 = 2 * t;                               // owned heads h0, h0 + 1
+    uint32_t* keys0 = P.keys + ((int64_t)b * P.n_ret + slot0 + min(h0, nh - 1)) * P.Ncap + n0;
+    uint32_t* keys1 = P.keys + ((int64_t)b * P.n_ret + slot0 + min(h0 + 1, nh - 1)) * P.Ncap + n0;
+    const bool own0 = h0 < nh, own1 = h0 + 1 < nh;
+    // ldmatrix row address of this lane: matrix m = lane/8 (rows +8 if m odd, bytes +16 if m >= 2)
+    const uint32_t lrow = (uint32_t)(((lane >> 3) & 1) * 8 + (lane & 7)) * 32u + (uint32_t)((lane >> 4) * 16);
+    const int ngroups = (nvalid + 15) / 16;
+    constexpr int NW = CONSUMERS / 32;
+    // four 16-row groups per warp at a time: their MMA chains are independent
+#pragma unroll 1
+    for (int base = warp; base < ngroups; base += 4 * NW) {
+        uint32_t a[4][4];
+        float c[4][4];
 #pragma unroll
-        for (int hh = 0; hh < G; ++hh) {
-            if (hh >= nh) break;
-            float s = 0.f;
+        for (int q = 0; q < 4; ++q) {
+            const int grp = min(base + q * NW, ngroups - 1);
+            asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                         : "=r"(a[q][0]), "=r"(a[q][1]), "=r"(a[q][2]), "=r"(a[q][3])
+                         : "r"(rows + (uint32_t)grp * 512u + lrow));
+            c[q][0] = c[q][1] = c[q][2] = c[q][3] = 0.f;
+        }
 #pragma unroll
-            for (int i = 0; i < R; ++i) s = fmaf(S.qi[hh][i], k[i], s);
-            const uint32_t key = f2key(s);
-            P.keys[((int64_t)b * P.n_ret + slot0 + hh) * P.Ncap + n] = key;
-            if (key > st.mk[hh]) {
-                st.mk[hh] = key;
-                st.am[hh] = (uint32_t)n;
+        for (int p = 0; p < 3; ++p)
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+                    "{%0,%1,%2,%3};"
+                    : "+f"(c[q][0]), "+f"(c[q][1]), "+f"(c[q][2]), "+f"(c[q][3])
+                    : "r"(a[q][0]), "r"(a[q][1]), "r"(a[q][2]), "r"(a[q][3]), "r"(st.b[p][0]), "r"(st.b[p][1]));
+        // per owned head: 8 values (rows g and g+8 of 4 groups, in row order)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            if (!(j ? own1 : own0)) continue;
+            uint32_t* kp = j ? keys1 : keys0;
+            uint32_t kb = 0u, rb = 0u, kmin = 0xFFFFFFFFu;
+            float mb = -INFINITY;
+            float v[8];
+            bool ok[8];
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int e = q * 2 + h;
+                    const int r = (base + q * NW) * 16 + g + 8 * h;
+                    ok[e] = r < nvalid;
+                    v[e] = ok[e] ? c[q][j + 2 * h] : -INFINITY;
+                    const uint32_t key = f2key(v[e]);
+                    if (ok[e]) {
+                        kp[r] = key;
+                        if (key > kb) {
+                            kb = key;
+                            rb = (uint32_t)(n0 + r);
+                        }
+                        kmin = min(kmin, key);
+                    }
+                    mb = fmaxf(mb, v[e]);
+                }
+            if (kb > st.mk[j]) {
+                st.mk[j] = kb;
+                st.am[j] = rb;
             }
-            st.nk[hh] = min(st.nk[hh], key);
-            constexpr float C = 0.25f * 1.4426950408889634f;   // (1/4) log2(e)
-            if (s > st.ms[hh]) {
-                st.sm[hh] = st.sm[hh] * exp2f((st.ms[hh] - s) * C) + 1.f;
-                st.ms[hh] = s;
-            } else {
-                st.sm[hh] += exp2f((s - st.ms[hh]) * C);
+            st.nk[j] = min(st.nk[j], kmin);
+            if (mb > st.ms[j]) {
+                st.sm[j] *= ex2_approx((st.ms[j] - mb) * C);
+                st.ms[j] = mb;
             }
+            float add = 0.f;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) add += ok[e] ? ex2_approx((v[e] - st.ms[j]) * C) : 0.f;
+            st.sm[j] += add;
         }
     }
 }
@@ -111,7 +206,7 @@ __device__ __forceinline__ void fold_ms(uint32_t& ka, float& sa, uint32_t kb, fl
 // whose best token alone reaches p, or whose p >= 1, are final; if all heads
 // of the group are final its block list is written here.
 template <int G>
-__device__ void score_decide(const StepParams& SP, StepSmem<G>& S, int b, int rgi, int L, int nch, int tid) {
+__device__ __forceinline__ void score_decide(const StepParams& SP, StepSmem<G>& S, int b, int rgi, int L, int nch, int tid) {
     const Params& P = SP.P;
     const int nh = P.rg_nh[rgi], slot0 = P.rg_slot0[rgi], g = P.rg_group[rgi];
     const int nblk = (L + BLK - 1) / BLK;
@@ -121,32 +216,32 @@ __device__ void score_decide(const StepParams& SP, StepSmem<G>& S, int b, int rg
     // every chunk of the group has folded its partials into its heads'
     // buckets (score_end): one warp per head reduces the 32 buckets and
     // re-arms them for the next call
-    __shared__ unsigned long long s_best[MAX_G], s_ms[MAX_G];
-    __shared__ uint32_t s_nmin[MAX_G];
+    __shared__ unsigned long long s_best[MAX_G];
+    __shared__ uint32_t s_nmin[MAX_G], s_flags[MAX_G];
+    __shared__ double s_zabs[MAX_G];
     {
         const int warp = tid >> 5, lane = tid & 31;
         for (int hh = warp; hh < nh; hh += CONSUMERS / 32) {
             HeadAgg* ag = P.agg + ((int64_t)b * P.n_ret + slot0 + hh) * AGG_BUCKETS + lane;
             unsigned long long best = __ldcg(&ag->best);
-            uint32_t nmin = __ldcg(&ag->nmin);
-            const unsigned long long ms = __ldcg(&ag->ms);
-            uint32_t km = (uint32_t)(ms >> 32);
-            float su = __uint_as_float((uint32_t)(ms & 0xFFFFFFFFull));
+            uint32_t nmin = __ldcg(&ag->nmin), flags = __ldcg(&ag->flags);
+            double zabs = __ldcg(&ag->zabs);
             ag->best = 0ull;
             ag->nmin = 0u;
-            ag->ms = 0ull;
+            ag->flags = 0u;
+            ag->zabs = 0.0;
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) {
                 best = max(best, __shfl_xor_sync(0xffffffffu, best, o));
                 nmin = max(nmin, __shfl_xor_sync(0xffffffffu, nmin, o));
-                const uint32_t km2 = __shfl_xor_sync(0xffffffffu, km, o);
-                const float s2 = __shfl_xor_sync(0xffffffffu, su, o);
-                fold_ms(km, su, km2, s2);
+                flags |= __shfl_xor_sync(0xffffffffu, flags, o);
+                zabs += __shfl_xor_sync(0xffffffffu, zabs, o);
             }
             if (lane == 0) {
                 s_best[hh] = best;
                 s_nmin[hh] = nmin;
-                s_ms[hh] = ((unsigned long long)km << 32) | __float_as_uint(su);
+                s_flags[hh] = flags;
+                s_zabs[hh] = zabs;
             }
         }
     }
@@ -159,8 +254,9 @@ __device__ void score_decide(const StepParams& SP, StepSmem<G>& S, int b, int rg
         const uint32_t a = 0xFFFFFFFFu - (uint32_t)(best & 0xFFFFFFFFull);
         const uint32_t mn = ~s_nmin[hh];
         const float smax = key2f(k);
-        // the folded sum's reference is the head's max score, i.e. smax
-        const double z = (double)__uint_as_float((uint32_t)(s_ms[hh] & 0xFFFFFFFFull));
+        // z = sum over tokens of exp((s - smax)/4); NaN when the fp64 sum was unusable
+        const double sm4 = (double)smax * 0.25;
+        const double z = (s_flags[hh] || sm4 > 600.0 || sm4 < -600.0) ? NAN : s_zabs[hh] * exp(-sm4);
         {
             const float pb = __ldg(P.p + b);
             HeadState h;
@@ -187,7 +283,7 @@ __device__ void score_decide(const StepParams& SP, StepSmem<G>& S, int b, int rg
                 h.mode = MODE_ALL;
                 h.kstar = (uint32_t)L;
                 h.tau_key = mn;
-            } else if (1.0 >= (double)pb * z * (1.0 + 1e-3)) {
+            } else if (z == z && 1.0 >= (double)pb * z * (1.0 + 1e-3)) {
                 h.mode = MODE_TOP1;   // the best token alone reaches p
                 h.kstar = 1;
                 h.tau_key = k;
@@ -304,19 +400,18 @@ __device__ void score_decide(const StepParams& SP, StepSmem<G>& S, int b, int rg
 }
 
 template <int G>
-__device__ void score_end(const StepParams& SP, StepSmem<G>& S, ScoreState<G>& st, int b, int rgi, int chunk, int L,
-                          int nch, int tid) {
+__device__ __forceinline__ void score_end(const StepParams& SP, StepSmem<G>& S, ScoreState<G>& st, int b, int rgi, int chunk,
+                                          int L, int nch, int tid) {
     const Params& P = SP.P;
     const int nh = P.rg_nh[rgi], slot0 = P.rg_slot0[rgi];
-    const int warp = tid >> 5, lane = tid & 31;
+    const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
 #pragma unroll
-    for (int hh = 0; hh < G; ++hh) {
-        if (hh >= nh) break;
-        uint32_t k = st.mk[hh], a = st.am[hh], mn = st.nk[hh];
-        uint32_t km = st.mk[hh];   // the running sum is relative to the max score, whose key is mk
-        float su = st.sm[hh];
+    for (int j = 0; j < 2; ++j) {
+        uint32_t k = st.mk[j], a = st.am[j], mn = st.nk[j];
+        uint32_t km = st.mk[j];   // the running sum is relative to the max score, whose key is mk
+        float su = st.sm[j];
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
+        for (int o = 4; o < 32; o <<= 1) {
             const uint32_t k2 = __shfl_xor_sync(0xffffffffu, k, o);
             const uint32_t a2 = __shfl_xor_sync(0xffffffffu, a, o);
             const uint32_t km2 = __shfl_xor_sync(0xffffffffu, km, o);
@@ -328,7 +423,8 @@ __device__ void score_end(const StepParams& SP, StepSmem<G>& S, ScoreState<G>& s
             }
             fold_ms(km, su, km2, s2);
         }
-        if (lane == 0) {
+        const int hh = 2 * t + j;
+        if (g == 0 && hh < nh) {
             S.w_key[hh][warp] = k;
             S.w_arg[hh][warp] = a;
             S.w_min[hh][warp] = mn;
@@ -349,19 +445,17 @@ __device__ void score_end(const StepParams& SP, StepSmem<G>& S, ScoreState<G>& s
             mn = min(mn, S.w_min[hh][w]);
             fold_ms(km, su, __float_as_uint(S.w_m[hh][w]), (float)S.w_sum[hh][w]);
         }
-        // fold this chunk into its bucket of the head's aggregate
+        // fold this chunk into its bucket of the head's aggregate: fire-and-forget
+        // atomics, the exp-sum as the fp64 sum of exp(s/4) (out of fp64's safe
+        // range the head takes the exact radix path instead)
         HeadAgg* ag = P.agg + ((int64_t)b * P.n_ret + slot0 + hh) * AGG_BUCKETS + (chunk % AGG_BUCKETS);
         atomicMax(&ag->best, ((unsigned long long)k << 32) | (0xFFFFFFFFu - a));
         atomicMax(&ag->nmin, ~mn);
-        unsigned long long old = __ldcg(&ag->ms), assumed;
-        do {
-            assumed = old;
-            uint32_t ka = (uint32_t)(assumed >> 32);
-            float sa = __uint_as_float((uint32_t)(assumed & 0xFFFFFFFFull));
-            fold_ms(ka, sa, km, su);
-            const unsigned long long nv = ((unsigned long long)ka << 32) | __float_as_uint(sa);
-            old = atomicCAS(&ag->ms, assumed, nv);
-        } while (old != assumed);
+        if (km != 0u) {
+            const double m4 = (double)key2f(km) * 0.25;
+            if (m4 > 600.0 || m4 < -600.0) atomicOr(&ag->flags, 1u);
+            else atomicAdd(&ag->zabs, (double)su * exp(m4));
+        }
     }
     if (!consumer_last(P.tick_score + b * P.n_rg + rgi, nch, &S.flag)) return;
     __threadfence();
@@ -374,14 +468,9 @@ __device__ void score_end(const StepParams& SP, StepSmem<G>& S, ScoreState<G>& s
 // exact radix select, block marking, block lists (consumers, L2-resident)
 // ===========================================================================
 template <int G>
-__device__ void radix_item(const StepParams& SP, StepSmem<G>& S, int j, int pass, int tid) {
+__device__ __forceinline__ void radix_item(const StepParams& SP, StepSmem<G>& S, int b, int slot, int chunk, int L, int pass, int tid) {
     const Params& P = SP.P;
-    const int k = j / P.nchunks, chunk = j % P.nchunks;
-    const uint32_t e = __ldcg(SP.rlist + k);
-    const int b = (int)(e >> 16), slot = (int)(e & 0xFFFFu);
-    const int L = __ldg(P.seq_lens + b);
     const int nch = (L + CHUNK - 1) / CHUNK;
-    if (chunk >= nch) return;
     const int64_t bs = (int64_t)b * P.n_ret + slot;
     HeadState* hsp = P.hs + bs;
     for (int d = tid; d < 256; d += CONSUMERS) {
@@ -390,10 +479,6 @@ __device__ void radix_item(const StepParams& SP, StepSmem<G>& S, int j, int pass
         S.hm[1][d] = 0;
         S.hm[2][d] = 0;
     }
-    consumer_sync();
-    const uint32_t prefix = __ldcg(&hsp->prefix);
-    const float smax = __ldcg(&hsp->smax);
-    const int shift = 24 - 8 * pass;
     const int n_begin = chunk * CHUNK, n_end = min(L, n_begin + CHUNK);
     const uint32_t* keys = P.keys + bs * P.Ncap;
     constexpr int PER = CHUNK / CONSUMERS;
@@ -403,6 +488,10 @@ __device__ void radix_item(const StepParams& SP, StepSmem<G>& S, int j, int pass
         const int n = n_begin + tid + i * CONSUMERS;
         kk[i] = (n < n_end) ? __ldcg(keys + n) : 0u;
     }
+    const uint32_t prefix = __ldcg(&hsp->prefix);
+    const float smax = __ldcg(&hsp->smax);
+    const int shift = 24 - 8 * pass;
+    consumer_sync();
     // Lanes holding the same digit are summed in the warp (match + redux):
     // the 2^-40 fixed-point mass (< 2^41) is split into 17-bit slices so the
     // 32-bit warp and shared sums stay exact; one leader per digit updates
@@ -511,14 +600,9 @@ __device__ void radix_item(const StepParams& SP, StepSmem<G>& S, int j, int pass
 }
 
 template <int G>
-__device__ void mark_item(const StepParams& SP, StepSmem<G>& S, int j, int tid) {
+__device__ __forceinline__ void mark_item(const StepParams& SP, StepSmem<G>& S, int b, int slot, int chunk, int L, int tid) {
     const Params& P = SP.P;
-    const int k = j / P.nchunks, chunk = j % P.nchunks;
-    const uint32_t e = __ldcg(SP.rlist + k);
-    const int b = (int)(e >> 16), slot = (int)(e & 0xFFFFu);
-    const int L = __ldg(P.seq_lens + b);
     const int nch = (L + CHUNK - 1) / CHUNK;
-    if (chunk >= nch) return;
     const int64_t bs = (int64_t)b * P.n_ret + slot;
     HeadState st;
     {
@@ -580,7 +664,7 @@ __device__ void mark_item(const StepParams& SP, StepSmem<G>& S, int j, int tid) 
 }
 
 template <int G>
-__device__ void blist_item(const StepParams& SP, StepSmem<G>& S, int gi, int tid) {
+__device__ __forceinline__ void blist_item(const StepParams& SP, StepSmem<G>& S, int gi, int tid) {
     const Params& P = SP.P;
     const uint32_t e = __ldcg(SP.rglist + gi);
     const int b = (int)(e >> 16), rgi = (int)(e & 0xFFFFu);
@@ -650,21 +734,41 @@ __device__ void blist_item(const StepParams& SP, StepSmem<G>& S, int gi, int tid
 // ===========================================================================
 // the persistent kernel
 // ===========================================================================
+// radix / mark item j -> (b, slot, chunk, L) in d; false when the chunk is
+// past the head's sequence length
+__device__ __forceinline__ bool resolve_chunk(const StepParams& SP, int j, Desc& d) {
+    const Params& P = SP.P;
+    const int k = j / P.nchunks, chunk = j % P.nchunks;
+    const uint32_t e = __ldcg(SP.rlist + k);
+    const int b = (int)(e >> 16), slot = (int)(e & 0xFFFFu);
+    const int L = __ldg(P.seq_lens + b);
+    if (chunk >= (L + CHUNK - 1) / CHUNK) return false;
+    d.b = b;
+    d.grp = slot;
+    d.item = chunk;
+    d.aux1 = L;
+    return true;
+}
+
 template <int G>
-__device__ void producer(const StepParams& SP, StepSmem<G>& S) {
+__device__ __forceinline__ void producer(const StepParams& SP, StepSmem<G>& S) {
     constexpr int NST = StepSmem<G>::NST;
     const Params& P = SP.P;
     Sync* sy = SP.sync;
     uint32_t t = 0;   // tiles published so far (same sequence the consumers follow)
     bool alive = true;
+    const bool acct = P.dbg_trace != nullptr;
+    unsigned long long a_slot = 0, a_dep = 0, a_claim = 0;
 
     auto acquire = [&]() -> int {
         const int st = (int)(t % NST);
         const uint32_t round = t / NST;
+        const uint64_t t0 = acct ? global_ns() : 0;
         if (round > 0 && !mbar_wait_bounded(&S.empty[st], (round - 1) & 1u)) {
             set_status(P, ST_TIMEOUT);
             alive = false;
         }
+        if (acct) a_slot += global_ns() - t0;
         return st;
     };
     auto publish_nodata = [&](const Desc& d) {
@@ -675,19 +779,27 @@ __device__ void producer(const StepParams& SP, StepSmem<G>& S) {
         ++t;
     };
     auto wait_for = [&](const uint32_t* ctr, uint32_t target) {
+        const uint64_t t0 = acct ? global_ns() : 0;
         if (alive && !wait_counter(ctr, target)) {
             set_status(P, ST_TIMEOUT);
             alive = false;
         }
+        if (acct) a_dep += global_ns() - t0;
+    };
+    auto claim = [&]() -> uint32_t {
+        const uint64_t t0 = acct ? global_ns() : 0;
+        const uint32_t v = atomicAdd(&sy->queue, 1u);
+        if (acct) a_claim += global_ns() - t0;
+        return v;
     };
 
     const int n_static = SP.n_score_items + SP.n_local_items;
-    uint32_t x = atomicAdd(&sy->queue, 1u);
+    uint32_t x = claim();
     while (alive && (int)x < n_static) {
         if ((int)x < SP.n_score_items) {
             // ---- index-score chunk (b, rgi, chunk) ----
-            const int per_b = P.n_rg * P.nchunks;
-            const int b = (int)x / per_b, rgi = ((int)x % per_b) / P.nchunks, chunk = (int)x % P.nchunks;
+            const int per_b = P.n_rg * P.nschunks;
+            const int b = (int)x / per_b, rgi = ((int)x % per_b) / P.nschunks, chunk = (int)x % P.nschunks;
             const int L = __ldg(P.seq_lens + b);
             if (!seq_ok(P, L)) {
                 if (chunk == 0) {   // this sequence's groups: no selection, no blocks
@@ -698,10 +810,10 @@ __device__ void producer(const StepParams& SP, StepSmem<G>& S) {
                     atomicAdd(&sy->groups_ready, 1u);
                 }
             } else {
-                const int nch = (L + CHUNK - 1) / CHUNK;
+                const int nch = (L + SCORE_CHUNK - 1) / SCORE_CHUNK;
                 if (chunk < nch) {
                     const int g = P.rg_group[rgi];
-                    const int n_begin = chunk * CHUNK, n_end = min(L, n_begin + CHUNK);
+                    const int n_begin = chunk * SCORE_CHUNK, n_end = min(L, n_begin + SCORE_CHUNK);
                     const int ntiles = (n_end - n_begin + SCORE_ROWS - 1) / SCORE_ROWS;
                     for (int ti = 0; ti < ntiles && alive; ++ti) {
                         const int n0 = n_begin + ti * SCORE_ROWS;
@@ -779,7 +891,7 @@ __device__ void producer(const StepParams& SP, StepSmem<G>& S) {
                 }
             }
         }
-        x = atomicAdd(&sy->queue, 1u);
+        x = claim();
     }
 
     // ---- retrieval heads: finish the selection, then their tiles ----
@@ -793,8 +905,8 @@ __device__ void producer(const StepParams& SP, StepSmem<G>& S) {
                 for (uint32_t j = atomicAdd(&sy->pass_claim[pass], 1u); j < nitems && alive;
                      j = atomicAdd(&sy->pass_claim[pass], 1u)) {
                     Desc d{};
+                    if (!resolve_chunk(SP, (int)j, d)) continue;
                     d.type = IT_RADIX;
-                    d.item = (int)j;
                     d.aux0 = pass;
                     publish_nodata(d);
                 }
@@ -802,8 +914,8 @@ __device__ void producer(const StepParams& SP, StepSmem<G>& S) {
             }
             for (uint32_t j = atomicAdd(&sy->mark_claim, 1u); j < nitems && alive; j = atomicAdd(&sy->mark_claim, 1u)) {
                 Desc d{};
+                if (!resolve_chunk(SP, (int)j, d)) continue;
                 d.type = IT_MARK;
-                d.item = (int)j;
                 publish_nodata(d);
             }
             wait_for(&sy->mark_done, nrad);
@@ -868,7 +980,7 @@ __device__ void producer(const StepParams& SP, StepSmem<G>& S) {
                     bulk_g2s(&S.stage[st][TILE_BYTES], P.v_cache + off, TILE_BYTES, &S.full[st]);
                     ++t;
                 }
-                r = (int)atomicAdd(&sy->queue, 1u) - n_static;
+                r = (int)claim() - n_static;
             }
         }
     }
@@ -879,39 +991,68 @@ __device__ void producer(const StepParams& SP, StepSmem<G>& S) {
     // tile published into each stage to have landed
     for (uint32_t i = (t > (uint32_t)NST ? t - NST : 0u); i < t; ++i)
         mbar_wait_bounded(&S.full[i % NST], (i / NST) & 1u);
+    if (acct) {
+        atomicAdd(P.dbg_trace + 26, a_slot);
+        atomicAdd(P.dbg_trace + 27, a_dep);
+        atomicAdd(P.dbg_trace + 28, a_claim);
+    }
 }
 
 template <int G>
-__device__ void consumers(const StepParams& SP, StepSmem<G>& S, int tid) {
+__device__ __forceinline__ void consumers(const StepParams& SP, StepSmem<G>& S, int tid) {
     constexpr int NST = StepSmem<G>::NST;
     const Params& P = SP.P;
     AttnCore<G> core;
     ScoreState<G> sc;
     uint32_t t = 0;
     const int warp = tid >> 5, lane = tid & 31;
+    // cycle accounting for the debug trace (thread 0), by category:
+    // 0 wait for data, 1 score begin, 2 score tile, 3 score release, 4 score
+    // epilogue, 5 attention begin, 6 attention tile, 7 attention epilogue,
+    // 8 data-less items
+    const bool acct = P.dbg_trace != nullptr && tid == 0;
+    if (acct)
+        for (int i = 0; i < 10; ++i) S.acct[i] = 0ull;
+    long long c_mark = acct ? clock64() : 0;
+    auto mark = [&](int cat) {
+        if (!acct) return;
+        const long long now = clock64();
+        S.acct[cat] += (unsigned long long)(now - c_mark);
+        c_mark = now;
+    };
     while (true) {
         const int st = (int)(t % NST);
         const uint32_t par = (t / NST) & 1u;
+        mark(8);   // whatever ran since the last mark and was not classified
         if (!mbar_wait_bounded(&S.full[st], par)) {
             set_status(P, ST_TIMEOUT);
             break;
         }
+        mark(0);
         const Desc d = S.desc[st];
         const uint8_t* data = &S.stage[st][0];
         ++t;
         if (d.type == IT_STOP) break;
         if (d.type == IT_SCORE) {
             if (d.tile == 0) score_begin<G>(P, S, sc, d.b, d.grp, tid);
+            mark(1);
             score_tile<G>(P, S, sc, data, d.b, d.grp, d.n0, d.nvalid, tid);
+            mark(2);
+            if (acct) S.acct[9] += 1;
             consumer_sync();
             if (lane == 0) mbar_arrive(&S.empty[st]);
-            if (d.tile == d.ntiles - 1) score_end<G>(SP, S, sc, d.b, d.grp, d.item, d.aux1, d.aux0, tid);
+            mark(3);
+            if (d.tile == d.ntiles - 1) {
+                score_end<G>(SP, S, sc, d.b, d.grp, d.item, d.aux1, d.aux0, tid);
+                mark(4);
+            }
             continue;
         }
         if (d.type == IT_LOCAL || d.type == IT_RET) {
             const bool local = d.type == IT_LOCAL;
             const int g = local ? P.lg_group[d.grp] : P.rg_group[d.grp];
             if (d.tile == 0) core.begin(P, S, d.b, g, tid);
+            mark(5);
             if (d.bad) {
                 if (tid == 0) set_status(P, ST_DEVICE_INPUT);
             } else {
@@ -924,6 +1065,7 @@ __device__ void consumers(const StepParams& SP, StepSmem<G>& S, int tid) {
                 core.tile(S, data, d.hmask, d.n0, d.nvalid, local, s_end, w_lo, tid);
             }
             if (lane == 0) mbar_arrive(&S.empty[st]);
+            mark(6);
             if (d.tile == d.ntiles - 1) {
                 float* parts;
                 uint32_t heads, *ctr;
@@ -946,15 +1088,19 @@ __device__ void consumers(const StepParams& SP, StepSmem<G>& S, int tid) {
                     combine_parts<G>(P, S, parts, nitems, heads, d.b, g, tid);
                     if (tid == 0) trace_max(P, local ? 2 : 4);
                 }
+                mark(7);
             }
             continue;
         }
         // data-less items: release the slot first
         consumer_sync();
         if (lane == 0) mbar_arrive(&S.empty[st]);
-        if (d.type == IT_RADIX) radix_item<G>(SP, S, d.item, d.aux0, tid);
-        else if (d.type == IT_MARK) mark_item<G>(SP, S, d.item, tid);
+        if (d.type == IT_RADIX) radix_item<G>(SP, S, d.b, d.grp, d.item, d.aux1, d.aux0, tid);
+        else if (d.type == IT_MARK) mark_item<G>(SP, S, d.b, d.grp, d.item, d.aux1, tid);
         else if (d.type == IT_BLIST) blist_item<G>(SP, S, d.item, tid);
+    }
+    if (acct) {
+        for (int i = 0; i < 10; ++i) atomicAdd(P.dbg_trace + 16 + i, S.acct[i]);
     }
     (void)warp;
 }
@@ -970,6 +1116,7 @@ __global__ void __launch_bounds__(STEP_THREADS, (G >= 8) ? 1 : 2) step_kernel(co
             mbar_init(&S.full[i], 1);
             mbar_init(&S.empty[i], CONSUMERS / 32);
         }
+        S.qi_tag = 0;
         mbar_fence_init();
     }
     if (tid == 0 && SP.P.dbg_trace) atomicCAS(SP.P.dbg_trace, 0ull, (unsigned long long)global_ns());

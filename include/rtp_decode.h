@@ -59,7 +59,8 @@ typedef enum rtp_status {
     RTP_ERR_WORKSPACE = 4,     /* workspace missing or smaller than rtp_workspace_size() */
     RTP_ERR_CUDA = 5,          /* a CUDA launch or query failed */
     RTP_ERR_DEVICE_INPUT = 6,  /* device-side: bad seq_len, p or page id (see rtp_get_status) */
-    RTP_ERR_TIMEOUT = 7        /* device-side: a bounded wait inside a kernel gave up */
+    RTP_ERR_TIMEOUT = 7,       /* device-side: a bounded wait inside a kernel gave up */
+    RTP_ERR_SCRATCH_LIMIT = 8  /* rtp_decode_step_noalloc: the sizes need more than RTP_NOALLOC_SCRATCH_BYTES */
 } rtp_status;
 
 /*
@@ -154,6 +155,49 @@ rtp_status rtp_decode_step(const rtp_dims* dims, const uint16_t* q_pre, const ui
  * it.  For tests and debugging; it blocks the host.
  */
 rtp_status rtp_get_status(const rtp_dims* dims, void* stream);
+
+/*
+ * rtp_decode_step_noalloc -- the same decode step as rtp_decode_step, for
+ * callers that must not allocate device memory.  (No counterpart in the
+ * paper: it is a packaging variant of the library, not part of the method.)
+ *
+ * Who needs it: code that runs where cudaMalloc is off limits -- a plugin
+ * inside an inference engine whose memory pool owns all device memory and
+ * whose budget leaves nothing for a private allocation, or a caller on a hot
+ * loop that cannot afford cudaMalloc's implicit device-wide synchronisation.
+ * Such a caller cannot hand rtp_decode_step a workspace, so this entry point
+ * uses a scratch array compiled into the library instead.
+ *
+ * Arguments are those of rtp_decode_step, except:
+ *   dims->workspace and dims->workspace_bytes are ignored;
+ *   device_status: optional DEVICE uint32; after the step, on `stream`, it
+ *     receives this call's device-side status (0 = none, otherwise an
+ *     rtp_status such as RTP_ERR_DEVICE_INPUT).  NULL = not reported.
+ *     rtp_get_status() does not see these calls.
+ * Scratch and its limit: one static device array of RTP_NOALLOC_SCRATCH_BYTES
+ *   (64 MiB), held on every GPU that loads the library until the process
+ *   exits.  Sizes whose rtp_workspace_size() exceeds it are rejected with
+ *   RTP_ERR_SCRATCH_LIMIT before anything is enqueued.
+ * Allocation: none -- no cudaMalloc, cudaFree or allocating library call.
+ *   The call enqueues two cudaMemsetAsync (clearing the parts of the scratch
+ *   that the kernel expects at zero, since the array keeps whatever the
+ *   previous call left), the kernel, and, with device_status, one 4-byte
+ *   device-to-device cudaMemcpyAsync.
+ * Set-up: the first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress, with that device current; the library is loaded
+ *   onto the device then if it was not yet).  Make that first call outside
+ *   any stream capture.  A failed lookup returns RTP_ERR_CUDA.
+ * Concurrency: every call on a device shares the one array.  Calls whose
+ *   work overlaps on the GPU (different streams without ordering between
+ *   them) race on it and produce wrong results; order them on one stream.
+ */
+#define RTP_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+
+rtp_status rtp_decode_step_noalloc(const rtp_dims* dims, const uint16_t* q_pre, const uint16_t* q_rope,
+                                   const uint16_t* k_idx, const uint16_t* k_cache, const uint16_t* v_cache,
+                                   const uint16_t* Wq_idx, const int32_t* seq_lens, const uint8_t* head_kind,
+                                   const float* p, int32_t window, int32_t sink, uint16_t* out,
+                                   uint32_t* device_status, void* stream);
 
 /* Static string naming a status code. */
 const char* rtp_status_string(rtp_status status);

@@ -15,11 +15,12 @@ from typing import Optional
 from .build import LIB as _LIB_PATH
 
 __all__ = ["RTP_OK", "RtpError", "RtpDims", "RtpDebug", "lib", "status_string", "workspace_size", "decode_step",
-           "get_status", "Step", "PHASES", "TIMING_EVENTS"]
+           "get_status", "Step", "PHASES", "TIMING_EVENTS", "decode_step_noalloc", "NOALLOC_SCRATCH_BYTES"]
 
 RTP_OK = 0
 _STATUS_NAMES = {0: "RTP_OK", 1: "RTP_ERR_NULL", 2: "RTP_ERR_SHAPE", 3: "RTP_ERR_UNSUPPORTED", 4: "RTP_ERR_WORKSPACE",
-                 5: "RTP_ERR_CUDA", 6: "RTP_ERR_DEVICE_INPUT", 7: "RTP_ERR_TIMEOUT"}
+                 5: "RTP_ERR_CUDA", 6: "RTP_ERR_DEVICE_INPUT", 7: "RTP_ERR_TIMEOUT",
+                 8: "RTP_ERR_SCRATCH_LIMIT"}
 
 
 class RtpError(RuntimeError):
@@ -65,6 +66,9 @@ def _load():
     L.rtp_workspace_size.restype = ctypes.c_size_t
     L.rtp_decode_step.argtypes = [ctypes.POINTER(RtpDims), vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, vp, vp]
     L.rtp_decode_step.restype = ctypes.c_int
+    L.rtp_decode_step_noalloc.argtypes = [ctypes.POINTER(RtpDims), vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, vp,
+                                          vp, vp]
+    L.rtp_decode_step_noalloc.restype = ctypes.c_int
     L.rtp_get_status.argtypes = [ctypes.POINTER(RtpDims), vp]
     L.rtp_get_status.restype = ctypes.c_int
     L.rtp_status_string.argtypes = [ctypes.c_int]
@@ -116,6 +120,26 @@ def decode_step(dims: RtpDims, q_pre, q_rope, k_idx, k_cache, v_cache, Wq_idx, s
                              int(window), int(sink), _ptr(out), st)
     if rc != RTP_OK:
         raise RtpError(rc, "rtp_decode_step")
+
+
+# RTP_NOALLOC_SCRATCH_BYTES of the C header: the static scratch of rtp_decode_step_noalloc
+NOALLOC_SCRATCH_BYTES = 64 << 20
+
+
+def decode_step_noalloc(dims: RtpDims, q_pre, q_rope, k_idx, k_cache, v_cache, Wq_idx, seq_lens, head_kind, p,
+                        window: int, sink: int, out, device_status=None, stream=None) -> None:
+    """rtp_decode_step_noalloc: the decode step for callers that must not
+    allocate device memory (an engine plugin whose pool owns the GPU's memory,
+    a loop that cannot take cudaMalloc's synchronisation).  The library uses
+    its own static scratch array; dims.workspace is ignored.  device_status is
+    an optional device uint32 tensor that receives the call's device-side
+    status.  Calls that overlap on the GPU race on the shared scratch."""
+    st = 0 if stream is None else (stream if isinstance(stream, int) else stream.cuda_stream)
+    rc = lib.rtp_decode_step_noalloc(ctypes.byref(dims), _ptr(q_pre), _ptr(q_rope), _ptr(k_idx), _ptr(k_cache),
+                                     _ptr(v_cache), _ptr(Wq_idx), _ptr(seq_lens), _head_kind_buf(head_kind), _ptr(p),
+                                     int(window), int(sink), _ptr(out), _ptr(device_status), st)
+    if rc != RTP_OK:
+        raise RtpError(rc, "rtp_decode_step_noalloc")
 
 
 def get_status(dims: RtpDims, stream=None) -> int:

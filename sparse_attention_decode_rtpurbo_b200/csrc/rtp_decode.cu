@@ -6,6 +6,7 @@
 
 #include <algorithm>
 #include <atomic>
+#include <mutex>
 
 #include "../../include/rtp_decode.h"
 #include "rtp_step_kernel.cuh"
@@ -277,6 +278,82 @@ extern "C" rtp_status rtp_get_status(const rtp_dims* dims, void* stream) {
     return (rtp_status)word;
 }
 
+// ---------------------------------------------------------------------------
+// Allocation-free variant.  Callers that may not allocate device memory (an
+// engine plugin whose pool owns every byte of the GPU, a loop that cannot take
+// cudaMalloc's device-wide synchronisation) get the same step with its scratch
+// in a device array built into the library.  The array is only reachable from
+// host code through the address looked up below: its host-side name is a
+// stand-in, not a device pointer.
+namespace rtp {
+
+static __device__ __align__(256) uint8_t noalloc_scratch[RTP_NOALLOC_SCRATCH_BYTES];
+
+constexpr int NOALLOC_MAX_DEVICES = 64;
+static std::atomic<void*> noalloc_addr[NOALLOC_MAX_DEVICES];
+static std::mutex noalloc_mutex;
+
+// Device address of noalloc_scratch on the current device, looked up once per
+// device (the lookup loads the module onto the device if needed).
+static cudaError_t noalloc_scratch_ptr(uint8_t** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= NOALLOC_MAX_DEVICES) return cudaErrorInvalidDevice;
+    void* a = noalloc_addr[dev].load(std::memory_order_acquire);
+    if (!a) {
+        std::lock_guard<std::mutex> lock(noalloc_mutex);
+        a = noalloc_addr[dev].load(std::memory_order_acquire);
+        if (!a) {
+            e = cudaGetSymbolAddress(&a, noalloc_scratch);
+            if (e != cudaSuccess) return e;
+            if (!a) return cudaErrorInvalidSymbol;
+            noalloc_addr[dev].store(a, std::memory_order_release);
+        }
+    }
+    *out = static_cast<uint8_t*>(a);
+    return cudaSuccess;
+}
+
+}  // namespace rtp
+
+extern "C" rtp_status rtp_decode_step_noalloc(const rtp_dims* dims, const uint16_t* q_pre, const uint16_t* q_rope,
+                                              const uint16_t* k_idx, const uint16_t* k_cache,
+                                              const uint16_t* v_cache, const uint16_t* Wq_idx,
+                                              const int32_t* seq_lens, const uint8_t* head_kind, const float* p,
+                                              int32_t window, int32_t sink, uint16_t* out, uint32_t* device_status,
+                                              void* stream) {
+    // every host-side check runs before anything is enqueued
+    if (!dims || !q_pre || !q_rope || !k_idx || !k_cache || !v_cache || !Wq_idx || !seq_lens || !head_kind || !p ||
+        !out)
+        return RTP_ERR_NULL;
+    if (window < 0 || sink < 0 || (int64_t)window + sink < 1) return RTP_ERR_SHAPE;
+    Plan pl;
+    rtp_status st = make_plan(dims, head_kind, window, sink, &pl);
+    if (st != RTP_OK) return st;
+    if (pl.total > RTP_NOALLOC_SCRATCH_BYTES) return RTP_ERR_SCRATCH_LIMIT;
+    uint8_t* ws = nullptr;
+    if (noalloc_scratch_ptr(&ws) != cudaSuccess) return RTP_ERR_CUDA;
+    cudaStream_t s = (cudaStream_t)stream;
+    // The array keeps the previous call's contents, possibly laid out for
+    // other sizes.  The kernel expects zero in the status word, the
+    // cross-CTA counters and ticket words ([0, o_keys)) and in the per-head
+    // bucket aggregates and radix histograms ([o_agg, o_chunk_cnt)); every
+    // other region is written before it is read.
+    if (cudaMemsetAsync(ws, 0, pl.o_keys, s) != cudaSuccess) return RTP_ERR_CUDA;
+    if (cudaMemsetAsync(ws + pl.o_agg, 0, pl.o_chunk_cnt - pl.o_agg, s) != cudaSuccess) return RTP_ERR_CUDA;
+    rtp_dims d = *dims;
+    d.workspace = ws;
+    d.workspace_bytes = RTP_NOALLOC_SCRATCH_BYTES;
+    st = rtp_decode_step(&d, q_pre, q_rope, k_idx, k_cache, v_cache, Wq_idx, seq_lens, head_kind, p, window, sink,
+                         out, stream);
+    if (st != RTP_OK) return st;
+    if (device_status &&
+        cudaMemcpyAsync(device_status, ws + pl.o_status, sizeof(uint32_t), cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+        return RTP_ERR_CUDA;
+    return RTP_OK;
+}
+
 extern "C" const char* rtp_status_string(rtp_status status) {
     switch (status) {
         case RTP_OK: return "ok";
@@ -287,6 +364,7 @@ extern "C" const char* rtp_status_string(rtp_status status) {
         case RTP_ERR_CUDA: return "CUDA error";
         case RTP_ERR_DEVICE_INPUT: return "device-side input error (seq_len, p or page id)";
         case RTP_ERR_TIMEOUT: return "a bounded wait inside a kernel timed out";
+        case RTP_ERR_SCRATCH_LIMIT: return "sizes need more scratch than the no-alloc entry point's static array";
     }
     return "unknown status";
 }

@@ -228,21 +228,29 @@ def main():
         flush_w.zero_()
         flush_r.sum(dtype=torch.int64)
 
-    # one step = one replay of a CUDA graph holding the rtp_decode_step launches
+    # one step = one replay of a CUDA graph holding one rtp_decode_step (its
+    # two kernels).  A second graph records phase events between the kernels
+    # (which serialises them); it is replayed separately for the per-kernel
+    # durations, never inside the timed steps.
     NE = rtp.TIMING_EVENTS
     inner = [torch.cuda.Event(enable_timing=True) for _ in range(NE)]
     for e in inner:
         e.record(stream)
     dc.run(stream)                               # eager warm-up (sets kernel attributes)
     torch.cuda.synchronize(dev)
-    dc.step.set_timing_events(inner)
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph):
+        dc.run(torch.cuda.current_stream(dev))
+    dc.step.set_timing_events(inner)
+    graph_ev = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph_ev):
         dc.run(torch.cuda.current_stream(dev))
     dc.step.set_timing_events(None)
     for _ in range(max(3, args.warmup)):
         flush()
         graph.replay()
+        flush()
+        graph_ev.replay()
     torch.cuda.synchronize(dev)
 
     sampler = ClockSampler(local_rank)
@@ -261,12 +269,16 @@ def main():
         z.record(stream)
         z.synchronize()
         step_ms.append(a.elapsed_time(z))
-        for k in range(len(rtp.PHASES)):
-            phase_acc[k] += inner[k].elapsed_time(inner[k + 1])
     torch.cuda.synchronize(dev)
     barrier()
     wall = time.perf_counter() - t_begin
     clocks = sampler.stop()
+    for i in range(args.steps):
+        flush()
+        graph_ev.replay()
+        inner[-1].synchronize()
+        for k in range(len(rtp.PHASES)):
+            phase_acc[k] += inner[k].elapsed_time(inner[k + 1])
     phase_ms = {n: phase_acc[k] / args.steps for k, n in enumerate(rtp.PHASES)}
     t_ms = statistics.mean(step_ms)
 
@@ -282,7 +294,10 @@ def main():
         torch.cuda.synchronize(dev)
         t = trace_buf.cpu().numpy().astype(np.float64)
         ev = {n: (t[k] - t[0]) / 1e3 if t[k] > 0 else None for k, n in enumerate(rtp.TRACE_EVENTS) if k}
-        ev.update({n: t[16 + k] for k, n in enumerate(rtp.TRACE_SUMS)})
+        for k, n in enumerate(rtp.TRACE_SUMS):
+            v = t[16 + k]
+            # timestamps (ns) become times since the start; cycle sums stay raw
+            ev[n] = ((v - t[0]) / 1e3 if v > 0 else None) if n in ("a_first_data", "a_consumers_done") else v
         tl.append(ev)
     dc.step.dims.debug = ctypes.POINTER(rtp.RtpDebug)()
     timeline = {n: (statistics.median([x[n] for x in tl]) if tl[0][n] is not None else None)
@@ -326,11 +341,16 @@ def main():
     tokens = float(case.seq_lens.sum())
     value = world * tokens / (t_ms * 1e-3)
     peak, peak_kind = hbm_peak()
-    # the whole step is one kernel launch (rtp::step_kernel): it is the dominant kernel
-    dom = "step"
-    ach = nbytes["total"] / (phase_ms[dom] * 1e-3) / 1e9
+    # two launches per step: rtp::stream_kernel (index cache + local heads'
+    # sink/window K/V) and, when there are retrieval heads,
+    # rtp::retrieve_kernel (kept K/V blocks; exact select when needed).
+    # The roofline is reported for the one that takes longer.
+    kbytes = {"stream": nbytes["index"] + nbytes["local"], "retrieve": nbytes["kept_kv"]}
+    has_ret = bool(case.head_kind.any())
+    dom = "retrieve" if has_ret and phase_ms["retrieve"] > phase_ms["stream"] else "stream"
+    ach = kbytes[dom] / (phase_ms[dom] * 1e-3) / 1e9
     step_gbs = nbytes["total"] / (t_ms * 1e-3) / 1e9
-    launches_per_step = 1
+    launches_per_step = 2 if has_ret else 1
 
     line = None
     if rank == 0:
@@ -354,12 +374,13 @@ def main():
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16 in, fp32 accumulate",
             "data": "synthetic (seeded; see DESIGN.md input recipe)",
             "config": dict(workload_config(case, args.workload), parallelism=f"replicas x{world}",
-                           dense_p1=bool(args.dense), timing="CUDA-graph replay of one rtp_decode_step per step; "
+                           dense_p1=bool(args.dense), timing="CUDA-graph replay of one rtp_decode_step (2 kernels, programmatic launch) per step; "
                            "CUDA events on the launching stream"),
             "wall_s_timed_loop": wall,
-            "roofline": {"bound": "hbm", "kernel": "rtp::step_kernel", "achieved": ach, "peak": peak, "unit": "GB/s",
+            "roofline": {"bound": "hbm", "kernel": f"rtp::{dom}_kernel", "achieved": ach, "peak": peak, "unit": "GB/s",
                          "frac": ach / peak, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, burst)",
-                         "traffic": None, "algorithmic_bytes_per_launch": nbytes["total"]},
+                         "traffic": None, "algorithmic_bytes_per_launch": kbytes[dom],
+                         "us_per_launch": phase_ms[dom] * 1e3},
             "step_roofline": {"algorithmic_bytes": nbytes, "achieved": step_gbs, "peak": peak, "unit": "GB/s",
                               "frac": step_gbs / peak},
             "phases_us": {n: phase_ms[n] * 1e3 for n in rtp.PHASES},

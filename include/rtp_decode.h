@@ -98,11 +98,13 @@ typedef struct rtp_debug {
  *   debug: host pointer to an rtp_debug of device pointers, or NULL.
  *   timing_events / n_timing_events: optional host array of cudaEvent_t
  *     handles (created by the caller).  When n_timing_events >=
- *     RTP_TIMING_EVENTS the call records event 0 on `stream` just before its
- *     kernel and event 1 just after it (external event nodes when the stream
- *     is being captured into a CUDA graph).
+ *     RTP_TIMING_EVENTS the call records, on `stream`, event 0 just before
+ *     its first kernel (index scores + local heads), event 1 between it and
+ *     the second kernel (exact select + retrieval heads; absent when no head
+ *     is a retrieval head) and event 2 after the last kernel (external event
+ *     nodes when the stream is being captured into a CUDA graph).
  */
-enum { RTP_TIMING_EVENTS = 2 };
+enum { RTP_TIMING_EVENTS = 3 };
 
 typedef struct rtp_dims {
     int32_t batch, num_q_heads, num_kv_heads;
@@ -179,9 +181,9 @@ rtp_status rtp_get_status(const rtp_dims* dims, void* stream);
  *   exits.  Sizes whose rtp_workspace_size() exceeds it are rejected with
  *   RTP_ERR_SCRATCH_LIMIT before anything is enqueued.
  * Allocation: none -- no cudaMalloc, cudaFree or allocating library call.
- *   The call enqueues two cudaMemsetAsync (clearing the parts of the scratch
- *   that the kernel expects at zero, since the array keeps whatever the
- *   previous call left), the kernel, and, with device_status, one 4-byte
+ *   The call enqueues one cudaMemsetAsync (clearing the part of the scratch
+ *   that the kernels expect at zero, since the array keeps whatever the
+ *   previous call left), the kernels, and, with device_status, one 4-byte
  *   device-to-device cudaMemcpyAsync.
  * Set-up: the first call on each device looks up the array's device address
  *   (cudaGetSymbolAddress, with that device current; the library is loaded

@@ -36,11 +36,12 @@ class RtpDebug(ctypes.Structure):
 
 
 TRACE_EVENTS = ["start", "select_done", "local_done", "lists_ready", "retrieval_done", "end", "select_start",
-                "local_combine_start", "radix1", "radix2", "radix3", "radix4", "mark"]
-# summed over CTAs (slots 16..28): consumer SM cycles by category, then producer ns
-TRACE_SUMS = ["cyc_wait", "cyc_score_begin", "cyc_score_tile", "cyc_score_release", "cyc_score_epilogue",
-              "cyc_attn_begin", "cyc_attn_tile", "cyc_attn_epilogue", "cyc_other", "n_score_tiles",
-              "ns_prod_slot", "ns_prod_dep", "ns_prod_claim"]
+                "stream_work_start", "radix1", "radix2", "radix3", "radix4", "mark", "ret_kernel_start", "pass0_hist",
+                "attn_start"]
+# debug sums (slots 16..): SM cycles of one thread per CTA by category, counts,
+# and the latest %globaltimer of two events
+TRACE_SUMS = ["a_cyc_wait", "a_cyc_score", "a_cyc_attn", "a_n_score", "a_n_attn", "a_cyc_split", "a_first_data",
+              "a_consumers_done", "b_cyc_pass_tile", "b_n_pass_tiles", "b_cyc_pass_wait", "b_cyc_pass_other"]
 
 
 class RtpDims(ctypes.Structure):
@@ -53,7 +54,7 @@ class RtpDims(ctypes.Structure):
                 ("n_timing_events", ctypes.c_int32)]
 
 
-PHASES = ["step"]
+PHASES = ["stream", "retrieve"]
 TIMING_EVENTS = len(PHASES) + 1
 
 

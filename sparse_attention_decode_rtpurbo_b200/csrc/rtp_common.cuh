@@ -1,24 +1,23 @@
 // Shared definitions of the RTPurbo decode-step kernels (sm_100a).
 #pragma once
+#include <cuda.h>   // CUtensorMap
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
 namespace rtp {
 
-constexpr int D = 128;          // head dimension
-constexpr int R = 16;           // indexer rank
-constexpr int BLK = 64;         // KV block (page) size in tokens
-constexpr int CHUNK = 2048;         // tokens per selection item (= 32 blocks = one bitmap word)
-constexpr int SCORE_CHUNK = 2048;   // tokens per index-score item (2 staged tiles)
-constexpr int SEL_THREADS = 256;
-constexpr int ATT_THREADS = 128;
-constexpr int STAGES = 3;                       // K/V tile ring depth of the attention kernels
-constexpr int TILE_BYTES = BLK * D * 2;         // one 64x128 bf16 tile = 16 KB
-constexpr int STAGE_BYTES = 2 * TILE_BYTES;     // K + V
-constexpr int PSTRIDE = 132;                    // floats per partial: m, l, 2 pad, acc[128]
-constexpr int MAX_G = 8, MAX_HQ = 128, MAX_HKV = 64;
-constexpr double FIX_SCALE = 1099511627776.0;   // 2^40: fixed-point unit of softmax mass
+constexpr int D = 128;            // head dimension
+constexpr int R = 16;             // indexer rank
+constexpr int BLK = 64;           // KV block (page) size in tokens
+constexpr int SROWS = 1024;       // k_idx rows per index tile (32 KB)
+constexpr int STAGE_BYTES = 32768;   // one ring stage: an index tile, or a 64-token K tile + V tile
+constexpr int KV_TILE = 16384;       // one 64 x 128 bf16 tile (two 64 x 64 TMA boxes, 128-byte swizzle)
+constexpr int CONSUMERS = 128;    // 4 compute warps
+constexpr int THREADS = CONSUMERS + 32;   // + 1 copy warp
+constexpr int PSTRIDE = 132;      // floats per split partial: m, l, 2 pad, acc[128]
+constexpr int MAX_G = 8, MAX_HQ = 128, MAX_HKV = 64, MAX_B = 1024;
+constexpr int AGG_BUCKETS = 32;
 
 enum SelMode : int32_t { MODE_SKIP = 0, MODE_TOP1 = 1, MODE_ALL = 2, MODE_RADIX = 3 };
 
@@ -26,12 +25,11 @@ enum SelMode : int32_t { MODE_SKIP = 0, MODE_TOP1 = 1, MODE_ALL = 2, MODE_RADIX 
 constexpr uint32_t ST_DEVICE_INPUT = 6;
 constexpr uint32_t ST_TIMEOUT = 7;
 
-// Per retrieval head and bucket (chunk mod AGG_BUCKETS), folded by score
-// chunks with fire-and-forget atomics (all-zero = empty, so a zero-filled
-// workspace is ready): best = (max key << 32) | ~argmax, nmin = ~(min key),
-// zabs = fp64 sum of exp(s/4), flags bit 0 = a chunk's scores left the range
-// where that sum is safe.  Buckets keep same-address atomics rare.
-constexpr int AGG_BUCKETS = 32;
+// Per retrieval head and bucket (split mod AGG_BUCKETS), folded by the
+// index-score splits with fire-and-forget atomics (all-zero = empty, so a
+// zero-filled workspace is ready): best = (max key << 32) | ~argmax,
+// nmin = ~(min key), zabs = fp64 sum of exp(s/4), flags bit 0 = a split's
+// scores left the range where that sum is safe.
 struct HeadAgg {
     unsigned long long best;
     uint32_t nmin, flags;
@@ -44,14 +42,25 @@ struct HeadState {
     uint32_t maxkey, argmax, minkey, pad0;
     double zrel;                            // sum over n < L of exp((s_n - smax)/4)
     unsigned long long target, mass_above;  // fixed-point masses (units of 2^-40)
-    uint32_t prefix, count_above, n_eq, n_tie, all_ties, kstar, tau_key, pad1;
+    uint32_t prefix, count_above, n_eq, n_tie, all_ties, kstar, tau_key;
+    uint32_t tie_idx;                       // largest index among the threshold ties kept
+};
+
+// Coordination words of one call (workspace; zero between calls).
+struct Sync {
+    uint32_t n_radix_heads;    // heads needing the exact select (list in rlist)
+    uint32_t n_radix_groups;   // (b, group) pairs holding such heads (list in rglist)
+    uint32_t any_ties;         // some radix head takes only part of its threshold ties
+    uint32_t barrier;          // grid barrier arrivals of the retrieval kernel
+    uint32_t exit_count;
+    uint32_t groups_decided;   // (b, retrieval group) pairs whose selection mode is known
+    uint32_t pad[26];
 };
 
 struct Params {
-    int B, Hq, Hkv, G, Ncap, nblk_cap, words_cap, mbps, num_pages, window, sink;
-    int n_ret, n_rg, n_lg, nchunks, nschunks;
-    int local_kb, local_items, ret_grid;
-    const uint16_t *q_pre, *q_rope, *k_idx, *k_cache, *v_cache, *Wq;
+    int B, Hq, Hkv, G, Ncap, nblk_cap, words_cap, ntiles_cap, mbps, num_pages, window, sink;
+    int n_ret, n_rg, n_lg;
+    const uint16_t *q_pre, *q_rope, *k_idx, *Wq;
     const int32_t *seq_lens, *block_table;
     const float* p;
     uint16_t* out;
@@ -62,14 +71,14 @@ struct Params {
     uint8_t slot_head[MAX_HQ], slot_rg[MAX_HQ];
     // workspace
     uint32_t* status;
-    uint32_t *tick_score, *tick_radix, *tick_local, *tick_ret;
-    uint32_t* keys;
+    Sync* sync;
+    uint32_t *rlist, *rglist;
+    uint32_t *tick_score, *tick_local, *tick_ret;
     HeadAgg* agg;
     HeadState* hs;
     uint32_t* hist_cnt;
     unsigned long long* hist_mass;
-    uint32_t* chunk_cnt;
-    uint32_t* tie_off;
+    uint32_t* tie_cnt;
     uint32_t* bitmap;
     uint32_t* blist;
     uint32_t* bcount;
@@ -85,11 +94,22 @@ struct Params {
     unsigned long long* dbg_trace;
 };
 
+// Kernel argument block: the tensor maps of the K and V caches (2-D:
+// rows x 128 bf16, 64 x 64 boxes, 128-byte swizzle) travel as grid constants.
+struct KParams {
+    CUtensorMap tmk, tmv;
+    Params P;
+};
+
 // ---------------------------------------------------------------------------
 // small helpers
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float bf_lo(uint32_t u) { return __uint_as_float(u << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(lo)) |
+           ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hi)) << 16);
+}
 
 // order-preserving map fp32 -> uint32 (larger float, larger key)
 __device__ __forceinline__ uint32_t f2key(float f) {
@@ -111,44 +131,20 @@ __device__ __forceinline__ void set_status(const Params& P, uint32_t code) { ato
 
 __device__ __forceinline__ bool seq_ok(const Params& P, int L) { return L >= 1 && L <= P.Ncap; }
 
-// Page id of block j of sequence b (paged layout), or -1 when out of range.
-__device__ __forceinline__ int page_of(const Params& P, int b, int j) {
-    int pg = __ldg(P.block_table + (int64_t)b * P.mbps + j);
-    return (pg >= 0 && pg < P.num_pages) ? pg : -1;
+// Page id of block j of sequence b (paged layout); an id outside
+// [0, num_pages) records an input error and reads page 0 instead.
+__device__ __forceinline__ int page_or_zero(const Params& P, int b, int j) {
+    const int pg = __ldg(P.block_table + (int64_t)b * P.mbps + j);
+    if (pg >= 0 && pg < P.num_pages) return pg;
+    set_status(P, ST_DEVICE_INPUT);
+    return 0;
 }
 
-// Element offset of row n of KV head g of sequence b in a cache of row width `dim`.
-__device__ __forceinline__ int64_t row_off(const Params& P, int b, int g, int n, int dim, bool* bad) {
-    if (P.block_table == nullptr) return (((int64_t)b * P.Hkv + g) * P.Ncap + n) * dim;
-    int pg = page_of(P, b, n / BLK);
-    if (pg < 0) {
-        *bad = true;
-        pg = 0;
-    }
-    return (((int64_t)pg * P.Hkv + g) * BLK + (n % BLK)) * dim;
+// First cache row (of `rows x dim` views) of block j of KV head g of sequence b.
+__device__ __forceinline__ int64_t block_row(const Params& P, int b, int g, int j) {
+    if (P.block_table == nullptr) return ((int64_t)b * P.Hkv + g) * P.Ncap + (int64_t)j * BLK;
+    return ((int64_t)page_or_zero(P, b, j) * P.Hkv + g) * BLK;
 }
-
-// Ticket: returns true in exactly one (the last) of `count` arrivals, and
-// re-arms the counter for the next call.  Caller has done __syncthreads().
-__device__ __forceinline__ bool last_arrival(uint32_t* ctr, uint32_t count, uint32_t* smem_flag) {
-    if (threadIdx.x == 0) {
-        __threadfence();
-        uint32_t t = atomicAdd(ctr, 1u);
-        bool last = (t == count - 1);
-        if (last) {
-            atomicExch(ctr, 0u);
-            __threadfence();
-        }
-        *smem_flag = last;
-    }
-    __syncthreads();
-    return *smem_flag != 0;
-}
-
-// ---------------------------------------------------------------------------
-// mbarrier + bulk copy (TMA engine, non-tensor form)
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
 // 2^x on the special-function unit (about 2 ulp; 0 for x = -inf)
 __device__ __forceinline__ float ex2_approx(float x) {
@@ -157,19 +153,59 @@ __device__ __forceinline__ float ex2_approx(float x) {
     return y;
 }
 
-// 16-byte load from a shared-memory address (explicit shared state space)
-__device__ __forceinline__ uint4 lds128(uint32_t addr) {
-    uint4 v;
-    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+__device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
 }
 
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+
+// optional timeline (debug): latest %globaltimer of event i
+__device__ __forceinline__ void trace_max(const Params& P, int i) {
+    if (P.dbg_trace) atomicMax(P.dbg_trace + i, (unsigned long long)global_ns());
+}
+
+// optional cycle accounting (debug, one thread per CTA): the SM cycles since
+// the previous mark are added to trace slot `slot`
+struct Acct {
+    unsigned long long* tr;
+    long long t;
+    __device__ __forceinline__ void init(const Params& P, bool me) {
+        tr = me ? P.dbg_trace : nullptr;
+        if (tr) t = clock64();
+    }
+    __device__ __forceinline__ void mark(int slot) {
+        if (!tr) return;
+        const long long now = clock64();
+        atomicAdd(tr + slot, (unsigned long long)(now - t));
+        t = now;
+    }
+    __device__ __forceinline__ void count(int slot) {
+        if (tr) atomicAdd(tr + slot, 1ull);
+    }
+};
+
+// ---------------------------------------------------------------------------
+// mbarrier, bulk copies and TMA tensor copies
+// ---------------------------------------------------------------------------
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
 }
 __device__ __forceinline__ void mbar_fence_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
 __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     uint32_t ok;
@@ -180,11 +216,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
-__device__ __forceinline__ uint64_t global_ns() {
-    uint64_t t;
-    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
-    return t;
-}
 // Bounded wait: gives up after about two seconds of wall time.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -194,26 +225,69 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
         if ((i & 255u) == 0 && global_ns() - t0 > 2000000000ull) return false;
     }
 }
+// Plain bulk copy global -> shared (16-byte aligned, size a multiple of 16).
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
     asm volatile(
         "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(smem_u32(dst)),
         "l"(src), "r"(bytes), "r"(smem_u32(bar))
         : "memory");
 }
+// One 2-D TMA box (x = column, y = row) into shared memory (1024-byte aligned
+// for the 128-byte swizzle).  x is 0 or 64 here: 128-byte aligned.
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
+            "r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
-// One 32-byte row read once: 256-bit load, not kept in L1, evicted early from L2.
-// The address must be 32-byte aligned.
-struct U8x32 {
-    uint32_t w[8];
-};
-__device__ __forceinline__ U8x32 ld_stream32(const void* p) {
-    U8x32 v;
-    asm volatile("ld.global.nc.L1::no_allocate.L2::evict_first.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-                 : "=r"(v.w[0]), "=r"(v.w[1]), "=r"(v.w[2]), "=r"(v.w[3]), "=r"(v.w[4]), "=r"(v.w[5]), "=r"(v.w[6]),
-                   "=r"(v.w[7])
-                 : "l"(p));
+// 16-byte load from a shared-memory address
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
     return v;
+}
+__device__ __forceinline__ void sts128_zero(uint32_t addr) {
+    asm volatile("st.shared.v4.u32 [%0], {%1,%1,%1,%1};" ::"r"(addr), "r"(0u) : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// warp-level tensor-core primitives (bf16 in, fp32 accumulate)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+// c += A(16x16, row) * B(16x8, col)
+__device__ __forceinline__ void mma_bf16(float* c, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                         uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// per-sequence geometry of the local heads' block list: sink blocks
+// [0, nA), then window blocks [bw0, bw0 + nv - nA)
+struct LocalGeom {
+    int s_end, w_lo, nA, bw0, nv;
+};
+__device__ __forceinline__ LocalGeom local_geom(const Params& P, int L) {
+    LocalGeom g;
+    g.s_end = min(P.sink, L);
+    g.w_lo = P.window > 0 ? max(0, L - P.window) : L;
+    g.nA = (g.s_end + BLK - 1) / BLK;
+    g.bw0 = max(g.w_lo / BLK, g.nA);
+    const int nB = P.window > 0 ? max(0, (L + BLK - 1) / BLK - g.bw0) : 0;
+    g.nv = g.nA + nB;
+    return g;
 }
 
 }  // namespace rtp

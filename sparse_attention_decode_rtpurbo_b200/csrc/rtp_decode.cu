@@ -1,31 +1,37 @@
-// C ABI of the RTPurbo decode step: argument checks, workspace layout and the
-// launch of the persistent sm_100a decode-step kernel (rtp_step.cuh, rtp_step_kernel.cuh).
+// C ABI of the RTPurbo decode step: argument checks, workspace layout, the
+// TMA tensor maps of the K/V caches, and the launches of the two sm_100a
+// kernels (rtp_stream.cuh: index scores + local heads; rtp_retrieve.cuh:
+// exact select when needed + retrieval heads).
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 #include <string.h>
+
+#include <stdio.h>
+#include <stdlib.h>
 
 #include <algorithm>
 #include <atomic>
 #include <mutex>
 
 #include "../../include/rtp_decode.h"
-#include "rtp_step_kernel.cuh"
+#include "rtp_retrieve.cuh"
 
 namespace rtp {
 
-constexpr int NSM_PLAN = 148;       // SMs of a B200: sizes the split counts
-constexpr int MAX_GRID = 148 * 4;   // upper bound of the persistent grid (partials are sized for it)
+constexpr int MAX_GRID = 148 * 4;   // upper bound of either grid (split partials are sized for it)
+constexpr int MAX_RET_GROUPS = 4096;   // B * (KV groups with retrieval heads) held in shared memory
 
 struct Plan {
-    int B, Hq, Hkv, G, Ncap, nblk_cap, words_cap, nchunks, nschunks;
+    int B, Hq, Hkv, G, Ncap, nblk_cap, words_cap, ntiles_cap;
     int n_ret, n_rg, n_lg;
-    int local_kb, local_items, ret_grid;
+    long long tiles_cap;   // upper bound of the streaming kernel's tiles
     uint8_t rg_group[MAX_HKV], rg_mask[MAX_HKV], rg_slot0[MAX_HKV], rg_nh[MAX_HKV];
     uint8_t lg_group[MAX_HKV], lg_mask[MAX_HKV];
     uint8_t slot_head[MAX_HQ], slot_rg[MAX_HQ];
-    // workspace byte offsets
-    size_t o_status, o_sync, o_rlist, o_rglist, o_tick_score, o_tick_radix, o_tick_local, o_tick_ret, o_keys, o_agg,
-        o_hs, o_hist_cnt, o_hist_mass, o_chunk_cnt, o_tie_off, o_bitmap, o_blist, o_bcount, o_lpart, o_rpart, total;
+    // workspace byte offsets; [0, zero_end) must be zero when a call starts
+    size_t o_status, o_sync, o_tick_score, o_tick_local, o_tick_ret, o_agg, o_hist_cnt, o_hist_mass, zero_end;
+    size_t o_rlist, o_rglist, o_hs, o_tie_cnt, o_bitmap, o_blist, o_bcount, o_lpart, o_rpart, total;
 };
 
 static size_t align_up(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -37,12 +43,15 @@ static rtp_status check_dims(const rtp_dims* d) {
     if (d->num_q_heads % d->num_kv_heads) return RTP_ERR_SHAPE;
     const int G = d->num_q_heads / d->num_kv_heads;
     if (G != 1 && G != 2 && G != 4 && G != 8) return RTP_ERR_UNSUPPORTED;
-    if (d->num_q_heads > MAX_HQ || d->num_kv_heads > MAX_HKV) return RTP_ERR_UNSUPPORTED;
+    if (d->num_q_heads > MAX_HQ || d->num_kv_heads > MAX_HKV || d->batch > MAX_B) return RTP_ERR_UNSUPPORTED;
     if (d->max_seq_len < BLK || d->max_seq_len % BLK) return RTP_ERR_SHAPE;
     if (d->max_seq_len > (1 << 28)) return RTP_ERR_UNSUPPORTED;
     if (d->block_table) {
         if (d->max_blocks_per_seq < 1 || d->num_pages < 1) return RTP_ERR_SHAPE;
         if ((int64_t)d->max_blocks_per_seq * BLK != d->max_seq_len) return RTP_ERR_SHAPE;
+        if ((int64_t)d->num_pages * d->num_kv_heads * BLK >= (1ll << 31)) return RTP_ERR_UNSUPPORTED;
+    } else if ((int64_t)d->batch * d->num_kv_heads * d->max_seq_len >= (1ll << 31)) {
+        return RTP_ERR_UNSUPPORTED;   // TMA row coordinates are 32-bit
     }
     return RTP_OK;
 }
@@ -59,8 +68,7 @@ static rtp_status make_plan(const rtp_dims* d, const uint8_t* head_kind, int win
     pl->Ncap = d->max_seq_len;
     pl->nblk_cap = pl->Ncap / BLK;
     pl->words_cap = (pl->nblk_cap + 31) / 32;
-    pl->nchunks = (pl->Ncap + CHUNK - 1) / CHUNK;
-    pl->nschunks = (pl->Ncap + SCORE_CHUNK - 1) / SCORE_CHUNK;
+    pl->ntiles_cap = (pl->Ncap + SROWS - 1) / SROWS;
     for (int g = 0; g < pl->Hkv; ++g) {
         uint32_t rm = 0, lm = 0;
         for (int i = 0; i < pl->G; ++i) {
@@ -88,17 +96,12 @@ static rtp_status make_plan(const rtp_dims* d, const uint8_t* head_kind, int win
             pl->lg_mask[l] = (uint8_t)lm;
         }
     }
-    // local heads: list of at most nv_max blocks per (b, group), cut into items
-    if (pl->n_lg) {
-        const int64_t nv_max = std::min<int64_t>(pl->nblk_cap, (sink + BLK - 1) / BLK + (window + BLK - 1) / BLK + 1);
-        const int64_t total = (int64_t)pl->B * pl->n_lg * nv_max;
-        pl->local_kb = (int)std::max<int64_t>(4, (total + 2 * NSM_PLAN - 1) / (2 * NSM_PLAN));
-        // the split combine keeps one weight per (head, split) in 512*G floats
-        pl->local_kb = (int)std::max<int64_t>(pl->local_kb, (nv_max + 511) / 512);
-        pl->local_items = (int)((nv_max + pl->local_kb - 1) / pl->local_kb);
+    if ((long long)pl->B * pl->n_rg > MAX_RET_GROUPS) return RTP_ERR_UNSUPPORTED;
+    {
+        const long long nv_max = std::min<long long>(
+            pl->nblk_cap, (sink + BLK - 1) / BLK + (window > 0 ? (window + BLK - 1) / BLK + 1 : 0));
+        pl->tiles_cap = (long long)pl->B * (pl->n_rg * (long long)pl->ntiles_cap + pl->n_lg * nv_max);
     }
-    pl->ret_grid = MAX_GRID;
-    // workspace layout
     const size_t BR = (size_t)pl->B * pl->n_ret, BG = (size_t)pl->B * pl->n_rg, BL = (size_t)pl->B * pl->n_lg;
     size_t o = 0;
     auto take = [&](size_t bytes) {
@@ -108,61 +111,148 @@ static rtp_status make_plan(const rtp_dims* d, const uint8_t* head_kind, int win
     };
     pl->o_status = take(64);
     pl->o_sync = take(sizeof(Sync));
-    pl->o_rlist = take(BR * 4);
-    pl->o_rglist = take(BG * 4);
     pl->o_tick_score = take(BG * 4);
-    pl->o_tick_radix = take(BR * 4);
     pl->o_tick_local = take(BL * 4);
     pl->o_tick_ret = take(BG * 4);
-    pl->o_keys = take(BR * pl->Ncap * 4);
     pl->o_agg = take(BR * AGG_BUCKETS * sizeof(HeadAgg));
-    pl->o_hs = take(BR * sizeof(HeadState));
     pl->o_hist_cnt = take(BR * 256 * 4);
     pl->o_hist_mass = take(BR * 256 * 8);
-    pl->o_chunk_cnt = take(BR * pl->nchunks * 256 * 4);
-    pl->o_tie_off = take(BR * pl->nchunks * 4);
+    pl->zero_end = o;
+    pl->o_rlist = take(BR * 4);
+    pl->o_rglist = take(BG * 4);
+    pl->o_hs = take(BR * sizeof(HeadState));
+    pl->o_tie_cnt = take(BR * pl->ntiles_cap * 4);
     pl->o_bitmap = take(BR * pl->words_cap * 4);
     pl->o_blist = take(BG * pl->nblk_cap * 4);
     pl->o_bcount = take(BG * 4);
-    // B*n_lg*local_items <= total/local_kb + B*n_lg <= 2*NSM_PLAN + B*n_lg for any window and sink
-    pl->o_lpart = take(((size_t)2 * NSM_PLAN + BL) * pl->G * PSTRIDE * 4);
-    pl->o_rpart = take(((size_t)pl->ret_grid + BG) * pl->G * PSTRIDE * 4);
+    // a split partial per (CTA, item) pair: slot = CTA + item index, at most grid + items
+    pl->o_lpart = take(((size_t)MAX_GRID + BL) * pl->G * PSTRIDE * 4);
+    pl->o_rpart = take(((size_t)MAX_GRID + BG) * pl->G * PSTRIDE * 4);
     pl->total = o;
     return RTP_OK;
 }
 
-template <int G>
-static cudaError_t launch_step(const Params& P, const Plan& pl, uint8_t* ws, cudaStream_t s, void* const* ev) {
-    const size_t smem = sizeof(StepSmem<G>);
-    static std::atomic<int> ctas_per_sm{0};
-    static std::atomic<int> num_sms{0};
-    if (!ctas_per_sm.load()) {
-        cudaError_t e = cudaFuncSetAttribute(step_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        int n = 0, dev = 0, sms = 0;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, step_kernel<G>, STEP_THREADS, smem);
-        if (e != cudaSuccess) return e;
-        if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-        if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-        num_sms.store(sms);
-        ctas_per_sm.store(std::max(1, n));
+// cuTensorMapEncodeTiled from the driver, looked up once.
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+static EncodeTiledFn encode_fn() {
+    static std::atomic<EncodeTiledFn> fn{nullptr};
+    EncodeTiledFn f = fn.load();
+    if (!f) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || !p)
+            return nullptr;
+        f = reinterpret_cast<EncodeTiledFn>(p);
+        fn.store(f);
     }
-    // under stream capture the records must become event nodes of the graph
-    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
-    if (ev) cudaStreamIsCapturing(s, &cap);
-    const unsigned ev_flags = (cap == cudaStreamCaptureStatusActive) ? cudaEventRecordExternal : cudaEventRecordDefault;
-    StepParams SP;
-    SP.P = P;
-    SP.sync = reinterpret_cast<Sync*>(ws + pl.o_sync);
-    SP.rlist = reinterpret_cast<uint32_t*>(ws + pl.o_rlist);
-    SP.rglist = reinterpret_cast<uint32_t*>(ws + pl.o_rglist);
-    SP.n_score_items = pl.B * pl.n_rg * pl.nschunks;
-    SP.n_local_items = pl.B * pl.n_lg * pl.local_items;
-    const int grid = std::min(MAX_GRID, ctas_per_sm.load() * num_sms.load());
-    if (ev) cudaEventRecordWithFlags((cudaEvent_t)ev[0], s, ev_flags);
-    step_kernel<G><<<grid, STEP_THREADS, smem, s>>>(SP);
+    return f;
+}
+
+// A [rows, 128] bf16 cache as 64 x 64 boxes with the 128-byte swizzle.
+static bool encode_cache_map(CUtensorMap* map, const void* base, long long rows) {
+    EncodeTiledFn f = encode_fn();
+    if (!f) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+    const cuuint32_t box[2] = {64, 64};
+    const cuuint32_t estr[2] = {1, 1};
+    return f(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Resident CTAs per SM of a kernel at a dynamic shared-memory size (cached).
+struct OccCache {
+    std::mutex mu;
+    const void* fn[16];
+    size_t smem[16];
+    int occ[16];
+    int n = 0;
+};
+static int occupancy(const void* fn, size_t smem) {
+    static OccCache c;
+    std::lock_guard<std::mutex> lock(c.mu);
+    for (int i = 0; i < c.n; ++i)
+        if (c.fn[i] == fn && c.smem[i] == smem) return c.occ[i];
+    // the limit is raised to the largest block allocation once (lowering it
+    // again for a smaller call would break a later larger one)
+    int dev = 0, maxs = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (cudaDeviceGetAttribute(&maxs, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) return 0;
+    if ((size_t)maxs < smem) return 0;
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, maxs) != cudaSuccess) return 0;
+    cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, THREADS, smem) != cudaSuccess) return 0;
+    const int slot = c.n < 16 ? c.n++ : 15;
+    c.fn[slot] = fn;
+    c.smem[slot] = smem;
+    c.occ[slot] = n;
+    return n;
+}
+
+// RTP_VERBOSE=1 in the environment: CUDA failures behind RTP_ERR_CUDA are
+// reported on stderr (what failed and the CUDA error string).
+static cudaError_t report(cudaError_t e, const char* what) {
+    static const bool verbose = getenv("RTP_VERBOSE") != nullptr;
+    if (e != cudaSuccess && verbose) fprintf(stderr, "rtp: %s: %s\n", what, cudaGetErrorString(e));
+    return e;
+}
+
+static int num_sms() {
+    static std::atomic<int> n{0};
+    int v = n.load();
+    if (!v) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+        n.store(v);
+    }
+    return v;
+}
+
+template <int G>
+static cudaError_t launch(const KParams& K, const Plan& pl, cudaStream_t s, void* const* ev, unsigned ev_flags) {
+    const int sms = num_sms();
+    if (!sms) return report(cudaErrorUnknown, "SM count");
+    // streaming kernel: as many resident CTAs as the tiles can use
+    {
+        const size_t smem = asmem_bytes<G>(pl.B);
+        const int occ = occupancy((const void*)stream_kernel<G>, smem);
+        if (occ < 1) return report(cudaErrorInvalidConfiguration, "stream kernel occupancy");
+        const long long grid = std::max(1ll, std::min<long long>(std::min(MAX_GRID, occ * sms), pl.tiles_cap));
+        stream_kernel<G><<<(unsigned)grid, THREADS, smem, s>>>(K);
+        cudaError_t e = report(cudaGetLastError(), "stream kernel launch");
+        if (e != cudaSuccess) return e;
+    }
     if (ev) cudaEventRecordWithFlags((cudaEvent_t)ev[1], s, ev_flags);
-    return cudaGetLastError();
+    if (pl.n_rg == 0) return cudaSuccess;
+    // retrieval kernel: one resident wave (its CTAs meet at grid barriers),
+    // launched as a programmatic dependent of the streaming kernel so that
+    // its launch overlaps that kernel's tail
+    {
+        const size_t smem = bsmem_bytes<G>(pl.B * pl.n_rg);
+        const int occ = occupancy((const void*)retrieve_kernel<G>, smem);
+        if (occ < 1) return report(cudaErrorInvalidConfiguration, "retrieval kernel occupancy");
+        const int grid = std::min(MAX_GRID, occ * sms);
+        cudaLaunchConfig_t cfg;
+        memset(&cfg, 0, sizeof(cfg));
+        cfg.gridDim = dim3((unsigned)grid);
+        cfg.blockDim = dim3(THREADS);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = s;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = ev ? 0 : 1;   // an event recorded in between orders the kernels anyway
+        cudaError_t e = report(cudaLaunchKernelEx(&cfg, retrieve_kernel<G>, K), "retrieval kernel launch");
+        if (e != cudaSuccess) return e;
+    }
+    return report(cudaGetLastError(), "retrieval kernel launch");
 }
 
 }  // namespace rtp
@@ -175,6 +265,8 @@ extern "C" size_t rtp_workspace_size(const rtp_dims* dims, const uint8_t* head_k
     return pl.total;
 }
 
+static bool aligned16(const void* p) { return ((uintptr_t)p & 15) == 0; }
+
 extern "C" rtp_status rtp_decode_step(const rtp_dims* dims, const uint16_t* q_pre, const uint16_t* q_rope,
                                       const uint16_t* k_idx, const uint16_t* k_cache, const uint16_t* v_cache,
                                       const uint16_t* Wq_idx, const int32_t* seq_lens, const uint8_t* head_kind,
@@ -183,14 +275,24 @@ extern "C" rtp_status rtp_decode_step(const rtp_dims* dims, const uint16_t* q_pr
         !out)
         return RTP_ERR_NULL;
     if (window < 0 || sink < 0 || (int64_t)window + sink < 1) return RTP_ERR_SHAPE;
+    if (!aligned16(q_pre) || !aligned16(q_rope) || !aligned16(k_idx) || !aligned16(k_cache) || !aligned16(v_cache) ||
+        !aligned16(Wq_idx) || !aligned16(out))
+        return RTP_ERR_UNSUPPORTED;
     Plan pl;
     rtp_status st = make_plan(dims, head_kind, window, sink, &pl);
     if (st != RTP_OK) return st;
     if (!dims->workspace || dims->workspace_bytes < pl.total || ((uintptr_t)dims->workspace & 255))
         return RTP_ERR_WORKSPACE;
 
-    Params P;
-    memset(&P, 0, sizeof(P));
+    KParams K;
+    memset(&K, 0, sizeof(K));
+    const long long rows =
+        dims->block_table ? (long long)dims->num_pages * pl.Hkv * BLK : (long long)pl.B * pl.Hkv * pl.Ncap;
+    if (!encode_cache_map(&K.tmk, k_cache, rows) || !encode_cache_map(&K.tmv, v_cache, rows)) {
+        report(cudaErrorInvalidValue, "K/V tensor map");
+        return RTP_ERR_CUDA;
+    }
+    Params& P = K.P;
     P.B = pl.B;
     P.Hq = pl.Hq;
     P.Hkv = pl.Hkv;
@@ -198,6 +300,7 @@ extern "C" rtp_status rtp_decode_step(const rtp_dims* dims, const uint16_t* q_pr
     P.Ncap = pl.Ncap;
     P.nblk_cap = pl.nblk_cap;
     P.words_cap = pl.words_cap;
+    P.ntiles_cap = pl.ntiles_cap;
     P.mbps = dims->max_blocks_per_seq;
     P.num_pages = dims->num_pages;
     P.window = window;
@@ -205,16 +308,9 @@ extern "C" rtp_status rtp_decode_step(const rtp_dims* dims, const uint16_t* q_pr
     P.n_ret = pl.n_ret;
     P.n_rg = pl.n_rg;
     P.n_lg = pl.n_lg;
-    P.nchunks = pl.nchunks;
-    P.nschunks = pl.nschunks;
-    P.local_kb = pl.local_kb;
-    P.local_items = pl.local_items;
-    P.ret_grid = pl.ret_grid;
     P.q_pre = q_pre;
     P.q_rope = q_rope;
     P.k_idx = k_idx;
-    P.k_cache = k_cache;
-    P.v_cache = v_cache;
     P.Wq = Wq_idx;
     P.seq_lens = seq_lens;
     P.block_table = dims->block_table;
@@ -230,17 +326,17 @@ extern "C" rtp_status rtp_decode_step(const rtp_dims* dims, const uint16_t* q_pr
     memcpy(P.slot_rg, pl.slot_rg, sizeof(P.slot_rg));
     uint8_t* ws = (uint8_t*)dims->workspace;
     P.status = (uint32_t*)(ws + pl.o_status);
+    P.sync = (Sync*)(ws + pl.o_sync);
+    P.rlist = (uint32_t*)(ws + pl.o_rlist);
+    P.rglist = (uint32_t*)(ws + pl.o_rglist);
     P.tick_score = (uint32_t*)(ws + pl.o_tick_score);
-    P.tick_radix = (uint32_t*)(ws + pl.o_tick_radix);
     P.tick_local = (uint32_t*)(ws + pl.o_tick_local);
     P.tick_ret = (uint32_t*)(ws + pl.o_tick_ret);
-    P.keys = (uint32_t*)(ws + pl.o_keys);
     P.agg = (HeadAgg*)(ws + pl.o_agg);
     P.hs = (HeadState*)(ws + pl.o_hs);
     P.hist_cnt = (uint32_t*)(ws + pl.o_hist_cnt);
     P.hist_mass = (unsigned long long*)(ws + pl.o_hist_mass);
-    P.chunk_cnt = (uint32_t*)(ws + pl.o_chunk_cnt);
-    P.tie_off = (uint32_t*)(ws + pl.o_tie_off);
+    P.tie_cnt = (uint32_t*)(ws + pl.o_tie_cnt);
     P.bitmap = (uint32_t*)(ws + pl.o_bitmap);
     P.blist = (uint32_t*)(ws + pl.o_blist);
     P.bcount = (uint32_t*)(ws + pl.o_bcount);
@@ -257,13 +353,19 @@ extern "C" rtp_status rtp_decode_step(const rtp_dims* dims, const uint16_t* q_pr
     }
     cudaStream_t s = (cudaStream_t)stream;
     void* const* ev = (dims->timing_events && dims->n_timing_events >= RTP_TIMING_EVENTS) ? dims->timing_events : nullptr;
+    // under stream capture the records must become event nodes of the graph
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (ev) cudaStreamIsCapturing(s, &cap);
+    const unsigned ev_flags = (cap == cudaStreamCaptureStatusActive) ? cudaEventRecordExternal : cudaEventRecordDefault;
+    if (ev) cudaEventRecordWithFlags((cudaEvent_t)ev[0], s, ev_flags);
     cudaError_t e;
     switch (pl.G) {
-        case 1: e = launch_step<1>(P, pl, ws, s, ev); break;
-        case 2: e = launch_step<2>(P, pl, ws, s, ev); break;
-        case 4: e = launch_step<4>(P, pl, ws, s, ev); break;
-        default: e = launch_step<8>(P, pl, ws, s, ev); break;
+        case 1: e = launch<1>(K, pl, s, ev, ev_flags); break;
+        case 2: e = launch<2>(K, pl, s, ev, ev_flags); break;
+        case 4: e = launch<4>(K, pl, s, ev, ev_flags); break;
+        default: e = launch<8>(K, pl, s, ev, ev_flags); break;
     }
+    if (ev) cudaEventRecordWithFlags((cudaEvent_t)ev[2], s, ev_flags);
     return e == cudaSuccess ? RTP_OK : RTP_ERR_CUDA;
 }
 
@@ -336,12 +438,11 @@ extern "C" rtp_status rtp_decode_step_noalloc(const rtp_dims* dims, const uint16
     if (noalloc_scratch_ptr(&ws) != cudaSuccess) return RTP_ERR_CUDA;
     cudaStream_t s = (cudaStream_t)stream;
     // The array keeps the previous call's contents, possibly laid out for
-    // other sizes.  The kernel expects zero in the status word, the
-    // cross-CTA counters and ticket words ([0, o_keys)) and in the per-head
-    // bucket aggregates and radix histograms ([o_agg, o_chunk_cnt)); every
+    // other sizes.  The kernels expect zero in the status word, the
+    // coordination and ticket words, the per-head bucket aggregates and the
+    // radix histograms, which the layout puts first ([0, zero_end)); every
     // other region is written before it is read.
-    if (cudaMemsetAsync(ws, 0, pl.o_keys, s) != cudaSuccess) return RTP_ERR_CUDA;
-    if (cudaMemsetAsync(ws + pl.o_agg, 0, pl.o_chunk_cnt - pl.o_agg, s) != cudaSuccess) return RTP_ERR_CUDA;
+    if (cudaMemsetAsync(ws, 0, pl.zero_end, s) != cudaSuccess) return RTP_ERR_CUDA;
     rtp_dims d = *dims;
     d.workspace = ws;
     d.workspace_bytes = RTP_NOALLOC_SCRATCH_BYTES;

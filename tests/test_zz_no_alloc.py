@@ -24,15 +24,15 @@ from tests.parity import ATOL, RTOL
 
 def test_oversize_and_null_rejected_on_host():
     """Refused before any CUDA call, so this runs without a GPU too."""
-    HK = [1] * 32
+    HK = [1] * 128
     fake = 4096                        # never dereferenced: the call returns first
     args = [fake] * 7 + [rtp._head_kind_buf(HK), fake, 64, 4, fake, None, None]
-    big = rtp.make_dims(1, 32, 8, 1 << 20)           # 32 retrieval heads x 1M tokens of score keys
+    big = rtp.make_dims(256, 128, 16, 8192)          # 256 x 128 retrieval heads of selection state
     assert rtp.workspace_size(big, HK) > rtp.NOALLOC_SCRATCH_BYTES
     rc = rtp.lib.rtp_decode_step_noalloc(ctypes.byref(big), *args)
     assert rc == 8, rtp.status_string(rc)             # RTP_ERR_SCRATCH_LIMIT
     assert "static array" in rtp.status_string(8)
-    small = rtp.make_dims(1, 32, 8, 4096)
+    small = rtp.make_dims(1, 128, 16, 4096)
     assert 0 < rtp.workspace_size(small, HK) <= rtp.NOALLOC_SCRATCH_BYTES
     bad = list(args)
     bad[0] = None                                     # q_pre

@@ -213,11 +213,16 @@ __device__ __forceinline__ void split_emit(const AttnScratch<G>& X, uint32_t hea
 }
 
 // Combine `nparts` split partials (stride G * PSTRIDE floats) of the heads in
-// `heads` into the bf16 outputs out0[h * D] (round to nearest even).
+// `heads` into the bf16 outputs out0[h * D] (round to nearest even).  The
+// split weights 2^(m_i - M) go to shared memory first (X.red, free once the
+// splits are emitted) so that each thread's loop over the splits issues
+// independent loads only.
 template <int G>
 __device__ __noinline__ void combine_splits(AttnScratch<G>& X, const float* parts, int nparts, uint32_t heads,
-                                               uint16_t* out0, int tid) {
+                                            uint16_t* out0, int tid) {
     const int warp = tid >> 5, lane = tid & 31;
+    float* wts = &X.red[0][0][0];   // [G][nparts]
+    const bool in_smem = nparts <= 4 * D;
     for (int h = warp; h < G; h += CONSUMERS / 32) {
         float M = -INFINITY;
         for (int i = lane; i < nparts; i += 32) {
@@ -227,12 +232,13 @@ __device__ __noinline__ void combine_splits(AttnScratch<G>& X, const float* part
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
         float den = 0.f;
-        if (M != -INFINITY)
-            for (int i = lane; i < nparts; i += 32) {
-                const float* pp = parts + ((int64_t)i * G + h) * PSTRIDE;
-                const float li = __ldcg(pp + 1);
-                if (li > 0.f) den = fmaf(li, ex2_approx(__ldcg(pp) - M), den);
-            }
+        for (int i = lane; i < nparts; i += 32) {
+            const float* pp = parts + ((int64_t)i * G + h) * PSTRIDE;
+            const float li = __ldcg(pp + 1);
+            const float w = (M != -INFINITY && li > 0.f) ? ex2_approx(__ldcg(pp) - M) : 0.f;
+            den = fmaf(li > 0.f ? li : 0.f, w, den);
+            if (in_smem) wts[h * nparts + i] = w;
+        }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
         if (lane == 0) {
@@ -246,20 +252,23 @@ __device__ __noinline__ void combine_splits(AttnScratch<G>& X, const float* part
         if (!((heads >> h) & 1u)) continue;
         const float den = X.cden[h], M = X.cm[h];
         if (!(den > 0.f)) continue;
-        float a0 = 0.f, a1 = 0.f;
+        float a[4] = {0.f, 0.f, 0.f, 0.f};
         int i = 0;
-        for (; i + 1 < nparts; i += 2) {
-            const float* p0 = parts + ((int64_t)i * G + h) * PSTRIDE;
-            const float* p1 = p0 + (int64_t)G * PSTRIDE;
-            const float l0 = __ldcg(p0 + 1), l1 = __ldcg(p1 + 1);
-            if (l0 > 0.f) a0 = fmaf(ex2_approx(__ldcg(p0) - M), __ldcg(p0 + 4 + tid), a0);
-            if (l1 > 0.f) a1 = fmaf(ex2_approx(__ldcg(p1) - M), __ldcg(p1 + 4 + tid), a1);
+        if (in_smem) {
+            for (; i + 4 <= nparts; i += 4) {
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    a[u] = fmaf(wts[h * nparts + i + u], __ldcg(parts + ((int64_t)(i + u) * G + h) * PSTRIDE + 4 + tid), a[u]);
+            }
+            for (; i < nparts; ++i)
+                a[0] = fmaf(wts[h * nparts + i], __ldcg(parts + ((int64_t)i * G + h) * PSTRIDE + 4 + tid), a[0]);
+        } else {
+            for (; i < nparts; ++i) {
+                const float* p0 = parts + ((int64_t)i * G + h) * PSTRIDE;
+                if (__ldcg(p0 + 1) > 0.f) a[0] = fmaf(ex2_approx(__ldcg(p0) - M), __ldcg(p0 + 4 + tid), a[0]);
+            }
         }
-        if (i < nparts) {
-            const float* p0 = parts + ((int64_t)i * G + h) * PSTRIDE;
-            if (__ldcg(p0 + 1) > 0.f) a0 = fmaf(ex2_approx(__ldcg(p0) - M), __ldcg(p0 + 4 + tid), a0);
-        }
-        out0[h * D + tid] = __bfloat16_as_ushort(__float2bfloat16_rn((a0 + a1) / den));
+        out0[h * D + tid] = __bfloat16_as_ushort(__float2bfloat16_rn(((a[0] + a[1]) + (a[2] + a[3])) / den));
     }
     consumer_sync();
 }

@@ -44,6 +44,8 @@ struct HeadState {
     unsigned long long target, mass_above;  // fixed-point masses (units of 2^-40)
     uint32_t prefix, count_above, n_eq, n_tie, all_ties, kstar, tau_key;
     uint32_t tie_idx;                       // largest index among the threshold ties kept
+    float dr, inv_w;                        // first select pass: bins of width dr/255 over smax - s in [0, dr)
+    uint32_t bstar, pad1;                   // the bin that holds the threshold
 };
 
 // Coordination words of one call (workspace; zero between calls).
@@ -54,13 +56,16 @@ struct Sync {
     uint32_t barrier;          // grid barrier arrivals of the retrieval kernel
     uint32_t exit_count;
     uint32_t groups_decided;   // (b, retrieval group) pairs whose selection mode is known
-    uint32_t pad[26];
+    uint32_t pass_done[8];     // radix heads whose step after select pass i is done
+    uint32_t groups_ready;     // radix groups whose block list is built
+    uint32_t pad[17];
 };
 
 struct Params {
     int B, Hq, Hkv, G, Ncap, nblk_cap, words_cap, ntiles_cap, mbps, num_pages, window, sink;
     int n_ret, n_rg, n_lg;
     const uint16_t *q_pre, *q_rope, *k_idx, *Wq;
+    const uint16_t *k_cache_ptr, *v_cache_ptr;   // the caches as plain pointers (the kernels read them through TMA maps)
     const int32_t *seq_lens, *block_table;
     const float* p;
     uint16_t* out;
@@ -73,12 +78,13 @@ struct Params {
     uint32_t* status;
     Sync* sync;
     uint32_t *rlist, *rglist;
-    uint32_t *tick_score, *tick_local, *tick_ret;
+    uint32_t *tick_score, *tick_local, *tick_ret, *tick_sel, *tick_grp;
     HeadAgg* agg;
     HeadState* hs;
     uint32_t* hist_cnt;
     unsigned long long* hist_mass;
     uint32_t* tie_cnt;
+    float* scores;   // [B * n_ret, Ncap] fp32 index scores, written by the streaming kernel, read by the select
     uint32_t* bitmap;
     uint32_t* blist;
     uint32_t* bcount;
@@ -119,6 +125,15 @@ __device__ __forceinline__ uint32_t f2key(float f) {
 __device__ __forceinline__ float key2f(uint32_t k) {
     uint32_t u = (k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k;
     return __uint_as_float(u);
+}
+
+// e^x for |x| <= 700 as an fp64 value: 2^(x log2 e) split into an integer
+// power (exact, ldexp) and a fractional one (fp32 special-function unit,
+// about 2 ulp of fp32).  Used where only a ~1e-6 relative accuracy matters.
+__device__ __forceinline__ double exp_wide(double x) {
+    const double y = x * 1.4426950408889634;
+    const double yi = floor(y);
+    return ldexp((double)exp2f((float)(y - yi)), (int)yi);
 }
 
 // softmax(s/4) weight of a score relative to the maximum score, in 2^-40 units

@@ -40,11 +40,13 @@ struct BSmem {
     AttnScratch<G> X;
     alignas(16) float qi[MAX_G][R];
     uint32_t hcnt[G][256];
-    uint32_t hm[G][3][256];   // 17-bit slices of the per-bin fixed-point mass
+    unsigned long long hmass[G][256];   // per-bin count and 2^-40 fixed-point mass
     unsigned long long dmass[256];
     uint32_t dcnt[256];
     uint32_t tmask[MAX_G];
     uint32_t tcnt[MAX_G];
+    uint8_t rlist_h[MAX_G];
+    uint32_t nrad_h;
     uint8_t tflag[SROWS];
     RDesc desc[NST];
     alignas(8) uint64_t full[NST], empty[NST];
@@ -117,206 +119,200 @@ struct RWalk {
     }
 };
 
-// The copy warp's part of a pass over the radix groups' index tiles.
-template <int G>
-__device__ __noinline__ void r_produce_index(const Params& P, BSmem<G>& S, RWalk wk, const int* pre, uint32_t& k,
-                                               int lane) {
-    constexpr int NST = BSmem<G>::NST;
-    RSeg sg;
-    while (wk.next(P, pre, sg)) {
-        const int g = P.rg_group[sg.rg];
-        for (int i = 0; i < sg.ntiles; ++i, ++k) {
-            const int st = (int)(k % NST);
-            const uint32_t round = k / NST;
-            bool ok = true;
-            if (lane == 0 && round > 0 && !mbar_wait_bounded(&S.empty[st], (round - 1) & 1u)) {
-                set_status(P, ST_TIMEOUT);
-                ok = false;
-            }
-            if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) {
-                S.abort = 1;
-                return;
-            }
-            uint8_t* dst = &S.stage[st][0];
-            const int n0 = (sg.first + i) * SROWS, nvalid = min(SROWS, sg.L - n0);
-            if (P.block_table == nullptr) {
-                if (lane == 0) {
-                    mbar_expect_tx(&S.full[st], (uint32_t)nvalid * R * 2);
-                    bulk_g2s(dst, P.k_idx + (((int64_t)sg.b * P.Hkv + g) * P.Ncap + n0) * R, (uint32_t)nvalid * R * 2,
-                             &S.full[st]);
-                }
-            } else {
-                const int np = (nvalid + BLK - 1) / BLK;
-                if (lane == 0) mbar_expect_tx(&S.full[st], (uint32_t)np * BLK * R * 2);
-                __syncwarp();
-                for (int q = lane; q < np; q += 32)
-                    bulk_g2s(dst + q * BLK * R * 2, P.k_idx + block_row(P, sg.b, g, n0 / BLK + q) * R, BLK * R * 2,
-                             &S.full[st]);
-            }
-            __syncwarp();
-        }
-    }
-}
-
-// Per-lane view of the radix state of the two heads (2t, 2t+1) a lane owns.
-struct RHeads {
-    bool on[2];
-    uint32_t prefix[2], tau[2], tie_idx[2];
-    float smax[2];
+// Per-thread view of the select state of one head.
+struct RHead {
+    uint32_t prefix, tau, tie_idx, bstar;
+    float smax, dr, inv_w;
 };
 
-__device__ __forceinline__ RHeads load_rheads(const Params& P, int b, int rg, int lane) {
-    const int nh = P.rg_nh[rg], slot0 = P.rg_slot0[rg], t = lane & 3;
-    RHeads r;
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-        const int hh = 2 * t + j;
-        r.on[j] = false;
-        r.prefix[j] = r.tau[j] = 0u;
-        r.tie_idx[j] = 0xFFFFFFFFu;
-        r.smax[j] = 0.f;
-        if (hh < nh) {
-            const HeadState* h = P.hs + (int64_t)b * P.n_ret + slot0 + hh;
-            r.on[j] = __ldcg(&h->mode) == MODE_RADIX;
-            r.prefix[j] = __ldcg(&h->prefix);
-            r.tau[j] = __ldcg(&h->tau_key);
-            r.tie_idx[j] = __ldcg(&h->tie_idx);
-            r.smax[j] = __ldcg(&h->smax);
-        }
-    }
+__device__ __forceinline__ RHead load_rhead(const HeadState* h) {
+    RHead r;
+    r.prefix = __ldcg(&h->prefix);
+    r.tau = __ldcg(&h->tau_key);
+    r.tie_idx = __ldcg(&h->tie_idx);
+    r.bstar = __ldcg(&h->bstar);
+    r.smax = __ldcg(&h->smax);
+    r.dr = __ldcg(&h->dr);
+    r.inv_w = __ldcg(&h->inv_w);
     return r;
 }
 
-// What a compute pass does with every (row, owned head) score of a tile.
-enum RPass : int { RP_HIST0 = 0, RP_HIST1, RP_HIST2, RP_HIST3, RP_TIES, RP_MARK };
+// First-pass bin of a score: 255 bins of width dr/255 over d = smax - s in
+// [0, dr) (d >= 0: smax is the maximum of the same fp32 scores), bin 255 for
+// d >= dr.  Every pass computes it with the same fp32 operations.
+__device__ __forceinline__ uint32_t score_bin(float s, float smax, float dr, float inv_w) {
+    const float d = smax - s;
+    return d < dr ? (uint32_t)min((int)(d * inv_w), 254) : 255u;
+}
 
-// The compute warps' part of a pass over the radix groups' index tiles.
+// What a pass does with every stored score of a radix head:
+// RP_BINS histograms the first-pass bins; RP_REF0..3 histogram the next 8
+// key bits of the scores in the threshold bin that match the key prefix
+// found so far; RP_TIES counts threshold ties per tile; RP_MARK marks blocks.
+enum RPass : int { RP_BINS = 0, RP_REF0, RP_REF1, RP_REF2, RP_REF3, RP_TIES, RP_MARK };
+
 template <int G>
-__device__ __noinline__ void r_consume_index(const Params& P, BSmem<G>& S, RWalk wk, const int* pre, uint32_t& k,
-                                               int pass, int tid) {
-    constexpr int NST = BSmem<G>::NST;
-    const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
+__device__ __noinline__ void r_digit(const Params& P, BSmem<G>& S, int b, int slot, int pass, int tid);
+template <int G>
+__device__ __noinline__ void r_tie_locate(const Params& P, BSmem<G>& S, int b, int slot, int tid);
+template <int G>
+__device__ __noinline__ void r_blist(const Params& P, BSmem<G>& S, int b, int rg, int tid);
+
+// One pass over the stored scores of this CTA's share of the radix groups'
+// 1024-token tiles (consumer threads; thread tid takes tokens n0 + tid + 128 u
+// of every radix head of the group at once).  At the end of each run of a
+// group's tiles the CTA folds its histograms into the heads' global ones;
+// per-head tickets elect the CTA that takes the head's next step (its digit,
+// its tie position, or, for the marks, the group's block list).
+template <int G>
+__device__ __noinline__ void r_pass(const Params& P, BSmem<G>& S, RWalk wk, const int* pre, int pass, int tid) {
+    constexpr int U = SROWS / CONSUMERS;
+    const int lane = tid & 31;
     RSeg sg;
     Acct ac;
     ac.init(P, tid == 0);
+    const int rp = pass - RP_REF0;
     while (wk.next(P, pre, sg)) {
         const int nh = P.rg_nh[sg.rg], slot0 = P.rg_slot0[sg.rg];
-        compute_qidx(P, S.qi, sg.b, sg.rg, tid);
+        const int64_t bs0 = (int64_t)sg.b * P.n_ret + slot0;
         for (int x = tid; x < G * 256; x += CONSUMERS) {
             (&S.hcnt[0][0])[x] = 0;
-            (&S.hm[0][0][0])[x] = 0;
-            (&S.hm[0][0][0])[x + G * 256] = 0;
-            (&S.hm[0][0][0])[x + 2 * G * 256] = 0;
+            (&S.hmass[0][0])[x] = 0ull;
         }
         if (tid < MAX_G) {
             S.tmask[tid] = 0;
             S.tcnt[tid] = 0;
         }
+        // the group's radix heads, then a flat loop over (tile, head) items
+        // with the next item's scores loaded while this one is processed
+        if (tid == 0) {
+            uint32_t n = 0;
+            for (int hh = 0; hh < nh; ++hh)
+                if (__ldcg(&P.hs[bs0 + hh].mode) == MODE_RADIX) S.rlist_h[n++] = (uint8_t)hh;
+            S.nrad_h = n;
+        }
         consumer_sync();
-        const QFrag qf = make_qfrag(S.qi, nh, lane);
-        const RHeads rh = load_rheads(P, sg.b, sg.rg, lane);
-        const int shift = pass <= RP_HIST3 ? 24 - 8 * pass : 0;
-        for (int i = 0; i < sg.ntiles; ++i, ++k) {
-            const int st = (int)(k % NST);
-            ac.mark(27);
-            if (!mbar_wait_bounded(&S.full[st], (k / NST) & 1u)) {
-                set_status(P, ST_TIMEOUT);
-                S.abort = 1;
-                return;
-            }
-            ac.mark(26);
-            const int tile = sg.first + i;
+        const int nr = (int)S.nrad_h;
+        const int nitems = sg.ntiles * nr;
+        float vn[U];
+        auto load_item = [&](int it, float* dst) {
+            const int tile = sg.first + it / nr, hh = S.rlist_h[it % nr];
             const int n0 = tile * SROWS, nvalid = min(SROWS, sg.L - n0);
-            const int ng = (nvalid + 15) / 16;
-            const uint32_t base = smem_u32(&S.stage[st][0]);
-            uint32_t bits[2] = {0u, 0u};
-            uint32_t cnt[2] = {0u, 0u};
+            const float* src = P.scores + (bs0 + hh) * P.Ncap + n0;
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int r = tid + u * CONSUMERS;
+                dst[u] = r < nvalid ? __ldcg(src + r) : 0.f;
+            }
+        };
+        if (nitems > 0) load_item(0, vn);
+        uint32_t ovf_n = 0u;
+        unsigned long long ovf_m = 0ull;
+        int cur_h = -1;
+        RHead rh;
 #pragma unroll 1
-            for (int grp = warp; grp < ng; grp += 4) {
-                float c[4];
-                score16(base, grp, lane, qf, c);
+        for (int it = 0; it < nitems; ++it) {
+            float v[U];
 #pragma unroll
-                for (int h = 0; h < 2; ++h)
+            for (int u = 0; u < U; ++u) v[u] = vn[u];
+            if (it + 1 < nitems) load_item(it + 1, vn);
+            const int tile = sg.first + it / nr, hh = S.rlist_h[it % nr];
+            const int n0 = tile * SROWS, nvalid = min(SROWS, sg.L - n0);
+            if (hh != cur_h) {
+                if (pass == RP_BINS && cur_h >= 0) {
+                    // out-of-range sums of the previous head
 #pragma unroll
-                    for (int j = 0; j < 2; ++j) {
-                        const int r = grp * 16 + g + 8 * h;
-                        const bool on = rh.on[j] && r < nvalid;
-                        const uint32_t key = f2key(c[j + 2 * h]);
-                        if (pass <= RP_HIST3) {
-                            const bool valid = on && (pass == 0 || (key >> (32 - 8 * pass)) == rh.prefix[j]);
-                            const uint32_t d = (key >> shift) & 255u;
-                            const uint32_t mv = valid ? ((uint32_t)(2 * t + j) << 8 | d) : 0xFFFFFFFFu;
-                            const uint32_t peers = __match_any_sync(0xffffffffu, mv);
-                            if (valid) {
-                                const unsigned long long ms = fixmass(key, rh.smax[j]);
-                                const uint32_t s0 = __reduce_add_sync(peers, (uint32_t)(ms & 0x1FFFFull));
-                                const uint32_t s1 = __reduce_add_sync(peers, (uint32_t)((ms >> 17) & 0x1FFFFull));
-                                const uint32_t s2 = __reduce_add_sync(peers, (uint32_t)(ms >> 34));
-                                if (lane == __ffs(peers) - 1) {
-                                    const int hh = 2 * t + j;
-                                    atomicAdd(&S.hcnt[hh][d], (uint32_t)__popc(peers));
-                                    atomicAdd(&S.hm[hh][0][d], s0);
-                                    atomicAdd(&S.hm[hh][1][d], s1);
-                                    atomicAdd(&S.hm[hh][2][d], s2);
-                                }
-                            }
-                        } else if (pass == RP_TIES) {
-                            cnt[j] += (on && key == rh.tau[j]) ? 1u : 0u;
+                    for (int o = 16; o > 0; o >>= 1) {
+                        ovf_n += __shfl_xor_sync(0xffffffffu, ovf_n, o);
+                        ovf_m += __shfl_xor_sync(0xffffffffu, ovf_m, o);
+                    }
+                    if (lane == 0 && ovf_n) {
+                        atomicAdd(&S.hcnt[cur_h][255], ovf_n);
+                        atomicAdd(&S.hmass[cur_h][255], ovf_m);
+                    }
+                    ovf_n = 0u;
+                    ovf_m = 0ull;
+                }
+                cur_h = hh;
+                rh = load_rhead(P.hs + bs0 + hh);
+            }
+            uint32_t bits = 0u, cnt = 0u;
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int r = tid + u * CONSUMERS;
+                const bool ok = r < nvalid;
+                const uint32_t key = f2key(v[u]);
+                if (pass == RP_BINS) {
+                    if (ok) {
+                        const uint32_t bn = score_bin(v[u], rh.smax, rh.dr, rh.inv_w);
+                        const unsigned long long ms = fixmass(key, rh.smax);
+                        if (bn < 255u) {
+                            atomicAdd(&S.hcnt[hh][bn], 1u);
+                            atomicAdd(&S.hmass[hh][bn], ms);
                         } else {
-                            const bool keep = on && (key > rh.tau[j] ||
-                                                     (key == rh.tau[j] && (uint32_t)(n0 + r) <= rh.tie_idx[j]));
-                            if (keep) bits[j] |= 1u << (grp >> 2);
+                            ovf_n += 1u;
+                            ovf_m += ms;
                         }
                     }
+                } else if (pass <= RP_REF3) {
+                    if (ok && score_bin(v[u], rh.smax, rh.dr, rh.inv_w) == rh.bstar &&
+                        (rp == 0 || (key >> (32 - 8 * rp)) == rh.prefix)) {
+                        const uint32_t d = (key >> (24 - 8 * rp)) & 255u;
+                        atomicAdd(&S.hcnt[hh][d], 1u);
+                        atomicAdd(&S.hmass[hh][d], fixmass(key, rh.smax));
+                    }
+                } else if (pass == RP_TIES) {
+                    cnt += (ok && key == rh.tau) ? 1u : 0u;
+                } else {
+                    const bool keep = ok && (key > rh.tau || (key == rh.tau && (uint32_t)(n0 + r) <= rh.tie_idx));
+                    // a warp's 32 tokens lie in one 64-token block: one vote per warp
+                    if (__any_sync(0xffffffffu, keep) && lane == 0) bits |= 1u << ((r / BLK) & 15);
+                }
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&S.empty[st]);
-            ac.mark(24);
-            ac.count(25);
             if (pass == RP_TIES || pass == RP_MARK) {
 #pragma unroll
-                for (int j = 0; j < 2; ++j) {
-#pragma unroll
-                    for (int o = 4; o < 32; o <<= 1) {
-                        bits[j] |= __shfl_xor_sync(0xffffffffu, bits[j], o);
-                        cnt[j] += __shfl_xor_sync(0xffffffffu, cnt[j], o);
-                    }
-                    if (g == 0 && 2 * t + j < nh) {
-                        if (bits[j]) atomicOr(&S.tmask[2 * t + j], bits[j]);
-                        if (cnt[j]) atomicAdd(&S.tcnt[2 * t + j], cnt[j]);
-                    }
+                for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+                if (lane == 0) {
+                    if (cnt) atomicAdd(&S.tcnt[hh], cnt);
+                    if (bits) atomicOr(&S.tmask[hh], bits);
                 }
                 consumer_sync();
-                if (tid < nh) {
-                    const int64_t bs = (int64_t)sg.b * P.n_ret + slot0 + tid;
-                    if (pass == RP_TIES) {
-                        P.tie_cnt[bs * P.ntiles_cap + tile] = S.tcnt[tid];
-                    } else if (S.tmask[tid]) {
-                        atomicOr(P.bitmap + bs * P.words_cap + tile / 2, S.tmask[tid] << ((tile & 1) * 16));
-                    }
-                    S.tmask[tid] = 0;
-                    S.tcnt[tid] = 0;
+                if (tid == 0) {
+                    const int64_t bs = bs0 + hh;
+                    if (pass == RP_TIES) P.tie_cnt[bs * P.ntiles_cap + tile] = S.tcnt[hh];
+                    else if (S.tmask[hh]) atomicOr(P.bitmap + bs * P.words_cap + tile / 2, S.tmask[hh] << ((tile & 1) * 16));
+                    S.tmask[hh] = 0;
+                    S.tcnt[hh] = 0;
                 }
                 consumer_sync();
             }
+            ac.mark(24);
+            ac.count(25);
         }
-        if (pass <= RP_HIST3) {
-            // this split's histograms -> the heads' global histograms
+        if (pass == RP_BINS && cur_h >= 0) {
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                ovf_n += __shfl_xor_sync(0xffffffffu, ovf_n, o);
+                ovf_m += __shfl_xor_sync(0xffffffffu, ovf_m, o);
+            }
+            if (lane == 0 && ovf_n) {
+                atomicAdd(&S.hcnt[cur_h][255], ovf_n);
+                atomicAdd(&S.hmass[cur_h][255], ovf_m);
+            }
+        }
+        if (pass <= RP_REF3) {
+            // this run's histograms -> the heads' global histograms
             consumer_sync();
             for (int x = tid; x < nh * 256; x += CONSUMERS) {
                 const int hh = x >> 8, d = x & 255;
                 const uint32_t c = S.hcnt[hh][d];
                 if (c) {
-                    const int64_t bs = (int64_t)sg.b * P.n_ret + slot0 + hh;
-                    const unsigned long long ms = (unsigned long long)S.hm[hh][0][d] +
-                                                  ((unsigned long long)S.hm[hh][1][d] << 17) +
-                                                  ((unsigned long long)S.hm[hh][2][d] << 34);
-                    atomicAdd(P.hist_cnt + bs * 256 + d, c);
-                    atomicAdd(P.hist_mass + bs * 256 + d, ms);
+                    atomicAdd(P.hist_cnt + (bs0 + hh) * 256 + d, c);
+                    atomicAdd(P.hist_mass + (bs0 + hh) * 256 + d, S.hmass[hh][d]);
                 }
             }
-            consumer_sync();
         }
+        consumer_sync();
     }
 }
 
@@ -326,9 +322,7 @@ __device__ __noinline__ void r_consume_index(const Params& P, BSmem<G>& S, RWalk
 // Pick the digit of pass `pass` for radix head `hx`: the largest digit d whose
 // bins >= d hold at least the target mass (over the tokens above the prefix).
 template <int G>
-__device__ __noinline__ void r_digit(const Params& P, BSmem<G>& S, int hx, int pass, int tid) {
-    const uint32_t e = __ldcg(P.rlist + hx);
-    const int b = (int)(e >> 16), slot = (int)(e & 0xFFFFu);
+__device__ __noinline__ void r_digit(const Params& P, BSmem<G>& S, int b, int slot, int pass, int tid) {
     const int64_t bs = (int64_t)b * P.n_ret + slot;
     uint32_t* gcnt = P.hist_cnt + bs * 256;
     unsigned long long* gmass = P.hist_mass + bs * 256;
@@ -341,7 +335,7 @@ __device__ __noinline__ void r_digit(const Params& P, BSmem<G>& S, int hx, int p
     consumer_sync();
     if (tid == 0) {
         HeadState st = P.hs[bs];
-        if (pass == 0) {
+        if (pass == RP_BINS) {
             unsigned long long z = 0;
             for (int d = 0; d < 256; ++d) z += S.dmass[d];
             const double pb = (double)__ldg(P.p + b);
@@ -349,42 +343,57 @@ __device__ __noinline__ void r_digit(const Params& P, BSmem<G>& S, int hx, int p
             if (tg > z) tg = z;
             if (tg == 0) tg = 1;
             st.target = tg;
-            st.mass_above = 0;
-            st.count_above = 0;
+            // bins ascend in smax - s: the first bin that completes the target
+            unsigned long long cum = 0;
+            uint32_t cabove = 0;
+            uint32_t bstar = 255;
+            for (int d = 0; d < 256; ++d) {
+                if (cum + S.dmass[d] >= tg) {
+                    bstar = (uint32_t)d;
+                    break;
+                }
+                cum += S.dmass[d];
+                cabove += S.dcnt[d];
+            }
+            st.bstar = bstar;
+            st.mass_above = cum;
+            st.count_above = cabove;
             st.prefix = 0;
-        }
-        unsigned long long cum = st.mass_above;
-        uint32_t cabove = st.count_above;
-        int dstar = 0;
-        for (int d = 255; d >= 0; --d) {
-            if (cum + S.dmass[d] >= st.target) {
-                dstar = d;
-                break;
+        } else {
+            const int rp = pass - RP_REF0;
+            unsigned long long cum = st.mass_above;
+            uint32_t cabove = st.count_above;
+            int dstar = 0;
+            for (int d = 255; d >= 0; --d) {
+                if (cum + S.dmass[d] >= st.target) {
+                    dstar = d;
+                    break;
+                }
+                cum += S.dmass[d];
+                cabove += S.dcnt[d];
             }
-            cum += S.dmass[d];
-            cabove += S.dcnt[d];
-        }
-        st.mass_above = cum;
-        st.count_above = cabove;
-        st.prefix = (st.prefix << 8) | (uint32_t)dstar;
-        if (pass == 3) {
-            st.tau_key = st.prefix;
-            st.n_eq = S.dcnt[dstar];
-            const unsigned long long m_tau = st.n_eq ? S.dmass[dstar] / st.n_eq : 0ull;
-            const unsigned long long need = st.target - st.mass_above;
-            uint32_t nt = st.n_eq;
-            if (m_tau > 0) {
-                const unsigned long long q = (need + m_tau - 1) / m_tau;
-                nt = (uint32_t)min((unsigned long long)st.n_eq, max(1ull, q));
+            st.mass_above = cum;
+            st.count_above = cabove;
+            st.prefix = (st.prefix << 8) | (uint32_t)dstar;
+            if (rp == 3) {
+                st.tau_key = st.prefix;
+                st.n_eq = S.dcnt[dstar];
+                const unsigned long long m_tau = st.n_eq ? S.dmass[dstar] / st.n_eq : 0ull;
+                const unsigned long long need = st.target - st.mass_above;
+                uint32_t nt = st.n_eq;
+                if (m_tau > 0) {
+                    const unsigned long long q = (need + m_tau - 1) / m_tau;
+                    nt = (uint32_t)min((unsigned long long)st.n_eq, max(1ull, q));
+                }
+                st.n_tie = nt;
+                st.all_ties = (nt == st.n_eq) ? 1u : 0u;
+                st.tie_idx = 0xFFFFFFFFu;
+                st.kstar = st.count_above + nt;
+                const int bh = b * P.Hq + P.slot_head[slot];
+                if (P.dbg_tau) P.dbg_tau[bh] = key2f(st.tau_key);
+                if (P.dbg_kstar) P.dbg_kstar[bh] = (int32_t)st.kstar;
+                if (!st.all_ties) atomicOr(&P.sync->any_ties, 1u);
             }
-            st.n_tie = nt;
-            st.all_ties = (nt == st.n_eq) ? 1u : 0u;
-            st.tie_idx = 0xFFFFFFFFu;
-            st.kstar = st.count_above + nt;
-            const int bh = b * P.Hq + P.slot_head[slot];
-            if (P.dbg_tau) P.dbg_tau[bh] = key2f(st.tau_key);
-            if (P.dbg_kstar) P.dbg_kstar[bh] = (int32_t)st.kstar;
-            if (!st.all_ties) atomicOr(&P.sync->any_ties, 1u);
         }
         P.hs[bs] = st;
     }
@@ -393,15 +402,11 @@ __device__ __noinline__ void r_digit(const Params& P, BSmem<G>& S, int hx, int p
 
 // For a radix head that keeps only n_tie of its n_eq threshold ties: find the
 // index of the n_tie-th tie in token order (per-tile counts, then a scan of
-// the one tile that holds it, re-scored exactly as in the passes).
+// the stored scores of the one tile that holds it).
 template <int G>
-__device__ __noinline__ void r_tie_locate(const Params& P, BSmem<G>& S, int hx, int tid) {
-    const uint32_t e = __ldcg(P.rlist + hx);
-    const int b = (int)(e >> 16), slot = (int)(e & 0xFFFFu);
+__device__ __noinline__ void r_tie_locate(const Params& P, BSmem<G>& S, int b, int slot, int tid) {
     const int64_t bs = (int64_t)b * P.n_ret + slot;
     if (__ldcg(&P.hs[bs].all_ties)) return;
-    const int rg = P.slot_rg[slot], g = P.rg_group[rg], slot0 = P.rg_slot0[rg], nh = P.rg_nh[rg];
-    const int hh = slot - slot0;
     const int L = __ldg(P.seq_lens + b);
     const int nt = (L + SROWS - 1) / SROWS;
     const uint32_t ntie = __ldcg(&P.hs[bs].n_tie), tau = __ldcg(&P.hs[bs].tau_key);
@@ -423,33 +428,10 @@ __device__ __noinline__ void r_tie_locate(const Params& P, BSmem<G>& S, int hx, 
     const int tile = (int)S.base;
     const uint32_t rank = S.flag;
     const int n0 = tile * SROWS, nvalid = min(SROWS, L - n0);
-    // stage the tile's rows with plain loads (no copy is in flight between passes)
-    uint8_t* rows = &S.stage[0][0];
-    for (int x = tid; x < nvalid * 2; x += CONSUMERS) {
-        const int r = x >> 1, half = x & 1;
-        const int n = n0 + r;
-        const int64_t row = block_row(P, b, g, n / BLK) + (n % BLK);
-        const uint4 v = __ldg(reinterpret_cast<const uint4*>(P.k_idx + row * R) + half);
-        *reinterpret_cast<uint4*>(rows + r * 32 + half * 16) = v;
-    }
-    compute_qidx(P, S.qi, b, rg, tid);
+    const float* sc = P.scores + bs * P.Ncap + n0;
+    for (int r = tid; r < SROWS; r += CONSUMERS) S.tflag[r] = (r < nvalid && f2key(__ldcg(sc + r)) == tau) ? 1 : 0;
     consumer_sync();
-    const int warp = tid >> 5, lane = tid & 31, gl = lane >> 2, t = lane & 3;
-    const QFrag qf = make_qfrag(S.qi, nh, lane);
-    const int ng = (nvalid + 15) / 16;
-    for (int grp = warp; grp < ng; grp += 4) {
-        float c[4];
-        score16(smem_u32(rows), grp, lane, qf, c);
-#pragma unroll
-        for (int h = 0; h < 2; ++h)
-#pragma unroll
-            for (int j = 0; j < 2; ++j)
-                if (2 * t + j == hh) {
-                    const int r = grp * 16 + gl + 8 * h;
-                    S.tflag[r] = (r < nvalid && f2key(c[j + 2 * h]) == tau) ? 1 : 0;
-                }
-    }
-    consumer_sync();
+    const int warp = tid >> 5, lane = tid & 31;
     if (warp == 0) {
         uint32_t cum = 0;
         int found = nvalid - 1;
@@ -458,7 +440,6 @@ __device__ __noinline__ void r_tie_locate(const Params& P, BSmem<G>& S, int hx, 
             const uint32_t bal = __ballot_sync(0xffffffffu, r < nvalid && S.tflag[r]);
             const uint32_t c = __popc(bal);
             if (cum + c >= rank) {
-                // the (rank - cum)-th set bit
                 uint32_t m = bal;
                 for (uint32_t q = 1; q < rank - cum; ++q) m &= m - 1;
                 found = r0 + __ffs(m) - 1;
@@ -474,9 +455,7 @@ __device__ __noinline__ void r_tie_locate(const Params& P, BSmem<G>& S, int hx, 
 // Block list of radix group i: union of its heads' block bitmaps, in
 // ascending block order, with the mask of heads that read each block.
 template <int G>
-__device__ __noinline__ void r_blist(const Params& P, BSmem<G>& S, int i, int tid) {
-    int b, rg;
-    radix_group(P, i, b, rg);
+__device__ __noinline__ void r_blist(const Params& P, BSmem<G>& S, int b, int rg, int tid) {
     const int L = __ldg(P.seq_lens + b);
     const int g = P.rg_group[rg], nh = P.rg_nh[rg], slot0 = P.rg_slot0[rg];
     const int nblk = (L + BLK - 1) / BLK;
@@ -690,7 +669,7 @@ __device__ __forceinline__ void warp_prefix(int* pre, int n, F cnt, int lane) {
 // the kernel
 // ---------------------------------------------------------------------------
 template <int G>
-__global__ void __launch_bounds__(THREADS, 1) retrieve_kernel(const __grid_constant__ KParams K) {
+__global__ void __launch_bounds__(THREADS, 2) retrieve_kernel(const __grid_constant__ KParams K) {
     extern __shared__ uint8_t smem_raw[];
     BSmem<G>& S = *reinterpret_cast<BSmem<G>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     constexpr int NST = BSmem<G>::NST;
@@ -734,37 +713,41 @@ __global__ void __launch_bounds__(THREADS, 1) retrieve_kernel(const __grid_const
         wk.t = (int)((long long)blockIdx.x * T / gridDim.x);
         wk.t1 = (int)((long long)(blockIdx.x + 1) * T / gridDim.x);
         wk.ngr = ngr;
-        for (int pass = 0; pass < 4 && ok; ++pass) {
-            if (copier) {
-                r_produce_index<G>(P, S, wk, pre, k, lane);
-            } else {
-                r_consume_index<G>(P, S, wk, pre, k, pass, tid);
-            }
+        for (int pass = RP_BINS; pass <= RP_REF3 && ok; ++pass) {
+            if (!copier) r_pass<G>(P, S, wk, pre, pass, tid);
             ok = grid_sync(P, S);
             if (!ok) break;
-            if (tid == 0 && pass == 0) trace_max(P, 14);
+            if (tid == 0 && pass == RP_BINS) trace_max(P, 14);
             if (!copier)
-                for (int hx = blockIdx.x; hx < (int)nrad; hx += gridDim.x) r_digit<G>(P, S, hx, pass, tid);
+                for (int hx = blockIdx.x; hx < (int)nrad; hx += gridDim.x) {
+                    const uint32_t e = __ldcg(P.rlist + hx);
+                    r_digit<G>(P, S, (int)(e >> 16), (int)(e & 0xFFFFu), pass, tid);
+                }
             ok = grid_sync(P, S);
-            if (tid == 0) trace_max(P, 8 + pass);
+            if (tid == 0 && pass > RP_BINS) trace_max(P, 8 + pass - RP_REF0);
         }
         if (ok && __ldcg(&P.sync->any_ties)) {
-            if (copier) r_produce_index<G>(P, S, wk, pre, k, lane);
-            else r_consume_index<G>(P, S, wk, pre, k, RP_TIES, tid);
+            if (!copier) r_pass<G>(P, S, wk, pre, RP_TIES, tid);
             ok = grid_sync(P, S);
             if (ok && !copier)
-                for (int hx = blockIdx.x; hx < (int)nrad; hx += gridDim.x) r_tie_locate<G>(P, S, hx, tid);
+                for (int hx = blockIdx.x; hx < (int)nrad; hx += gridDim.x) {
+                    const uint32_t e = __ldcg(P.rlist + hx);
+                    r_tie_locate<G>(P, S, (int)(e >> 16), (int)(e & 0xFFFFu), tid);
+                }
             ok = ok && grid_sync(P, S);
         }
         if (ok) {
-            if (copier) r_produce_index<G>(P, S, wk, pre, k, lane);
-            else r_consume_index<G>(P, S, wk, pre, k, RP_MARK, tid);
+            if (!copier) r_pass<G>(P, S, wk, pre, RP_MARK, tid);
             ok = grid_sync(P, S);
             if (tid == 0) trace_max(P, 12);
         }
         if (ok) {
             if (!copier)
-                for (int i = blockIdx.x; i < ngr; i += gridDim.x) r_blist<G>(P, S, i, tid);
+                for (int i = blockIdx.x; i < ngr; i += gridDim.x) {
+                    int b, rg;
+                    radix_group(P, i, b, rg);
+                    r_blist<G>(P, S, b, rg, tid);
+                }
             ok = grid_sync(P, S);
         }
     }
@@ -785,6 +768,18 @@ __global__ void __launch_bounds__(THREADS, 1) retrieve_kernel(const __grid_const
         else r_consume_attn<G>(K, S, k, tid);
         if (tid == 0) trace_max(P, 4);
     }
+    // the stored scores are dead now: drop their L2 lines without writing
+    // them back (each CTA a slice of every retrieval head's used range)
+    if (ok) {
+        for (int bs = 0; bs < P.B * P.n_ret; ++bs) {
+            const int L = __ldg(P.seq_lens + bs / P.n_ret);
+            if (!seq_ok(P, L)) continue;
+            const char* base = reinterpret_cast<const char*>(P.scores + (int64_t)bs * P.Ncap);
+            const int nlines = (L * 4 + 127) / 128;
+            for (int x = blockIdx.x * THREADS + tid; x < nlines; x += gridDim.x * THREADS)
+                asm volatile("discard.global.L2 [%0], 128;" ::"l"(base + (int64_t)x * 128) : "memory");
+        }
+    }
     // the last CTA out clears the call's coordination words
     __syncthreads();
     if (tid == 0) {
@@ -796,6 +791,8 @@ __global__ void __launch_bounds__(THREADS, 1) retrieve_kernel(const __grid_const
             P.sync->any_ties = 0;
             P.sync->barrier = 0;
             P.sync->groups_decided = 0;
+            for (int i = 0; i < 8; ++i) P.sync->pass_done[i] = 0;
+            P.sync->groups_ready = 0;
             P.sync->exit_count = 0;
             __threadfence();
         }

@@ -33,6 +33,8 @@ struct ASmem {
     uint32_t d_nmin[MAX_G], d_flags[MAX_G], d_arg[MAX_G];
     double d_zabs[MAX_G];
     int d_mode[MAX_G];
+    uint32_t d_list[MAX_G], d_cnt;
+    int pend_b, pend_rg, pend_L;   // best-token blocks this CTA attends after its share (d_list)
     uint32_t flag;
     int tot_s, tot_l, nact;
     int pre[2];   // really [2 * (B + 1)]: tiles before sequence b (score, then local)
@@ -197,7 +199,7 @@ __device__ __noinline__ void decide_group(const Params& P, ASmem<G>& S, int b, i
         const float smax = key2f(k);
         // z = sum over tokens of exp((s - smax)/4); NaN when the fp64 sum was unusable
         const double sm4 = (double)smax * 0.25;
-        const double z = (S.d_flags[hh] || sm4 > 600.0 || sm4 < -600.0) ? NAN : S.d_zabs[hh] * exp(-sm4);
+        const double z = (S.d_flags[hh] || sm4 > 600.0 || sm4 < -600.0) ? NAN : S.d_zabs[hh] * exp_wide(-sm4);
         HeadState h;
         h.smax = smax;
         h.maxkey = k;
@@ -229,6 +231,19 @@ __device__ __noinline__ void decide_group(const Params& P, ASmem<G>& S, int b, i
         } else {
             h.mode = MODE_RADIX;
             h.kstar = 0;
+        }
+        // first select pass: 255 bins over smax - s in [0, dr), dr large
+        // enough that the tokens beyond it cannot hold the last 1 - p of the
+        // mass (otherwise the select continues in the overflow bin)
+        {
+            const float omp = pb < 1.f ? fmaxf(1.f - pb, 1e-6f) : 1e-6f;
+            const float zz = (z == z && z >= 1.0) ? (float)fmin(z, 1e30) : 1.f;
+            float dr = 4.f * (__logf((float)L) - __logf(omp) - __logf(zz)) + 8.f;
+            dr = fminf(fmaxf(dr, 8.f), 400.f);
+            h.dr = dr;
+            h.inv_w = 255.f / dr;
+            h.bstar = 0;
+            h.pad1 = 0;
         }
         P.hs[(int64_t)b * P.n_ret + slot] = h;
         const int bh = b * P.Hq + P.slot_head[slot];
@@ -312,25 +327,41 @@ __device__ __noinline__ void decide_group(const Params& P, ASmem<G>& S, int b, i
             list[j] = ((uint32_t)j << 8) | hm;
         }
         if (tid == 0) P.bcount[bg] = (uint32_t)nblk;
-    } else if (tid == 0) {
-        uint32_t cnt = 0;
-        int last = -1;
-        while (true) {
-            int bj = 0x7FFFFFFF;
-            for (int hh = 0; hh < nh; ++hh)
-                if (S.d_mode[hh] == MODE_TOP1) {
-                    const int j = (int)(S.d_arg[hh] / BLK);
-                    if (j > last && j < bj) bj = j;
-                }
-            if (bj == 0x7FFFFFFF) break;
-            uint32_t hm = 0;
-            for (int hh = 0; hh < nh; ++hh)
-                if (S.d_mode[hh] == MODE_TOP1 && (int)(S.d_arg[hh] / BLK) == bj)
-                    hm |= 1u << (P.slot_head[slot0 + hh] - g * P.G);
-            list[cnt++] = ((uint32_t)bj << 8) | hm;
-            last = bj;
+    } else {
+        // only best-token blocks: the distinct argmax blocks, ascending, are
+        // attended by this CTA after its share (the first such group of the
+        // CTA; a later one goes to the retrieval kernel)
+        if (tid == 0) {
+            uint32_t lst[MAX_G];
+            uint32_t cnt = 0;
+            int last = -1;
+            while (true) {
+                int bj = 0x7FFFFFFF;
+                for (int hh = 0; hh < nh; ++hh)
+                    if (S.d_mode[hh] == MODE_TOP1) {
+                        const int j = (int)(S.d_arg[hh] / BLK);
+                        if (j > last && j < bj) bj = j;
+                    }
+                if (bj == 0x7FFFFFFF) break;
+                uint32_t hm = 0;
+                for (int hh = 0; hh < nh; ++hh)
+                    if (S.d_mode[hh] == MODE_TOP1 && (int)(S.d_arg[hh] / BLK) == bj)
+                        hm |= 1u << (P.slot_head[slot0 + hh] - g * P.G);
+                lst[cnt++] = ((uint32_t)bj << 8) | hm;
+                last = bj;
+            }
+            if (S.d_cnt != 0 || cnt == 0) {
+                for (uint32_t e = 0; e < cnt; ++e) list[e] = lst[e];
+                P.bcount[bg] = cnt;
+            } else {
+                for (uint32_t e = 0; e < cnt; ++e) S.d_list[e] = lst[e];
+                S.d_cnt = cnt;
+                S.pend_b = b;
+                S.pend_rg = rg;
+                S.pend_L = L;
+                P.bcount[bg] = 0;
+            }
         }
-        P.bcount[bg] = cnt;
     }
     consumer_sync();
     if (tid == 0) {
@@ -374,7 +405,7 @@ __device__ __forceinline__ int fold_head(int t, int j) {
 // four at a time (independent MMA chains).
 template <bool NH4, bool FULL>
 __device__ __forceinline__ void score_tile(uint32_t tile, int n0, int nvalid, int nh, bool track_min, const QFrag& q,
-                                           ScoreFold& f, int warp, int lane) {
+                                           ScoreFold& f, float* sbase, int ncap, int warp, int lane) {
     const int g = lane >> 2, t = lane & 3;
     const int ng = FULL ? SROWS / 16 : (nvalid + 15) / 16;
     constexpr float C = 0.25f * 1.4426950408889634f;   // (1/4) log2(e)
@@ -409,6 +440,8 @@ __device__ __forceinline__ void score_tile(uint32_t tile, int n0, int nvalid, in
                     rr[e] = (uint32_t)r;
                     const float x = NH4 ? c[q4][j] : c[q4][j + 2 * h];
                     v[e] = (FULL || r < nvalid) ? x : -INFINITY;
+                    // kept for the exact select (L2-resident until it is read or dropped)
+                    if (FULL || r < nvalid) sbase[(int64_t)fold_head<NH4>(t, j) * ncap + n0 + r] = x;
                 }
             float mb = v[0];
 #pragma unroll
@@ -506,7 +539,7 @@ __device__ __forceinline__ void score_split_end(const Params& P, ASmem<G>& S, co
         if (m != -INFINITY) {
             const double m4 = (double)m * 0.25;
             if (m4 > 600.0 || m4 < -600.0) atomicOr(&ag->flags, 1u);
-            else atomicAdd(&ag->zabs, (double)s * exp(m4));
+            else atomicAdd(&ag->zabs, (double)s * exp_wide(m4));
         }
     }
 }
@@ -564,10 +597,12 @@ __device__ __forceinline__ void a_producer(const KParams& K, ASmem<G>& S, AWalk 
         }
     }
     // never leave the CTA with copies in flight: wait (bounded) for the last
-    // tile issued into each stage to land
+    // tile issued into each stage to land, then tell the compute warps
     if (lane == 0)
         for (uint32_t i = (k > (uint32_t)NST ? k - NST : 0u); i < k; ++i)
             mbar_wait_bounded(&S.full[i % NST], (i / NST) & 1u);
+    __syncwarp();
+    asm volatile("bar.arrive 2, 160;" ::: "memory");
 }
 
 // ---------------------------------------------------------------------------
@@ -616,12 +651,13 @@ __device__ __forceinline__ void a_consumers(const KParams& K, ASmem<G>& S, AWalk
                 first_data = false;
                 const int n0 = (sg.first + i) * SROWS, nvalid = min(SROWS, sg.L - n0);
                 const uint32_t tile = smem_u32(&S.stage[st][0]);
+                float* sbase = P.scores + ((int64_t)sg.b * P.n_ret + P.rg_slot0[sg.grp]) * P.Ncap;
                 if (nvalid == SROWS) {
-                    if (nh4) score_tile<true, true>(tile, n0, nvalid, nh, track_min, qf, f, warp, lane);
-                    else score_tile<false, true>(tile, n0, nvalid, nh, track_min, qf, f, warp, lane);
+                    if (nh4) score_tile<true, true>(tile, n0, nvalid, nh, track_min, qf, f, sbase, P.Ncap, warp, lane);
+                    else score_tile<false, true>(tile, n0, nvalid, nh, track_min, qf, f, sbase, P.Ncap, warp, lane);
                 } else {
-                    if (nh4) score_tile<true, false>(tile, n0, nvalid, nh, track_min, qf, f, warp, lane);
-                    else score_tile<false, false>(tile, n0, nvalid, nh, track_min, qf, f, warp, lane);
+                    if (nh4) score_tile<true, false>(tile, n0, nvalid, nh, track_min, qf, f, sbase, P.Ncap, warp, lane);
+                    else score_tile<false, false>(tile, n0, nvalid, nh, track_min, qf, f, sbase, P.Ncap, warp, lane);
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&S.empty[st]);
@@ -637,14 +673,14 @@ __device__ __forceinline__ void a_consumers(const KParams& K, ASmem<G>& S, AWalk
                 consumer_sync();
                 if (tid == 0) trace_max(P, 1);
             }
-            ac.mark(21);
+            ac.mark(28);
         } else {
             // ---- local heads of (b, local group): sink + window blocks
             const int g = P.lg_group[sg.grp];
             const uint32_t heads = P.lg_mask[sg.grp];
             const LocalGeom lg = local_geom(P, sg.L);
             attn.begin(P, sg.b, g, lane);
-            ac.mark(21);
+            ac.mark(29);
             for (int i = 0; i < sg.ntiles; ++i, ++k) {
                 const int st = (int)(k % NST);
                 if (!mbar_wait_bounded(&S.full[st], (k / NST) & 1u)) {
@@ -686,8 +722,51 @@ __device__ __forceinline__ void a_consumers(const KParams& K, ASmem<G>& S, AWalk
                     if (tid == 0) trace_max(P, 2);
                 }
             }
-            ac.mark(21);
+            ac.mark(30);
         }
+    }
+    // best-token blocks selected by this CTA: attended here, through the same
+    // ring (the copy warp has finished: it signals barrier 2 when done)
+    asm volatile("bar.sync 2, 160;" ::: "memory");
+    if (S.d_cnt > 0) {
+        const int b = S.pend_b, rg = S.pend_rg, L = S.pend_L, g = P.rg_group[rg];
+        const int cnt = (int)S.d_cnt;
+        attn.begin(P, b, g, lane);
+        for (int e0 = 0; e0 < cnt; e0 += NST) {
+            const int ne = min(NST, cnt - e0);
+            if (tid == 0) {
+                for (int e = 0; e < ne; ++e) {
+                    const int st = (int)((k + e) % NST);
+                    const int j = (int)(S.d_list[e0 + e] >> 8);
+                    const int row = (int)block_row(P, b, g, j);
+                    uint8_t* dst = &S.stage[st][0];
+                    mbar_expect_tx(&S.full[st], STAGE_BYTES);
+                    tma_load_2d(dst, &K.tmk, 0, row, &S.full[st]);
+                    tma_load_2d(dst + 8192, &K.tmk, 64, row, &S.full[st]);
+                    tma_load_2d(dst + KV_TILE, &K.tmv, 0, row, &S.full[st]);
+                    tma_load_2d(dst + KV_TILE + 8192, &K.tmv, 64, row, &S.full[st]);
+                }
+            }
+            for (int e = 0; e < ne; ++e, ++k) {
+                const int st = (int)(k % NST);
+                if (!mbar_wait_bounded(&S.full[st], (k / NST) & 1u)) {
+                    set_status(P, ST_TIMEOUT);
+                    return;
+                }
+                const uint32_t ent = S.d_list[e0 + e];
+                const int j = (int)(ent >> 8);
+                const uint32_t base = smem_u32(&S.stage[st][0]);
+                const bool zeroed =
+                    attn.tile(base, base + KV_TILE, warp, lane, j * BLK, min(BLK, L - j * BLK), ent & 0xFFu, false, 0, 0);
+                if (zeroed) fence_proxy_async();
+            }
+            consumer_sync();
+        }
+        attn.finish(S.X, warp, lane);
+        consumer_sync();
+        split_emit<G>(S.X, P.rg_mask[rg], nullptr, P.out + ((int64_t)b * P.Hq + g * G) * D, tid);
+        consumer_sync();
+        if (tid == 0) trace_max(P, 4);
     }
     if (tid == 0) trace_max(P, 23);
 }
@@ -711,6 +790,7 @@ __global__ void __launch_bounds__(THREADS, 2) stream_kernel(const __grid_constan
         }
         mbar_fence_init();
         if (P.dbg_trace) atomicCAS(P.dbg_trace, 0ull, (unsigned long long)global_ns());
+        S.d_cnt = 0;
     }
     // the retrieval kernel may be scheduled now; it waits for this grid's
     // completion before it reads anything this grid writes

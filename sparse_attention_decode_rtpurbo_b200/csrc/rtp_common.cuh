@@ -18,6 +18,7 @@ constexpr int THREADS = CONSUMERS + 32;   // + 1 copy warp
 constexpr int PSTRIDE = 132;      // floats per split partial: m, l, 2 pad, acc[128]
 constexpr int MAX_G = 8, MAX_HQ = 128, MAX_HKV = 64, MAX_B = 1024;
 constexpr int AGG_BUCKETS = 32;
+constexpr int CAND_CAP = 4096;    // threshold-bin tokens selected inside one CTA
 
 enum SelMode : int32_t { MODE_SKIP = 0, MODE_TOP1 = 1, MODE_ALL = 2, MODE_RADIX = 3 };
 
@@ -45,7 +46,7 @@ struct HeadState {
     uint32_t prefix, count_above, n_eq, n_tie, all_ties, kstar, tau_key;
     uint32_t tie_idx;                       // largest index among the threshold ties kept
     float dr, inv_w;                        // first select pass: bins of width dr/255 over smax - s in [0, dr)
-    uint32_t bstar, pad1;                   // the bin that holds the threshold
+    uint32_t bstar, n_cand;                 // the bin that holds the threshold, and its token count
 };
 
 // Coordination words of one call (workspace; zero between calls).
@@ -56,9 +57,10 @@ struct Sync {
     uint32_t barrier;          // grid barrier arrivals of the retrieval kernel
     uint32_t exit_count;
     uint32_t groups_decided;   // (b, retrieval group) pairs whose selection mode is known
-    uint32_t pass_done[8];     // radix heads whose step after select pass i is done
-    uint32_t groups_ready;     // radix groups whose block list is built
-    uint32_t pad[17];
+    uint32_t pass_done[8];     // (unused)
+    uint32_t groups_ready;     // (unused)
+    uint32_t any_global;       // some radix head's threshold bin is too large for the in-CTA select
+    uint32_t pad[16];
 };
 
 struct Params {
@@ -85,6 +87,8 @@ struct Params {
     unsigned long long* hist_mass;
     uint32_t* tie_cnt;
     float* scores;   // [B * n_ret, Ncap] fp32 index scores, written by the streaming kernel, read by the select
+    uint32_t* cand_cnt;              // [B * n_ret] candidates gathered from the threshold bin
+    unsigned long long* cand;        // [B * n_ret, CAND_CAP] (key << 32 | token index)
     uint32_t* bitmap;
     uint32_t* blist;
     uint32_t* bcount;

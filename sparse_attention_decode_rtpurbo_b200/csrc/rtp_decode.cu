@@ -30,8 +30,8 @@ struct Plan {
     uint8_t lg_group[MAX_HKV], lg_mask[MAX_HKV];
     uint8_t slot_head[MAX_HQ], slot_rg[MAX_HQ];
     // workspace byte offsets; [0, zero_end) must be zero when a call starts
-    size_t o_status, o_sync, o_tick_score, o_tick_local, o_tick_ret, o_tick_sel, o_tick_grp, o_agg, o_hist_cnt, o_hist_mass, zero_end;
-    size_t o_rlist, o_rglist, o_hs, o_tie_cnt, o_scores, o_bitmap, o_blist, o_bcount, o_lpart, o_rpart, total;
+    size_t o_status, o_sync, o_tick_score, o_tick_local, o_tick_ret, o_tick_sel, o_tick_grp, o_cand_cnt, o_agg, o_hist_cnt, o_hist_mass, zero_end;
+    size_t o_rlist, o_rglist, o_hs, o_tie_cnt, o_scores, o_cand, o_bitmap, o_blist, o_bcount, o_lpart, o_rpart, total;
 };
 
 static size_t align_up(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -116,6 +116,7 @@ static rtp_status make_plan(const rtp_dims* d, const uint8_t* head_kind, int win
     pl->o_tick_ret = take(BG * 4);
     pl->o_tick_sel = take(BR * 4);
     pl->o_tick_grp = take(BG * 4);
+    pl->o_cand_cnt = take(BR * 4);
     pl->o_agg = take(BR * AGG_BUCKETS * sizeof(HeadAgg));
     pl->o_hist_cnt = take(BR * 256 * 4);
     pl->o_hist_mass = take(BR * 256 * 8);
@@ -125,6 +126,7 @@ static rtp_status make_plan(const rtp_dims* d, const uint8_t* head_kind, int win
     pl->o_hs = take(BR * sizeof(HeadState));
     pl->o_tie_cnt = take(BR * pl->ntiles_cap * 4);
     pl->o_scores = take(BR * (size_t)pl->Ncap * 4);
+    pl->o_cand = take(BR * (size_t)CAND_CAP * 8);
     pl->o_bitmap = take(BR * pl->words_cap * 4);
     pl->o_blist = take(BG * pl->nblk_cap * 4);
     pl->o_bcount = take(BG * 4);
@@ -345,6 +347,8 @@ extern "C" rtp_status rtp_decode_step(const rtp_dims* dims, const uint16_t* q_pr
     P.hist_mass = (unsigned long long*)(ws + pl.o_hist_mass);
     P.tie_cnt = (uint32_t*)(ws + pl.o_tie_cnt);
     P.scores = (float*)(ws + pl.o_scores);
+    P.cand_cnt = (uint32_t*)(ws + pl.o_cand_cnt);
+    P.cand = (unsigned long long*)(ws + pl.o_cand);
     P.bitmap = (uint32_t*)(ws + pl.o_bitmap);
     P.blist = (uint32_t*)(ws + pl.o_blist);
     P.bcount = (uint32_t*)(ws + pl.o_bcount);

@@ -47,6 +47,8 @@ struct BSmem {
     uint32_t tcnt[MAX_G];
     uint8_t rlist_h[MAX_G];
     uint32_t nrad_h;
+    uint32_t lsel_prefix, lsel_count, lsel_neq;
+    unsigned long long lsel_mass, lsel_meq;
     uint8_t tflag[SROWS];
     RDesc desc[NST];
     alignas(8) uint64_t full[NST], empty[NST];
@@ -121,7 +123,7 @@ struct RWalk {
 
 // Per-thread view of the select state of one head.
 struct RHead {
-    uint32_t prefix, tau, tie_idx, bstar;
+    uint32_t prefix, tau, tie_idx, bstar, n_cand;
     float smax, dr, inv_w;
 };
 
@@ -131,6 +133,7 @@ __device__ __forceinline__ RHead load_rhead(const HeadState* h) {
     r.tau = __ldcg(&h->tau_key);
     r.tie_idx = __ldcg(&h->tie_idx);
     r.bstar = __ldcg(&h->bstar);
+    r.n_cand = __ldcg(&h->n_cand);
     r.smax = __ldcg(&h->smax);
     r.dr = __ldcg(&h->dr);
     r.inv_w = __ldcg(&h->inv_w);
@@ -146,10 +149,12 @@ __device__ __forceinline__ uint32_t score_bin(float s, float smax, float dr, flo
 }
 
 // What a pass does with every stored score of a radix head:
-// RP_BINS histograms the first-pass bins; RP_REF0..3 histogram the next 8
-// key bits of the scores in the threshold bin that match the key prefix
-// found so far; RP_TIES counts threshold ties per tile; RP_MARK marks blocks.
-enum RPass : int { RP_BINS = 0, RP_REF0, RP_REF1, RP_REF2, RP_REF3, RP_TIES, RP_MARK };
+// RP_BINS histograms the first-pass bins; RP_COMPACT gathers the tokens of
+// the threshold bin (when at most CAND_CAP) for a select inside one CTA;
+// otherwise RP_REF0..3 histogram the next 8 key bits of the scores in the
+// threshold bin that match the key prefix found so far and RP_TIES counts
+// threshold ties per tile; RP_MARK marks blocks.
+enum RPass : int { RP_BINS = 0, RP_REF0, RP_REF1, RP_REF2, RP_REF3, RP_TIES, RP_MARK, RP_COMPACT };
 
 template <int G>
 __device__ __noinline__ void r_digit(const Params& P, BSmem<G>& S, int b, int slot, int pass, int tid);
@@ -187,8 +192,13 @@ __device__ __noinline__ void r_pass(const Params& P, BSmem<G>& S, RWalk wk, cons
         // with the next item's scores loaded while this one is processed
         if (tid == 0) {
             uint32_t n = 0;
-            for (int hh = 0; hh < nh; ++hh)
-                if (__ldcg(&P.hs[bs0 + hh].mode) == MODE_RADIX) S.rlist_h[n++] = (uint8_t)hh;
+            for (int hh = 0; hh < nh; ++hh) {
+                const HeadState* h = P.hs + bs0 + hh;
+                if (__ldcg(&h->mode) != MODE_RADIX) continue;
+                const bool local = __ldcg(&h->n_cand) <= (uint32_t)CAND_CAP;
+                const bool want = (pass == RP_BINS || pass == RP_MARK) ? true : (pass == RP_COMPACT ? local : !local);
+                if (want) S.rlist_h[n++] = (uint8_t)hh;
+            }
             S.nrad_h = n;
         }
         consumer_sync();
@@ -263,6 +273,19 @@ __device__ __noinline__ void r_pass(const Params& P, BSmem<G>& S, RWalk wk, cons
                     }
                 } else if (pass == RP_TIES) {
                     cnt += (ok && key == rh.tau) ? 1u : 0u;
+                } else if (pass == RP_COMPACT) {
+                    const bool in = ok && score_bin(v[u], rh.smax, rh.dr, rh.inv_w) == rh.bstar;
+                    const uint32_t bal = __ballot_sync(0xffffffffu, in);
+                    if (bal) {
+                        uint32_t base = 0;
+                        if (lane == 0) base = atomicAdd(P.cand_cnt + bs0 + hh, (uint32_t)__popc(bal));
+                        base = __shfl_sync(0xffffffffu, base, 0);
+                        if (in) {
+                            const uint32_t pos = base + __popc(bal & ((1u << lane) - 1u));
+                            if (pos < (uint32_t)CAND_CAP)
+                                P.cand[(bs0 + hh) * CAND_CAP + pos] = ((unsigned long long)key << 32) | (uint32_t)(n0 + r);
+                        }
+                    }
                 } else {
                     const bool keep = ok && (key > rh.tau || (key == rh.tau && (uint32_t)(n0 + r) <= rh.tie_idx));
                     // a warp's 32 tokens lie in one 64-token block: one vote per warp
@@ -356,9 +379,11 @@ __device__ __noinline__ void r_digit(const Params& P, BSmem<G>& S, int b, int sl
                 cabove += S.dcnt[d];
             }
             st.bstar = bstar;
+            st.n_cand = S.dcnt[bstar];
             st.mass_above = cum;
             st.count_above = cabove;
             st.prefix = 0;
+            if (st.n_cand > (uint32_t)CAND_CAP) atomicOr(&P.sync->any_global, 1u);
         } else {
             const int rp = pass - RP_REF0;
             unsigned long long cum = st.mass_above;
@@ -396,6 +421,129 @@ __device__ __noinline__ void r_digit(const Params& P, BSmem<G>& S, int b, int sl
             }
         }
         P.hs[bs] = st;
+    }
+    consumer_sync();
+}
+
+// Threshold of a radix head whose threshold bin holds at most CAND_CAP
+// tokens, inside one CTA: the bin's (key, index) pairs, gathered by the
+// compaction pass, go to shared memory; four 8-bit MSD passes over the keys
+// (count and fixed-point mass per digit, cumulative from the mass above the
+// bin) give tau and the number of its ties to keep, and a four-pass select
+// over the tie indices gives the largest tie index kept (ties toward the
+// lower index).
+template <int G>
+__device__ __noinline__ void r_local_select(const Params& P, BSmem<G>& S, int b, int slot, int tid) {
+    const int64_t bs = (int64_t)b * P.n_ret + slot;
+    const uint32_t ncand = __ldcg(&P.hs[bs].n_cand);
+    if (ncand > (uint32_t)CAND_CAP) return;
+    uint32_t* keys = reinterpret_cast<uint32_t*>(&S.stage[0][0]);
+    uint32_t* idx = keys + CAND_CAP;
+    const int n = (int)ncand;
+    for (int i = tid; i < n; i += CONSUMERS) {
+        const unsigned long long c = __ldcg(P.cand + bs * CAND_CAP + i);
+        keys[i] = (uint32_t)(c >> 32);
+        idx[i] = (uint32_t)(c & 0xFFFFFFFFull);
+    }
+    const float smax = __ldcg(&P.hs[bs].smax);
+    if (tid == 0) {
+        S.lsel_prefix = 0;
+        S.lsel_mass = __ldcg(&P.hs[bs].mass_above);
+        S.lsel_count = __ldcg(&P.hs[bs].count_above);
+    }
+    const unsigned long long target = __ldcg(&P.hs[bs].target);
+    for (int rp = 0; rp < 4; ++rp) {
+        for (int d = tid; d < 256; d += CONSUMERS) {
+            S.hcnt[0][d] = 0;
+            S.hmass[0][d] = 0ull;
+        }
+        consumer_sync();
+        const uint32_t prefix = S.lsel_prefix;
+        for (int i = tid; i < n; i += CONSUMERS) {
+            const uint32_t key = keys[i];
+            if (rp > 0 && (key >> (32 - 8 * rp)) != prefix) continue;
+            const uint32_t d = (key >> (24 - 8 * rp)) & 255u;
+            atomicAdd(&S.hcnt[0][d], 1u);
+            atomicAdd(&S.hmass[0][d], fixmass(key, smax));
+        }
+        consumer_sync();
+        if (tid == 0) {
+            unsigned long long cum = S.lsel_mass;
+            uint32_t cabove = S.lsel_count;
+            int dstar = 0;
+            for (int d = 255; d >= 0; --d) {
+                if (cum + S.hmass[0][d] >= target) {
+                    dstar = d;
+                    break;
+                }
+                cum += S.hmass[0][d];
+                cabove += S.hcnt[0][d];
+            }
+            S.lsel_mass = cum;
+            S.lsel_count = cabove;
+            S.lsel_prefix = (prefix << 8) | (uint32_t)dstar;
+            S.lsel_neq = S.hcnt[0][dstar];
+            S.lsel_meq = S.hmass[0][dstar];
+        }
+        consumer_sync();
+    }
+    const uint32_t tau = S.lsel_prefix, n_eq = S.lsel_neq, count_above = S.lsel_count;
+    uint32_t n_tie = n_eq;
+    {
+        const unsigned long long m_tau = n_eq ? S.lsel_meq / n_eq : 0ull;
+        const unsigned long long need = target - S.lsel_mass;
+        if (m_tau > 0) {
+            const unsigned long long q = (need + m_tau - 1) / m_tau;
+            n_tie = (uint32_t)min((unsigned long long)n_eq, max(1ull, q));
+        }
+    }
+    // the n_tie-th smallest index among the ties (only when some ties are left out)
+    uint32_t tie_idx = 0xFFFFFFFFu;
+    if (n_tie < n_eq) {
+        if (tid == 0) {
+            S.lsel_prefix = 0;
+            S.lsel_count = n_tie;   // rank still wanted
+        }
+        for (int rp = 0; rp < 4; ++rp) {
+            for (int d = tid; d < 256; d += CONSUMERS) S.hcnt[0][d] = 0;
+            consumer_sync();
+            const uint32_t prefix = S.lsel_prefix;
+            for (int i = tid; i < n; i += CONSUMERS) {
+                if (keys[i] != tau) continue;
+                const uint32_t x = idx[i];
+                if (rp > 0 && (x >> (32 - 8 * rp)) != prefix) continue;
+                atomicAdd(&S.hcnt[0][(x >> (24 - 8 * rp)) & 255u], 1u);
+            }
+            consumer_sync();
+            if (tid == 0) {
+                uint32_t rank = S.lsel_count, cum = 0;
+                int dstar = 255;
+                for (int d = 0; d < 256; ++d) {
+                    if (cum + S.hcnt[0][d] >= rank) {
+                        dstar = d;
+                        break;
+                    }
+                    cum += S.hcnt[0][d];
+                }
+                S.lsel_count = rank - cum;
+                S.lsel_prefix = (prefix << 8) | (uint32_t)dstar;
+            }
+            consumer_sync();
+        }
+        tie_idx = S.lsel_prefix;
+    }
+    if (tid == 0) {
+        HeadState* h = P.hs + bs;
+        h->tau_key = tau;
+        h->n_eq = n_eq;
+        h->n_tie = n_tie;
+        h->all_ties = n_tie == n_eq ? 1u : 0u;
+        h->tie_idx = tie_idx;
+        h->kstar = count_above + n_tie;
+        const int bh = b * P.Hq + P.slot_head[slot];
+        if (P.dbg_tau) P.dbg_tau[bh] = key2f(tau);
+        if (P.dbg_kstar) P.dbg_kstar[bh] = (int32_t)(count_above + n_tie);
+        P.cand_cnt[bs] = 0;
     }
     consumer_sync();
 }
@@ -713,18 +861,43 @@ __global__ void __launch_bounds__(THREADS, 2) retrieve_kernel(const __grid_const
         wk.t = (int)((long long)blockIdx.x * T / gridDim.x);
         wk.t1 = (int)((long long)(blockIdx.x + 1) * T / gridDim.x);
         wk.ngr = ngr;
-        for (int pass = RP_BINS; pass <= RP_REF3 && ok; ++pass) {
+        // first pass: bins; then the threshold bin's tokens are gathered and
+        // selected inside one CTA per head, or, for a bin of more than
+        // CAND_CAP tokens, refined by four more passes over all scores
+        if (!copier) r_pass<G>(P, S, wk, pre, RP_BINS, tid);
+        ok = grid_sync(P, S);
+        if (ok && !copier)
+            for (int hx = blockIdx.x; hx < (int)nrad; hx += gridDim.x) {
+                const uint32_t e = __ldcg(P.rlist + hx);
+                r_digit<G>(P, S, (int)(e >> 16), (int)(e & 0xFFFFu), RP_BINS, tid);
+            }
+        ok = ok && grid_sync(P, S);
+        if (tid == 0) trace_max(P, 14);
+        if (ok) {
+            if (!copier) r_pass<G>(P, S, wk, pre, RP_COMPACT, tid);
+            ok = grid_sync(P, S);
+        }
+        if (ok && !copier)
+            for (int hx = blockIdx.x; hx < (int)nrad; hx += gridDim.x) {
+                const uint32_t e = __ldcg(P.rlist + hx);
+                r_local_select<G>(P, S, (int)(e >> 16), (int)(e & 0xFFFFu), tid);
+            }
+        if (ok) ok = grid_sync(P, S);
+        if (tid == 0) trace_max(P, 8);
+        const bool global = ok && __ldcg(&P.sync->any_global) != 0;
+        for (int pass = RP_REF0; global && pass <= RP_REF3 && ok; ++pass) {
             if (!copier) r_pass<G>(P, S, wk, pre, pass, tid);
             ok = grid_sync(P, S);
             if (!ok) break;
-            if (tid == 0 && pass == RP_BINS) trace_max(P, 14);
             if (!copier)
                 for (int hx = blockIdx.x; hx < (int)nrad; hx += gridDim.x) {
                     const uint32_t e = __ldcg(P.rlist + hx);
-                    r_digit<G>(P, S, (int)(e >> 16), (int)(e & 0xFFFFu), pass, tid);
+                    const int64_t bs = (int64_t)(e >> 16) * P.n_ret + (e & 0xFFFFu);
+                    if (__ldcg(&P.hs[bs].n_cand) > (uint32_t)CAND_CAP)
+                        r_digit<G>(P, S, (int)(e >> 16), (int)(e & 0xFFFFu), pass, tid);
                 }
             ok = grid_sync(P, S);
-            if (tid == 0 && pass > RP_BINS) trace_max(P, 8 + pass - RP_REF0);
+            if (tid == 0) trace_max(P, 8 + pass - RP_REF0);
         }
         if (ok && __ldcg(&P.sync->any_ties)) {
             if (!copier) r_pass<G>(P, S, wk, pre, RP_TIES, tid);
@@ -732,7 +905,9 @@ __global__ void __launch_bounds__(THREADS, 2) retrieve_kernel(const __grid_const
             if (ok && !copier)
                 for (int hx = blockIdx.x; hx < (int)nrad; hx += gridDim.x) {
                     const uint32_t e = __ldcg(P.rlist + hx);
-                    r_tie_locate<G>(P, S, (int)(e >> 16), (int)(e & 0xFFFFu), tid);
+                    const int64_t bs = (int64_t)(e >> 16) * P.n_ret + (e & 0xFFFFu);
+                    if (__ldcg(&P.hs[bs].n_cand) > (uint32_t)CAND_CAP)
+                        r_tie_locate<G>(P, S, (int)(e >> 16), (int)(e & 0xFFFFu), tid);
                 }
             ok = ok && grid_sync(P, S);
         }
@@ -793,6 +968,7 @@ __global__ void __launch_bounds__(THREADS, 2) retrieve_kernel(const __grid_const
             P.sync->groups_decided = 0;
             for (int i = 0; i < 8; ++i) P.sync->pass_done[i] = 0;
             P.sync->groups_ready = 0;
+            P.sync->any_global = 0;
             P.sync->exit_count = 0;
             __threadfence();
         }

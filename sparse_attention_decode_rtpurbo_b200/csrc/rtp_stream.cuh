@@ -243,7 +243,7 @@ __device__ __noinline__ void decide_group(const Params& P, ASmem<G>& S, int b, i
             h.dr = dr;
             h.inv_w = 255.f / dr;
             h.bstar = 0;
-            h.pad1 = 0;
+            h.n_cand = 0;
         }
         P.hs[(int64_t)b * P.n_ret + slot] = h;
         const int bh = b * P.Hq + P.slot_head[slot];

@@ -26,7 +26,9 @@
  * Conventions
  *   - Every tensor pointer is DEVICE memory owned by the caller unless marked
  *     host.  bf16 tensors are passed as uint16_t bit patterns.  Strides are
- *     the dense row-major strides of the stated shapes.
+ *     the dense row-major strides of the stated shapes.  The bf16 tensors and
+ *     `out` must be 16-byte aligned (else RTP_ERR_UNSUPPORTED): the caches
+ *     are read by TMA / bulk copies.
  *   - The library allocates no memory.  Scratch lives in a caller-allocated
  *     device workspace of rtp_workspace_size() bytes.  Zero-fill it once
  *     after allocation (cudaMemset); every call leaves it ready for the next.
@@ -86,7 +88,10 @@ typedef struct rtp_debug {
 
 /*
  * Sizes and layout of one call.
- *   batch, num_q_heads (Hq), num_kv_heads (Hkv): Hq % Hkv == 0, Hq/Hkv <= 8.
+ *   batch, num_q_heads (Hq), num_kv_heads (Hkv): Hq % Hkv == 0, Hq/Hkv in
+ *     {1, 2, 4, 8}, batch <= 1024, Hq <= 128, Hkv <= 64, batch x (KV heads
+ *     with a retrieval head) <= 4096, and fewer than 2^31 cache rows of 128
+ *     (batch x Hkv x max_seq_len, or num_pages x Hkv x 64).
  *   head_dim must be 128, idx_dim 16, block_size 64.
  *   max_seq_len: per-sequence capacity in tokens, a multiple of 64.
  *     Contiguous layout: caches are [batch, Hkv, max_seq_len, dim].

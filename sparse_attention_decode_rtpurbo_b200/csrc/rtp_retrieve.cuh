@@ -834,13 +834,9 @@ __global__ void __launch_bounds__(THREADS, 2) retrieve_kernel(const __grid_const
         S.gen = 0;
         S.abort = 0;
     }
-    // everything below reads the selection results of the streaming kernel,
-    // which may still be streaming local heads: wait for every group's
-    // decision (written before the count, with a fence)
-    if (tid == 0 && !wait_counter(&P.sync->groups_decided, (uint32_t)(P.B * P.n_rg))) {
-        set_status(P, ST_TIMEOUT);
-        S.abort = 1;
-    }
+    // everything below reads the streaming kernel's results: wait for that
+    // grid to complete (this launch overlaps only its tail)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     __syncthreads();
     if (tid == 0) trace_max(P, 13);
     uint32_t k = 0;

@@ -25,9 +25,9 @@ struct ASmem {
     static constexpr int NST = (G >= 8) ? 2 : 3;
     alignas(1024) uint8_t stage[NST][STAGE_BYTES];
     AttnScratch<G> X;
-    alignas(16) float qi[MAX_G][R];
-    float w_m[4][MAX_G], w_s[4][MAX_G], w_bv[4][MAX_G], w_mn[4][MAX_G];
-    uint32_t w_bi[4][MAX_G];
+    alignas(16) float qi[G][R];
+    float w_m[4][G], w_s[4][G], w_bv[4][G], w_mn[4][G];
+    uint32_t w_bi[4][G];
     alignas(8) uint64_t full[NST], empty[NST];
     unsigned long long d_best[MAX_G];
     uint32_t d_nmin[MAX_G], d_flags[MAX_G], d_arg[MAX_G];
@@ -42,7 +42,7 @@ struct ASmem {
 
 template <int G>
 constexpr size_t asmem_bytes(int B) {
-    return sizeof(ASmem<G>) + sizeof(int) * 2 * (size_t)(B + 1) + 1024;   // + alignment slack
+    return sizeof(ASmem<G>) + sizeof(int) * 2 * (size_t)(B + 1);
 }
 
 // One run of consecutive tiles of a single item inside a CTA's share.
@@ -134,6 +134,23 @@ struct AWalk {
     }
 };
 
+// The best-token blocks a CTA selected (decide_group), as one more attention
+// segment after its share: type 2, tiles = the block list in shared memory.
+template <typename SM>
+__device__ __forceinline__ Seg best_token_seg(const SM& S) {
+    Seg s;
+    s.type = 2;
+    s.b = S.pend_b;
+    s.grp = S.pend_rg;
+    s.L = S.pend_L;
+    s.item_idx = 0;
+    s.item_t0 = 0;
+    s.item_tiles = (int)S.d_cnt;
+    s.first = 0;
+    s.ntiles = (int)S.d_cnt;
+    return s;
+}
+
 // Ticket among the consumer threads with a variable increment: true in the
 // CTA whose addition completes `total`; it re-arms the counter.
 __device__ __forceinline__ bool ticket_add(uint32_t* ctr, uint32_t add, uint32_t total, uint32_t* smem_flag) {
@@ -159,7 +176,7 @@ __device__ __forceinline__ bool ticket_add(uint32_t* ctr, uint32_t add, uint32_t
 // final here; if every head of the group is final its block list is written
 // at once, otherwise its radix heads are registered for the exact select.
 template <int G>
-__device__ __noinline__ void decide_group(const Params& P, ASmem<G>& S, int b, int rg, int L, float pb, int tid) {
+__device__ __forceinline__ void decide_group(const Params& P, ASmem<G>& S, int b, int rg, int L, float pb, int tid) {
     const int nh = P.rg_nh[rg], slot0 = P.rg_slot0[rg], g = P.rg_group[rg];
     const int nblk = (L + BLK - 1) / BLK;
     const int nwords = (nblk + 31) / 32;
@@ -311,8 +328,6 @@ __device__ __noinline__ void decide_group(const Params& P, ASmem<G>& S, int b, i
                 }
             const uint32_t gi = atomicAdd(&P.sync->n_radix_groups, 1u);
             P.rglist[gi] = ((uint32_t)b << 16) | (uint32_t)rg;
-            __threadfence();
-            atomicAdd(&P.sync->groups_decided, 1u);
         }
         return;
     }
@@ -362,11 +377,6 @@ __device__ __noinline__ void decide_group(const Params& P, ASmem<G>& S, int b, i
                 P.bcount[bg] = 0;
             }
         }
-    }
-    consumer_sync();
-    if (tid == 0) {
-        __threadfence();
-        atomicAdd(&P.sync->groups_decided, 1u);
     }
 }
 
@@ -554,8 +564,18 @@ __device__ __forceinline__ void a_producer(const KParams& K, ASmem<G>& S, AWalk 
     const Params& P = K.P;
     uint32_t k = 0;
     bool alive = true;
-    for (Seg sg = wk.next(P, pre_s, pre_l, S.tot_s); sg.type >= 0 && alive; sg = wk.next(P, pre_s, pre_l, S.tot_s)) {
-        const int g = sg.type == 0 ? P.rg_group[sg.grp] : P.lg_group[sg.grp];
+    bool extra = false;
+    for (Seg sg = wk.next(P, pre_s, pre_l, S.tot_s);; sg = extra ? Seg{-1} : wk.next(P, pre_s, pre_l, S.tot_s)) {
+        if (sg.type < 0 || !alive) {
+            if (extra) break;
+            // share issued: meet the compute warps, then issue the best-token
+            // blocks their group decision put in shared memory (if any)
+            extra = true;
+            asm volatile("bar.sync 3, 160;" ::: "memory");
+            if (!alive || S.d_cnt == 0) break;
+            sg = best_token_seg(S);
+        }
+        const int g = sg.type == 0 ? P.rg_group[sg.grp] : (sg.type == 1 ? P.lg_group[sg.grp] : P.rg_group[sg.grp]);
         const LocalGeom lg = local_geom(P, sg.L);
         for (int i = 0; i < sg.ntiles; ++i, ++k) {
             const int st = (int)(k % NST);
@@ -585,7 +605,7 @@ __device__ __forceinline__ void a_producer(const KParams& K, ASmem<G>& S, AWalk 
                                  &S.full[st]);
                 }
             } else if (lane == 0) {
-                const int j = ti < lg.nA ? ti : lg.bw0 + (ti - lg.nA);
+                const int j = sg.type == 1 ? (ti < lg.nA ? ti : lg.bw0 + (ti - lg.nA)) : (int)(S.d_list[ti] >> 8);
                 const int row = (int)block_row(P, sg.b, g, j);
                 mbar_expect_tx(&S.full[st], STAGE_BYTES);
                 tma_load_2d(dst, &K.tmk, 0, row, &S.full[st]);
@@ -601,8 +621,6 @@ __device__ __forceinline__ void a_producer(const KParams& K, ASmem<G>& S, AWalk 
     if (lane == 0)
         for (uint32_t i = (k > (uint32_t)NST ? k - NST : 0u); i < k; ++i)
             mbar_wait_bounded(&S.full[i % NST], (i / NST) & 1u);
-    __syncwarp();
-    asm volatile("bar.arrive 2, 160;" ::: "memory");
 }
 
 // ---------------------------------------------------------------------------
@@ -622,7 +640,17 @@ __device__ __forceinline__ void a_consumers(const KParams& K, ASmem<G>& S, AWalk
     Acct ac;
     ac.init(P, tid == 0);
     bool first_data = true;
-    for (Seg sg = wk.next(P, pre_s, pre_l, S.tot_s); sg.type >= 0; sg = wk.next(P, pre_s, pre_l, S.tot_s)) {
+    bool extra = false;
+    for (Seg sg = wk.next(P, pre_s, pre_l, S.tot_s);; sg = extra ? Seg{-1} : wk.next(P, pre_s, pre_l, S.tot_s)) {
+        if (sg.type < 0) {
+            if (extra) break;
+            // share done: meet the copy warp, then the best-token blocks this
+            // CTA selected (if any) follow through the ring as one more segment
+            extra = true;
+            asm volatile("bar.sync 3, 160;" ::: "memory");
+            if (S.d_cnt == 0) break;
+            sg = best_token_seg(S);
+        }
         if (sg.type == 0) {
             // ---- index scores of (b, retrieval group): q_idx while the first tile is in flight
             const int nh = P.rg_nh[sg.grp];
@@ -644,6 +672,7 @@ __device__ __forceinline__ void a_consumers(const KParams& K, ASmem<G>& S, AWalk
                 const int st = (int)(k % NST);
                 if (!mbar_wait_bounded(&S.full[st], (k / NST) & 1u)) {
                     set_status(P, ST_TIMEOUT);
+                    if (!extra) asm volatile("bar.arrive 3, 160;" ::: "memory");
                     return;
                 }
                 ac.mark(16);
@@ -675,9 +704,12 @@ __device__ __forceinline__ void a_consumers(const KParams& K, ASmem<G>& S, AWalk
             }
             ac.mark(28);
         } else {
-            // ---- local heads of (b, local group): sink + window blocks
-            const int g = P.lg_group[sg.grp];
-            const uint32_t heads = P.lg_mask[sg.grp];
+            // ---- attention: local heads of (b, local group) over sink + window
+            // blocks (type 1), or the best-token blocks this CTA selected for
+            // (b, retrieval group) (type 2), through the same code
+            const bool local = sg.type == 1;
+            const int g = local ? P.lg_group[sg.grp] : P.rg_group[sg.grp];
+            const uint32_t heads = local ? P.lg_mask[sg.grp] : P.rg_mask[sg.grp];
             const LocalGeom lg = local_geom(P, sg.L);
             attn.begin(P, sg.b, g, lane);
             ac.mark(29);
@@ -685,16 +717,25 @@ __device__ __forceinline__ void a_consumers(const KParams& K, ASmem<G>& S, AWalk
                 const int st = (int)(k % NST);
                 if (!mbar_wait_bounded(&S.full[st], (k / NST) & 1u)) {
                     set_status(P, ST_TIMEOUT);
+                    if (!extra) asm volatile("bar.arrive 3, 160;" ::: "memory");
                     return;
                 }
                 ac.mark(16);
                 if (first_data && tid == 0) trace_max(P, 22);
                 first_data = false;
                 const int ti = sg.first + i;
-                const int j = ti < lg.nA ? ti : lg.bw0 + (ti - lg.nA);
+                int j;
+                uint32_t hm;
+                if (local) {
+                    j = ti < lg.nA ? ti : lg.bw0 + (ti - lg.nA);
+                    hm = heads;
+                } else {
+                    j = (int)(S.d_list[ti] >> 8);
+                    hm = S.d_list[ti] & 0xFFu;
+                }
                 const uint32_t base = smem_u32(&S.stage[st][0]);
-                const bool zeroed = attn.tile(base, base + KV_TILE, warp, lane, j * BLK, min(BLK, sg.L - j * BLK),
-                                              heads, true, lg.s_end, lg.w_lo);
+                const bool zeroed = attn.tile(base, base + KV_TILE, warp, lane, j * BLK, min(BLK, sg.L - j * BLK), hm,
+                                              local, lg.s_end, lg.w_lo);
                 if (zeroed) fence_proxy_async();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&S.empty[st]);
@@ -707,7 +748,7 @@ __device__ __forceinline__ void a_consumers(const KParams& K, ASmem<G>& S, AWalk
             if (sg.ntiles == sg.item_tiles) {
                 split_emit<G>(S.X, heads, nullptr, out0, tid);
                 consumer_sync();
-                if (tid == 0) trace_max(P, 2);
+                if (tid == 0) trace_max(P, local ? 2 : 4);
             } else {
                 const int c = (int)blockIdx.x;
                 float* part = P.lpart + ((int64_t)c + sg.item_idx) * G * PSTRIDE;
@@ -725,49 +766,6 @@ __device__ __forceinline__ void a_consumers(const KParams& K, ASmem<G>& S, AWalk
             ac.mark(30);
         }
     }
-    // best-token blocks selected by this CTA: attended here, through the same
-    // ring (the copy warp has finished: it signals barrier 2 when done)
-    asm volatile("bar.sync 2, 160;" ::: "memory");
-    if (S.d_cnt > 0) {
-        const int b = S.pend_b, rg = S.pend_rg, L = S.pend_L, g = P.rg_group[rg];
-        const int cnt = (int)S.d_cnt;
-        attn.begin(P, b, g, lane);
-        for (int e0 = 0; e0 < cnt; e0 += NST) {
-            const int ne = min(NST, cnt - e0);
-            if (tid == 0) {
-                for (int e = 0; e < ne; ++e) {
-                    const int st = (int)((k + e) % NST);
-                    const int j = (int)(S.d_list[e0 + e] >> 8);
-                    const int row = (int)block_row(P, b, g, j);
-                    uint8_t* dst = &S.stage[st][0];
-                    mbar_expect_tx(&S.full[st], STAGE_BYTES);
-                    tma_load_2d(dst, &K.tmk, 0, row, &S.full[st]);
-                    tma_load_2d(dst + 8192, &K.tmk, 64, row, &S.full[st]);
-                    tma_load_2d(dst + KV_TILE, &K.tmv, 0, row, &S.full[st]);
-                    tma_load_2d(dst + KV_TILE + 8192, &K.tmv, 64, row, &S.full[st]);
-                }
-            }
-            for (int e = 0; e < ne; ++e, ++k) {
-                const int st = (int)(k % NST);
-                if (!mbar_wait_bounded(&S.full[st], (k / NST) & 1u)) {
-                    set_status(P, ST_TIMEOUT);
-                    return;
-                }
-                const uint32_t ent = S.d_list[e0 + e];
-                const int j = (int)(ent >> 8);
-                const uint32_t base = smem_u32(&S.stage[st][0]);
-                const bool zeroed =
-                    attn.tile(base, base + KV_TILE, warp, lane, j * BLK, min(BLK, L - j * BLK), ent & 0xFFu, false, 0, 0);
-                if (zeroed) fence_proxy_async();
-            }
-            consumer_sync();
-        }
-        attn.finish(S.X, warp, lane);
-        consumer_sync();
-        split_emit<G>(S.X, P.rg_mask[rg], nullptr, P.out + ((int64_t)b * P.Hq + g * G) * D, tid);
-        consumer_sync();
-        if (tid == 0) trace_max(P, 4);
-    }
     if (tid == 0) trace_max(P, 23);
 }
 
@@ -776,11 +774,17 @@ __device__ __forceinline__ void a_consumers(const KParams& K, ASmem<G>& S, AWalk
 // ---------------------------------------------------------------------------
 template <int G>
 __global__ void __launch_bounds__(THREADS, 2) stream_kernel(const __grid_constant__ KParams K) {
-    extern __shared__ uint8_t smem_raw[];
-    ASmem<G>& S = *reinterpret_cast<ASmem<G>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    extern __shared__ __align__(1024) uint8_t smem_raw[];   // no static shared memory: the base is aligned
+    ASmem<G>& S = *reinterpret_cast<ASmem<G>*>(smem_raw);
     constexpr int NST = ASmem<G>::NST;
     const Params& P = K.P;
     const int tid = threadIdx.x;
+    // the 128-byte-swizzled TMA boxes need 1024-byte aligned stages: refuse
+    // (status RTP_ERR_CUDA) rather than copy into a misaligned ring
+    if (smem_u32(smem_raw) & 1023u) {
+        if (tid == 0) set_status(P, 5u);
+        return;
+    }
     int* pre_s = S.pre;
     int* pre_l = S.pre + (P.B + 1);
     if (tid == 0) {
@@ -811,8 +815,6 @@ __global__ void __launch_bounds__(THREADS, 2) stream_kernel(const __grid_constan
                     // an invalid length: no outputs for this sequence, no blocks
                     set_status(P, ST_DEVICE_INPUT);
                     for (int rg = 0; rg < P.n_rg; ++rg) P.bcount[b * P.n_rg + rg] = 0;
-                    __threadfence();
-                    atomicAdd(&P.sync->groups_decided, (uint32_t)P.n_rg);
                 }
             }
             int is = ns, il = nl;

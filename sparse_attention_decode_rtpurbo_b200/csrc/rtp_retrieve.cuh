@@ -837,11 +837,13 @@ __global__ void __launch_bounds__(THREADS, 2) retrieve_kernel(const __grid_const
     // everything below reads the streaming kernel's results: wait for that
     // grid to complete (this launch overlaps only its tail)
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (tid == 0) S.base = __ldcg(&P.sync->kb_work);
     __syncthreads();
+    const bool work = S.base != 0;   // nothing left when every group was settled in the streaming kernel
     if (tid == 0) trace_max(P, 13);
     uint32_t k = 0;
     bool ok = S.abort == 0;
-    const uint32_t nrad = ok ? __ldcg(&P.sync->n_radix_heads) : 0u;
+    const uint32_t nrad = (ok && work) ? __ldcg(&P.sync->n_radix_heads) : 0u;
     if (nrad > 0) {
         // ---- exact select of the radix heads
         const int ngr = (int)__ldcg(&P.sync->n_radix_groups);
@@ -923,7 +925,7 @@ __global__ void __launch_bounds__(THREADS, 2) retrieve_kernel(const __grid_const
         }
     }
     if (tid == 0) trace_max(P, 3);
-    if (ok) {
+    if (ok && work) {
         // ---- block-sparse attention over every group's block list
         const int ngroups = P.B * P.n_rg;
         if (tid < 32)
@@ -961,7 +963,7 @@ __global__ void __launch_bounds__(THREADS, 2) retrieve_kernel(const __grid_const
             P.sync->n_radix_groups = 0;
             P.sync->any_ties = 0;
             P.sync->barrier = 0;
-            P.sync->groups_decided = 0;
+            P.sync->kb_work = 0;
             for (int i = 0; i < 8; ++i) P.sync->pass_done[i] = 0;
             P.sync->groups_ready = 0;
             P.sync->any_global = 0;

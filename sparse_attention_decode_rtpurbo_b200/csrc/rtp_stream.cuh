@@ -328,6 +328,7 @@ __device__ __forceinline__ void decide_group(const Params& P, ASmem<G>& S, int b
                 }
             const uint32_t gi = atomicAdd(&P.sync->n_radix_groups, 1u);
             P.rglist[gi] = ((uint32_t)b << 16) | (uint32_t)rg;
+            atomicAdd(&P.sync->kb_work, 1u);
         }
         return;
     }
@@ -341,7 +342,10 @@ __device__ __forceinline__ void decide_group(const Params& P, ASmem<G>& S, int b
                     hm |= 1u << (P.slot_head[slot0 + hh] - g * P.G);
             list[j] = ((uint32_t)j << 8) | hm;
         }
-        if (tid == 0) P.bcount[bg] = (uint32_t)nblk;
+        if (tid == 0) {
+            P.bcount[bg] = (uint32_t)nblk;
+            atomicAdd(&P.sync->kb_work, 1u);
+        }
     } else {
         // only best-token blocks: the distinct argmax blocks, ascending, are
         // attended by this CTA after its share (the first such group of the
@@ -368,6 +372,7 @@ __device__ __forceinline__ void decide_group(const Params& P, ASmem<G>& S, int b
             if (S.d_cnt != 0 || cnt == 0) {
                 for (uint32_t e = 0; e < cnt; ++e) list[e] = lst[e];
                 P.bcount[bg] = cnt;
+                if (cnt) atomicAdd(&P.sync->kb_work, 1u);
             } else {
                 for (uint32_t e = 0; e < cnt; ++e) S.d_list[e] = lst[e];
                 S.d_cnt = cnt;

@@ -215,29 +215,51 @@ __device__ __forceinline__ void split_emit(const AttnScratch<G>& X, uint32_t hea
 // Combine `nparts` split partials (stride G * PSTRIDE floats) of the heads in
 // `heads` into the bf16 outputs out0[h * D] (round to nearest even).  The
 // split weights 2^(m_i - M) go to shared memory first (X.red, free once the
-// splits are emitted) so that each thread's loop over the splits issues
-// independent loads only.
+// splits are emitted, as [part][head]); then thread d sums column d of every
+// head with 8 parts x G heads of loads in flight at a time, so that a
+// combine costs about nparts / 8 memory round trips rather than one per part.
 template <int G>
 __device__ __noinline__ void combine_splits(AttnScratch<G>& X, const float* parts, int nparts, uint32_t heads,
                                             uint16_t* out0, int tid) {
     const int warp = tid >> 5, lane = tid & 31;
-    float* wts = &X.red[0][0][0];   // [G][nparts]
+    float* wts = &X.red[0][0][0];   // [nparts][G]
     const bool in_smem = nparts <= 4 * D;
     for (int h = warp; h < G; h += CONSUMERS / 32) {
+        // (m, l) of parts lane and lane + 32 stay in registers
+        float mr[2], lr[2];
         float M = -INFINITY;
-        for (int i = lane; i < nparts; i += 32) {
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            const int i = lane + 32 * r;
+            mr[r] = -INFINITY;
+            lr[r] = 0.f;
+            if (i < nparts) {
+                const float* pp = parts + ((int64_t)i * G + h) * PSTRIDE;
+                mr[r] = __ldcg(pp);
+                lr[r] = __ldcg(pp + 1);
+            }
+            if (lr[r] > 0.f) M = fmaxf(M, mr[r]);
+        }
+        for (int i = lane + 64; i < nparts; i += 32) {
             const float* pp = parts + ((int64_t)i * G + h) * PSTRIDE;
             if (__ldcg(pp + 1) > 0.f) M = fmaxf(M, __ldcg(pp));
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
         float den = 0.f;
-        for (int i = lane; i < nparts; i += 32) {
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            const int i = lane + 32 * r;
+            const float w = (M != -INFINITY && lr[r] > 0.f) ? ex2_approx(mr[r] - M) : 0.f;
+            den = fmaf(lr[r] > 0.f ? lr[r] : 0.f, w, den);
+            if (in_smem && i < nparts) wts[i * G + h] = w;
+        }
+        for (int i = lane + 64; i < nparts; i += 32) {
             const float* pp = parts + ((int64_t)i * G + h) * PSTRIDE;
             const float li = __ldcg(pp + 1);
             const float w = (M != -INFINITY && li > 0.f) ? ex2_approx(__ldcg(pp) - M) : 0.f;
             den = fmaf(li > 0.f ? li : 0.f, w, den);
-            if (in_smem) wts[h * nparts + i] = w;
+            if (in_smem) wts[i * G + h] = w;
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
@@ -247,28 +269,45 @@ __device__ __noinline__ void combine_splits(AttnScratch<G>& X, const float* part
         }
     }
     consumer_sync();
-#pragma unroll 1
-    for (int h = 0; h < G; ++h) {
-        if (!((heads >> h) & 1u)) continue;
-        const float den = X.cden[h], M = X.cm[h];
-        if (!(den > 0.f)) continue;
-        float a[4] = {0.f, 0.f, 0.f, 0.f};
-        int i = 0;
-        if (in_smem) {
-            for (; i + 4 <= nparts; i += 4) {
+    if (in_smem) {
+        constexpr int U = G >= 8 ? 4 : 8;   // parts per batch (registers)
+        float acc[G];
 #pragma unroll
-                for (int u = 0; u < 4; ++u)
-                    a[u] = fmaf(wts[h * nparts + i + u], __ldcg(parts + ((int64_t)(i + u) * G + h) * PSTRIDE + 4 + tid), a[u]);
-            }
-            for (; i < nparts; ++i)
-                a[0] = fmaf(wts[h * nparts + i], __ldcg(parts + ((int64_t)i * G + h) * PSTRIDE + 4 + tid), a[0]);
-        } else {
-            for (; i < nparts; ++i) {
-                const float* p0 = parts + ((int64_t)i * G + h) * PSTRIDE;
-                if (__ldcg(p0 + 1) > 0.f) a[0] = fmaf(ex2_approx(__ldcg(p0) - M), __ldcg(p0 + 4 + tid), a[0]);
-            }
+        for (int h = 0; h < G; ++h) acc[h] = 0.f;
+        const float* col = parts + 4 + tid;
+        for (int i = 0; i < nparts; i += U) {
+            float v[U][G];
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+#pragma unroll
+                for (int h = 0; h < G; ++h)
+                    v[u][h] = (i + u < nparts && ((heads >> h) & 1u))
+                                  ? __ldcg(col + ((int64_t)(i + u) * G + h) * PSTRIDE) : 0.f;
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+#pragma unroll
+                for (int h = 0; h < G; ++h)
+                    if (i + u < nparts) acc[h] = fmaf(wts[(i + u) * G + h], v[u][h], acc[h]);
         }
-        out0[h * D + tid] = __bfloat16_as_ushort(__float2bfloat16_rn(((a[0] + a[1]) + (a[2] + a[3])) / den));
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            const float den = X.cden[h];
+            if (((heads >> h) & 1u) && den > 0.f)
+                out0[h * D + tid] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[h] / den));
+        }
+    } else {
+#pragma unroll 1
+        for (int h = 0; h < G; ++h) {
+            if (!((heads >> h) & 1u)) continue;
+            const float den = X.cden[h], M = X.cm[h];
+            if (!(den > 0.f)) continue;
+            float a = 0.f;
+            for (int i = 0; i < nparts; ++i) {
+                const float* p0 = parts + ((int64_t)i * G + h) * PSTRIDE;
+                if (__ldcg(p0 + 1) > 0.f) a = fmaf(ex2_approx(__ldcg(p0) - M), __ldcg(p0 + 4 + tid), a);
+            }
+            out0[h * D + tid] = __bfloat16_as_ushort(__float2bfloat16_rn(a / den));
+        }
     }
     consumer_sync();
 }
@@ -285,33 +324,55 @@ struct QFrag {
 };
 
 // q_idx[hh][r] = Wq_idx[h] . q_pre[b,h] (fp32, fixed summation order) for the
-// nh retrieval heads of group rg, by the 128 consumer threads.
-__device__ __forceinline__ void compute_qidx(const Params& P, float (*qi)[R], int b, int rg, int tid) {
-    const int nh = P.rg_nh[rg], slot0 = P.rg_slot0[rg];
-    const int npair = nh * R;   // <= 128
-    const int tpp = CONSUMERS / npair >= 8 ? 8 : (CONSUMERS / npair >= 4 ? 4 : (CONSUMERS / npair >= 2 ? 2 : 1));
-    const int pr = tid / tpp, part = tid % tpp;
+// nh retrieval heads of group rg, by the 128 consumer threads: TPP threads per
+// (head, r) pair, each over D / TPP elements, with every load of a thread
+// issued before its first product (one or two memory round trips, not D / 8).
+template <int TPP>
+__device__ __forceinline__ void qidx_pairs(const Params& P, const HeadTab& T, float (*qi)[R], int b, int rg,
+                                           int tid) {
+    constexpr int SPAN = D / TPP, NV = SPAN / 8;
+    const int nh = T.rg_nh[rg], slot0 = T.rg_slot0[rg];
+    const int pr = tid / TPP, part = tid % TPP;
     float a = 0.f;
-    if (pr < npair) {
+    if (pr < nh * R) {
         const int hh = pr / R, r = pr % R;
-        const int h = P.slot_head[slot0 + hh];
-        const int span = D / tpp;
-        const uint4* w = reinterpret_cast<const uint4*>(P.Wq + ((int64_t)h * R + r) * D + part * span);
-        const uint4* q = reinterpret_cast<const uint4*>(P.q_pre + ((int64_t)b * P.Hq + h) * D + part * span);
-        for (int i = 0; i < span / 8; ++i) {
-            const uint4 wv = __ldg(w + i), qv = __ldg(q + i);
-            a = fmaf(bf_lo(wv.x), bf_lo(qv.x), a);
-            a = fmaf(bf_hi(wv.x), bf_hi(qv.x), a);
-            a = fmaf(bf_lo(wv.y), bf_lo(qv.y), a);
-            a = fmaf(bf_hi(wv.y), bf_hi(qv.y), a);
-            a = fmaf(bf_lo(wv.z), bf_lo(qv.z), a);
-            a = fmaf(bf_hi(wv.z), bf_hi(qv.z), a);
-            a = fmaf(bf_lo(wv.w), bf_lo(qv.w), a);
-            a = fmaf(bf_hi(wv.w), bf_hi(qv.w), a);
+        const int h = T.slot_head[slot0 + hh];
+        const uint4* w = reinterpret_cast<const uint4*>(P.Wq + ((int64_t)h * R + r) * D + part * SPAN);
+        const uint4* q = reinterpret_cast<const uint4*>(P.q_pre + ((int64_t)b * P.Hq + h) * D + part * SPAN);
+        constexpr int NB = NV < 8 ? NV : 8;   // loads in flight per operand (register budget)
+#pragma unroll
+        for (int i0 = 0; i0 < NV; i0 += NB) {
+            uint4 wv[NB], qv[NB];
+#pragma unroll
+            for (int i = 0; i < NB; ++i) {
+                wv[i] = __ldg(w + i0 + i);
+                qv[i] = __ldg(q + i0 + i);
+            }
+#pragma unroll
+            for (int i = 0; i < NB; ++i) {
+                a = fmaf(bf_lo(wv[i].x), bf_lo(qv[i].x), a);
+                a = fmaf(bf_hi(wv[i].x), bf_hi(qv[i].x), a);
+                a = fmaf(bf_lo(wv[i].y), bf_lo(qv[i].y), a);
+                a = fmaf(bf_hi(wv[i].y), bf_hi(qv[i].y), a);
+                a = fmaf(bf_lo(wv[i].z), bf_lo(qv[i].z), a);
+                a = fmaf(bf_hi(wv[i].z), bf_hi(qv[i].z), a);
+                a = fmaf(bf_lo(wv[i].w), bf_lo(qv[i].w), a);
+                a = fmaf(bf_hi(wv[i].w), bf_hi(qv[i].w), a);
+            }
         }
     }
-    for (int o = 1; o < tpp; o <<= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-    if (pr < npair && part == 0) qi[pr / R][pr % R] = a;
+#pragma unroll
+    for (int o = 1; o < TPP; o <<= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+    if (pr < nh * R && part == 0) qi[pr / R][pr % R] = a;
+}
+
+__device__ __forceinline__ void compute_qidx(const Params& P, const HeadTab& T, float (*qi)[R], int b, int rg,
+                                             int tid) {
+    const int npair = T.rg_nh[rg] * R;   // <= 128
+    if (npair <= CONSUMERS / 8) qidx_pairs<8>(P, T, qi, b, rg, tid);
+    else if (npair <= CONSUMERS / 4) qidx_pairs<4>(P, T, qi, b, rg, tid);
+    else if (npair <= CONSUMERS / 2) qidx_pairs<2>(P, T, qi, b, rg, tid);
+    else qidx_pairs<1>(P, T, qi, b, rg, tid);
 }
 
 // B fragment of this lane (column g = lane/4 = head g; k = 2t, 2t+1, 2t+8, 2t+9)

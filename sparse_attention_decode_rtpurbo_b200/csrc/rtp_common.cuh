@@ -63,6 +63,25 @@ struct Sync {
     uint32_t pad[16];
 };
 
+// Head split (host-derived): retrieval groups (KV heads with >= 1 retrieval
+// head), local groups (KV heads with >= 1 local head), retrieval slots (one
+// per retrieval query head).  The kernels read it with run-time indices, so
+// each CTA copies it to shared memory once (copy_tab) instead of indexing the
+// parameter block on its critical paths.
+struct alignas(16) HeadTab {
+    uint8_t rg_group[MAX_HKV], rg_mask[MAX_HKV], rg_slot0[MAX_HKV], rg_nh[MAX_HKV];
+    uint8_t lg_group[MAX_HKV], lg_mask[MAX_HKV];
+    uint8_t slot_head[MAX_HQ], slot_rg[MAX_HQ];
+};
+static_assert(sizeof(HeadTab) % 16 == 0, "HeadTab copies as 16-byte words");
+
+// the table copied by `n` threads (t = 0 .. n-1) into shared memory
+__device__ __forceinline__ void copy_tab(const HeadTab& src, HeadTab& dst, int t, int n) {
+    const uint4* a = reinterpret_cast<const uint4*>(&src);
+    uint4* d = reinterpret_cast<uint4*>(&dst);
+    for (int i = t; i < (int)(sizeof(HeadTab) / 16); i += n) d[i] = a[i];
+}
+
 struct Params {
     int B, Hq, Hkv, G, Ncap, nblk_cap, words_cap, ntiles_cap, mbps, num_pages, window, sink;
     int n_ret, n_rg, n_lg;
@@ -71,11 +90,7 @@ struct Params {
     const int32_t *seq_lens, *block_table;
     const float* p;
     uint16_t* out;
-    // head split (host-derived): retrieval groups (KV heads with >= 1 retrieval head),
-    // local groups (KV heads with >= 1 local head), retrieval slots (one per retrieval query head)
-    uint8_t rg_group[MAX_HKV], rg_mask[MAX_HKV], rg_slot0[MAX_HKV], rg_nh[MAX_HKV];
-    uint8_t lg_group[MAX_HKV], lg_mask[MAX_HKV];
-    uint8_t slot_head[MAX_HQ], slot_rg[MAX_HQ];
+    HeadTab tab;
     // workspace
     uint32_t* status;
     Sync* sync;

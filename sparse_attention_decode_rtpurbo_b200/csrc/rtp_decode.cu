@@ -323,14 +323,14 @@ extern "C" rtp_status rtp_decode_step(const rtp_dims* dims, const uint16_t* q_pr
     P.block_table = dims->block_table;
     P.p = p;
     P.out = out;
-    memcpy(P.rg_group, pl.rg_group, sizeof(P.rg_group));
-    memcpy(P.rg_mask, pl.rg_mask, sizeof(P.rg_mask));
-    memcpy(P.rg_slot0, pl.rg_slot0, sizeof(P.rg_slot0));
-    memcpy(P.rg_nh, pl.rg_nh, sizeof(P.rg_nh));
-    memcpy(P.lg_group, pl.lg_group, sizeof(P.lg_group));
-    memcpy(P.lg_mask, pl.lg_mask, sizeof(P.lg_mask));
-    memcpy(P.slot_head, pl.slot_head, sizeof(P.slot_head));
-    memcpy(P.slot_rg, pl.slot_rg, sizeof(P.slot_rg));
+    memcpy(P.tab.rg_group, pl.rg_group, sizeof(P.tab.rg_group));
+    memcpy(P.tab.rg_mask, pl.rg_mask, sizeof(P.tab.rg_mask));
+    memcpy(P.tab.rg_slot0, pl.rg_slot0, sizeof(P.tab.rg_slot0));
+    memcpy(P.tab.rg_nh, pl.rg_nh, sizeof(P.tab.rg_nh));
+    memcpy(P.tab.lg_group, pl.lg_group, sizeof(P.tab.lg_group));
+    memcpy(P.tab.lg_mask, pl.lg_mask, sizeof(P.tab.lg_mask));
+    memcpy(P.tab.slot_head, pl.slot_head, sizeof(P.tab.slot_head));
+    memcpy(P.tab.slot_rg, pl.slot_rg, sizeof(P.tab.slot_rg));
     uint8_t* ws = (uint8_t*)dims->workspace;
     P.status = (uint32_t*)(ws + pl.o_status);
     P.sync = (Sync*)(ws + pl.o_sync);

@@ -55,6 +55,7 @@ struct BSmem {
     uint32_t flag, gen, abort, base;
     int kept[MAX_G];
     uint32_t wsum[4];
+    HeadTab tab;
     int pre[2];   // really [max(B * n_rg, 1) + 1]: tiles before group i (radix groups, then all groups)
 };
 
@@ -178,7 +179,7 @@ __device__ __noinline__ void r_pass(const Params& P, BSmem<G>& S, RWalk wk, cons
     ac.init(P, tid == 0);
     const int rp = pass - RP_REF0;
     while (wk.next(P, pre, sg)) {
-        const int nh = P.rg_nh[sg.rg], slot0 = P.rg_slot0[sg.rg];
+        const int nh = S.tab.rg_nh[sg.rg], slot0 = S.tab.rg_slot0[sg.rg];
         const int64_t bs0 = (int64_t)sg.b * P.n_ret + slot0;
         for (int x = tid; x < G * 256; x += CONSUMERS) {
             (&S.hcnt[0][0])[x] = 0;
@@ -414,7 +415,7 @@ __device__ __noinline__ void r_digit(const Params& P, BSmem<G>& S, int b, int sl
                 st.all_ties = (nt == st.n_eq) ? 1u : 0u;
                 st.tie_idx = 0xFFFFFFFFu;
                 st.kstar = st.count_above + nt;
-                const int bh = b * P.Hq + P.slot_head[slot];
+                const int bh = b * P.Hq + S.tab.slot_head[slot];
                 if (P.dbg_tau) P.dbg_tau[bh] = key2f(st.tau_key);
                 if (P.dbg_kstar) P.dbg_kstar[bh] = (int32_t)st.kstar;
                 if (!st.all_ties) atomicOr(&P.sync->any_ties, 1u);
@@ -540,7 +541,7 @@ __device__ __noinline__ void r_local_select(const Params& P, BSmem<G>& S, int b,
         h->all_ties = n_tie == n_eq ? 1u : 0u;
         h->tie_idx = tie_idx;
         h->kstar = count_above + n_tie;
-        const int bh = b * P.Hq + P.slot_head[slot];
+        const int bh = b * P.Hq + S.tab.slot_head[slot];
         if (P.dbg_tau) P.dbg_tau[bh] = key2f(tau);
         if (P.dbg_kstar) P.dbg_kstar[bh] = (int32_t)(count_above + n_tie);
         P.cand_cnt[bs] = 0;
@@ -605,7 +606,7 @@ __device__ __noinline__ void r_tie_locate(const Params& P, BSmem<G>& S, int b, i
 template <int G>
 __device__ __noinline__ void r_blist(const Params& P, BSmem<G>& S, int b, int rg, int tid) {
     const int L = __ldg(P.seq_lens + b);
-    const int g = P.rg_group[rg], nh = P.rg_nh[rg], slot0 = P.rg_slot0[rg];
+    const int g = S.tab.rg_group[rg], nh = S.tab.rg_nh[rg], slot0 = S.tab.rg_slot0[rg];
     const int nblk = (L + BLK - 1) / BLK;
     const int nwords = (nblk + 31) / 32;
     const int bg = b * P.n_rg + rg;
@@ -627,7 +628,7 @@ __device__ __noinline__ void r_blist(const Params& P, BSmem<G>& S, int b, int rg
                 uni |= wh[hh];
                 if (wh[hh]) atomicAdd(&S.kept[hh], __popc(wh[hh]));
                 if (P.dbg_bitmap)
-                    P.dbg_bitmap[((int64_t)b * P.Hq + P.slot_head[slot0 + hh]) * P.words_cap + w] = wh[hh];
+                    P.dbg_bitmap[((int64_t)b * P.Hq + S.tab.slot_head[slot0 + hh]) * P.words_cap + w] = wh[hh];
             }
         }
         const uint32_t c = __popc(uni);
@@ -648,7 +649,7 @@ __device__ __noinline__ void r_blist(const Params& P, BSmem<G>& S, int b, int rg
             uint32_t hm = 0;
 #pragma unroll
             for (int hh = 0; hh < MAX_G; ++hh)
-                if ((wh[hh] >> jb) & 1u) hm |= 1u << (P.slot_head[slot0 + hh] - g * P.G);
+                if ((wh[hh] >> jb) & 1u) hm |= 1u << (S.tab.slot_head[slot0 + hh] - g * P.G);
             list[pos++] = ((uint32_t)(w * 32 + jb) << 8) | hm;
         }
         consumer_sync();
@@ -658,7 +659,7 @@ __device__ __noinline__ void r_blist(const Params& P, BSmem<G>& S, int b, int rg
     if (tid < nh && P.dbg_kept) {
         const int slot = slot0 + tid;
         if (__ldcg(&P.hs[(int64_t)b * P.n_ret + slot].mode) == MODE_RADIX)
-            P.dbg_kept[b * P.Hq + P.slot_head[slot]] = S.kept[tid];
+            P.dbg_kept[b * P.Hq + S.tab.slot_head[slot]] = S.kept[tid];
     }
     if (tid == 0) P.bcount[bg] = S.base;
     consumer_sync();
@@ -687,7 +688,7 @@ __device__ __forceinline__ void r_produce_attn(const KParams& K, BSmem<G>& S, co
     while (t < t1) {
         while (pre[gi + 1] <= t) ++gi;
         const int cnt = pre[gi + 1] - pre[gi];
-        const int b = gi / P.n_rg, rg = gi % P.n_rg, g = P.rg_group[rg];
+        const int b = gi / P.n_rg, rg = gi % P.n_rg, g = S.tab.rg_group[rg];
         const int L = __ldg(P.seq_lens + b);
         const int first = t - pre[gi];
         const int nseg = min(cnt - first, t1 - t);
@@ -766,7 +767,7 @@ __device__ __forceinline__ void r_consume_attn(const KParams& K, BSmem<G>& S, ui
         ++k;
         const RDesc d = S.desc[st];
         if (d.type != 0) break;
-        const int g = P.rg_group[d.rg];
+        const int g = S.tab.rg_group[d.rg];
         if (d.flags & 1) attn.begin(P, d.b, g, lane);
         const uint32_t base = smem_u32(&S.stage[st][0]);
         const bool zeroed = attn.tile(base, base + KV_TILE, warp, lane, d.n0, d.nvalid, d.hmask, false, 0, 0);
@@ -776,7 +777,7 @@ __device__ __forceinline__ void r_consume_attn(const KParams& K, BSmem<G>& S, ui
         if (d.flags & 2) {
             attn.finish(S.X, warp, lane);
             consumer_sync();
-            const uint32_t heads = P.rg_mask[d.rg];
+            const uint32_t heads = S.tab.rg_mask[d.rg];
             const int gi = d.b * P.n_rg + d.rg;
             uint16_t* out0 = P.out + ((int64_t)d.b * P.Hq + g * G) * D;
             if (d.seg_tiles == d.item_tiles) {
@@ -834,6 +835,7 @@ __global__ void __launch_bounds__(THREADS, 2) retrieve_kernel(const __grid_const
         S.gen = 0;
         S.abort = 0;
     }
+    if (tid >= 32) copy_tab(P.tab, S.tab, tid - 32, THREADS - 32);
     // everything below reads the streaming kernel's results: wait for that
     // grid to complete (this launch overlaps only its tail)
     asm volatile("griddepcontrol.wait;" ::: "memory");

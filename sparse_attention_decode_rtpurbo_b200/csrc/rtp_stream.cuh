@@ -37,6 +37,7 @@ struct ASmem {
     int pend_b, pend_rg, pend_L;   // best-token blocks this CTA attends after its share (d_list)
     uint32_t flag;
     int tot_s, tot_l, nact;
+    HeadTab tab;
     int pre[2];   // really [2 * (B + 1)]: tiles before sequence b (score, then local)
 };
 
@@ -177,7 +178,7 @@ __device__ __forceinline__ bool ticket_add(uint32_t* ctr, uint32_t add, uint32_t
 // at once, otherwise its radix heads are registered for the exact select.
 template <int G>
 __device__ __forceinline__ void decide_group(const Params& P, ASmem<G>& S, int b, int rg, int L, float pb, int tid) {
-    const int nh = P.rg_nh[rg], slot0 = P.rg_slot0[rg], g = P.rg_group[rg];
+    const int nh = S.tab.rg_nh[rg], slot0 = S.tab.rg_slot0[rg], g = S.tab.rg_group[rg];
     const int nblk = (L + BLK - 1) / BLK;
     const int nwords = (nblk + 31) / 32;
     {
@@ -263,7 +264,7 @@ __device__ __forceinline__ void decide_group(const Params& P, ASmem<G>& S, int b
             h.n_cand = 0;
         }
         P.hs[(int64_t)b * P.n_ret + slot] = h;
-        const int bh = b * P.Hq + P.slot_head[slot];
+        const int bh = b * P.Hq + S.tab.slot_head[slot];
         if (P.dbg_smax) P.dbg_smax[bh] = smax;
         if (P.dbg_Z) P.dbg_Z[bh] = z;
         if (h.mode != MODE_RADIX) {
@@ -281,7 +282,7 @@ __device__ __forceinline__ void decide_group(const Params& P, ASmem<G>& S, int b
         any_radix |= S.d_mode[hh] == MODE_RADIX;
         if (S.d_mode[hh] == MODE_ALL) {
             any_all = true;
-            all_mask |= 1u << (P.slot_head[slot0 + hh] - g * P.G);
+            all_mask |= 1u << (S.tab.slot_head[slot0 + hh] - g * P.G);
         }
     }
     const int bg = b * P.n_rg + rg;
@@ -313,7 +314,7 @@ __device__ __forceinline__ void decide_group(const Params& P, ASmem<G>& S, int b
                 }
                 if (any_radix) P.bitmap[((int64_t)b * P.n_ret + slot) * P.words_cap + w] = word;
                 if (P.dbg_bitmap && mode != MODE_RADIX)
-                    P.dbg_bitmap[((int64_t)b * P.Hq + P.slot_head[slot]) * P.words_cap + w] = word;
+                    P.dbg_bitmap[((int64_t)b * P.Hq + S.tab.slot_head[slot]) * P.words_cap + w] = word;
             }
         }
     }
@@ -339,7 +340,7 @@ __device__ __forceinline__ void decide_group(const Params& P, ASmem<G>& S, int b
             uint32_t hm = all_mask;
             for (int hh = 0; hh < nh; ++hh)
                 if (S.d_mode[hh] == MODE_TOP1 && (int)(S.d_arg[hh] / BLK) == j)
-                    hm |= 1u << (P.slot_head[slot0 + hh] - g * P.G);
+                    hm |= 1u << (S.tab.slot_head[slot0 + hh] - g * P.G);
             list[j] = ((uint32_t)j << 8) | hm;
         }
         if (tid == 0) {
@@ -351,35 +352,38 @@ __device__ __forceinline__ void decide_group(const Params& P, ASmem<G>& S, int b
         // attended by this CTA after its share (the first such group of the
         // CTA; a later one goes to the retrieval kernel)
         if (tid == 0) {
-            uint32_t lst[MAX_G];
+            // heads' argmax blocks in registers (fixed indices), then the
+            // distinct ones ascending, written straight to their destination
+            int bj_h[MAX_G];
+#pragma unroll
+            for (int hh = 0; hh < MAX_G; ++hh)
+                bj_h[hh] = (hh < nh && S.d_mode[hh] == MODE_TOP1) ? (int)(S.d_arg[hh] / BLK) : 0x7FFFFFFF;
+            const bool defer = S.d_cnt == 0;
+            uint32_t* dst = defer ? S.d_list : list;
             uint32_t cnt = 0;
             int last = -1;
             while (true) {
                 int bj = 0x7FFFFFFF;
-                for (int hh = 0; hh < nh; ++hh)
-                    if (S.d_mode[hh] == MODE_TOP1) {
-                        const int j = (int)(S.d_arg[hh] / BLK);
-                        if (j > last && j < bj) bj = j;
-                    }
+#pragma unroll
+                for (int hh = 0; hh < MAX_G; ++hh)
+                    if (bj_h[hh] > last && bj_h[hh] < bj) bj = bj_h[hh];
                 if (bj == 0x7FFFFFFF) break;
                 uint32_t hm = 0;
-                for (int hh = 0; hh < nh; ++hh)
-                    if (S.d_mode[hh] == MODE_TOP1 && (int)(S.d_arg[hh] / BLK) == bj)
-                        hm |= 1u << (P.slot_head[slot0 + hh] - g * P.G);
-                lst[cnt++] = ((uint32_t)bj << 8) | hm;
+#pragma unroll
+                for (int hh = 0; hh < MAX_G; ++hh)
+                    if (bj_h[hh] == bj) hm |= 1u << (S.tab.slot_head[slot0 + hh] - g * P.G);
+                dst[cnt++] = ((uint32_t)bj << 8) | hm;
                 last = bj;
             }
-            if (S.d_cnt != 0 || cnt == 0) {
-                for (uint32_t e = 0; e < cnt; ++e) list[e] = lst[e];
-                P.bcount[bg] = cnt;
-                if (cnt) atomicAdd(&P.sync->kb_work, 1u);
-            } else {
-                for (uint32_t e = 0; e < cnt; ++e) S.d_list[e] = lst[e];
+            if (defer && cnt != 0) {
                 S.d_cnt = cnt;
                 S.pend_b = b;
                 S.pend_rg = rg;
                 S.pend_L = L;
                 P.bcount[bg] = 0;
+            } else {
+                P.bcount[bg] = cnt;
+                if (cnt) atomicAdd(&P.sync->kb_work, 1u);
             }
         }
     }
@@ -503,7 +507,7 @@ __device__ __forceinline__ void fold_pair(float& m, float& s, float m2, float s2
 template <int G, bool NH4>
 __device__ __forceinline__ void score_split_end(const Params& P, ASmem<G>& S, const ScoreFold& f0, int b, int rg,
                                                 int bucket, int tid) {
-    const int nh = P.rg_nh[rg], slot0 = P.rg_slot0[rg];
+    const int nh = S.tab.rg_nh[rg], slot0 = S.tab.rg_slot0[rg];
     const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
     ScoreFold f = f0;
 #pragma unroll
@@ -580,7 +584,7 @@ __device__ __forceinline__ void a_producer(const KParams& K, ASmem<G>& S, AWalk 
             if (!alive || S.d_cnt == 0) break;
             sg = best_token_seg(S);
         }
-        const int g = sg.type == 0 ? P.rg_group[sg.grp] : (sg.type == 1 ? P.lg_group[sg.grp] : P.rg_group[sg.grp]);
+        const int g = sg.type == 0 ? S.tab.rg_group[sg.grp] : (sg.type == 1 ? S.tab.lg_group[sg.grp] : S.tab.rg_group[sg.grp]);
         const LocalGeom lg = local_geom(P, sg.L);
         for (int i = 0; i < sg.ntiles; ++i, ++k) {
             const int st = (int)(k % NST);
@@ -658,11 +662,11 @@ __device__ __forceinline__ void a_consumers(const KParams& K, ASmem<G>& S, AWalk
         }
         if (sg.type == 0) {
             // ---- index scores of (b, retrieval group): q_idx while the first tile is in flight
-            const int nh = P.rg_nh[sg.grp];
+            const int nh = S.tab.rg_nh[sg.grp];
             const int tag = sg.item_idx;
             if (tag != q_tag) {
                 q_tag = tag;
-                compute_qidx(P, S.qi, sg.b, sg.grp, tid);
+                compute_qidx(P, S.tab, S.qi, sg.b, sg.grp, tid);
                 consumer_sync();
                 qf = make_qfrag(S.qi, nh, lane);
                 consumer_sync();
@@ -685,7 +689,7 @@ __device__ __forceinline__ void a_consumers(const KParams& K, ASmem<G>& S, AWalk
                 first_data = false;
                 const int n0 = (sg.first + i) * SROWS, nvalid = min(SROWS, sg.L - n0);
                 const uint32_t tile = smem_u32(&S.stage[st][0]);
-                float* sbase = P.scores + ((int64_t)sg.b * P.n_ret + P.rg_slot0[sg.grp]) * P.Ncap;
+                float* sbase = P.scores + ((int64_t)sg.b * P.n_ret + S.tab.rg_slot0[sg.grp]) * P.Ncap;
                 if (nvalid == SROWS) {
                     if (nh4) score_tile<true, true>(tile, n0, nvalid, nh, track_min, qf, f, sbase, P.Ncap, warp, lane);
                     else score_tile<false, true>(tile, n0, nvalid, nh, track_min, qf, f, sbase, P.Ncap, warp, lane);
@@ -713,8 +717,8 @@ __device__ __forceinline__ void a_consumers(const KParams& K, ASmem<G>& S, AWalk
             // blocks (type 1), or the best-token blocks this CTA selected for
             // (b, retrieval group) (type 2), through the same code
             const bool local = sg.type == 1;
-            const int g = local ? P.lg_group[sg.grp] : P.rg_group[sg.grp];
-            const uint32_t heads = local ? P.lg_mask[sg.grp] : P.rg_mask[sg.grp];
+            const int g = local ? S.tab.lg_group[sg.grp] : S.tab.rg_group[sg.grp];
+            const uint32_t heads = local ? S.tab.lg_mask[sg.grp] : S.tab.rg_mask[sg.grp];
             const LocalGeom lg = local_geom(P, sg.L);
             attn.begin(P, sg.b, g, lane);
             ac.mark(29);
@@ -804,6 +808,7 @@ __global__ void __launch_bounds__(THREADS, 2) stream_kernel(const __grid_constan
     // the retrieval kernel may be scheduled now; it waits for this grid's
     // completion before it reads anything this grid writes
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    if (tid >= 32) copy_tab(P.tab, S.tab, tid - 32, THREADS - 32);
     // tiles per sequence (score tiles of all retrieval groups, then local
     // tiles of all local groups), prefix-summed by warp 0
     if (tid < 32) {
@@ -847,8 +852,10 @@ __global__ void __launch_bounds__(THREADS, 2) stream_kernel(const __grid_constan
         }
     }
     __syncthreads();
-    // every CTA takes an equal, contiguous share of the tiles: index tiles
-    // of all retrieval groups first, then the local tiles
+    // every CTA takes an equal, contiguous share of the index tiles of all
+    // retrieval groups, then one of the local tiles: the scores (and with
+    // them the selection) finish early, the local heads' streaming after
+    // them covers the decisions' latency
     AWalk wk;
     int nact;
     cta_share((long long)S.tot_s + S.tot_l, wk.t, wk.t1, nact);

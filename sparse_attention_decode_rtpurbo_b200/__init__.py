@@ -41,8 +41,8 @@ TRACE_EVENTS = ["start", "select_done", "local_done", "lists_ready", "retrieval_
 # debug sums (slots 16..): SM cycles of one thread per CTA by category, counts,
 # and the latest %globaltimer of two events
 TRACE_SUMS = ["a_cyc_wait", "a_cyc_score", "a_cyc_attn", "a_n_score", "a_n_attn", "a_cyc_score_begin",
-              "a_first_data", "a_consumers_done", "b_cyc_pass_tile", "b_n_pass_tiles", "b_cyc_pass_wait",
-              "b_cyc_pass_other", "a_cyc_score_end", "a_cyc_local_begin", "a_cyc_local_end"]
+              "a_first_data", "a_consumers_done", "b_cyc_bins", "b_n_pass_tiles", "b_cyc_compact",
+              "b_cyc_mark", "a_cyc_score_end", "a_cyc_local_begin", "a_cyc_local_end"]
 
 
 class RtpDims(ctypes.Structure):

@@ -84,6 +84,7 @@ __device__ __forceinline__ void copy_tab(const HeadTab& src, HeadTab& dst, int t
 
 struct Params {
     int B, Hq, Hkv, G, Ncap, nblk_cap, words_cap, ntiles_cap, mbps, num_pages, window, sink;
+    int sstride;   // row stride of the stored scores: ntiles_cap * SROWS (whole 4 KB tiles)
     int n_ret, n_rg, n_lg;
     const uint16_t *q_pre, *q_rope, *k_idx, *Wq;
     const uint16_t *k_cache_ptr, *v_cache_ptr;   // the caches as plain pointers (the kernels read them through TMA maps)
@@ -101,7 +102,7 @@ struct Params {
     uint32_t* hist_cnt;
     unsigned long long* hist_mass;
     uint32_t* tie_cnt;
-    float* scores;   // [B * n_ret, Ncap] fp32 index scores, written by the streaming kernel, read by the select
+    float* scores;   // [B * n_ret, sstride] fp32 index scores, written by the streaming kernel, read by the select
     uint32_t* cand_cnt;              // [B * n_ret] candidates gathered from the threshold bin
     unsigned long long* cand;        // [B * n_ret, CAND_CAP] (key << 32 | token index)
     uint32_t* bitmap;

@@ -125,7 +125,7 @@ static rtp_status make_plan(const rtp_dims* d, const uint8_t* head_kind, int win
     pl->o_rglist = take(BG * 4);
     pl->o_hs = take(BR * sizeof(HeadState));
     pl->o_tie_cnt = take(BR * pl->ntiles_cap * 4);
-    pl->o_scores = take(BR * (size_t)pl->Ncap * 4);
+    pl->o_scores = take(BR * (size_t)pl->ntiles_cap * SROWS * 4);
     pl->o_cand = take(BR * (size_t)CAND_CAP * 8);
     pl->o_bitmap = take(BR * pl->words_cap * 4);
     pl->o_blist = take(BG * pl->nblk_cap * 4);
@@ -303,6 +303,7 @@ extern "C" rtp_status rtp_decode_step(const rtp_dims* dims, const uint16_t* q_pr
     P.Hkv = pl.Hkv;
     P.G = pl.G;
     P.Ncap = pl.Ncap;
+    P.sstride = pl.ntiles_cap * SROWS;
     P.nblk_cap = pl.nblk_cap;
     P.words_cap = pl.words_cap;
     P.ntiles_cap = pl.ntiles_cap;

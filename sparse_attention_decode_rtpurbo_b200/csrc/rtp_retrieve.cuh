@@ -33,25 +33,62 @@ struct RDesc {
     int32_t c0, nsplits;  // first CTA holding a split of the group, number of splits
 };
 
+// Select state of one radix head as the passes read it.
+struct RHead {
+    uint32_t prefix, tau, tie_idx, bstar, n_cand;
+    float smax, dr, inv_w;
+};
+
+// Per-bin histograms of the select passes in shared memory: a count and the
+// 2^-40 fixed-point mass held as three partial sums, of bits 0-15, 16-31 and
+// 32 up of every token's mass (mass = m[0] + m[1] 2^16 + m[2] 2^32).  All
+// four are 32-bit atomics, which the shared-memory units resolve without
+// retries even when a warp's lanes collide; a partial sum cannot wrap while a
+// bin gathers at most 65536 tokens between flushes.
+template <int G>
+struct RHist {
+    uint32_t cnt[G][256];
+    uint32_t m[3][G][256];
+};
+constexpr int HIST_FLUSH_TOKENS = 65536;
+
+template <int G>
+__device__ __forceinline__ void hist_add(RHist<G>& H, int h, int d, uint32_t n, unsigned long long ms) {
+    atomicAdd(&H.cnt[h][d], n);
+    atomicAdd(&H.m[0][h][d], (uint32_t)(ms & 0xFFFFull));
+    atomicAdd(&H.m[1][h][d], (uint32_t)((ms >> 16) & 0xFFFFull));
+    atomicAdd(&H.m[2][h][d], (uint32_t)(ms >> 32));
+}
+template <int G>
+__device__ __forceinline__ unsigned long long hist_mass(const RHist<G>& H, int h, int d) {
+    return (unsigned long long)H.m[0][h][d] + ((unsigned long long)H.m[1][h][d] << 16) +
+           ((unsigned long long)H.m[2][h][d] << 32);
+}
+
 template <int G>
 struct BSmem {
     static constexpr int NST = 2;
     alignas(1024) uint8_t stage[NST][STAGE_BYTES];
-    AttnScratch<G> X;
+    union {
+        AttnScratch<G> X;   // attention phase
+        RHist<G> H;         // select phase
+    };
     alignas(16) float qi[MAX_G][R];
-    uint32_t hcnt[G][256];
-    unsigned long long hmass[G][256];   // per-bin count and 2^-40 fixed-point mass
     unsigned long long dmass[256];
     uint32_t dcnt[256];
     uint32_t tmask[MAX_G];
     uint32_t tcnt[MAX_G];
     uint8_t rlist_h[MAX_G];
+    uint32_t want_mask;   // bit hx: this pass processes radix head rlist_h[hx]
+    RHead rhs[MAX_G];   // select state of the segment's radix heads (r_pass)
     uint32_t nrad_h;
     uint32_t lsel_prefix, lsel_count, lsel_neq;
     unsigned long long lsel_mass, lsel_meq;
     uint8_t tflag[SROWS];
     RDesc desc[NST];
     alignas(8) uint64_t full[NST], empty[NST];
+    alignas(8) uint64_t res_bar;   // the resident score tiles have landed
+    uint32_t resident;             // this CTA's score tiles sit in the stage buffers
     uint32_t flag, gen, abort, base;
     int kept[MAX_G];
     uint32_t wsum[4];
@@ -62,6 +99,17 @@ struct BSmem {
 template <int G>
 constexpr size_t bsmem_bytes(int ngroups) {
     return sizeof(BSmem<G>) + sizeof(int) * (size_t)(ngroups + 1) + 1024;
+}
+
+// The CTA's BSmem, 1024-byte aligned inside the dynamic shared memory.  It is
+// derived by offset arithmetic on the shared array, so the compiler keeps it
+// in the shared state space (native shared loads, stores and atomics) also in
+// the helpers that are not inlined.
+template <int G>
+__device__ __forceinline__ BSmem<G>& bsmem() {
+    extern __shared__ uint8_t rtp_dyn_smem[];
+    const uint32_t pad = (1024u - (smem_u32(rtp_dyn_smem) & 1023u)) & 1023u;
+    return *reinterpret_cast<BSmem<G>*>(rtp_dyn_smem + pad);
 }
 
 __device__ __forceinline__ bool wait_counter(const uint32_t* p, uint32_t target) {
@@ -122,12 +170,6 @@ struct RWalk {
     }
 };
 
-// Per-thread view of the select state of one head.
-struct RHead {
-    uint32_t prefix, tau, tie_idx, bstar, n_cand;
-    float smax, dr, inv_w;
-};
-
 __device__ __forceinline__ RHead load_rhead(const HeadState* h) {
     RHead r;
     r.prefix = __ldcg(&h->prefix);
@@ -158,11 +200,11 @@ __device__ __forceinline__ uint32_t score_bin(float s, float smax, float dr, flo
 enum RPass : int { RP_BINS = 0, RP_REF0, RP_REF1, RP_REF2, RP_REF3, RP_TIES, RP_MARK, RP_COMPACT };
 
 template <int G>
-__device__ __noinline__ void r_digit(const Params& P, BSmem<G>& S, int b, int slot, int pass, int tid);
+__device__ __noinline__ void r_digit(const Params& P, int b, int slot, int pass, int tid);
 template <int G>
-__device__ __noinline__ void r_tie_locate(const Params& P, BSmem<G>& S, int b, int slot, int tid);
+__device__ __noinline__ void r_tie_locate(const Params& P, int b, int slot, int tid);
 template <int G>
-__device__ __noinline__ void r_blist(const Params& P, BSmem<G>& S, int b, int rg, int tid);
+__device__ __noinline__ void r_blist(const Params& P, int b, int rg, int tid);
 
 // One pass over the stored scores of this CTA's share of the radix groups'
 // 1024-token tiles (consumer threads; thread tid takes tokens n0 + tid + 128 u
@@ -170,147 +212,196 @@ __device__ __noinline__ void r_blist(const Params& P, BSmem<G>& S, int b, int rg
 // group's tiles the CTA folds its histograms into the heads' global ones;
 // per-head tickets elect the CTA that takes the head's next step (its digit,
 // its tie position, or, for the marks, the group's block list).
-template <int G>
-__device__ __noinline__ void r_pass(const Params& P, BSmem<G>& S, RWalk wk, const int* pre, int pass, int tid) {
+template <int G, int pass>
+__device__ __noinline__ void r_pass(const Params& P, RWalk wk, const int* pre, int tid) {
+    BSmem<G>& S = bsmem<G>();
     constexpr int U = SROWS / CONSUMERS;
     const int lane = tid & 31;
     RSeg sg;
     Acct ac;
     ac.init(P, tid == 0);
     const int rp = pass - RP_REF0;
+    const bool resident = S.resident != 0;
+    if (resident && !mbar_wait_bounded(&S.res_bar, 0u)) set_status(P, ST_TIMEOUT);
+    int sbase = 0;
     while (wk.next(P, pre, sg)) {
         const int nh = S.tab.rg_nh[sg.rg], slot0 = S.tab.rg_slot0[sg.rg];
         const int64_t bs0 = (int64_t)sg.b * P.n_ret + slot0;
-        for (int x = tid; x < G * 256; x += CONSUMERS) {
-            (&S.hcnt[0][0])[x] = 0;
-            (&S.hmass[0][0])[x] = 0ull;
-        }
+        for (int x = tid; x < 4 * G * 256; x += CONSUMERS) (&S.H.cnt[0][0])[x] = 0;
         if (tid < MAX_G) {
             S.tmask[tid] = 0;
             S.tcnt[tid] = 0;
         }
-        // the group's radix heads, then a flat loop over (tile, head) items
-        // with the next item's scores loaded while this one is processed
+        // the group's radix heads (then their select state, once per run),
+        // then a flat loop over (tile, head) items
         if (tid == 0) {
-            uint32_t n = 0;
+            uint32_t n = 0, wm = 0;
             for (int hh = 0; hh < nh; ++hh) {
                 const HeadState* h = P.hs + bs0 + hh;
                 if (__ldcg(&h->mode) != MODE_RADIX) continue;
                 const bool local = __ldcg(&h->n_cand) <= (uint32_t)CAND_CAP;
                 const bool want = (pass == RP_BINS || pass == RP_MARK) ? true : (pass == RP_COMPACT ? local : !local);
-                if (want) S.rlist_h[n++] = (uint8_t)hh;
+                if (want) wm |= 1u << n;
+                S.rlist_h[n++] = (uint8_t)hh;
             }
             S.nrad_h = n;
+            S.want_mask = wm;
         }
         consumer_sync();
         const int nr = (int)S.nrad_h;
+        const uint32_t wantm = S.want_mask;
+        if (tid < nr) S.rhs[tid] = load_rhead(P.hs + bs0 + S.rlist_h[tid]);
         const int nitems = sg.ntiles * nr;
+        // this CTA's histograms -> the heads' global ones (at the end of the
+        // run, and every 64 tiles so that no partial sum can wrap)
+        auto flush = [&]() {
+            consumer_sync();
+            for (int x = tid; x < nh * 256; x += CONSUMERS) {
+                const int hh = x >> 8, d = x & 255;
+                const uint32_t c = S.H.cnt[hh][d];
+                if (c) {
+                    atomicAdd(P.hist_cnt + (bs0 + hh) * 256 + d, c);
+                    atomicAdd(P.hist_mass + (bs0 + hh) * 256 + d, hist_mass(S.H, hh, d));
+                    S.H.cnt[hh][d] = 0;
+                    S.H.m[0][hh][d] = 0;
+                    S.H.m[1][hh][d] = 0;
+                    S.H.m[2][hh][d] = 0;
+                }
+            }
+            consumer_sync();
+        };
+        // items of every radix head in (tile, head) order: resident ones from
+        // the stage buffers (slot sbase + it), else from the stored scores
+        const float* res = reinterpret_cast<const float*>(&S.stage[0][0]) + (size_t)sbase * SROWS;
         float vn[U];
-        auto load_item = [&](int it, float* dst) {
-            const int tile = sg.first + it / nr, hh = S.rlist_h[it % nr];
+        auto load_item = [&](int it, int tile, int hx, float* dst) {
+            const int hh = S.rlist_h[hx];
             const int n0 = tile * SROWS, nvalid = min(SROWS, sg.L - n0);
-            const float* src = P.scores + (bs0 + hh) * P.Ncap + n0;
+            const float* src = resident ? res + (size_t)it * SROWS : P.scores + (bs0 + hh) * P.sstride + n0;
 #pragma unroll
             for (int u = 0; u < U; ++u) {
                 const int r = tid + u * CONSUMERS;
-                dst[u] = r < nvalid ? __ldcg(src + r) : 0.f;
+                dst[u] = r < nvalid ? (resident ? src[r] : __ldcg(src + r)) : 0.f;
             }
         };
-        if (nitems > 0) load_item(0, vn);
+        if (nitems > 0) load_item(0, sg.first, 0, vn);
+        consumer_sync();   // S.rhs
         uint32_t ovf_n = 0u;
         unsigned long long ovf_m = 0ull;
         int cur_h = -1;
-        RHead rh;
+        // item it = (tile, head hx), walked without divisions
+        int tile = sg.first - 1, hx = nr - 1;
 #pragma unroll 1
         for (int it = 0; it < nitems; ++it) {
+            if (++hx == nr) {
+                hx = 0;
+                ++tile;
+            }
             float v[U];
 #pragma unroll
             for (int u = 0; u < U; ++u) v[u] = vn[u];
-            if (it + 1 < nitems) load_item(it + 1, vn);
-            const int tile = sg.first + it / nr, hh = S.rlist_h[it % nr];
-            const int n0 = tile * SROWS, nvalid = min(SROWS, sg.L - n0);
-            if (hh != cur_h) {
-                if (pass == RP_BINS && cur_h >= 0) {
-                    // out-of-range sums of the previous head
-#pragma unroll
-                    for (int o = 16; o > 0; o >>= 1) {
-                        ovf_n += __shfl_xor_sync(0xffffffffu, ovf_n, o);
-                        ovf_m += __shfl_xor_sync(0xffffffffu, ovf_m, o);
-                    }
-                    if (lane == 0 && ovf_n) {
-                        atomicAdd(&S.hcnt[cur_h][255], ovf_n);
-                        atomicAdd(&S.hmass[cur_h][255], ovf_m);
-                    }
-                    ovf_n = 0u;
-                    ovf_m = 0ull;
-                }
-                cur_h = hh;
-                rh = load_rhead(P.hs + bs0 + hh);
+            if (it + 1 < nitems) {
+                if (hx + 1 == nr) load_item(it + 1, tile + 1, 0, vn);
+                else load_item(it + 1, tile, hx + 1, vn);
             }
+            const int hh = S.rlist_h[hx];
+            const int n0 = tile * SROWS, nvalid = min(SROWS, sg.L - n0);
+            if (pass <= RP_REF3 && hx == 0 && tile > sg.first && ((tile - sg.first) & (HIST_FLUSH_TOKENS / SROWS - 1)) == 0) {
+                // every 64 tiles: no partial sum can wrap (the overflow bin's
+                // register sums join at the head's next switch)
+                flush();
+            }
+            if (!((wantm >> hx) & 1u)) continue;   // (uniform over the CTA)
+            if (pass == RP_BINS && hh != cur_h && cur_h >= 0) {
+                // out-of-range sums of the previous head
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    ovf_n += __shfl_xor_sync(0xffffffffu, ovf_n, o);
+                    ovf_m += __shfl_xor_sync(0xffffffffu, ovf_m, o);
+                }
+                if (lane == 0 && ovf_n) hist_add(S.H, cur_h, 255, ovf_n, ovf_m);
+                ovf_n = 0u;
+                ovf_m = 0ull;
+            }
+            cur_h = hh;
+            const RHead rh = S.rhs[hx];
             uint32_t bits = 0u, cnt = 0u;
+            uint32_t bal[U];
 #pragma unroll
             for (int u = 0; u < U; ++u) {
                 const int r = tid + u * CONSUMERS;
                 const bool ok = r < nvalid;
                 const uint32_t key = f2key(v[u]);
-                if (pass == RP_BINS) {
+                if constexpr (pass == RP_BINS) {
                     if (ok) {
                         const uint32_t bn = score_bin(v[u], rh.smax, rh.dr, rh.inv_w);
                         const unsigned long long ms = fixmass(key, rh.smax);
                         if (bn < 255u) {
-                            atomicAdd(&S.hcnt[hh][bn], 1u);
-                            atomicAdd(&S.hmass[hh][bn], ms);
+                            hist_add(S.H, hh, (int)bn, 1u, ms);
                         } else {
                             ovf_n += 1u;
                             ovf_m += ms;
                         }
                     }
-                } else if (pass <= RP_REF3) {
+                } else if constexpr (pass <= RP_REF3) {
                     if (ok && score_bin(v[u], rh.smax, rh.dr, rh.inv_w) == rh.bstar &&
                         (rp == 0 || (key >> (32 - 8 * rp)) == rh.prefix)) {
                         const uint32_t d = (key >> (24 - 8 * rp)) & 255u;
-                        atomicAdd(&S.hcnt[hh][d], 1u);
-                        atomicAdd(&S.hmass[hh][d], fixmass(key, rh.smax));
+                        hist_add(S.H, hh, (int)d, 1u, fixmass(key, rh.smax));
                     }
-                } else if (pass == RP_TIES) {
+                } else if constexpr (pass == RP_TIES) {
                     cnt += (ok && key == rh.tau) ? 1u : 0u;
-                } else if (pass == RP_COMPACT) {
+                } else if constexpr (pass == RP_COMPACT) {
+                    // ballots only: the warp's candidates of the item go out below
                     const bool in = ok && score_bin(v[u], rh.smax, rh.dr, rh.inv_w) == rh.bstar;
-                    const uint32_t bal = __ballot_sync(0xffffffffu, in);
-                    if (bal) {
-                        uint32_t base = 0;
-                        if (lane == 0) base = atomicAdd(P.cand_cnt + bs0 + hh, (uint32_t)__popc(bal));
-                        base = __shfl_sync(0xffffffffu, base, 0);
-                        if (in) {
-                            const uint32_t pos = base + __popc(bal & ((1u << lane) - 1u));
-                            if (pos < (uint32_t)CAND_CAP)
-                                P.cand[(bs0 + hh) * CAND_CAP + pos] = ((unsigned long long)key << 32) | (uint32_t)(n0 + r);
-                        }
-                    }
+                    bal[u] = __ballot_sync(0xffffffffu, in);
                 } else {
                     const bool keep = ok && (key > rh.tau || (key == rh.tau && (uint32_t)(n0 + r) <= rh.tie_idx));
                     // a warp's 32 tokens lie in one 64-token block: one vote per warp
                     if (__any_sync(0xffffffffu, keep) && lane == 0) bits |= 1u << ((r / BLK) & 15);
                 }
             }
-            if (pass == RP_TIES || pass == RP_MARK) {
+            if constexpr (pass == RP_COMPACT) {
+                // one reservation per warp and item, then the candidates in
+                // ballot order
+                uint32_t tot = 0;
+#pragma unroll
+                for (int u = 0; u < U; ++u) tot += __popc(bal[u]);
+                if (tot) {
+                    uint32_t base = 0;
+                    if (lane == 0) base = atomicAdd(P.cand_cnt + bs0 + hh, tot);
+                    base = __shfl_sync(0xffffffffu, base, 0);
+#pragma unroll
+                    for (int u = 0; u < U; ++u) {
+                        if ((bal[u] >> lane) & 1u) {
+                            const uint32_t pos = base + __popc(bal[u] & ((1u << lane) - 1u));
+                            if (pos < (uint32_t)CAND_CAP) {
+                                const int r = tid + u * CONSUMERS;
+                                P.cand[(bs0 + hh) * CAND_CAP + pos] =
+                                    ((unsigned long long)f2key(v[u]) << 32) | (uint32_t)(n0 + r);
+                            }
+                        }
+                        base += __popc(bal[u]);
+                    }
+                }
+            }
+            if constexpr (pass == RP_MARK) {
+                // the warp's blocks straight into the head's bitmap (zeroed
+                // when the group was registered for the select)
+                if (lane == 0 && bits)
+                    atomicOr(P.bitmap + (bs0 + hh) * P.words_cap + tile / 2, bits << ((tile & 1) * 16));
+            } else if constexpr (pass == RP_TIES) {
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
-                if (lane == 0) {
-                    if (cnt) atomicAdd(&S.tcnt[hh], cnt);
-                    if (bits) atomicOr(&S.tmask[hh], bits);
-                }
+                if (lane == 0 && cnt) atomicAdd(&S.tcnt[hh], cnt);
                 consumer_sync();
                 if (tid == 0) {
-                    const int64_t bs = bs0 + hh;
-                    if (pass == RP_TIES) P.tie_cnt[bs * P.ntiles_cap + tile] = S.tcnt[hh];
-                    else if (S.tmask[hh]) atomicOr(P.bitmap + bs * P.words_cap + tile / 2, S.tmask[hh] << ((tile & 1) * 16));
-                    S.tmask[hh] = 0;
+                    P.tie_cnt[(bs0 + hh) * P.ntiles_cap + tile] = S.tcnt[hh];
                     S.tcnt[hh] = 0;
                 }
                 consumer_sync();
             }
-            ac.mark(24);
+            ac.mark(pass == RP_COMPACT ? 26 : (pass == RP_MARK ? 27 : 24));
             ac.count(25);
         }
         if (pass == RP_BINS && cur_h >= 0) {
@@ -319,24 +410,52 @@ __device__ __noinline__ void r_pass(const Params& P, BSmem<G>& S, RWalk wk, cons
                 ovf_n += __shfl_xor_sync(0xffffffffu, ovf_n, o);
                 ovf_m += __shfl_xor_sync(0xffffffffu, ovf_m, o);
             }
-            if (lane == 0 && ovf_n) {
-                atomicAdd(&S.hcnt[cur_h][255], ovf_n);
-                atomicAdd(&S.hmass[cur_h][255], ovf_m);
-            }
+            if (lane == 0 && ovf_n) hist_add(S.H, cur_h, 255, ovf_n, ovf_m);
         }
-        if (pass <= RP_REF3) {
-            // this run's histograms -> the heads' global histograms
-            consumer_sync();
-            for (int x = tid; x < nh * 256; x += CONSUMERS) {
-                const int hh = x >> 8, d = x & 255;
-                const uint32_t c = S.hcnt[hh][d];
-                if (c) {
-                    atomicAdd(P.hist_cnt + (bs0 + hh) * 256 + d, c);
-                    atomicAdd(P.hist_mass + (bs0 + hh) * 256 + d, S.hmass[hh][d]);
-                }
-            }
-        }
+        if constexpr (pass <= RP_REF3) flush();
         consumer_sync();
+        sbase += nitems;
+    }
+}
+
+// The copy warp at the start of the select: when this CTA's share of score
+// items (every radix head of its tiles) fits the two stage buffers, all of
+// them are copied there at once (one 4 KB bulk copy per item, in the order
+// the passes walk them) and every pass then reads shared memory only.
+constexpr int RES_ITEMS = 2 * STAGE_BYTES / (SROWS * 4);
+template <int G>
+__device__ __noinline__ void r_load_scores(const Params& P, RWalk wk, const int* pre, int lane) {
+    BSmem<G>& S = bsmem<G>();
+    if (lane != 0) return;
+    int items = 0;
+    {
+        RWalk w2 = wk;
+        RSeg sg;
+        while (w2.next(P, pre, sg)) {
+            const int nh = S.tab.rg_nh[sg.rg], slot0 = S.tab.rg_slot0[sg.rg];
+            int nr = 0;
+            for (int hh = 0; hh < nh; ++hh)
+                nr += __ldcg(&P.hs[(int64_t)sg.b * P.n_ret + slot0 + hh].mode) == MODE_RADIX;
+            items += sg.ntiles * nr;
+        }
+    }
+    if (items == 0 || items > RES_ITEMS) {
+        S.resident = 0;
+        return;
+    }
+    S.resident = 1;
+    mbar_expect_tx(&S.res_bar, (uint32_t)items * SROWS * 4);
+    uint8_t* dst = &S.stage[0][0];
+    RSeg sg;
+    while (wk.next(P, pre, sg)) {
+        const int nh = S.tab.rg_nh[sg.rg], slot0 = S.tab.rg_slot0[sg.rg];
+        const int64_t bs0 = (int64_t)sg.b * P.n_ret + slot0;
+        for (int t = 0; t < sg.ntiles; ++t)
+            for (int hh = 0; hh < nh; ++hh) {
+                if (__ldcg(&P.hs[bs0 + hh].mode) != MODE_RADIX) continue;
+                bulk_g2s(dst, P.scores + (bs0 + hh) * P.sstride + (int64_t)(sg.first + t) * SROWS, SROWS * 4, &S.res_bar);
+                dst += SROWS * 4;
+            }
     }
 }
 
@@ -346,7 +465,8 @@ __device__ __noinline__ void r_pass(const Params& P, BSmem<G>& S, RWalk wk, cons
 // Pick the digit of pass `pass` for radix head `hx`: the largest digit d whose
 // bins >= d hold at least the target mass (over the tokens above the prefix).
 template <int G>
-__device__ __noinline__ void r_digit(const Params& P, BSmem<G>& S, int b, int slot, int pass, int tid) {
+__device__ __noinline__ void r_digit(const Params& P, int b, int slot, int pass, int tid) {
+    BSmem<G>& S = bsmem<G>();
     const int64_t bs = (int64_t)b * P.n_ret + slot;
     uint32_t* gcnt = P.hist_cnt + bs * 256;
     unsigned long long* gmass = P.hist_mass + bs * 256;
@@ -434,38 +554,66 @@ __device__ __noinline__ void r_digit(const Params& P, BSmem<G>& S, int b, int sl
 // over the tie indices gives the largest tie index kept (ties toward the
 // lower index).
 template <int G>
-__device__ __noinline__ void r_local_select(const Params& P, BSmem<G>& S, int b, int slot, int tid) {
+__device__ __noinline__ void r_local_select(const Params& P, int b, int slot, int tid) {
+    BSmem<G>& S = bsmem<G>();
+    constexpr int CPT = CAND_CAP / CONSUMERS;   // candidates per thread, kept in registers
     const int64_t bs = (int64_t)b * P.n_ret + slot;
     const uint32_t ncand = __ldcg(&P.hs[bs].n_cand);
     if (ncand > (uint32_t)CAND_CAP) return;
-    uint32_t* keys = reinterpret_cast<uint32_t*>(&S.stage[0][0]);
-    uint32_t* idx = keys + CAND_CAP;
     const int n = (int)ncand;
-    for (int i = tid; i < n; i += CONSUMERS) {
-        const unsigned long long c = __ldcg(P.cand + bs * CAND_CAP + i);
-        keys[i] = (uint32_t)(c >> 32);
-        idx[i] = (uint32_t)(c & 0xFFFFFFFFull);
+    uint32_t keys[CPT], idx[CPT];
+#pragma unroll
+    for (int j = 0; j < CPT; ++j) {
+        const int i = tid + j * CONSUMERS;
+        keys[j] = 0u;
+        idx[j] = 0u;
+        if (i < n) {
+            const unsigned long long c = __ldcg(P.cand + bs * CAND_CAP + i);
+            keys[j] = (uint32_t)(c >> 32);
+            idx[j] = (uint32_t)(c & 0xFFFFFFFFull);
+        }
     }
+    // the leading digits every candidate shares (one threshold bin: often
+    // one or two) need no pass
+    uint32_t kand = 0xFFFFFFFFu, kor = 0u;
+#pragma unroll
+    for (int j = 0; j < CPT; ++j)
+        if (tid + j * CONSUMERS < n) {
+            kand &= keys[j];
+            kor |= keys[j];
+        }
+    kand = __reduce_and_sync(0xffffffffu, kand);
+    kor = __reduce_or_sync(0xffffffffu, kor);
+    if ((tid & 31) == 0) {
+        S.wsum[tid >> 5] = kand;
+        S.tcnt[tid >> 5] = kor;
+    }
+    consumer_sync();
+    kand = S.wsum[0] & S.wsum[1] & S.wsum[2] & S.wsum[3];
+    kor = S.tcnt[0] | S.tcnt[1] | S.tcnt[2] | S.tcnt[3];
+    const int rp0 = n > 0 ? min(__clz(kand ^ kor) / 8, 3) : 0;
     const float smax = __ldcg(&P.hs[bs].smax);
+    consumer_sync();
     if (tid == 0) {
-        S.lsel_prefix = 0;
+        S.lsel_prefix = rp0 > 0 ? kand >> (32 - 8 * rp0) : 0u;
         S.lsel_mass = __ldcg(&P.hs[bs].mass_above);
         S.lsel_count = __ldcg(&P.hs[bs].count_above);
     }
     const unsigned long long target = __ldcg(&P.hs[bs].target);
-    for (int rp = 0; rp < 4; ++rp) {
+    for (int rp = rp0; rp < 4; ++rp) {
         for (int d = tid; d < 256; d += CONSUMERS) {
-            S.hcnt[0][d] = 0;
-            S.hmass[0][d] = 0ull;
+            S.H.cnt[0][d] = 0;
+            S.H.m[0][0][d] = 0;
+            S.H.m[1][0][d] = 0;
+            S.H.m[2][0][d] = 0;
         }
         consumer_sync();
         const uint32_t prefix = S.lsel_prefix;
-        for (int i = tid; i < n; i += CONSUMERS) {
-            const uint32_t key = keys[i];
-            if (rp > 0 && (key >> (32 - 8 * rp)) != prefix) continue;
-            const uint32_t d = (key >> (24 - 8 * rp)) & 255u;
-            atomicAdd(&S.hcnt[0][d], 1u);
-            atomicAdd(&S.hmass[0][d], fixmass(key, smax));
+#pragma unroll
+        for (int j = 0; j < CPT; ++j) {
+            const uint32_t key = keys[j];
+            if (tid + j * CONSUMERS >= n || (rp > 0 && (key >> (32 - 8 * rp)) != prefix)) continue;
+            hist_add(S.H, 0, (int)((key >> (24 - 8 * rp)) & 255u), 1u, fixmass(key, smax));
         }
         consumer_sync();
         if (tid == 0) {
@@ -473,18 +621,19 @@ __device__ __noinline__ void r_local_select(const Params& P, BSmem<G>& S, int b,
             uint32_t cabove = S.lsel_count;
             int dstar = 0;
             for (int d = 255; d >= 0; --d) {
-                if (cum + S.hmass[0][d] >= target) {
+                const unsigned long long md = hist_mass(S.H, 0, d);
+                if (cum + md >= target) {
                     dstar = d;
                     break;
                 }
-                cum += S.hmass[0][d];
-                cabove += S.hcnt[0][d];
+                cum += md;
+                cabove += S.H.cnt[0][d];
             }
             S.lsel_mass = cum;
             S.lsel_count = cabove;
             S.lsel_prefix = (prefix << 8) | (uint32_t)dstar;
-            S.lsel_neq = S.hcnt[0][dstar];
-            S.lsel_meq = S.hmass[0][dstar];
+            S.lsel_neq = S.H.cnt[0][dstar];
+            S.lsel_meq = hist_mass(S.H, 0, dstar);
         }
         consumer_sync();
     }
@@ -506,25 +655,26 @@ __device__ __noinline__ void r_local_select(const Params& P, BSmem<G>& S, int b,
             S.lsel_count = n_tie;   // rank still wanted
         }
         for (int rp = 0; rp < 4; ++rp) {
-            for (int d = tid; d < 256; d += CONSUMERS) S.hcnt[0][d] = 0;
+            for (int d = tid; d < 256; d += CONSUMERS) S.H.cnt[0][d] = 0;
             consumer_sync();
             const uint32_t prefix = S.lsel_prefix;
-            for (int i = tid; i < n; i += CONSUMERS) {
-                if (keys[i] != tau) continue;
-                const uint32_t x = idx[i];
+#pragma unroll
+            for (int j = 0; j < CPT; ++j) {
+                if (tid + j * CONSUMERS >= n || keys[j] != tau) continue;
+                const uint32_t x = idx[j];
                 if (rp > 0 && (x >> (32 - 8 * rp)) != prefix) continue;
-                atomicAdd(&S.hcnt[0][(x >> (24 - 8 * rp)) & 255u], 1u);
+                atomicAdd(&S.H.cnt[0][(x >> (24 - 8 * rp)) & 255u], 1u);
             }
             consumer_sync();
             if (tid == 0) {
                 uint32_t rank = S.lsel_count, cum = 0;
                 int dstar = 255;
                 for (int d = 0; d < 256; ++d) {
-                    if (cum + S.hcnt[0][d] >= rank) {
+                    if (cum + S.H.cnt[0][d] >= rank) {
                         dstar = d;
                         break;
                     }
-                    cum += S.hcnt[0][d];
+                    cum += S.H.cnt[0][d];
                 }
                 S.lsel_count = rank - cum;
                 S.lsel_prefix = (prefix << 8) | (uint32_t)dstar;
@@ -553,7 +703,8 @@ __device__ __noinline__ void r_local_select(const Params& P, BSmem<G>& S, int b,
 // index of the n_tie-th tie in token order (per-tile counts, then a scan of
 // the stored scores of the one tile that holds it).
 template <int G>
-__device__ __noinline__ void r_tie_locate(const Params& P, BSmem<G>& S, int b, int slot, int tid) {
+__device__ __noinline__ void r_tie_locate(const Params& P, int b, int slot, int tid) {
+    BSmem<G>& S = bsmem<G>();
     const int64_t bs = (int64_t)b * P.n_ret + slot;
     if (__ldcg(&P.hs[bs].all_ties)) return;
     const int L = __ldg(P.seq_lens + b);
@@ -577,7 +728,7 @@ __device__ __noinline__ void r_tie_locate(const Params& P, BSmem<G>& S, int b, i
     const int tile = (int)S.base;
     const uint32_t rank = S.flag;
     const int n0 = tile * SROWS, nvalid = min(SROWS, L - n0);
-    const float* sc = P.scores + bs * P.Ncap + n0;
+    const float* sc = P.scores + bs * P.sstride + n0;
     for (int r = tid; r < SROWS; r += CONSUMERS) S.tflag[r] = (r < nvalid && f2key(__ldcg(sc + r)) == tau) ? 1 : 0;
     consumer_sync();
     const int warp = tid >> 5, lane = tid & 31;
@@ -604,7 +755,8 @@ __device__ __noinline__ void r_tie_locate(const Params& P, BSmem<G>& S, int b, i
 // Block list of radix group i: union of its heads' block bitmaps, in
 // ascending block order, with the mask of heads that read each block.
 template <int G>
-__device__ __noinline__ void r_blist(const Params& P, BSmem<G>& S, int b, int rg, int tid) {
+__device__ __noinline__ void r_blist(const Params& P, int b, int rg, int tid) {
+    BSmem<G>& S = bsmem<G>();
     const int L = __ldg(P.seq_lens + b);
     const int g = S.tab.rg_group[rg], nh = S.tab.rg_nh[rg], slot0 = S.tab.rg_slot0[rg];
     const int nblk = (L + BLK - 1) / BLK;
@@ -615,22 +767,26 @@ __device__ __noinline__ void r_blist(const Params& P, BSmem<G>& S, int b, int rg
     if (tid < MAX_G) S.kept[tid] = 0;
     if (tid == 0) S.base = 0;
     consumer_sync();
-    for (int w0 = 0; w0 < nwords; w0 += CONSUMERS) {
-        const int w = w0 + tid;
+    // thread tid takes 16 consecutive blocks (half a bitmap word) per round
+    const int nhalf = (nblk + 15) / 16;
+    for (int h0 = 0; h0 < nhalf; h0 += CONSUMERS) {
+        const int hw = h0 + tid, w = hw >> 1;
         uint32_t uni = 0;
-        uint32_t wh[MAX_G];
+        uint32_t hb[MAX_G];
 #pragma unroll
         for (int hh = 0; hh < MAX_G; ++hh) {
-            wh[hh] = 0;
-            if (hh < nh && w < nwords) {
-                wh[hh] = __ldcg(P.bitmap + ((int64_t)b * P.n_ret + slot0 + hh) * P.words_cap + w);
-                if (w == nwords - 1 && (nblk & 31)) wh[hh] &= (1u << (nblk & 31)) - 1u;
-                uni |= wh[hh];
-                if (wh[hh]) atomicAdd(&S.kept[hh], __popc(wh[hh]));
-                if (P.dbg_bitmap)
-                    P.dbg_bitmap[((int64_t)b * P.Hq + S.tab.slot_head[slot0 + hh]) * P.words_cap + w] = wh[hh];
+            hb[hh] = 0;
+            if (hh < nh && hw < nhalf) {
+                uint32_t word = __ldcg(P.bitmap + ((int64_t)b * P.n_ret + slot0 + hh) * P.words_cap + w);
+                if (w == nwords - 1 && (nblk & 31)) word &= (1u << (nblk & 31)) - 1u;
+                if (P.dbg_bitmap && (hw & 1) == 0)
+                    P.dbg_bitmap[((int64_t)b * P.Hq + S.tab.slot_head[slot0 + hh]) * P.words_cap + w] = word;
+                hb[hh] = (word >> ((hw & 1) * 16)) & 0xFFFFu;
+                uni |= hb[hh];
+                if (hb[hh]) atomicAdd(&S.kept[hh], __popc(hb[hh]));
             }
         }
+        // exclusive scan of the per-thread counts over the CTA
         const uint32_t c = __popc(uni);
         uint32_t incl = c;
 #pragma unroll
@@ -649,8 +805,8 @@ __device__ __noinline__ void r_blist(const Params& P, BSmem<G>& S, int b, int rg
             uint32_t hm = 0;
 #pragma unroll
             for (int hh = 0; hh < MAX_G; ++hh)
-                if ((wh[hh] >> jb) & 1u) hm |= 1u << (S.tab.slot_head[slot0 + hh] - g * P.G);
-            list[pos++] = ((uint32_t)(w * 32 + jb) << 8) | hm;
+                if ((hb[hh] >> jb) & 1u) hm |= 1u << (S.tab.slot_head[slot0 + hh] - g * P.G);
+            list[pos++] = ((uint32_t)(hw * 16 + jb) << 8) | hm;
         }
         consumer_sync();
         if (tid == 0) S.base += S.wsum[0] + S.wsum[1] + S.wsum[2] + S.wsum[3];
@@ -819,8 +975,7 @@ __device__ __forceinline__ void warp_prefix(int* pre, int n, F cnt, int lane) {
 // ---------------------------------------------------------------------------
 template <int G>
 __global__ void __launch_bounds__(THREADS, 2) retrieve_kernel(const __grid_constant__ KParams K) {
-    extern __shared__ uint8_t smem_raw[];
-    BSmem<G>& S = *reinterpret_cast<BSmem<G>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    BSmem<G>& S = bsmem<G>();
     constexpr int NST = BSmem<G>::NST;
     const Params& P = K.P;
     const int tid = threadIdx.x, lane = tid & 31;
@@ -831,9 +986,11 @@ __global__ void __launch_bounds__(THREADS, 2) retrieve_kernel(const __grid_const
             mbar_init(&S.full[i], 1);
             mbar_init(&S.empty[i], CONSUMERS / 32);
         }
+        mbar_init(&S.res_bar, 1);
         mbar_fence_init();
         S.gen = 0;
         S.abort = 0;
+        S.resident = 0;
     }
     if (tid >= 32) copy_tab(P.tab, S.tab, tid - 32, THREADS - 32);
     // everything below reads the streaming kernel's results: wait for that
@@ -861,32 +1018,39 @@ __global__ void __launch_bounds__(THREADS, 2) retrieve_kernel(const __grid_const
         wk.t = (int)((long long)blockIdx.x * T / gridDim.x);
         wk.t1 = (int)((long long)(blockIdx.x + 1) * T / gridDim.x);
         wk.ngr = ngr;
+        if (copier && tid == CONSUMERS) r_load_scores<G>(P, wk, pre, 0);
+        __syncthreads();
         // first pass: bins; then the threshold bin's tokens are gathered and
         // selected inside one CTA per head, or, for a bin of more than
         // CAND_CAP tokens, refined by four more passes over all scores
-        if (!copier) r_pass<G>(P, S, wk, pre, RP_BINS, tid);
+        if (!copier) r_pass<G, RP_BINS>(P, wk, pre, tid);
         ok = grid_sync(P, S);
         if (ok && !copier)
             for (int hx = blockIdx.x; hx < (int)nrad; hx += gridDim.x) {
                 const uint32_t e = __ldcg(P.rlist + hx);
-                r_digit<G>(P, S, (int)(e >> 16), (int)(e & 0xFFFFu), RP_BINS, tid);
+                r_digit<G>(P, (int)(e >> 16), (int)(e & 0xFFFFu), RP_BINS, tid);
             }
         ok = ok && grid_sync(P, S);
         if (tid == 0) trace_max(P, 14);
         if (ok) {
-            if (!copier) r_pass<G>(P, S, wk, pre, RP_COMPACT, tid);
+            if (!copier) r_pass<G, RP_COMPACT>(P, wk, pre, tid);
             ok = grid_sync(P, S);
         }
         if (ok && !copier)
             for (int hx = blockIdx.x; hx < (int)nrad; hx += gridDim.x) {
                 const uint32_t e = __ldcg(P.rlist + hx);
-                r_local_select<G>(P, S, (int)(e >> 16), (int)(e & 0xFFFFu), tid);
+                r_local_select<G>(P, (int)(e >> 16), (int)(e & 0xFFFFu), tid);
             }
         if (ok) ok = grid_sync(P, S);
         if (tid == 0) trace_max(P, 8);
         const bool global = ok && __ldcg(&P.sync->any_global) != 0;
         for (int pass = RP_REF0; global && pass <= RP_REF3 && ok; ++pass) {
-            if (!copier) r_pass<G>(P, S, wk, pre, pass, tid);
+            if (!copier) {
+                if (pass == RP_REF0) r_pass<G, RP_REF0>(P, wk, pre, tid);
+                else if (pass == RP_REF1) r_pass<G, RP_REF1>(P, wk, pre, tid);
+                else if (pass == RP_REF2) r_pass<G, RP_REF2>(P, wk, pre, tid);
+                else r_pass<G, RP_REF3>(P, wk, pre, tid);
+            }
             ok = grid_sync(P, S);
             if (!ok) break;
             if (!copier)
@@ -894,25 +1058,25 @@ __global__ void __launch_bounds__(THREADS, 2) retrieve_kernel(const __grid_const
                     const uint32_t e = __ldcg(P.rlist + hx);
                     const int64_t bs = (int64_t)(e >> 16) * P.n_ret + (e & 0xFFFFu);
                     if (__ldcg(&P.hs[bs].n_cand) > (uint32_t)CAND_CAP)
-                        r_digit<G>(P, S, (int)(e >> 16), (int)(e & 0xFFFFu), pass, tid);
+                        r_digit<G>(P, (int)(e >> 16), (int)(e & 0xFFFFu), pass, tid);
                 }
             ok = grid_sync(P, S);
             if (tid == 0) trace_max(P, 8 + pass - RP_REF0);
         }
         if (ok && __ldcg(&P.sync->any_ties)) {
-            if (!copier) r_pass<G>(P, S, wk, pre, RP_TIES, tid);
+            if (!copier) r_pass<G, RP_TIES>(P, wk, pre, tid);
             ok = grid_sync(P, S);
             if (ok && !copier)
                 for (int hx = blockIdx.x; hx < (int)nrad; hx += gridDim.x) {
                     const uint32_t e = __ldcg(P.rlist + hx);
                     const int64_t bs = (int64_t)(e >> 16) * P.n_ret + (e & 0xFFFFu);
                     if (__ldcg(&P.hs[bs].n_cand) > (uint32_t)CAND_CAP)
-                        r_tie_locate<G>(P, S, (int)(e >> 16), (int)(e & 0xFFFFu), tid);
+                        r_tie_locate<G>(P, (int)(e >> 16), (int)(e & 0xFFFFu), tid);
                 }
             ok = ok && grid_sync(P, S);
         }
         if (ok) {
-            if (!copier) r_pass<G>(P, S, wk, pre, RP_MARK, tid);
+            if (!copier) r_pass<G, RP_MARK>(P, wk, pre, tid);
             ok = grid_sync(P, S);
             if (tid == 0) trace_max(P, 12);
         }
@@ -921,7 +1085,7 @@ __global__ void __launch_bounds__(THREADS, 2) retrieve_kernel(const __grid_const
                 for (int i = blockIdx.x; i < ngr; i += gridDim.x) {
                     int b, rg;
                     radix_group(P, i, b, rg);
-                    r_blist<G>(P, S, b, rg, tid);
+                    r_blist<G>(P, b, rg, tid);
                 }
             ok = grid_sync(P, S);
         }
@@ -949,7 +1113,7 @@ __global__ void __launch_bounds__(THREADS, 2) retrieve_kernel(const __grid_const
         for (int bs = 0; bs < P.B * P.n_ret; ++bs) {
             const int L = __ldg(P.seq_lens + bs / P.n_ret);
             if (!seq_ok(P, L)) continue;
-            const char* base = reinterpret_cast<const char*>(P.scores + (int64_t)bs * P.Ncap);
+            const char* base = reinterpret_cast<const char*>(P.scores + (int64_t)bs * P.sstride);
             const int nlines = (L * 4 + 127) / 128;
             for (int x = blockIdx.x * THREADS + tid; x < nlines; x += gridDim.x * THREADS)
                 asm volatile("discard.global.L2 [%0], 128;" ::"l"(base + (int64_t)x * 128) : "memory");

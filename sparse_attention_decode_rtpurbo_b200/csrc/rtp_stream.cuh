@@ -689,13 +689,13 @@ __device__ __forceinline__ void a_consumers(const KParams& K, ASmem<G>& S, AWalk
                 first_data = false;
                 const int n0 = (sg.first + i) * SROWS, nvalid = min(SROWS, sg.L - n0);
                 const uint32_t tile = smem_u32(&S.stage[st][0]);
-                float* sbase = P.scores + ((int64_t)sg.b * P.n_ret + S.tab.rg_slot0[sg.grp]) * P.Ncap;
+                float* sbase = P.scores + ((int64_t)sg.b * P.n_ret + S.tab.rg_slot0[sg.grp]) * P.sstride;
                 if (nvalid == SROWS) {
-                    if (nh4) score_tile<true, true>(tile, n0, nvalid, nh, track_min, qf, f, sbase, P.Ncap, warp, lane);
-                    else score_tile<false, true>(tile, n0, nvalid, nh, track_min, qf, f, sbase, P.Ncap, warp, lane);
+                    if (nh4) score_tile<true, true>(tile, n0, nvalid, nh, track_min, qf, f, sbase, P.sstride, warp, lane);
+                    else score_tile<false, true>(tile, n0, nvalid, nh, track_min, qf, f, sbase, P.sstride, warp, lane);
                 } else {
-                    if (nh4) score_tile<true, false>(tile, n0, nvalid, nh, track_min, qf, f, sbase, P.Ncap, warp, lane);
-                    else score_tile<false, false>(tile, n0, nvalid, nh, track_min, qf, f, sbase, P.Ncap, warp, lane);
+                    if (nh4) score_tile<true, false>(tile, n0, nvalid, nh, track_min, qf, f, sbase, P.sstride, warp, lane);
+                    else score_tile<false, false>(tile, n0, nvalid, nh, track_min, qf, f, sbase, P.sstride, warp, lane);
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&S.empty[st]);

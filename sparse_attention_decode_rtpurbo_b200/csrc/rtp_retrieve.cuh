@@ -1109,7 +1109,7 @@ __global__ void __launch_bounds__(THREADS, 2) retrieve_kernel(const __grid_const
     }
     // the stored scores are dead now: drop their L2 lines without writing
     // them back (each CTA a slice of every retrieval head's used range)
-    if (ok) {
+    if (ok || !work) {
         for (int bs = 0; bs < P.B * P.n_ret; ++bs) {
             const int L = __ldg(P.seq_lens + bs / P.n_ret);
             if (!seq_ok(P, L)) continue;
@@ -1119,9 +1119,10 @@ __global__ void __launch_bounds__(THREADS, 2) retrieve_kernel(const __grid_const
                 asm volatile("discard.global.L2 [%0], 128;" ::"l"(base + (int64_t)x * 128) : "memory");
         }
     }
-    // the last CTA out clears the call's coordination words
+    // the last CTA out clears the call's coordination words (none was set
+    // when every group was settled in the streaming kernel: no count then)
     __syncthreads();
-    if (tid == 0) {
+    if (work && tid == 0) {
         trace_max(P, 5);
         __threadfence();
         if (atomicAdd(&P.sync->exit_count, 1u) == gridDim.x - 1) {

@@ -42,7 +42,7 @@ TRACE_EVENTS = ["start", "select_done", "local_done", "lists_ready", "retrieval_
 # and the latest %globaltimer of two events
 TRACE_SUMS = ["a_cyc_wait", "a_cyc_score", "a_cyc_attn", "a_n_score", "a_n_attn", "a_cyc_score_begin",
               "a_first_data", "a_consumers_done", "b_cyc_bins", "b_n_pass_tiles", "b_cyc_compact",
-              "b_cyc_mark", "a_cyc_score_end", "a_cyc_local_begin", "a_cyc_local_end"]
+              "b_cyc_mark", "a_cyc_score_end", "a_cyc_local_begin", "a_cyc_local_end", "b_cyc_grid_sync"]
 
 
 class RtpDims(ctypes.Structure):

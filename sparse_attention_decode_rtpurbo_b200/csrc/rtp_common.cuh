@@ -210,24 +210,33 @@ __device__ __forceinline__ void trace_max(const Params& P, int i) {
 }
 
 // optional cycle accounting (debug, one thread per CTA): the SM cycles since
-// the previous mark are added to trace slot `slot`
+// the previous mark are added to sum `slot` (16..31) of the CTA's shared
+// array `sums`, which acct_flush adds to the trace once at the CTA's end (a
+// global atomic per mark from every CTA would serialise in L2 and distort
+// what it measures)
+constexpr int ACCT_SLOTS = 16;
 struct Acct {
-    unsigned long long* tr;
+    unsigned long long* sums;
     long long t;
-    __device__ __forceinline__ void init(const Params& P, bool me) {
-        tr = me ? P.dbg_trace : nullptr;
-        if (tr) t = clock64();
+    __device__ __forceinline__ void init(const Params& P, unsigned long long* s, bool me) {
+        sums = (me && P.dbg_trace) ? s : nullptr;
+        if (sums) t = clock64();
     }
     __device__ __forceinline__ void mark(int slot) {
-        if (!tr) return;
+        if (!sums) return;
         const long long now = clock64();
-        atomicAdd(tr + slot, (unsigned long long)(now - t));
+        sums[slot - 16] += (unsigned long long)(now - t);
         t = now;
     }
     __device__ __forceinline__ void count(int slot) {
-        if (tr) atomicAdd(tr + slot, 1ull);
+        if (sums) sums[slot - 16] += 1ull;
     }
 };
+__device__ __forceinline__ void acct_flush(const Params& P, unsigned long long* sums) {
+    if (!P.dbg_trace) return;
+    for (int i = 0; i < ACCT_SLOTS; ++i)
+        if (sums[i]) atomicAdd(P.dbg_trace + 16 + i, sums[i]);
+}
 
 // ---------------------------------------------------------------------------
 // mbarrier, bulk copies and TMA tensor copies

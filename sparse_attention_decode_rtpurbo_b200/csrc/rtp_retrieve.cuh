@@ -90,6 +90,9 @@ struct BSmem {
     alignas(8) uint64_t res_bar;   // the resident score tiles have landed
     uint32_t resident;             // this CTA's score tiles sit in the stage buffers
     uint32_t flag, gen, abort, base;
+    unsigned long long acct[ACCT_SLOTS];   // debug cycle sums of thread 0
+    unsigned long long sc_k[4], hit_k;     // bin_search: per-warp key sums, key sum before the hit
+    uint32_t sc_a[4], hit_a, hit_pos;      // bin_search: per-warp aux sums, aux sum before the hit, hit position
     int kept[MAX_G];
     uint32_t wsum[4];
     HeadTab tab;
@@ -219,7 +222,7 @@ __device__ __noinline__ void r_pass(const Params& P, RWalk wk, const int* pre, i
     const int lane = tid & 31;
     RSeg sg;
     Acct ac;
-    ac.init(P, tid == 0);
+    ac.init(P, S.acct, tid == 0);
     const int rp = pass - RP_REF0;
     const bool resident = S.resident != 0;
     if (resident && !mbar_wait_bounded(&S.res_bar, 0u)) set_status(P, ST_TIMEOUT);
@@ -464,6 +467,62 @@ __device__ __noinline__ void r_load_scores(const Params& P, RWalk wk, const int*
 // ---------------------------------------------------------------------------
 // Pick the digit of pass `pass` for radix head `hx`: the largest digit d whose
 // bins >= d hold at least the target mass (over the tokens above the prefix).
+// Search over 256 bins by the 128 compute threads (two walk positions
+// each, warp scans, one cross-warp step): walking the bins from 255 down
+// (desc) or from 0 up, the first position i whose inclusive key sum reaches
+// `need`.  Leaves in shared memory the position (255 when none does), the
+// key and aux sums of the positions before it (all positions when none
+// does).  The bin of position i is 255 - i (desc) or i.
+template <int G, typename KF, typename AF>
+__device__ __forceinline__ void bin_search(BSmem<G>& S, KF key_of, AF aux_of, bool desc, unsigned long long need,
+                                           int tid) {
+    const int warp = tid >> 5, lane = tid & 31;
+    const int i0 = 2 * tid;
+    const int d0 = desc ? 255 - i0 : i0, d1 = desc ? 254 - i0 : i0 + 1;
+    const unsigned long long k0 = key_of(d0), k1 = key_of(d1);
+    const uint32_t a0 = aux_of(d0), a1 = aux_of(d1);
+    unsigned long long ik = k0 + k1;
+    uint32_t ia = a0 + a1;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const unsigned long long xk = __shfl_up_sync(0xffffffffu, ik, o);
+        const uint32_t xa = __shfl_up_sync(0xffffffffu, ia, o);
+        if (lane >= o) {
+            ik += xk;
+            ia += xa;
+        }
+    }
+    if (lane == 31) {
+        S.sc_k[warp] = ik;
+        S.sc_a[warp] = ia;
+    }
+    consumer_sync();
+    unsigned long long ok_ = 0;
+    uint32_t oa = 0;
+    for (int w = 0; w < warp; ++w) {
+        ok_ += S.sc_k[w];
+        oa += S.sc_a[w];
+    }
+    if (tid == 0) {
+        S.hit_pos = 255;
+        S.hit_k = S.sc_k[0] + S.sc_k[1] + S.sc_k[2] + S.sc_k[3];
+        S.hit_a = S.sc_a[0] + S.sc_a[1] + S.sc_a[2] + S.sc_a[3];
+    }
+    consumer_sync();
+    const unsigned long long e0 = ok_ + ik - (k0 + k1), e1 = e0 + k0;
+    const uint32_t f0 = oa + ia - (a0 + a1), f1 = f0 + a0;
+    if (e0 + k0 >= need && (i0 == 0 || e0 < need)) {
+        S.hit_pos = (uint32_t)i0;
+        S.hit_k = e0;
+        S.hit_a = f0;
+    } else if (e1 + k1 >= need && e1 < need) {
+        S.hit_pos = (uint32_t)i0 + 1;
+        S.hit_k = e1;
+        S.hit_a = f1;
+    }
+    consumer_sync();
+}
+
 template <int G>
 __device__ __noinline__ void r_digit(const Params& P, int b, int slot, int pass, int tid) {
     BSmem<G>& S = bsmem<G>();
@@ -477,47 +536,42 @@ __device__ __noinline__ void r_digit(const Params& P, int b, int slot, int pass,
         gmass[d] = 0ull;
     }
     consumer_sync();
-    if (tid == 0) {
-        HeadState st = P.hs[bs];
-        if (pass == RP_BINS) {
-            unsigned long long z = 0;
-            for (int d = 0; d < 256; ++d) z += S.dmass[d];
-            const double pb = (double)__ldg(P.p + b);
-            unsigned long long tg = (unsigned long long)ceil(pb * (double)z);
-            if (tg > z) tg = z;
-            if (tg == 0) tg = 1;
+    auto mass_of = [&](int d) { return S.dmass[d]; };
+    auto cnt_of = [&](int d) { return S.dcnt[d]; };
+    if (pass == RP_BINS) {
+        // z = the total mass; bins ascend in smax - s: the first bin that
+        // completes the target ceil(p z)
+        bin_search(S, mass_of, cnt_of, false, ~0ull, tid);
+        const unsigned long long z = S.hit_k;
+        const double pb = (double)__ldg(P.p + b);
+        unsigned long long tg = (unsigned long long)ceil(pb * (double)z);
+        if (tg > z) tg = z;
+        if (tg == 0) tg = 1;
+        bin_search(S, mass_of, cnt_of, false, tg, tid);
+        if (tid == 0) {
+            HeadState st = P.hs[bs];
             st.target = tg;
-            // bins ascend in smax - s: the first bin that completes the target
-            unsigned long long cum = 0;
-            uint32_t cabove = 0;
-            uint32_t bstar = 255;
-            for (int d = 0; d < 256; ++d) {
-                if (cum + S.dmass[d] >= tg) {
-                    bstar = (uint32_t)d;
-                    break;
-                }
-                cum += S.dmass[d];
-                cabove += S.dcnt[d];
-            }
+            const uint32_t bstar = S.hit_pos;
             st.bstar = bstar;
             st.n_cand = S.dcnt[bstar];
-            st.mass_above = cum;
-            st.count_above = cabove;
+            st.mass_above = S.hit_k;
+            st.count_above = S.hit_a;
             st.prefix = 0;
             if (st.n_cand > (uint32_t)CAND_CAP) atomicOr(&P.sync->any_global, 1u);
-        } else {
+            P.hs[bs] = st;
+        }
+        consumer_sync();
+        return;
+    }
+    const unsigned long long tgt = __ldcg(&P.hs[bs].target), above = __ldcg(&P.hs[bs].mass_above);
+    bin_search(S, mass_of, cnt_of, true, tgt > above ? tgt - above : 0ull, tid);
+    if (tid == 0) {
+        HeadState st = P.hs[bs];
+        {
             const int rp = pass - RP_REF0;
-            unsigned long long cum = st.mass_above;
-            uint32_t cabove = st.count_above;
-            int dstar = 0;
-            for (int d = 255; d >= 0; --d) {
-                if (cum + S.dmass[d] >= st.target) {
-                    dstar = d;
-                    break;
-                }
-                cum += S.dmass[d];
-                cabove += S.dcnt[d];
-            }
+            const int dstar = 255 - (int)S.hit_pos;
+            const unsigned long long cum = st.mass_above + S.hit_k;
+            const uint32_t cabove = st.count_above + S.hit_a;
             st.mass_above = cum;
             st.count_above = cabove;
             st.prefix = (st.prefix << 8) | (uint32_t)dstar;
@@ -616,21 +670,14 @@ __device__ __noinline__ void r_local_select(const Params& P, int b, int slot, in
             hist_add(S.H, 0, (int)((key >> (24 - 8 * rp)) & 255u), 1u, fixmass(key, smax));
         }
         consumer_sync();
+        // the highest digit whose mass completes the target (digits descend)
+        const unsigned long long base = S.lsel_mass;
+        bin_search(S, [&](int d) { return hist_mass(S.H, 0, d); }, [&](int d) { return S.H.cnt[0][d]; }, true,
+                   target > base ? target - base : 0ull, tid);
         if (tid == 0) {
-            unsigned long long cum = S.lsel_mass;
-            uint32_t cabove = S.lsel_count;
-            int dstar = 0;
-            for (int d = 255; d >= 0; --d) {
-                const unsigned long long md = hist_mass(S.H, 0, d);
-                if (cum + md >= target) {
-                    dstar = d;
-                    break;
-                }
-                cum += md;
-                cabove += S.H.cnt[0][d];
-            }
-            S.lsel_mass = cum;
-            S.lsel_count = cabove;
+            const int dstar = 255 - (int)S.hit_pos;
+            S.lsel_mass = base + S.hit_k;
+            S.lsel_count += S.hit_a;
             S.lsel_prefix = (prefix << 8) | (uint32_t)dstar;
             S.lsel_neq = S.H.cnt[0][dstar];
             S.lsel_meq = hist_mass(S.H, 0, dstar);
@@ -666,18 +713,13 @@ __device__ __noinline__ void r_local_select(const Params& P, int b, int slot, in
                 atomicAdd(&S.H.cnt[0][(x >> (24 - 8 * rp)) & 255u], 1u);
             }
             consumer_sync();
+            // the lowest index digit that reaches the wanted rank
+            const uint32_t rank = S.lsel_count;
+            bin_search(S, [&](int d) { return (unsigned long long)S.H.cnt[0][d]; }, [&](int d) { return 0u; }, false,
+                       rank, tid);
             if (tid == 0) {
-                uint32_t rank = S.lsel_count, cum = 0;
-                int dstar = 255;
-                for (int d = 0; d < 256; ++d) {
-                    if (cum + S.H.cnt[0][d] >= rank) {
-                        dstar = d;
-                        break;
-                    }
-                    cum += S.H.cnt[0][d];
-                }
-                S.lsel_count = rank - cum;
-                S.lsel_prefix = (prefix << 8) | (uint32_t)dstar;
+                S.lsel_count = rank - (uint32_t)S.hit_k;
+                S.lsel_prefix = (prefix << 8) | S.hit_pos;
             }
             consumer_sync();
         }
@@ -980,6 +1022,13 @@ __global__ void __launch_bounds__(THREADS, 2) retrieve_kernel(const __grid_const
     const Params& P = K.P;
     const int tid = threadIdx.x, lane = tid & 31;
     const bool copier = tid >= CONSUMERS;
+    // grid barrier; thread 0's wait goes to debug sum 31
+    auto gsync = [&]() {
+        const long long t0 = clock64();
+        const bool r = grid_sync(P, S);
+        if (tid == 0 && P.dbg_trace) S.acct[15] += (unsigned long long)(clock64() - t0);
+        return r;
+    };
     int* pre = S.pre;
     if (tid == 0) {
         for (int i = 0; i < NST; ++i) {
@@ -990,6 +1039,7 @@ __global__ void __launch_bounds__(THREADS, 2) retrieve_kernel(const __grid_const
         mbar_fence_init();
         S.gen = 0;
         S.abort = 0;
+        for (int i = 0; i < ACCT_SLOTS; ++i) S.acct[i] = 0ull;
         S.resident = 0;
     }
     if (tid >= 32) copy_tab(P.tab, S.tab, tid - 32, THREADS - 32);
@@ -1024,24 +1074,24 @@ __global__ void __launch_bounds__(THREADS, 2) retrieve_kernel(const __grid_const
         // selected inside one CTA per head, or, for a bin of more than
         // CAND_CAP tokens, refined by four more passes over all scores
         if (!copier) r_pass<G, RP_BINS>(P, wk, pre, tid);
-        ok = grid_sync(P, S);
+        ok = gsync();
         if (ok && !copier)
             for (int hx = blockIdx.x; hx < (int)nrad; hx += gridDim.x) {
                 const uint32_t e = __ldcg(P.rlist + hx);
                 r_digit<G>(P, (int)(e >> 16), (int)(e & 0xFFFFu), RP_BINS, tid);
             }
-        ok = ok && grid_sync(P, S);
+        ok = ok && gsync();
         if (tid == 0) trace_max(P, 14);
         if (ok) {
             if (!copier) r_pass<G, RP_COMPACT>(P, wk, pre, tid);
-            ok = grid_sync(P, S);
+            ok = gsync();
         }
         if (ok && !copier)
             for (int hx = blockIdx.x; hx < (int)nrad; hx += gridDim.x) {
                 const uint32_t e = __ldcg(P.rlist + hx);
                 r_local_select<G>(P, (int)(e >> 16), (int)(e & 0xFFFFu), tid);
             }
-        if (ok) ok = grid_sync(P, S);
+        if (ok) ok = gsync();
         if (tid == 0) trace_max(P, 8);
         const bool global = ok && __ldcg(&P.sync->any_global) != 0;
         for (int pass = RP_REF0; global && pass <= RP_REF3 && ok; ++pass) {
@@ -1051,7 +1101,7 @@ __global__ void __launch_bounds__(THREADS, 2) retrieve_kernel(const __grid_const
                 else if (pass == RP_REF2) r_pass<G, RP_REF2>(P, wk, pre, tid);
                 else r_pass<G, RP_REF3>(P, wk, pre, tid);
             }
-            ok = grid_sync(P, S);
+            ok = gsync();
             if (!ok) break;
             if (!copier)
                 for (int hx = blockIdx.x; hx < (int)nrad; hx += gridDim.x) {
@@ -1060,12 +1110,12 @@ __global__ void __launch_bounds__(THREADS, 2) retrieve_kernel(const __grid_const
                     if (__ldcg(&P.hs[bs].n_cand) > (uint32_t)CAND_CAP)
                         r_digit<G>(P, (int)(e >> 16), (int)(e & 0xFFFFu), pass, tid);
                 }
-            ok = grid_sync(P, S);
+            ok = gsync();
             if (tid == 0) trace_max(P, 8 + pass - RP_REF0);
         }
         if (ok && __ldcg(&P.sync->any_ties)) {
             if (!copier) r_pass<G, RP_TIES>(P, wk, pre, tid);
-            ok = grid_sync(P, S);
+            ok = gsync();
             if (ok && !copier)
                 for (int hx = blockIdx.x; hx < (int)nrad; hx += gridDim.x) {
                     const uint32_t e = __ldcg(P.rlist + hx);
@@ -1073,11 +1123,11 @@ __global__ void __launch_bounds__(THREADS, 2) retrieve_kernel(const __grid_const
                     if (__ldcg(&P.hs[bs].n_cand) > (uint32_t)CAND_CAP)
                         r_tie_locate<G>(P, (int)(e >> 16), (int)(e & 0xFFFFu), tid);
                 }
-            ok = ok && grid_sync(P, S);
+            ok = ok && gsync();
         }
         if (ok) {
             if (!copier) r_pass<G, RP_MARK>(P, wk, pre, tid);
-            ok = grid_sync(P, S);
+            ok = gsync();
             if (tid == 0) trace_max(P, 12);
         }
         if (ok) {
@@ -1087,7 +1137,7 @@ __global__ void __launch_bounds__(THREADS, 2) retrieve_kernel(const __grid_const
                     radix_group(P, i, b, rg);
                     r_blist<G>(P, b, rg, tid);
                 }
-            ok = grid_sync(P, S);
+            ok = gsync();
         }
     }
     if (tid == 0) trace_max(P, 3);
@@ -1107,6 +1157,7 @@ __global__ void __launch_bounds__(THREADS, 2) retrieve_kernel(const __grid_const
         else r_consume_attn<G>(K, S, k, tid);
         if (tid == 0) trace_max(P, 4);
     }
+    if (tid == 0) acct_flush(P, S.acct);
     // the stored scores are dead now: drop their L2 lines without writing
     // them back (each CTA a slice of every retrieval head's used range)
     if (ok || !work) {

@@ -36,6 +36,7 @@ struct ASmem {
     uint32_t d_list[MAX_G], d_cnt;
     int pend_b, pend_rg, pend_L;   // best-token blocks this CTA attends after its share (d_list)
     uint32_t flag;
+    unsigned long long acct[ACCT_SLOTS];   // debug cycle sums of thread 0
     int tot_s, tot_l, nact;
     HeadTab tab;
     int pre[2];   // really [2 * (B + 1)]: tiles before sequence b (score, then local)
@@ -258,6 +259,11 @@ __device__ __forceinline__ void decide_group(const Params& P, ASmem<G>& S, int b
             const float zz = (z == z && z >= 1.0) ? (float)fmin(z, 1e30) : 1.f;
             float dr = 4.f * (__logf((float)L) - __logf(omp) - __logf(zz)) + 8.f;
             dr = fminf(fmaxf(dr, 8.f), 400.f);
+            // no wider than the scores' own spread (a little more, so that the
+            // lowest score lands in bin 254 at most): concentrated scores then
+            // spread over all the bins instead of colliding in a few
+            const float range = smax - key2f(mn);
+            if (range >= 0.f) dr = fminf(dr, range + fmaxf(range * 0x1p-10f, 1e-6f));
             h.dr = dr;
             h.inv_w = 255.f / dr;
             h.bstar = 0;
@@ -647,7 +653,7 @@ __device__ __forceinline__ void a_consumers(const KParams& K, ASmem<G>& S, AWalk
     MmaAttn<G> attn;
     attn.init();
     Acct ac;
-    ac.init(P, tid == 0);
+    ac.init(P, S.acct, tid == 0);
     bool first_data = true;
     bool extra = false;
     for (Seg sg = wk.next(P, pre_s, pre_l, S.tot_s);; sg = extra ? Seg{-1} : wk.next(P, pre_s, pre_l, S.tot_s)) {
@@ -675,7 +681,7 @@ __device__ __forceinline__ void a_consumers(const KParams& K, ASmem<G>& S, AWalk
             f.reset();
             const bool nh4 = nh <= 4;
             const float pb = __ldg(P.p + sg.b);
-            const bool track_min = !(pb < 1.f);
+            const bool track_min = true;   // (the threshold when p >= 1; the select's bin range otherwise)
             ac.mark(21);
             for (int i = 0; i < sg.ntiles; ++i, ++k) {
                 const int st = (int)(k % NST);
@@ -775,7 +781,10 @@ __device__ __forceinline__ void a_consumers(const KParams& K, ASmem<G>& S, AWalk
             ac.mark(30);
         }
     }
-    if (tid == 0) trace_max(P, 23);
+    if (tid == 0) {
+        trace_max(P, 23);
+        acct_flush(P, S.acct);
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -804,6 +813,7 @@ __global__ void __launch_bounds__(THREADS, 2) stream_kernel(const __grid_constan
         mbar_fence_init();
         if (P.dbg_trace) atomicCAS(P.dbg_trace, 0ull, (unsigned long long)global_ns());
         S.d_cnt = 0;
+        for (int i = 0; i < ACCT_SLOTS; ++i) S.acct[i] = 0ull;
     }
     // the retrieval kernel may be scheduled now; it waits for this grid's
     // completion before it reads anything this grid writes

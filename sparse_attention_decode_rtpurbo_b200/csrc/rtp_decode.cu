@@ -219,16 +219,27 @@ static int num_sms() {
     return v;
 }
 
+// Test knob: RTP_GRID_CAP=n (n >= 1) caps both grids at n CTAs, so that small
+// tests reach the paths that only long shares take (select passes reading
+// the stored scores from global memory, histogram flushes every 64 tiles).
+// Read at every call; results do not depend on the grid.
+static int grid_cap() {
+    const char* v = getenv("RTP_GRID_CAP");
+    const int n = v ? atoi(v) : 0;
+    return n >= 1 ? n : MAX_GRID;
+}
+
 template <int G>
 static cudaError_t launch(const KParams& K, const Plan& pl, cudaStream_t s, void* const* ev, unsigned ev_flags) {
     const int sms = num_sms();
     if (!sms) return report(cudaErrorUnknown, "SM count");
+    const int cap = std::min(MAX_GRID, grid_cap());
     // streaming kernel: as many resident CTAs as the tiles can use
     {
         const size_t smem = asmem_bytes<G>(pl.B);
         const int occ = occupancy((const void*)stream_kernel<G>, smem);
         if (occ < 1) return report(cudaErrorInvalidConfiguration, "stream kernel occupancy");
-        const long long grid = std::max(1ll, std::min<long long>(std::min(MAX_GRID, occ * sms), pl.tiles_cap));
+        const long long grid = std::max(1ll, std::min<long long>(std::min(cap, occ * sms), pl.tiles_cap));
         stream_kernel<G><<<(unsigned)grid, THREADS, smem, s>>>(K);
         cudaError_t e = report(cudaGetLastError(), "stream kernel launch");
         if (e != cudaSuccess) return e;
@@ -242,7 +253,7 @@ static cudaError_t launch(const KParams& K, const Plan& pl, cudaStream_t s, void
         const size_t smem = bsmem_bytes<G>(pl.B * pl.n_rg);
         const int occ = occupancy((const void*)retrieve_kernel<G>, smem);
         if (occ < 1) return report(cudaErrorInvalidConfiguration, "retrieval kernel occupancy");
-        const int grid = std::min(MAX_GRID, occ * sms);
+        const int grid = std::min(cap, occ * sms);
         cudaLaunchConfig_t cfg;
         memset(&cfg, 0, sizeof(cfg));
         cfg.gridDim = dim3((unsigned)grid);

@@ -141,3 +141,47 @@ def test_full_size_workloads(w):
     case = synth.workload(w)
     fails, stats, gpu, ref = run_both(case)
     assert not fails, "\n".join(fails[:20])
+
+
+def _ties_at_tau(case, ref, b, h):
+    s = oracle.index_scores(case, b, h)[: int(case.seq_lens[b])]
+    return int(np.count_nonzero(s == ref["tau"][b, h]))
+
+
+def test_refine_passes_many_ties():
+    """Few integer score levels over 64K tokens: the threshold bin holds more
+    than 4096 tokens, so the select refines the threshold over all stored
+    scores (four 8-bit passes), counts threshold ties per tile and locates the
+    last tie kept.  Block sets, k* and tau must be exact."""
+    done = deep = 0
+    for seed in range(8):
+        case = synth.integer_case(seed, B=1, Hkv=2, G=4, L=65536, p=0.9, qmax=1, kmax=1)
+        ref = oracle.decode_step(case)
+        assert ref["rc"] == 0
+        ret = np.nonzero(case.head_kind)[0]
+        # where p falls inside the mass of the last kept token: the count of
+        # ties kept is robust to mass rounding unless p sits at an end
+        lo, hi = ref["cum_before"][0, ret], ref["cum_at"][0, ret]
+        frac = (0.9 - lo) / np.maximum(hi - lo, 1e-300)
+        if np.any((frac < 1e-3) | (frac > 1 - 1e-3)):
+            continue
+        deep += max(_ties_at_tau(case, ref, 0, h) for h in ret) > 4096
+        dc = DeviceCase(case)
+        dc.run()
+        fails, _ = compare(case, dc.results(), ref, exact_sets=True, check_kstar=True, check_tau=True)
+        assert not fails, f"seed {seed}:\n" + "\n".join(fails[:10])
+        done += 1
+    assert done >= 4 and deep >= 2, (done, deep)
+
+
+@pytest.mark.parametrize("cap,w,scale", [(3, 5, 8), (7, 3, 1)])
+def test_small_grid_long_shares(monkeypatch, cap, w, scale):
+    """Both grids capped at a few CTAs (RTP_GRID_CAP): every CTA's share of
+    stored score tiles exceeds the shared-memory stages, so the select passes
+    read them from global memory; with 7 CTAs over 4 x 128K, shares of more
+    than 64 tiles of one group flush the shared histograms mid-run.  Results
+    must not change."""
+    monkeypatch.setenv("RTP_GRID_CAP", str(cap))
+    case = synth.workload(w, scale=scale)
+    fails, stats, gpu, ref = run_both(case)
+    assert not fails, "\n".join(fails[:20])

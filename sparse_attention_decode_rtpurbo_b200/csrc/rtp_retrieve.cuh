@@ -224,12 +224,23 @@ __device__ __noinline__ void r_pass(const Params& P, RWalk wk, const int* pre, i
     Acct ac;
     ac.init(P, S.acct, tid == 0);
     const int rp = pass - RP_REF0;
+    // the parameters this loop uses, read once: through a reference into the
+    // parameter block they would be read again after every global atomic
+    const int n_ret = P.n_ret, sstride = P.sstride, words_cap = P.words_cap, ntiles_cap = P.ntiles_cap;
+    const HeadState* const hs = P.hs;
+    const float* const scores = P.scores;
+    uint32_t* const hist_cnt = P.hist_cnt;
+    unsigned long long* const hist_mass_g = P.hist_mass;
+    uint32_t* const cand_cnt = P.cand_cnt;
+    unsigned long long* const cand = P.cand;
+    uint32_t* const bitmap = P.bitmap;
+    uint32_t* const tie_cnt = P.tie_cnt;
     const bool resident = S.resident != 0;
     if (resident && !mbar_wait_bounded(&S.res_bar, 0u)) set_status(P, ST_TIMEOUT);
     int sbase = 0;
     while (wk.next(P, pre, sg)) {
         const int nh = S.tab.rg_nh[sg.rg], slot0 = S.tab.rg_slot0[sg.rg];
-        const int64_t bs0 = (int64_t)sg.b * P.n_ret + slot0;
+        const int64_t bs0 = (int64_t)sg.b * n_ret + slot0;
         for (int x = tid; x < 4 * G * 256; x += CONSUMERS) (&S.H.cnt[0][0])[x] = 0;
         if (tid < MAX_G) {
             S.tmask[tid] = 0;
@@ -240,7 +251,7 @@ __device__ __noinline__ void r_pass(const Params& P, RWalk wk, const int* pre, i
         if (tid == 0) {
             uint32_t n = 0, wm = 0;
             for (int hh = 0; hh < nh; ++hh) {
-                const HeadState* h = P.hs + bs0 + hh;
+                const HeadState* h = hs + bs0 + hh;
                 if (__ldcg(&h->mode) != MODE_RADIX) continue;
                 const bool local = __ldcg(&h->n_cand) <= (uint32_t)CAND_CAP;
                 const bool want = (pass == RP_BINS || pass == RP_MARK) ? true : (pass == RP_COMPACT ? local : !local);
@@ -253,7 +264,7 @@ __device__ __noinline__ void r_pass(const Params& P, RWalk wk, const int* pre, i
         consumer_sync();
         const int nr = (int)S.nrad_h;
         const uint32_t wantm = S.want_mask;
-        if (tid < nr) S.rhs[tid] = load_rhead(P.hs + bs0 + S.rlist_h[tid]);
+        if (tid < nr) S.rhs[tid] = load_rhead(hs + bs0 + S.rlist_h[tid]);
         const int nitems = sg.ntiles * nr;
         // this CTA's histograms -> the heads' global ones (at the end of the
         // run, and every 64 tiles so that no partial sum can wrap)
@@ -263,8 +274,8 @@ __device__ __noinline__ void r_pass(const Params& P, RWalk wk, const int* pre, i
                 const int hh = x >> 8, d = x & 255;
                 const uint32_t c = S.H.cnt[hh][d];
                 if (c) {
-                    atomicAdd(P.hist_cnt + (bs0 + hh) * 256 + d, c);
-                    atomicAdd(P.hist_mass + (bs0 + hh) * 256 + d, hist_mass(S.H, hh, d));
+                    atomicAdd(hist_cnt + (bs0 + hh) * 256 + d, c);
+                    atomicAdd(hist_mass_g + (bs0 + hh) * 256 + d, hist_mass(S.H, hh, d));
                     S.H.cnt[hh][d] = 0;
                     S.H.m[0][hh][d] = 0;
                     S.H.m[1][hh][d] = 0;
@@ -280,7 +291,7 @@ __device__ __noinline__ void r_pass(const Params& P, RWalk wk, const int* pre, i
         auto load_item = [&](int it, int tile, int hx, float* dst) {
             const int hh = S.rlist_h[hx];
             const int n0 = tile * SROWS, nvalid = min(SROWS, sg.L - n0);
-            const float* src = resident ? res + (size_t)it * SROWS : P.scores + (bs0 + hh) * P.sstride + n0;
+            const float* src = resident ? res + (size_t)it * SROWS : scores + (bs0 + hh) * sstride + n0;
 #pragma unroll
             for (int u = 0; u < U; ++u) {
                 const int r = tid + u * CONSUMERS;
@@ -372,7 +383,7 @@ __device__ __noinline__ void r_pass(const Params& P, RWalk wk, const int* pre, i
                 for (int u = 0; u < U; ++u) tot += __popc(bal[u]);
                 if (tot) {
                     uint32_t base = 0;
-                    if (lane == 0) base = atomicAdd(P.cand_cnt + bs0 + hh, tot);
+                    if (lane == 0) base = atomicAdd(cand_cnt + bs0 + hh, tot);
                     base = __shfl_sync(0xffffffffu, base, 0);
 #pragma unroll
                     for (int u = 0; u < U; ++u) {
@@ -380,7 +391,7 @@ __device__ __noinline__ void r_pass(const Params& P, RWalk wk, const int* pre, i
                             const uint32_t pos = base + __popc(bal[u] & ((1u << lane) - 1u));
                             if (pos < (uint32_t)CAND_CAP) {
                                 const int r = tid + u * CONSUMERS;
-                                P.cand[(bs0 + hh) * CAND_CAP + pos] =
+                                cand[(bs0 + hh) * CAND_CAP + pos] =
                                     ((unsigned long long)f2key(v[u]) << 32) | (uint32_t)(n0 + r);
                             }
                         }
@@ -392,14 +403,14 @@ __device__ __noinline__ void r_pass(const Params& P, RWalk wk, const int* pre, i
                 // the warp's blocks straight into the head's bitmap (zeroed
                 // when the group was registered for the select)
                 if (lane == 0 && bits)
-                    atomicOr(P.bitmap + (bs0 + hh) * P.words_cap + tile / 2, bits << ((tile & 1) * 16));
+                    atomicOr(bitmap + (bs0 + hh) * words_cap + tile / 2, bits << ((tile & 1) * 16));
             } else if constexpr (pass == RP_TIES) {
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
                 if (lane == 0 && cnt) atomicAdd(&S.tcnt[hh], cnt);
                 consumer_sync();
                 if (tid == 0) {
-                    P.tie_cnt[(bs0 + hh) * P.ntiles_cap + tile] = S.tcnt[hh];
+                    tie_cnt[(bs0 + hh) * ntiles_cap + tile] = S.tcnt[hh];
                     S.tcnt[hh] = 0;
                 }
                 consumer_sync();

@@ -300,6 +300,65 @@ __device__ __noinline__ void r_pass(const Params& P, RWalk wk, const int* pre, i
         };
         if (nitems > 0) load_item(0, sg.first, 0, vn);
         consumer_sync();   // S.rhs
+        if constexpr (pass == RP_COMPACT) {
+            if (resident) {
+                // resident scores: count the threshold-bin tokens per head,
+                // reserve each head's range with one atomic, then write (one
+                // global round trip per head and run instead of per item)
+                for (int sub = 0; sub < 2; ++sub) {
+                    int tile = sg.first - 1, hx = nr - 1;
+#pragma unroll 1
+                    for (int it = 0; it < nitems; ++it) {
+                        if (++hx == nr) {
+                            hx = 0;
+                            ++tile;
+                        }
+                        if (!((wantm >> hx) & 1u)) continue;
+                        const RHead rh = S.rhs[hx];
+                        const int n0 = tile * SROWS, nvalid = min(SROWS, sg.L - n0);
+                        const float* src = res + (size_t)it * SROWS;
+                        uint32_t bal[U], tot = 0;
+                        float v[U];
+#pragma unroll
+                        for (int u = 0; u < U; ++u) {
+                            const int r = tid + u * CONSUMERS;
+                            v[u] = src[r];
+                            bal[u] = __ballot_sync(0xffffffffu,
+                                                   r < nvalid && score_bin(v[u], rh.smax, rh.dr, rh.inv_w) == rh.bstar);
+                            tot += __popc(bal[u]);
+                        }
+                        if (sub == 0) {
+                            if (lane == 0 && tot) atomicAdd(&S.tcnt[hx], tot);
+                        } else if (tot) {
+                            uint32_t off = 0;
+                            if (lane == 0) off = atomicAdd(&S.tcnt[hx], tot);
+                            uint32_t pos = S.tmask[hx] + __shfl_sync(0xffffffffu, off, 0);
+#pragma unroll
+                            for (int u = 0; u < U; ++u) {
+                                if ((bal[u] >> lane) & 1u) {
+                                    const uint32_t pp = pos + __popc(bal[u] & ((1u << lane) - 1u));
+                                    if (pp < (uint32_t)CAND_CAP)
+                                        cand[(bs0 + S.rlist_h[hx]) * CAND_CAP + pp] =
+                                            ((unsigned long long)f2key(v[u]) << 32) | (uint32_t)(n0 + tid + u * CONSUMERS);
+                                }
+                                pos += __popc(bal[u]);
+                            }
+                        }
+                    }
+                    consumer_sync();
+                    if (sub == 0) {
+                        if (tid < nr && ((wantm >> tid) & 1u)) {
+                            S.tmask[tid] = atomicAdd(cand_cnt + bs0 + S.rlist_h[tid], S.tcnt[tid]);
+                            S.tcnt[tid] = 0;
+                        }
+                        consumer_sync();
+                    }
+                }
+                ac.mark(26);
+                sbase += nitems;
+                continue;
+            }
+        }
         uint32_t ovf_n = 0u;
         unsigned long long ovf_m = 0ull;
         int cur_h = -1;

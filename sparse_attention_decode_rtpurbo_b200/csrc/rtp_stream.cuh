@@ -599,6 +599,12 @@ __device__ __forceinline__ void a_producer(const KParams& K, ASmem<G>& S, AWalk 
                 set_status(P, ST_TIMEOUT);
                 alive = false;
             }
+            // the second tile waits for the first to land: every CTA's first
+            // tile then arrives within ~10 MB of requests, not ~30 MB
+            if (lane == 0 && k == 1 && alive && !mbar_wait_bounded(&S.full[0], 0u)) {
+                set_status(P, ST_TIMEOUT);
+                alive = false;
+            }
             alive = __shfl_sync(0xffffffffu, alive ? 1 : 0, 0) != 0;
             if (!alive) break;
             uint8_t* dst = &S.stage[st][0];

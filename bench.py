@@ -319,7 +319,7 @@ def main():
     t_ms = statistics.mean(step_ms)
 
     # ---- timeline of one step (debug trace, separate untimed replays) ----
-    trace_buf = torch.zeros(32, dtype=torch.int64, device=dev)
+    trace_buf = torch.zeros(rtp.TRACE_WORDS, dtype=torch.int64, device=dev)
     tdbg = rtp.RtpDebug(trace=trace_buf.data_ptr())
     dc.step.dims.debug = ctypes.pointer(tdbg)
     tl = []

@@ -76,13 +76,15 @@ typedef struct rtp_debug {
     float* smax;             /* [B*Hq] largest index score s */
     double* Z;               /* [B*Hq] sum over n < L of exp((s_n - smax)/4) */
     uint32_t* block_bitmap;  /* [B*Hq*words], words = ceil(ceil(capacity/64)/32); bit j%32 of word j/32 = block j kept */
-    /* [32] %globaltimer nanoseconds, zero them before the call: 0 kernel start, 1 last selection
-     * decided, 2 last local-head combine done, 3 last block list final, 4 last retrieval combine
-     * done, 5 kernel end, 6 last selection started (all index scores of a group done),
-     * 7 last local-head combine started, 8-11 last radix pass 1-4 done, 12 last block mark done;
-     * summed over CTAs: 16-24 consumer SM cycles waiting for data, in score begin / tile /
-     * release / epilogue, attention begin / tile / epilogue, other; 25 score tiles; 26-28
-     * producer ns waiting for a free stage, on other CTAs, for queue claims */
+    /* [48] debug trace, zeroed by the caller before the call.
+     * 0-15: latest %globaltimer ns over CTAs of: 0 first CTA start, 1 group decision done,
+     *   2 local-head output done, 3 block lists final, 4 retrieval attention done, 5 CTA end,
+     *   6 group decision started, 7 streaming shares assigned, 8-11 selection steps done
+     *   (local select / refine passes 2-4), 12 block marks done, 13 retrieval kernel started,
+     *   14 first selection pass and digits done, 15 retrieval attention started.
+     * 16-47: sums over CTAs of one thread's SM cycles (or counts) by phase; the Python
+     *   binding's TRACE_SUMS names them in order (slots 22 and 23 are %globaltimer events:
+     *   first index tile consumed, last streaming share done). */
     unsigned long long* trace;
 } rtp_debug;
 

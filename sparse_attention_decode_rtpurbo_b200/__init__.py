@@ -42,7 +42,10 @@ TRACE_EVENTS = ["start", "select_done", "local_done", "lists_ready", "retrieval_
 # and the latest %globaltimer of two events
 TRACE_SUMS = ["a_cyc_wait", "a_cyc_score", "a_cyc_attn", "a_n_score", "a_n_attn", "a_cyc_score_begin",
               "a_first_data", "a_consumers_done", "b_cyc_bins", "b_n_pass_tiles", "b_cyc_compact",
-              "b_cyc_mark", "a_cyc_score_end", "a_cyc_local_begin", "a_cyc_local_end", "b_cyc_grid_sync"]
+              "b_cyc_mark", "a_cyc_score_end", "a_cyc_local_begin", "a_cyc_local_end", "b_cyc_grid_sync",
+              "b_attn_wait", "b_attn_tile", "b_attn_end", "b_n_attn", "b_prod_wait", "b_cyc_digit", "b_cyc_local_select",
+              "b_cyc_blist", "b_cyc_res_wait"]
+TRACE_WORDS = 48
 
 
 class RtpDims(ctypes.Structure):

@@ -210,11 +210,11 @@ __device__ __forceinline__ void trace_max(const Params& P, int i) {
 }
 
 // optional cycle accounting (debug, one thread per CTA): the SM cycles since
-// the previous mark are added to sum `slot` (16..31) of the CTA's shared
+// the previous mark are added to sum `slot` (16..47) of the CTA's shared
 // array `sums`, which acct_flush adds to the trace once at the CTA's end (a
 // global atomic per mark from every CTA would serialise in L2 and distort
 // what it measures)
-constexpr int ACCT_SLOTS = 16;
+constexpr int ACCT_SLOTS = 32;   // debug sums 16..47
 struct Acct {
     unsigned long long* sums;
     long long t;

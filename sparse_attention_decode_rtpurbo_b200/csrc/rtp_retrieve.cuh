@@ -236,7 +236,11 @@ __device__ __noinline__ void r_pass(const Params& P, RWalk wk, const int* pre, i
     uint32_t* const bitmap = P.bitmap;
     uint32_t* const tie_cnt = P.tie_cnt;
     const bool resident = S.resident != 0;
-    if (resident && !mbar_wait_bounded(&S.res_bar, 0u)) set_status(P, ST_TIMEOUT);
+    if (resident) {
+        const long long tq = clock64();
+        if (!mbar_wait_bounded(&S.res_bar, 0u)) set_status(P, ST_TIMEOUT);
+        if (tid == 0 && P.dbg_trace) S.acct[40 - 16] += (unsigned long long)(clock64() - tq);
+    }
     int sbase = 0;
     while (wk.next(P, pre, sg)) {
         const int nh = S.tab.rg_nh[sg.rg], slot0 = S.tab.rg_slot0[sg.rg];
@@ -946,10 +950,12 @@ __device__ __forceinline__ void r_produce_attn(const KParams& K, BSmem<G>& S, co
     const Params& P = K.P;
     auto acquire = [&](int st, uint32_t round) -> bool {
         bool ok = true;
+        const long long t0 = clock64();
         if (lane == 0 && round > 0 && !mbar_wait_bounded(&S.empty[st], (round - 1) & 1u)) {
             set_status(P, ST_TIMEOUT);
             ok = false;
         }
+        if (lane == 0 && P.dbg_trace) S.acct[36 - 16] += (unsigned long long)(clock64() - t0);
         return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
     };
     int gi = t < t1 ? last_le(pre, ngroups + 1, t) : 0;
@@ -1026,12 +1032,15 @@ __device__ __forceinline__ void r_consume_attn(const KParams& K, BSmem<G>& S, ui
     const int warp = tid >> 5, lane = tid & 31;
     MmaAttn<G> attn;
     attn.init();
+    Acct ac;
+    ac.init(P, S.acct, tid == 0);
     while (true) {
         const int st = (int)(k % NST);
         if (!mbar_wait_bounded(&S.full[st], (k / NST) & 1u)) {
             set_status(P, ST_TIMEOUT);
             return;
         }
+        ac.mark(32);
         ++k;
         const RDesc d = S.desc[st];
         if (d.type != 0) break;
@@ -1042,6 +1051,8 @@ __device__ __forceinline__ void r_consume_attn(const KParams& K, BSmem<G>& S, ui
         if (zeroed) fence_proxy_async();
         __syncwarp();
         if (lane == 0) mbar_arrive(&S.empty[st]);
+        ac.mark(33);
+        ac.count(35);
         if (d.flags & 2) {
             attn.finish(S.X, warp, lane);
             consumer_sync();
@@ -1059,6 +1070,7 @@ __device__ __forceinline__ void r_consume_attn(const KParams& K, BSmem<G>& S, ui
                     combine_splits<G>(S.X, P.rpart + ((int64_t)d.c0 + gi) * G * PSTRIDE, d.nsplits, heads, out0, tid);
                 }
             }
+            ac.mark(34);
         }
     }
 }
@@ -1148,7 +1160,9 @@ __global__ void __launch_bounds__(THREADS, 2) retrieve_kernel(const __grid_const
         if (ok && !copier)
             for (int hx = blockIdx.x; hx < (int)nrad; hx += gridDim.x) {
                 const uint32_t e = __ldcg(P.rlist + hx);
+                const long long tq = clock64();
                 r_digit<G>(P, (int)(e >> 16), (int)(e & 0xFFFFu), RP_BINS, tid);
+                if (tid == 0 && P.dbg_trace) S.acct[37 - 16] += (unsigned long long)(clock64() - tq);
             }
         ok = ok && gsync();
         if (tid == 0) trace_max(P, 14);
@@ -1159,7 +1173,9 @@ __global__ void __launch_bounds__(THREADS, 2) retrieve_kernel(const __grid_const
         if (ok && !copier)
             for (int hx = blockIdx.x; hx < (int)nrad; hx += gridDim.x) {
                 const uint32_t e = __ldcg(P.rlist + hx);
+                const long long tq = clock64();
                 r_local_select<G>(P, (int)(e >> 16), (int)(e & 0xFFFFu), tid);
+                if (tid == 0 && P.dbg_trace) S.acct[38 - 16] += (unsigned long long)(clock64() - tq);
             }
         if (ok) ok = gsync();
         if (tid == 0) trace_max(P, 8);
@@ -1205,7 +1221,9 @@ __global__ void __launch_bounds__(THREADS, 2) retrieve_kernel(const __grid_const
                 for (int i = blockIdx.x; i < ngr; i += gridDim.x) {
                     int b, rg;
                     radix_group(P, i, b, rg);
+                    const long long tq = clock64();
                     r_blist<G>(P, b, rg, tid);
+                    if (tid == 0 && P.dbg_trace) S.acct[39 - 16] += (unsigned long long)(clock64() - tq);
                 }
             ok = gsync();
         }

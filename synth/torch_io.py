@@ -52,7 +52,7 @@ class DeviceCase:
                 "smax": torch.full((BH,), float("nan"), dtype=torch.float32, device=device),
                 "Z": torch.full((BH,), float("nan"), dtype=torch.float64, device=device),
                 "block_bitmap": torch.zeros((BH * self.words,), dtype=torch.int32, device=device),
-                "trace": torch.zeros((32,), dtype=torch.int64, device=device),
+                "trace": torch.zeros((rtp.TRACE_WORDS,), dtype=torch.int64, device=device),
             }
             self.dbg_struct = rtp.RtpDebug(*(self.dbg[k].data_ptr() for k in
                                              ("tau", "kstar", "kept_blocks", "smax", "Z", "block_bitmap", "trace")))

@@ -153,7 +153,10 @@ __device__ __forceinline__ float key2f(uint32_t k) {
 __device__ __forceinline__ double exp_wide(double x) {
     const double y = x * 1.4426950408889634;
     const double yi = floor(y);
-    return ldexp((double)exp2f((float)(y - yi)), (int)yi);
+    // f in [1, 2] times 2^yi, by adding yi to f's exponent field (the result
+    // is a normal double for |x| <= 700: the same value ldexp would give)
+    const double f = (double)exp2f((float)(y - yi));
+    return __longlong_as_double(__double_as_longlong(f) + ((long long)(int)yi << 52));
 }
 
 // softmax(s/4) weight of a score relative to the maximum score, in 2^-40 units
@@ -284,6 +287,19 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
             "r"(smem_u32(dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
         : "memory");
+}
+// L2 prefetch (a hint: nothing to wait for) of one 2-D TMA box, and of the
+// K and V boxes of one 64-row block (x as for the loads: 16-byte aligned)
+__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int x, int y) {
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(reinterpret_cast<uint64_t>(map)),
+                 "r"(x), "r"(y)
+                 : "memory");
+}
+__device__ __forceinline__ void kv_prefetch_l2(const CUtensorMap* mk, const CUtensorMap* mv, int row) {
+    tma_prefetch_2d(mk, 0, row);
+    tma_prefetch_2d(mk, 64, row);
+    tma_prefetch_2d(mv, 0, row);
+    tma_prefetch_2d(mv, 64, row);
 }
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 

@@ -178,7 +178,8 @@ __device__ __forceinline__ bool ticket_add(uint32_t* ctr, uint32_t add, uint32_t
 // final here; if every head of the group is final its block list is written
 // at once, otherwise its radix heads are registered for the exact select.
 template <int G>
-__device__ __forceinline__ void decide_group(const Params& P, ASmem<G>& S, int b, int rg, int L, float pb, int tid) {
+__device__ __forceinline__ void decide_group(const KParams& K, ASmem<G>& S, int b, int rg, int L, float pb, int tid) {
+    const Params& P = K.P;
     const int nh = S.tab.rg_nh[rg], slot0 = S.tab.rg_slot0[rg], g = S.tab.rg_group[rg];
     const int nblk = (L + BLK - 1) / BLK;
     const int nwords = (nblk + 31) / 32;
@@ -205,6 +206,10 @@ __device__ __forceinline__ void decide_group(const Params& P, ASmem<G>& S, int b
                 S.d_nmin[hh] = nmin;
                 S.d_flags[hh] = flags;
                 S.d_zabs[hh] = zabs;
+                // the best token's block into L2 now: if the head keeps only
+                // that token, this CTA attends it right after the decision
+                const uint32_t a = 0xFFFFFFFFu - (uint32_t)(best & 0xFFFFFFFFull);
+                if (a < (uint32_t)L) kv_prefetch_l2(&K.tmk, &K.tmv, (int)block_row(P, b, g, (int)(a / BLK)));
             }
         }
     }
@@ -719,7 +724,7 @@ __device__ __forceinline__ void a_consumers(const KParams& K, ASmem<G>& S, AWalk
             if (ticket_add(P.tick_score + sg.item_idx, (uint32_t)sg.ntiles, (uint32_t)sg.item_tiles, &S.flag)) {
                 __threadfence();
                 if (tid == 0) trace_max(P, 6);
-                decide_group<G>(P, S, sg.b, sg.grp, sg.L, pb, tid);
+                decide_group<G>(K, S, sg.b, sg.grp, sg.L, pb, tid);
                 consumer_sync();
                 if (tid == 0) trace_max(P, 1);
             }

@@ -171,6 +171,50 @@ __device__ __forceinline__ bool ticket_add(uint32_t* ctr, uint32_t add, uint32_t
     return *smem_flag != 0;
 }
 
+// The group's list when its heads keep only their best tokens (thread 0):
+// the distinct argmax blocks, ascending, with their head masks; the first
+// such group of a CTA is attended by that CTA after its share, a later one
+// goes to the retrieval kernel.
+template <int G>
+__device__ __forceinline__ void best_token_list(const Params& P, ASmem<G>& S, int b, int rg, int L, int nh, int slot0,
+                                                int g) {
+    const int bg = b * P.n_rg + rg;
+    uint32_t* list = P.blist + (int64_t)bg * P.nblk_cap;
+    // heads' argmax blocks in registers (fixed indices), then the
+    // distinct ones ascending, written straight to their destination
+    int bj_h[MAX_G];
+#pragma unroll
+    for (int hh = 0; hh < MAX_G; ++hh)
+        bj_h[hh] = (hh < nh && S.d_mode[hh] == MODE_TOP1) ? (int)(S.d_arg[hh] / BLK) : 0x7FFFFFFF;
+    const bool defer = S.d_cnt == 0;
+    uint32_t* dst = defer ? S.d_list : list;
+    uint32_t cnt = 0;
+    int last = -1;
+    while (true) {
+        int bj = 0x7FFFFFFF;
+#pragma unroll
+        for (int hh = 0; hh < MAX_G; ++hh)
+            if (bj_h[hh] > last && bj_h[hh] < bj) bj = bj_h[hh];
+        if (bj == 0x7FFFFFFF) break;
+        uint32_t hm = 0;
+#pragma unroll
+        for (int hh = 0; hh < MAX_G; ++hh)
+            if (bj_h[hh] == bj) hm |= 1u << (S.tab.slot_head[slot0 + hh] - g * P.G);
+        dst[cnt++] = ((uint32_t)bj << 8) | hm;
+        last = bj;
+    }
+    if (defer && cnt != 0) {
+        S.d_cnt = cnt;
+        S.pend_b = b;
+        S.pend_rg = rg;
+        S.pend_L = L;
+        P.bcount[bg] = 0;
+    } else {
+        P.bcount[bg] = cnt;
+        if (cnt) atomicAdd(&P.sync->kb_work, 1u);
+    }
+}
+
 // ---------------------------------------------------------------------------
 // selection of one retrieval group, by the last of its score splits
 // ---------------------------------------------------------------------------
@@ -224,69 +268,83 @@ __device__ __forceinline__ void decide_group(const KParams& K, ASmem<G>& S, int 
         // z = sum over tokens of exp((s - smax)/4); NaN when the fp64 sum was unusable
         const double sm4 = (double)smax * 0.25;
         const double z = (S.d_flags[hh] || sm4 > 600.0 || sm4 < -600.0) ? NAN : S.d_zabs[hh] * exp_wide(-sm4);
-        HeadState h;
-        h.smax = smax;
-        h.maxkey = k;
-        h.argmax = a;
-        h.minkey = mn;
-        h.pad0 = 0;
-        h.zrel = z;
-        h.target = 0;
-        h.mass_above = 0;
-        h.prefix = 0;
-        h.count_above = 0;
-        h.n_eq = 0;
-        h.n_tie = 0;
-        h.all_ties = 1;
-        h.tau_key = 0;
-        h.tie_idx = 0xFFFFFFFFu;
+        int mode;
+        uint32_t kstar = 0, tau_key = 0;
         if (!(pb > 0.f)) {
-            h.mode = MODE_SKIP;
-            h.kstar = 0;
+            mode = MODE_SKIP;
             set_status(P, ST_DEVICE_INPUT);
         } else if (pb >= 1.f) {
-            h.mode = MODE_ALL;
-            h.kstar = (uint32_t)L;
-            h.tau_key = mn;
+            mode = MODE_ALL;
+            kstar = (uint32_t)L;
+            tau_key = mn;
         } else if (z == z && 1.0 >= (double)pb * z * (1.0 + 1e-3)) {
-            h.mode = MODE_TOP1;   // the best token alone reaches p
-            h.kstar = 1;
-            h.tau_key = k;
+            mode = MODE_TOP1;   // the best token alone reaches p
+            kstar = 1;
+            tau_key = k;
         } else {
-            h.mode = MODE_RADIX;
-            h.kstar = 0;
+            mode = MODE_RADIX;
         }
-        // first select pass: 255 bins over smax - s in [0, dr), dr large
-        // enough that the tokens beyond it cannot hold the last 1 - p of the
-        // mass (otherwise the select continues in the overflow bin)
-        {
-            const float omp = pb < 1.f ? fmaxf(1.f - pb, 1e-6f) : 1e-6f;
+        HeadState* hs = P.hs + (int64_t)b * P.n_ret + slot;
+        if (mode == MODE_RADIX) {
+            // the exact select's state; its first pass bins smax - s into 255
+            // bins over [0, dr), dr large enough that the tokens beyond it
+            // cannot hold the last 1 - p of the mass (otherwise the select
+            // continues in the overflow bin), and no wider than the scores'
+            // own spread (a little more, so the lowest score lands in bin 254
+            // at most): concentrated scores then spread over all the bins
+            HeadState h;
+            h.mode = mode;
+            h.smax = smax;
+            h.maxkey = k;
+            h.argmax = a;
+            h.minkey = mn;
+            h.pad0 = 0;
+            h.zrel = z;
+            h.target = 0;
+            h.mass_above = 0;
+            h.prefix = 0;
+            h.count_above = 0;
+            h.n_eq = 0;
+            h.n_tie = 0;
+            h.all_ties = 1;
+            h.tau_key = 0;
+            h.tie_idx = 0xFFFFFFFFu;
+            h.kstar = 0;
+            const float omp = fmaxf(1.f - pb, 1e-6f);
             const float zz = (z == z && z >= 1.0) ? (float)fmin(z, 1e30) : 1.f;
             float dr = 4.f * (__logf((float)L) - __logf(omp) - __logf(zz)) + 8.f;
             dr = fminf(fmaxf(dr, 8.f), 400.f);
-            // no wider than the scores' own spread (a little more, so that the
-            // lowest score lands in bin 254 at most): concentrated scores then
-            // spread over all the bins instead of colliding in a few
             const float range = smax - key2f(mn);
             if (range >= 0.f) dr = fminf(dr, range + fmaxf(range * 0x1p-10f, 1e-6f));
             h.dr = dr;
             h.inv_w = 255.f / dr;
             h.bstar = 0;
             h.n_cand = 0;
+            *hs = h;
+        } else {
+            hs->mode = mode;   // (read by the select of a group that has radix heads too)
         }
-        P.hs[(int64_t)b * P.n_ret + slot] = h;
         const int bh = b * P.Hq + S.tab.slot_head[slot];
         if (P.dbg_smax) P.dbg_smax[bh] = smax;
         if (P.dbg_Z) P.dbg_Z[bh] = z;
-        if (h.mode != MODE_RADIX) {
-            if (P.dbg_tau) P.dbg_tau[bh] = key2f(h.tau_key);
-            if (P.dbg_kstar) P.dbg_kstar[bh] = (int32_t)h.kstar;
-            if (P.dbg_kept) P.dbg_kept[bh] = h.mode == MODE_TOP1 ? 1 : (h.mode == MODE_ALL ? nblk : 0);
+        if (mode != MODE_RADIX) {
+            if (P.dbg_tau) P.dbg_tau[bh] = key2f(tau_key);
+            if (P.dbg_kstar) P.dbg_kstar[bh] = (int32_t)kstar;
+            if (P.dbg_kept) P.dbg_kept[bh] = mode == MODE_TOP1 ? 1 : (mode == MODE_ALL ? nblk : 0);
         }
-        S.d_mode[hh] = h.mode;
+        S.d_mode[hh] = mode;
         S.d_arg[hh] = a;
     }
     consumer_sync();
+    {
+        // the common case first: every head keeps its best token only
+        bool top1 = P.dbg_bitmap == nullptr;
+        for (int hh = 0; hh < nh; ++hh) top1 = top1 && S.d_mode[hh] == MODE_TOP1;
+        if (top1) {
+            if (tid == 0) best_token_list<G>(P, S, b, rg, L, nh, slot0, g);
+            return;
+        }
+    }
     bool any_radix = false, any_all = false;
     uint32_t all_mask = 0;
     for (int hh = 0; hh < nh; ++hh) {
@@ -362,41 +420,7 @@ __device__ __forceinline__ void decide_group(const KParams& K, ASmem<G>& S, int 
         // only best-token blocks: the distinct argmax blocks, ascending, are
         // attended by this CTA after its share (the first such group of the
         // CTA; a later one goes to the retrieval kernel)
-        if (tid == 0) {
-            // heads' argmax blocks in registers (fixed indices), then the
-            // distinct ones ascending, written straight to their destination
-            int bj_h[MAX_G];
-#pragma unroll
-            for (int hh = 0; hh < MAX_G; ++hh)
-                bj_h[hh] = (hh < nh && S.d_mode[hh] == MODE_TOP1) ? (int)(S.d_arg[hh] / BLK) : 0x7FFFFFFF;
-            const bool defer = S.d_cnt == 0;
-            uint32_t* dst = defer ? S.d_list : list;
-            uint32_t cnt = 0;
-            int last = -1;
-            while (true) {
-                int bj = 0x7FFFFFFF;
-#pragma unroll
-                for (int hh = 0; hh < MAX_G; ++hh)
-                    if (bj_h[hh] > last && bj_h[hh] < bj) bj = bj_h[hh];
-                if (bj == 0x7FFFFFFF) break;
-                uint32_t hm = 0;
-#pragma unroll
-                for (int hh = 0; hh < MAX_G; ++hh)
-                    if (bj_h[hh] == bj) hm |= 1u << (S.tab.slot_head[slot0 + hh] - g * P.G);
-                dst[cnt++] = ((uint32_t)bj << 8) | hm;
-                last = bj;
-            }
-            if (defer && cnt != 0) {
-                S.d_cnt = cnt;
-                S.pend_b = b;
-                S.pend_rg = rg;
-                S.pend_L = L;
-                P.bcount[bg] = 0;
-            } else {
-                P.bcount[bg] = cnt;
-                if (cnt) atomicAdd(&P.sync->kb_work, 1u);
-            }
-        }
+        if (tid == 0) best_token_list<G>(P, S, b, rg, L, nh, slot0, g);
     }
 }
 

@@ -1066,7 +1066,6 @@ __device__ __forceinline__ void r_consume_attn(const KParams& K, BSmem<G>& S, ui
                 float* part = P.rpart + ((int64_t)blockIdx.x + gi) * G * PSTRIDE;
                 split_emit<G>(S.X, heads, part, nullptr, tid);
                 if (ticket_add(P.tick_ret + gi, (uint32_t)d.seg_tiles, (uint32_t)d.item_tiles, &S.flag)) {
-                    __threadfence();
                     combine_splits<G>(S.X, P.rpart + ((int64_t)d.c0 + gi) * G * PSTRIDE, d.nsplits, heads, out0, tid);
                 }
             }

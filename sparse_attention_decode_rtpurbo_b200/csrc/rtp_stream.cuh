@@ -154,7 +154,11 @@ __device__ __forceinline__ Seg best_token_seg(const SM& S) {
 }
 
 // Ticket among the consumer threads with a variable increment: true in the
-// CTA whose addition completes `total`; it re-arms the counter.
+// CTA whose addition completes `total`.  The fence before the addition
+// publishes this CTA's writes; the fence after it, in the CTA that completes
+// the count, orders its later reads of the other CTAs' writes (and, through
+// the CTA barrier, those of its other threads).  That CTA re-arms the counter
+// with a plain store: the next addition to it comes from a later launch.
 __device__ __forceinline__ bool ticket_add(uint32_t* ctr, uint32_t add, uint32_t total, uint32_t* smem_flag) {
     consumer_sync();
     if (threadIdx.x == 0) {
@@ -162,8 +166,8 @@ __device__ __forceinline__ bool ticket_add(uint32_t* ctr, uint32_t add, uint32_t
         const uint32_t old = atomicAdd(ctr, add);
         const bool last = old + add == total;
         if (last) {
-            atomicExch(ctr, 0u);
             __threadfence();
+            *reinterpret_cast<volatile uint32_t*>(ctr) = 0u;
         }
         *smem_flag = last;
     }
@@ -746,7 +750,6 @@ __device__ __forceinline__ void a_consumers(const KParams& K, ASmem<G>& S, AWalk
             if (nh4) score_split_end<G, true>(P, S, f, sg.b, sg.grp, sg.first, tid);
             else score_split_end<G, false>(P, S, f, sg.b, sg.grp, sg.first, tid);
             if (ticket_add(P.tick_score + sg.item_idx, (uint32_t)sg.ntiles, (uint32_t)sg.item_tiles, &S.flag)) {
-                __threadfence();
                 if (tid == 0) trace_max(P, 6);
                 decide_group<G>(K, S, sg.b, sg.grp, sg.L, pb, tid);
                 consumer_sync();
@@ -804,7 +807,6 @@ __device__ __forceinline__ void a_consumers(const KParams& K, ASmem<G>& S, AWalk
                 float* part = P.lpart + ((int64_t)c + sg.item_idx) * G * PSTRIDE;
                 split_emit<G>(S.X, heads, part, nullptr, tid);
                 if (ticket_add(P.tick_local + sg.item_idx, (uint32_t)sg.ntiles, (uint32_t)sg.item_tiles, &S.flag)) {
-                    __threadfence();
                     const long long T = (long long)S.tot_s + S.tot_l;
                     const int c0 = cta_of_tile(S.tot_s + sg.item_t0, T, S.nact);
                     const int c1 = cta_of_tile(S.tot_s + sg.item_t0 + sg.item_tiles - 1, T, S.nact);

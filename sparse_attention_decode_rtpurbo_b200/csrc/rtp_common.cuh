@@ -156,7 +156,8 @@ __device__ __forceinline__ double exp_wide(double x) {
     // f in [1, 2] times 2^yi, by adding yi to f's exponent field (the result
     // is a normal double for |x| <= 700: the same value ldexp would give)
     const double f = (double)exp2f((float)(y - yi));
-    return __longlong_as_double(__double_as_longlong(f) + ((long long)(int)yi << 52));
+    const unsigned long long e = (unsigned long long)(long long)(int)yi << 52;   // two's complement exponent step
+    return __longlong_as_double((long long)((unsigned long long)__double_as_longlong(f) + e));
 }
 
 // softmax(s/4) weight of a score relative to the maximum score, in 2^-40 units

@@ -184,26 +184,30 @@ __device__ __forceinline__ void best_token_list(const Params& P, ASmem<G>& S, in
                                                 int g) {
     const int bg = b * P.n_rg + rg;
     uint32_t* list = P.blist + (int64_t)bg * P.nblk_cap;
-    // heads' argmax blocks in registers (fixed indices), then the
-    // distinct ones ascending, written straight to their destination
-    int bj_h[MAX_G];
-#pragma unroll
-    for (int hh = 0; hh < MAX_G; ++hh)
-        bj_h[hh] = (hh < nh && S.d_mode[hh] == MODE_TOP1) ? (int)(S.d_arg[hh] / BLK) : 0x7FFFFFFF;
+    // the distinct argmax blocks ascending, written straight to their
+    // destination (short loops, not unrolled: this runs once per group, on
+    // code that is rarely in the instruction cache)
     const bool defer = S.d_cnt == 0;
     uint32_t* dst = defer ? S.d_list : list;
     uint32_t cnt = 0;
     int last = -1;
+#pragma unroll 1
     while (true) {
         int bj = 0x7FFFFFFF;
-#pragma unroll
-        for (int hh = 0; hh < MAX_G; ++hh)
-            if (bj_h[hh] > last && bj_h[hh] < bj) bj = bj_h[hh];
-        if (bj == 0x7FFFFFFF) break;
         uint32_t hm = 0;
-#pragma unroll
-        for (int hh = 0; hh < MAX_G; ++hh)
-            if (bj_h[hh] == bj) hm |= 1u << (S.tab.slot_head[slot0 + hh] - g * P.G);
+#pragma unroll 1
+        for (int hh = 0; hh < nh; ++hh) {
+            if (S.d_mode[hh] != MODE_TOP1) continue;
+            const int j = (int)(S.d_arg[hh] / BLK);
+            const uint32_t bit = 1u << (S.tab.slot_head[slot0 + hh] - g * P.G);
+            if (j > last && j < bj) {
+                bj = j;
+                hm = bit;
+            } else if (j == bj) {
+                hm |= bit;
+            }
+        }
+        if (bj == 0x7FFFFFFF) break;
         dst[cnt++] = ((uint32_t)bj << 8) | hm;
         last = bj;
     }

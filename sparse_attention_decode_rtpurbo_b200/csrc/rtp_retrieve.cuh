@@ -680,14 +680,16 @@ __device__ __noinline__ void r_digit(const Params& P, int b, int slot, int pass,
 // (count and fixed-point mass per digit, cumulative from the mass above the
 // bin) give tau and the number of its ties to keep, and a four-pass select
 // over the tie indices gives the largest tie index kept (ties toward the
-// lower index).
-template <int G>
+// lower index).  CPT candidates per thread, kept in registers: an instance
+// for at most 1024 candidates (8 per thread) and one for CAND_CAP; the
+// smaller one is a quarter of the code, which matters for code that runs
+// once per head and per step.
+template <int G, int CPT>
 __device__ __noinline__ void r_local_select(const Params& P, int b, int slot, int tid) {
     BSmem<G>& S = bsmem<G>();
-    constexpr int CPT = CAND_CAP / CONSUMERS;   // candidates per thread, kept in registers
     const int64_t bs = (int64_t)b * P.n_ret + slot;
     const uint32_t ncand = __ldcg(&P.hs[bs].n_cand);
-    if (ncand > (uint32_t)CAND_CAP) return;
+    if (ncand > (uint32_t)(CPT * CONSUMERS)) return;
     const int n = (int)ncand;
     uint32_t keys[CPT], idx[CPT];
 #pragma unroll
@@ -1173,7 +1175,11 @@ __global__ void __launch_bounds__(THREADS, 2) retrieve_kernel(const __grid_const
             for (int hx = blockIdx.x; hx < (int)nrad; hx += gridDim.x) {
                 const uint32_t e = __ldcg(P.rlist + hx);
                 const long long tq = clock64();
-                r_local_select<G>(P, (int)(e >> 16), (int)(e & 0xFFFFu), tid);
+                const int64_t bsx = (int64_t)(e >> 16) * P.n_ret + (e & 0xFFFFu);
+                if (__ldcg(&P.hs[bsx].n_cand) <= 8u * CONSUMERS)
+                    r_local_select<G, 8>(P, (int)(e >> 16), (int)(e & 0xFFFFu), tid);
+                else
+                    r_local_select<G, CAND_CAP / CONSUMERS>(P, (int)(e >> 16), (int)(e & 0xFFFFu), tid);
                 if (tid == 0 && P.dbg_trace) S.acct[38 - 16] += (unsigned long long)(clock64() - tq);
             }
         if (ok) ok = gsync();

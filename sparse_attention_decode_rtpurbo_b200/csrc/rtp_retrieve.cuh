@@ -890,9 +890,9 @@ __device__ __noinline__ void r_blist(const Params& P, int b, int rg, int tid) {
     for (int h0 = 0; h0 < nhalf; h0 += CONSUMERS) {
         const int hw = h0 + tid, w = hw >> 1;
         uint32_t uni = 0;
-        uint32_t hb[MAX_G];
+        uint32_t hb[G];   // a group has at most G heads
 #pragma unroll
-        for (int hh = 0; hh < MAX_G; ++hh) {
+        for (int hh = 0; hh < G; ++hh) {
             hb[hh] = 0;
             if (hh < nh && hw < nhalf) {
                 uint32_t word = __ldcg(P.bitmap + ((int64_t)b * P.n_ret + slot0 + hh) * P.words_cap + w);
@@ -922,7 +922,7 @@ __device__ __noinline__ void r_blist(const Params& P, int b, int rg, int tid) {
             uni &= uni - 1;
             uint32_t hm = 0;
 #pragma unroll
-            for (int hh = 0; hh < MAX_G; ++hh)
+            for (int hh = 0; hh < G; ++hh)
                 if ((hb[hh] >> jb) & 1u) hm |= 1u << (S.tab.slot_head[slot0 + hh] - g * P.G);
             list[pos++] = ((uint32_t)(hw * 16 + jb) << 8) | hm;
         }

@@ -202,8 +202,8 @@ __device__ __forceinline__ uint32_t score_bin(float s, float smax, float dr, flo
 // threshold ties per tile; RP_MARK marks blocks.
 enum RPass : int { RP_BINS = 0, RP_REF0, RP_REF1, RP_REF2, RP_REF3, RP_TIES, RP_MARK, RP_COMPACT };
 
-template <int G>
-__device__ __noinline__ void r_digit(const Params& P, int b, int slot, int pass, int tid);
+template <int G, int pass>
+__device__ __noinline__ void r_digit(const Params& P, int b, int slot, int tid);
 template <int G>
 __device__ __noinline__ void r_tie_locate(const Params& P, int b, int slot, int tid);
 template <int G>
@@ -597,8 +597,8 @@ __device__ __forceinline__ void bin_search(BSmem<G>& S, KF key_of, AF aux_of, bo
     consumer_sync();
 }
 
-template <int G>
-__device__ __noinline__ void r_digit(const Params& P, int b, int slot, int pass, int tid) {
+template <int G, int pass>
+__device__ __noinline__ void r_digit(const Params& P, int b, int slot, int tid) {
     BSmem<G>& S = bsmem<G>();
     const int64_t bs = (int64_t)b * P.n_ret + slot;
     uint32_t* gcnt = P.hist_cnt + bs * 256;
@@ -612,7 +612,7 @@ __device__ __noinline__ void r_digit(const Params& P, int b, int slot, int pass,
     consumer_sync();
     auto mass_of = [&](int d) { return S.dmass[d]; };
     auto cnt_of = [&](int d) { return S.dcnt[d]; };
-    if (pass == RP_BINS) {
+    if constexpr (pass == RP_BINS) {
         // z = the total mass; bins ascend in smax - s: the first bin that
         // completes the target ceil(p z)
         bin_search(S, mass_of, cnt_of, false, ~0ull, tid);
@@ -1162,7 +1162,7 @@ __global__ void __launch_bounds__(THREADS, 2) retrieve_kernel(const __grid_const
             for (int hx = blockIdx.x; hx < (int)nrad; hx += gridDim.x) {
                 const uint32_t e = __ldcg(P.rlist + hx);
                 const long long tq = clock64();
-                r_digit<G>(P, (int)(e >> 16), (int)(e & 0xFFFFu), RP_BINS, tid);
+                r_digit<G, RP_BINS>(P, (int)(e >> 16), (int)(e & 0xFFFFu), tid);
                 if (tid == 0 && P.dbg_trace) S.acct[37 - 16] += (unsigned long long)(clock64() - tq);
             }
         ok = ok && gsync();
@@ -1199,7 +1199,10 @@ __global__ void __launch_bounds__(THREADS, 2) retrieve_kernel(const __grid_const
                     const uint32_t e = __ldcg(P.rlist + hx);
                     const int64_t bs = (int64_t)(e >> 16) * P.n_ret + (e & 0xFFFFu);
                     if (__ldcg(&P.hs[bs].n_cand) > (uint32_t)CAND_CAP)
-                        r_digit<G>(P, (int)(e >> 16), (int)(e & 0xFFFFu), pass, tid);
+                        if (pass == RP_REF0) r_digit<G, RP_REF0>(P, (int)(e >> 16), (int)(e & 0xFFFFu), tid);
+                        else if (pass == RP_REF1) r_digit<G, RP_REF1>(P, (int)(e >> 16), (int)(e & 0xFFFFu), tid);
+                        else if (pass == RP_REF2) r_digit<G, RP_REF2>(P, (int)(e >> 16), (int)(e & 0xFFFFu), tid);
+                        else r_digit<G, RP_REF3>(P, (int)(e >> 16), (int)(e & 0xFFFFu), tid);
                 }
             ok = gsync();
             if (tid == 0) trace_max(P, 8 + pass - RP_REF0);

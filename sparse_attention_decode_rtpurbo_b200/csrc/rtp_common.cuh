@@ -57,8 +57,6 @@ struct Sync {
     uint32_t barrier;          // grid barrier arrivals of the retrieval kernel
     uint32_t exit_count;
     uint32_t kb_work;          // groups left to the retrieval kernel (a select, or blocks to attend)
-    uint32_t pass_done[8];     // (unused)
-    uint32_t groups_ready;     // (unused)
     uint32_t any_global;       // some radix head's threshold bin is too large for the in-CTA select
     uint32_t pad[16];
 };

@@ -1278,8 +1278,6 @@ __global__ void __launch_bounds__(THREADS, 2) retrieve_kernel(const __grid_const
             P.sync->any_ties = 0;
             P.sync->barrier = 0;
             P.sync->kb_work = 0;
-            for (int i = 0; i < 8; ++i) P.sync->pass_done[i] = 0;
-            P.sync->groups_ready = 0;
             P.sync->any_global = 0;
             P.sync->exit_count = 0;
             __threadfence();

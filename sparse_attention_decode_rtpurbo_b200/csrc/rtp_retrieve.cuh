@@ -1278,6 +1278,13 @@ __global__ void __launch_bounds__(THREADS, 2) retrieve_kernel(const __grid_const
             P.sync->any_ties = 0;
             P.sync->barrier = 0;
             P.sync->kb_work = 0;
+            if (__ldcg(P.status) != 0) {
+                // an aborted call may leave select histograms behind
+                for (int64_t i = 0; i < (int64_t)P.B * P.n_ret * 256; ++i) {
+                    P.hist_cnt[i] = 0;
+                    P.hist_mass[i] = 0ull;
+                }
+            }
             P.sync->any_global = 0;
             P.sync->exit_count = 0;
             __threadfence();

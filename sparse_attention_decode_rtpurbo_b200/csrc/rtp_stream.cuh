@@ -363,17 +363,9 @@ __device__ __forceinline__ void decide_group(const KParams& K, ASmem<G>& S, int 
         }
     }
     const int bg = b * P.n_rg + rg;
-    if (any_radix) {
-        // the exact select starts from zero histograms and bitmaps
-        for (int hh = 0; hh < nh; ++hh) {
-            if (S.d_mode[hh] != MODE_RADIX) continue;
-            const int64_t bs = (int64_t)b * P.n_ret + slot0 + hh;
-            for (int x = tid; x < 256; x += CONSUMERS) {
-                P.hist_cnt[bs * 256 + x] = 0;
-                P.hist_mass[bs * 256 + x] = 0ull;
-            }
-        }
-    }
+    // (the exact select's histograms are zero already: they lie in the
+    // workspace region every call leaves at zero, the digit step clears each
+    // after reading it, and an aborted call clears them all)
     // bitmap words of the heads (read by the block-list builder of a group
     // with radix heads, and by the debug sink)
     if (any_radix || P.dbg_bitmap != nullptr) {

@@ -88,6 +88,41 @@ __device__ __forceinline__ void cta_share(long long T, int& t0, int& t1, int& na
     }
 }
 
+// The streaming kernel shares tile weight, not tiles: an index tile counts
+// W_SCORE, a local tile W_LOCAL.  Index tiles cost more (MMA scores, fold,
+// stored scores) and the group decision and best-token attention follow
+// the last index split, so index CTAs take fewer tiles and the two paths
+// end closer together.  Tile t's weight starts at tile_w0(t); a CTA's share
+// is a contiguous weight range, never shorter than one tile.
+constexpr int W_SCORE = 5, W_LOCAL = 4;
+__device__ __forceinline__ long long tile_w0(long long t, long long Ts) {
+    return t < Ts ? t * W_SCORE : Ts * W_SCORE + (t - Ts) * W_LOCAL;
+}
+// smallest t with tile_w0(t) >= w
+__device__ __forceinline__ long long first_tile_at(long long w, long long Ts) {
+    const long long ws = Ts * W_SCORE;
+    return w <= ws ? (w + W_SCORE - 1) / W_SCORE : Ts + (w - ws + W_LOCAL - 1) / W_LOCAL;
+}
+// This CTA's tiles [t0, t1) of Ts index and Tl local tiles over the first
+// nact CTAs: CTA c takes the tiles whose weight starts in
+// [c W / nact, (c + 1) W / nact).
+__device__ __forceinline__ void cta_wshare(long long Ts, long long Tl, int& t0, int& t1, int& nact) {
+    const long long W = Ts * W_SCORE + Tl * W_LOCAL;
+    const long long cap = W / W_SCORE;   // spans of at least W_SCORE: every CTA owns a tile
+    nact = (int)(cap < (long long)gridDim.x ? cap : (long long)gridDim.x);
+    if ((int)blockIdx.x < nact) {
+        t0 = (int)first_tile_at((long long)blockIdx.x * W / nact, Ts);
+        t1 = (int)first_tile_at((long long)(blockIdx.x + 1) * W / nact, Ts);
+    } else {
+        t0 = t1 = 0;
+    }
+}
+// the CTA owning tile t under cta_wshare
+__device__ __forceinline__ int cta_of_wtile(long long t, long long Ts, long long Tl, int nact) {
+    const long long W = Ts * W_SCORE + Tl * W_LOCAL;
+    return (int)(((tile_w0(t, Ts) + 1) * nact + W - 1) / W) - 1;
+}
+
 // A CTA's share: tiles [t, t1) of the sequence (index tiles, then local
 // tiles from tot_s on), then optionally local tiles [tot_s + l0, tot_s + l1);
 // item_t0 of a local item counts from the start of the local tiles.
@@ -803,9 +838,8 @@ __device__ __forceinline__ void a_consumers(const KParams& K, ASmem<G>& S, AWalk
                 float* part = P.lpart + ((int64_t)c + sg.item_idx) * G * PSTRIDE;
                 split_emit<G>(S.X, heads, part, nullptr, tid);
                 if (ticket_add(P.tick_local + sg.item_idx, (uint32_t)sg.ntiles, (uint32_t)sg.item_tiles, &S.flag)) {
-                    const long long T = (long long)S.tot_s + S.tot_l;
-                    const int c0 = cta_of_tile(S.tot_s + sg.item_t0, T, S.nact);
-                    const int c1 = cta_of_tile(S.tot_s + sg.item_t0 + sg.item_tiles - 1, T, S.nact);
+                    const int c0 = cta_of_wtile(S.tot_s + sg.item_t0, S.tot_s, S.tot_l, S.nact);
+                    const int c1 = cta_of_wtile(S.tot_s + sg.item_t0 + sg.item_tiles - 1, S.tot_s, S.tot_l, S.nact);
                     combine_splits<G>(S.X, P.lpart + ((int64_t)c0 + sg.item_idx) * G * PSTRIDE, c1 - c0 + 1, heads,
                                       out0, tid);
                     if (tid == 0) trace_max(P, 2);
@@ -895,13 +929,11 @@ __global__ void __launch_bounds__(THREADS, 2) stream_kernel(const __grid_constan
         }
     }
     __syncthreads();
-    // every CTA takes an equal, contiguous share of the index tiles of all
-    // retrieval groups, then one of the local tiles: the scores (and with
-    // them the selection) finish early, the local heads' streaming after
-    // them covers the decisions' latency
+    // every CTA takes a contiguous share of equal weight of the step's tiles
+    // (index tiles of all retrieval groups first, then the local tiles)
     AWalk wk;
     int nact;
-    cta_share((long long)S.tot_s + S.tot_l, wk.t, wk.t1, nact);
+    cta_wshare(S.tot_s, S.tot_l, wk.t, wk.t1, nact);
     wk.l0 = wk.l1 = 0;
     if (tid == 0) {
         S.nact = nact;

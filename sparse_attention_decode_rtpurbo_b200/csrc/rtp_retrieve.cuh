@@ -1,13 +1,18 @@
 // Retrieval kernel of the decode step (sm_100a), launched after the
-// streaming kernel:
-//   1. (only when some head needs it) the exact top-p select: an MSD radix
-//      select over the order-preserving u32 keys of the fp32 index scores,
-//      four passes of 256 bins of count and 2^-40 fixed-point softmax mass,
-//      scores recomputed from the index cache on the tensor cores; then the
-//      threshold ties (lowest indices first), block marking and the groups'
-//      block lists.  Passes are separated by grid barriers: the grid is one
-//      resident wave and no CTA of it depends on work that is not already
-//      running (the streaming kernel it follows never waits on it).
+// streaming kernel (programmatic dependent launch; it waits for that grid):
+//   1. (only when some head needs it) the exact top-p select over the fp32
+//      index scores the streaming kernel stored: a first pass bins smax - s
+//      (255 bins, count and 2^-40 fixed-point softmax mass), a 256-bin search
+//      picks the bin that completes ceil(p Z), a compaction pass gathers that
+//      bin's tokens and one CTA per head selects inside them (8-bit MSD
+//      digits over the order-preserving u32 keys, ties toward the lowest
+//      index); a bin of more than 4096 tokens takes four refine passes over
+//      all scores instead.  A mark pass sets block bits, one CTA per group
+//      builds its block list.  Each CTA holds its share of the scores in
+//      shared memory when it fits.  Passes are separated by grid barriers:
+//      the grid is one resident wave and no CTA of it depends on work that
+//      is not already running (the streaming kernel it follows never waits
+//      on it).
 //   2. block-sparse attention of the retrieval heads over their groups'
 //      block lists, split evenly over the CTAs (TMA-staged K/V, tensor
 //      cores), and the log-sum-exp combine of the splits.
@@ -211,10 +216,12 @@ __device__ __noinline__ void r_blist(const Params& P, int b, int rg, int tid);
 
 // One pass over the stored scores of this CTA's share of the radix groups'
 // 1024-token tiles (consumer threads; thread tid takes tokens n0 + tid + 128 u
-// of every radix head of the group at once).  At the end of each run of a
-// group's tiles the CTA folds its histograms into the heads' global ones;
-// per-head tickets elect the CTA that takes the head's next step (its digit,
-// its tie position, or, for the marks, the group's block list).
+// of one radix head's tile per item; items walk (tile, head) in order).  The
+// scores come from the stage buffers when the share is resident there, else
+// from global memory.  Histogram passes fold the CTA's shared histograms into
+// the heads' global ones at the end of each run of a group's tiles (and every
+// 64 tiles); the compaction and mark passes write candidates and bitmap bits.
+// The per-head steps between passes run after a grid barrier.
 template <int G, int pass>
 __device__ __noinline__ void r_pass(const Params& P, RWalk wk, const int* pre, int tid) {
     BSmem<G>& S = bsmem<G>();

@@ -1,5 +1,5 @@
 // Streaming kernel of the decode step (sm_100a): every CTA streams a
-// contiguous, equal share of the step's 32 KB tiles -- first the index-cache
+// contiguous share of equal weight of the step's 32 KB tiles -- first the index-cache
 // tiles of the retrieval groups (1024 tokens of k_idx each), then the K/V
 // tiles of the local heads' sink + window blocks -- through a shared-memory
 // ring fed by one copy warp (bulk copies for k_idx, 2-D TMA boxes with the

@@ -176,6 +176,19 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def max_over_ranks(values, world, device):
+    """Each rank's timings -> the maximum over the ranks, on every rank (the
+    replicas' device times; the whole job is as slow as its slowest rank)."""
+    import torch
+
+    vals = torch.tensor(list(values), dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+    return [float(v) for v in vals]
+
+
 def run_reference(args, rank):
     """The oracle (fp64 C, OpenMP over heads) on the host cores, same workload."""
     if rank != 0:
@@ -368,11 +381,9 @@ def main():
         raise SystemExit("device status set during the timed steps")
 
     # ---- max over ranks ----
-    vals = torch.tensor([t_ms, e2e_t] + [phase_ms[n] for n in rtp.PHASES], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
-    t_ms, e2e_t = float(vals[0]), float(vals[1])
-    phase_ms = {n: float(vals[2 + k]) for k, n in enumerate(rtp.PHASES)}
+    vals = max_over_ranks([t_ms, e2e_t] + [phase_ms[n] for n in rtp.PHASES], world, dev)
+    t_ms, e2e_t = vals[0], vals[1]
+    phase_ms = {n: vals[2 + k] for k, n in enumerate(rtp.PHASES)}
 
     tokens = float(case.seq_lens.sum())
     value = world * tokens / (t_ms * 1e-3)

@@ -420,6 +420,8 @@ def make_case(name: str, *, B: int, Hkv: int, G: int, seq_lens: Sequence[int], r
                 cnt = 0
                 plist, tlist = [], []
                 taken = set()
+                if hi - lo < len(aims) * n_needles:
+                    raise ValueError(f"needle range [{lo}, {hi}) holds fewer than {len(aims) * n_needles} positions")
                 for h in aims:
                     for i in range(n_needles):
                         while True:

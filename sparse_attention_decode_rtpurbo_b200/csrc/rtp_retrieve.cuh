@@ -1255,7 +1255,10 @@ __global__ void __launch_bounds__(THREADS, 2) retrieve_kernel(const __grid_const
         if (tid == 0) trace_max(P, 15);
         const long long T = pre[ngroups];
         int t0, t1, nact;
-        cta_share(T, t0, t1, nact);
+        // at least 4 tiles per CTA: with few tiles, a CTA of one tile pays a
+        // whole load latency and the group's last CTA combines one partial
+        // per tile
+        cta_share(T, t0, t1, nact, 4);
         if (copier) r_produce_attn<G>(K, S, pre, ngroups, t0, t1, T, nact, k, lane);
         else r_consume_attn<G>(K, S, k, tid);
         if (tid == 0) trace_max(P, 4);

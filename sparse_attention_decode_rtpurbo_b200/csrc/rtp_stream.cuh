@@ -76,10 +76,13 @@ __device__ __forceinline__ int cta_of_tile(long long t, long long T, int nact) {
     return (int)(((t + 1) * nact + T - 1) / T) - 1;
 }
 
-// This CTA's share [t0, t1) of T tiles over the first min(grid, T) CTAs
-// (nact of them).
-__device__ __forceinline__ void cta_share(long long T, int& t0, int& t1, int& nact) {
-    nact = (int)(T < (long long)gridDim.x ? T : (long long)gridDim.x);
+// This CTA's share [t0, t1) of T tiles over the first nact CTAs: min(grid,
+// T / min_per) of them (at least one when T > 0), so that a share holds at
+// least min_per tiles when there are few (and is never empty).
+__device__ __forceinline__ void cta_share(long long T, int& t0, int& t1, int& nact, int min_per = 1) {
+    long long want = T / min_per;
+    if (want < 1 && T > 0) want = 1;
+    nact = (int)(want < (long long)gridDim.x ? want : (long long)gridDim.x);
     if ((int)blockIdx.x < nact) {
         t0 = (int)((long long)blockIdx.x * T / nact);
         t1 = (int)((long long)(blockIdx.x + 1) * T / nact);

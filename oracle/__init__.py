@@ -52,6 +52,9 @@ def _L():
         lib.oracle_decode_step.argtypes = [i32, i32, i32, i64, vp, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32,
                                            i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, i64]
         lib.oracle_decode_step.restype = i32
+        lib.oracle_index_append.argtypes = [i32, i32, i64, vp, i32, vp, i32, vp, vp, vp]
+        lib.oracle_bf16_rne.argtypes = [dbl]
+        lib.oracle_bf16_rne.restype = ctypes.c_uint16
         _lib = lib
     return _lib
 
@@ -137,3 +140,32 @@ def decode_step(case, nthreads: int = 0) -> Dict[str, np.ndarray]:
                                  _p(res["kept_blocks"]), nblk)
     res["rc"] = rc
     return res
+
+
+def bf16_rne(x: float) -> int:
+    """The bf16 bit pattern nearest to x (ties to the even significand)."""
+    return int(_L().oracle_bf16_rne(float(x)))
+
+
+def index_append(k_pre: np.ndarray, Wk: np.ndarray, pos: np.ndarray, k_idx: np.ndarray,
+                 block_table: Optional[np.ndarray] = None) -> np.ndarray:
+    """k_idx rows pos[b] + t of KV head g <- bf16(W^K_g k^pre[b, g, t]).
+
+    k_pre: uint16 (bf16) [B, Hkv, T, 128]; Wk: uint16 [Hkv, 16, 128]; pos:
+    int32 [B]; k_idx: the cache, uint16, contiguous [B, Hkv, Ncap, 16] or,
+    with block_table int32 [B, max_blocks], paged [pages, Hkv, 64, 16].
+    Returns an updated copy of k_idx."""
+    k_pre = np.ascontiguousarray(k_pre, dtype=np.uint16)
+    Wk = np.ascontiguousarray(Wk, dtype=np.uint16)
+    pos = np.ascontiguousarray(pos, dtype=np.int32)
+    out = np.array(k_idx, dtype=np.uint16, copy=True, order="C")
+    B, Hkv, T = k_pre.shape[:3]
+    if block_table is None:
+        ncap, bt, mbps = out.shape[2], None, 0
+    else:
+        bt = np.ascontiguousarray(block_table, dtype=np.int32)
+        mbps = bt.shape[1]
+        ncap = mbps * BLK
+    _L().oracle_index_append(B, Hkv, ncap, _p(bt), mbps, _p(k_pre), T, _p(Wk), _p(pos), _p(out))
+    return out
+

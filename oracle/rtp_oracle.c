@@ -283,3 +283,56 @@ int oracle_decode_step(int B, int Hq, int Hkv, int64_t Ncap, const int32_t* bloc
     }
     return bad ? 6 : 0;
 }
+
+/*
+ * Index-cache append (the step before the decode hot path): for each new
+ * token t of sequence b and each KV head g,
+ *     k_idx[b, g, pos_b + t] = bf16( W^K_g k^pre[b, g, t] )
+ * (review, Method: "Adaptive sparse attention" -- the retrieval key
+ * k^idx_n = W^K_h k^pre_n, kept as a 16-dim bf16 cache; W^K is per KV head
+ * under GQA).  The dot product is taken in fp64 from the exact bf16 upcasts,
+ * summed in index order, then rounded once to bf16.
+ */
+
+/* nearest bf16 to x, ties to the even significand: bf16 keeps the sign, the
+ * 8 exponent bits and the top 7 fraction bits of an IEEE binary32. */
+static uint16_t bf16_rne(double x) {
+    if (isnan(x)) return 0x7FC0;
+    uint16_t sign = signbit(x) ? 0x8000 : 0;
+    double a = fabs(x);
+    if (a == 0.0) return sign;
+    int e;
+    double m = frexp(a, &e);                 /* a = m 2^e, 0.5 <= m < 1 */
+    int be = e - 1 + 127;                    /* biased exponent of a normal bf16 */
+    if (be >= 1) {
+        double q = nearbyint(ldexp(m, 8));   /* 8 significant bits: 128 .. 256 */
+        if (q == 256.0) {
+            q = 128.0;
+            be += 1;
+        }
+        if (be >= 255) return (uint16_t)(sign | 0x7F80);   /* overflow: infinity */
+        return (uint16_t)(sign | (be << 7) | ((int)q - 128));
+    }
+    /* subnormal: multiples of 2^-133 */
+    double q = nearbyint(ldexp(a, 133));
+    return (uint16_t)(sign | (int)q);        /* q = 128 lands on the smallest normal */
+}
+
+void oracle_index_append(int B, int Hkv, int64_t Ncap, const int32_t* block_table, int mbps, const uint16_t* k_pre,
+                         int T, const uint16_t* Wk, const int32_t* pos, uint16_t* k_idx) {
+    geom g = {B, Hkv, Hkv, Ncap, block_table, mbps};
+    for (int b = 0; b < B; ++b)
+        for (int kv = 0; kv < Hkv; ++kv)
+            for (int t = 0; t < T; ++t) {
+                const uint16_t* kp = k_pre + (((int64_t)b * Hkv + kv) * T + t) * ORC_D;
+                uint16_t* dst = (uint16_t*)row(&g, k_idx, ORC_R, b, kv, (int64_t)pos[b] + t);
+                for (int r = 0; r < ORC_R; ++r) {
+                    const uint16_t* w = Wk + ((int64_t)kv * ORC_R + r) * ORC_D;
+                    double acc = 0.0;
+                    for (int i = 0; i < ORC_D; ++i) acc += bf(w[i]) * bf(kp[i]);
+                    dst[r] = bf16_rne(acc);
+                }
+            }
+}
+
+uint16_t oracle_bf16_rne(double x) { return bf16_rne(x); }

@@ -377,3 +377,126 @@ def test_invalid_p_is_an_error():
     c = synth.workload(1, scale=4)
     c.p[:] = 0.0
     assert oracle.decode_step(c)["rc"] == 6
+
+
+# ---------------------------------------------------------------------------
+# index-cache append: k_idx_n = bf16(W^K_g k^pre_n)
+# ---------------------------------------------------------------------------
+def _bf16_exact_rne(v):
+    """Nearest bf16 bits of the exact rational v, ties to even: written from
+    the format (sign, 8-bit exponent, 7 stored fraction bits), independent of
+    the oracle's C rounding."""
+    from fractions import Fraction
+
+    v = Fraction(v)
+    if v == 0:
+        return 0
+    sign = 0x8000 if v < 0 else 0
+    a = abs(v)
+    e = a.numerator.bit_length() - a.denominator.bit_length()
+    while Fraction(2) ** e > a:
+        e -= 1
+    while Fraction(2) ** (e + 1) <= a:
+        e += 1                                   # 2^e <= a < 2^(e+1)
+    if e < -126:                                 # subnormal: multiples of 2^-133
+        q, rem = divmod(a * 2 ** 133, 1)
+        q = int(q) + (1 if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and int(q) % 2) else 0)
+        return sign | q
+    q, rem = divmod(a / Fraction(2) ** e * 128, 1)  # 128 <= q < 256
+    q = int(q) + (1 if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and int(q) % 2) else 0)
+    if q == 256:
+        q, e = 128, e + 1
+    if e + 127 >= 255:
+        return sign | 0x7F80
+    return sign | ((e + 127) << 7) | (q - 128)
+
+
+def _bf16_value(b):
+    from fractions import Fraction
+
+    s = -1 if b & 0x8000 else 1
+    ex, fr = (b >> 7) & 0xFF, b & 0x7F
+    if ex == 0:
+        return s * Fraction(fr) * Fraction(2) ** -133
+    return s * (128 + fr) * Fraction(2) ** (ex - 127 - 7)
+
+
+def test_bf16_rounding_ties_to_even_and_edges():
+    assert oracle.bf16_rne(1.0) == 0x3F80
+    assert oracle.bf16_rne(1 + 2 ** -8) == 0x3F80          # halfway 1 | 1+2^-7: the even one
+    assert oracle.bf16_rne(1 + 3 * 2 ** -8) == 0x3F82      # halfway 1+2^-7 | 1+2^-6: the even one
+    assert oracle.bf16_rne(1 + 2 ** -8 + 2 ** -30) == 0x3F81
+    assert oracle.bf16_rne(-2.5) == 0xC020
+    assert oracle.bf16_rne(2.0 ** -133) == 0x0001          # smallest subnormal
+    assert oracle.bf16_rne(2.0 ** -126) == 0x0080          # smallest normal
+    assert oracle.bf16_rne(3.5e38) == 0x7F80               # beyond the largest finite: infinity
+    rng = np.random.default_rng(7)
+    xs = np.concatenate([rng.standard_normal(2000) * 10.0 ** rng.integers(-40, 38, 2000),
+                         rng.standard_normal(500)])
+    for x in xs:
+        assert oracle.bf16_rne(float(x)) == _bf16_exact_rne(float(x)), x
+
+
+def _append_case(seed, B=2, Hkv=3, T=5, ncap=64, paged=False):
+    rng = np.random.default_rng(seed)
+    k_pre = synth.to_bf16(rng.standard_normal((B, Hkv, T, 128)))
+    Wk = synth.to_bf16(rng.standard_normal((Hkv, 16, 128)) / np.sqrt(128))
+    pos = rng.integers(0, ncap - T + 1, B).astype(np.int32)
+    if paged:
+        mbps = ncap // 64
+        pages = rng.permutation(B * mbps).astype(np.int32)
+        bt = pages.reshape(B, mbps)
+        cache = rng.integers(0, 2 ** 16, (B * mbps, Hkv, 64, 16)).astype(np.uint16)
+    else:
+        bt = None
+        cache = rng.integers(0, 2 ** 16, (B, Hkv, ncap, 16)).astype(np.uint16)
+    return k_pre, Wk, pos, cache, bt
+
+
+def _row(cache, bt, b, g, n):
+    if bt is None:
+        return cache[b, g, n]
+    return cache[bt[b, n // 64], g, n % 64]
+
+
+@pytest.mark.parametrize("paged", [False, True])
+def test_index_append_exact_dot_and_untouched_rows(paged):
+    """Brute force in exact rationals: every written row is the nearest bf16
+    of the exact dot product; every other row keeps its old bits."""
+    from fractions import Fraction
+
+    k_pre, Wk, pos, cache, bt = _append_case(3, paged=paged, ncap=128)
+    out = oracle.index_append(k_pre, Wk, pos, cache, block_table=bt)
+    B, Hkv, T = k_pre.shape[:3]
+    written = set()
+    for b in range(B):
+        for g in range(Hkv):
+            for t in range(T):
+                n = int(pos[b]) + t
+                written.add((b, g, n))
+                got = _row(out, bt, b, g, n)
+                for r in range(16):
+                    exact = sum(_bf16_value(int(Wk[g, r, i])) * _bf16_value(int(k_pre[b, g, t, i]))
+                                for i in range(128))
+                    assert int(got[r]) == _bf16_exact_rne(exact), (b, g, t, r)
+    ncap = 128
+    for b in range(B):
+        for g in range(Hkv):
+            for n in range(ncap):
+                if (b, g, n) not in written:
+                    assert np.array_equal(_row(out, bt, b, g, n), _row(cache, bt, b, g, n))
+
+
+def test_index_append_identity_projection_copies_inputs():
+    """W^K = [I_16 | 0]: the cache row is the first 16 entries of k^pre, bit
+    for bit (bf16 values are exact in fp64 and round to themselves)."""
+    k_pre, Wk, pos, cache, bt = _append_case(5)
+    Wk = np.zeros_like(Wk)
+    one = synth.to_bf16(np.ones(1))[0]
+    for r in range(16):
+        Wk[:, r, r] = one
+    out = oracle.index_append(k_pre, Wk, pos, cache)
+    for b in range(k_pre.shape[0]):
+        for g in range(k_pre.shape[1]):
+            for t in range(k_pre.shape[2]):
+                assert np.array_equal(out[b, g, pos[b] + t], k_pre[b, g, t, :16])

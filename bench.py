@@ -45,6 +45,8 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--dense", action="store_true", help="p = 1 for every sequence (dense comparator)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--op", choices=["decode", "append"], default="decode",
+                    help="append: time the index-cache append instead of the decode step")
     return ap.parse_args()
 
 
@@ -65,10 +67,11 @@ PROFILED = {"stream": ("profiles/stream_kernel_w4_1m.md", "w4-1m"),
 
 
 def kernel_source_hash():
-    import glob
+    """Hash of the sources that define the two profiled kernels (the decode
+    step's streaming and retrieval kernels and the helpers they include)."""
     import hashlib
-    pkg = os.path.join(ROOT, "sparse_attention_decode_rtpurbo_b200")
-    files = sorted(glob.glob(os.path.join(pkg, "csrc", "*.cu*"))) + [os.path.join(ROOT, "include", "rtp_decode.h")]
+    csrc = os.path.join(ROOT, "sparse_attention_decode_rtpurbo_b200", "csrc")
+    files = [os.path.join(csrc, f) for f in ("rtp_common.cuh", "rtp_attn.cuh", "rtp_stream.cuh", "rtp_retrieve.cuh")]
     h = hashlib.sha256()
     for p in files:
         h.update(os.path.basename(p).encode())
@@ -220,8 +223,50 @@ def run_reference(args, rank):
     print(json.dumps(line), flush=True)
 
 
+def bench_append(args):
+    """rtp_index_append alone: a decode-sized append (one new token for each
+    of 16 sequences x 8 KV heads) and a 32K-token chunk of one sequence; HBM
+    bytes = k_pre read (256 B) + k_idx written (32 B) per token and KV head
+    (W^K, 32 KB, stays in L2).  L2 flushed before every timed call."""
+    import torch
+
+    import sparse_attention_decode_rtpurbo_b200 as rtp
+
+    dev = torch.device("cuda", 0)
+    flush_w = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    peak, peak_kind = hbm_peak()
+    for name, B, Hkv, T, ncap in [("decode 16x8 heads x 1 token", 16, 8, 1, 65536),
+                                  ("chunk 1x8 heads x 32768 tokens", 1, 8, 32768, 65536)]:
+        g = torch.Generator(device=dev).manual_seed(1)
+        k_pre = torch.randn((B, Hkv, T, 128), generator=g, device=dev).to(torch.bfloat16)
+        Wk = (torch.randn((Hkv, 16, 128), generator=g, device=dev) / 11.3).to(torch.bfloat16)
+        pos = torch.zeros(B, dtype=torch.int32, device=dev)
+        cache = torch.zeros((B, Hkv, ncap, 16), dtype=torch.bfloat16, device=dev)
+        dims = rtp.make_dims(B, Hkv, Hkv, ncap)
+        stream = torch.cuda.current_stream()
+        ts = []
+        for i in range(args.warmup + args.steps):
+            flush_w.zero_()
+            a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            rtp.index_append(dims, k_pre, Wk, pos, T, cache, None, stream)
+            z.record(stream)
+            z.synchronize()
+            if i >= args.warmup:
+                ts.append(a.elapsed_time(z))
+        t_ms = statistics.median(ts)
+        nbytes = B * Hkv * T * (256 + 32)
+        gbs = nbytes / (t_ms * 1e-3) / 1e9
+        print(json.dumps({"metric": "index-cache append (rtp_index_append)", "op": "append", "case": name,
+                          "value": gbs, "unit": "GB/s", "us_per_call": t_ms * 1e3, "bytes": nbytes,
+                          "peak": peak, "frac": gbs / peak, "peak_source": peak_kind, "steps": args.steps,
+                          "warmup": args.warmup, "l2": "flushed (256 MB write) before every call"}), flush=True)
+
+
 def main():
     args = parse()
+    if args.op == "append":
+        return bench_append(args)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

@@ -209,6 +209,46 @@ rtp_status rtp_decode_step_noalloc(const rtp_dims* dims, const uint16_t* q_pre, 
                                    uint32_t* device_status, void* stream);
 
 /* Static string naming a status code. */
+/*
+ * rtp_index_append -- write the retrieval keys of new tokens into the index
+ * cache that rtp_decode_step reads (the step before the decode hot path).
+ *
+ * Source: "Full Attention Strikes Back" (RTPurbo) review, Method: "Adaptive
+ * sparse attention": the retrieval key k^idx_n = W^K k^pre_n, a rank-16
+ * projection of the pre-RoPE key kept as a 16-dim bf16 cache; W^K is per KV
+ * head under GQA.
+ *
+ * For every sequence b < batch, KV head g < num_kv_heads and new token
+ * t < num_new:
+ *     k_idx row (b, g, pos[b] + t) = bf16( W^K[g] (16 x 128) . k_pre[b, g, t] )
+ * each of the 16 entries the fp64 sum, in index order, of the 128 exact
+ * products of bf16 values, rounded once to bf16 (round to nearest even).
+ *
+ *   dims     : batch, num_kv_heads, head_dim 128, idx_dim 16, block_size 64,
+ *              max_seq_len (the cache capacity, a multiple of 64) and, for a
+ *              paged cache, block_table / max_blocks_per_seq / num_pages as for
+ *              rtp_decode_step.  num_q_heads, workspace, debug and timing
+ *              fields are not used.
+ *   k_pre    : device bf16 [batch, num_kv_heads, num_new, 128], 16-byte aligned.
+ *   Wk_idx   : device bf16 [num_kv_heads, 16, 128], 16-byte aligned.
+ *   pos      : device int32 [batch]: the cache row of each sequence's first
+ *              new token (its current length, for an append).
+ *   num_new  : new tokens per sequence (0: nothing is enqueued).
+ *   k_idx    : device bf16 index cache, contiguous [batch, num_kv_heads,
+ *              max_seq_len, 16] or paged [num_pages, num_kv_heads, 64, 16]
+ *              (page id = block_table[b, n / 64]), 8-byte aligned; only the
+ *              rows above are written.  Owned by the caller.
+ *   device_status : optional device uint32: a row outside [0, max_seq_len)
+ *              or a page id outside [0, num_pages) is skipped and sets it to
+ *              RTP_ERR_DEVICE_INPUT if it was 0.  NULL: not reported.
+ *   stream   : the cudaStream_t the kernel is enqueued on.
+ * Returns RTP_OK, or RTP_ERR_NULL / RTP_ERR_SHAPE / RTP_ERR_UNSUPPORTED
+ * (unaligned k_pre, Wk_idx or k_idx, sizes beyond the limits of rtp_dims) before
+ * anything is enqueued, or RTP_ERR_CUDA if the launch failed.
+ */
+rtp_status rtp_index_append(const rtp_dims* dims, const uint16_t* k_pre, const uint16_t* Wk_idx, const int32_t* pos,
+                            int32_t num_new, uint16_t* k_idx, uint32_t* device_status, void* stream);
+
 const char* rtp_status_string(rtp_status status);
 
 #ifdef __cplusplus

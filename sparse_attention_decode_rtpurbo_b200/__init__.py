@@ -75,6 +75,8 @@ def _load():
                                           vp, vp]
     L.rtp_decode_step_noalloc.restype = ctypes.c_int
     L.rtp_get_status.argtypes = [ctypes.POINTER(RtpDims), vp]
+    L.rtp_index_append.argtypes = [ctypes.POINTER(RtpDims), vp, vp, vp, i32, vp, vp, vp]
+    L.rtp_index_append.restype = ctypes.c_int
     L.rtp_get_status.restype = ctypes.c_int
     L.rtp_status_string.argtypes = [ctypes.c_int]
     L.rtp_status_string.restype = ctypes.c_char_p
@@ -145,6 +147,18 @@ def decode_step_noalloc(dims: RtpDims, q_pre, q_rope, k_idx, k_cache, v_cache, W
                                      int(window), int(sink), _ptr(out), _ptr(device_status), st)
     if rc != RTP_OK:
         raise RtpError(rc, "rtp_decode_step_noalloc")
+
+
+def index_append(dims: RtpDims, k_pre, Wk_idx, pos, num_new: int, k_idx, device_status=None, stream=None) -> None:
+    """rtp_index_append: rows pos[b] + t of the index cache k_idx receive
+    bf16(W^K[g] . k_pre[b, g, t]) for the num_new new tokens of every sequence
+    (dims gives the cache geometry).  device_status: optional device uint32
+    tensor set to RTP_ERR_DEVICE_INPUT by a row or page id out of range."""
+    st = 0 if stream is None else (stream if isinstance(stream, int) else stream.cuda_stream)
+    rc = lib.rtp_index_append(ctypes.byref(dims), _ptr(k_pre), _ptr(Wk_idx), _ptr(pos), int(num_new), _ptr(k_idx),
+                              _ptr(device_status), st)
+    if rc != RTP_OK:
+        raise RtpError(rc, "rtp_index_append")
 
 
 def get_status(dims: RtpDims, stream=None) -> int:

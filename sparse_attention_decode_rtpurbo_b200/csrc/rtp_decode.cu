@@ -16,6 +16,7 @@
 
 #include "../../include/rtp_decode.h"
 #include "rtp_retrieve.cuh"
+#include "rtp_append.cuh"
 
 namespace rtp {
 
@@ -477,6 +478,45 @@ extern "C" rtp_status rtp_decode_step_noalloc(const rtp_dims* dims, const uint16
         cudaMemcpyAsync(device_status, ws + pl.o_status, sizeof(uint32_t), cudaMemcpyDeviceToDevice, s) != cudaSuccess)
         return RTP_ERR_CUDA;
     return RTP_OK;
+}
+
+// ---------------------------------------------------------------------------
+// index-cache append
+// ---------------------------------------------------------------------------
+extern "C" rtp_status rtp_index_append(const rtp_dims* d, const uint16_t* k_pre, const uint16_t* Wk_idx,
+                                       const int32_t* pos, int32_t num_new, uint16_t* k_idx, uint32_t* device_status,
+                                       void* stream) {
+    if (!d) return RTP_ERR_NULL;
+    if (d->head_dim != D || d->idx_dim != R || d->block_size != BLK) return RTP_ERR_UNSUPPORTED;
+    if (d->batch < 1 || d->num_kv_heads < 1 || num_new < 0) return RTP_ERR_SHAPE;
+    if (d->batch > MAX_B || d->num_kv_heads > MAX_HKV) return RTP_ERR_UNSUPPORTED;
+    if (d->max_seq_len < BLK || d->max_seq_len % BLK || num_new > d->max_seq_len) return RTP_ERR_SHAPE;
+    if (d->block_table) {
+        if (d->max_blocks_per_seq < 1 || d->num_pages < 1) return RTP_ERR_SHAPE;
+        if ((int64_t)d->max_blocks_per_seq * BLK != d->max_seq_len) return RTP_ERR_SHAPE;
+    }
+    if (num_new == 0) return RTP_OK;
+    if (!k_pre || !Wk_idx || !pos || !k_idx) return RTP_ERR_NULL;
+    if (((uintptr_t)k_pre | (uintptr_t)Wk_idx) & 15u) return RTP_ERR_UNSUPPORTED;   // 16-byte vector loads
+    if ((uintptr_t)k_idx & 7u) return RTP_ERR_UNSUPPORTED;                            // 8-byte stores of 4 entries
+    AppendParams A;
+    A.B = d->batch;
+    A.Hkv = d->num_kv_heads;
+    A.T = num_new;
+    A.Ncap = d->max_seq_len;
+    A.mbps = d->block_table ? d->max_blocks_per_seq : 0;
+    A.num_pages = d->block_table ? d->num_pages : 0;
+    A.k_pre = k_pre;
+    A.Wk = Wk_idx;
+    A.pos = pos;
+    A.block_table = d->block_table;
+    A.k_idx = k_idx;
+    A.status = device_status;
+    const int64_t total = (int64_t)A.B * A.Hkv * A.T * (R / APPEND_ROWS);
+    const int64_t grid = (total + APPEND_THREADS - 1) / APPEND_THREADS;
+    if (grid > 0x7FFFFFFF) return RTP_ERR_UNSUPPORTED;
+    index_append_kernel<<<(unsigned)grid, APPEND_THREADS, 0, (cudaStream_t)stream>>>(A);
+    return report(cudaGetLastError(), "index append launch") == cudaSuccess ? RTP_OK : RTP_ERR_CUDA;
 }
 
 extern "C" const char* rtp_status_string(rtp_status status) {

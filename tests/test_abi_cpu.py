@@ -89,3 +89,19 @@ def test_status_strings():
     assert "unknown" in rtp.status_string(99)
     with pytest.raises(rtp.RtpError):
         rtp.decode_step(dims(), 1, 1, 1, 1, 1, 1, 1, HK, 1, 64, 4, 1)
+
+
+def test_index_append_host_side_checks():
+    """rtp_index_append: bad arguments are refused before any CUDA call."""
+    fake = 4096   # never dereferenced: every call below returns first
+    d = dims()
+    call = lambda dd, *a: rtp.lib.rtp_index_append(ctypes.byref(dd) if dd is not None else None, *a)
+    assert call(None, fake, fake, fake, 1, fake, None, None) == 1                      # NULL dims
+    assert call(d, None, fake, fake, 1, fake, None, None) == 1                         # NULL k_pre
+    assert call(d, fake, fake, fake, 0, fake, None, None) == 0                         # nothing to append
+    assert call(d, fake, fake, fake, -1, fake, None, None) == 2                        # negative count
+    assert call(d, fake, fake, fake, 4097, fake, None, None) == 2                      # more than the capacity
+    assert call(dims(max_seq_len=100), fake, fake, fake, 1, fake, None, None) == 2     # capacity not a multiple of 64
+    assert call(d, fake + 2, fake, fake, 1, fake, None, None) == 3                     # k_pre not 16-byte aligned
+    assert call(d, fake, fake, fake, 1, fake + 4, None, None) == 3                     # k_idx not 8-byte aligned
+    assert call(dims(num_kv_heads=65, num_q_heads=65), fake, fake, fake, 1, fake, None, None) == 3

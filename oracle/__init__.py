@@ -53,6 +53,11 @@ def _L():
                                            i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, i64]
         lib.oracle_decode_step.restype = i32
         lib.oracle_index_append.argtypes = [i32, i32, i64, vp, i32, vp, i32, vp, vp, vp]
+        lib.oracle_topk.argtypes = [vp, i64, i64, vp, vp]
+        lib.oracle_topk.restype = i32
+        lib.oracle_decode_step_topk.argtypes = [i32, i32, i32, i64, vp, i32, vp, vp, vp, vp, vp, vp, vp, vp, i64, i32,
+                                                i32, i32, vp, vp, vp, vp, i64]
+        lib.oracle_decode_step_topk.restype = i32
         lib.oracle_bf16_rne.argtypes = [dbl]
         lib.oracle_bf16_rne.restype = ctypes.c_uint16
         _lib = lib
@@ -86,6 +91,19 @@ def topp(s: np.ndarray, p: float) -> Dict[str, object]:
         raise ValueError(f"oracle_topp rc={rc}")
     return {"order": order, "kstar": int(k.value), "kept": np.sort(order[:k.value]), "zmax": zm.value, "Z": Z.value,
             "cum_before": cb.value, "cum_at": ca.value}
+
+
+def topk(s: np.ndarray, k: int) -> Dict[str, object]:
+    """Static Top-K on raw index scores s: the first min(k, L) tokens under
+    (s desc, n asc)."""
+    s = np.ascontiguousarray(s, dtype=np.float64)
+    L = s.size
+    order = np.empty(L, dtype=np.int64)
+    kk = ctypes.c_int64()
+    rc = _L().oracle_topk(_p(s), L, int(k), _p(order), ctypes.byref(kk))
+    if rc != 0:
+        raise ValueError(f"oracle_topk rc={rc}")
+    return {"order": order, "kstar": int(kk.value), "kept": np.sort(order[:kk.value])}
 
 
 def _geom(case):
@@ -138,6 +156,27 @@ def decode_step(case, nthreads: int = 0) -> Dict[str, np.ndarray]:
                                  int(nthreads), _p(res["out"]), _p(res["kstar"]), _p(res["tau"]), _p(res["zmax"]),
                                  _p(res["Z"]), _p(res["cum_before"]), _p(res["cum_at"]), _p(res["next_s"]),
                                  _p(res["kept_blocks"]), nblk)
+    res["rc"] = rc
+    return res
+
+
+def decode_step_topk(case, k: int, nthreads: int = 0) -> Dict[str, np.ndarray]:
+    """The decode step with every retrieval head keeping its static top-k
+    (case.p unused).  Returns out, kstar, tau and kept_blocks."""
+    B, Hq, Hkv, Ncap, bt, mbps = _geom(case)
+    nblk = (Ncap + BLK - 1) // BLK
+    res = {
+        "out": np.zeros((B, Hq, D), dtype=np.float64),
+        "kstar": np.zeros((B, Hq), dtype=np.int64),
+        "tau": np.full((B, Hq), np.nan),
+        "kept_blocks": np.zeros((B, Hq, nblk), dtype=np.uint8),
+    }
+    hk = np.ascontiguousarray(case.head_kind, dtype=np.uint8)
+    rc = _L().oracle_decode_step_topk(B, Hq, Hkv, Ncap, _p(bt), mbps, _p(case.q_pre), _p(case.q_rope),
+                                      _p(case.k_idx), _p(case.k_cache), _p(case.v_cache), _p(case.Wq_idx),
+                                      _p(np.ascontiguousarray(case.seq_lens, dtype=np.int32)), _p(hk), int(k),
+                                      int(case.window), int(case.sink), int(nthreads), _p(res["out"]),
+                                      _p(res["kstar"]), _p(res["tau"]), _p(res["kept_blocks"]), nblk)
     res["rc"] = rc
     return res
 

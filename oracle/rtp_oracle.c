@@ -141,6 +141,28 @@ int oracle_topp(const double* s, int64_t L, double p, int64_t* order, int64_t* k
     return 0;
 }
 
+/*
+ * Static Top-K (the pages' fixed-budget ablation, k = 4096 in the review's
+ * comparison of top-k against top-p): the k highest index scores, ties
+ * toward the lower index -- the first min(k, L) tokens under (s desc, n asc).
+ * Outputs order[0..L) and *kstar = min(k, L).
+ */
+int oracle_topk(const double* s, int64_t L, int64_t K, int64_t* order, int64_t* kstar_out) {
+    if (L <= 0) return 2;
+    if (K < 1) return 6;
+    scored* v = (scored*)malloc(sizeof(scored) * (size_t)L);
+    for (int64_t n = 0; n < L; ++n) {
+        v[n].s = s[n];
+        v[n].n = n;
+    }
+    qsort(v, (size_t)L, sizeof(scored), by_score_then_index);
+    if (order)
+        for (int64_t i = 0; i < L; ++i) order[i] = v[i].n;
+    free(v);
+    if (kstar_out) *kstar_out = K < L ? K : L;
+    return 0;
+}
+
 /* index scores s_n = (W^Q_h q^pre) . k_idx_n for n < L (fp64) */
 static void index_scores(const geom* g, const uint16_t* q_pre, const uint16_t* Wq, const uint16_t* k_idx, int b,
                          int h, int64_t L, double* s) {
@@ -222,12 +244,14 @@ static int64_t local_positions(int64_t L, int window, int sink, int64_t* pos) {
  *   next_s (score of token k*+1 in the order, NaN when k* = L),
  *   kept_blocks [B,Hq,nblk_cap] (1 = block kept).
  */
-int oracle_decode_step(int B, int Hq, int Hkv, int64_t Ncap, const int32_t* block_table, int mbps,
+/* the decode step; topk > 0 selects each retrieval head's static top-k
+ * (p unused) instead of its dynamic top-p */
+static int decode_step(int B, int Hq, int Hkv, int64_t Ncap, const int32_t* block_table, int mbps,
                        const uint16_t* q_pre, const uint16_t* q_rope, const uint16_t* k_idx, const uint16_t* k_cache,
                        const uint16_t* v_cache, const uint16_t* Wq_idx, const int32_t* seq_lens,
-                       const uint8_t* head_kind, const float* p, int window, int sink, int nthreads, double* out,
-                       int64_t* kstar, double* tau, double* zmax, double* Z, double* cum_before, double* cum_at,
-                       double* next_s, uint8_t* kept_blocks, int64_t nblk_cap) {
+                       const uint8_t* head_kind, const float* p, int64_t topk, int window, int sink, int nthreads,
+                       double* out, int64_t* kstar, double* tau, double* zmax, double* Z, double* cum_before,
+                       double* cum_at, double* next_s, uint8_t* kept_blocks, int64_t nblk_cap) {
     geom g = {B, Hq, Hkv, Ncap, block_table, mbps};
     int bad = 0;
 #ifdef _OPENMP
@@ -246,7 +270,7 @@ int oracle_decode_step(int B, int Hq, int Hkv, int64_t Ncap, const int32_t* bloc
             np = local_positions(L, window, sink, pos);
             if (kstar) kstar[bh] = np;
         } else {
-            double pb = (double)p[b];
+            double pb = topk > 0 ? 1.0 : (double)p[b];
             if (!(pb > 0.0)) {
                 bad = 1;
                 free(pos);
@@ -258,6 +282,7 @@ int oracle_decode_step(int B, int Hq, int Hkv, int64_t Ncap, const int32_t* bloc
             int64_t k;
             double zm, Zs, cb, ca;
             oracle_topp(s, L, pb, order, &k, &zm, &Zs, &cb, &ca);
+            if (topk > 0) oracle_topk(s, L, topk, order, &k);   /* same order, count k */
             uint8_t* keep = (uint8_t*)calloc((size_t)((L + ORC_BLK - 1) / ORC_BLK), 1);
             for (int64_t i = 0; i < k; ++i) keep[order[i] / ORC_BLK] = 1;
             for (int64_t n = 0; n < L; ++n)
@@ -282,6 +307,30 @@ int oracle_decode_step(int B, int Hq, int Hkv, int64_t Ncap, const int32_t* bloc
         free(pos);
     }
     return bad ? 6 : 0;
+}
+
+int oracle_decode_step(int B, int Hq, int Hkv, int64_t Ncap, const int32_t* block_table, int mbps,
+                       const uint16_t* q_pre, const uint16_t* q_rope, const uint16_t* k_idx, const uint16_t* k_cache,
+                       const uint16_t* v_cache, const uint16_t* Wq_idx, const int32_t* seq_lens,
+                       const uint8_t* head_kind, const float* p, int window, int sink, int nthreads, double* out,
+                       int64_t* kstar, double* tau, double* zmax, double* Z, double* cum_before, double* cum_at,
+                       double* next_s, uint8_t* kept_blocks, int64_t nblk_cap) {
+    return decode_step(B, Hq, Hkv, Ncap, block_table, mbps, q_pre, q_rope, k_idx, k_cache, v_cache, Wq_idx, seq_lens,
+                       head_kind, p, 0, window, sink, nthreads, out, kstar, tau, zmax, Z, cum_before, cum_at, next_s,
+                       kept_blocks, nblk_cap);
+}
+
+/* the same step with every retrieval head keeping its static top-k (k >= 1) */
+int oracle_decode_step_topk(int B, int Hq, int Hkv, int64_t Ncap, const int32_t* block_table, int mbps,
+                            const uint16_t* q_pre, const uint16_t* q_rope, const uint16_t* k_idx,
+                            const uint16_t* k_cache, const uint16_t* v_cache, const uint16_t* Wq_idx,
+                            const int32_t* seq_lens, const uint8_t* head_kind, int64_t topk, int window, int sink,
+                            int nthreads, double* out, int64_t* kstar, double* tau, uint8_t* kept_blocks,
+                            int64_t nblk_cap) {
+    if (topk < 1) return 6;
+    return decode_step(B, Hq, Hkv, Ncap, block_table, mbps, q_pre, q_rope, k_idx, k_cache, v_cache, Wq_idx, seq_lens,
+                       head_kind, NULL, topk, window, sink, nthreads, out, kstar, tau, NULL, NULL, NULL, NULL, NULL,
+                       kept_blocks, nblk_cap);
 }
 
 /*

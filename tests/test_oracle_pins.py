@@ -500,3 +500,66 @@ def test_index_append_identity_projection_copies_inputs():
         for g in range(k_pre.shape[1]):
             for t in range(k_pre.shape[2]):
                 assert np.array_equal(out[b, g, pos[b] + t], k_pre[b, g, t, :16])
+
+
+# ---------------------------------------------------------------------------
+# static top-k (the fixed-budget variant): the k highest scores, ties low index
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("seed", range(12))
+def test_topk_brute_force_dominance(seed):
+    """Brute force on tiny inputs: among all subsets of size min(k, L) exactly
+    one has every member beat every non-member under (s desc, n asc), and it
+    is the oracle's."""
+    rng = np.random.default_rng(seed)
+    L = int(rng.integers(1, 11))
+    s = rng.integers(-3, 4, L).astype(np.float64)       # integer scores: many ties
+    k = int(rng.integers(1, L + 3))
+    beats = lambda a, b: s[a] > s[b] or (s[a] == s[b] and a < b)
+    m = min(k, L)
+    winners = [set(c) for c in itertools.combinations(range(L), m)
+               if all(beats(a, b) for a in c for b in range(L) if b not in c)]
+    assert len(winners) == 1
+    r = oracle.topk(s, k)
+    assert r["kstar"] == m
+    assert set(r["kept"].tolist()) == winners[0]
+
+
+def test_topk_closed_forms():
+    # all scores equal: the first k indices
+    r = oracle.topk(np.zeros(1000), 300)
+    assert r["kept"].tolist() == list(range(300))
+    # k = 1: the maximum, lowest index among equal maxima
+    s = np.array([1.0, 5.0, 2.0, 5.0, -1.0])
+    assert oracle.topk(s, 1)["kept"].tolist() == [1]
+    # k >= L keeps everything
+    assert oracle.topk(s, 99)["kstar"] == 5
+    with pytest.raises(ValueError):
+        oracle.topk(s, 0)
+
+
+def test_topk_step_with_k_at_least_L_is_dense():
+    """k >= L keeps every token: the step equals the top-p step with p = 1."""
+    case = synth.workload(1)
+    dense = case.__class__(**{**case.__dict__})
+    dense.p = np.ones_like(case.p)
+    a = oracle.decode_step_topk(case, 1 << 20)
+    b = oracle.decode_step(dense)
+    assert a["rc"] == 0 and b["rc"] == 0
+    ret = np.nonzero(case.head_kind)[0]
+    assert np.array_equal(a["kept_blocks"][:, ret], b["kept_blocks"][:, ret])
+    assert np.max(np.abs(a["out"] - b["out"])) < 1e-12
+
+
+def test_topk_step_keeps_the_blocks_of_its_k_best():
+    """The step's kept blocks are the blocks of the k best tokens of each
+    retrieval head (scores recomputed independently by index_scores)."""
+    case = synth.workload(1)
+    k = 200
+    r = oracle.decode_step_topk(case, k)
+    assert r["rc"] == 0
+    for h in np.nonzero(case.head_kind)[0]:
+        s = oracle.index_scores(case, 0, h)[: int(case.seq_lens[0])]
+        best = sorted(range(s.size), key=lambda n: (-s[n], n))[:k]
+        blocks = sorted({n // 64 for n in best})
+        assert np.nonzero(r["kept_blocks"][0, h])[0].tolist() == blocks
+        assert r["kstar"][0, h] == k

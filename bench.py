@@ -106,7 +106,7 @@ def workload_config(case, wl):
 
 
 def algorithmic_bytes(case, kept):
-    """North-star byte count of one step: index cache of every retrieval KV
+    """Algorithmic byte count of one step (the roofline numerator): index cache of every retrieval KV
     group + the union of kept K/V blocks per retrieval group (rows < L) +
     sink/window rows of every local KV group.  512 B per K+V row, 32 B per
     index row."""
@@ -464,7 +464,7 @@ def main():
             "warmup": args.warmup, "ms_per_step": t_ms, "us_per_step": t_ms * 1e3,
             "us_per_step_p10_p90": [float(np.percentile(step_ms, 10)) * 1e3, float(np.percentile(step_ms, 90)) * 1e3],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16 in, fp32 accumulate",
-            "data": "synthetic (seeded; see DESIGN.md input recipe)",
+            "data": "synthetic (seeded generators in synth/, shaped like the pages' workloads)",
             "config": dict(workload_config(case, args.workload), parallelism=f"replicas x{world}",
                            dense_p1=bool(args.dense), timing="CUDA-graph replay of one rtp_decode_step (2 kernels, programmatic launch) per step; "
                            "CUDA events on the launching stream"),

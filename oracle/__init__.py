@@ -53,6 +53,7 @@ def _L():
                                            i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, i64]
         lib.oracle_decode_step.restype = i32
         lib.oracle_index_append.argtypes = [i32, i32, i64, vp, i32, vp, i32, vp, vp, vp]
+        lib.oracle_kv_append.argtypes = [i32, i32, i64, vp, i32, vp, vp, i32, vp, vp, vp, vp, vp, vp, vp]
         lib.oracle_topk.argtypes = [vp, i64, i64, vp, vp]
         lib.oracle_topk.restype = i32
         lib.oracle_decode_step_topk.argtypes = [i32, i32, i32, i64, vp, i32, vp, vp, vp, vp, vp, vp, vp, vp, i64, i32,
@@ -179,6 +180,37 @@ def decode_step_topk(case, k: int, nthreads: int = 0) -> Dict[str, np.ndarray]:
                                       _p(res["kstar"]), _p(res["tau"]), _p(res["kept_blocks"]), nblk)
     res["rc"] = rc
     return res
+
+
+def kv_append(k_pre: np.ndarray, v_new: np.ndarray, Wk: np.ndarray, rope_cos: np.ndarray, rope_sin: np.ndarray,
+              pos: np.ndarray, k_idx: np.ndarray, k_cache: np.ndarray, v_cache: np.ndarray,
+              block_table: Optional[np.ndarray] = None):
+    """The KV-cache write of new tokens with the index-cache append: rows
+    n = pos[b] + t of KV head g get k_idx = bf16(W^K_g k^pre), k_cache =
+    bf16(RoPE_n(k^pre)) (pairs (i, i+64) rotated by rope_cos/rope_sin row n,
+    fp32 [positions, 64]) and v_cache = v_new.  k_pre, v_new: uint16 (bf16)
+    [B, Hkv, T, 128]; caches contiguous [B, Hkv, Ncap, dim] or, with
+    block_table, paged [pages, Hkv, 64, dim].  Returns updated copies
+    (k_idx, k_cache, v_cache)."""
+    k_pre = np.ascontiguousarray(k_pre, dtype=np.uint16)
+    v_new = np.ascontiguousarray(v_new, dtype=np.uint16)
+    Wk = np.ascontiguousarray(Wk, dtype=np.uint16)
+    rc = np.ascontiguousarray(rope_cos, dtype=np.float32)
+    rs = np.ascontiguousarray(rope_sin, dtype=np.float32)
+    pos = np.ascontiguousarray(pos, dtype=np.int32)
+    outs = [np.array(a, dtype=np.uint16, copy=True, order="C") for a in (k_idx, k_cache, v_cache)]
+    B, Hkv, T = k_pre.shape[:3]
+    if block_table is None:
+        ncap, bt, mbps = outs[0].shape[2], None, 0
+    else:
+        bt = np.ascontiguousarray(block_table, dtype=np.int32)
+        mbps = bt.shape[1]
+        ncap = mbps * BLK
+    if int(pos.min()) < 0 or int(pos.max()) + T > ncap or rc.shape != rs.shape or rc.shape[0] < ncap:
+        raise ValueError("kv_append: positions beyond the cache or the angle table")
+    _L().oracle_kv_append(B, Hkv, ncap, _p(bt), mbps, _p(k_pre), _p(v_new), T, _p(Wk), _p(rc), _p(rs), _p(pos),
+                          _p(outs[0]), _p(outs[1]), _p(outs[2]))
+    return tuple(outs)
 
 
 def bf16_rne(x: float) -> int:

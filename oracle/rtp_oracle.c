@@ -384,4 +384,46 @@ void oracle_index_append(int B, int Hkv, int64_t Ncap, const int32_t* block_tabl
             }
 }
 
+/*
+ * KV-cache write of new tokens, with the index-cache append in the same step:
+ * for each new token t of sequence b, at cache position n = pos_b + t, and
+ * each KV head g,
+ *     k_idx[b, g, n]   = bf16( W^K_g k^pre )          (as oracle_index_append)
+ *     k_cache[b, g, n] = bf16( RoPE_n(k^pre) )
+ *     v_cache[b, g, n] = v[b, g, t]                   (bits copied)
+ * The indexer reads keys before RoPE and the attention after it (review,
+ * Method: "Adaptive sparse attention" -- s_h from W^Q q^pre and W^K k^pre,
+ * exact attention on the RoPE'd q and k; Insight 2: RoPE rotates each
+ * frequency pair by an angle proportional to the position).  RoPE_n rotates
+ * the pairs (i, i + 64), i < 64, by the caller's angle table, row n:
+ *     y_i      = k_i cos_{n,i} - k_{i+64} sin_{n,i}
+ *     y_{i+64} = k_{i+64} cos_{n,i} + k_i sin_{n,i}
+ * (cos, sin: fp32 [positions, 64]).  A product of a bf16 and an fp32 value
+ * is exact in fp64; each y is the two products' sum rounded once to fp64
+ * (a fused multiply-add onto the exact second product), then to bf16.
+ */
+void oracle_kv_append(int B, int Hkv, int64_t Ncap, const int32_t* block_table, int mbps, const uint16_t* k_pre,
+                      const uint16_t* v_new, int T, const uint16_t* Wk, const float* rope_cos, const float* rope_sin,
+                      const int32_t* pos, uint16_t* k_idx, uint16_t* k_cache, uint16_t* v_cache) {
+    geom g = {B, Hkv, Hkv, Ncap, block_table, mbps};
+    oracle_index_append(B, Hkv, Ncap, block_table, mbps, k_pre, T, Wk, pos, k_idx);
+    for (int b = 0; b < B; ++b)
+        for (int kv = 0; kv < Hkv; ++kv)
+            for (int t = 0; t < T; ++t) {
+                const int64_t n = (int64_t)pos[b] + t;
+                const int64_t src = (((int64_t)b * Hkv + kv) * T + t) * ORC_D;
+                const uint16_t* kp = k_pre + src;
+                const float* c = rope_cos + n * 64;
+                const float* sn = rope_sin + n * 64;
+                uint16_t* kd = (uint16_t*)row(&g, k_cache, ORC_D, b, kv, n);
+                uint16_t* vd = (uint16_t*)row(&g, v_cache, ORC_D, b, kv, n);
+                for (int i = 0; i < 64; ++i) {
+                    const double lo = bf(kp[i]), hi = bf(kp[i + 64]);
+                    kd[i] = bf16_rne(fma(lo, (double)c[i], -(hi * (double)sn[i])));
+                    kd[i + 64] = bf16_rne(fma(hi, (double)c[i], lo * (double)sn[i]));
+                }
+                memcpy(vd, v_new + src, ORC_D * sizeof(uint16_t));
+            }
+}
+
 uint16_t oracle_bf16_rne(double x) { return bf16_rne(x); }

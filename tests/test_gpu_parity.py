@@ -124,6 +124,19 @@ def test_device_input_errors_set_status():
     dc.seq_lens[0] = 300
     dc.run()
     assert dc.step.status() == 0
+    ref = oracle.decode_step(case)
+    for bad in (0, -7):
+        # an empty or negative length is an input error too; the other
+        # sequence's outputs are still those of the oracle
+        dc.seq_lens[0] = bad
+        dc.out.zero_()
+        dc.run()
+        assert dc.step.status() == 6
+        got = dc.out.float().cpu().numpy()[1]
+        assert np.all(np.abs(got - ref["out"][1]) <= 4e-3 + 1e-2 * np.abs(ref["out"][1]))
+    dc.seq_lens[0] = 300
+    dc.run()
+    assert dc.step.status() == 0
 
 
 def test_bad_page_id_sets_status():

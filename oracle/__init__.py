@@ -57,7 +57,7 @@ def _L():
         lib.oracle_ring_row.argtypes = [i64, i32, i32]
         lib.oracle_ring_row.restype = i64
         lib.oracle_ring_write.argtypes = [i32, i32, i32, i32, vp, vp, i32, vp, vp, vp]
-        lib.oracle_attend_ring.argtypes = [i32, i32, i32, i32, i32, vp, vp, vp, i32, i32, i64, i32, vp]
+        lib.oracle_attend_ring.argtypes = [i32, i32, i32, i32, i32, vp, vp, vp, i32, i32, i64, i32, i32, vp]
         lib.oracle_attend_ring.restype = i32
         lib.oracle_topk.argtypes = [vp, i64, i64, vp, vp]
         lib.oracle_topk.restype = i32
@@ -218,14 +218,14 @@ def kv_append(k_pre: np.ndarray, v_new: np.ndarray, Wk: np.ndarray, rope_cos: np
     return tuple(outs)
 
 
-def ring_row(n: int, sink: int, W: int) -> int:
-    """Row of position n in a local head's ring of sink + W rows."""
-    return int(_L().oracle_ring_row(int(n), int(sink), int(W)))
+def ring_row(n: int, S0: int, W: int) -> int:
+    """Row of position n in a local head's ring of S0 + W rows."""
+    return int(_L().oracle_ring_row(int(n), int(S0), int(W)))
 
 
 def ring_write(k_new: np.ndarray, v_new: np.ndarray, pos: np.ndarray, k_ring: np.ndarray, v_ring: np.ndarray,
-               sink: int, W: int):
-    """Rings [B, Hkv, sink + W, 128] (uint16 bf16) after writing the new rows
+               S0: int, W: int):
+    """Rings [B, Hkv, S0 + W, 128] (uint16 bf16) after writing the new rows
     [B, Hkv, T, 128] of positions pos[b] + t in order.  Returns updated copies."""
     k_new = np.ascontiguousarray(k_new, dtype=np.uint16)
     v_new = np.ascontiguousarray(v_new, dtype=np.uint16)
@@ -233,25 +233,26 @@ def ring_write(k_new: np.ndarray, v_new: np.ndarray, pos: np.ndarray, k_ring: np
     kr = np.array(k_ring, dtype=np.uint16, copy=True, order="C")
     vr = np.array(v_ring, dtype=np.uint16, copy=True, order="C")
     B, Hkv, T = k_new.shape[:3]
-    if kr.shape != (B, Hkv, sink + W, D) or vr.shape != kr.shape or W < 1 or sink < 0 or int(pos.min()) < 0:
-        raise ValueError("ring_write: ring shape, W, sink or positions")
-    _L().oracle_ring_write(B, Hkv, sink, W, _p(k_new), _p(v_new), T, _p(pos), _p(kr), _p(vr))
+    if kr.shape != (B, Hkv, S0 + W, D) or vr.shape != kr.shape or W < 1 or S0 < 0 or int(pos.min()) < 0:
+        raise ValueError("ring_write: ring shape, W, S0 or positions")
+    _L().oracle_ring_write(B, Hkv, S0, W, _p(k_new), _p(v_new), T, _p(pos), _p(kr), _p(vr))
     return kr, vr
 
 
 def attend_ring(q_rope: np.ndarray, k_ring: np.ndarray, v_ring: np.ndarray, b: int, h: int, L: int, window: int,
-                sink: int, W: int) -> np.ndarray:
-    """Local head h of sequence b at length L, its keys and values read from
-    the rings (window <= W)."""
+                sink: int, S0: int, W: int) -> np.ndarray:
+    """Local head h of sequence b at length L (sink <= S0, window <= W), its
+    keys and values read from the rings."""
     q = np.ascontiguousarray(q_rope, dtype=np.uint16)
     kr = np.ascontiguousarray(k_ring, dtype=np.uint16)
     vr = np.ascontiguousarray(v_ring, dtype=np.uint16)
     B, Hq = q.shape[:2]
     Hkv = kr.shape[1]
     out = np.empty(D, dtype=np.float64)
-    rc = _L().oracle_attend_ring(B, Hq, Hkv, sink, W, _p(q), _p(kr), _p(vr), b, h, int(L), int(window), _p(out))
+    rc = _L().oracle_attend_ring(B, Hq, Hkv, S0, W, _p(q), _p(kr), _p(vr), b, h, int(L), int(window), int(sink),
+                                 _p(out))
     if rc != 0:
-        raise ValueError("attend_ring: window larger than the ring's W")
+        raise ValueError("attend_ring: sink beyond S0 or window beyond W")
     return out
 
 

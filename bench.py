@@ -109,7 +109,9 @@ def algorithmic_bytes(case, kept):
     """Algorithmic byte count of one step (the roofline numerator): index cache of every retrieval KV
     group + the union of kept K/V blocks per retrieval group (rows < L) +
     sink/window rows of every local KV group.  512 B per K+V row, 32 B per
-    index row."""
+    index row.  A KV group with both kinds of heads counts the union of the
+    rows it reads once (its sink/window rows inside kept blocks are not
+    counted again under "local")."""
     import synth
 
     G = case.G
@@ -120,15 +122,16 @@ def algorithmic_bytes(case, kept):
         rows = np.minimum(64, L - 64 * np.arange(nblk))
         for g in range(case.Hkv):
             heads = range(g * G, (g + 1) * G)
+            uni = np.zeros(nblk, dtype=bool)
             if any(case.head_kind[h] for h in heads):
                 idx += L * 32
-                uni = np.zeros(nblk, dtype=bool)
                 for h in heads:
                     if case.head_kind[h]:
                         uni |= kept[b, h, :nblk].astype(bool)
                 kv += int(rows[uni].sum()) * 512
             if any(not case.head_kind[h] for h in heads):
-                loc += synth.local_positions(L, case.window, case.sink).size * 512
+                pos = synth.local_positions(L, case.window, case.sink)
+                loc += int(np.count_nonzero(~uni[pos // 64])) * 512
     return {"index": idx, "kept_kv": kv, "local": loc, "total": idx + kv + loc}
 
 

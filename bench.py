@@ -111,13 +111,14 @@ def algorithmic_bytes(case, kept):
     """Algorithmic byte count of one step (the roofline numerator): index cache of every retrieval KV
     group + the union of kept K/V blocks per retrieval group (rows < L) +
     sink/window rows of every local KV group.  512 B per K+V row, 32 B per
-    index row.  A KV group with both kinds of heads counts the union of the
-    rows it reads once (its sink/window rows inside kept blocks are not
-    counted again under "local")."""
+    index row.  "local" counts every sink/window row (the streaming kernel
+    reads them all); a KV group with both kinds of heads reads some rows for
+    both ("shared": its sink/window rows inside kept blocks), and the step's
+    total counts those once."""
     import synth
 
     G = case.G
-    idx = kv = loc = 0
+    idx = kv = loc = shared = 0
     for b in range(case.B):
         L = int(case.seq_lens[b])
         nblk = (L + 63) // 64
@@ -133,8 +134,9 @@ def algorithmic_bytes(case, kept):
                 kv += int(rows[uni].sum()) * 512
             if any(not case.head_kind[h] for h in heads):
                 pos = synth.local_positions(L, case.window, case.sink)
-                loc += int(np.count_nonzero(~uni[pos // 64])) * 512
-    return {"index": idx, "kept_kv": kv, "local": loc, "total": idx + kv + loc}
+                loc += pos.size * 512
+                shared += int(np.count_nonzero(uni[pos // 64])) * 512
+    return {"index": idx, "kept_kv": kv, "local": loc, "shared": shared, "total": idx + kv + loc - shared}
 
 
 class ClockSampler:

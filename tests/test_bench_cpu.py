@@ -49,6 +49,7 @@ def test_algorithmic_bytes_by_hand():
     assert got["index"] == 200 * 32
     assert got["kept_kv"] == (64 + 8) * 512
     assert got["local"] == (4 + 50) * 512     # sink 0..3 and window 150..199
+    assert got["shared"] == 0
     assert got["total"] == got["index"] + got["kept_kv"] + got["local"]
 
     # one KV group with both kinds: heads 0 (retrieval) and 1 (local)
@@ -58,6 +59,8 @@ def test_algorithmic_bytes_by_hand():
     kept = np.zeros((1, 2, case.Ncap // 64), np.uint8)
     kept[0, 0, [0, 2]] = 1                   # blocks 0 (rows 0..63) and 2 (rows 128..191)
     got = bench.algorithmic_bytes(case, kept)
-    # local rows: sink 0..3 (in block 0: already read), window 150..191 (in block 2: read), 192..199 (new)
+    # local rows: sink 0..3 (in block 0), window 150..191 (in block 2), 192..199 (in no kept block)
     assert got["kept_kv"] == 128 * 512
-    assert got["local"] == 8 * 512
+    assert got["local"] == (4 + 50) * 512
+    assert got["shared"] == (4 + 42) * 512
+    assert got["total"] == got["index"] + (128 + 8) * 512

@@ -874,3 +874,38 @@ def test_oracle_results_do_not_depend_on_the_thread_count():
     c = oracle.decode_step_topk(case, 100, nthreads=1)
     d = oracle.decode_step_topk(case, 100, nthreads=8)
     assert np.array_equal(c["out"], d["out"]) and np.array_equal(c["kept_blocks"], d["kept_blocks"])
+
+
+@pytest.mark.parametrize("paged", [False, True])
+def test_generator_poisons_every_row_no_head_may_read(paged):
+    """The parity inputs' NaN rows: rows >= L of every KV head, the whole index
+    cache of local-only KV heads and their K/V outside the sink and window are
+    NaN; every row some head may read is finite.  (A stray read on the GPU
+    then shows up as a non-finite output.)"""
+    case = synth.make_case("poison", B=2, Hkv=3, G=2, seq_lens=[700, 130], ret_groups=[0], p=[0.9, 0.9],
+                           window=100, sink=4, seed=12, regimes=["gaussian", "gaussian"], paged=paged)
+    nan_k, nan_v, nan_i = (np.isnan(synth.from_bf16(a)).all(axis=-1) for a in (case.k_cache, case.v_cache,
+                                                                             case.k_idx))
+    fin_k, fin_v, fin_i = (np.isfinite(synth.from_bf16(a)).all(axis=-1) for a in (case.k_cache, case.v_cache,
+                                                                                case.k_idx))
+
+    def row(arr, b, g, n):
+        return arr[b, g, n] if case.block_table is None else arr[case.block_table[b, n // 64], g, n % 64]
+
+    for b in range(case.B):
+        L = int(case.seq_lens[b])
+        local = set(range(min(4, L))) | set(range(max(0, L - 100), L))
+        # paged: only mapped blocks have rows (-1 = no page)
+        nrows = case.Ncap if case.block_table is None else int(np.count_nonzero(case.block_table[b] >= 0)) * 64
+        for g in range(case.Hkv):
+            retrieval = g == 0
+            for n in range(nrows):
+                readable_kv = n < L and (retrieval or n in local)
+                readable_idx = n < L and retrieval
+                assert row(fin_k if readable_kv else nan_k, b, g, n), (b, g, n, "k")
+                assert row(fin_v if readable_kv else nan_v, b, g, n), (b, g, n, "v")
+                assert row(fin_i if readable_idx else nan_i, b, g, n), (b, g, n, "k_idx")
+    if case.block_table is not None:
+        unmapped = sorted(set(range(case.num_pages)) - set(case.block_table[case.block_table >= 0].tolist()))
+        for pg in unmapped:
+            assert nan_k[pg].all() and nan_v[pg].all() and nan_i[pg].all(), pg

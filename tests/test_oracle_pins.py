@@ -909,3 +909,17 @@ def test_generator_poisons_every_row_no_head_may_read(paged):
         unmapped = sorted(set(range(case.num_pages)) - set(case.block_table[case.block_table >= 0].tolist()))
         for pg in unmapped:
             assert nan_k[pg].all() and nan_v[pg].all() and nan_i[pg].all(), pg
+
+
+def test_regimes_keep_the_fractions_the_recipe_states():
+    """The input recipe's regimes, measured by the oracle on the 4 x 128K
+    workload (reduced 8x): needle-peaked sequences keep one token per head,
+    the diffuse one ~15 % of its tokens on average over heads, the plain
+    Gaussian one (p = 0.95) ~60-80 %."""
+    case = synth.workload(3, scale=8)
+    ref = oracle.decode_step(case)
+    ret = np.nonzero(case.head_kind)[0]
+    frac = [ref["kstar"][b, ret] / int(case.seq_lens[b]) for b in range(case.B)]
+    assert np.all(ref["kstar"][0, ret] == 1) and np.all(ref["kstar"][1, ret] == 1)      # needle, needle
+    assert 0.10 <= frac[2].mean() <= 0.20                                               # diffuse
+    assert 0.60 <= frac[3].mean() <= 0.80                                               # gaussian

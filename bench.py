@@ -44,6 +44,8 @@ def parse():
     ap.add_argument("--scale", type=int, default=1, help="divide the workload's context lengths (profiling runs)")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--dense", action="store_true", help="p = 1 for every sequence (dense comparator)")
+    ap.add_argument("--topk", type=int, default=0,
+                    help="static top-k selection with this k (the fixed-budget variant) instead of top-p")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--op", choices=["decode", "append"], default="decode",
                     help="append: time the index-cache append instead of the decode step")
@@ -192,6 +194,10 @@ def max_over_ranks(values, world, device):
     return [float(v) for v in vals]
 
 
+def selection_name(args):
+    return f"static top-k, k={args.topk}" if args.topk > 0 else ("top-p, p=1 (dense)" if args.dense else "top-p")
+
+
 def run_reference(args, rank):
     """The oracle (fp64 C, OpenMP over heads) on the host cores, same workload."""
     if rank != 0:
@@ -203,12 +209,19 @@ def run_reference(args, rank):
     if args.dense:
         case.p[:] = 1.0
     cores = os.cpu_count() or 1
+
+    def step():
+        if args.topk > 0:
+            oracle.decode_step_topk(case, args.topk, nthreads=cores)
+        else:
+            oracle.decode_step(case, nthreads=cores)
+
     for _ in range(args.warmup):
-        oracle.decode_step(case, nthreads=cores)
+        step()
     ts = []
     for _ in range(args.steps):
         t0 = time.perf_counter()
-        oracle.decode_step(case, nthreads=cores)
+        step()
         ts.append(time.perf_counter() - t0)
     t = statistics.mean(ts)
     tokens = float(case.seq_lens.sum())
@@ -216,7 +229,7 @@ def run_reference(args, rank):
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": workload_config(case, args.workload),
+            "config": dict(workload_config(case, args.workload), selection=selection_name(args)),
             "cpu_baseline": {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
                              "sample": f"whole decode step of the workload per timed step ({args.steps} steps)"},
             "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -296,6 +309,7 @@ def main():
     if args.dense:
         case.p[:] = 1.0
     dc = DeviceCase(case, device=dev, debug=True)
+    dc.topk = max(0, args.topk)
     stream = torch.cuda.current_stream(dev)
 
     # one debug step: kept blocks for the algorithmic byte count
@@ -403,7 +417,8 @@ def main():
     hlens = torch.from_numpy(case.seq_lens.astype(np.int32)).pin_memory()
     hp = torch.from_numpy(case.p.astype(np.float32)).pin_memory()
     hout = torch.empty(dc.out.shape, dtype=torch.bfloat16).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in (hq_pre, hq_rope, hlens, hp))
+    h_in = (hq_pre, hq_rope, hlens) if dc.topk > 0 else (hq_pre, hq_rope, hlens, hp)   # (top-k takes no p)
+    h2d = sum(t.numel() * t.element_size() for t in h_in)
     d2h = hout.numel() * hout.element_size()
     e2e_ms = []
     for i in range(max(3, args.warmup) + args.steps):
@@ -414,7 +429,8 @@ def main():
         dc.q_pre.copy_(hq_pre, non_blocking=True)
         dc.q_rope.copy_(hq_rope, non_blocking=True)
         dc.seq_lens.copy_(hlens, non_blocking=True)
-        dc.p.copy_(hp, non_blocking=True)
+        if dc.topk == 0:
+            dc.p.copy_(hp, non_blocking=True)
         graph.replay()
         hout.copy_(dc.out, non_blocking=True)
         z.record(stream)
@@ -451,10 +467,16 @@ def main():
             import oracle
 
             cores = os.cpu_count() or 1
-            oracle.decode_step(case, nthreads=cores)
+            def oracle_step():
+                if args.topk > 0:
+                    oracle.decode_step_topk(case, args.topk, nthreads=cores)
+                else:
+                    oracle.decode_step(case, nthreads=cores)
+
+            oracle_step()
             reps, t0 = 0, time.perf_counter()
             while time.perf_counter() - t0 < 10.0 and reps < 50:
-                oracle.decode_step(case, nthreads=cores)
+                oracle_step()
                 reps += 1
             tc = (time.perf_counter() - t0) / reps
             cpu = {"value": tokens / tc, "unit": UNIT, "cores": cores, "kind": "oracle",
@@ -466,12 +488,13 @@ def main():
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16 in, fp32 accumulate",
             "data": "synthetic (seeded generators in synth/, shaped like the pages' workloads)",
             "config": dict(workload_config(case, args.workload), parallelism=f"replicas x{world}",
-                           dense_p1=bool(args.dense), timing="CUDA-graph replay of one rtp_decode_step (2 kernels, programmatic launch) per step; "
+                           dense_p1=bool(args.dense), selection=selection_name(args), timing="CUDA-graph replay of one rtp_decode_step (2 kernels, programmatic launch) per step; "
                            "CUDA events on the launching stream"),
             "wall_s_timed_loop": wall,
             "roofline": {"bound": "hbm", "kernel": f"rtp::{dom}_kernel", "achieved": ach, "peak": peak, "unit": "GB/s",
                          "frac": ach / peak, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, burst)",
-                         "traffic": profiled_traffic(dom, case.name), "algorithmic_bytes_per_launch": kbytes[dom],
+                         "traffic": profiled_traffic(dom, case.name) if selection_name(args) == "top-p" else None,
+                         "algorithmic_bytes_per_launch": kbytes[dom],
                          "us_per_launch": phase_ms[dom] * 1e3},
             "step_roofline": {"algorithmic_bytes": nbytes, "achieved": step_gbs, "peak": peak, "unit": "GB/s",
                               "frac": step_gbs / peak},

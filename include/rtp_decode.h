@@ -159,6 +159,28 @@ rtp_status rtp_decode_step(const rtp_dims* dims, const uint16_t* q_pre, const ui
                            const float* p, int32_t window, int32_t sink, uint16_t* out, void* stream);
 
 /*
+ * rtp_decode_step_topk -- the decode step with the static top-k selection in
+ * place of dynamic top-p: every retrieval head keeps its min(topk, L) best
+ * tokens under the order (score descending, token index ascending), widened
+ * to 64-token blocks, and attends over them exactly as rtp_decode_step does.
+ * Local heads are unchanged.  This is the fixed-budget variant that the
+ * paper's experiments compare against (review on dongryeollee1.github.io,
+ * Experiments: the static top-k baseline at k = 4096; Method, "Insight 3":
+ * a fixed budget against a query-dependent one).
+ *
+ * Arguments are those of rtp_decode_step, with p replaced by
+ *   topk: tokens kept per retrieval head, >= 1 (the same for every sequence
+ *     and head); topk >= L keeps every block of that sequence, topk = 1 keeps
+ *     the block of the best-scoring token (lowest index among equal maxima).
+ * Returns RTP_ERR_SHAPE for topk < 1; every other check, the workspace and
+ * the error behaviour are those of rtp_decode_step (same workspace size).
+ */
+rtp_status rtp_decode_step_topk(const rtp_dims* dims, const uint16_t* q_pre, const uint16_t* q_rope,
+                                const uint16_t* k_idx, const uint16_t* k_cache, const uint16_t* v_cache,
+                                const uint16_t* Wq_idx, const int32_t* seq_lens, const uint8_t* head_kind,
+                                int32_t topk, int32_t window, int32_t sink, uint16_t* out, void* stream);
+
+/*
  * Synchronises `stream`, returns the first device-side error recorded in the
  * workspace since the last call to this function (RTP_OK if none) and clears
  * it.  For tests and debugging; it blocks the host.

@@ -71,6 +71,8 @@ def _load():
     L.rtp_workspace_size.restype = ctypes.c_size_t
     L.rtp_decode_step.argtypes = [ctypes.POINTER(RtpDims), vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, vp, vp]
     L.rtp_decode_step.restype = ctypes.c_int
+    L.rtp_decode_step_topk.argtypes = [ctypes.POINTER(RtpDims), vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, vp, vp]
+    L.rtp_decode_step_topk.restype = ctypes.c_int
     L.rtp_decode_step_noalloc.argtypes = [ctypes.POINTER(RtpDims), vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, vp,
                                           vp, vp]
     L.rtp_decode_step_noalloc.restype = ctypes.c_int
@@ -127,6 +129,18 @@ def decode_step(dims: RtpDims, q_pre, q_rope, k_idx, k_cache, v_cache, Wq_idx, s
                              int(window), int(sink), _ptr(out), st)
     if rc != RTP_OK:
         raise RtpError(rc, "rtp_decode_step")
+
+
+def decode_step_topk(dims: RtpDims, q_pre, q_rope, k_idx, k_cache, v_cache, Wq_idx, seq_lens, head_kind, topk: int,
+                     window: int, sink: int, out, stream=None) -> None:
+    """rtp_decode_step_topk: the decode step with every retrieval head keeping
+    its static top-k tokens (topk >= 1) instead of the dynamic top-p set."""
+    st = 0 if stream is None else (stream if isinstance(stream, int) else stream.cuda_stream)
+    rc = lib.rtp_decode_step_topk(ctypes.byref(dims), _ptr(q_pre), _ptr(q_rope), _ptr(k_idx), _ptr(k_cache),
+                                  _ptr(v_cache), _ptr(Wq_idx), _ptr(seq_lens), _head_kind_buf(head_kind), int(topk),
+                                  int(window), int(sink), _ptr(out), st)
+    if rc != RTP_OK:
+        raise RtpError(rc, "rtp_decode_step_topk")
 
 
 # RTP_NOALLOC_SCRATCH_BYTES of the C header: the static scratch of rtp_decode_step_noalloc
@@ -191,6 +205,10 @@ class Step:
     def __call__(self, q_pre, q_rope, k_idx, k_cache, v_cache, Wq_idx, seq_lens, p, window, sink, out, stream=None):
         decode_step(self.dims, q_pre, q_rope, k_idx, k_cache, v_cache, Wq_idx, seq_lens, self.head_kind, p, window,
                     sink, out, stream)
+
+    def topk(self, q_pre, q_rope, k_idx, k_cache, v_cache, Wq_idx, seq_lens, topk, window, sink, out, stream=None):
+        decode_step_topk(self.dims, q_pre, q_rope, k_idx, k_cache, v_cache, Wq_idx, seq_lens, self.head_kind, topk,
+                         window, sink, out, stream)
 
     def status(self, stream=None) -> int:
         return get_status(self.dims, stream)

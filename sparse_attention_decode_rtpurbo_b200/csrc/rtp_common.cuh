@@ -87,7 +87,8 @@ struct Params {
     const uint16_t *q_pre, *q_rope, *k_idx, *Wq;
     const uint16_t *k_cache_ptr, *v_cache_ptr;   // the caches as plain pointers (the kernels read them through TMA maps)
     const int32_t *seq_lens, *block_table;
-    const float* p;
+    const float* p;   // top-p mass per sequence (unused, may be null, under static top-k)
+    int topk;         // 0: dynamic top-p; k >= 1: every retrieval head keeps its k best tokens
     uint16_t* out;
     HeadTab tab;
     // workspace

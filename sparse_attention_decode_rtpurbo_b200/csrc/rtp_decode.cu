@@ -284,13 +284,17 @@ extern "C" size_t rtp_workspace_size(const rtp_dims* dims, const uint8_t* head_k
 
 static bool aligned16(const void* p) { return ((uintptr_t)p & 15) == 0; }
 
-extern "C" rtp_status rtp_decode_step(const rtp_dims* dims, const uint16_t* q_pre, const uint16_t* q_rope,
-                                      const uint16_t* k_idx, const uint16_t* k_cache, const uint16_t* v_cache,
-                                      const uint16_t* Wq_idx, const int32_t* seq_lens, const uint8_t* head_kind,
-                                      const float* p, int32_t window, int32_t sink, uint16_t* out, void* stream) {
-    if (!dims || !q_pre || !q_rope || !k_idx || !k_cache || !v_cache || !Wq_idx || !seq_lens || !head_kind || !p ||
-        !out)
+// The decode step with a caller workspace: dynamic top-p (p, topk = 0) or
+// static top-k (topk >= 1, p unused).
+static rtp_status decode_step_ws(const rtp_dims* dims, const uint16_t* q_pre, const uint16_t* q_rope,
+                                 const uint16_t* k_idx, const uint16_t* k_cache, const uint16_t* v_cache,
+                                 const uint16_t* Wq_idx, const int32_t* seq_lens, const uint8_t* head_kind,
+                                 const float* p, int32_t topk, int32_t window, int32_t sink, uint16_t* out,
+                                 void* stream) {
+    if (!dims || !q_pre || !q_rope || !k_idx || !k_cache || !v_cache || !Wq_idx || !seq_lens || !head_kind ||
+        (topk == 0 && !p) || !out)
         return RTP_ERR_NULL;
+    if (topk < 0) return RTP_ERR_SHAPE;
     if (window < 0 || sink < 0 || (int64_t)window + sink < 1) return RTP_ERR_SHAPE;
     if (!aligned16(q_pre) || !aligned16(q_rope) || !aligned16(k_idx) || !aligned16(k_cache) || !aligned16(v_cache) ||
         !aligned16(Wq_idx) || !aligned16(out))
@@ -334,7 +338,8 @@ extern "C" rtp_status rtp_decode_step(const rtp_dims* dims, const uint16_t* q_pr
     P.Wq = Wq_idx;
     P.seq_lens = seq_lens;
     P.block_table = dims->block_table;
-    P.p = p;
+    P.p = topk > 0 ? nullptr : p;
+    P.topk = topk;
     P.out = out;
     memcpy(P.tab.rg_group, pl.rg_group, sizeof(P.tab.rg_group));
     memcpy(P.tab.rg_mask, pl.rg_mask, sizeof(P.tab.rg_mask));
@@ -392,6 +397,25 @@ extern "C" rtp_status rtp_decode_step(const rtp_dims* dims, const uint16_t* q_pr
     }
     if (ev) cudaEventRecordWithFlags((cudaEvent_t)ev[2], s, ev_flags);
     return e == cudaSuccess ? RTP_OK : RTP_ERR_CUDA;
+}
+
+extern "C" rtp_status rtp_decode_step(const rtp_dims* dims, const uint16_t* q_pre, const uint16_t* q_rope,
+                                      const uint16_t* k_idx, const uint16_t* k_cache, const uint16_t* v_cache,
+                                      const uint16_t* Wq_idx, const int32_t* seq_lens, const uint8_t* head_kind,
+                                      const float* p, int32_t window, int32_t sink, uint16_t* out, void* stream) {
+    if (!p) return RTP_ERR_NULL;
+    return decode_step_ws(dims, q_pre, q_rope, k_idx, k_cache, v_cache, Wq_idx, seq_lens, head_kind, p, 0, window,
+                          sink, out, stream);
+}
+
+extern "C" rtp_status rtp_decode_step_topk(const rtp_dims* dims, const uint16_t* q_pre, const uint16_t* q_rope,
+                                           const uint16_t* k_idx, const uint16_t* k_cache, const uint16_t* v_cache,
+                                           const uint16_t* Wq_idx, const int32_t* seq_lens,
+                                           const uint8_t* head_kind, int32_t topk, int32_t window, int32_t sink,
+                                           uint16_t* out, void* stream) {
+    if (topk < 1) return RTP_ERR_SHAPE;
+    return decode_step_ws(dims, q_pre, q_rope, k_idx, k_cache, v_cache, Wq_idx, seq_lens, head_kind, nullptr, topk,
+                          window, sink, out, stream);
 }
 
 extern "C" rtp_status rtp_get_status(const rtp_dims* dims, void* stream) {

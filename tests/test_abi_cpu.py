@@ -76,6 +76,30 @@ def test_host_side_errors_launch_nothing():
     assert _call(d4) == 3                             # RTP_ERR_UNSUPPORTED
 
 
+def _call_topk(d, topk, window=64, sink=4, ptr=256, **nulls):
+    args = {k: ptr for k in ("q_pre", "q_rope", "k_idx", "k_cache", "v_cache", "Wq", "seq_lens", "out")}
+    args.update(nulls)
+    return rtp.lib.rtp_decode_step_topk(ctypes.byref(d), args["q_pre"], args["q_rope"], args["k_idx"],
+                                        args["k_cache"], args["v_cache"], args["Wq"], args["seq_lens"],
+                                        rtp._head_kind_buf(HK), topk, window, sink, args["out"], None)
+
+
+def test_topk_host_side_checks():
+    """rtp_decode_step_topk: k < 1 is refused; p is not an argument, so the
+    remaining checks (nulls, local set, workspace) are rtp_decode_step's."""
+    d = dims()
+    assert _call_topk(d, 0) == 2                      # RTP_ERR_SHAPE: k must be >= 1
+    assert _call_topk(d, -5) == 2
+    assert _call_topk(d, 4096, q_pre=None) == 1       # RTP_ERR_NULL
+    assert _call_topk(d, 4096, window=0, sink=0) == 2
+    assert _call_topk(d, 4096) == 4                   # RTP_ERR_WORKSPACE: none given (the checks passed)
+    assert _call_topk(d, 1 << 30) == 4                # any k >= 1 is valid (k >= L keeps every block)
+    d4 = dims()
+    d4.idx_dim = 32
+    assert _call_topk(d4, 16) == 3
+    assert _call(d, p=None) == 1                      # the top-p step still needs p
+
+
 def test_paged_geometry_checks():
     d = dims(block_table=4096, max_blocks_per_seq=32, num_pages=10)   # 32*64 != 4096
     assert rtp.workspace_size(d, HK) == 0

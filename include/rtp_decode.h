@@ -230,7 +230,6 @@ rtp_status rtp_decode_step_noalloc(const rtp_dims* dims, const uint16_t* q_pre, 
                                    const float* p, int32_t window, int32_t sink, uint16_t* out,
                                    uint32_t* device_status, void* stream);
 
-/* Static string naming a status code. */
 /*
  * rtp_index_append -- write the retrieval keys of new tokens into the index
  * cache that rtp_decode_step reads (the step before the decode hot path).
@@ -271,6 +270,7 @@ rtp_status rtp_decode_step_noalloc(const rtp_dims* dims, const uint16_t* q_pre, 
 rtp_status rtp_index_append(const rtp_dims* dims, const uint16_t* k_pre, const uint16_t* Wk_idx, const int32_t* pos,
                             int32_t num_new, uint16_t* k_idx, uint32_t* device_status, void* stream);
 
+/* Static string naming a status code. */
 const char* rtp_status_string(rtp_status status);
 
 #ifdef __cplusplus

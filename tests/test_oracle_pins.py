@@ -503,6 +503,229 @@ def test_index_append_identity_projection_copies_inputs():
 
 
 # ---------------------------------------------------------------------------
+# KV-cache write with the index-cache append: k_cache = bf16(RoPE_n(k^pre)),
+# v_cache = v, k_idx = bf16(W^K k^pre), rows n = pos_b + t
+# ---------------------------------------------------------------------------
+def _kv_case(seed, B=2, Hkv=2, T=3, ncap=128, paged=False):
+    k_pre, Wk, pos, kidx, bt = _append_case(seed, B=B, Hkv=Hkv, T=T, ncap=ncap, paged=paged)
+    rng = np.random.default_rng(1000 + seed)
+    v_new = synth.to_bf16(rng.standard_normal(k_pre.shape))
+    ang = rng.uniform(-np.pi, np.pi, (ncap, 64))
+    cos, sin = np.cos(ang).astype(np.float32), np.sin(ang).astype(np.float32)
+    shape = kidx.shape[:3] + (128,)
+    kc = rng.integers(0, 2 ** 16, shape).astype(np.uint16)
+    vc = rng.integers(0, 2 ** 16, shape).astype(np.uint16)
+    return k_pre, v_new, Wk, cos, sin, pos, kidx, kc, vc, bt
+
+
+@pytest.mark.parametrize("paged", [False, True])
+def test_kv_append_exact_rationals_and_untouched_rows(paged):
+    """Brute force in exact rationals: every written key element is the
+    nearest bf16 of k_i cos - k_(i+64) sin (resp. k_(i+64) cos + k_i sin)
+    with the table's fp32 values; value rows are the new values bit for bit;
+    index rows are the nearest bf16 of the exact projection; every other row
+    of the three caches keeps its old bits."""
+    from fractions import Fraction
+
+    k_pre, v_new, Wk, cos, sin, pos, kidx, kc, vc, bt = _kv_case(11, paged=paged)
+    o_idx, o_k, o_v = oracle.kv_append(k_pre, v_new, Wk, cos, sin, pos, kidx, kc, vc, block_table=bt)
+    B, Hkv, T = k_pre.shape[:3]
+    written = set()
+    for b in range(B):
+        for g in range(Hkv):
+            for t in range(T):
+                n = int(pos[b]) + t
+                written.add((b, g, n))
+                kv = [_bf16_value(int(x)) for x in k_pre[b, g, t]]
+                got = _row(o_k, bt, b, g, n)
+                for i in range(64):
+                    c, sn = Fraction(float(cos[n, i])), Fraction(float(sin[n, i]))
+                    assert int(got[i]) == _bf16_exact_rne(kv[i] * c - kv[i + 64] * sn), (b, g, t, i)
+                    assert int(got[i + 64]) == _bf16_exact_rne(kv[i + 64] * c + kv[i] * sn), (b, g, t, i + 64)
+                assert np.array_equal(_row(o_v, bt, b, g, n), v_new[b, g, t])
+                gi = _row(o_idx, bt, b, g, n)
+                for r in (0, 7, 15):
+                    exact = sum(_bf16_value(int(Wk[g, r, i])) * kv[i] for i in range(128))
+                    assert int(gi[r]) == _bf16_exact_rne(exact), (b, g, t, r)
+    for b in range(B):
+        for g in range(Hkv):
+            for n in range(128):
+                if (b, g, n) not in written:
+                    for new, old in ((o_idx, kidx), (o_k, kc), (o_v, vc)):
+                        assert np.array_equal(_row(new, bt, b, g, n), _row(old, bt, b, g, n))
+
+
+def test_kv_append_quarter_turns_permute_and_negate():
+    """Angles 0, 90, 180 and 270 degrees (cos, sin in {0, 1, -1}): the key
+    row is k, (-k_hi, k_lo), -k and (k_hi, -k_lo), exactly (up to the sign of
+    zero), which fixes the pairing (i, i + 64) and the direction of rotation."""
+    k_pre, v_new, Wk, cos, sin, pos, kidx, kc, vc, bt = _kv_case(12, B=1, Hkv=1, T=4, ncap=64)
+    pos[:] = 10
+    turns = [(1.0, 0.0), (0.0, 1.0), (-1.0, 0.0), (0.0, -1.0)]
+    for t, (c, sn) in enumerate(turns):
+        cos[10 + t, :], sin[10 + t, :] = c, sn
+    _, o_k, _ = oracle.kv_append(k_pre, v_new, Wk, cos, sin, pos, kidx, kc, vc)
+    for t in range(4):
+        k = synth.from_bf16(k_pre[0, 0, t])
+        lo, hi = k[:64], k[64:]
+        want = [np.concatenate([lo, hi]), np.concatenate([-hi, lo]), np.concatenate([-lo, -hi]),
+                np.concatenate([hi, -lo])][t]
+        assert np.array_equal(synth.from_bf16(o_k[0, 0, 10 + t]), want), t
+
+
+def test_kv_append_one_hot_keys_give_the_table():
+    """k = e_i gives y_i = cos, y_(i+64) = sin; k = e_(i+64) gives
+    y_i = -sin, y_(i+64) = cos; every other element is zero."""
+    k_pre, v_new, Wk, cos, sin, pos, kidx, kc, vc, bt = _kv_case(13, B=1, Hkv=1, T=2, ncap=64)
+    one = synth.to_bf16(np.ones(1))[0]
+    for i in (0, 5, 63):
+        k_pre[:] = 0
+        k_pre[0, 0, 0, i] = one
+        k_pre[0, 0, 1, i + 64] = one
+        pos[:] = 20
+        _, o_k, _ = oracle.kv_append(k_pre, v_new, Wk, cos, sin, pos, kidx, kc, vc)
+        a = synth.from_bf16(o_k[0, 0, 20])
+        b = synth.from_bf16(o_k[0, 0, 21])
+        c, sn = float(cos[20, i]), float(sin[21, i])
+        assert a[i] == synth.from_bf16(synth.to_bf16(np.array([c])))[0]
+        assert a[i + 64] == synth.from_bf16(synth.to_bf16(np.array([float(sin[20, i])])))[0]
+        assert b[i] == synth.from_bf16(synth.to_bf16(np.array([-sn])))[0]
+        assert b[i + 64] == synth.from_bf16(synth.to_bf16(np.array([float(cos[21, i])])))[0]
+        mask = np.ones(128, bool)
+        mask[[i, i + 64]] = False
+        assert np.all(a[mask] == 0) and np.all(b[mask] == 0)
+
+
+def test_kv_append_with_position_angles_matches_the_generator():
+    """With the angle table n theta_i (theta_i = 1e6^(-2i/128), rounded to
+    fp32), the written keys are the generator's RoPE'd keys (exact angles,
+    computed by its own code) to within one bf16 step, nearly all bit for
+    bit: the table row of token t is its cache position pos_b + t."""
+    k_pre, v_new, Wk, cos, sin, pos, kidx, kc, vc, bt = _kv_case(14, B=2, Hkv=2, T=6, ncap=4096)
+    n = np.arange(4096, dtype=np.float64)[:, None]
+    ang = n * synth.THETA ** (-2.0 * np.arange(64) / 128.0)[None, :]
+    cos, sin = np.cos(ang).astype(np.float32), np.sin(ang).astype(np.float32)
+    _, o_k, _ = oracle.kv_append(k_pre, v_new, Wk, cos, sin, pos, kidx, kc, vc)
+    same = total = 0
+    for b in range(2):
+        p = pos[b] + np.arange(6)
+        for g in range(2):
+            want = synth.rope_rows(k_pre[b, g], p)
+            got = o_k[b, g, p]
+            d = np.abs(got.astype(np.int32) - want.astype(np.int32))
+            d = np.where((got ^ want) & 0x8000, 0, d)         # (compare magnitudes only when signs agree)
+            assert np.all(np.abs(synth.from_bf16(got) - synth.from_bf16(want)) <=
+                          2.0 ** -7 * np.maximum(np.abs(synth.from_bf16(want)), 2.0 ** -126))
+            same += int(np.count_nonzero(got == want))
+            total += got.size
+            assert d.max() <= 1
+    assert same >= 0.99 * total, (same, total)
+
+
+def test_kv_append_refuses_positions_beyond_the_cache():
+    k_pre, v_new, Wk, cos, sin, pos, kidx, kc, vc, bt = _kv_case(15, ncap=64)
+    pos[0] = 62                                            # 62 + 3 > 64
+    with pytest.raises(ValueError):
+        oracle.kv_append(k_pre, v_new, Wk, cos, sin, pos, kidx, kc, vc)
+
+
+# ---------------------------------------------------------------------------
+# local heads' ring cache: sink + W rows per (sequence, KV head)
+# ---------------------------------------------------------------------------
+def _marker_rows(positions):
+    """bf16 rows whose first four entries spell the position in base 16
+    (small integers are exact in bf16); the rest zero."""
+    rows = np.zeros((len(positions), 128))
+    for i, n in enumerate(positions):
+        for d in range(4):
+            rows[i, d] = (n >> (4 * d)) & 15
+        rows[i, 4] = 1.0                        # a written row is never all-zero
+    return synth.to_bf16(rows)
+
+
+def _marker_of(row_bits):
+    v = synth.from_bf16(row_bits)
+    if v[4] != 1.0:
+        return None
+    return int(sum(int(v[d]) << (4 * d) for d in range(4)))
+
+
+@pytest.mark.parametrize("S0,W,L,chunk", [(4, 16, 3, 1), (4, 16, 20, 1), (4, 16, 21, 7), (4, 16, 100, 1),
+                                           (4, 16, 100, 40), (0, 8, 50, 3), (3, 1, 9, 2), (64, 64, 1000, 64),
+                                           (64, 128, 1000, 100), (2, 7, 300, 300)])
+def test_ring_keeps_the_head_rows_and_the_last_W_positions(S0, W, L, chunk):
+    """Positions 0 .. L-1 written in order (chunks of `chunk`): the ring then
+    holds exactly [0, min(S0, L)) and the last W positions past S0, each in
+    the row the layout gives it; unwritten rows stay unwritten."""
+    B, Hkv = 1, 1
+    kr = np.zeros((B, Hkv, S0 + W, 128), np.uint16)
+    vr = np.zeros_like(kr)
+    start = 0
+    while start < L:
+        T = min(chunk, L - start)
+        rows = _marker_rows(range(start, start + T)).reshape(B, Hkv, T, 128)
+        kr, vr = oracle.ring_write(rows, rows, np.array([start], np.int32), kr, vr, S0, W)
+        start += T
+    held = {}
+    for r in range(S0 + W):
+        m = _marker_of(kr[0, 0, r])
+        assert m == _marker_of(vr[0, 0, r])
+        if m is not None:
+            held[m] = r
+    want = set(range(min(S0, L))) | set(range(max(S0, L - W), L))
+    assert set(held) == want
+    for n, r in held.items():
+        assert r == oracle.ring_row(n, S0, W)
+        assert (r < S0) == (n < S0)
+
+
+def test_ring_blocks_occupy_aligned_slots():
+    """With S0 = 64 and W a multiple of 64, the 64 positions of any block
+    j >= 1 lie in 64 consecutive rows starting at a multiple of 64."""
+    for W in (64, 256, 4096):
+        for j in (1, 2, 63, 64, 65, 1000):
+            rows = [oracle.ring_row(64 * j + o, 64, W) for o in range(64)]
+            assert rows[0] % 64 == 0 and rows == list(range(rows[0], rows[0] + 64))
+            assert 64 <= rows[0] < 64 + W
+
+
+@pytest.mark.parametrize("L,window,sink,S0,W", [(3000, 256, 4, 64, 256), (3000, 100, 4, 64, 256),
+                                                (200, 256, 4, 64, 256), (3, 256, 4, 64, 256),
+                                                (700, 64, 0, 0, 64), (700, 0, 4, 4, 64), (5000, 1, 0, 0, 1),
+                                                (3001, 200, 4, 4, 200)])
+def test_ring_attention_equals_the_local_head_output(L, window, sink, S0, W):
+    """A local head that reads its keys and values from the ring gives the
+    decode step's local-head output on the full cache, bit for bit (same
+    positions, same order of summation)."""
+    case = synth.make_case("ring", B=2, Hkv=2, G=2, seq_lens=[L, max(1, L // 3)], ret_groups=[], p=[0.9, 0.9],
+                           window=window, sink=sink, seed=L + window, regimes=["gaussian", "gaussian"])
+    ref = oracle.decode_step(case)
+    for b in range(case.B):
+        Lb = int(case.seq_lens[b])
+        kr = np.zeros((case.B, case.Hkv, S0 + W, 128), np.uint16)
+        vr = np.zeros_like(kr)
+        for start in range(0, Lb, 512):
+            T = min(512, Lb - start)
+            pos = np.full(case.B, start, np.int32)
+            kr, vr = oracle.ring_write(case.k_cache[:, :, start:start + T], case.v_cache[:, :, start:start + T],
+                                       pos, kr, vr, S0, W)
+        for h in range(case.Hq):
+            got = oracle.attend_ring(case.q_rope, kr, vr, b, h, Lb, window, sink, S0, W)
+            assert np.array_equal(got, ref["out"][b, h]), (b, h)
+
+
+def test_ring_refuses_a_window_or_sink_it_cannot_hold():
+    case = synth.make_case("ring-w", B=1, Hkv=1, G=1, seq_lens=[100], ret_groups=[], p=[0.9], window=32, sink=4,
+                           seed=3, regimes=["gaussian"])
+    kr = np.zeros((1, 1, 64 + 16, 128), np.uint16)
+    with pytest.raises(ValueError):
+        oracle.attend_ring(case.q_rope, kr, kr, 0, 0, 100, 32, 4, 64, 16)     # window 32 > W 16
+    kr = np.zeros((1, 1, 2 + 64, 128), np.uint16)
+    with pytest.raises(ValueError):
+        oracle.attend_ring(case.q_rope, kr, kr, 0, 0, 100, 32, 4, 2, 64)      # sink 4 > S0 2
+
+
+# ---------------------------------------------------------------------------
 # static top-k (the fixed-budget variant): the k highest scores, ties low index
 # ---------------------------------------------------------------------------
 @pytest.mark.parametrize("seed", range(12))

@@ -159,6 +159,36 @@ rtp_status rtp_decode_step(const rtp_dims* dims, const uint16_t* q_pre, const ui
                            const float* p, int32_t window, int32_t sink, uint16_t* out, void* stream);
 
 /*
+ * rtp_decode_step_ring -- the decode step for a model whose local KV heads
+ * keep only their sink and sliding window (review, Method: "Adaptive sparse
+ * attention": local heads attend to a sink and a window, so they need no
+ * long-context cache; Insight 1: most heads are local).  Local heads of KV
+ * heads that serve no retrieval head read their keys and values from rings
+ * instead of k_cache / v_cache; every other read is rtp_decode_step's.
+ *
+ * Ring layout, per sequence b and KV head g (rows of 128 bf16):
+ *   rows 0 .. 63      : positions 0 .. 63 (the sink, 64 >= sink);
+ *   rows 64 .. 63 + W : position n >= 64 in row 64 + (n mod W).
+ * Writing positions in order, each new one overwrites the one W places
+ * before it, so after L tokens the ring holds [0, min(64, L)) and
+ * [max(64, L - W), L); W (ring_W) must be a multiple of 64 and >= window.
+ *
+ * Arguments are those of rtp_decode_step, plus
+ *   k_ring, v_ring : device bf16 [batch, num_kv_heads, 64 + ring_W, 128],
+ *     16-byte aligned (rows of KV heads with retrieval heads are not read).
+ *   ring_W : the window region's rows, a multiple of 64, >= window.
+ * Rows of k_cache / v_cache for KV heads without retrieval heads are not read.
+ * Returns RTP_ERR_NULL for a NULL ring, RTP_ERR_SHAPE for ring_W not a
+ * multiple of 64 or below window (or below 64) or sink > 64; otherwise as
+ * rtp_decode_step (same workspace size).
+ */
+rtp_status rtp_decode_step_ring(const rtp_dims* dims, const uint16_t* q_pre, const uint16_t* q_rope,
+                                const uint16_t* k_idx, const uint16_t* k_cache, const uint16_t* v_cache,
+                                const uint16_t* k_ring, const uint16_t* v_ring, int32_t ring_W,
+                                const uint16_t* Wq_idx, const int32_t* seq_lens, const uint8_t* head_kind,
+                                const float* p, int32_t window, int32_t sink, uint16_t* out, void* stream);
+
+/*
  * rtp_decode_step_topk -- the decode step with the static top-k selection in
  * place of dynamic top-p: every retrieval head keeps its min(topk, L) best
  * tokens under the order (score descending, token index ascending), widened

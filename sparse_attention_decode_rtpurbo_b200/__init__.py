@@ -73,6 +73,9 @@ def _load():
     L.rtp_decode_step.restype = ctypes.c_int
     L.rtp_decode_step_topk.argtypes = [ctypes.POINTER(RtpDims), vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, vp, vp]
     L.rtp_decode_step_topk.restype = ctypes.c_int
+    L.rtp_decode_step_ring.argtypes = [ctypes.POINTER(RtpDims), vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, i32,
+                                       i32, vp, vp]
+    L.rtp_decode_step_ring.restype = ctypes.c_int
     L.rtp_decode_step_noalloc.argtypes = [ctypes.POINTER(RtpDims), vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, vp,
                                           vp, vp]
     L.rtp_decode_step_noalloc.restype = ctypes.c_int
@@ -129,6 +132,19 @@ def decode_step(dims: RtpDims, q_pre, q_rope, k_idx, k_cache, v_cache, Wq_idx, s
                              int(window), int(sink), _ptr(out), st)
     if rc != RTP_OK:
         raise RtpError(rc, "rtp_decode_step")
+
+
+def decode_step_ring(dims: RtpDims, q_pre, q_rope, k_idx, k_cache, v_cache, k_ring, v_ring, ring_W: int, Wq_idx,
+                     seq_lens, head_kind, p, window: int, sink: int, out, stream=None) -> None:
+    """rtp_decode_step_ring: the decode step with the local-only KV heads'
+    keys and values read from rings [B, Hkv, 64 + ring_W, 128] (block 0 in
+    rows 0..63, position n >= 64 in row 64 + n % ring_W)."""
+    st = 0 if stream is None else (stream if isinstance(stream, int) else stream.cuda_stream)
+    rc = lib.rtp_decode_step_ring(ctypes.byref(dims), _ptr(q_pre), _ptr(q_rope), _ptr(k_idx), _ptr(k_cache),
+                                  _ptr(v_cache), _ptr(k_ring), _ptr(v_ring), int(ring_W), _ptr(Wq_idx), _ptr(seq_lens),
+                                  _head_kind_buf(head_kind), _ptr(p), int(window), int(sink), _ptr(out), st)
+    if rc != RTP_OK:
+        raise RtpError(rc, "rtp_decode_step_ring")
 
 
 def decode_step_topk(dims: RtpDims, q_pre, q_rope, k_idx, k_cache, v_cache, Wq_idx, seq_lens, head_kind, topk: int,
@@ -205,6 +221,11 @@ class Step:
     def __call__(self, q_pre, q_rope, k_idx, k_cache, v_cache, Wq_idx, seq_lens, p, window, sink, out, stream=None):
         decode_step(self.dims, q_pre, q_rope, k_idx, k_cache, v_cache, Wq_idx, seq_lens, self.head_kind, p, window,
                     sink, out, stream)
+
+    def ring(self, q_pre, q_rope, k_idx, k_cache, v_cache, k_ring, v_ring, ring_W, Wq_idx, seq_lens, p, window, sink,
+             out, stream=None):
+        decode_step_ring(self.dims, q_pre, q_rope, k_idx, k_cache, v_cache, k_ring, v_ring, ring_W, Wq_idx, seq_lens,
+                         self.head_kind, p, window, sink, out, stream)
 
     def topk(self, q_pre, q_rope, k_idx, k_cache, v_cache, Wq_idx, seq_lens, topk, window, sink, out, stream=None):
         decode_step_topk(self.dims, q_pre, q_rope, k_idx, k_cache, v_cache, Wq_idx, seq_lens, self.head_kind, topk,

@@ -713,12 +713,17 @@ __device__ __forceinline__ void a_producer(const KParams& K, ASmem<G>& S, AWalk 
                 }
             } else if (lane == 0) {
                 const int j = sg.type == 1 ? (ti < lg.nA ? ti : lg.bw0 + (ti - lg.nA)) : (int)(S.d_list[ti] >> 8);
-                const int row = (int)block_row(P, sg.b, g, j);
+                // local groups without retrieval heads may keep only a ring of
+                // their sink and window (the tiles' position masks stay as they are)
+                const bool ring = sg.type == 1 && ((P.ring_lg_mask >> sg.grp) & 1ull);
+                const int row = ring ? (int)ring_block_row(P, sg.b, g, j) : (int)block_row(P, sg.b, g, j);
+                const CUtensorMap* mk = ring ? &K.tmk_r : &K.tmk;
+                const CUtensorMap* mv = ring ? &K.tmv_r : &K.tmv;
                 mbar_expect_tx(&S.full[st], STAGE_BYTES);
-                tma_load_2d(dst, &K.tmk, 0, row, &S.full[st]);
-                tma_load_2d(dst + 8192, &K.tmk, 64, row, &S.full[st]);
-                tma_load_2d(dst + KV_TILE, &K.tmv, 0, row, &S.full[st]);
-                tma_load_2d(dst + KV_TILE + 8192, &K.tmv, 64, row, &S.full[st]);
+                tma_load_2d(dst, mk, 0, row, &S.full[st]);
+                tma_load_2d(dst + 8192, mk, 64, row, &S.full[st]);
+                tma_load_2d(dst + KV_TILE, mv, 0, row, &S.full[st]);
+                tma_load_2d(dst + KV_TILE + 8192, mv, 64, row, &S.full[st]);
             }
             __syncwarp();
         }

@@ -129,3 +129,23 @@ def test_index_append_host_side_checks():
     assert call(d, fake + 2, fake, fake, 1, fake, None, None) == 3                     # k_pre not 16-byte aligned
     assert call(d, fake, fake, fake, 1, fake + 4, None, None) == 3                     # k_idx not 8-byte aligned
     assert call(dims(num_kv_heads=65, num_q_heads=65), fake, fake, fake, 1, fake, None, None) == 3
+
+
+def test_ring_host_side_checks():
+    """rtp_decode_step_ring: ring sizes are checked before any CUDA call."""
+    fake = 4096
+
+    def call(d, W=128, window=64, sink=4, kr=fake, vr=fake, p=fake):
+        return rtp.lib.rtp_decode_step_ring(ctypes.byref(d), fake, fake, fake, fake, fake, kr, vr, W, fake, fake,
+                                            rtp._head_kind_buf(HK), p, window, sink, fake, None)
+
+    d = dims()
+    assert call(d, kr=None) == 1
+    assert call(d, vr=None) == 1
+    assert call(d, p=None) == 1
+    assert call(d, W=96) == 2                        # not a multiple of 64
+    assert call(d, W=64, window=65) == 2             # the window does not fit
+    assert call(d, W=0, window=0) == 2
+    assert call(d, sink=65) == 2                     # the sink must fit the 64 head rows
+    assert call(d, kr=fake + 8) == 3
+    assert call(d) == 4                              # checks passed; no workspace given

@@ -231,6 +231,8 @@ __device__ __noinline__ void r_pass(const Params& P, RWalk wk, const int* pre, i
     Acct ac;
     ac.init(P, S.acct, tid == 0);
     const int rp = pass - RP_REF0;
+    // key bits above the refine pass's digit (the prefix found so far); unused in pass RP_REF0
+    constexpr int psh = (pass > RP_REF0 && pass <= RP_REF3) ? 32 - 8 * (pass - RP_REF0) : 0;
     // the parameters this loop uses, read once: through a reference into the
     // parameter block they would be read again after every global atomic
     const int n_ret = P.n_ret, sstride = P.sstride, words_cap = P.words_cap, ntiles_cap = P.ntiles_cap;
@@ -430,7 +432,7 @@ __device__ __noinline__ void r_pass(const Params& P, RWalk wk, const int* pre, i
                     }
                 } else if constexpr (pass <= RP_REF3) {
                     if (ok && score_bin(v[u], rh.smax, rh.dr, rh.inv_w) == rh.bstar &&
-                        (rp == 0 || (key >> (32 - 8 * rp)) == rh.prefix)) {
+                        (rp == 0 || (key >> psh) == rh.prefix)) {
                         const uint32_t d = (key >> (24 - 8 * rp)) & 255u;
                         hist_add(S.H, hh, (int)d, 1u, unit ? 1ull : fixmass(key, rh.smax));
                     }

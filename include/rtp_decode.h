@@ -189,6 +189,31 @@ rtp_status rtp_decode_step_ring(const rtp_dims* dims, const uint16_t* q_pre, con
                                 const float* p, int32_t window, int32_t sink, uint16_t* out, void* stream);
 
 /*
+ * rtp_ring_write -- write the key and value rows of new tokens of the local-
+ * only KV heads into their rings (the layout of rtp_decode_step_ring: rows
+ * 0 .. 63 hold positions 0 .. 63, position n >= 64 goes to row 64 + n mod W).
+ * The result is that of writing the tokens t = 0 .. num_new-1 of each
+ * sequence in order: a token whose row a later token of the same call also
+ * takes is not written.
+ *   dims     : batch, num_kv_heads, head_dim 128, block_size 64 (other fields
+ *              unused).
+ *   k_new, v_new : device bf16 [batch, num_kv_heads, num_new, 128] (RoPE'd
+ *              keys, values), 16-byte aligned.
+ *   pos      : device int32 [batch], position of each sequence's first new token.
+ *   ring_W   : the rings' window rows, a multiple of 64.
+ *   k_ring, v_ring : device bf16 [batch, num_kv_heads, 64 + ring_W, 128],
+ *              16-byte aligned; owned by the caller.
+ *   device_status : optional device uint32, set to RTP_ERR_DEVICE_INPUT for a
+ *              negative position (that sequence is skipped).
+ * Returns RTP_ERR_NULL / RTP_ERR_SHAPE / RTP_ERR_UNSUPPORTED before anything
+ * is enqueued, RTP_ERR_CUDA if the launch failed, else RTP_OK (num_new = 0:
+ * nothing is enqueued).
+ */
+rtp_status rtp_ring_write(const rtp_dims* dims, const uint16_t* k_new, const uint16_t* v_new, const int32_t* pos,
+                          int32_t num_new, int32_t ring_W, uint16_t* k_ring, uint16_t* v_ring,
+                          uint32_t* device_status, void* stream);
+
+/*
  * rtp_decode_step_topk -- the decode step with the static top-k selection in
  * place of dynamic top-p: every retrieval head keeps its min(topk, L) best
  * tokens under the order (score descending, token index ascending), widened

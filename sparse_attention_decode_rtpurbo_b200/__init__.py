@@ -76,6 +76,8 @@ def _load():
     L.rtp_decode_step_ring.argtypes = [ctypes.POINTER(RtpDims), vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, i32,
                                        i32, vp, vp]
     L.rtp_decode_step_ring.restype = ctypes.c_int
+    L.rtp_ring_write.argtypes = [ctypes.POINTER(RtpDims), vp, vp, vp, i32, i32, vp, vp, vp, vp]
+    L.rtp_ring_write.restype = ctypes.c_int
     L.rtp_decode_step_noalloc.argtypes = [ctypes.POINTER(RtpDims), vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, vp,
                                           vp, vp]
     L.rtp_decode_step_noalloc.restype = ctypes.c_int
@@ -145,6 +147,17 @@ def decode_step_ring(dims: RtpDims, q_pre, q_rope, k_idx, k_cache, v_cache, k_ri
                                   _head_kind_buf(head_kind), _ptr(p), int(window), int(sink), _ptr(out), st)
     if rc != RTP_OK:
         raise RtpError(rc, "rtp_decode_step_ring")
+
+
+def ring_write(dims: RtpDims, k_new, v_new, pos, num_new: int, ring_W: int, k_ring, v_ring, device_status=None,
+               stream=None) -> None:
+    """rtp_ring_write: the new key and value rows of every sequence into the
+    local heads' rings [B, Hkv, 64 + ring_W, 128], as if written in order."""
+    st = 0 if stream is None else (stream if isinstance(stream, int) else stream.cuda_stream)
+    rc = lib.rtp_ring_write(ctypes.byref(dims), _ptr(k_new), _ptr(v_new), _ptr(pos), int(num_new), int(ring_W),
+                            _ptr(k_ring), _ptr(v_ring), _ptr(device_status), st)
+    if rc != RTP_OK:
+        raise RtpError(rc, "rtp_ring_write")
 
 
 def decode_step_topk(dims: RtpDims, q_pre, q_rope, k_idx, k_cache, v_cache, Wq_idx, seq_lens, head_kind, topk: int,

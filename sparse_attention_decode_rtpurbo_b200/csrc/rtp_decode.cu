@@ -543,6 +543,39 @@ extern "C" rtp_status rtp_decode_step_noalloc(const rtp_dims* dims, const uint16
 }
 
 // ---------------------------------------------------------------------------
+// local heads' ring write
+// ---------------------------------------------------------------------------
+extern "C" rtp_status rtp_ring_write(const rtp_dims* d, const uint16_t* k_new, const uint16_t* v_new,
+                                     const int32_t* pos, int32_t num_new, int32_t ring_W, uint16_t* k_ring,
+                                     uint16_t* v_ring, uint32_t* device_status, void* stream) {
+    if (!d) return RTP_ERR_NULL;
+    if (d->head_dim != D || d->block_size != BLK) return RTP_ERR_UNSUPPORTED;
+    if (d->batch < 1 || d->num_kv_heads < 1 || num_new < 0) return RTP_ERR_SHAPE;
+    if (d->batch > MAX_B || d->num_kv_heads > MAX_HKV) return RTP_ERR_UNSUPPORTED;
+    if (ring_W < BLK || ring_W % BLK) return RTP_ERR_SHAPE;
+    if (num_new == 0) return RTP_OK;
+    if (!k_new || !v_new || !pos || !k_ring || !v_ring) return RTP_ERR_NULL;
+    if (((uintptr_t)k_new | (uintptr_t)v_new | (uintptr_t)k_ring | (uintptr_t)v_ring) & 15u)
+        return RTP_ERR_UNSUPPORTED;
+    RingParams A;
+    A.B = d->batch;
+    A.Hkv = d->num_kv_heads;
+    A.T = num_new;
+    A.W = ring_W;
+    A.k_new = k_new;
+    A.v_new = v_new;
+    A.pos = pos;
+    A.k_ring = k_ring;
+    A.v_ring = v_ring;
+    A.status = device_status;
+    const int64_t threads = (int64_t)A.B * A.Hkv * A.T * 32;
+    const int64_t grid = (threads + 255) / 256;
+    if (grid > 0x7FFFFFFF) return RTP_ERR_UNSUPPORTED;
+    ring_write_kernel<<<(unsigned)grid, 256, 0, (cudaStream_t)stream>>>(A);
+    return report(cudaGetLastError(), "ring write launch") == cudaSuccess ? RTP_OK : RTP_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
 // index-cache append
 // ---------------------------------------------------------------------------
 extern "C" rtp_status rtp_index_append(const rtp_dims* d, const uint16_t* k_pre, const uint16_t* Wk_idx,

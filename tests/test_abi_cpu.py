@@ -149,3 +149,21 @@ def test_ring_host_side_checks():
     assert call(d, sink=65) == 2                     # the sink must fit the 64 head rows
     assert call(d, kr=fake + 8) == 3
     assert call(d) == 4                              # checks passed; no workspace given
+
+
+def test_ring_write_host_side_checks():
+    fake = 4096
+
+    def call(d, n=1, W=128, kn=fake, vn=fake, kr=fake, vr=fake, pos=fake):
+        return rtp.lib.rtp_ring_write(ctypes.byref(d) if d is not None else None, kn, vn, pos, n, W, kr, vr, None,
+                                      None)
+
+    d = dims()
+    assert call(None) == 1
+    assert call(d, n=0) == 0                         # nothing to write
+    assert call(d, n=-1) == 2
+    assert call(d, W=96) == 2
+    assert call(d, W=0) == 2
+    assert call(d, kr=None) == 1
+    assert call(d, pos=None) == 1
+    assert call(d, vn=fake + 4) == 3

@@ -87,3 +87,29 @@ def test_ring_windows(window, sink, W):
     case = synth.make_case("ring-w", B=1, Hkv=2, G=4, seq_lens=[3333], ret_groups=[], p=[0.9], window=window,
                            sink=sink, seed=31, regimes=["gaussian"], paged=True)
     assert run_ring(case, W) == []
+
+
+@pytest.mark.parametrize("B,Hkv,T,W,starts", [(2, 3, 1, 64, [0, 63]), (2, 2, 37, 128, [60, 500]),
+                                              (1, 2, 300, 64, [10]), (3, 1, 700, 256, [0, 64, 1000])])
+def test_ring_write_bit_exact(B, Hkv, T, W, starts):
+    """rtp_ring_write against the oracle's in-order writes: chunks that cross
+    the head rows, wrap the window rows several times (T > W: only each
+    row's last token lands), and untouched rows."""
+    import sparse_attention_decode_rtpurbo_b200 as rtp
+
+    rng = np.random.default_rng(T + W)
+    k_new = synth.to_bf16(rng.standard_normal((B, Hkv, T, 128)))
+    v_new = synth.to_bf16(rng.standard_normal((B, Hkv, T, 128)))
+    kr = rng.integers(0, 2 ** 16, (B, Hkv, S0 + W, 128)).astype(np.uint16)
+    vr = rng.integers(0, 2 ** 16, (B, Hkv, S0 + W, 128)).astype(np.uint16)
+    pos = np.array(starts, np.int32)
+    ref_k, ref_v = oracle.ring_write(k_new, v_new, pos, kr, vr, S0, W)
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16) if a.dtype == np.uint16 else a).cuda()
+    kn_d, vn_d, kr_d, vr_d, pos_d = dev(k_new), dev(v_new), dev(kr), dev(vr), dev(pos)
+    dims = rtp.make_dims(B, Hkv, Hkv, 64)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    rtp.ring_write(dims, kn_d, vn_d, pos_d, T, W, kr_d, vr_d, status, torch.cuda.current_stream())
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    assert np.array_equal(kr_d.cpu().numpy().view(np.uint16), ref_k)
+    assert np.array_equal(vr_d.cpu().numpy().view(np.uint16), ref_v)

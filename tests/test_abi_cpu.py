@@ -167,3 +167,14 @@ def test_ring_write_host_side_checks():
     assert call(d, kr=None) == 1
     assert call(d, pos=None) == 1
     assert call(d, vn=fake + 4) == 3
+
+
+def test_binding_refuses_host_and_strided_tensors():
+    """The binding passes tensors by address: a host tensor or a strided view
+    is refused before the library is called."""
+    import torch
+
+    with pytest.raises(ValueError, match="device memory"):
+        rtp.decode_step(dims(), torch.zeros(8), 1, 1, 1, 1, 1, 1, HK, 1, 64, 4, 1)
+    with pytest.raises(ValueError, match="contiguous"):
+        rtp.decode_step(dims(), torch.zeros(8, 8).t(), 1, 1, 1, 1, 1, 1, HK, 1, 64, 4, 1)

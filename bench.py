@@ -44,6 +44,8 @@ def parse():
     ap.add_argument("--scale", type=int, default=1, help="divide the workload's context lengths (profiling runs)")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--dense", action="store_true", help="p = 1 for every sequence (dense comparator)")
+    ap.add_argument("--topk", type=int, default=0,
+                    help="static top-k selection with this k (the fixed-budget variant) instead of top-p")
     ap.add_argument("--dense-comparator", action="store_true",
                     help="also time the same captured step with p = 1 and add it to the line as dense_comparator")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -199,6 +201,10 @@ def max_over_ranks(values, world, device):
     return [float(v) for v in vals]
 
 
+def selection_name(args):
+    return f"static top-k, k={args.topk}" if args.topk > 0 else ("top-p, p=1 (dense)" if args.dense else "top-p")
+
+
 def cpu_model():
     """The host CPU's model name (from /proc/cpuinfo), or None."""
     try:
@@ -211,14 +217,17 @@ def cpu_model():
     return None
 
 
-def oracle_single_thread(case, tokens, budget_s=5.0):
+def oracle_single_thread(case, tokens, topk=0, budget_s=5.0):
     """The oracle on one host thread: whole steps until about budget_s have
     passed (at least one).  Returns a dict for the cpu_baseline entry."""
     import oracle
 
     reps, t0 = 0, time.perf_counter()
     while reps == 0 or (time.perf_counter() - t0 < budget_s and reps < 20):
-        oracle.decode_step(case, nthreads=1)
+        if topk > 0:
+            oracle.decode_step_topk(case, topk, nthreads=1)
+        else:
+            oracle.decode_step(case, nthreads=1)
         reps += 1
     t = (time.perf_counter() - t0) / reps
     return {"value": tokens / t, "s_per_step": t, "sample": f"{reps} whole decode steps, 1 thread"}
@@ -235,21 +244,28 @@ def run_reference(args, rank):
     if args.dense:
         case.p[:] = 1.0
     cores = os.cpu_count() or 1
+
+    def step():
+        if args.topk > 0:
+            oracle.decode_step_topk(case, args.topk, nthreads=cores)
+        else:
+            oracle.decode_step(case, nthreads=cores)
+
     for _ in range(args.warmup):
-        oracle.decode_step(case, nthreads=cores)
+        step()
     ts = []
     for _ in range(args.steps):
         t0 = time.perf_counter()
-        oracle.decode_step(case, nthreads=cores)
+        step()
         ts.append(time.perf_counter() - t0)
     t = statistics.mean(ts)
     tokens = float(case.seq_lens.sum())
     v = tokens / t
-    single = oracle_single_thread(case, tokens)
+    single = oracle_single_thread(case, tokens, args.topk)
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": workload_config(case, args.workload),
+            "config": dict(workload_config(case, args.workload), selection=selection_name(args)),
             "cpu_baseline": {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "cpu_model": cpu_model(),
                              "sample": f"whole decode step of the workload per timed step ({args.steps} steps)",
                              "single_thread": single},
@@ -330,6 +346,7 @@ def main():
     if args.dense:
         case.p[:] = 1.0
     dc = DeviceCase(case, device=dev, debug=True)
+    dc.topk = max(0, args.topk)
     stream = torch.cuda.current_stream(dev)
 
     # one debug step: kept blocks for the algorithmic byte count
@@ -437,7 +454,8 @@ def main():
     hlens = torch.from_numpy(case.seq_lens.astype(np.int32)).pin_memory()
     hp = torch.from_numpy(case.p.astype(np.float32)).pin_memory()
     hout = torch.empty(dc.out.shape, dtype=torch.bfloat16).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in (hq_pre, hq_rope, hlens, hp))
+    h_in = (hq_pre, hq_rope, hlens) if dc.topk > 0 else (hq_pre, hq_rope, hlens, hp)   # (top-k takes no p)
+    h2d = sum(t.numel() * t.element_size() for t in h_in)
     d2h = hout.numel() * hout.element_size()
     e2e_ms = []
     for i in range(max(3, args.warmup) + args.steps):
@@ -448,7 +466,8 @@ def main():
         dc.q_pre.copy_(hq_pre, non_blocking=True)
         dc.q_rope.copy_(hq_rope, non_blocking=True)
         dc.seq_lens.copy_(hlens, non_blocking=True)
-        dc.p.copy_(hp, non_blocking=True)
+        if dc.topk == 0:
+            dc.p.copy_(hp, non_blocking=True)
         graph.replay()
         hout.copy_(dc.out, non_blocking=True)
         z.record(stream)
@@ -463,7 +482,7 @@ def main():
     # sequence (every block of every retrieval head), the stand-in for the
     # pages' dense-attention baseline; the graph reads p from dc.p ----
     dense_ms, dense_status = 0.0, 0
-    if args.dense_comparator and not args.dense and case.head_kind.any():
+    if args.dense_comparator and not args.dense and args.topk == 0 and case.head_kind.any():
         dc.p.fill_(1.0)
         dts = []
         for i in range(max(3, args.warmup) + args.steps):
@@ -507,15 +526,21 @@ def main():
             import oracle
 
             cores = os.cpu_count() or 1
-            oracle.decode_step(case, nthreads=cores)
+            def oracle_step():
+                if args.topk > 0:
+                    oracle.decode_step_topk(case, args.topk, nthreads=cores)
+                else:
+                    oracle.decode_step(case, nthreads=cores)
+
+            oracle_step()
             reps, t0 = 0, time.perf_counter()
             while time.perf_counter() - t0 < 10.0 and reps < 50:
-                oracle.decode_step(case, nthreads=cores)
+                oracle_step()
                 reps += 1
             tc = (time.perf_counter() - t0) / reps
             cpu = {"value": tokens / tc, "unit": UNIT, "cores": cores, "kind": "oracle", "cpu_model": cpu_model(),
                    "sample": f"{reps} whole decode steps of this workload (fp64 C oracle, OpenMP over heads)",
-                   "single_thread": oracle_single_thread(case, tokens)}
+                   "single_thread": oracle_single_thread(case, tokens, args.topk)}
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": t_ms, "us_per_step": t_ms * 1e3,
@@ -523,12 +548,13 @@ def main():
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16 in, fp32 accumulate",
             "data": "synthetic (seeded generators in synth/, shaped like the pages' workloads)",
             "config": dict(workload_config(case, args.workload), parallelism=f"replicas x{world}",
-                           dense_p1=bool(args.dense), timing="CUDA-graph replay of one rtp_decode_step (2 kernels, programmatic launch) per step; "
+                           dense_p1=bool(args.dense), selection=selection_name(args), timing="CUDA-graph replay of one rtp_decode_step (2 kernels, programmatic launch) per step; "
                            "CUDA events on the launching stream"),
             "wall_s_timed_loop": wall,
             "roofline": {"bound": "hbm", "kernel": f"rtp::{dom}_kernel", "achieved": ach, "peak": peak, "unit": "GB/s",
                          "frac": ach / peak, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, burst)",
-                         "traffic": profiled_traffic(dom, case.name), "algorithmic_bytes_per_launch": kbytes[dom],
+                         "traffic": profiled_traffic(dom, case.name) if selection_name(args) == "top-p" else None,
+                         "algorithmic_bytes_per_launch": kbytes[dom],
                          "us_per_launch": phase_ms[dom] * 1e3},
             "step_roofline": {"algorithmic_bytes": nbytes, "achieved": step_gbs, "peak": peak, "unit": "GB/s",
                               "frac": step_gbs / peak},

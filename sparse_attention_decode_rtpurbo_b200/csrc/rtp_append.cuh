@@ -90,3 +90,46 @@ __global__ void __launch_bounds__(APPEND_THREADS) index_append_kernel(const __gr
 }
 
 }  // namespace rtp
+
+namespace rtp {
+
+// Ring write: new key and value rows of local-only KV heads into their rings
+// of 64 + W rows (position n < 64 in row n, n >= 64 in row 64 + n mod W).
+// One warp per (sequence, KV head, new token): lanes 0..15 copy the key row,
+// 16..31 the value row, 16 bytes each.  A token whose row a later token of
+// the same call also maps to (n >= 64 and n + W <= the call's last position)
+// is skipped, so the result is that of writing the tokens in order, whatever
+// the order the warps run in.
+struct RingParams {
+    int B, Hkv, T, W;
+    const uint16_t* k_new;     // [B, Hkv, T, 128]
+    const uint16_t* v_new;
+    const int32_t* pos;        // [B]
+    uint16_t* k_ring;          // [B, Hkv, 64 + W, 128]
+    uint16_t* v_ring;
+    uint32_t* status;          // optional: RTP_ERR_DEVICE_INPUT for a negative position
+};
+
+__global__ void __launch_bounds__(256) ring_write_kernel(const __grid_constant__ RingParams A) {
+    const int64_t w = ((int64_t)blockIdx.x * 256 + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    const int64_t total = (int64_t)A.B * A.Hkv * A.T;
+    if (w >= total) return;
+    const int t = (int)(w % A.T);
+    const int b = (int)(w / ((int64_t)A.T * A.Hkv));
+    const int64_t p0 = (int64_t)__ldg(A.pos + b);
+    const int64_t n = p0 + t;
+    if (p0 < 0) {
+        if (A.status && lane == 0) atomicCAS(A.status, 0u, ST_DEVICE_INPUT);
+        return;
+    }
+    if (n >= BLK && n + A.W <= p0 + A.T - 1) return;   // a later token of this call takes the row
+    const int64_t slot = n < BLK ? n : BLK + n % A.W;
+    const int64_t ring_row = (w / A.T) * (BLK + A.W) + slot;   // (b, g) = w / T
+    const int c = lane & 15;
+    const uint4* src = reinterpret_cast<const uint4*>((lane < 16 ? A.k_new : A.v_new) + w * D) + c;
+    uint4* dst = reinterpret_cast<uint4*>((lane < 16 ? A.k_ring : A.v_ring) + ring_row * D) + c;
+    *dst = __ldg(src);
+}
+
+}  // namespace rtp

@@ -231,6 +231,8 @@ __device__ __noinline__ void r_pass(const Params& P, RWalk wk, const int* pre, i
     Acct ac;
     ac.init(P, S.acct, tid == 0);
     const int rp = pass - RP_REF0;
+    // key bits above the refine pass's digit (the prefix found so far); unused in pass RP_REF0
+    constexpr int psh = (pass > RP_REF0 && pass <= RP_REF3) ? 32 - 8 * (pass - RP_REF0) : 0;
     // the parameters this loop uses, read once: through a reference into the
     // parameter block they would be read again after every global atomic
     const int n_ret = P.n_ret, sstride = P.sstride, words_cap = P.words_cap, ntiles_cap = P.ntiles_cap;
@@ -242,6 +244,7 @@ __device__ __noinline__ void r_pass(const Params& P, RWalk wk, const int* pre, i
     unsigned long long* const cand = P.cand;
     uint32_t* const bitmap = P.bitmap;
     uint32_t* const tie_cnt = P.tie_cnt;
+    const bool unit = P.topk > 0;   // static top-k: every token weighs 1 (the histograms count)
     const bool resident = S.resident != 0;
     if (resident) {
         const long long tq = clock64();
@@ -419,7 +422,7 @@ __device__ __noinline__ void r_pass(const Params& P, RWalk wk, const int* pre, i
                 if constexpr (pass == RP_BINS) {
                     if (ok) {
                         const uint32_t bn = score_bin(v[u], rh.smax, rh.dr, rh.inv_w);
-                        const unsigned long long ms = fixmass(key, rh.smax);
+                        const unsigned long long ms = unit ? 1ull : fixmass(key, rh.smax);
                         if (bn < 255u) {
                             hist_add(S.H, hh, (int)bn, 1u, ms);
                         } else {
@@ -429,9 +432,9 @@ __device__ __noinline__ void r_pass(const Params& P, RWalk wk, const int* pre, i
                     }
                 } else if constexpr (pass <= RP_REF3) {
                     if (ok && score_bin(v[u], rh.smax, rh.dr, rh.inv_w) == rh.bstar &&
-                        (rp == 0 || (key >> (32 - 8 * rp)) == rh.prefix)) {
+                        (rp == 0 || (key >> psh) == rh.prefix)) {
                         const uint32_t d = (key >> (24 - 8 * rp)) & 255u;
-                        hist_add(S.H, hh, (int)d, 1u, fixmass(key, rh.smax));
+                        hist_add(S.H, hh, (int)d, 1u, unit ? 1ull : fixmass(key, rh.smax));
                     }
                 } else if constexpr (pass == RP_TIES) {
                     cnt += (ok && key == rh.tau) ? 1u : 0u;
@@ -621,11 +624,17 @@ __device__ __noinline__ void r_digit(const Params& P, int b, int slot, int tid) 
     auto cnt_of = [&](int d) { return S.dcnt[d]; };
     if constexpr (pass == RP_BINS) {
         // z = the total mass; bins ascend in smax - s: the first bin that
-        // completes the target ceil(p z)
+        // completes the target ceil(p z) (top-k: masses are counts, z = L,
+        // and the target is k)
         bin_search(S, mass_of, cnt_of, false, ~0ull, tid);
         const unsigned long long z = S.hit_k;
-        const double pb = (double)__ldg(P.p + b);
-        unsigned long long tg = (unsigned long long)ceil(pb * (double)z);
+        unsigned long long tg;
+        if (P.topk > 0) {
+            tg = (unsigned long long)P.topk;
+        } else {
+            const double pb = (double)__ldg(P.p + b);
+            tg = (unsigned long long)ceil(pb * (double)z);
+        }
         if (tg > z) tg = z;
         if (tg == 0) tg = 1;
         bin_search(S, mass_of, cnt_of, false, tg, tid);
@@ -737,6 +746,7 @@ __device__ __noinline__ void r_local_select(const Params& P, int b, int slot, in
         S.lsel_count = __ldcg(&P.hs[bs].count_above);
     }
     const unsigned long long target = __ldcg(&P.hs[bs].target);
+    const bool unit = P.topk > 0;   // static top-k: every token weighs 1
     for (int rp = rp0; rp < 4; ++rp) {
         for (int d = tid; d < 256; d += CONSUMERS) {
             S.H.cnt[0][d] = 0;
@@ -750,7 +760,7 @@ __device__ __noinline__ void r_local_select(const Params& P, int b, int slot, in
         for (int j = 0; j < CPT; ++j) {
             const uint32_t key = keys[j];
             if (tid + j * CONSUMERS >= n || (rp > 0 && (key >> (32 - 8 * rp)) != prefix)) continue;
-            hist_add(S.H, 0, (int)((key >> (24 - 8 * rp)) & 255u), 1u, fixmass(key, smax));
+            hist_add(S.H, 0, (int)((key >> (24 - 8 * rp)) & 255u), 1u, unit ? 1ull : fixmass(key, smax));
         }
         consumer_sync();
         // the highest digit whose mass completes the target (digits descend)

@@ -123,17 +123,17 @@ __global__ void __launch_bounds__(APPEND_THREADS) append_kernel(const __grid_con
             uint32_t ylo[4], yhi[4];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                uint16_t a[2], b[2];
+                uint16_t lo_out[2], hi_out[2];
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
                     const double kl = (double)(e ? bf_hi(lu[j]) : bf_lo(lu[j]));
                     const double kh = (double)(e ? bf_hi(hu[j]) : bf_lo(hu[j]));
                     const double c = (double)cv[2 * j + e], s = (double)sv[2 * j + e];
-                    a[e] = __bfloat16_as_ushort(__double2bfloat16(fma(kl, c, -(kh * s))));
-                    b[e] = __bfloat16_as_ushort(__double2bfloat16(fma(kh, c, kl * s)));
+                    lo_out[e] = __bfloat16_as_ushort(__double2bfloat16(fma(kl, c, -(kh * s))));
+                    hi_out[e] = __bfloat16_as_ushort(__double2bfloat16(fma(kh, c, kl * s)));
                 }
-                ylo[j] = (uint32_t)a[0] | ((uint32_t)a[1] << 16);
-                yhi[j] = (uint32_t)b[0] | ((uint32_t)b[1] << 16);
+                ylo[j] = (uint32_t)lo_out[0] | ((uint32_t)lo_out[1] << 16);
+                yhi[j] = (uint32_t)hi_out[0] | ((uint32_t)hi_out[1] << 16);
             }
             kd[2 * q + h] = make_uint4(ylo[0], ylo[1], ylo[2], ylo[3]);
             kd[8 + 2 * q + h] = make_uint4(yhi[0], yhi[1], yhi[2], yhi[3]);

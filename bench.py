@@ -193,6 +193,31 @@ def max_over_ranks(values, world, device):
     return [float(v) for v in vals]
 
 
+def cpu_model():
+    """The host CPU's model name (from /proc/cpuinfo), or None."""
+    try:
+        with open("/proc/cpuinfo") as fh:
+            for line in fh:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
+def oracle_single_thread(case, tokens, budget_s=5.0):
+    """The oracle on one host thread: whole steps until about budget_s have
+    passed (at least one).  Returns a dict for the cpu_baseline entry."""
+    import oracle
+
+    reps, t0 = 0, time.perf_counter()
+    while reps == 0 or (time.perf_counter() - t0 < budget_s and reps < 20):
+        oracle.decode_step(case, nthreads=1)
+        reps += 1
+    t = (time.perf_counter() - t0) / reps
+    return {"value": tokens / t, "s_per_step": t, "sample": f"{reps} whole decode steps, 1 thread"}
+
+
 def run_reference(args, rank):
     """The oracle (fp64 C, OpenMP over heads) on the host cores, same workload."""
     if rank != 0:
@@ -214,12 +239,14 @@ def run_reference(args, rank):
     t = statistics.mean(ts)
     tokens = float(case.seq_lens.sum())
     v = tokens / t
+    single = oracle_single_thread(case, tokens)
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": workload_config(case, args.workload),
-            "cpu_baseline": {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
-                             "sample": f"whole decode step of the workload per timed step ({args.steps} steps)"},
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "cpu_model": cpu_model(),
+                             "sample": f"whole decode step of the workload per timed step ({args.steps} steps)",
+                             "single_thread": single},
             "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -472,8 +499,9 @@ def main():
                 oracle.decode_step(case, nthreads=cores)
                 reps += 1
             tc = (time.perf_counter() - t0) / reps
-            cpu = {"value": tokens / tc, "unit": UNIT, "cores": cores, "kind": "oracle",
-                   "sample": f"{reps} whole decode steps of this workload (fp64 C oracle, OpenMP over heads)"}
+            cpu = {"value": tokens / tc, "unit": UNIT, "cores": cores, "kind": "oracle", "cpu_model": cpu_model(),
+                   "sample": f"{reps} whole decode steps of this workload (fp64 C oracle, OpenMP over heads)",
+                   "single_thread": oracle_single_thread(case, tokens)}
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": t_ms, "us_per_step": t_ms * 1e3,

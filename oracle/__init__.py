@@ -54,6 +54,11 @@ def _L():
         lib.oracle_decode_step.restype = i32
         lib.oracle_index_append.argtypes = [i32, i32, i64, vp, i32, vp, i32, vp, vp, vp]
         lib.oracle_kv_append.argtypes = [i32, i32, i64, vp, i32, vp, vp, i32, vp, vp, vp, vp, vp, vp, vp]
+        lib.oracle_ring_row.argtypes = [i64, i32, i32]
+        lib.oracle_ring_row.restype = i64
+        lib.oracle_ring_write.argtypes = [i32, i32, i32, i32, vp, vp, i32, vp, vp, vp]
+        lib.oracle_attend_ring.argtypes = [i32, i32, i32, i32, i32, vp, vp, vp, i32, i32, i64, i32, i32, vp]
+        lib.oracle_attend_ring.restype = i32
         lib.oracle_topk.argtypes = [vp, i64, i64, vp, vp]
         lib.oracle_topk.restype = i32
         lib.oracle_decode_step_topk.argtypes = [i32, i32, i32, i64, vp, i32, vp, vp, vp, vp, vp, vp, vp, vp, i64, i32,
@@ -211,6 +216,44 @@ def kv_append(k_pre: np.ndarray, v_new: np.ndarray, Wk: np.ndarray, rope_cos: np
     _L().oracle_kv_append(B, Hkv, ncap, _p(bt), mbps, _p(k_pre), _p(v_new), T, _p(Wk), _p(rc), _p(rs), _p(pos),
                           _p(outs[0]), _p(outs[1]), _p(outs[2]))
     return tuple(outs)
+
+
+def ring_row(n: int, S0: int, W: int) -> int:
+    """Row of position n in a local head's ring of S0 + W rows."""
+    return int(_L().oracle_ring_row(int(n), int(S0), int(W)))
+
+
+def ring_write(k_new: np.ndarray, v_new: np.ndarray, pos: np.ndarray, k_ring: np.ndarray, v_ring: np.ndarray,
+               S0: int, W: int):
+    """Rings [B, Hkv, S0 + W, 128] (uint16 bf16) after writing the new rows
+    [B, Hkv, T, 128] of positions pos[b] + t in order.  Returns updated copies."""
+    k_new = np.ascontiguousarray(k_new, dtype=np.uint16)
+    v_new = np.ascontiguousarray(v_new, dtype=np.uint16)
+    pos = np.ascontiguousarray(pos, dtype=np.int32)
+    kr = np.array(k_ring, dtype=np.uint16, copy=True, order="C")
+    vr = np.array(v_ring, dtype=np.uint16, copy=True, order="C")
+    B, Hkv, T = k_new.shape[:3]
+    if kr.shape != (B, Hkv, S0 + W, D) or vr.shape != kr.shape or W < 1 or S0 < 0 or int(pos.min()) < 0:
+        raise ValueError("ring_write: ring shape, W, S0 or positions")
+    _L().oracle_ring_write(B, Hkv, S0, W, _p(k_new), _p(v_new), T, _p(pos), _p(kr), _p(vr))
+    return kr, vr
+
+
+def attend_ring(q_rope: np.ndarray, k_ring: np.ndarray, v_ring: np.ndarray, b: int, h: int, L: int, window: int,
+                sink: int, S0: int, W: int) -> np.ndarray:
+    """Local head h of sequence b at length L (sink <= S0, window <= W), its
+    keys and values read from the rings."""
+    q = np.ascontiguousarray(q_rope, dtype=np.uint16)
+    kr = np.ascontiguousarray(k_ring, dtype=np.uint16)
+    vr = np.ascontiguousarray(v_ring, dtype=np.uint16)
+    B, Hq = q.shape[:2]
+    Hkv = kr.shape[1]
+    out = np.empty(D, dtype=np.float64)
+    rc = _L().oracle_attend_ring(B, Hq, Hkv, S0, W, _p(q), _p(kr), _p(vr), b, h, int(L), int(window), int(sink),
+                                 _p(out))
+    if rc != 0:
+        raise ValueError("attend_ring: sink beyond S0 or window beyond W")
+    return out
 
 
 def bf16_rne(x: float) -> int:

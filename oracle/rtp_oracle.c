@@ -426,4 +426,52 @@ void oracle_kv_append(int B, int Hkv, int64_t Ncap, const int32_t* block_table, 
             }
 }
 
+/*
+ * Local heads' ring cache: a local head reads only the first `sink` tokens
+ * and the last `window` ones (review, Method: "Adaptive sparse attention" --
+ * local heads keep a sink and a sliding window; Insight 1: only a minority of
+ * heads needs the long context), so its KV head can keep C = S0 + W rows per
+ * sequence (S0 >= sink, W >= window) instead of the whole context.  Reading
+ * of the layout (the pages give none): position n < S0 lives in row n;
+ * position n >= S0 lives in row S0 + (n mod W), so each new position
+ * overwrites the one W places before it.  With S0 and W multiples of 64,
+ * every 64-token block of the context occupies whole aligned 64-row slots.
+ * After positions 0 .. L-1 are written in order, the rows hold
+ * [0, min(S0, L)) and [max(S0, L - W), L).
+ */
+int64_t oracle_ring_row(int64_t n, int S0, int W) { return n < S0 ? n : S0 + n % W; }
+
+/* Write the rows of positions pos_b + t, t = 0 .. T-1, in that order (a later
+ * position overwrites an earlier one of the same row): rings [B, Hkv, C, 128],
+ * new rows [B, Hkv, T, 128]. */
+void oracle_ring_write(int B, int Hkv, int S0, int W, const uint16_t* k_new, const uint16_t* v_new, int T,
+                       const int32_t* pos, uint16_t* k_ring, uint16_t* v_ring) {
+    const int64_t C = (int64_t)S0 + W;
+    for (int b = 0; b < B; ++b)
+        for (int kv = 0; kv < Hkv; ++kv)
+            for (int t = 0; t < T; ++t) {
+                const int64_t src = (((int64_t)b * Hkv + kv) * T + t) * ORC_D;
+                const int64_t dst =
+                    (((int64_t)b * Hkv + kv) * C + oracle_ring_row((int64_t)pos[b] + t, S0, W)) * ORC_D;
+                memcpy(k_ring + dst, k_new + src, ORC_D * sizeof(uint16_t));
+                memcpy(v_ring + dst, v_new + src, ORC_D * sizeof(uint16_t));
+            }
+}
+
+/* Local head h of sequence b at length L: the attention over
+ * [0, min(sink, L)) U [max(0, L - window), L), each key and value read from
+ * its ring row.  Returns 0, or 2 if sink > S0 or window > W (positions the
+ * ring does not hold). */
+int oracle_attend_ring(int B, int Hq, int Hkv, int S0, int W, const uint16_t* q_rope, const uint16_t* k_ring,
+                       const uint16_t* v_ring, int b, int h, int64_t L, int window, int sink, double* out) {
+    if (window > W || sink > S0) return 2;
+    geom g = {B, Hq, Hkv, (int64_t)S0 + W, NULL, 0};
+    int64_t* pos = (int64_t*)malloc(sizeof(int64_t) * (size_t)(L > 0 ? L : 1));
+    const int64_t np = local_positions(L, window, sink, pos);
+    for (int64_t i = 0; i < np; ++i) pos[i] = oracle_ring_row(pos[i], S0, W);
+    attend(&g, q_rope, k_ring, v_ring, b, h, pos, np, out);
+    free(pos);
+    return 0;
+}
+
 uint16_t oracle_bf16_rne(double x) { return bf16_rne(x); }

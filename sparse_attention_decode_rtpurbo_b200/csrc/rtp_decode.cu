@@ -170,23 +170,26 @@ static bool encode_cache_map(CUtensorMap* map, const void* base, long long rows)
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Resident CTAs per SM of a kernel at a dynamic shared-memory size (cached).
+// Resident CTAs per SM of a kernel at a dynamic shared-memory size on the
+// current device (cached per device: the shared-memory limit a kernel is
+// given below is a per-device setting).
 struct OccCache {
     std::mutex mu;
     const void* fn[16];
     size_t smem[16];
+    int dev[16];
     int occ[16];
     int n = 0;
 };
 static int occupancy(const void* fn, size_t smem) {
     static OccCache c;
-    std::lock_guard<std::mutex> lock(c.mu);
-    for (int i = 0; i < c.n; ++i)
-        if (c.fn[i] == fn && c.smem[i] == smem) return c.occ[i];
-    // the limit is raised to the largest block allocation once (lowering it
-    // again for a smaller call would break a later larger one)
     int dev = 0, maxs = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    std::lock_guard<std::mutex> lock(c.mu);
+    for (int i = 0; i < c.n; ++i)
+        if (c.fn[i] == fn && c.smem[i] == smem && c.dev[i] == dev) return c.occ[i];
+    // the limit is raised to the largest block allocation once (lowering it
+    // again for a smaller call would break a later larger one)
     if (cudaDeviceGetAttribute(&maxs, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) return 0;
     if ((size_t)maxs < smem) return 0;
     if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, maxs) != cudaSuccess) return 0;
@@ -196,6 +199,7 @@ static int occupancy(const void* fn, size_t smem) {
     const int slot = c.n < 16 ? c.n++ : 15;
     c.fn[slot] = fn;
     c.smem[slot] = smem;
+    c.dev[slot] = dev;
     c.occ[slot] = n;
     return n;
 }
@@ -208,14 +212,17 @@ static cudaError_t report(cudaError_t e, const char* what) {
     return e;
 }
 
+// SM count of the current device (cached per device).
 static int num_sms() {
-    static std::atomic<int> n{0};
-    int v = n.load();
+    constexpr int MAXDEV = 64;
+    static std::atomic<int> n[MAXDEV];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (dev < 0 || dev >= MAXDEV) return 0;
+    int v = n[dev].load();
     if (!v) {
-        int dev = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess) return 0;
         if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-        n.store(v);
+        n[dev].store(v);
     }
     return v;
 }

@@ -25,12 +25,13 @@ def blocks_to_positions(kept: np.ndarray, L: int) -> np.ndarray:
 
 
 def compare(case, gpu, ref, *, exact_sets: bool = False, check_kstar: bool = False, check_tau: bool = False,
-            heads=None):
-    """Returns a list of failure strings (empty = pass) and a stats dict."""
+            heads=None, batches=None):
+    """Returns a list of failure strings (empty = pass) and a stats dict.
+    heads / batches: compare only these query heads / sequences."""
     fails = []
     stats = {"set_diffs": 0, "heads": 0, "max_err": 0.0}
     assert gpu["status"] == 0, f"device status {gpu['status']}"
-    for b in range(case.B):
+    for b in (range(case.B) if batches is None else batches):
         L = int(case.seq_lens[b])
         nblk = (L + 63) // 64
         for h in (range(case.Hq) if heads is None else heads):

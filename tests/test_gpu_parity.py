@@ -124,6 +124,20 @@ def test_device_input_errors_set_status():
     dc.seq_lens[0] = 300
     dc.run()
     assert dc.step.status() == 0
+    ref = oracle.decode_step(case)
+    for bad in (0, -7):
+        # an empty or negative length is an input error too; the other
+        # sequence's results still match the oracle's
+        dc.seq_lens[0] = bad
+        dc.run()
+        res = dc.results()
+        assert res["status"] == 6
+        res["status"] = 0
+        fails, _ = compare(case, res, ref, batches=[1])
+        assert not fails, "\n".join(fails[:10])
+    dc.seq_lens[0] = 300
+    dc.run()
+    assert dc.step.status() == 0
 
 
 def test_bad_page_id_sets_status():

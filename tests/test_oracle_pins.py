@@ -630,6 +630,102 @@ def test_kv_append_refuses_positions_beyond_the_cache():
 
 
 # ---------------------------------------------------------------------------
+# local heads' ring cache: sink + W rows per (sequence, KV head)
+# ---------------------------------------------------------------------------
+def _marker_rows(positions):
+    """bf16 rows whose first four entries spell the position in base 16
+    (small integers are exact in bf16); the rest zero."""
+    rows = np.zeros((len(positions), 128))
+    for i, n in enumerate(positions):
+        for d in range(4):
+            rows[i, d] = (n >> (4 * d)) & 15
+        rows[i, 4] = 1.0                        # a written row is never all-zero
+    return synth.to_bf16(rows)
+
+
+def _marker_of(row_bits):
+    v = synth.from_bf16(row_bits)
+    if v[4] != 1.0:
+        return None
+    return int(sum(int(v[d]) << (4 * d) for d in range(4)))
+
+
+@pytest.mark.parametrize("S0,W,L,chunk", [(4, 16, 3, 1), (4, 16, 20, 1), (4, 16, 21, 7), (4, 16, 100, 1),
+                                           (4, 16, 100, 40), (0, 8, 50, 3), (3, 1, 9, 2), (64, 64, 1000, 64),
+                                           (64, 128, 1000, 100), (2, 7, 300, 300)])
+def test_ring_keeps_the_head_rows_and_the_last_W_positions(S0, W, L, chunk):
+    """Positions 0 .. L-1 written in order (chunks of `chunk`): the ring then
+    holds exactly [0, min(S0, L)) and the last W positions past S0, each in
+    the row the layout gives it; unwritten rows stay unwritten."""
+    B, Hkv = 1, 1
+    kr = np.zeros((B, Hkv, S0 + W, 128), np.uint16)
+    vr = np.zeros_like(kr)
+    start = 0
+    while start < L:
+        T = min(chunk, L - start)
+        rows = _marker_rows(range(start, start + T)).reshape(B, Hkv, T, 128)
+        kr, vr = oracle.ring_write(rows, rows, np.array([start], np.int32), kr, vr, S0, W)
+        start += T
+    held = {}
+    for r in range(S0 + W):
+        m = _marker_of(kr[0, 0, r])
+        assert m == _marker_of(vr[0, 0, r])
+        if m is not None:
+            held[m] = r
+    want = set(range(min(S0, L))) | set(range(max(S0, L - W), L))
+    assert set(held) == want
+    for n, r in held.items():
+        assert r == oracle.ring_row(n, S0, W)
+        assert (r < S0) == (n < S0)
+
+
+def test_ring_blocks_occupy_aligned_slots():
+    """With S0 = 64 and W a multiple of 64, the 64 positions of any block
+    j >= 1 lie in 64 consecutive rows starting at a multiple of 64."""
+    for W in (64, 256, 4096):
+        for j in (1, 2, 63, 64, 65, 1000):
+            rows = [oracle.ring_row(64 * j + o, 64, W) for o in range(64)]
+            assert rows[0] % 64 == 0 and rows == list(range(rows[0], rows[0] + 64))
+            assert 64 <= rows[0] < 64 + W
+
+
+@pytest.mark.parametrize("L,window,sink,S0,W", [(3000, 256, 4, 64, 256), (3000, 100, 4, 64, 256),
+                                                (200, 256, 4, 64, 256), (3, 256, 4, 64, 256),
+                                                (700, 64, 0, 0, 64), (700, 0, 4, 4, 64), (5000, 1, 0, 0, 1),
+                                                (3001, 200, 4, 4, 200)])
+def test_ring_attention_equals_the_local_head_output(L, window, sink, S0, W):
+    """A local head that reads its keys and values from the ring gives the
+    decode step's local-head output on the full cache, bit for bit (same
+    positions, same order of summation)."""
+    case = synth.make_case("ring", B=2, Hkv=2, G=2, seq_lens=[L, max(1, L // 3)], ret_groups=[], p=[0.9, 0.9],
+                           window=window, sink=sink, seed=L + window, regimes=["gaussian", "gaussian"])
+    ref = oracle.decode_step(case)
+    for b in range(case.B):
+        Lb = int(case.seq_lens[b])
+        kr = np.zeros((case.B, case.Hkv, S0 + W, 128), np.uint16)
+        vr = np.zeros_like(kr)
+        for start in range(0, Lb, 512):
+            T = min(512, Lb - start)
+            pos = np.full(case.B, start, np.int32)
+            kr, vr = oracle.ring_write(case.k_cache[:, :, start:start + T], case.v_cache[:, :, start:start + T],
+                                       pos, kr, vr, S0, W)
+        for h in range(case.Hq):
+            got = oracle.attend_ring(case.q_rope, kr, vr, b, h, Lb, window, sink, S0, W)
+            assert np.array_equal(got, ref["out"][b, h]), (b, h)
+
+
+def test_ring_refuses_a_window_or_sink_it_cannot_hold():
+    case = synth.make_case("ring-w", B=1, Hkv=1, G=1, seq_lens=[100], ret_groups=[], p=[0.9], window=32, sink=4,
+                           seed=3, regimes=["gaussian"])
+    kr = np.zeros((1, 1, 64 + 16, 128), np.uint16)
+    with pytest.raises(ValueError):
+        oracle.attend_ring(case.q_rope, kr, kr, 0, 0, 100, 32, 4, 64, 16)     # window 32 > W 16
+    kr = np.zeros((1, 1, 2 + 64, 128), np.uint16)
+    with pytest.raises(ValueError):
+        oracle.attend_ring(case.q_rope, kr, kr, 0, 0, 100, 32, 4, 2, 64)      # sink 4 > S0 2
+
+
+# ---------------------------------------------------------------------------
 # static top-k (the fixed-budget variant): the k highest scores, ties low index
 # ---------------------------------------------------------------------------
 @pytest.mark.parametrize("seed", range(12))

@@ -132,3 +132,14 @@ def test_kv_append_host_side_checks():
     bad = dims()
     bad.head_dim = 64
     assert call(bad) == 3
+
+
+def test_binding_refuses_host_and_strided_tensors():
+    """The binding passes tensors by address: a host tensor or a strided view
+    is refused before the library is called."""
+    import torch
+
+    with pytest.raises(ValueError, match="device memory"):
+        rtp.decode_step(dims(), torch.zeros(8), 1, 1, 1, 1, 1, 1, HK, 1, 64, 4, 1)
+    with pytest.raises(ValueError, match="contiguous"):
+        rtp.decode_step(dims(), torch.zeros(8, 8).t(), 1, 1, 1, 1, 1, 1, HK, 1, 64, 4, 1)

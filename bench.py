@@ -49,8 +49,9 @@ def parse():
     ap.add_argument("--dense-comparator", action="store_true",
                     help="also time the same captured step with p = 1 and add it to the line as dense_comparator")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--op", choices=["decode", "append"], default="decode",
-                    help="append: time the index-cache append instead of the decode step")
+    ap.add_argument("--op", choices=["decode", "append", "kv_append"], default="decode",
+                    help="append: time the index-cache append instead of the decode step; "
+                         "kv_append: the KV-cache write with the index append")
     return ap.parse_args()
 
 
@@ -274,10 +275,14 @@ def run_reference(args, rank):
 
 
 def bench_append(args):
-    """rtp_index_append alone: a decode-sized append (one new token for each
-    of 16 sequences x 8 KV heads) and a 32K-token chunk of one sequence; HBM
-    bytes = k_pre read (256 B) + k_idx written (32 B) per token and KV head
-    (W^K, 32 KB, stays in L2).  L2 flushed before every timed call."""
+    """rtp_index_append alone (--op append) or rtp_kv_append (--op kv_append):
+    a decode-sized append (one new token for each of 16 sequences x 8 KV
+    heads) and a 32K-token chunk of one sequence.  HBM bytes per token and KV
+    head: k_pre read (256 B) + k_idx written (32 B); kv_append adds the new
+    value read (256 B) and the key and value rows written (512 B), and the
+    angle table row (512 B) once per position.  W^K (32 KB) stays in L2.  L2
+    flushed before every timed call."""
+    kv = args.op == "kv_append"
     import torch
 
     import sparse_attention_decode_rtpurbo_b200 as rtp
@@ -292,6 +297,12 @@ def bench_append(args):
         Wk = (torch.randn((Hkv, 16, 128), generator=g, device=dev) / 11.3).to(torch.bfloat16)
         pos = torch.zeros(B, dtype=torch.int32, device=dev)
         cache = torch.zeros((B, Hkv, ncap, 16), dtype=torch.bfloat16, device=dev)
+        if kv:
+            v_new = torch.randn((B, Hkv, T, 128), generator=g, device=dev).to(torch.bfloat16)
+            ang = torch.rand((ncap, 64), generator=g, device=dev, dtype=torch.float64) * 6.283
+            rc, rs = torch.cos(ang).float(), torch.sin(ang).float()
+            kc = torch.zeros((B, Hkv, ncap, 128), dtype=torch.bfloat16, device=dev)
+            vc = torch.zeros((B, Hkv, ncap, 128), dtype=torch.bfloat16, device=dev)
         dims = rtp.make_dims(B, Hkv, Hkv, ncap)
         stream = torch.cuda.current_stream()
         ts = []
@@ -299,15 +310,19 @@ def bench_append(args):
             flush_w.zero_()
             a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(stream)
-            rtp.index_append(dims, k_pre, Wk, pos, T, cache, None, stream)
+            if kv:
+                rtp.kv_append(dims, k_pre, v_new, Wk, rc, rs, pos, T, cache, kc, vc, None, stream)
+            else:
+                rtp.index_append(dims, k_pre, Wk, pos, T, cache, None, stream)
             z.record(stream)
             z.synchronize()
             if i >= args.warmup:
                 ts.append(a.elapsed_time(z))
         t_ms = statistics.median(ts)
-        nbytes = B * Hkv * T * (256 + 32)
+        nbytes = B * Hkv * T * (256 + 32 + (256 + 512 if kv else 0)) + (T * 512 if kv else 0)
         gbs = nbytes / (t_ms * 1e-3) / 1e9
-        print(json.dumps({"metric": "index-cache append (rtp_index_append)", "op": "append", "case": name,
+        metric = "KV-cache write + index append (rtp_kv_append)" if kv else "index-cache append (rtp_index_append)"
+        print(json.dumps({"metric": metric, "op": args.op, "case": name,
                           "value": gbs, "unit": "GB/s", "us_per_call": t_ms * 1e3, "bytes": nbytes,
                           "peak": peak, "frac": gbs / peak, "peak_source": peak_kind, "steps": args.steps,
                           "warmup": args.warmup, "l2": "flushed (256 MB write) before every call"}), flush=True)
@@ -315,7 +330,7 @@ def bench_append(args):
 
 def main():
     args = parse()
-    if args.op == "append":
+    if args.op in ("append", "kv_append"):
         return bench_append(args)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -325,6 +325,46 @@ rtp_status rtp_decode_step_noalloc(const rtp_dims* dims, const uint16_t* q_pre, 
 rtp_status rtp_index_append(const rtp_dims* dims, const uint16_t* k_pre, const uint16_t* Wk_idx, const int32_t* pos,
                             int32_t num_new, uint16_t* k_idx, uint32_t* device_status, void* stream);
 
+/*
+ * rtp_kv_append -- the KV-cache write of new tokens with the index-cache
+ * append in the same kernel: the key and value rows that rtp_decode_step's
+ * attention reads and the index rows its scoring reads, from one read of the
+ * new pre-RoPE keys.
+ *
+ * Source: review, Method: "Adaptive sparse attention" (the indexer projects
+ * pre-RoPE keys, the attention uses RoPE'd keys) and Insight 2 (RoPE rotates
+ * each frequency pair by an angle proportional to the position).
+ *
+ * For every sequence b, KV head g and new token t, at cache row n = pos[b] + t:
+ *     k_idx row (b, g, n)   = as rtp_index_append
+ *     k_cache row (b, g, n) = bf16( RoPE_n(k_pre[b, g, t]) )
+ *     v_cache row (b, g, n) = v_new[b, g, t]   (bits copied)
+ * RoPE_n rotates the pairs (i, i + 64), i < 64 (rotate-half pairing), by the
+ * caller's angle table row n:
+ *     y_i = k_i cos[n][i] - k_{i+64} sin[n][i],  y_{i+64} = k_{i+64} cos[n][i] + k_i sin[n][i]
+ * each computed as one fp64 fused multiply-add onto the other (exact)
+ * product, then rounded to bf16 (round to nearest even).  The table carries
+ * the model's own RoPE (base, scaling); the kernels never compute angles.
+ *
+ *   dims, k_pre, Wk_idx, pos, num_new, k_idx, device_status, stream: as
+ *              rtp_index_append.
+ *   v_new    : device bf16 [batch, num_kv_heads, num_new, 128], 16-byte aligned.
+ *   rope_cos, rope_sin : device fp32 [max_seq_len, 64], 16-byte aligned; row n
+ *              holds cos and sin of the angles of cache position n.
+ *   k_cache, v_cache : device bf16 caches in rtp_decode_step's layout
+ *              (contiguous [batch, num_kv_heads, max_seq_len, 128] or paged
+ *              [num_pages, num_kv_heads, 64, 128]), 16-byte aligned; only the
+ *              rows above are written.  Owned by the caller.
+ * A row or page id out of range is skipped in all three caches (and reported
+ * through device_status).  Returns the codes of rtp_index_append; also
+ * RTP_ERR_NULL for a NULL k_cache, v_cache, v_new or table, and
+ * RTP_ERR_UNSUPPORTED for one that is not 16-byte aligned.
+ */
+rtp_status rtp_kv_append(const rtp_dims* dims, const uint16_t* k_pre, const uint16_t* v_new, const uint16_t* Wk_idx,
+                         const float* rope_cos, const float* rope_sin, const int32_t* pos, int32_t num_new,
+                         uint16_t* k_idx, uint16_t* k_cache, uint16_t* v_cache, uint32_t* device_status,
+                         void* stream);
+
 /* Static string naming a status code. */
 const char* rtp_status_string(rtp_status status);
 

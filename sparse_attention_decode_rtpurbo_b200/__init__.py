@@ -84,6 +84,8 @@ def _load():
     L.rtp_get_status.argtypes = [ctypes.POINTER(RtpDims), vp]
     L.rtp_index_append.argtypes = [ctypes.POINTER(RtpDims), vp, vp, vp, i32, vp, vp, vp]
     L.rtp_index_append.restype = ctypes.c_int
+    L.rtp_kv_append.argtypes = [ctypes.POINTER(RtpDims), vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp]
+    L.rtp_kv_append.restype = ctypes.c_int
     L.rtp_get_status.restype = ctypes.c_int
     L.rtp_status_string.argtypes = [ctypes.c_int]
     L.rtp_status_string.restype = ctypes.c_char_p
@@ -210,6 +212,19 @@ def index_append(dims: RtpDims, k_pre, Wk_idx, pos, num_new: int, k_idx, device_
                               _ptr(device_status), st)
     if rc != RTP_OK:
         raise RtpError(rc, "rtp_index_append")
+
+
+def kv_append(dims: RtpDims, k_pre, v_new, Wk_idx, rope_cos, rope_sin, pos, num_new: int, k_idx, k_cache, v_cache,
+              device_status=None, stream=None) -> None:
+    """rtp_kv_append: for the num_new new tokens of every sequence, cache rows
+    n = pos[b] + t receive k_idx = bf16(W^K[g] . k_pre), k_cache =
+    bf16(RoPE_n(k_pre)) with the angle table rows rope_cos[n], rope_sin[n]
+    (fp32 [max_seq_len, 64]), and v_cache = v_new."""
+    st = 0 if stream is None else (stream if isinstance(stream, int) else stream.cuda_stream)
+    rc = lib.rtp_kv_append(ctypes.byref(dims), _ptr(k_pre), _ptr(v_new), _ptr(Wk_idx), _ptr(rope_cos), _ptr(rope_sin),
+                           _ptr(pos), int(num_new), _ptr(k_idx), _ptr(k_cache), _ptr(v_cache), _ptr(device_status), st)
+    if rc != RTP_OK:
+        raise RtpError(rc, "rtp_kv_append")
 
 
 def get_status(dims: RtpDims, stream=None) -> int:

@@ -578,9 +578,12 @@ extern "C" rtp_status rtp_ring_write(const rtp_dims* d, const uint16_t* k_new, c
 // ---------------------------------------------------------------------------
 // index-cache append
 // ---------------------------------------------------------------------------
-extern "C" rtp_status rtp_index_append(const rtp_dims* d, const uint16_t* k_pre, const uint16_t* Wk_idx,
-                                       const int32_t* pos, int32_t num_new, uint16_t* k_idx, uint32_t* device_status,
-                                       void* stream) {
+// The index-cache append, with the KV-cache write when k_cache is given.
+static rtp_status append_impl(const rtp_dims* d, const uint16_t* k_pre, const uint16_t* v_new, const uint16_t* Wk_idx,
+                              const float* rope_cos, const float* rope_sin, const int32_t* pos, int32_t num_new,
+                              uint16_t* k_idx, uint16_t* k_cache, uint16_t* v_cache, uint32_t* device_status,
+                              void* stream) {
+    const bool kv = k_cache != nullptr;
     if (!d) return RTP_ERR_NULL;
     if (d->head_dim != D || d->idx_dim != R || d->block_size != BLK) return RTP_ERR_UNSUPPORTED;
     if (d->batch < 1 || d->num_kv_heads < 1 || num_new < 0) return RTP_ERR_SHAPE;
@@ -592,9 +595,14 @@ extern "C" rtp_status rtp_index_append(const rtp_dims* d, const uint16_t* k_pre,
     }
     if (num_new == 0) return RTP_OK;
     if (!k_pre || !Wk_idx || !pos || !k_idx) return RTP_ERR_NULL;
+    if (kv && (!v_new || !rope_cos || !rope_sin || !v_cache)) return RTP_ERR_NULL;
     if (((uintptr_t)k_pre | (uintptr_t)Wk_idx) & 15u) return RTP_ERR_UNSUPPORTED;   // 16-byte vector loads
     if ((uintptr_t)k_idx & 7u) return RTP_ERR_UNSUPPORTED;                            // 8-byte stores of 4 entries
+    if (kv && (((uintptr_t)v_new | (uintptr_t)rope_cos | (uintptr_t)rope_sin | (uintptr_t)k_cache |
+                (uintptr_t)v_cache) & 15u))
+        return RTP_ERR_UNSUPPORTED;                                                    // 16-byte loads and stores
     AppendParams A;
+    memset(&A, 0, sizeof(A));
     A.B = d->batch;
     A.Hkv = d->num_kv_heads;
     A.T = num_new;
@@ -607,11 +615,33 @@ extern "C" rtp_status rtp_index_append(const rtp_dims* d, const uint16_t* k_pre,
     A.block_table = d->block_table;
     A.k_idx = k_idx;
     A.status = device_status;
+    A.v_new = v_new;
+    A.rope_cos = rope_cos;
+    A.rope_sin = rope_sin;
+    A.k_cache = k_cache;
+    A.v_cache = v_cache;
     const int64_t total = (int64_t)A.B * A.Hkv * A.T * (R / APPEND_ROWS);
     const int64_t grid = (total + APPEND_THREADS - 1) / APPEND_THREADS;
     if (grid > 0x7FFFFFFF) return RTP_ERR_UNSUPPORTED;
-    index_append_kernel<<<(unsigned)grid, APPEND_THREADS, 0, (cudaStream_t)stream>>>(A);
-    return report(cudaGetLastError(), "index append launch") == cudaSuccess ? RTP_OK : RTP_ERR_CUDA;
+    if (kv) append_kernel<true><<<(unsigned)grid, APPEND_THREADS, 0, (cudaStream_t)stream>>>(A);
+    else append_kernel<false><<<(unsigned)grid, APPEND_THREADS, 0, (cudaStream_t)stream>>>(A);
+    return report(cudaGetLastError(), "append launch") == cudaSuccess ? RTP_OK : RTP_ERR_CUDA;
+}
+
+extern "C" rtp_status rtp_index_append(const rtp_dims* d, const uint16_t* k_pre, const uint16_t* Wk_idx,
+                                       const int32_t* pos, int32_t num_new, uint16_t* k_idx, uint32_t* device_status,
+                                       void* stream) {
+    return append_impl(d, k_pre, nullptr, Wk_idx, nullptr, nullptr, pos, num_new, k_idx, nullptr, nullptr,
+                       device_status, stream);
+}
+
+extern "C" rtp_status rtp_kv_append(const rtp_dims* d, const uint16_t* k_pre, const uint16_t* v_new,
+                                    const uint16_t* Wk_idx, const float* rope_cos, const float* rope_sin,
+                                    const int32_t* pos, int32_t num_new, uint16_t* k_idx, uint16_t* k_cache,
+                                    uint16_t* v_cache, uint32_t* device_status, void* stream) {
+    if (!k_cache) return RTP_ERR_NULL;
+    return append_impl(d, k_pre, v_new, Wk_idx, rope_cos, rope_sin, pos, num_new, k_idx, k_cache, v_cache,
+                       device_status, stream);
 }
 
 extern "C" const char* rtp_status_string(rtp_status status) {

@@ -169,6 +169,33 @@ def test_ring_write_host_side_checks():
     assert call(d, vn=fake + 4) == 3
 
 
+def test_kv_append_host_side_checks():
+    """rtp_kv_append: bad arguments are refused before any CUDA call."""
+    fake = 4096   # never dereferenced: every call below returns first
+    d = dims()
+
+    def call(dd, k_pre=fake, v_new=fake, wk=fake, cs=fake, sn=fake, pos=fake, n=1, kidx=fake, kc=fake, vc=fake):
+        return rtp.lib.rtp_kv_append(ctypes.byref(dd) if dd is not None else None, k_pre, v_new, wk, cs, sn, pos, n,
+                                     kidx, kc, vc, None, None)
+
+    assert call(None) == 1                           # NULL dims
+    assert call(d, kc=None) == 1                     # NULL key cache
+    assert call(d, vc=None) == 1                     # NULL value cache
+    assert call(d, v_new=None) == 1                  # NULL new values
+    assert call(d, cs=None) == 1                     # NULL angle table
+    assert call(d, n=0) == 0                         # nothing to append
+    assert call(d, n=-1) == 2
+    assert call(d, n=4097) == 2                      # more than the capacity
+    assert call(d, v_new=fake + 8) == 3              # 16-byte alignment of every row-wise operand
+    assert call(d, sn=fake + 4) == 3
+    assert call(d, kc=fake + 2) == 3
+    assert call(d, vc=fake + 8) == 3
+    assert call(d, kidx=fake + 4) == 3               # k_idx: 8-byte aligned, as rtp_index_append
+    bad = dims()
+    bad.head_dim = 64
+    assert call(bad) == 3
+
+
 def test_binding_refuses_host_and_strided_tensors():
     """The binding passes tensors by address: a host tensor or a strided view
     is refused before the library is called."""

@@ -237,11 +237,32 @@ static int grid_cap() {
     return n >= 1 ? n : MAX_GRID;
 }
 
+// RTP_SINGLE_LAUNCH=1 in the environment (read at every call): the step
+// runs as one launch (step_kernel: streaming phase, grid barrier, retrieval
+// phase) instead of two.  Results do not depend on it.
+static bool single_launch() {
+    const char* v = getenv("RTP_SINGLE_LAUNCH");
+    return v && atoi(v) == 1;
+}
+
 template <int G>
 static cudaError_t launch(const KParams& K, const Plan& pl, cudaStream_t s, void* const* ev, unsigned ev_flags) {
     const int sms = num_sms();
     if (!sms) return report(cudaErrorUnknown, "SM count");
     const int cap = std::min(MAX_GRID, grid_cap());
+    if (pl.n_rg > 0 && single_launch()) {
+        // one resident wave with room for either phase's shared memory (the
+        // retrieval phase's grid barriers need every CTA resident; surplus
+        // CTAs take no share of the streaming phase)
+        const size_t smem = std::max(asmem_bytes<G>(pl.B), bsmem_bytes<G>(pl.B * pl.n_rg));
+        const int occ = occupancy((const void*)step_kernel<G>, smem);
+        if (occ < 1) return report(cudaErrorInvalidConfiguration, "step kernel occupancy");
+        const int grid = std::min(cap, occ * sms);
+        step_kernel<G><<<(unsigned)grid, THREADS, smem, s>>>(K);
+        cudaError_t e = report(cudaGetLastError(), "step kernel launch");
+        if (ev) cudaEventRecordWithFlags((cudaEvent_t)ev[1], s, ev_flags);   // (no phase boundary to mark)
+        return e;
+    }
     // streaming kernel: as many resident CTAs as the tiles can use
     {
         const size_t smem = asmem_bytes<G>(pl.B);

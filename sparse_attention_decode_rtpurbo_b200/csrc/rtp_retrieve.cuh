@@ -1113,23 +1113,14 @@ __device__ __forceinline__ void warp_prefix(int* pre, int n, F cnt, int lane) {
 }
 
 // ---------------------------------------------------------------------------
-// the kernel
+// the retrieval phase: its shared-memory set-up, and its body once the
+// streaming phase's results are visible (after the streaming grid completed,
+// or, in the single launch, after a grid barrier)
 // ---------------------------------------------------------------------------
 template <int G>
-__global__ void __launch_bounds__(THREADS, 2) retrieve_kernel(const __grid_constant__ KParams K) {
+__device__ __forceinline__ void r_setup(const Params& P, int tid) {
     BSmem<G>& S = bsmem<G>();
     constexpr int NST = BSmem<G>::NST;
-    const Params& P = K.P;
-    const int tid = threadIdx.x, lane = tid & 31;
-    const bool copier = tid >= CONSUMERS;
-    // grid barrier; thread 0's wait goes to debug sum 31
-    auto gsync = [&]() {
-        const long long t0 = clock64();
-        const bool r = grid_sync(P, S);
-        if (tid == 0 && P.dbg_trace) S.acct[15] += (unsigned long long)(clock64() - t0);
-        return r;
-    };
-    int* pre = S.pre;
     if (tid == 0) {
         for (int i = 0; i < NST; ++i) {
             mbar_init(&S.full[i], 1);
@@ -1143,9 +1134,24 @@ __global__ void __launch_bounds__(THREADS, 2) retrieve_kernel(const __grid_const
         S.resident = 0;
     }
     if (tid >= 32) copy_tab(P.tab, S.tab, tid - 32, THREADS - 32);
-    // everything below reads the streaming kernel's results: wait for that
-    // grid to complete (this launch overlaps only its tail)
-    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// single: the single launch, whose transition barrier always counts in
+// P.sync->barrier, so the last CTA out always clears the coordination words
+template <int G>
+__device__ __forceinline__ void r_body(const KParams& K, bool single) {
+    BSmem<G>& S = bsmem<G>();
+    const Params& P = K.P;
+    const int tid = threadIdx.x, lane = tid & 31;
+    const bool copier = tid >= CONSUMERS;
+    // grid barrier; thread 0's wait goes to debug sum 31
+    auto gsync = [&]() {
+        const long long t0 = clock64();
+        const bool r = grid_sync(P, S);
+        if (tid == 0 && P.dbg_trace) S.acct[15] += (unsigned long long)(clock64() - t0);
+        return r;
+    };
+    int* pre = S.pre;
     if (tid == 0) S.base = __ldcg(&P.sync->kb_work);
     __syncthreads();
     const bool work = S.base != 0;   // nothing left when every group was settled in the streaming kernel
@@ -1287,9 +1293,10 @@ __global__ void __launch_bounds__(THREADS, 2) retrieve_kernel(const __grid_const
         }
     }
     // the last CTA out clears the call's coordination words (none was set
-    // when every group was settled in the streaming kernel: no count then)
+    // when every group was settled in the streaming kernel: no count then,
+    // except for the single launch's transition barrier)
     __syncthreads();
-    if (work && tid == 0) {
+    if ((work || single) && tid == 0) {
         trace_max(P, 5);
         __threadfence();
         if (atomicAdd(&P.sync->exit_count, 1u) == gridDim.x - 1) {
@@ -1310,6 +1317,54 @@ __global__ void __launch_bounds__(THREADS, 2) retrieve_kernel(const __grid_const
             __threadfence();
         }
     }
+}
+
+__device__ __forceinline__ void mbar_inval(uint64_t* bar) {
+    asm volatile("mbarrier.inval.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// The whole decode step in one launch: the streaming phase, then (after a
+// grid barrier that stands for the retrieval kernel's wait on the streaming
+// grid) the retrieval phase in the same shared memory.  When every group was
+// settled in the streaming phase, the CTAs only clear the call's words and
+// drop the stored scores: no second launch.  One resident wave (the
+// retrieval phase's grid barriers need it).
+template <int G>
+__global__ void __launch_bounds__(THREADS, 2) step_kernel(const __grid_constant__ KParams K) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const Params& P = K.P;
+    const int tid = threadIdx.x;
+    if (smem_u32(smem_raw) & 1023u) {   // (the same for every CTA: none waits for another)
+        if (tid == 0) set_status(P, 5u);
+        return;
+    }
+    s_body<G, true>(K);
+    __syncthreads();
+    // the streaming phase's ring barriers end here (no copy is in flight:
+    // its copy warp waited for its last tiles); the memory becomes the
+    // retrieval phase's
+    if (tid == 0) {
+        ASmem<G>& A = *reinterpret_cast<ASmem<G>*>(smem_raw);
+        for (int i = 0; i < ASmem<G>::NST; ++i) {
+            mbar_inval(&A.full[i]);
+            mbar_inval(&A.empty[i]);
+        }
+    }
+    __syncthreads();
+    r_setup<G>(P, tid);
+    __syncthreads();
+    grid_sync(P, bsmem<G>());   // a timeout sets S.abort: the body then skips its work
+    r_body<G>(K, true);
+}
+
+template <int G>
+__global__ void __launch_bounds__(THREADS, 2) retrieve_kernel(const __grid_constant__ KParams K) {
+    const int tid = threadIdx.x;
+    r_setup<G>(K.P, tid);
+    // everything below reads the streaming kernel's results: wait for that
+    // grid to complete (this launch overlaps only its tail)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    r_body<G>(K, false);
 }
 
 }  // namespace rtp

@@ -884,8 +884,10 @@ __device__ __forceinline__ void a_consumers(const KParams& K, ASmem<G>& S, AWalk
 // ---------------------------------------------------------------------------
 // the kernel
 // ---------------------------------------------------------------------------
-template <int G>
-__global__ void __launch_bounds__(THREADS, 2) stream_kernel(const __grid_constant__ KParams K) {
+// The streaming phase.  SINGLE: part of the single launch (no dependent
+// grid to release; every thread returns here, the copy warp included).
+template <int G, bool SINGLE>
+__device__ __forceinline__ void s_body(const KParams& K) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];   // no static shared memory: the base is aligned
     ASmem<G>& S = *reinterpret_cast<ASmem<G>*>(smem_raw);
     constexpr int NST = ASmem<G>::NST;
@@ -911,7 +913,7 @@ __global__ void __launch_bounds__(THREADS, 2) stream_kernel(const __grid_constan
     }
     // the retrieval kernel may be scheduled now; it waits for this grid's
     // completion before it reads anything this grid writes
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    if constexpr (!SINGLE) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (tid >= 32) copy_tab(P.tab, S.tab, tid - 32, THREADS - 32);
     // tiles per sequence (score tiles of all retrieval groups, then local
     // tiles of all local groups), prefix-summed by warp 0
@@ -973,6 +975,11 @@ __global__ void __launch_bounds__(THREADS, 2) stream_kernel(const __grid_constan
     }
     a_consumers<G>(K, S, wk, pre_s, pre_l, tid);
     if (tid == 0) trace_max(P, 5);
+}
+
+template <int G>
+__global__ void __launch_bounds__(THREADS, 2) stream_kernel(const __grid_constant__ KParams K) {
+    s_body<G, false>(K);
 }
 
 }  // namespace rtp

@@ -54,6 +54,7 @@ def _L():
         lib.oracle_decode_step.restype = i32
         lib.oracle_index_append.argtypes = [i32, i32, i64, vp, i32, vp, i32, vp, vp, vp]
         lib.oracle_kv_append.argtypes = [i32, i32, i64, vp, i32, vp, vp, i32, vp, vp, vp, vp, vp, vp, vp]
+        lib.oracle_prefill.argtypes = [i32, i32, i32, i64, vp, i32, vp, vp, vp, vp, vp, i32, i32, i32, vp]
         lib.oracle_ring_row.argtypes = [i64, i32, i32]
         lib.oracle_ring_row.restype = i64
         lib.oracle_ring_write.argtypes = [i32, i32, i32, i32, vp, vp, i32, vp, vp, vp]
@@ -216,6 +217,24 @@ def kv_append(k_pre: np.ndarray, v_new: np.ndarray, Wk: np.ndarray, rope_cos: np
     _L().oracle_kv_append(B, Hkv, ncap, _p(bt), mbps, _p(k_pre), _p(v_new), T, _p(Wk), _p(rc), _p(rs), _p(pos),
                           _p(outs[0]), _p(outs[1]), _p(outs[2]))
     return tuple(outs)
+
+
+def prefill(case, q: np.ndarray, pos: np.ndarray) -> np.ndarray:
+    """Prefill attention of T queries per sequence (q: uint16 bf16 [B, Hq, T,
+    128], RoPE'd) at positions pos[b] + t, over the case's caches: retrieval
+    heads attend to [0, m], local heads to the sink and the last `window`
+    positions up to m.  Returns out [B, Hq, T, 128] fp64."""
+    B, Hq, Hkv, Ncap, bt, mbps = _geom(case)
+    q = np.ascontiguousarray(q, dtype=np.uint16)
+    pos = np.ascontiguousarray(pos, dtype=np.int32)
+    T = q.shape[2]
+    if q.shape[:2] != (B, Hq) or int(pos.min()) < 0 or int(pos.max()) + T > Ncap:
+        raise ValueError("prefill: query shape or positions beyond the cache")
+    out = np.empty((B, Hq, T, D), dtype=np.float64)
+    _L().oracle_prefill(B, Hq, Hkv, Ncap, _p(bt), mbps, _p(q), _p(case.k_cache), _p(case.v_cache),
+                        _p(np.ascontiguousarray(case.head_kind, dtype=np.uint8)), _p(pos), T, int(case.window),
+                        int(case.sink), _p(out))
+    return out
 
 
 def ring_row(n: int, S0: int, W: int) -> int:

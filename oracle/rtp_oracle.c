@@ -191,10 +191,18 @@ void oracle_index_scores(int B, int Hq, int Hkv, int64_t Ncap, const int32_t* bl
 }
 
 /* exact softmax attention of head h of sequence b over the positions pos[0..npos) */
+static void attend_q(const geom* g, const uint16_t* q, const uint16_t* k_cache, const uint16_t* v_cache, int b,
+                     int kv, const int64_t* pos, int64_t npos, double* out);
+
 static void attend(const geom* g, const uint16_t* q_rope, const uint16_t* k_cache, const uint16_t* v_cache, int b,
                    int h, const int64_t* pos, int64_t npos, double* out) {
-    int G = g->Hq / g->Hkv, kv = h / G;
-    const uint16_t* q = q_rope + ((int64_t)b * g->Hq + h) * ORC_D;
+    const int G = g->Hq / g->Hkv;
+    attend_q(g, q_rope + ((int64_t)b * g->Hq + h) * ORC_D, k_cache, v_cache, b, h / G, pos, npos, out);
+}
+
+/* softmax(q . k_n / sqrt(128)) over the positions, times v_n, for one query vector q of KV head kv */
+static void attend_q(const geom* g, const uint16_t* q, const uint16_t* k_cache, const uint16_t* v_cache, int b,
+                     int kv, const int64_t* pos, int64_t npos, double* out) {
     double qd[ORC_D];
     for (int d = 0; d < ORC_D; ++d) qd[d] = bf(q[d]);
     double* a = (double*)malloc(sizeof(double) * (size_t)(npos > 0 ? npos : 1));
@@ -472,6 +480,41 @@ int oracle_attend_ring(int B, int Hq, int Hkv, int S0, int W, const uint16_t* q_
     attend(&g, q_rope, k_ring, v_ring, b, h, pos, np, out);
     free(pos);
     return 0;
+}
+
+/*
+ * Prefill attention of a chunk of T queries per sequence (the pages' second
+ * workload; review, Method: "Adaptive sparse attention" -- in prefill the
+ * retrieval heads attend densely and the local heads to their sink and
+ * sliding window; Experiments: the prefill speedups).  Query t of sequence b
+ * sits at position m = pos_b + t and attends causally, itself included:
+ *   retrieval head : positions [0, m]
+ *   local head     : [0, min(sink, m + 1)) U [max(0, m + 1 - window), m + 1)
+ * (the decode step's sets at length L = m + 1).  The cache must already hold
+ * the keys and values of positions up to pos_b + T - 1.  q: [B, Hq, T, 128]
+ * bf16 (RoPE'd); out: [B, Hq, T, 128] fp64.
+ */
+void oracle_prefill(int B, int Hq, int Hkv, int64_t Ncap, const int32_t* block_table, int mbps, const uint16_t* q,
+                    const uint16_t* k_cache, const uint16_t* v_cache, const uint8_t* head_kind, const int32_t* pos,
+                    int T, int window, int sink, double* out) {
+    geom g = {B, Hq, Hkv, Ncap, block_table, mbps};
+    const int G = Hq / Hkv;
+    int64_t* ps = (int64_t*)malloc(sizeof(int64_t) * (size_t)(Ncap > 0 ? Ncap : 1));
+    for (int b = 0; b < B; ++b)
+        for (int h = 0; h < Hq; ++h)
+            for (int t = 0; t < T; ++t) {
+                const int64_t L = (int64_t)pos[b] + t + 1;     /* positions 0 .. m */
+                int64_t np;
+                if (head_kind[h]) {
+                    for (int64_t n = 0; n < L; ++n) ps[n] = n;
+                    np = L;
+                } else {
+                    np = local_positions(L, window, sink, ps);
+                }
+                const int64_t qi = ((int64_t)b * Hq + h) * T + t;
+                attend_q(&g, q + qi * ORC_D, k_cache, v_cache, b, h / G, ps, np, out + qi * ORC_D);
+            }
+    free(ps);
 }
 
 uint16_t oracle_bf16_rne(double x) { return bf16_rne(x); }

@@ -91,10 +91,18 @@ def status_string(code: int) -> str:
 
 
 def _ptr(x) -> Optional[int]:
+    """The device address of an argument: None, a raw address (int), or a
+    tensor, which must be contiguous and in device memory (the library reads
+    it as a dense array at that address)."""
     if x is None:
         return None
     if isinstance(x, int):
         return x
+    if hasattr(x, "is_contiguous"):
+        if not x.is_contiguous():
+            raise ValueError("rtp: tensor arguments must be contiguous")
+        if not getattr(x, "is_cuda", False):
+            raise ValueError("rtp: tensor arguments must be in device memory")
     return x.data_ptr()
 
 

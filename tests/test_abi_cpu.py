@@ -105,3 +105,14 @@ def test_index_append_host_side_checks():
     assert call(d, fake + 2, fake, fake, 1, fake, None, None) == 3                     # k_pre not 16-byte aligned
     assert call(d, fake, fake, fake, 1, fake + 4, None, None) == 3                     # k_idx not 8-byte aligned
     assert call(dims(num_kv_heads=65, num_q_heads=65), fake, fake, fake, 1, fake, None, None) == 3
+
+
+def test_binding_refuses_host_and_strided_tensors():
+    """The binding passes tensors by address: a host tensor or a strided view
+    is refused before the library is called."""
+    import torch
+
+    with pytest.raises(ValueError, match="device memory"):
+        rtp.decode_step(dims(), torch.zeros(8), 1, 1, 1, 1, 1, 1, HK, 1, 64, 4, 1)
+    with pytest.raises(ValueError, match="contiguous"):
+        rtp.decode_step(dims(), torch.zeros(8, 8).t(), 1, 1, 1, 1, 1, 1, HK, 1, 64, 4, 1)

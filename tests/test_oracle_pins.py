@@ -726,6 +726,81 @@ def test_ring_refuses_a_window_or_sink_it_cannot_hold():
 
 
 # ---------------------------------------------------------------------------
+# prefill: causal attention of a chunk of queries, dense for retrieval heads,
+# sink + window for local heads
+# ---------------------------------------------------------------------------
+def _prefill_case(L, window, sink, paged=False, seed=5):
+    # mixed KV groups (retrieval and local heads in each): every cache row valid
+    hk = np.array([1, 0, 0, 1, 1, 0, 0, 1], np.uint8)
+    return synth.make_case("prefill", B=2, Hkv=2, G=4, seq_lens=[L, L - 7], ret_groups=[], head_kind=hk,
+                           p=[1.0, 1.0], window=window, sink=sink, seed=seed, regimes=["gaussian", "gaussian"],
+                           paged=paged)
+
+
+@pytest.mark.parametrize("paged", [False, True])
+def test_prefill_uniform_keys_give_the_mean_of_the_attended_values(paged):
+    """All keys equal: every query weighs its attended positions equally, so
+    its output is the mean of their values.  Values spell the position in
+    base 8, so the mean fixes the position set: [0, m] for retrieval heads,
+    the sink and the last `window` positions up to m for local heads."""
+    L, window, sink, T = 300, 40, 3, 50
+    case = _prefill_case(L, window, sink, paged=paged)
+    ones = synth.to_bf16(np.full(128, 0.25))
+    vals = np.zeros((case.Ncap, 128))
+    n = np.arange(case.Ncap)
+    vals[:, 0], vals[:, 1], vals[:, 2], vals[:, 3] = n % 8, (n // 8) % 8, (n // 64) % 8, 1.0
+    vrows = synth.to_bf16(vals)
+    for b in range(case.B):
+        for g in range(case.Hkv):
+            for m in range(int(case.seq_lens[b])):
+                if case.block_table is None:
+                    case.k_cache[b, g, m], case.v_cache[b, g, m] = ones, vrows[m]
+                else:
+                    pg = case.block_table[b, m // 64]
+                    case.k_cache[pg, g, m % 64], case.v_cache[pg, g, m % 64] = ones, vrows[m]
+    pos = np.array([L - T, L - 7 - T], np.int32)
+    rng = np.random.default_rng(1)
+    q = synth.to_bf16(rng.standard_normal((case.B, case.Hq, T, 128)))
+    out = oracle.prefill(case, q, pos)
+    for b in range(case.B):
+        for h in range(case.Hq):
+            for t in range(T):
+                m = int(pos[b]) + t
+                if case.head_kind[h]:
+                    S = np.arange(m + 1)
+                else:
+                    S = np.array(sorted(set(range(min(sink, m + 1))) | set(range(max(0, m + 1 - window), m + 1))))
+                want = [np.mean(S % 8), np.mean((S // 8) % 8), np.mean((S // 64) % 8), 1.0]
+                assert np.allclose(out[b, h, t, :4], want, rtol=0, atol=1e-12), (b, h, t)
+
+
+def test_prefill_first_position_attends_only_itself():
+    case = _prefill_case(200, 16, 4)
+    rng = np.random.default_rng(2)
+    q = synth.to_bf16(rng.standard_normal((case.B, case.Hq, 3, 128)))
+    out = oracle.prefill(case, q, np.zeros(case.B, np.int32))
+    for b in range(case.B):
+        for h in range(case.Hq):
+            assert np.array_equal(out[b, h, 0], synth.from_bf16(case.v_cache[b, h // 4, 0]))
+
+
+@pytest.mark.parametrize("paged", [False, True])
+def test_prefill_last_query_is_the_decode_step(paged):
+    """The chunk's last query, at position L - 1 with the decode query's
+    vector, attends exactly the decode step's positions at length L (p = 1 for
+    the retrieval heads): the same output, bit for bit."""
+    L, T = 900, 33
+    case = _prefill_case(L, 100, 4, paged=paged, seed=9)
+    ref = oracle.decode_step(case)
+    rng = np.random.default_rng(3)
+    q = synth.to_bf16(rng.standard_normal((case.B, case.Hq, T, 128)))
+    q[:, :, T - 1] = case.q_rope
+    pos = (case.seq_lens - T).astype(np.int32)
+    out = oracle.prefill(case, q, pos)
+    assert np.array_equal(out[:, :, T - 1], ref["out"])
+
+
+# ---------------------------------------------------------------------------
 # static top-k (the fixed-budget variant): the k highest scores, ties low index
 # ---------------------------------------------------------------------------
 @pytest.mark.parametrize("seed", range(12))

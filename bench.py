@@ -44,6 +44,8 @@ def parse():
     ap.add_argument("--scale", type=int, default=1, help="divide the workload's context lengths (profiling runs)")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--dense", action="store_true", help="p = 1 for every sequence (dense comparator)")
+    ap.add_argument("--dense-comparator", action="store_true",
+                    help="also time the same captured step with p = 1 and add it to the line as dense_comparator")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--op", choices=["decode", "append"], default="decode",
                     help="append: time the index-cache append instead of the decode step")
@@ -109,7 +111,9 @@ def algorithmic_bytes(case, kept):
     """Algorithmic byte count of one step (the roofline numerator): index cache of every retrieval KV
     group + the union of kept K/V blocks per retrieval group (rows < L) +
     sink/window rows of every local KV group.  512 B per K+V row, 32 B per
-    index row."""
+    index row.  A KV group with both kinds of heads counts the union of the
+    rows it reads once (its sink/window rows inside kept blocks are not
+    counted again under "local")."""
     import synth
 
     G = case.G
@@ -120,15 +124,16 @@ def algorithmic_bytes(case, kept):
         rows = np.minimum(64, L - 64 * np.arange(nblk))
         for g in range(case.Hkv):
             heads = range(g * G, (g + 1) * G)
+            uni = np.zeros(nblk, dtype=bool)
             if any(case.head_kind[h] for h in heads):
                 idx += L * 32
-                uni = np.zeros(nblk, dtype=bool)
                 for h in heads:
                     if case.head_kind[h]:
                         uni |= kept[b, h, :nblk].astype(bool)
                 kv += int(rows[uni].sum()) * 512
             if any(not case.head_kind[h] for h in heads):
-                loc += synth.local_positions(L, case.window, case.sink).size * 512
+                pos = synth.local_positions(L, case.window, case.sink)
+                loc += int(np.count_nonzero(~uni[pos // 64])) * 512
     return {"index": idx, "kept_kv": kv, "local": loc, "total": idx + kv + loc}
 
 
@@ -482,10 +487,32 @@ def main():
     if dc.step.status() != 0:
         raise SystemExit("device status set during the timed steps")
 
+    # ---- dense comparator: the same captured step with p = 1 for every
+    # sequence (every block of every retrieval head), the stand-in for the
+    # pages' dense-attention baseline; the graph reads p from dc.p ----
+    dense_ms, dense_status = 0.0, 0
+    if args.dense_comparator and not args.dense and case.head_kind.any():
+        dc.p.fill_(1.0)
+        dts = []
+        for i in range(max(3, args.warmup) + args.steps):
+            flush()
+            a = torch.cuda.Event(enable_timing=True)
+            z = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            graph.replay()
+            z.record(stream)
+            z.synchronize()
+            if i >= max(3, args.warmup):
+                dts.append(a.elapsed_time(z))
+        dc.p.copy_(torch.from_numpy(case.p.astype(np.float32)).to(dev))
+        torch.cuda.synchronize(dev)
+        dense_status = dc.step.status()          # reported, not fatal: the main line stands
+        dense_ms = statistics.mean(dts)
+
     # ---- max over ranks ----
-    vals = max_over_ranks([t_ms, e2e_t] + [phase_ms[n] for n in rtp.PHASES], world, dev)
-    t_ms, e2e_t = vals[0], vals[1]
-    phase_ms = {n: vals[2 + k] for k, n in enumerate(rtp.PHASES)}
+    vals = max_over_ranks([t_ms, e2e_t, dense_ms] + [phase_ms[n] for n in rtp.PHASES], world, dev)
+    t_ms, e2e_t, dense_ms = vals[0], vals[1], vals[2]
+    phase_ms = {n: vals[3 + k] for k, n in enumerate(rtp.PHASES)}
 
     tokens = float(case.seq_lens.sum())
     value = world * tokens / (t_ms * 1e-3)
@@ -541,6 +568,11 @@ def main():
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clocks,
             "cpu_baseline": cpu,
+            "dense_comparator": ({"us_per_step": dense_ms * 1e3, "value": world * tokens / (dense_ms * 1e-3),
+                                  "unit": UNIT, "speedup_of_sparse": dense_ms / t_ms,
+                                  "device_status": dense_status,
+                                  "what": "the same step with p = 1 (every block of every retrieval head)"}
+                                 if dense_ms > 0 else None),
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -52,3 +52,37 @@ def test_stage_inputs_views_and_one_copy():
     dbuf.copy_(hbuf)
     for t, v in zip(tensors, views):
         assert torch.equal(v.view(torch.uint8), t.view(torch.uint8))
+
+
+def test_algorithmic_bytes_by_hand():
+    """The roofline numerator on hand-countable cases: index rows per
+    retrieval group, the union of the group's kept blocks (the last block
+    partial), sink/window rows per local group, and a group with both kinds
+    counting the rows it reads once."""
+    import numpy as np
+
+    import bench
+    import synth
+
+    # two KV groups of 2 heads: group 0 retrieval, group 1 local; L = 200 (4 blocks, last 8 rows)
+    case = synth.make_case("bytes", B=1, Hkv=2, G=2, seq_lens=[200], ret_groups=[0], p=[0.9], window=50, sink=4,
+                           seed=1, regimes=["gaussian"])
+    kept = np.zeros((1, 4, case.Ncap // 64), np.uint8)
+    kept[0, 0, [0, 3]] = 1                   # head 0: blocks 0 and 3 (64 + 8 rows)
+    kept[0, 1, [3]] = 1                      # head 1: block 3 again (union)
+    got = bench.algorithmic_bytes(case, kept)
+    assert got["index"] == 200 * 32
+    assert got["kept_kv"] == (64 + 8) * 512
+    assert got["local"] == (4 + 50) * 512     # sink 0..3 and window 150..199
+    assert got["total"] == got["index"] + got["kept_kv"] + got["local"]
+
+    # one KV group with both kinds: heads 0 (retrieval) and 1 (local)
+    hk = np.array([1, 0], np.uint8)
+    case = synth.make_case("bytes-mixed", B=1, Hkv=1, G=2, seq_lens=[200], ret_groups=[], head_kind=hk, p=[0.9],
+                           window=50, sink=4, seed=2, regimes=["gaussian"])
+    kept = np.zeros((1, 2, case.Ncap // 64), np.uint8)
+    kept[0, 0, [0, 2]] = 1                   # blocks 0 (rows 0..63) and 2 (rows 128..191)
+    got = bench.algorithmic_bytes(case, kept)
+    # local rows: sink 0..3 (in block 0: already read), window 150..191 (in block 2: read), 192..199 (new)
+    assert got["kept_kv"] == 128 * 512
+    assert got["local"] == 8 * 512

@@ -861,3 +861,16 @@ def test_topk_step_keeps_the_blocks_of_its_k_best():
         blocks = sorted({n // 64 for n in best})
         assert np.nonzero(r["kept_blocks"][0, h])[0].tolist() == blocks
         assert r["kstar"][0, h] == k
+
+
+def test_oracle_results_do_not_depend_on_the_thread_count():
+    """The oracle parallelises over (sequence, head) only: one thread and
+    many give the same bits (the benchmark times both)."""
+    case = synth.workload(5, scale=64)
+    a = oracle.decode_step(case, nthreads=1)
+    b = oracle.decode_step(case, nthreads=8)
+    for k in ("out", "kstar", "tau", "kept_blocks"):
+        assert np.array_equal(a[k], b[k], equal_nan=(k == "tau")), k
+    c = oracle.decode_step_topk(case, 100, nthreads=1)
+    d = oracle.decode_step_topk(case, 100, nthreads=8)
+    assert np.array_equal(c["out"], d["out"]) and np.array_equal(c["kept_blocks"], d["kept_blocks"])

@@ -189,6 +189,36 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def stage_inputs(tensors, host_arrays, device, pin=True):
+    """One device buffer for a step's per-step inputs, each at a 256-byte
+    aligned offset, and its host twin (pinned): views into the device buffer
+    take the place of `tensors` (same shapes and dtypes, same values), so a
+    step's inputs cross in one host-to-device copy.  host_arrays: the host
+    values of the same tensors (numpy, same element sizes).  Returns
+    (device buffer, host buffer, views)."""
+    import torch
+
+    offs, off = [], 0
+    for t in tensors:
+        off = (off + 255) // 256 * 256
+        offs.append(off)
+        off += t.numel() * t.element_size()
+    dbuf = torch.empty(off, dtype=torch.uint8, device=device)
+    hbuf = torch.zeros(off, dtype=torch.uint8)
+    if pin:
+        hbuf = hbuf.pin_memory()
+    views = []
+    for t, o, a in zip(tensors, offs, host_arrays):
+        n = t.numel() * t.element_size()
+        v = dbuf[o:o + n].view(t.dtype).view(t.shape)
+        v.copy_(t)
+        views.append(v)
+        raw = np.ascontiguousarray(a).view(np.uint8).reshape(-1)
+        assert raw.size == n, "host array and tensor sizes differ"
+        hbuf[o:o + n].copy_(torch.from_numpy(raw))
+    return dbuf, hbuf, views
+
+
 def max_over_ranks(values, world, device):
     """Each rank's timings -> the maximum over the ranks, on every rank (the
     replicas' device times; the whole job is as slow as its slowest rank)."""
@@ -362,6 +392,13 @@ def main():
         case.p[:] = 1.0
     dc = DeviceCase(case, device=dev, debug=True)
     dc.topk = max(0, args.topk)
+    # the per-step inputs (queries, lengths, p) share one device buffer, so the
+    # end-to-end leg moves them in one host-to-device copy; set before any
+    # step is captured, so the graphs take these addresses
+    dbuf, hbuf, views = stage_inputs(
+        [dc.q_pre, dc.q_rope, dc.seq_lens, dc.p],
+        [case.q_pre, case.q_rope, case.seq_lens.astype(np.int32), case.p.astype(np.float32)], dev)
+    dc.q_pre, dc.q_rope, dc.seq_lens, dc.p = views
     stream = torch.cuda.current_stream(dev)
 
     # one debug step: kept blocks for the algorithmic byte count
@@ -463,14 +500,9 @@ def main():
     timeline = {n: (statistics.median([x[n] for x in tl]) if tl[0][n] is not None else None)
                 for n in tl[0]}
 
-    # ---- end to end: host query/len/p -> device, step, output -> host ----
-    hq_pre = torch.from_numpy(case.q_pre.view(np.int16)).view(torch.bfloat16).pin_memory()
-    hq_rope = torch.from_numpy(case.q_rope.view(np.int16)).view(torch.bfloat16).pin_memory()
-    hlens = torch.from_numpy(case.seq_lens.astype(np.int32)).pin_memory()
-    hp = torch.from_numpy(case.p.astype(np.float32)).pin_memory()
+    # ---- end to end: host query/len/p -> device (one staged copy), step, output -> host ----
     hout = torch.empty(dc.out.shape, dtype=torch.bfloat16).pin_memory()
-    h_in = (hq_pre, hq_rope, hlens) if dc.topk > 0 else (hq_pre, hq_rope, hlens, hp)   # (top-k takes no p)
-    h2d = sum(t.numel() * t.element_size() for t in h_in)
+    h2d = hbuf.numel()
     d2h = hout.numel() * hout.element_size()
     e2e_ms = []
     for i in range(max(3, args.warmup) + args.steps):
@@ -478,11 +510,7 @@ def main():
         a = torch.cuda.Event(enable_timing=True)
         z = torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        dc.q_pre.copy_(hq_pre, non_blocking=True)
-        dc.q_rope.copy_(hq_rope, non_blocking=True)
-        dc.seq_lens.copy_(hlens, non_blocking=True)
-        if dc.topk == 0:
-            dc.p.copy_(hp, non_blocking=True)
+        dbuf.copy_(hbuf, non_blocking=True)
         graph.replay()
         hout.copy_(dc.out, non_blocking=True)
         z.record(stream)

@@ -44,11 +44,14 @@ def parse():
     ap.add_argument("--scale", type=int, default=1, help="divide the workload's context lengths (profiling runs)")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--dense", action="store_true", help="p = 1 for every sequence (dense comparator)")
+    ap.add_argument("--topk", type=int, default=0,
+                    help="static top-k selection with this k (the fixed-budget variant) instead of top-p")
     ap.add_argument("--dense-comparator", action="store_true",
                     help="also time the same captured step with p = 1 and add it to the line as dense_comparator")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--op", choices=["decode", "append"], default="decode",
-                    help="append: time the index-cache append instead of the decode step")
+    ap.add_argument("--op", choices=["decode", "append", "kv_append"], default="decode",
+                    help="append: time the index-cache append instead of the decode step; "
+                         "kv_append: the KV-cache write with the index append")
     return ap.parse_args()
 
 
@@ -186,6 +189,36 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def stage_inputs(tensors, host_arrays, device, pin=True):
+    """One device buffer for a step's per-step inputs, each at a 256-byte
+    aligned offset, and its host twin (pinned): views into the device buffer
+    take the place of `tensors` (same shapes and dtypes, same values), so a
+    step's inputs cross in one host-to-device copy.  host_arrays: the host
+    values of the same tensors (numpy, same element sizes).  Returns
+    (device buffer, host buffer, views)."""
+    import torch
+
+    offs, off = [], 0
+    for t in tensors:
+        off = (off + 255) // 256 * 256
+        offs.append(off)
+        off += t.numel() * t.element_size()
+    dbuf = torch.empty(off, dtype=torch.uint8, device=device)
+    hbuf = torch.zeros(off, dtype=torch.uint8)
+    if pin:
+        hbuf = hbuf.pin_memory()
+    views = []
+    for t, o, a in zip(tensors, offs, host_arrays):
+        n = t.numel() * t.element_size()
+        v = dbuf[o:o + n].view(t.dtype).view(t.shape)
+        v.copy_(t)
+        views.append(v)
+        raw = np.ascontiguousarray(a).view(np.uint8).reshape(-1)
+        assert raw.size == n, "host array and tensor sizes differ"
+        hbuf[o:o + n].copy_(torch.from_numpy(raw))
+    return dbuf, hbuf, views
+
+
 def max_over_ranks(values, world, device):
     """Each rank's timings -> the maximum over the ranks, on every rank (the
     replicas' device times; the whole job is as slow as its slowest rank)."""
@@ -197,6 +230,10 @@ def max_over_ranks(values, world, device):
 
         dist.all_reduce(vals, op=dist.ReduceOp.MAX)
     return [float(v) for v in vals]
+
+
+def selection_name(args):
+    return f"static top-k, k={args.topk}" if args.topk > 0 else ("top-p, p=1 (dense)" if args.dense else "top-p")
 
 
 def cpu_model():
@@ -211,14 +248,17 @@ def cpu_model():
     return None
 
 
-def oracle_single_thread(case, tokens, budget_s=5.0):
+def oracle_single_thread(case, tokens, topk=0, budget_s=5.0):
     """The oracle on one host thread: whole steps until about budget_s have
     passed (at least one).  Returns a dict for the cpu_baseline entry."""
     import oracle
 
     reps, t0 = 0, time.perf_counter()
     while reps == 0 or (time.perf_counter() - t0 < budget_s and reps < 20):
-        oracle.decode_step(case, nthreads=1)
+        if topk > 0:
+            oracle.decode_step_topk(case, topk, nthreads=1)
+        else:
+            oracle.decode_step(case, nthreads=1)
         reps += 1
     t = (time.perf_counter() - t0) / reps
     return {"value": tokens / t, "s_per_step": t, "sample": f"{reps} whole decode steps, 1 thread"}
@@ -235,21 +275,28 @@ def run_reference(args, rank):
     if args.dense:
         case.p[:] = 1.0
     cores = os.cpu_count() or 1
+
+    def step():
+        if args.topk > 0:
+            oracle.decode_step_topk(case, args.topk, nthreads=cores)
+        else:
+            oracle.decode_step(case, nthreads=cores)
+
     for _ in range(args.warmup):
-        oracle.decode_step(case, nthreads=cores)
+        step()
     ts = []
     for _ in range(args.steps):
         t0 = time.perf_counter()
-        oracle.decode_step(case, nthreads=cores)
+        step()
         ts.append(time.perf_counter() - t0)
     t = statistics.mean(ts)
     tokens = float(case.seq_lens.sum())
     v = tokens / t
-    single = oracle_single_thread(case, tokens)
+    single = oracle_single_thread(case, tokens, args.topk)
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": workload_config(case, args.workload),
+            "config": dict(workload_config(case, args.workload), selection=selection_name(args)),
             "cpu_baseline": {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "cpu_model": cpu_model(),
                              "sample": f"whole decode step of the workload per timed step ({args.steps} steps)",
                              "single_thread": single},
@@ -258,10 +305,14 @@ def run_reference(args, rank):
 
 
 def bench_append(args):
-    """rtp_index_append alone: a decode-sized append (one new token for each
-    of 16 sequences x 8 KV heads) and a 32K-token chunk of one sequence; HBM
-    bytes = k_pre read (256 B) + k_idx written (32 B) per token and KV head
-    (W^K, 32 KB, stays in L2).  L2 flushed before every timed call."""
+    """rtp_index_append alone (--op append) or rtp_kv_append (--op kv_append):
+    a decode-sized append (one new token for each of 16 sequences x 8 KV
+    heads) and a 32K-token chunk of one sequence.  HBM bytes per token and KV
+    head: k_pre read (256 B) + k_idx written (32 B); kv_append adds the new
+    value read (256 B) and the key and value rows written (512 B), and the
+    angle table row (512 B) once per position.  W^K (32 KB) stays in L2.  L2
+    flushed before every timed call."""
+    kv = args.op == "kv_append"
     import torch
 
     import sparse_attention_decode_rtpurbo_b200 as rtp
@@ -276,6 +327,12 @@ def bench_append(args):
         Wk = (torch.randn((Hkv, 16, 128), generator=g, device=dev) / 11.3).to(torch.bfloat16)
         pos = torch.zeros(B, dtype=torch.int32, device=dev)
         cache = torch.zeros((B, Hkv, ncap, 16), dtype=torch.bfloat16, device=dev)
+        if kv:
+            v_new = torch.randn((B, Hkv, T, 128), generator=g, device=dev).to(torch.bfloat16)
+            ang = torch.rand((ncap, 64), generator=g, device=dev, dtype=torch.float64) * 6.283
+            rc, rs = torch.cos(ang).float(), torch.sin(ang).float()
+            kc = torch.zeros((B, Hkv, ncap, 128), dtype=torch.bfloat16, device=dev)
+            vc = torch.zeros((B, Hkv, ncap, 128), dtype=torch.bfloat16, device=dev)
         dims = rtp.make_dims(B, Hkv, Hkv, ncap)
         stream = torch.cuda.current_stream()
         ts = []
@@ -283,15 +340,19 @@ def bench_append(args):
             flush_w.zero_()
             a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(stream)
-            rtp.index_append(dims, k_pre, Wk, pos, T, cache, None, stream)
+            if kv:
+                rtp.kv_append(dims, k_pre, v_new, Wk, rc, rs, pos, T, cache, kc, vc, None, stream)
+            else:
+                rtp.index_append(dims, k_pre, Wk, pos, T, cache, None, stream)
             z.record(stream)
             z.synchronize()
             if i >= args.warmup:
                 ts.append(a.elapsed_time(z))
         t_ms = statistics.median(ts)
-        nbytes = B * Hkv * T * (256 + 32)
+        nbytes = B * Hkv * T * (256 + 32 + (256 + 512 if kv else 0)) + (T * 512 if kv else 0)
         gbs = nbytes / (t_ms * 1e-3) / 1e9
-        print(json.dumps({"metric": "index-cache append (rtp_index_append)", "op": "append", "case": name,
+        metric = "KV-cache write + index append (rtp_kv_append)" if kv else "index-cache append (rtp_index_append)"
+        print(json.dumps({"metric": metric, "op": args.op, "case": name,
                           "value": gbs, "unit": "GB/s", "us_per_call": t_ms * 1e3, "bytes": nbytes,
                           "peak": peak, "frac": gbs / peak, "peak_source": peak_kind, "steps": args.steps,
                           "warmup": args.warmup, "l2": "flushed (256 MB write) before every call"}), flush=True)
@@ -299,7 +360,7 @@ def bench_append(args):
 
 def main():
     args = parse()
-    if args.op == "append":
+    if args.op in ("append", "kv_append"):
         return bench_append(args)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -330,6 +391,14 @@ def main():
     if args.dense:
         case.p[:] = 1.0
     dc = DeviceCase(case, device=dev, debug=True)
+    dc.topk = max(0, args.topk)
+    # the per-step inputs (queries, lengths, p) share one device buffer, so the
+    # end-to-end leg moves them in one host-to-device copy; set before any
+    # step is captured, so the graphs take these addresses
+    dbuf, hbuf, views = stage_inputs(
+        [dc.q_pre, dc.q_rope, dc.seq_lens, dc.p],
+        [case.q_pre, case.q_rope, case.seq_lens.astype(np.int32), case.p.astype(np.float32)], dev)
+    dc.q_pre, dc.q_rope, dc.seq_lens, dc.p = views
     stream = torch.cuda.current_stream(dev)
 
     # one debug step: kept blocks for the algorithmic byte count
@@ -431,13 +500,9 @@ def main():
     timeline = {n: (statistics.median([x[n] for x in tl]) if tl[0][n] is not None else None)
                 for n in tl[0]}
 
-    # ---- end to end: host query/len/p -> device, step, output -> host ----
-    hq_pre = torch.from_numpy(case.q_pre.view(np.int16)).view(torch.bfloat16).pin_memory()
-    hq_rope = torch.from_numpy(case.q_rope.view(np.int16)).view(torch.bfloat16).pin_memory()
-    hlens = torch.from_numpy(case.seq_lens.astype(np.int32)).pin_memory()
-    hp = torch.from_numpy(case.p.astype(np.float32)).pin_memory()
+    # ---- end to end: host query/len/p -> device (one staged copy), step, output -> host ----
     hout = torch.empty(dc.out.shape, dtype=torch.bfloat16).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in (hq_pre, hq_rope, hlens, hp))
+    h2d = hbuf.numel()
     d2h = hout.numel() * hout.element_size()
     e2e_ms = []
     for i in range(max(3, args.warmup) + args.steps):
@@ -445,10 +510,7 @@ def main():
         a = torch.cuda.Event(enable_timing=True)
         z = torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        dc.q_pre.copy_(hq_pre, non_blocking=True)
-        dc.q_rope.copy_(hq_rope, non_blocking=True)
-        dc.seq_lens.copy_(hlens, non_blocking=True)
-        dc.p.copy_(hp, non_blocking=True)
+        dbuf.copy_(hbuf, non_blocking=True)
         graph.replay()
         hout.copy_(dc.out, non_blocking=True)
         z.record(stream)
@@ -463,7 +525,7 @@ def main():
     # sequence (every block of every retrieval head), the stand-in for the
     # pages' dense-attention baseline; the graph reads p from dc.p ----
     dense_ms, dense_status = 0.0, 0
-    if args.dense_comparator and not args.dense and case.head_kind.any():
+    if args.dense_comparator and not args.dense and args.topk == 0 and case.head_kind.any():
         dc.p.fill_(1.0)
         dts = []
         for i in range(max(3, args.warmup) + args.steps):
@@ -507,15 +569,21 @@ def main():
             import oracle
 
             cores = os.cpu_count() or 1
-            oracle.decode_step(case, nthreads=cores)
+            def oracle_step():
+                if args.topk > 0:
+                    oracle.decode_step_topk(case, args.topk, nthreads=cores)
+                else:
+                    oracle.decode_step(case, nthreads=cores)
+
+            oracle_step()
             reps, t0 = 0, time.perf_counter()
             while time.perf_counter() - t0 < 10.0 and reps < 50:
-                oracle.decode_step(case, nthreads=cores)
+                oracle_step()
                 reps += 1
             tc = (time.perf_counter() - t0) / reps
             cpu = {"value": tokens / tc, "unit": UNIT, "cores": cores, "kind": "oracle", "cpu_model": cpu_model(),
                    "sample": f"{reps} whole decode steps of this workload (fp64 C oracle, OpenMP over heads)",
-                   "single_thread": oracle_single_thread(case, tokens)}
+                   "single_thread": oracle_single_thread(case, tokens, args.topk)}
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": t_ms, "us_per_step": t_ms * 1e3,
@@ -523,12 +591,13 @@ def main():
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16 in, fp32 accumulate",
             "data": "synthetic (seeded generators in synth/, shaped like the pages' workloads)",
             "config": dict(workload_config(case, args.workload), parallelism=f"replicas x{world}",
-                           dense_p1=bool(args.dense), timing="CUDA-graph replay of one rtp_decode_step (2 kernels, programmatic launch) per step; "
+                           dense_p1=bool(args.dense), selection=selection_name(args), timing="CUDA-graph replay of one rtp_decode_step (2 kernels, programmatic launch) per step; "
                            "CUDA events on the launching stream"),
             "wall_s_timed_loop": wall,
             "roofline": {"bound": "hbm", "kernel": f"rtp::{dom}_kernel", "achieved": ach, "peak": peak, "unit": "GB/s",
                          "frac": ach / peak, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, burst)",
-                         "traffic": profiled_traffic(dom, case.name), "algorithmic_bytes_per_launch": kbytes[dom],
+                         "traffic": profiled_traffic(dom, case.name) if selection_name(args) == "top-p" else None,
+                         "algorithmic_bytes_per_launch": kbytes[dom],
                          "us_per_launch": phase_ms[dom] * 1e3},
             "step_roofline": {"algorithmic_bytes": nbytes, "achieved": step_gbs, "peak": peak, "unit": "GB/s",
                               "frac": step_gbs / peak},

@@ -159,6 +159,83 @@ rtp_status rtp_decode_step(const rtp_dims* dims, const uint16_t* q_pre, const ui
                            const float* p, int32_t window, int32_t sink, uint16_t* out, void* stream);
 
 /*
+ * rtp_decode_step_ring -- the decode step for a model whose local KV heads
+ * keep only their sink and sliding window (review, Method: "Adaptive sparse
+ * attention": local heads attend to a sink and a window, so they need no
+ * long-context cache; Insight 1: most heads are local).  Local heads of KV
+ * heads that serve no retrieval head read their keys and values from rings
+ * instead of k_cache / v_cache; every other read is rtp_decode_step's.
+ *
+ * Ring layout, per sequence b and KV head g (rows of 128 bf16):
+ *   rows 0 .. 63      : positions 0 .. 63 (the sink, 64 >= sink);
+ *   rows 64 .. 63 + W : position n >= 64 in row 64 + (n mod W).
+ * Writing positions in order, each new one overwrites the one W places
+ * before it, so after L tokens the ring holds [0, min(64, L)) and
+ * [max(64, L - W), L); W (ring_W) must be a multiple of 64 and >= window.
+ *
+ * Arguments are those of rtp_decode_step, plus
+ *   k_ring, v_ring : device bf16 [batch, num_kv_heads, 64 + ring_W, 128],
+ *     16-byte aligned (rows of KV heads with retrieval heads are not read).
+ *   ring_W : the window region's rows, a multiple of 64, >= window.
+ * Rows of k_cache / v_cache for KV heads without retrieval heads are not read.
+ * Returns RTP_ERR_NULL for a NULL ring, RTP_ERR_SHAPE for ring_W not a
+ * multiple of 64 or below window (or below 64) or sink > 64; otherwise as
+ * rtp_decode_step (same workspace size).
+ */
+rtp_status rtp_decode_step_ring(const rtp_dims* dims, const uint16_t* q_pre, const uint16_t* q_rope,
+                                const uint16_t* k_idx, const uint16_t* k_cache, const uint16_t* v_cache,
+                                const uint16_t* k_ring, const uint16_t* v_ring, int32_t ring_W,
+                                const uint16_t* Wq_idx, const int32_t* seq_lens, const uint8_t* head_kind,
+                                const float* p, int32_t window, int32_t sink, uint16_t* out, void* stream);
+
+/*
+ * rtp_ring_write -- write the key and value rows of new tokens of the local-
+ * only KV heads into their rings (the layout of rtp_decode_step_ring: rows
+ * 0 .. 63 hold positions 0 .. 63, position n >= 64 goes to row 64 + n mod W).
+ * The result is that of writing the tokens t = 0 .. num_new-1 of each
+ * sequence in order: a token whose row a later token of the same call also
+ * takes is not written.
+ *   dims     : batch, num_kv_heads, head_dim 128, block_size 64 (other fields
+ *              unused).
+ *   k_new, v_new : device bf16 [batch, num_kv_heads, num_new, 128] (RoPE'd
+ *              keys, values), 16-byte aligned.
+ *   pos      : device int32 [batch], position of each sequence's first new token.
+ *   ring_W   : the rings' window rows, a multiple of 64.
+ *   k_ring, v_ring : device bf16 [batch, num_kv_heads, 64 + ring_W, 128],
+ *              16-byte aligned; owned by the caller.
+ *   device_status : optional device uint32, set to RTP_ERR_DEVICE_INPUT for a
+ *              negative position (that sequence is skipped).
+ * Returns RTP_ERR_NULL / RTP_ERR_SHAPE / RTP_ERR_UNSUPPORTED before anything
+ * is enqueued, RTP_ERR_CUDA if the launch failed, else RTP_OK (num_new = 0:
+ * nothing is enqueued).
+ */
+rtp_status rtp_ring_write(const rtp_dims* dims, const uint16_t* k_new, const uint16_t* v_new, const int32_t* pos,
+                          int32_t num_new, int32_t ring_W, uint16_t* k_ring, uint16_t* v_ring,
+                          uint32_t* device_status, void* stream);
+
+/*
+ * rtp_decode_step_topk -- the decode step with the static top-k selection in
+ * place of dynamic top-p: every retrieval head keeps its min(topk, L) best
+ * tokens under the order (score descending, token index ascending), widened
+ * to 64-token blocks, and attends over them exactly as rtp_decode_step does.
+ * Local heads are unchanged.  This is the fixed-budget variant that the
+ * paper's experiments compare against (review on dongryeollee1.github.io,
+ * Experiments: the static top-k baseline at k = 4096; Method, "Insight 3":
+ * a fixed budget against a query-dependent one).
+ *
+ * Arguments are those of rtp_decode_step, with p replaced by
+ *   topk: tokens kept per retrieval head, >= 1 (the same for every sequence
+ *     and head); topk >= L keeps every block of that sequence, topk = 1 keeps
+ *     the block of the best-scoring token (lowest index among equal maxima).
+ * Returns RTP_ERR_SHAPE for topk < 1; every other check, the workspace and
+ * the error behaviour are those of rtp_decode_step (same workspace size).
+ */
+rtp_status rtp_decode_step_topk(const rtp_dims* dims, const uint16_t* q_pre, const uint16_t* q_rope,
+                                const uint16_t* k_idx, const uint16_t* k_cache, const uint16_t* v_cache,
+                                const uint16_t* Wq_idx, const int32_t* seq_lens, const uint8_t* head_kind,
+                                int32_t topk, int32_t window, int32_t sink, uint16_t* out, void* stream);
+
+/*
  * Synchronises `stream`, returns the first device-side error recorded in the
  * workspace since the last call to this function (RTP_OK if none) and clears
  * it.  For tests and debugging; it blocks the host.
@@ -247,6 +324,46 @@ rtp_status rtp_decode_step_noalloc(const rtp_dims* dims, const uint16_t* q_pre, 
  */
 rtp_status rtp_index_append(const rtp_dims* dims, const uint16_t* k_pre, const uint16_t* Wk_idx, const int32_t* pos,
                             int32_t num_new, uint16_t* k_idx, uint32_t* device_status, void* stream);
+
+/*
+ * rtp_kv_append -- the KV-cache write of new tokens with the index-cache
+ * append in the same kernel: the key and value rows that rtp_decode_step's
+ * attention reads and the index rows its scoring reads, from one read of the
+ * new pre-RoPE keys.
+ *
+ * Source: review, Method: "Adaptive sparse attention" (the indexer projects
+ * pre-RoPE keys, the attention uses RoPE'd keys) and Insight 2 (RoPE rotates
+ * each frequency pair by an angle proportional to the position).
+ *
+ * For every sequence b, KV head g and new token t, at cache row n = pos[b] + t:
+ *     k_idx row (b, g, n)   = as rtp_index_append
+ *     k_cache row (b, g, n) = bf16( RoPE_n(k_pre[b, g, t]) )
+ *     v_cache row (b, g, n) = v_new[b, g, t]   (bits copied)
+ * RoPE_n rotates the pairs (i, i + 64), i < 64 (rotate-half pairing), by the
+ * caller's angle table row n:
+ *     y_i = k_i cos[n][i] - k_{i+64} sin[n][i],  y_{i+64} = k_{i+64} cos[n][i] + k_i sin[n][i]
+ * each computed as one fp64 fused multiply-add onto the other (exact)
+ * product, then rounded to bf16 (round to nearest even).  The table carries
+ * the model's own RoPE (base, scaling); the kernels never compute angles.
+ *
+ *   dims, k_pre, Wk_idx, pos, num_new, k_idx, device_status, stream: as
+ *              rtp_index_append.
+ *   v_new    : device bf16 [batch, num_kv_heads, num_new, 128], 16-byte aligned.
+ *   rope_cos, rope_sin : device fp32 [max_seq_len, 64], 16-byte aligned; row n
+ *              holds cos and sin of the angles of cache position n.
+ *   k_cache, v_cache : device bf16 caches in rtp_decode_step's layout
+ *              (contiguous [batch, num_kv_heads, max_seq_len, 128] or paged
+ *              [num_pages, num_kv_heads, 64, 128]), 16-byte aligned; only the
+ *              rows above are written.  Owned by the caller.
+ * A row or page id out of range is skipped in all three caches (and reported
+ * through device_status).  Returns the codes of rtp_index_append; also
+ * RTP_ERR_NULL for a NULL k_cache, v_cache, v_new or table, and
+ * RTP_ERR_UNSUPPORTED for one that is not 16-byte aligned.
+ */
+rtp_status rtp_kv_append(const rtp_dims* dims, const uint16_t* k_pre, const uint16_t* v_new, const uint16_t* Wk_idx,
+                         const float* rope_cos, const float* rope_sin, const int32_t* pos, int32_t num_new,
+                         uint16_t* k_idx, uint16_t* k_cache, uint16_t* v_cache, uint32_t* device_status,
+                         void* stream);
 
 /* Static string naming a status code. */
 const char* rtp_status_string(rtp_status status);

@@ -71,12 +71,21 @@ def _load():
     L.rtp_workspace_size.restype = ctypes.c_size_t
     L.rtp_decode_step.argtypes = [ctypes.POINTER(RtpDims), vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, vp, vp]
     L.rtp_decode_step.restype = ctypes.c_int
+    L.rtp_decode_step_topk.argtypes = [ctypes.POINTER(RtpDims), vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, vp, vp]
+    L.rtp_decode_step_topk.restype = ctypes.c_int
+    L.rtp_decode_step_ring.argtypes = [ctypes.POINTER(RtpDims), vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, i32,
+                                       i32, vp, vp]
+    L.rtp_decode_step_ring.restype = ctypes.c_int
+    L.rtp_ring_write.argtypes = [ctypes.POINTER(RtpDims), vp, vp, vp, i32, i32, vp, vp, vp, vp]
+    L.rtp_ring_write.restype = ctypes.c_int
     L.rtp_decode_step_noalloc.argtypes = [ctypes.POINTER(RtpDims), vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, vp,
                                           vp, vp]
     L.rtp_decode_step_noalloc.restype = ctypes.c_int
     L.rtp_get_status.argtypes = [ctypes.POINTER(RtpDims), vp]
     L.rtp_index_append.argtypes = [ctypes.POINTER(RtpDims), vp, vp, vp, i32, vp, vp, vp]
     L.rtp_index_append.restype = ctypes.c_int
+    L.rtp_kv_append.argtypes = [ctypes.POINTER(RtpDims), vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp]
+    L.rtp_kv_append.restype = ctypes.c_int
     L.rtp_get_status.restype = ctypes.c_int
     L.rtp_status_string.argtypes = [ctypes.c_int]
     L.rtp_status_string.restype = ctypes.c_char_p
@@ -137,6 +146,42 @@ def decode_step(dims: RtpDims, q_pre, q_rope, k_idx, k_cache, v_cache, Wq_idx, s
         raise RtpError(rc, "rtp_decode_step")
 
 
+def decode_step_ring(dims: RtpDims, q_pre, q_rope, k_idx, k_cache, v_cache, k_ring, v_ring, ring_W: int, Wq_idx,
+                     seq_lens, head_kind, p, window: int, sink: int, out, stream=None) -> None:
+    """rtp_decode_step_ring: the decode step with the local-only KV heads'
+    keys and values read from rings [B, Hkv, 64 + ring_W, 128] (block 0 in
+    rows 0..63, position n >= 64 in row 64 + n % ring_W)."""
+    st = 0 if stream is None else (stream if isinstance(stream, int) else stream.cuda_stream)
+    rc = lib.rtp_decode_step_ring(ctypes.byref(dims), _ptr(q_pre), _ptr(q_rope), _ptr(k_idx), _ptr(k_cache),
+                                  _ptr(v_cache), _ptr(k_ring), _ptr(v_ring), int(ring_W), _ptr(Wq_idx), _ptr(seq_lens),
+                                  _head_kind_buf(head_kind), _ptr(p), int(window), int(sink), _ptr(out), st)
+    if rc != RTP_OK:
+        raise RtpError(rc, "rtp_decode_step_ring")
+
+
+def ring_write(dims: RtpDims, k_new, v_new, pos, num_new: int, ring_W: int, k_ring, v_ring, device_status=None,
+               stream=None) -> None:
+    """rtp_ring_write: the new key and value rows of every sequence into the
+    local heads' rings [B, Hkv, 64 + ring_W, 128], as if written in order."""
+    st = 0 if stream is None else (stream if isinstance(stream, int) else stream.cuda_stream)
+    rc = lib.rtp_ring_write(ctypes.byref(dims), _ptr(k_new), _ptr(v_new), _ptr(pos), int(num_new), int(ring_W),
+                            _ptr(k_ring), _ptr(v_ring), _ptr(device_status), st)
+    if rc != RTP_OK:
+        raise RtpError(rc, "rtp_ring_write")
+
+
+def decode_step_topk(dims: RtpDims, q_pre, q_rope, k_idx, k_cache, v_cache, Wq_idx, seq_lens, head_kind, topk: int,
+                     window: int, sink: int, out, stream=None) -> None:
+    """rtp_decode_step_topk: the decode step with every retrieval head keeping
+    its static top-k tokens (topk >= 1) instead of the dynamic top-p set."""
+    st = 0 if stream is None else (stream if isinstance(stream, int) else stream.cuda_stream)
+    rc = lib.rtp_decode_step_topk(ctypes.byref(dims), _ptr(q_pre), _ptr(q_rope), _ptr(k_idx), _ptr(k_cache),
+                                  _ptr(v_cache), _ptr(Wq_idx), _ptr(seq_lens), _head_kind_buf(head_kind), int(topk),
+                                  int(window), int(sink), _ptr(out), st)
+    if rc != RTP_OK:
+        raise RtpError(rc, "rtp_decode_step_topk")
+
+
 # RTP_NOALLOC_SCRATCH_BYTES of the C header: the static scratch of rtp_decode_step_noalloc
 NOALLOC_SCRATCH_BYTES = 64 << 20
 
@@ -169,6 +214,19 @@ def index_append(dims: RtpDims, k_pre, Wk_idx, pos, num_new: int, k_idx, device_
         raise RtpError(rc, "rtp_index_append")
 
 
+def kv_append(dims: RtpDims, k_pre, v_new, Wk_idx, rope_cos, rope_sin, pos, num_new: int, k_idx, k_cache, v_cache,
+              device_status=None, stream=None) -> None:
+    """rtp_kv_append: for the num_new new tokens of every sequence, cache rows
+    n = pos[b] + t receive k_idx = bf16(W^K[g] . k_pre), k_cache =
+    bf16(RoPE_n(k_pre)) with the angle table rows rope_cos[n], rope_sin[n]
+    (fp32 [max_seq_len, 64]), and v_cache = v_new."""
+    st = 0 if stream is None else (stream if isinstance(stream, int) else stream.cuda_stream)
+    rc = lib.rtp_kv_append(ctypes.byref(dims), _ptr(k_pre), _ptr(v_new), _ptr(Wk_idx), _ptr(rope_cos), _ptr(rope_sin),
+                           _ptr(pos), int(num_new), _ptr(k_idx), _ptr(k_cache), _ptr(v_cache), _ptr(device_status), st)
+    if rc != RTP_OK:
+        raise RtpError(rc, "rtp_kv_append")
+
+
 def get_status(dims: RtpDims, stream=None) -> int:
     st = 0 if stream is None else (stream if isinstance(stream, int) else stream.cuda_stream)
     return int(lib.rtp_get_status(ctypes.byref(dims), st))
@@ -199,6 +257,15 @@ class Step:
     def __call__(self, q_pre, q_rope, k_idx, k_cache, v_cache, Wq_idx, seq_lens, p, window, sink, out, stream=None):
         decode_step(self.dims, q_pre, q_rope, k_idx, k_cache, v_cache, Wq_idx, seq_lens, self.head_kind, p, window,
                     sink, out, stream)
+
+    def ring(self, q_pre, q_rope, k_idx, k_cache, v_cache, k_ring, v_ring, ring_W, Wq_idx, seq_lens, p, window, sink,
+             out, stream=None):
+        decode_step_ring(self.dims, q_pre, q_rope, k_idx, k_cache, v_cache, k_ring, v_ring, ring_W, Wq_idx, seq_lens,
+                         self.head_kind, p, window, sink, out, stream)
+
+    def topk(self, q_pre, q_rope, k_idx, k_cache, v_cache, Wq_idx, seq_lens, topk, window, sink, out, stream=None):
+        decode_step_topk(self.dims, q_pre, q_rope, k_idx, k_cache, v_cache, Wq_idx, seq_lens, self.head_kind, topk,
+                         window, sink, out, stream)
 
     def status(self, stream=None) -> int:
         return get_status(self.dims, stream)

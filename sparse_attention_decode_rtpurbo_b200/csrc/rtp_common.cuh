@@ -87,7 +87,14 @@ struct Params {
     const uint16_t *q_pre, *q_rope, *k_idx, *Wq;
     const uint16_t *k_cache_ptr, *v_cache_ptr;   // the caches as plain pointers (the kernels read them through TMA maps)
     const int32_t *seq_lens, *block_table;
-    const float* p;
+    const float* p;   // top-p mass per sequence (unused, may be null, under static top-k)
+    int topk;         // 0: dynamic top-p; k >= 1: every retrieval head keeps its k best tokens
+    // local heads' ring cache: local groups i with bit i of ring_lg_mask read
+    // their sink and window from rings of ring_rows = 64 + ring_W rows per
+    // (sequence, KV head): block 0 in rows 0..63, block j >= 1 in the 64 rows
+    // from 64 + (64 j mod ring_W)
+    unsigned long long ring_lg_mask;
+    int ring_W, ring_rows;
     uint16_t* out;
     HeadTab tab;
     // workspace
@@ -122,6 +129,7 @@ struct Params {
 // rows x 128 bf16, 64 x 64 boxes, 128-byte swizzle) travel as grid constants.
 struct KParams {
     CUtensorMap tmk, tmv;
+    CUtensorMap tmk_r, tmv_r;   // the local heads' rings (encoded only when they are given)
     Params P;
 };
 
@@ -175,6 +183,12 @@ __device__ __forceinline__ int page_or_zero(const Params& P, int b, int j) {
     if (pg >= 0 && pg < P.num_pages) return pg;
     set_status(P, ST_DEVICE_INPUT);
     return 0;
+}
+
+// First ring row (of the `rows x 128` ring views) of block j of KV head g of sequence b.
+__device__ __forceinline__ int64_t ring_block_row(const Params& P, int b, int g, int j) {
+    const int slot = j == 0 ? 0 : BLK + (int)(((int64_t)j * BLK) % P.ring_W);
+    return ((int64_t)b * P.Hkv + g) * P.ring_rows + slot;
 }
 
 // First cache row (of `rows x dim` views) of block j of KV head g of sequence b.

@@ -237,11 +237,32 @@ static int grid_cap() {
     return n >= 1 ? n : MAX_GRID;
 }
 
+// RTP_SINGLE_LAUNCH=1 in the environment (read at every call): the step
+// runs as one launch (step_kernel: streaming phase, grid barrier, retrieval
+// phase) instead of two.  Results do not depend on it.
+static bool single_launch() {
+    const char* v = getenv("RTP_SINGLE_LAUNCH");
+    return v && atoi(v) == 1;
+}
+
 template <int G>
 static cudaError_t launch(const KParams& K, const Plan& pl, cudaStream_t s, void* const* ev, unsigned ev_flags) {
     const int sms = num_sms();
     if (!sms) return report(cudaErrorUnknown, "SM count");
     const int cap = std::min(MAX_GRID, grid_cap());
+    if (pl.n_rg > 0 && single_launch()) {
+        // one resident wave with room for either phase's shared memory (the
+        // retrieval phase's grid barriers need every CTA resident; surplus
+        // CTAs take no share of the streaming phase)
+        const size_t smem = std::max(asmem_bytes<G>(pl.B), bsmem_bytes<G>(pl.B * pl.n_rg));
+        const int occ = occupancy((const void*)step_kernel<G>, smem);
+        if (occ < 1) return report(cudaErrorInvalidConfiguration, "step kernel occupancy");
+        const int grid = std::min(cap, occ * sms);
+        step_kernel<G><<<(unsigned)grid, THREADS, smem, s>>>(K);
+        cudaError_t e = report(cudaGetLastError(), "step kernel launch");
+        if (ev) cudaEventRecordWithFlags((cudaEvent_t)ev[1], s, ev_flags);   // (no phase boundary to mark)
+        return e;
+    }
     // streaming kernel: as many resident CTAs as the tiles can use
     {
         const size_t smem = asmem_bytes<G>(pl.B);
@@ -291,16 +312,23 @@ extern "C" size_t rtp_workspace_size(const rtp_dims* dims, const uint8_t* head_k
 
 static bool aligned16(const void* p) { return ((uintptr_t)p & 15) == 0; }
 
-extern "C" rtp_status rtp_decode_step(const rtp_dims* dims, const uint16_t* q_pre, const uint16_t* q_rope,
-                                      const uint16_t* k_idx, const uint16_t* k_cache, const uint16_t* v_cache,
-                                      const uint16_t* Wq_idx, const int32_t* seq_lens, const uint8_t* head_kind,
-                                      const float* p, int32_t window, int32_t sink, uint16_t* out, void* stream) {
-    if (!dims || !q_pre || !q_rope || !k_idx || !k_cache || !v_cache || !Wq_idx || !seq_lens || !head_kind || !p ||
-        !out)
+// The decode step with a caller workspace: dynamic top-p (p, topk = 0) or
+// static top-k (topk >= 1, p unused).
+// (and, with k_ring, the local heads' rings of 64 + ring_W rows).
+static rtp_status decode_step_ws(const rtp_dims* dims, const uint16_t* q_pre, const uint16_t* q_rope,
+                                 const uint16_t* k_idx, const uint16_t* k_cache, const uint16_t* v_cache,
+                                 const uint16_t* k_ring, const uint16_t* v_ring, int32_t ring_W,
+                                 const uint16_t* Wq_idx, const int32_t* seq_lens, const uint8_t* head_kind,
+                                 const float* p, int32_t topk, int32_t window, int32_t sink, uint16_t* out,
+                                 void* stream) {
+    if (!dims || !q_pre || !q_rope || !k_idx || !k_cache || !v_cache || !Wq_idx || !seq_lens || !head_kind ||
+        (topk == 0 && !p) || !out || (k_ring && !v_ring))
         return RTP_ERR_NULL;
+    if (topk < 0) return RTP_ERR_SHAPE;
     if (window < 0 || sink < 0 || (int64_t)window + sink < 1) return RTP_ERR_SHAPE;
+    if (k_ring && (ring_W < BLK || ring_W % BLK || ring_W < window || sink > BLK)) return RTP_ERR_SHAPE;
     if (!aligned16(q_pre) || !aligned16(q_rope) || !aligned16(k_idx) || !aligned16(k_cache) || !aligned16(v_cache) ||
-        !aligned16(Wq_idx) || !aligned16(out))
+        !aligned16(Wq_idx) || !aligned16(out) || (k_ring && (!aligned16(k_ring) || !aligned16(v_ring))))
         return RTP_ERR_UNSUPPORTED;
     Plan pl;
     rtp_status st = make_plan(dims, head_kind, window, sink, &pl);
@@ -316,7 +344,24 @@ extern "C" rtp_status rtp_decode_step(const rtp_dims* dims, const uint16_t* q_pr
         report(cudaErrorInvalidValue, "K/V tensor map");
         return RTP_ERR_CUDA;
     }
+    unsigned long long ring_mask = 0;
+    if (k_ring) {
+        // the rings serve the local groups whose KV head has no retrieval head
+        for (int i = 0; i < pl.n_lg; ++i) {
+            bool pure = true;
+            for (int r = 0; r < pl.n_rg; ++r) pure = pure && pl.rg_group[r] != pl.lg_group[i];
+            if (pure) ring_mask |= 1ull << i;
+        }
+        const long long ring_rows = (long long)pl.B * pl.Hkv * (BLK + ring_W);
+        if (!encode_cache_map(&K.tmk_r, k_ring, ring_rows) || !encode_cache_map(&K.tmv_r, v_ring, ring_rows)) {
+            report(cudaErrorInvalidValue, "ring tensor map");
+            return RTP_ERR_CUDA;
+        }
+    }
     Params& P = K.P;
+    P.ring_lg_mask = ring_mask;
+    P.ring_W = k_ring ? ring_W : 0;
+    P.ring_rows = k_ring ? BLK + ring_W : 0;
     P.B = pl.B;
     P.Hq = pl.Hq;
     P.Hkv = pl.Hkv;
@@ -341,7 +386,8 @@ extern "C" rtp_status rtp_decode_step(const rtp_dims* dims, const uint16_t* q_pr
     P.Wq = Wq_idx;
     P.seq_lens = seq_lens;
     P.block_table = dims->block_table;
-    P.p = p;
+    P.p = topk > 0 ? nullptr : p;
+    P.topk = topk;
     P.out = out;
     memcpy(P.tab.rg_group, pl.rg_group, sizeof(P.tab.rg_group));
     memcpy(P.tab.rg_mask, pl.rg_mask, sizeof(P.tab.rg_mask));
@@ -399,6 +445,36 @@ extern "C" rtp_status rtp_decode_step(const rtp_dims* dims, const uint16_t* q_pr
     }
     if (ev) cudaEventRecordWithFlags((cudaEvent_t)ev[2], s, ev_flags);
     return e == cudaSuccess ? RTP_OK : RTP_ERR_CUDA;
+}
+
+extern "C" rtp_status rtp_decode_step(const rtp_dims* dims, const uint16_t* q_pre, const uint16_t* q_rope,
+                                      const uint16_t* k_idx, const uint16_t* k_cache, const uint16_t* v_cache,
+                                      const uint16_t* Wq_idx, const int32_t* seq_lens, const uint8_t* head_kind,
+                                      const float* p, int32_t window, int32_t sink, uint16_t* out, void* stream) {
+    if (!p) return RTP_ERR_NULL;
+    return decode_step_ws(dims, q_pre, q_rope, k_idx, k_cache, v_cache, nullptr, nullptr, 0, Wq_idx, seq_lens,
+                          head_kind, p, 0, window, sink, out, stream);
+}
+
+extern "C" rtp_status rtp_decode_step_ring(const rtp_dims* dims, const uint16_t* q_pre, const uint16_t* q_rope,
+                                           const uint16_t* k_idx, const uint16_t* k_cache, const uint16_t* v_cache,
+                                           const uint16_t* k_ring, const uint16_t* v_ring, int32_t ring_W,
+                                           const uint16_t* Wq_idx, const int32_t* seq_lens,
+                                           const uint8_t* head_kind, const float* p, int32_t window, int32_t sink,
+                                           uint16_t* out, void* stream) {
+    if (!p || !k_ring || !v_ring) return RTP_ERR_NULL;
+    return decode_step_ws(dims, q_pre, q_rope, k_idx, k_cache, v_cache, k_ring, v_ring, ring_W, Wq_idx, seq_lens,
+                          head_kind, p, 0, window, sink, out, stream);
+}
+
+extern "C" rtp_status rtp_decode_step_topk(const rtp_dims* dims, const uint16_t* q_pre, const uint16_t* q_rope,
+                                           const uint16_t* k_idx, const uint16_t* k_cache, const uint16_t* v_cache,
+                                           const uint16_t* Wq_idx, const int32_t* seq_lens,
+                                           const uint8_t* head_kind, int32_t topk, int32_t window, int32_t sink,
+                                           uint16_t* out, void* stream) {
+    if (topk < 1) return RTP_ERR_SHAPE;
+    return decode_step_ws(dims, q_pre, q_rope, k_idx, k_cache, v_cache, nullptr, nullptr, 0, Wq_idx, seq_lens,
+                          head_kind, nullptr, topk, window, sink, out, stream);
 }
 
 extern "C" rtp_status rtp_get_status(const rtp_dims* dims, void* stream) {
@@ -488,11 +564,47 @@ extern "C" rtp_status rtp_decode_step_noalloc(const rtp_dims* dims, const uint16
 }
 
 // ---------------------------------------------------------------------------
+// local heads' ring write
+// ---------------------------------------------------------------------------
+extern "C" rtp_status rtp_ring_write(const rtp_dims* d, const uint16_t* k_new, const uint16_t* v_new,
+                                     const int32_t* pos, int32_t num_new, int32_t ring_W, uint16_t* k_ring,
+                                     uint16_t* v_ring, uint32_t* device_status, void* stream) {
+    if (!d) return RTP_ERR_NULL;
+    if (d->head_dim != D || d->block_size != BLK) return RTP_ERR_UNSUPPORTED;
+    if (d->batch < 1 || d->num_kv_heads < 1 || num_new < 0) return RTP_ERR_SHAPE;
+    if (d->batch > MAX_B || d->num_kv_heads > MAX_HKV) return RTP_ERR_UNSUPPORTED;
+    if (ring_W < BLK || ring_W % BLK) return RTP_ERR_SHAPE;
+    if (num_new == 0) return RTP_OK;
+    if (!k_new || !v_new || !pos || !k_ring || !v_ring) return RTP_ERR_NULL;
+    if (((uintptr_t)k_new | (uintptr_t)v_new | (uintptr_t)k_ring | (uintptr_t)v_ring) & 15u)
+        return RTP_ERR_UNSUPPORTED;
+    RingParams A;
+    A.B = d->batch;
+    A.Hkv = d->num_kv_heads;
+    A.T = num_new;
+    A.W = ring_W;
+    A.k_new = k_new;
+    A.v_new = v_new;
+    A.pos = pos;
+    A.k_ring = k_ring;
+    A.v_ring = v_ring;
+    A.status = device_status;
+    const int64_t threads = (int64_t)A.B * A.Hkv * A.T * 32;
+    const int64_t grid = (threads + 255) / 256;
+    if (grid > 0x7FFFFFFF) return RTP_ERR_UNSUPPORTED;
+    ring_write_kernel<<<(unsigned)grid, 256, 0, (cudaStream_t)stream>>>(A);
+    return report(cudaGetLastError(), "ring write launch") == cudaSuccess ? RTP_OK : RTP_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
 // index-cache append
 // ---------------------------------------------------------------------------
-extern "C" rtp_status rtp_index_append(const rtp_dims* d, const uint16_t* k_pre, const uint16_t* Wk_idx,
-                                       const int32_t* pos, int32_t num_new, uint16_t* k_idx, uint32_t* device_status,
-                                       void* stream) {
+// The index-cache append, with the KV-cache write when k_cache is given.
+static rtp_status append_impl(const rtp_dims* d, const uint16_t* k_pre, const uint16_t* v_new, const uint16_t* Wk_idx,
+                              const float* rope_cos, const float* rope_sin, const int32_t* pos, int32_t num_new,
+                              uint16_t* k_idx, uint16_t* k_cache, uint16_t* v_cache, uint32_t* device_status,
+                              void* stream) {
+    const bool kv = k_cache != nullptr;
     if (!d) return RTP_ERR_NULL;
     if (d->head_dim != D || d->idx_dim != R || d->block_size != BLK) return RTP_ERR_UNSUPPORTED;
     if (d->batch < 1 || d->num_kv_heads < 1 || num_new < 0) return RTP_ERR_SHAPE;
@@ -504,9 +616,14 @@ extern "C" rtp_status rtp_index_append(const rtp_dims* d, const uint16_t* k_pre,
     }
     if (num_new == 0) return RTP_OK;
     if (!k_pre || !Wk_idx || !pos || !k_idx) return RTP_ERR_NULL;
+    if (kv && (!v_new || !rope_cos || !rope_sin || !v_cache)) return RTP_ERR_NULL;
     if (((uintptr_t)k_pre | (uintptr_t)Wk_idx) & 15u) return RTP_ERR_UNSUPPORTED;   // 16-byte vector loads
     if ((uintptr_t)k_idx & 7u) return RTP_ERR_UNSUPPORTED;                            // 8-byte stores of 4 entries
+    if (kv && (((uintptr_t)v_new | (uintptr_t)rope_cos | (uintptr_t)rope_sin | (uintptr_t)k_cache |
+                (uintptr_t)v_cache) & 15u))
+        return RTP_ERR_UNSUPPORTED;                                                    // 16-byte loads and stores
     AppendParams A;
+    memset(&A, 0, sizeof(A));
     A.B = d->batch;
     A.Hkv = d->num_kv_heads;
     A.T = num_new;
@@ -519,11 +636,33 @@ extern "C" rtp_status rtp_index_append(const rtp_dims* d, const uint16_t* k_pre,
     A.block_table = d->block_table;
     A.k_idx = k_idx;
     A.status = device_status;
+    A.v_new = v_new;
+    A.rope_cos = rope_cos;
+    A.rope_sin = rope_sin;
+    A.k_cache = k_cache;
+    A.v_cache = v_cache;
     const int64_t total = (int64_t)A.B * A.Hkv * A.T * (R / APPEND_ROWS);
     const int64_t grid = (total + APPEND_THREADS - 1) / APPEND_THREADS;
     if (grid > 0x7FFFFFFF) return RTP_ERR_UNSUPPORTED;
-    index_append_kernel<<<(unsigned)grid, APPEND_THREADS, 0, (cudaStream_t)stream>>>(A);
-    return report(cudaGetLastError(), "index append launch") == cudaSuccess ? RTP_OK : RTP_ERR_CUDA;
+    if (kv) append_kernel<true><<<(unsigned)grid, APPEND_THREADS, 0, (cudaStream_t)stream>>>(A);
+    else append_kernel<false><<<(unsigned)grid, APPEND_THREADS, 0, (cudaStream_t)stream>>>(A);
+    return report(cudaGetLastError(), "append launch") == cudaSuccess ? RTP_OK : RTP_ERR_CUDA;
+}
+
+extern "C" rtp_status rtp_index_append(const rtp_dims* d, const uint16_t* k_pre, const uint16_t* Wk_idx,
+                                       const int32_t* pos, int32_t num_new, uint16_t* k_idx, uint32_t* device_status,
+                                       void* stream) {
+    return append_impl(d, k_pre, nullptr, Wk_idx, nullptr, nullptr, pos, num_new, k_idx, nullptr, nullptr,
+                       device_status, stream);
+}
+
+extern "C" rtp_status rtp_kv_append(const rtp_dims* d, const uint16_t* k_pre, const uint16_t* v_new,
+                                    const uint16_t* Wk_idx, const float* rope_cos, const float* rope_sin,
+                                    const int32_t* pos, int32_t num_new, uint16_t* k_idx, uint16_t* k_cache,
+                                    uint16_t* v_cache, uint32_t* device_status, void* stream) {
+    if (!k_cache) return RTP_ERR_NULL;
+    return append_impl(d, k_pre, v_new, Wk_idx, rope_cos, rope_sin, pos, num_new, k_idx, k_cache, v_cache,
+                       device_status, stream);
 }
 
 extern "C" const char* rtp_status_string(rtp_status status) {

@@ -231,6 +231,8 @@ __device__ __noinline__ void r_pass(const Params& P, RWalk wk, const int* pre, i
     Acct ac;
     ac.init(P, S.acct, tid == 0);
     const int rp = pass - RP_REF0;
+    // key bits above the refine pass's digit (the prefix found so far); unused in pass RP_REF0
+    constexpr int psh = (pass > RP_REF0 && pass <= RP_REF3) ? 32 - 8 * (pass - RP_REF0) : 0;
     // the parameters this loop uses, read once: through a reference into the
     // parameter block they would be read again after every global atomic
     const int n_ret = P.n_ret, sstride = P.sstride, words_cap = P.words_cap, ntiles_cap = P.ntiles_cap;
@@ -242,6 +244,7 @@ __device__ __noinline__ void r_pass(const Params& P, RWalk wk, const int* pre, i
     unsigned long long* const cand = P.cand;
     uint32_t* const bitmap = P.bitmap;
     uint32_t* const tie_cnt = P.tie_cnt;
+    const bool unit = P.topk > 0;   // static top-k: every token weighs 1 (the histograms count)
     const bool resident = S.resident != 0;
     if (resident) {
         const long long tq = clock64();
@@ -419,7 +422,7 @@ __device__ __noinline__ void r_pass(const Params& P, RWalk wk, const int* pre, i
                 if constexpr (pass == RP_BINS) {
                     if (ok) {
                         const uint32_t bn = score_bin(v[u], rh.smax, rh.dr, rh.inv_w);
-                        const unsigned long long ms = fixmass(key, rh.smax);
+                        const unsigned long long ms = unit ? 1ull : fixmass(key, rh.smax);
                         if (bn < 255u) {
                             hist_add(S.H, hh, (int)bn, 1u, ms);
                         } else {
@@ -429,9 +432,9 @@ __device__ __noinline__ void r_pass(const Params& P, RWalk wk, const int* pre, i
                     }
                 } else if constexpr (pass <= RP_REF3) {
                     if (ok && score_bin(v[u], rh.smax, rh.dr, rh.inv_w) == rh.bstar &&
-                        (rp == 0 || (key >> (32 - 8 * rp)) == rh.prefix)) {
+                        (rp == 0 || (key >> psh) == rh.prefix)) {
                         const uint32_t d = (key >> (24 - 8 * rp)) & 255u;
-                        hist_add(S.H, hh, (int)d, 1u, fixmass(key, rh.smax));
+                        hist_add(S.H, hh, (int)d, 1u, unit ? 1ull : fixmass(key, rh.smax));
                     }
                 } else if constexpr (pass == RP_TIES) {
                     cnt += (ok && key == rh.tau) ? 1u : 0u;
@@ -621,11 +624,17 @@ __device__ __noinline__ void r_digit(const Params& P, int b, int slot, int tid) 
     auto cnt_of = [&](int d) { return S.dcnt[d]; };
     if constexpr (pass == RP_BINS) {
         // z = the total mass; bins ascend in smax - s: the first bin that
-        // completes the target ceil(p z)
+        // completes the target ceil(p z) (top-k: masses are counts, z = L,
+        // and the target is k)
         bin_search(S, mass_of, cnt_of, false, ~0ull, tid);
         const unsigned long long z = S.hit_k;
-        const double pb = (double)__ldg(P.p + b);
-        unsigned long long tg = (unsigned long long)ceil(pb * (double)z);
+        unsigned long long tg;
+        if (P.topk > 0) {
+            tg = (unsigned long long)P.topk;
+        } else {
+            const double pb = (double)__ldg(P.p + b);
+            tg = (unsigned long long)ceil(pb * (double)z);
+        }
         if (tg > z) tg = z;
         if (tg == 0) tg = 1;
         bin_search(S, mass_of, cnt_of, false, tg, tid);
@@ -737,6 +746,7 @@ __device__ __noinline__ void r_local_select(const Params& P, int b, int slot, in
         S.lsel_count = __ldcg(&P.hs[bs].count_above);
     }
     const unsigned long long target = __ldcg(&P.hs[bs].target);
+    const bool unit = P.topk > 0;   // static top-k: every token weighs 1
     for (int rp = rp0; rp < 4; ++rp) {
         for (int d = tid; d < 256; d += CONSUMERS) {
             S.H.cnt[0][d] = 0;
@@ -750,7 +760,7 @@ __device__ __noinline__ void r_local_select(const Params& P, int b, int slot, in
         for (int j = 0; j < CPT; ++j) {
             const uint32_t key = keys[j];
             if (tid + j * CONSUMERS >= n || (rp > 0 && (key >> (32 - 8 * rp)) != prefix)) continue;
-            hist_add(S.H, 0, (int)((key >> (24 - 8 * rp)) & 255u), 1u, fixmass(key, smax));
+            hist_add(S.H, 0, (int)((key >> (24 - 8 * rp)) & 255u), 1u, unit ? 1ull : fixmass(key, smax));
         }
         consumer_sync();
         // the highest digit whose mass completes the target (digits descend)
@@ -1103,23 +1113,14 @@ __device__ __forceinline__ void warp_prefix(int* pre, int n, F cnt, int lane) {
 }
 
 // ---------------------------------------------------------------------------
-// the kernel
+// the retrieval phase: its shared-memory set-up, and its body once the
+// streaming phase's results are visible (after the streaming grid completed,
+// or, in the single launch, after a grid barrier)
 // ---------------------------------------------------------------------------
 template <int G>
-__global__ void __launch_bounds__(THREADS, 2) retrieve_kernel(const __grid_constant__ KParams K) {
+__device__ __forceinline__ void r_setup(const Params& P, int tid) {
     BSmem<G>& S = bsmem<G>();
     constexpr int NST = BSmem<G>::NST;
-    const Params& P = K.P;
-    const int tid = threadIdx.x, lane = tid & 31;
-    const bool copier = tid >= CONSUMERS;
-    // grid barrier; thread 0's wait goes to debug sum 31
-    auto gsync = [&]() {
-        const long long t0 = clock64();
-        const bool r = grid_sync(P, S);
-        if (tid == 0 && P.dbg_trace) S.acct[15] += (unsigned long long)(clock64() - t0);
-        return r;
-    };
-    int* pre = S.pre;
     if (tid == 0) {
         for (int i = 0; i < NST; ++i) {
             mbar_init(&S.full[i], 1);
@@ -1133,9 +1134,24 @@ __global__ void __launch_bounds__(THREADS, 2) retrieve_kernel(const __grid_const
         S.resident = 0;
     }
     if (tid >= 32) copy_tab(P.tab, S.tab, tid - 32, THREADS - 32);
-    // everything below reads the streaming kernel's results: wait for that
-    // grid to complete (this launch overlaps only its tail)
-    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// single: the single launch, whose transition barrier always counts in
+// P.sync->barrier, so the last CTA out always clears the coordination words
+template <int G>
+__device__ __forceinline__ void r_body(const KParams& K, bool single) {
+    BSmem<G>& S = bsmem<G>();
+    const Params& P = K.P;
+    const int tid = threadIdx.x, lane = tid & 31;
+    const bool copier = tid >= CONSUMERS;
+    // grid barrier; thread 0's wait goes to debug sum 31
+    auto gsync = [&]() {
+        const long long t0 = clock64();
+        const bool r = grid_sync(P, S);
+        if (tid == 0 && P.dbg_trace) S.acct[15] += (unsigned long long)(clock64() - t0);
+        return r;
+    };
+    int* pre = S.pre;
     if (tid == 0) S.base = __ldcg(&P.sync->kb_work);
     __syncthreads();
     const bool work = S.base != 0;   // nothing left when every group was settled in the streaming kernel
@@ -1277,9 +1293,10 @@ __global__ void __launch_bounds__(THREADS, 2) retrieve_kernel(const __grid_const
         }
     }
     // the last CTA out clears the call's coordination words (none was set
-    // when every group was settled in the streaming kernel: no count then)
+    // when every group was settled in the streaming kernel: no count then,
+    // except for the single launch's transition barrier)
     __syncthreads();
-    if (work && tid == 0) {
+    if ((work || single) && tid == 0) {
         trace_max(P, 5);
         __threadfence();
         if (atomicAdd(&P.sync->exit_count, 1u) == gridDim.x - 1) {
@@ -1300,6 +1317,54 @@ __global__ void __launch_bounds__(THREADS, 2) retrieve_kernel(const __grid_const
             __threadfence();
         }
     }
+}
+
+__device__ __forceinline__ void mbar_inval(uint64_t* bar) {
+    asm volatile("mbarrier.inval.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// The whole decode step in one launch: the streaming phase, then (after a
+// grid barrier that stands for the retrieval kernel's wait on the streaming
+// grid) the retrieval phase in the same shared memory.  When every group was
+// settled in the streaming phase, the CTAs only clear the call's words and
+// drop the stored scores: no second launch.  One resident wave (the
+// retrieval phase's grid barriers need it).
+template <int G>
+__global__ void __launch_bounds__(THREADS, 2) step_kernel(const __grid_constant__ KParams K) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const Params& P = K.P;
+    const int tid = threadIdx.x;
+    if (smem_u32(smem_raw) & 1023u) {   // (the same for every CTA: none waits for another)
+        if (tid == 0) set_status(P, 5u);
+        return;
+    }
+    s_body<G, true>(K);
+    __syncthreads();
+    // the streaming phase's ring barriers end here (no copy is in flight:
+    // its copy warp waited for its last tiles); the memory becomes the
+    // retrieval phase's
+    if (tid == 0) {
+        ASmem<G>& A = *reinterpret_cast<ASmem<G>*>(smem_raw);
+        for (int i = 0; i < ASmem<G>::NST; ++i) {
+            mbar_inval(&A.full[i]);
+            mbar_inval(&A.empty[i]);
+        }
+    }
+    __syncthreads();
+    r_setup<G>(P, tid);
+    __syncthreads();
+    grid_sync(P, bsmem<G>());   // a timeout sets S.abort: the body then skips its work
+    r_body<G>(K, true);
+}
+
+template <int G>
+__global__ void __launch_bounds__(THREADS, 2) retrieve_kernel(const __grid_constant__ KParams K) {
+    const int tid = threadIdx.x;
+    r_setup<G>(K.P, tid);
+    // everything below reads the streaming kernel's results: wait for that
+    // grid to complete (this launch overlaps only its tail)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    r_body<G>(K, false);
 }
 
 }  // namespace rtp

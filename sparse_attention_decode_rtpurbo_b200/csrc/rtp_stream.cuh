@@ -267,6 +267,9 @@ __device__ __forceinline__ void best_token_list(const Params& P, ASmem<G>& S, in
 // Heads whose best token alone reaches p (TOP1) or whose p >= 1 (ALL) are
 // final here; if every head of the group is final its block list is written
 // at once, otherwise its radix heads are registered for the exact select.
+// Under static top-k (P.topk = k >= 1) the same three outcomes are k >= L
+// (ALL), k = 1 (TOP1: the argmax, lowest index among equal maxima) and any
+// other k (the exact select, counting tokens instead of summing mass).
 template <int G>
 __device__ __forceinline__ void decide_group(const KParams& K, ASmem<G>& S, int b, int rg, int L, float pb, int tid) {
     const Params& P = K.P;
@@ -316,7 +319,20 @@ __device__ __forceinline__ void decide_group(const KParams& K, ASmem<G>& S, int 
         const double z = (S.d_flags[hh] || sm4 > 600.0 || sm4 < -600.0) ? NAN : S.d_zabs[hh] * exp_wide(-sm4);
         int mode;
         uint32_t kstar = 0, tau_key = 0;
-        if (!(pb > 0.f)) {
+        const int topk = P.topk;
+        if (topk > 0) {
+            if (topk >= L) {
+                mode = MODE_ALL;
+                kstar = (uint32_t)L;
+                tau_key = mn;
+            } else if (topk == 1) {
+                mode = MODE_TOP1;
+                kstar = 1;
+                tau_key = k;
+            } else {
+                mode = MODE_RADIX;
+            }
+        } else if (!(pb > 0.f)) {
             mode = MODE_SKIP;
             set_status(P, ST_DEVICE_INPUT);
         } else if (pb >= 1.f) {
@@ -356,10 +372,13 @@ __device__ __forceinline__ void decide_group(const KParams& K, ASmem<G>& S, int 
             h.tau_key = 0;
             h.tie_idx = 0xFFFFFFFFu;
             h.kstar = 0;
-            const float omp = fmaxf(1.f - pb, 1e-6f);
-            const float zz = (z == z && z >= 1.0) ? (float)fmin(z, 1e30) : 1.f;
-            float dr = 4.f * (__logf((float)L) - __logf(omp) - __logf(zz)) + 8.f;
-            dr = fminf(fmaxf(dr, 8.f), 400.f);
+            float dr = 400.f;   // top-k: the k-th score may lie anywhere in the range
+            if (topk == 0) {
+                const float omp = fmaxf(1.f - pb, 1e-6f);
+                const float zz = (z == z && z >= 1.0) ? (float)fmin(z, 1e30) : 1.f;
+                dr = 4.f * (__logf((float)L) - __logf(omp) - __logf(zz)) + 8.f;
+                dr = fminf(fmaxf(dr, 8.f), 400.f);
+            }
             const float range = smax - key2f(mn);
             if (range >= 0.f) dr = fminf(dr, range + fmaxf(range * 0x1p-10f, 1e-6f));
             h.dr = dr;
@@ -694,12 +713,17 @@ __device__ __forceinline__ void a_producer(const KParams& K, ASmem<G>& S, AWalk 
                 }
             } else if (lane == 0) {
                 const int j = sg.type == 1 ? (ti < lg.nA ? ti : lg.bw0 + (ti - lg.nA)) : (int)(S.d_list[ti] >> 8);
-                const int row = (int)block_row(P, sg.b, g, j);
+                // local groups without retrieval heads may keep only a ring of
+                // their sink and window (the tiles' position masks stay as they are)
+                const bool ring = sg.type == 1 && ((P.ring_lg_mask >> sg.grp) & 1ull);
+                const int row = ring ? (int)ring_block_row(P, sg.b, g, j) : (int)block_row(P, sg.b, g, j);
+                const CUtensorMap* mk = ring ? &K.tmk_r : &K.tmk;
+                const CUtensorMap* mv = ring ? &K.tmv_r : &K.tmv;
                 mbar_expect_tx(&S.full[st], STAGE_BYTES);
-                tma_load_2d(dst, &K.tmk, 0, row, &S.full[st]);
-                tma_load_2d(dst + 8192, &K.tmk, 64, row, &S.full[st]);
-                tma_load_2d(dst + KV_TILE, &K.tmv, 0, row, &S.full[st]);
-                tma_load_2d(dst + KV_TILE + 8192, &K.tmv, 64, row, &S.full[st]);
+                tma_load_2d(dst, mk, 0, row, &S.full[st]);
+                tma_load_2d(dst + 8192, mk, 64, row, &S.full[st]);
+                tma_load_2d(dst + KV_TILE, mv, 0, row, &S.full[st]);
+                tma_load_2d(dst + KV_TILE + 8192, mv, 64, row, &S.full[st]);
             }
             __syncwarp();
         }
@@ -753,7 +777,7 @@ __device__ __forceinline__ void a_consumers(const KParams& K, ASmem<G>& S, AWalk
             ScoreFold f;
             f.reset();
             const bool nh4 = nh <= 4;
-            const float pb = __ldg(P.p + sg.b);
+            const float pb = P.p ? __ldg(P.p + sg.b) : 1.f;   // (no p under static top-k)
             const bool track_min = true;   // (the threshold when p >= 1; the select's bin range otherwise)
             ac.mark(21);
             for (int i = 0; i < sg.ntiles; ++i, ++k) {
@@ -860,8 +884,10 @@ __device__ __forceinline__ void a_consumers(const KParams& K, ASmem<G>& S, AWalk
 // ---------------------------------------------------------------------------
 // the kernel
 // ---------------------------------------------------------------------------
-template <int G>
-__global__ void __launch_bounds__(THREADS, 2) stream_kernel(const __grid_constant__ KParams K) {
+// The streaming phase.  SINGLE: part of the single launch (no dependent
+// grid to release; every thread returns here, the copy warp included).
+template <int G, bool SINGLE>
+__device__ __forceinline__ void s_body(const KParams& K) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];   // no static shared memory: the base is aligned
     ASmem<G>& S = *reinterpret_cast<ASmem<G>*>(smem_raw);
     constexpr int NST = ASmem<G>::NST;
@@ -887,7 +913,7 @@ __global__ void __launch_bounds__(THREADS, 2) stream_kernel(const __grid_constan
     }
     // the retrieval kernel may be scheduled now; it waits for this grid's
     // completion before it reads anything this grid writes
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    if constexpr (!SINGLE) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (tid >= 32) copy_tab(P.tab, S.tab, tid - 32, THREADS - 32);
     // tiles per sequence (score tiles of all retrieval groups, then local
     // tiles of all local groups), prefix-summed by warp 0
@@ -949,6 +975,11 @@ __global__ void __launch_bounds__(THREADS, 2) stream_kernel(const __grid_constan
     }
     a_consumers<G>(K, S, wk, pre_s, pre_l, tid);
     if (tid == 0) trace_max(P, 5);
+}
+
+template <int G>
+__global__ void __launch_bounds__(THREADS, 2) stream_kernel(const __grid_constant__ KParams K) {
+    s_body<G, false>(K);
 }
 
 }  // namespace rtp

@@ -56,15 +56,40 @@ class DeviceCase:
             }
             self.dbg_struct = rtp.RtpDebug(*(self.dbg[k].data_ptr() for k in
                                              ("tau", "kstar", "kept_blocks", "smax", "Z", "block_bitmap", "trace")))
+        self.topk = 0   # > 0: run() takes the static top-k variant with this k
+        self.ring_W = 0  # > 0: run() reads the local-only KV heads from k_ring / v_ring (attach_ring)
+        self.k_ring = self.v_ring = None
         self.step = rtp.Step(c.B, c.Hq, c.Hkv, c.Ncap, c.head_kind, block_table=self.block_table,
                              num_pages=c.num_pages, device=device, debug=self.dbg_struct)
 
+    def attach_ring(self, k_ring: np.ndarray, v_ring: np.ndarray, ring_W: int):
+        """Rings [B, Hkv, 64 + ring_W, 128] (uint16 bf16) for the local-only KV heads."""
+        self.k_ring = bf16_tensor(k_ring, self.device)
+        self.v_ring = bf16_tensor(v_ring, self.device)
+        self.ring_W = int(ring_W)
+
     def run(self, stream=None):
         c = self.case
+        if self.topk > 0:
+            return self.run_topk(self.topk, stream)
+        if self.ring_W > 0:
+            if stream is None:
+                stream = torch.cuda.current_stream(self.out.device)
+            return self.step.ring(self.q_pre, self.q_rope, self.k_idx, self.k_cache, self.v_cache, self.k_ring,
+                                  self.v_ring, self.ring_W, self.Wq, self.seq_lens, self.p, c.window, c.sink,
+                                  self.out, stream)
         if stream is None:
             stream = torch.cuda.current_stream(self.out.device)
         self.step(self.q_pre, self.q_rope, self.k_idx, self.k_cache, self.v_cache, self.Wq, self.seq_lens, self.p,
                   c.window, c.sink, self.out, stream)
+
+    def run_topk(self, k: int, stream=None):
+        """The static top-k variant of the step (every retrieval head keeps k tokens)."""
+        c = self.case
+        if stream is None:
+            stream = torch.cuda.current_stream(self.out.device)
+        self.step.topk(self.q_pre, self.q_rope, self.k_idx, self.k_cache, self.v_cache, self.Wq, self.seq_lens, k,
+                       c.window, c.sink, self.out, stream)
 
     def results(self) -> Dict[str, np.ndarray]:
         torch.cuda.synchronize()

@@ -76,6 +76,30 @@ def test_host_side_errors_launch_nothing():
     assert _call(d4) == 3                             # RTP_ERR_UNSUPPORTED
 
 
+def _call_topk(d, topk, window=64, sink=4, ptr=256, **nulls):
+    args = {k: ptr for k in ("q_pre", "q_rope", "k_idx", "k_cache", "v_cache", "Wq", "seq_lens", "out")}
+    args.update(nulls)
+    return rtp.lib.rtp_decode_step_topk(ctypes.byref(d), args["q_pre"], args["q_rope"], args["k_idx"],
+                                        args["k_cache"], args["v_cache"], args["Wq"], args["seq_lens"],
+                                        rtp._head_kind_buf(HK), topk, window, sink, args["out"], None)
+
+
+def test_topk_host_side_checks():
+    """rtp_decode_step_topk: k < 1 is refused; p is not an argument, so the
+    remaining checks (nulls, local set, workspace) are rtp_decode_step's."""
+    d = dims()
+    assert _call_topk(d, 0) == 2                      # RTP_ERR_SHAPE: k must be >= 1
+    assert _call_topk(d, -5) == 2
+    assert _call_topk(d, 4096, q_pre=None) == 1       # RTP_ERR_NULL
+    assert _call_topk(d, 4096, window=0, sink=0) == 2
+    assert _call_topk(d, 4096) == 4                   # RTP_ERR_WORKSPACE: none given (the checks passed)
+    assert _call_topk(d, 1 << 30) == 4                # any k >= 1 is valid (k >= L keeps every block)
+    d4 = dims()
+    d4.idx_dim = 32
+    assert _call_topk(d4, 16) == 3
+    assert _call(d, p=None) == 1                      # the top-p step still needs p
+
+
 def test_paged_geometry_checks():
     d = dims(block_table=4096, max_blocks_per_seq=32, num_pages=10)   # 32*64 != 4096
     assert rtp.workspace_size(d, HK) == 0
@@ -105,6 +129,71 @@ def test_index_append_host_side_checks():
     assert call(d, fake + 2, fake, fake, 1, fake, None, None) == 3                     # k_pre not 16-byte aligned
     assert call(d, fake, fake, fake, 1, fake + 4, None, None) == 3                     # k_idx not 8-byte aligned
     assert call(dims(num_kv_heads=65, num_q_heads=65), fake, fake, fake, 1, fake, None, None) == 3
+
+
+def test_ring_host_side_checks():
+    """rtp_decode_step_ring: ring sizes are checked before any CUDA call."""
+    fake = 4096
+
+    def call(d, W=128, window=64, sink=4, kr=fake, vr=fake, p=fake):
+        return rtp.lib.rtp_decode_step_ring(ctypes.byref(d), fake, fake, fake, fake, fake, kr, vr, W, fake, fake,
+                                            rtp._head_kind_buf(HK), p, window, sink, fake, None)
+
+    d = dims()
+    assert call(d, kr=None) == 1
+    assert call(d, vr=None) == 1
+    assert call(d, p=None) == 1
+    assert call(d, W=96) == 2                        # not a multiple of 64
+    assert call(d, W=64, window=65) == 2             # the window does not fit
+    assert call(d, W=0, window=0) == 2
+    assert call(d, sink=65) == 2                     # the sink must fit the 64 head rows
+    assert call(d, kr=fake + 8) == 3
+    assert call(d) == 4                              # checks passed; no workspace given
+
+
+def test_ring_write_host_side_checks():
+    fake = 4096
+
+    def call(d, n=1, W=128, kn=fake, vn=fake, kr=fake, vr=fake, pos=fake):
+        return rtp.lib.rtp_ring_write(ctypes.byref(d) if d is not None else None, kn, vn, pos, n, W, kr, vr, None,
+                                      None)
+
+    d = dims()
+    assert call(None) == 1
+    assert call(d, n=0) == 0                         # nothing to write
+    assert call(d, n=-1) == 2
+    assert call(d, W=96) == 2
+    assert call(d, W=0) == 2
+    assert call(d, kr=None) == 1
+    assert call(d, pos=None) == 1
+    assert call(d, vn=fake + 4) == 3
+
+
+def test_kv_append_host_side_checks():
+    """rtp_kv_append: bad arguments are refused before any CUDA call."""
+    fake = 4096   # never dereferenced: every call below returns first
+    d = dims()
+
+    def call(dd, k_pre=fake, v_new=fake, wk=fake, cs=fake, sn=fake, pos=fake, n=1, kidx=fake, kc=fake, vc=fake):
+        return rtp.lib.rtp_kv_append(ctypes.byref(dd) if dd is not None else None, k_pre, v_new, wk, cs, sn, pos, n,
+                                     kidx, kc, vc, None, None)
+
+    assert call(None) == 1                           # NULL dims
+    assert call(d, kc=None) == 1                     # NULL key cache
+    assert call(d, vc=None) == 1                     # NULL value cache
+    assert call(d, v_new=None) == 1                  # NULL new values
+    assert call(d, cs=None) == 1                     # NULL angle table
+    assert call(d, n=0) == 0                         # nothing to append
+    assert call(d, n=-1) == 2
+    assert call(d, n=4097) == 2                      # more than the capacity
+    assert call(d, v_new=fake + 8) == 3              # 16-byte alignment of every row-wise operand
+    assert call(d, sn=fake + 4) == 3
+    assert call(d, kc=fake + 2) == 3
+    assert call(d, vc=fake + 8) == 3
+    assert call(d, kidx=fake + 4) == 3               # k_idx: 8-byte aligned, as rtp_index_append
+    bad = dims()
+    bad.head_dim = 64
+    assert call(bad) == 3
 
 
 def test_binding_refuses_host_and_strided_tensors():

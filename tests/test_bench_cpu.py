@@ -29,6 +29,31 @@ def test_kernel_source_hash_is_stable_and_short():
     assert h == bench.kernel_source_hash() and len(h) == 16 and int(h, 16) >= 0
 
 
+def test_stage_inputs_views_and_one_copy():
+    """The staged inputs: views with the tensors' shapes, dtypes and values at
+    256-byte aligned offsets; one copy of the host buffer reproduces them."""
+    import numpy as np
+    import torch
+
+    import bench
+
+    q = np.arange(2 * 3 * 128, dtype=np.float64).reshape(2, 3, 128) / 7.0
+    q_bits = np.asarray(torch.from_numpy(q).to(torch.bfloat16).view(torch.int16).numpy()).view(np.uint16)
+    lens = np.array([5, 9], np.int32)
+    p = np.array([0.9, 0.5], np.float32)
+    tensors = [torch.from_numpy(q_bits.view(np.int16)).view(torch.bfloat16), torch.from_numpy(lens.copy()),
+               torch.from_numpy(p.copy())]
+    dbuf, hbuf, views = bench.stage_inputs(tensors, [q_bits, lens, p], "cpu", pin=False)
+    for t, v in zip(tensors, views):
+        assert v.dtype == t.dtype and v.shape == t.shape and torch.equal(v.view(torch.uint8), t.view(torch.uint8))
+        assert (v.data_ptr() - dbuf.data_ptr()) % 256 == 0
+    for v in views:
+        v.zero_()
+    dbuf.copy_(hbuf)
+    for t, v in zip(tensors, views):
+        assert torch.equal(v.view(torch.uint8), t.view(torch.uint8))
+
+
 def test_algorithmic_bytes_by_hand():
     """The roofline numerator on hand-countable cases: index rows per
     retrieval group, the union of the group's kept blocks (the last block

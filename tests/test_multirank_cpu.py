@@ -74,7 +74,7 @@ def test_reference_arm_other_ranks_do_no_work(capsys):
     sys.path.insert(0, ROOT)
     import bench
 
-    args = Namespace(workload=1, scale=1, dense=False, warmup=0, steps=1, gpus=2)
+    args = Namespace(workload=1, scale=1, dense=False, topk=0, warmup=0, steps=1, gpus=2)
     bench.run_reference(args, rank=1)
     assert capsys.readouterr().out == ""
     bench.run_reference(args, rank=0)

@@ -46,8 +46,10 @@ def parse():
     ap.add_argument("--dense", action="store_true", help="p = 1 for every sequence (dense comparator)")
     ap.add_argument("--topk", type=int, default=0,
                     help="static top-k selection with this k (the fixed-budget variant) instead of top-p")
-    ap.add_argument("--dense-comparator", action="store_true",
-                    help="also time the same captured step with p = 1 and add it to the line as dense_comparator")
+    ap.add_argument("--no-dense-comparator", action="store_true",
+                    help="skip timing the same captured step with p = 1 (the line's dense_comparator)")
+    ap.add_argument("--no-per-workload", action="store_true",
+                    help="time only the headline workload (skip the 32K, 4 x 128K and ragged lines)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--op", choices=["decode", "append", "kv_append"], default="decode",
                     help="append: time the index-cache append instead of the decode step; "
@@ -358,6 +360,193 @@ def bench_append(args):
                           "warmup": args.warmup, "l2": "flushed (256 MB write) before every call"}), flush=True)
 
 
+class StepBench:
+    """One workload on the device, ready to time: its inputs staged in one
+    device buffer (so the end-to-end leg makes one host-to-device copy), a
+    CUDA graph of one rtp_decode_step, and a second graph that records the
+    library's phase events between its kernels."""
+
+    def __init__(self, case, args, dev, flush):
+        import ctypes
+
+        import torch
+
+        import sparse_attention_decode_rtpurbo_b200 as rtp
+        from synth.torch_io import DeviceCase
+
+        self.case, self.dev, self.flush = case, dev, flush
+        self.stream = torch.cuda.current_stream(dev)
+        dc = DeviceCase(case, device=dev, debug=True)
+        dc.topk = max(0, args.topk)
+        self.dbuf, self.hbuf, views = stage_inputs(
+            [dc.q_pre, dc.q_rope, dc.seq_lens, dc.p],
+            [case.q_pre, case.q_rope, case.seq_lens.astype(np.int32), case.p.astype(np.float32)], dev)
+        dc.q_pre, dc.q_rope, dc.seq_lens, dc.p = views
+        self.dc = dc
+        # one debug step: kept blocks for the algorithmic byte count
+        dc.run(self.stream)
+        res = dc.results()
+        if res["status"] != 0:
+            raise SystemExit(f"device status {res['status']}")
+        self.nbytes = algorithmic_bytes(case, res["kept"])
+        ret = np.nonzero(case.head_kind)[0]
+        self.kept_tokens = float(np.mean([res["kstar"][b, h] / case.seq_lens[b] for b in range(case.B)
+                                          for h in ret])) if ret.size else 0.0
+        self.kept_blocks = float(np.mean([res["kept_blocks"][b, h] / ((case.seq_lens[b] + 63) // 64)
+                                          for b in range(case.B) for h in ret])) if ret.size else 0.0
+        dc.step.dims.debug = ctypes.POINTER(rtp.RtpDebug)()   # timed steps run without diagnostics
+        self.inner = [torch.cuda.Event(enable_timing=True) for _ in range(rtp.TIMING_EVENTS)]
+        for e in self.inner:
+            e.record(self.stream)
+        dc.run(self.stream)                                   # eager warm-up (sets kernel attributes)
+        torch.cuda.synchronize(dev)
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            dc.run(torch.cuda.current_stream(dev))
+        dc.step.set_timing_events(self.inner)
+        self.graph_ev = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph_ev):
+            dc.run(torch.cuda.current_stream(dev))
+        dc.step.set_timing_events(None)
+
+    def warm(self, n):
+        import torch
+
+        for _ in range(n):
+            self.flush()
+            self.graph.replay()
+            self.flush()
+            self.graph_ev.replay()
+        torch.cuda.synchronize(self.dev)
+
+    def timed(self, steps, replay=None):
+        """Device time (ms) of each of `steps` graph replays, L2 flushed before each."""
+        import torch
+
+        replay = replay or self.graph.replay
+        out = []
+        for _ in range(steps):
+            self.flush()
+            a = torch.cuda.Event(enable_timing=True)
+            z = torch.cuda.Event(enable_timing=True)
+            a.record(self.stream)
+            replay()
+            z.record(self.stream)
+            z.synchronize()
+            out.append(a.elapsed_time(z))
+        return out
+
+    def phases(self, steps):
+        import sparse_attention_decode_rtpurbo_b200 as rtp
+
+        acc = [0.0] * len(rtp.PHASES)
+        for _ in range(steps):
+            self.flush()
+            self.graph_ev.replay()
+            self.inner[-1].synchronize()
+            for k in range(len(rtp.PHASES)):
+                acc[k] += self.inner[k].elapsed_time(self.inner[k + 1])
+        return {n: acc[k] / steps for k, n in enumerate(rtp.PHASES)}
+
+    def timeline(self, reps=5):
+        """Median over `reps` debug-traced steps of the library's timeline (us since the first CTA)."""
+        import ctypes
+
+        import torch
+
+        import sparse_attention_decode_rtpurbo_b200 as rtp
+
+        dc = self.dc
+        trace_buf = torch.zeros(rtp.TRACE_WORDS, dtype=torch.int64, device=self.dev)
+        tdbg = rtp.RtpDebug(trace=trace_buf.data_ptr())
+        dc.step.dims.debug = ctypes.pointer(tdbg)
+        tl = []
+        for _ in range(reps):
+            self.flush()
+            trace_buf.zero_()
+            dc.run(self.stream)
+            torch.cuda.synchronize(self.dev)
+            t = trace_buf.cpu().numpy().astype(np.float64)
+            ev = {n: (t[k] - t[0]) / 1e3 if t[k] > 0 else None for k, n in enumerate(rtp.TRACE_EVENTS) if k}
+            for k, n in enumerate(rtp.TRACE_SUMS):
+                v = t[16 + k]
+                ev[n] = ((v - t[0]) / 1e3 if v > 0 else None) if n in rtp.TRACE_SUM_EVENTS else v
+            tl.append(ev)
+        dc.step.dims.debug = ctypes.POINTER(rtp.RtpDebug)()
+        return {n: (statistics.median([x[n] for x in tl]) if tl[0][n] is not None else None) for n in tl[0]}
+
+    def e2e(self, steps, warmup):
+        """End to end through the public call: each step copies the staged
+        per-step inputs host -> device (one pinned copy), calls
+        rtp_decode_step eagerly through the Python binding (argument
+        checks, workspace plan and tensor maps on the host every call), and
+        copies the output device -> host.  Also the same with the captured
+        graph in place of the eager call."""
+        import torch
+
+        dc = self.dc
+        hout = torch.empty(dc.out.shape, dtype=torch.bfloat16).pin_memory()
+
+        def leg(call):
+            ts = []
+            for i in range(warmup + steps):
+                self.flush()
+                a = torch.cuda.Event(enable_timing=True)
+                z = torch.cuda.Event(enable_timing=True)
+                a.record(self.stream)
+                self.dbuf.copy_(self.hbuf, non_blocking=True)
+                call()
+                hout.copy_(dc.out, non_blocking=True)
+                z.record(self.stream)
+                z.synchronize()
+                if i >= warmup:
+                    ts.append(a.elapsed_time(z))
+            return statistics.mean(ts)
+
+        eager = leg(lambda: dc.run(self.stream))
+        graph = leg(self.graph.replay)
+        return eager, graph, self.hbuf.numel(), hout.numel() * hout.element_size()
+
+    def dense(self, steps, warmup):
+        """The same captured step with p = 1 for every sequence (every block
+        of every retrieval head): the stand-in for the pages' dense-attention
+        baseline.  Returns (mean ms, device status)."""
+        import torch
+
+        dc, case = self.dc, self.case
+        dc.p.fill_(1.0)
+        dts = self.timed(warmup + steps)[warmup:]
+        dc.p.copy_(torch.from_numpy(case.p.astype(np.float32)).to(self.dev))
+        torch.cuda.synchronize(self.dev)
+        return statistics.mean(dts), dc.step.status()
+
+    def status(self):
+        return self.dc.step.status()
+
+
+def step_summary(sb, step_ms, peak, dense_ms=0.0, dense_status=0):
+    """us/step (mean, median, p10/p90), context-tokens/s and the step's HBM fraction."""
+    t_ms = statistics.mean(step_ms)
+    tokens = float(sb.case.seq_lens.sum())
+    gbs = sb.nbytes["total"] / (t_ms * 1e-3) / 1e9
+    d = {"us_per_step": t_ms * 1e3, "us_per_step_median": statistics.median(step_ms) * 1e3,
+         "us_per_step_p10_p90": [float(np.percentile(step_ms, 10)) * 1e3, float(np.percentile(step_ms, 90)) * 1e3],
+         "context_tokens_per_s": tokens / (t_ms * 1e-3),
+         "step_roofline": {"algorithmic_bytes": sb.nbytes, "achieved": gbs, "peak": peak, "unit": "GB/s",
+                           "frac": gbs / peak},
+         "sparsity": {"kept_token_frac": sb.kept_tokens, "kept_block_frac": sb.kept_blocks}}
+    if dense_ms > 0:
+        d["dense_comparator"] = {"us_per_step": dense_ms * 1e3, "value": tokens / (dense_ms * 1e-3), "unit": UNIT,
+                                 "speedup_of_sparse": dense_ms / t_ms, "device_status": dense_status,
+                                 "what": "the same step with p = 1 (every block of every retrieval head)"}
+    return d
+
+
+# the other workloads of the metric's range (32K to 1M), timed after the
+# headline with fewer steps; the 4K workload is a parity case only
+OTHER_WORKLOADS = (2, 3, 5)
+
+
 def main():
     args = parse()
     if args.op in ("append", "kv_append"):
@@ -374,7 +563,6 @@ def main():
 
     import sparse_attention_decode_rtpurbo_b200 as rtp
     import synth
-    from synth.torch_io import DeviceCase
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
@@ -387,35 +575,6 @@ def main():
         if world > 1:
             dist.barrier()
 
-    case = synth.workload(args.workload, scale=args.scale)
-    if args.dense:
-        case.p[:] = 1.0
-    dc = DeviceCase(case, device=dev, debug=True)
-    dc.topk = max(0, args.topk)
-    # the per-step inputs (queries, lengths, p) share one device buffer, so the
-    # end-to-end leg moves them in one host-to-device copy; set before any
-    # step is captured, so the graphs take these addresses
-    dbuf, hbuf, views = stage_inputs(
-        [dc.q_pre, dc.q_rope, dc.seq_lens, dc.p],
-        [case.q_pre, case.q_rope, case.seq_lens.astype(np.int32), case.p.astype(np.float32)], dev)
-    dc.q_pre, dc.q_rope, dc.seq_lens, dc.p = views
-    stream = torch.cuda.current_stream(dev)
-
-    # one debug step: kept blocks for the algorithmic byte count
-    dc.run(stream)
-    res = dc.results()
-    if res["status"] != 0:
-        raise SystemExit(f"device status {res['status']}")
-    nbytes = algorithmic_bytes(case, res["kept"])
-    ret = np.nonzero(case.head_kind)[0]
-    kept_tokens = float(np.mean([res["kstar"][b, h] / case.seq_lens[b] for b in range(case.B) for h in ret])) \
-        if ret.size else 0.0
-    kept_blocks = float(np.mean([res["kept_blocks"][b, h] / ((case.seq_lens[b] + 63) // 64)
-                                 for b in range(case.B) for h in ret])) if ret.size else 0.0
-    import ctypes
-
-    dc.step.dims.debug = ctypes.POINTER(rtp.RtpDebug)()   # timed steps run without diagnostics
-
     # L2 flush between timed steps: write 256 MB, then read another 256 MB so
     # the dirty lines of the write are evicted before the step, not during it
     flush_w = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
@@ -425,128 +584,37 @@ def main():
         flush_w.zero_()
         flush_r.sum(dtype=torch.int64)
 
-    # one step = one replay of a CUDA graph holding one rtp_decode_step (its
-    # two kernels).  A second graph records phase events between the kernels
-    # (which serialises them); it is replayed separately for the per-kernel
-    # durations, never inside the timed steps.
-    NE = rtp.TIMING_EVENTS
-    inner = [torch.cuda.Event(enable_timing=True) for _ in range(NE)]
-    for e in inner:
-        e.record(stream)
-    dc.run(stream)                               # eager warm-up (sets kernel attributes)
-    torch.cuda.synchronize(dev)
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph):
-        dc.run(torch.cuda.current_stream(dev))
-    dc.step.set_timing_events(inner)
-    graph_ev = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph_ev):
-        dc.run(torch.cuda.current_stream(dev))
-    dc.step.set_timing_events(None)
-    for _ in range(max(3, args.warmup)):
-        flush()
-        graph.replay()
-        flush()
-        graph_ev.replay()
-    torch.cuda.synchronize(dev)
+    case = synth.workload(args.workload, scale=args.scale)
+    if args.dense:
+        case.p[:] = 1.0
+    sb = StepBench(case, args, dev, flush)
+    sb.warm(max(3, args.warmup))
 
     sampler = ClockSampler(local_rank)
     sampler.start()
     time.sleep(0.3)
     barrier()
     torch.cuda.synchronize(dev)
-    step_ms, phase_acc = [], [0.0] * len(rtp.PHASES)
     t_begin = time.perf_counter()
-    for i in range(args.steps):
-        flush()
-        a = torch.cuda.Event(enable_timing=True)
-        z = torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        graph.replay()
-        z.record(stream)
-        z.synchronize()
-        step_ms.append(a.elapsed_time(z))
+    step_ms = sb.timed(args.steps)
     torch.cuda.synchronize(dev)
     barrier()
     wall = time.perf_counter() - t_begin
     clocks = sampler.stop()
-    for i in range(args.steps):
-        flush()
-        graph_ev.replay()
-        inner[-1].synchronize()
-        for k in range(len(rtp.PHASES)):
-            phase_acc[k] += inner[k].elapsed_time(inner[k + 1])
-    phase_ms = {n: phase_acc[k] / args.steps for k, n in enumerate(rtp.PHASES)}
-    t_ms = statistics.mean(step_ms)
-
-    # ---- timeline of one step (debug trace, separate untimed replays) ----
-    trace_buf = torch.zeros(rtp.TRACE_WORDS, dtype=torch.int64, device=dev)
-    tdbg = rtp.RtpDebug(trace=trace_buf.data_ptr())
-    dc.step.dims.debug = ctypes.pointer(tdbg)
-    tl = []
-    for _ in range(5):
-        flush()
-        trace_buf.zero_()
-        dc.run(stream)
-        torch.cuda.synchronize(dev)
-        t = trace_buf.cpu().numpy().astype(np.float64)
-        ev = {n: (t[k] - t[0]) / 1e3 if t[k] > 0 else None for k, n in enumerate(rtp.TRACE_EVENTS) if k}
-        for k, n in enumerate(rtp.TRACE_SUMS):
-            v = t[16 + k]
-            # timestamps (ns) become times since the start; cycle sums stay raw
-            ev[n] = ((v - t[0]) / 1e3 if v > 0 else None) if n in ("a_first_data", "a_consumers_done") else v
-        tl.append(ev)
-    dc.step.dims.debug = ctypes.POINTER(rtp.RtpDebug)()
-    timeline = {n: (statistics.median([x[n] for x in tl]) if tl[0][n] is not None else None)
-                for n in tl[0]}
-
-    # ---- end to end: host query/len/p -> device (one staged copy), step, output -> host ----
-    hout = torch.empty(dc.out.shape, dtype=torch.bfloat16).pin_memory()
-    h2d = hbuf.numel()
-    d2h = hout.numel() * hout.element_size()
-    e2e_ms = []
-    for i in range(max(3, args.warmup) + args.steps):
-        flush()
-        a = torch.cuda.Event(enable_timing=True)
-        z = torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        dbuf.copy_(hbuf, non_blocking=True)
-        graph.replay()
-        hout.copy_(dc.out, non_blocking=True)
-        z.record(stream)
-        z.synchronize()
-        if i >= max(3, args.warmup):
-            e2e_ms.append(a.elapsed_time(z))
-    e2e_t = statistics.mean(e2e_ms)
-    if dc.step.status() != 0:
+    phase_ms = sb.phases(args.steps)
+    timeline = sb.timeline()
+    e2e_t, e2e_graph_t, h2d, d2h = sb.e2e(args.steps, max(3, args.warmup))
+    if sb.status() != 0:
         raise SystemExit("device status set during the timed steps")
-
-    # ---- dense comparator: the same captured step with p = 1 for every
-    # sequence (every block of every retrieval head), the stand-in for the
-    # pages' dense-attention baseline; the graph reads p from dc.p ----
     dense_ms, dense_status = 0.0, 0
-    if args.dense_comparator and not args.dense and args.topk == 0 and case.head_kind.any():
-        dc.p.fill_(1.0)
-        dts = []
-        for i in range(max(3, args.warmup) + args.steps):
-            flush()
-            a = torch.cuda.Event(enable_timing=True)
-            z = torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            graph.replay()
-            z.record(stream)
-            z.synchronize()
-            if i >= max(3, args.warmup):
-                dts.append(a.elapsed_time(z))
-        dc.p.copy_(torch.from_numpy(case.p.astype(np.float32)).to(dev))
-        torch.cuda.synchronize(dev)
-        dense_status = dc.step.status()          # reported, not fatal: the main line stands
-        dense_ms = statistics.mean(dts)
+    if not args.no_dense_comparator and not args.dense and args.topk == 0 and case.head_kind.any():
+        dense_ms, dense_status = sb.dense(args.steps, max(3, args.warmup))
 
     # ---- max over ranks ----
-    vals = max_over_ranks([t_ms, e2e_t, dense_ms] + [phase_ms[n] for n in rtp.PHASES], world, dev)
-    t_ms, e2e_t, dense_ms = vals[0], vals[1], vals[2]
-    phase_ms = {n: vals[3 + k] for k, n in enumerate(rtp.PHASES)}
+    t_ms = statistics.mean(step_ms)
+    vals = max_over_ranks([t_ms, e2e_t, e2e_graph_t, dense_ms] + [phase_ms[n] for n in rtp.PHASES], world, dev)
+    t_ms, e2e_t, e2e_graph_t, dense_ms = vals[:4]
+    phase_ms = {n: vals[4 + k] for k, n in enumerate(rtp.PHASES)}
 
     tokens = float(case.seq_lens.sum())
     value = world * tokens / (t_ms * 1e-3)
@@ -555,12 +623,34 @@ def main():
     # sink/window K/V) and, when there are retrieval heads,
     # rtp::retrieve_kernel (kept K/V blocks; exact select when needed).
     # The roofline is reported for the one that takes longer.
+    nbytes = sb.nbytes
     kbytes = {"stream": nbytes["index"] + nbytes["local"], "retrieve": nbytes["kept_kv"]}
     has_ret = bool(case.head_kind.any())
     dom = "retrieve" if has_ret and phase_ms["retrieve"] > phase_ms["stream"] else "stream"
     ach = kbytes[dom] / (phase_ms[dom] * 1e-3) / 1e9
-    step_gbs = nbytes["total"] / (t_ms * 1e-3) / 1e9
     launches_per_step = 2 if has_ret else 1
+    summary = step_summary(sb, step_ms, peak, dense_ms, dense_status)
+    del sb
+    torch.cuda.empty_cache()
+
+    # ---- the metric's other context lengths (32K, 4 x 128K, ragged paged) ----
+    per_workload = {}
+    if args.workload == 4 and args.scale == 1 and not args.dense and args.topk == 0 and not args.no_per_workload:
+        for wl in OTHER_WORKLOADS:
+            c2 = synth.workload(wl)
+            s2 = StepBench(c2, args, dev, flush)
+            s2.warm(3)
+            ms2 = s2.timed(max(5, args.steps // 2))
+            dm2, ds2 = s2.dense(max(5, args.steps // 2), 3) if c2.head_kind.any() else (0.0, 0)
+            st2 = s2.status()
+            ms2_max = max_over_ranks([statistics.mean(ms2), dm2], world, dev)
+            entry = step_summary(s2, ms2, peak, dm2, ds2)
+            entry["us_per_step_max_over_ranks"] = ms2_max[0] * 1e3
+            entry["config"] = workload_config(c2, wl)
+            entry["device_status"] = st2
+            per_workload[synth.WORKLOADS[wl]] = entry
+            del s2
+            torch.cuda.empty_cache()
 
     line = None
     if rank == 0:
@@ -587,33 +677,34 @@ def main():
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": t_ms, "us_per_step": t_ms * 1e3,
-            "us_per_step_p10_p90": [float(np.percentile(step_ms, 10)) * 1e3, float(np.percentile(step_ms, 90)) * 1e3],
+            "us_per_step_median": summary["us_per_step_median"],
+            "us_per_step_p10_p90": summary["us_per_step_p10_p90"],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16 in, fp32 accumulate",
             "data": "synthetic (seeded generators in synth/, shaped like the pages' workloads)",
             "config": dict(workload_config(case, args.workload), parallelism=f"replicas x{world}",
                            dense_p1=bool(args.dense), selection=selection_name(args), timing="CUDA-graph replay of one rtp_decode_step (2 kernels, programmatic launch) per step; "
-                           "CUDA events on the launching stream"),
+                           "CUDA events on the launching stream; value from the mean step time"),
             "wall_s_timed_loop": wall,
             "roofline": {"bound": "hbm", "kernel": f"rtp::{dom}_kernel", "achieved": ach, "peak": peak, "unit": "GB/s",
                          "frac": ach / peak, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, burst)",
                          "traffic": profiled_traffic(dom, case.name) if selection_name(args) == "top-p" else None,
                          "algorithmic_bytes_per_launch": kbytes[dom],
                          "us_per_launch": phase_ms[dom] * 1e3},
-            "step_roofline": {"algorithmic_bytes": nbytes, "achieved": step_gbs, "peak": peak, "unit": "GB/s",
-                              "frac": step_gbs / peak},
+            "step_roofline": summary["step_roofline"],
             "phases_us": {n: phase_ms[n] * 1e3 for n in rtp.PHASES},
             "timeline_us": timeline,
-            "sparsity": {"kept_token_frac": kept_tokens, "kept_block_frac": kept_blocks},
+            "sparsity": summary["sparsity"],
             "e2e": {"value": world * tokens / (e2e_t * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h, "us_per_step": e2e_t * 1e3},
+                    "d2h_bytes_per_step": d2h, "us_per_step": e2e_t * 1e3,
+                    "what": "eager rtp_decode_step through the Python binding per step (host checks, plan and "
+                            "tensor maps included), inputs host->device in one pinned copy, output device->host",
+                    "graph_replay": {"value": world * tokens / (e2e_graph_t * 1e-3), "us_per_step": e2e_graph_t * 1e3,
+                                     "what": "the same with the captured graph in place of the eager call"}},
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clocks,
             "cpu_baseline": cpu,
-            "dense_comparator": ({"us_per_step": dense_ms * 1e3, "value": world * tokens / (dense_ms * 1e-3),
-                                  "unit": UNIT, "speedup_of_sparse": dense_ms / t_ms,
-                                  "device_status": dense_status,
-                                  "what": "the same step with p = 1 (every block of every retrieval head)"}
-                                 if dense_ms > 0 else None),
+            "dense_comparator": summary.get("dense_comparator"),
+            "per_workload": per_workload or None,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -82,9 +82,12 @@ typedef struct rtp_debug {
      *   6 group decision started, 7 streaming shares assigned, 8-11 selection steps done
      *   (local select / refine passes 2-4), 12 block marks done, 13 retrieval kernel started,
      *   14 first selection pass and digits done, 15 retrieval attention started.
-     * 16-47: sums over CTAs of one thread's SM cycles (or counts) by phase; the Python
+     * 16-40: sums over CTAs of one thread's SM cycles (or counts) by phase; the Python
      *   binding's TRACE_SUMS names them in order (slots 22 and 23 are %globaltimer events:
-     *   first index tile consumed, last streaming share done). */
+     *   first index tile consumed, last streaming share done).
+     * 43-47: latest %globaltimer ns over CTAs of: 43 a group decision reduced its
+     *   buckets, 44 ... decided its heads' modes, 46 an index split took its ticket,
+     *   47 an index split reduced its scores (41, 42 and 45 unused). */
     unsigned long long* trace;
 } rtp_debug;
 
@@ -129,7 +132,9 @@ typedef struct rtp_dims {
 /*
  * Bytes of device workspace rtp_decode_step needs for these sizes and this
  * head split (head_kind is a HOST array of num_q_heads bytes, 1 = retrieval,
- * 0 = local).  Returns 0 if the sizes are invalid or unsupported.
+ * 0 = local: the score scratch and the per-head state scale with the number
+ * of retrieval heads, so the size depends on the split, not on the sizes
+ * alone).  Returns 0 if the sizes are invalid or unsupported.
  */
 size_t rtp_workspace_size(const rtp_dims* dims, const uint8_t* head_kind);
 
@@ -142,7 +147,11 @@ size_t rtp_workspace_size(const rtp_dims* dims, const uint8_t* head_kind);
  *   v_cache   same layout as k_cache, bf16 values
  *   Wq_idx    [Hq, 16, 128] bf16 indexer query projections (rows of local heads unused)
  *   seq_lens  [B] int32, 1 <= L <= cap (device)
- *   head_kind [Hq] uint8, HOST memory: 1 = retrieval head, 0 = local head
+ *   head_kind [Hq] uint8, HOST memory: 1 = retrieval head, 0 = local head.
+ *             (A host array, where a device array would match the rest: the
+ *             head split is fixed per layer by offline calibration, and the
+ *             host needs it to size the grids and the workspace exactly, so
+ *             the call reads it without a device-to-host copy.)
  *   p         [B] fp32 top-p mass per sequence, in (0, 1]; >= 1 keeps all tokens (device)
  *   window, sink: local heads' sliding window and sink sizes, >= 0, window + sink >= 1
  *   out       [B, Hq, 128] bf16 (round to nearest even)
@@ -269,10 +278,15 @@ rtp_status rtp_get_status(const rtp_dims* dims, void* stream);
  *   that the kernels expect at zero, since the array keeps whatever the
  *   previous call left), the kernels, and, with device_status, one 4-byte
  *   device-to-device cudaMemcpyAsync.
- * Set-up: the first call on each device looks up the array's device address
- *   (cudaGetSymbolAddress, with that device current; the library is loaded
- *   onto the device then if it was not yet).  Make that first call outside
- *   any stream capture.  A failed lookup returns RTP_ERR_CUDA.
+ * Set-up: every call looks up the array's device address in the current
+ *   device's context (cudaGetSymbolAddress, with that device current), so a
+ *   context that was reset and made again is followed.  The first call in a
+ *   context also loads the library's kernels into it: make that first call
+ *   outside any stream capture.  A failed lookup returns RTP_ERR_CUDA and
+ *   enqueues nothing.
+ * Host-side errors (RTP_ERR_NULL, _SHAPE, _UNSUPPORTED, _SCRATCH_LIMIT,
+ *   a failed lookup or tensor-map encoding) return before anything is
+ *   enqueued, as for rtp_decode_step.
  * Concurrency: every call on a device shares the one array.  Calls whose
  *   work overlaps on the GPU (different streams without ordering between
  *   them) race on it and produce wrong results; order them on one stream.

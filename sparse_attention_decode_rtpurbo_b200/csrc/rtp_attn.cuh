@@ -46,7 +46,9 @@ struct MmaAttn {
 
     __device__ __forceinline__ void init() { q_tag = -1; }
 
-    __device__ __forceinline__ void begin(const Params& P, int b, int g, int lane) {
+    // arrive: the CTA's first segment (named barrier 4 lets the copy warp
+    // issue the first tile once the query loads are on their way)
+    __device__ __forceinline__ void begin(const Params& P, int b, int g, int lane, bool arrive = false) {
         const int tag = b * P.Hkv + g;
         if (tag != q_tag) {
             q_tag = tag;
@@ -59,6 +61,7 @@ struct MmaAttn {
                 qa[kk][1] = hr < G ? __ldg(q + 8 * kk + 4 + t) : 0u;
             }
         }
+        if (arrive) asm volatile("bar.arrive 4, 160;" ::: "memory");
         m = -INFINITY;
         l = 0.f;
 #pragma unroll
@@ -329,36 +332,40 @@ struct QFrag {
 // issued before its first product (one or two memory round trips, not D / 8).
 template <int TPP>
 __device__ __forceinline__ void qidx_pairs(const Params& P, const HeadTab& T, float (*qi)[R], int b, int rg,
-                                           int tid) {
+                                           int tid, bool arrive) {
     constexpr int SPAN = D / TPP, NV = SPAN / 8;
     const int nh = T.rg_nh[rg], slot0 = T.rg_slot0[rg];
     const int pr = tid / TPP, part = tid % TPP;
+    // threads beyond the nh x 16 pairs load pair 0's operands (valid
+    // addresses, no branch around the loads) and store nothing
+    const int pe = pr < nh * R ? pr : 0;
+    const int hh = pe / R, r = pe % R;
+    const int h = T.slot_head[slot0 + hh];
+    const uint4* w = reinterpret_cast<const uint4*>(P.Wq + ((int64_t)h * R + r) * D + part * SPAN);
+    const uint4* q = reinterpret_cast<const uint4*>(P.q_pre + ((int64_t)b * P.Hq + h) * D + part * SPAN);
+    constexpr int NB = NV < 8 ? NV : 8;   // loads in flight per operand (register budget)
     float a = 0.f;
-    if (pr < nh * R) {
-        const int hh = pr / R, r = pr % R;
-        const int h = T.slot_head[slot0 + hh];
-        const uint4* w = reinterpret_cast<const uint4*>(P.Wq + ((int64_t)h * R + r) * D + part * SPAN);
-        const uint4* q = reinterpret_cast<const uint4*>(P.q_pre + ((int64_t)b * P.Hq + h) * D + part * SPAN);
-        constexpr int NB = NV < 8 ? NV : 8;   // loads in flight per operand (register budget)
 #pragma unroll
-        for (int i0 = 0; i0 < NV; i0 += NB) {
-            uint4 wv[NB], qv[NB];
+    for (int i0 = 0; i0 < NV; i0 += NB) {
+        uint4 wv[NB], qv[NB];
 #pragma unroll
-            for (int i = 0; i < NB; ++i) {
-                wv[i] = __ldg(w + i0 + i);
-                qv[i] = __ldg(q + i0 + i);
-            }
+        for (int i = 0; i < NB; ++i) {
+            wv[i] = __ldg(w + i0 + i);
+            qv[i] = __ldg(q + i0 + i);
+        }
+        // the CTA's first segment: its copy warp issues the first tile only
+        // once these loads are on their way (named barrier 4)
+        if (i0 == 0 && arrive) asm volatile("bar.arrive 4, 160;" ::: "memory");
 #pragma unroll
-            for (int i = 0; i < NB; ++i) {
-                a = fmaf(bf_lo(wv[i].x), bf_lo(qv[i].x), a);
-                a = fmaf(bf_hi(wv[i].x), bf_hi(qv[i].x), a);
-                a = fmaf(bf_lo(wv[i].y), bf_lo(qv[i].y), a);
-                a = fmaf(bf_hi(wv[i].y), bf_hi(qv[i].y), a);
-                a = fmaf(bf_lo(wv[i].z), bf_lo(qv[i].z), a);
-                a = fmaf(bf_hi(wv[i].z), bf_hi(qv[i].z), a);
-                a = fmaf(bf_lo(wv[i].w), bf_lo(qv[i].w), a);
-                a = fmaf(bf_hi(wv[i].w), bf_hi(qv[i].w), a);
-            }
+        for (int i = 0; i < NB; ++i) {
+            a = fmaf(bf_lo(wv[i].x), bf_lo(qv[i].x), a);
+            a = fmaf(bf_hi(wv[i].x), bf_hi(qv[i].x), a);
+            a = fmaf(bf_lo(wv[i].y), bf_lo(qv[i].y), a);
+            a = fmaf(bf_hi(wv[i].y), bf_hi(qv[i].y), a);
+            a = fmaf(bf_lo(wv[i].z), bf_lo(qv[i].z), a);
+            a = fmaf(bf_hi(wv[i].z), bf_hi(qv[i].z), a);
+            a = fmaf(bf_lo(wv[i].w), bf_lo(qv[i].w), a);
+            a = fmaf(bf_hi(wv[i].w), bf_hi(qv[i].w), a);
         }
     }
 #pragma unroll
@@ -367,12 +374,12 @@ __device__ __forceinline__ void qidx_pairs(const Params& P, const HeadTab& T, fl
 }
 
 __device__ __forceinline__ void compute_qidx(const Params& P, const HeadTab& T, float (*qi)[R], int b, int rg,
-                                             int tid) {
+                                             int tid, bool arrive = false) {
     const int npair = T.rg_nh[rg] * R;   // <= 128
-    if (npair <= CONSUMERS / 8) qidx_pairs<8>(P, T, qi, b, rg, tid);
-    else if (npair <= CONSUMERS / 4) qidx_pairs<4>(P, T, qi, b, rg, tid);
-    else if (npair <= CONSUMERS / 2) qidx_pairs<2>(P, T, qi, b, rg, tid);
-    else qidx_pairs<1>(P, T, qi, b, rg, tid);
+    if (npair <= CONSUMERS / 8) qidx_pairs<8>(P, T, qi, b, rg, tid, arrive);
+    else if (npair <= CONSUMERS / 4) qidx_pairs<4>(P, T, qi, b, rg, tid, arrive);
+    else if (npair <= CONSUMERS / 2) qidx_pairs<2>(P, T, qi, b, rg, tid, arrive);
+    else qidx_pairs<1>(P, T, qi, b, rg, tid, arrive);
 }
 
 // B fragment of this lane (column g = lane/4 = head g; k = 2t, 2t+1, 2t+8, 2t+9)

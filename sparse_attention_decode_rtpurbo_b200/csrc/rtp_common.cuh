@@ -58,7 +58,8 @@ struct Sync {
     uint32_t exit_count;
     uint32_t kb_work;          // groups left to the retrieval kernel (a select, or blocks to attend)
     uint32_t any_global;       // some radix head's threshold bin is too large for the in-CTA select
-    uint32_t pad[16];
+    uint32_t n_decided;        // (b, group) pairs decided so far (a count the single launch waits for)
+    uint32_t pad[15];
 };
 
 // Head split (host-derived): retrieval groups (KV heads with >= 1 retrieval
@@ -313,6 +314,10 @@ __device__ __forceinline__ void kv_prefetch_l2(const CUtensorMap* mk, const CUte
     tma_prefetch_2d(mk, 64, row);
     tma_prefetch_2d(mv, 0, row);
     tma_prefetch_2d(mv, 64, row);
+}
+// L2 prefetch of the 128-byte line at p (a hint: nothing to wait for)
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 

@@ -258,8 +258,18 @@ static cudaError_t launch(const KParams& K, const Plan& pl, cudaStream_t s, void
         const int occ = occupancy((const void*)step_kernel<G>, smem);
         if (occ < 1) return report(cudaErrorInvalidConfiguration, "step kernel occupancy");
         const int grid = std::min(cap, occ * sms);
-        step_kernel<G><<<(unsigned)grid, THREADS, smem, s>>>(K);
-        cudaError_t e = report(cudaGetLastError(), "step kernel launch");
+        cudaLaunchConfig_t cfg;
+        memset(&cfg, 0, sizeof(cfg));
+        cfg.gridDim = dim3((unsigned)grid);
+        cfg.blockDim = dim3(THREADS);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = s;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeCooperative;   // every CTA resident: the grid barrier's premise
+        attr[0].val.cooperative = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        cudaError_t e = report(cudaLaunchKernelEx(&cfg, step_kernel<G>, K), "step kernel launch");
         if (ev) cudaEventRecordWithFlags((cudaEvent_t)ev[1], s, ev_flags);   // (no phase boundary to mark)
         return e;
     }
@@ -289,11 +299,16 @@ static cudaError_t launch(const KParams& K, const Plan& pl, cudaStream_t s, void
         cfg.blockDim = dim3(THREADS);
         cfg.dynamicSmemBytes = smem;
         cfg.stream = s;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        // cooperative: the driver places every CTA at once or refuses the
+        // launch, so the grid barriers never wait on a CTA that kernels of
+        // other streams keep from starting
+        cudaLaunchAttribute attr[2];
+        attr[0].id = cudaLaunchAttributeCooperative;
+        attr[0].val.cooperative = 1;
+        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[1].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
-        cfg.numAttrs = ev ? 0 : 1;   // an event recorded in between orders the kernels anyway
+        cfg.numAttrs = ev ? 1 : 2;   // an event recorded in between orders the kernels anyway
         cudaError_t e = report(cudaLaunchKernelEx(&cfg, retrieve_kernel<G>, K), "retrieval kernel launch");
         if (e != cudaSuccess) return e;
     }
@@ -320,7 +335,7 @@ static rtp_status decode_step_ws(const rtp_dims* dims, const uint16_t* q_pre, co
                                  const uint16_t* k_ring, const uint16_t* v_ring, int32_t ring_W,
                                  const uint16_t* Wq_idx, const int32_t* seq_lens, const uint8_t* head_kind,
                                  const float* p, int32_t topk, int32_t window, int32_t sink, uint16_t* out,
-                                 void* stream) {
+                                 void* stream, bool clear_first = false) {
     if (!dims || !q_pre || !q_rope || !k_idx || !k_cache || !v_cache || !Wq_idx || !seq_lens || !head_kind ||
         (topk == 0 && !p) || !out || (k_ring && !v_ring))
         return RTP_ERR_NULL;
@@ -430,6 +445,9 @@ static rtp_status decode_step_ws(const rtp_dims* dims, const uint16_t* q_pre, co
         P.dbg_trace = dims->debug->trace;
     }
     cudaStream_t s = (cudaStream_t)stream;
+    // (the no-alloc entry point: the scratch's zero region is cleared only
+    // now that every host-side check has passed)
+    if (clear_first && cudaMemsetAsync(ws, 0, pl.zero_end, s) != cudaSuccess) return RTP_ERR_CUDA;
     void* const* ev = (dims->timing_events && dims->n_timing_events >= RTP_TIMING_EVENTS) ? dims->timing_events : nullptr;
     // under stream capture the records must become event nodes of the graph
     cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
@@ -499,28 +517,16 @@ namespace rtp {
 
 static __device__ __align__(256) uint8_t noalloc_scratch[RTP_NOALLOC_SCRATCH_BYTES];
 
-constexpr int NOALLOC_MAX_DEVICES = 64;
-static std::atomic<void*> noalloc_addr[NOALLOC_MAX_DEVICES];
-static std::mutex noalloc_mutex;
-
-// Device address of noalloc_scratch on the current device, looked up once per
-// device (the lookup loads the module onto the device if needed).
+// Device address of noalloc_scratch in the current device's context, looked
+// up on every call: the address belongs to the module as loaded into that
+// context, and a context that was destroyed and made again (cudaDeviceReset)
+// may hold the module at another address.  The lookup loads the module into
+// the context if it is not loaded yet; after that it is a table lookup.
 static cudaError_t noalloc_scratch_ptr(uint8_t** out) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    void* a = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&a, noalloc_scratch);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= NOALLOC_MAX_DEVICES) return cudaErrorInvalidDevice;
-    void* a = noalloc_addr[dev].load(std::memory_order_acquire);
-    if (!a) {
-        std::lock_guard<std::mutex> lock(noalloc_mutex);
-        a = noalloc_addr[dev].load(std::memory_order_acquire);
-        if (!a) {
-            e = cudaGetSymbolAddress(&a, noalloc_scratch);
-            if (e != cudaSuccess) return e;
-            if (!a) return cudaErrorInvalidSymbol;
-            noalloc_addr[dev].store(a, std::memory_order_release);
-        }
-    }
+    if (!a) return cudaErrorInvalidSymbol;
     *out = static_cast<uint8_t*>(a);
     return cudaSuccess;
 }
@@ -538,6 +544,9 @@ extern "C" rtp_status rtp_decode_step_noalloc(const rtp_dims* dims, const uint16
         !out)
         return RTP_ERR_NULL;
     if (window < 0 || sink < 0 || (int64_t)window + sink < 1) return RTP_ERR_SHAPE;
+    if (!aligned16(q_pre) || !aligned16(q_rope) || !aligned16(k_idx) || !aligned16(k_cache) || !aligned16(v_cache) ||
+        !aligned16(Wq_idx) || !aligned16(out))
+        return RTP_ERR_UNSUPPORTED;
     Plan pl;
     rtp_status st = make_plan(dims, head_kind, window, sink, &pl);
     if (st != RTP_OK) return st;
@@ -549,13 +558,14 @@ extern "C" rtp_status rtp_decode_step_noalloc(const rtp_dims* dims, const uint16
     // other sizes.  The kernels expect zero in the status word, the
     // coordination and ticket words, the per-head bucket aggregates and the
     // radix histograms, which the layout puts first ([0, zero_end)); every
-    // other region is written before it is read.
-    if (cudaMemsetAsync(ws, 0, pl.zero_end, s) != cudaSuccess) return RTP_ERR_CUDA;
+    // other region is written before it is read.  The step clears that
+    // region itself, after its host-side checks, so that a call refused on
+    // the host enqueues nothing.
     rtp_dims d = *dims;
     d.workspace = ws;
     d.workspace_bytes = RTP_NOALLOC_SCRATCH_BYTES;
-    st = rtp_decode_step(&d, q_pre, q_rope, k_idx, k_cache, v_cache, Wq_idx, seq_lens, head_kind, p, window, sink,
-                         out, stream);
+    st = decode_step_ws(&d, q_pre, q_rope, k_idx, k_cache, v_cache, nullptr, nullptr, 0, Wq_idx, seq_lens, head_kind,
+                        p, 0, window, sink, out, stream, true);
     if (st != RTP_OK) return st;
     if (device_status &&
         cudaMemcpyAsync(device_status, ws + pl.o_status, sizeof(uint32_t), cudaMemcpyDeviceToDevice, s) != cudaSuccess)

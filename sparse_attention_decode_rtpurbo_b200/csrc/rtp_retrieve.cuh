@@ -1136,6 +1136,41 @@ __device__ __forceinline__ void r_setup(const Params& P, int tid) {
     if (tid >= 32) copy_tab(P.tab, S.tab, tid - 32, THREADS - 32);
 }
 
+// The call's coordination words back to zero, by the last CTA out of the
+// call's last kernel (after an aborted call also the select histograms it
+// may have left).
+__device__ __noinline__ void clear_call_words(const Params& P) {
+    P.sync->n_radix_heads = 0;
+    P.sync->n_radix_groups = 0;
+    P.sync->any_ties = 0;
+    P.sync->barrier = 0;
+    P.sync->kb_work = 0;
+    if (__ldcg(P.status) != 0) {
+        for (int64_t i = 0; i < (int64_t)P.B * P.n_ret * 256; ++i) {
+            P.hist_cnt[i] = 0;
+            P.hist_mass[i] = 0ull;
+        }
+    }
+    P.sync->any_global = 0;
+    P.sync->n_decided = 0;
+    P.sync->exit_count = 0;
+    __threadfence();
+}
+
+// The stored scores are dead once the select is done (or was not needed):
+// drop their L2 lines without writing them back (each CTA a slice of every
+// retrieval head's used range).
+__device__ __forceinline__ void drop_scores(const Params& P, int tid) {
+    for (int bs = 0; bs < P.B * P.n_ret; ++bs) {
+        const int L = __ldg(P.seq_lens + bs / P.n_ret);
+        if (!seq_ok(P, L)) continue;
+        const char* base = reinterpret_cast<const char*>(P.scores + (int64_t)bs * P.sstride);
+        const int nlines = (L * 4 + 127) / 128;
+        for (int x = blockIdx.x * THREADS + tid; x < nlines; x += gridDim.x * THREADS)
+            asm volatile("discard.global.L2 [%0], 128;" ::"l"(base + (int64_t)x * 128) : "memory");
+    }
+}
+
 // single: the single launch, whose transition barrier always counts in
 // P.sync->barrier, so the last CTA out always clears the coordination words
 template <int G>
@@ -1153,6 +1188,9 @@ __device__ __forceinline__ void r_body(const KParams& K, bool single) {
     };
     int* pre = S.pre;
     if (tid == 0) S.base = __ldcg(&P.sync->kb_work);
+    // (two launches: the streaming grid is complete, nothing else counts the
+    // decisions of this call)
+    if (!single && blockIdx.x == 0 && tid == 0) P.sync->n_decided = 0;
     __syncthreads();
     const bool work = S.base != 0;   // nothing left when every group was settled in the streaming kernel
     if (tid == 0) trace_max(P, 13);
@@ -1280,18 +1318,7 @@ __device__ __forceinline__ void r_body(const KParams& K, bool single) {
         if (tid == 0) trace_max(P, 4);
     }
     if (tid == 0) acct_flush(P, S.acct);
-    // the stored scores are dead now: drop their L2 lines without writing
-    // them back (each CTA a slice of every retrieval head's used range)
-    if (ok || !work) {
-        for (int bs = 0; bs < P.B * P.n_ret; ++bs) {
-            const int L = __ldg(P.seq_lens + bs / P.n_ret);
-            if (!seq_ok(P, L)) continue;
-            const char* base = reinterpret_cast<const char*>(P.scores + (int64_t)bs * P.sstride);
-            const int nlines = (L * 4 + 127) / 128;
-            for (int x = blockIdx.x * THREADS + tid; x < nlines; x += gridDim.x * THREADS)
-                asm volatile("discard.global.L2 [%0], 128;" ::"l"(base + (int64_t)x * 128) : "memory");
-        }
-    }
+    if (ok || !work) drop_scores(P, tid);
     // the last CTA out clears the call's coordination words (none was set
     // when every group was settled in the streaming kernel: no count then,
     // except for the single launch's transition barrier)
@@ -1299,23 +1326,7 @@ __device__ __forceinline__ void r_body(const KParams& K, bool single) {
     if ((work || single) && tid == 0) {
         trace_max(P, 5);
         __threadfence();
-        if (atomicAdd(&P.sync->exit_count, 1u) == gridDim.x - 1) {
-            P.sync->n_radix_heads = 0;
-            P.sync->n_radix_groups = 0;
-            P.sync->any_ties = 0;
-            P.sync->barrier = 0;
-            P.sync->kb_work = 0;
-            if (__ldcg(P.status) != 0) {
-                // an aborted call may leave select histograms behind
-                for (int64_t i = 0; i < (int64_t)P.B * P.n_ret * 256; ++i) {
-                    P.hist_cnt[i] = 0;
-                    P.hist_mass[i] = 0ull;
-                }
-            }
-            P.sync->any_global = 0;
-            P.sync->exit_count = 0;
-            __threadfence();
-        }
+        if (atomicAdd(&P.sync->exit_count, 1u) == gridDim.x - 1) clear_call_words(P);
     }
 }
 
@@ -1343,8 +1354,9 @@ __global__ void __launch_bounds__(THREADS, 2) step_kernel(const __grid_constant_
     // the streaming phase's ring barriers end here (no copy is in flight:
     // its copy warp waited for its last tiles); the memory becomes the
     // retrieval phase's
+    ASmem<G>& A = *reinterpret_cast<ASmem<G>*>(smem_raw);
+    const uint32_t ngroups = (uint32_t)A.n_vgroups;
     if (tid == 0) {
-        ASmem<G>& A = *reinterpret_cast<ASmem<G>*>(smem_raw);
         for (int i = 0; i < ASmem<G>::NST; ++i) {
             mbar_inval(&A.full[i]);
             mbar_inval(&A.empty[i]);
@@ -1353,7 +1365,29 @@ __global__ void __launch_bounds__(THREADS, 2) step_kernel(const __grid_constant_
     __syncthreads();
     r_setup<G>(P, tid);
     __syncthreads();
-    grid_sync(P, bsmem<G>());   // a timeout sets S.abort: the body then skips its work
+    // wait until every group is decided (the deciding CTAs are running: each
+    // took its group's last ticket); if none was left to the retrieval
+    // phase, drop the stored scores and leave without a grid barrier
+    BSmem<G>& S = bsmem<G>();
+    if (tid == 0) {
+        if (!wait_counter(&P.sync->n_decided, ngroups)) {
+            set_status(P, ST_TIMEOUT);
+            S.abort = 1;
+        }
+        S.base = __ldcg(&P.sync->kb_work);
+    }
+    __syncthreads();
+    if (S.base == 0u || S.abort != 0u) {
+        drop_scores(P, tid);
+        __syncthreads();
+        if (tid == 0) {
+            // the last CTA out clears the call's words
+            __threadfence();
+            if (atomicAdd(&P.sync->exit_count, 1u) == gridDim.x - 1) clear_call_words(P);
+        }
+        return;
+    }
+    grid_sync(P, S);   // a timeout sets S.abort: the body then skips its work
     r_body<G>(K, true);
 }
 

@@ -38,6 +38,7 @@ struct ASmem {
     uint32_t flag;
     unsigned long long acct[ACCT_SLOTS];   // debug cycle sums of thread 0
     int tot_s, tot_l, nact;
+    int n_vgroups;   // (b, retrieval group) pairs of sequences with a valid length
     HeadTab tab;
     int pre[2];   // really [2 * (B + 1)]: tiles before sequence b (score, then local)
 };
@@ -271,7 +272,8 @@ __device__ __forceinline__ void best_token_list(const Params& P, ASmem<G>& S, in
 // (ALL), k = 1 (TOP1: the argmax, lowest index among equal maxima) and any
 // other k (the exact select, counting tokens instead of summing mass).
 template <int G>
-__device__ __forceinline__ void decide_group(const KParams& K, ASmem<G>& S, int b, int rg, int L, float pb, int tid) {
+__device__ __forceinline__ void decide_group_body(const KParams& K, ASmem<G>& S, int b, int rg, int L, float pb,
+                                                  int tid) {
     const Params& P = K.P;
     const int nh = S.tab.rg_nh[rg], slot0 = S.tab.rg_slot0[rg], g = S.tab.rg_group[rg];
     const int nblk = (L + BLK - 1) / BLK;
@@ -307,6 +309,7 @@ __device__ __forceinline__ void decide_group(const KParams& K, ASmem<G>& S, int 
         }
     }
     consumer_sync();
+    if (tid == 0) trace_max(P, 43);
     if (tid < nh) {
         const int hh = tid, slot = slot0 + hh;
         const unsigned long long best = S.d_best[hh];
@@ -401,10 +404,12 @@ __device__ __forceinline__ void decide_group(const KParams& K, ASmem<G>& S, int 
         S.d_arg[hh] = a;
     }
     consumer_sync();
+    if (tid == 0) trace_max(P, 44);
     {
         // the common case first: every head keeps its best token only
-        bool top1 = P.dbg_bitmap == nullptr;
+        bool top1 = true;
         for (int hh = 0; hh < nh; ++hh) top1 = top1 && S.d_mode[hh] == MODE_TOP1;
+        top1 = top1 && P.dbg_bitmap == nullptr;
         if (top1) {
             if (tid == 0) best_token_list<G>(P, S, b, rg, L, nh, slot0, g);
             return;
@@ -478,6 +483,19 @@ __device__ __forceinline__ void decide_group(const KParams& K, ASmem<G>& S, int 
         // attended by this CTA after its share (the first such group of the
         // CTA; a later one goes to the retrieval kernel)
         if (tid == 0) best_token_list<G>(P, S, b, rg, L, nh, slot0, g);
+    }
+}
+
+// The decision of one group, then the count of decided groups (the single
+// launch waits for all of them before it either leaves or goes on to the
+// retrieval phase).
+template <int G>
+__device__ __forceinline__ void decide_group(const KParams& K, ASmem<G>& S, int b, int rg, int L, float pb, int tid) {
+    decide_group_body<G>(K, S, b, rg, L, pb, tid);
+    consumer_sync();
+    if (tid == 0) {
+        __threadfence();
+        atomicAdd(&K.P.sync->n_decided, 1u);
     }
 }
 
@@ -668,9 +686,9 @@ __device__ __forceinline__ void a_producer(const KParams& K, ASmem<G>& S, AWalk 
     bool extra = false;
     for (Seg sg = wk.next(P, pre_s, pre_l, S.tot_s);; sg = extra ? Seg{-1} : wk.next(P, pre_s, pre_l, S.tot_s)) {
         if (sg.type < 0 || !alive) {
-            if (extra) break;
-            // share issued: meet the compute warps, then issue the best-token
-            // blocks their group decision put in shared memory (if any)
+            // share (or one more round) issued: meet the compute warps, then
+            // issue the best-token blocks their group decision left in d_list,
+            // until a round leaves none
             extra = true;
             asm volatile("bar.sync 3, 160;" ::: "memory");
             if (!alive || S.d_cnt == 0) break;
@@ -678,6 +696,10 @@ __device__ __forceinline__ void a_producer(const KParams& K, ASmem<G>& S, AWalk 
         }
         const int g = sg.type == 0 ? S.tab.rg_group[sg.grp] : (sg.type == 1 ? S.tab.lg_group[sg.grp] : S.tab.rg_group[sg.grp]);
         const LocalGeom lg = local_geom(P, sg.L);
+        // the first tile of the share waits until the compute warps' query
+        // loads are issued: those few lines then reach this SM ahead of the
+        // 32 KB tile, not behind the whole grid's first burst
+        if (k == 0 && sg.type != 2) asm volatile("bar.sync 4, 160;" ::: "memory");
         for (int i = 0; i < sg.ntiles; ++i, ++k) {
             const int st = (int)(k % NST);
             const uint32_t round = k / NST;
@@ -752,12 +774,14 @@ __device__ __forceinline__ void a_consumers(const KParams& K, ASmem<G>& S, AWalk
     Acct ac;
     ac.init(P, S.acct, tid == 0);
     bool first_data = true;
+    bool first_seg = true;   // its query loads release the copy warp's first tile (barrier 4)
     bool extra = false;
     for (Seg sg = wk.next(P, pre_s, pre_l, S.tot_s);; sg = extra ? Seg{-1} : wk.next(P, pre_s, pre_l, S.tot_s)) {
         if (sg.type < 0) {
-            if (extra) break;
-            // share done: meet the copy warp, then the best-token blocks this
-            // CTA selected (if any) follow through the ring as one more segment
+            // share done (or one more round of it): meet the copy warp; the
+            // best-token blocks of a group this CTA decided (left in d_list)
+            // follow through the ring as one more segment, and the rounds
+            // end when none are left
             extra = true;
             asm volatile("bar.sync 3, 160;" ::: "memory");
             if (S.d_cnt == 0) break;
@@ -769,7 +793,8 @@ __device__ __forceinline__ void a_consumers(const KParams& K, ASmem<G>& S, AWalk
             const int tag = sg.item_idx;
             if (tag != q_tag) {
                 q_tag = tag;
-                compute_qidx(P, S.tab, S.qi, sg.b, sg.grp, tid);
+                compute_qidx(P, S.tab, S.qi, sg.b, sg.grp, tid, first_seg);
+                first_seg = false;
                 consumer_sync();
                 qf = make_qfrag(S.qi, nh, lane);
                 consumer_sync();
@@ -783,8 +808,11 @@ __device__ __forceinline__ void a_consumers(const KParams& K, ASmem<G>& S, AWalk
             for (int i = 0; i < sg.ntiles; ++i, ++k) {
                 const int st = (int)(k % NST);
                 if (!mbar_wait_bounded(&S.full[st], (k / NST) & 1u)) {
+                    // release the copy warp's next round barrier with no
+                    // blocks left, so that it stops too
                     set_status(P, ST_TIMEOUT);
-                    if (!extra) asm volatile("bar.arrive 3, 160;" ::: "memory");
+                    S.d_cnt = 0;
+                    asm volatile("bar.arrive 3, 160;" ::: "memory");
                     return;
                 }
                 ac.mark(16);
@@ -807,7 +835,11 @@ __device__ __forceinline__ void a_consumers(const KParams& K, ASmem<G>& S, AWalk
             }
             if (nh4) score_split_end<G, true>(P, S, f, sg.b, sg.grp, sg.first, tid);
             else score_split_end<G, false>(P, S, f, sg.b, sg.grp, sg.first, tid);
-            if (ticket_add(P.tick_score + sg.item_idx, (uint32_t)sg.ntiles, (uint32_t)sg.item_tiles, &S.flag)) {
+            if (tid == 0) trace_max(P, 47);
+            const bool won =
+                ticket_add(P.tick_score + sg.item_idx, (uint32_t)sg.ntiles, (uint32_t)sg.item_tiles, &S.flag);
+            if (tid == 0) trace_max(P, 46);
+            if (won) {
                 if (tid == 0) trace_max(P, 6);
                 decide_group<G>(K, S, sg.b, sg.grp, sg.L, pb, tid);
                 consumer_sync();
@@ -822,13 +854,17 @@ __device__ __forceinline__ void a_consumers(const KParams& K, ASmem<G>& S, AWalk
             const int g = local ? S.tab.lg_group[sg.grp] : S.tab.rg_group[sg.grp];
             const uint32_t heads = local ? S.tab.lg_mask[sg.grp] : S.tab.rg_mask[sg.grp];
             const LocalGeom lg = local_geom(P, sg.L);
-            attn.begin(P, sg.b, g, lane);
+            attn.begin(P, sg.b, g, lane, first_seg && sg.type == 1);
+            first_seg = false;
             ac.mark(29);
             for (int i = 0; i < sg.ntiles; ++i, ++k) {
                 const int st = (int)(k % NST);
                 if (!mbar_wait_bounded(&S.full[st], (k / NST) & 1u)) {
+                    // release the copy warp's next round barrier with no
+                    // blocks left, so that it stops too
                     set_status(P, ST_TIMEOUT);
-                    if (!extra) asm volatile("bar.arrive 3, 160;" ::: "memory");
+                    S.d_cnt = 0;
+                    asm volatile("bar.arrive 3, 160;" ::: "memory");
                     return;
                 }
                 ac.mark(16);
@@ -859,7 +895,11 @@ __device__ __forceinline__ void a_consumers(const KParams& K, ASmem<G>& S, AWalk
             if (sg.ntiles == sg.item_tiles) {
                 split_emit<G>(S.X, heads, nullptr, out0, tid);
                 consumer_sync();
-                if (tid == 0) trace_max(P, local ? 2 : 4);
+                if (tid == 0) {
+                    if (sg.type == 2) S.d_cnt = 0;   // this round's blocks are done
+                    trace_max(P, local ? 2 : 4);
+                }
+                consumer_sync();
             } else {
                 const int c = (int)blockIdx.x;
                 float* part = P.lpart + ((int64_t)c + sg.item_idx) * G * PSTRIDE;
@@ -901,6 +941,25 @@ __device__ __forceinline__ void s_body(const KParams& K) {
     }
     int* pre_s = S.pre;
     int* pre_l = S.pre + (P.B + 1);
+    if (tid >= CONSUMERS) {
+        // the queries and the retrieval heads' indexer projections into L2
+        // first (every CTA a few 128-byte lines), ahead of the tile traffic
+        const int lane = tid - CONSUMERS;
+        const int nw = P.n_ret * (R * D * 2 / 128), nq = P.B * P.n_ret * 2, nr = P.B * P.Hq * 2;
+        for (int x = (int)blockIdx.x * 32 + lane; x < nw + nq + nr; x += (int)gridDim.x * 32) {
+            const char* a;
+            if (x < nw) {
+                a = reinterpret_cast<const char*>(P.Wq + (int64_t)P.tab.slot_head[x / 32] * R * D) + (x % 32) * 128;
+            } else if (x < nw + nq) {
+                const int y = x - nw, bs = y >> 1;
+                a = reinterpret_cast<const char*>(P.q_pre + ((int64_t)(bs / P.n_ret) * P.Hq +
+                                                             P.tab.slot_head[bs % P.n_ret]) * D) + (y & 1) * 128;
+            } else {
+                a = reinterpret_cast<const char*>(P.q_rope) + (int64_t)(x - nw - nq) * 128;
+            }
+            prefetch_l2(a);
+        }
+    }
     if (tid == 0) {
         for (int i = 0; i < NST; ++i) {
             mbar_init(&S.full[i], 1);
@@ -918,13 +977,15 @@ __device__ __forceinline__ void s_body(const KParams& K) {
     // tiles per sequence (score tiles of all retrieval groups, then local
     // tiles of all local groups), prefix-summed by warp 0
     if (tid < 32) {
-        int run_s = 0, run_l = 0;
+        int run_s = 0, run_l = 0, nvalid = 0;
         for (int b0 = 0; b0 < P.B; b0 += 32) {
             const int b = b0 + tid;
             int ns = 0, nl = 0;
+            bool okb = false;
             if (b < P.B) {
                 const int L = __ldg(P.seq_lens + b);
-                if (seq_ok(P, L)) {
+                okb = seq_ok(P, L);
+                if (okb) {
                     ns = P.n_rg * ((L + SROWS - 1) / SROWS);
                     nl = P.n_lg ? P.n_lg * local_geom(P, L).nv : 0;
                 } else if (blockIdx.x == 0) {
@@ -949,8 +1010,10 @@ __device__ __forceinline__ void s_body(const KParams& K) {
             }
             run_s += __shfl_sync(0xffffffffu, is, 31);
             run_l += __shfl_sync(0xffffffffu, il, 31);
+            nvalid += __popc(__ballot_sync(0xffffffffu, okb));
         }
         if (tid == 0) {
+            S.n_vgroups = nvalid * P.n_rg;
             pre_s[P.B] = run_s;
             pre_l[P.B] = run_l;
             S.tot_s = run_s;

@@ -199,3 +199,18 @@ def test_small_grid_long_shares(monkeypatch, cap, w, scale):
     case = synth.workload(w, scale=scale)
     fails, stats, gpu, ref = run_both(case)
     assert not fails, "\n".join(fails[:20])
+
+
+@pytest.mark.parametrize("regime", ["diffuse", "gaussian"])
+def test_full_size_1m_exact_select(regime):
+    """The 1M workload's shape (B=1, L=2^20, 8 KV x GQA 4, group 0 retrieval,
+    p=0.9, window 4096, sink 4) with a score field that no single token
+    settles: every retrieval head goes through the exact select with 2^20
+    scores (the first pass's bin range, the overflow bin and the candidate
+    caps at that length), then the block-list attention."""
+    case = synth.make_case(f"w4-1m-{regime}", B=1, Hkv=8, G=4, seq_lens=[1 << 20], ret_groups=[0], p=[0.9],
+                           window=4096, sink=4, seed=3, regimes=[regime])
+    fails, stats, gpu, ref = run_both(case)
+    assert not fails, "\n".join(fails[:20])
+    ret = np.nonzero(case.head_kind)[0]
+    assert np.all(gpu["kstar"][0, ret] > 1)          # the select ran: no head was settled by its best token

@@ -51,9 +51,10 @@ def parse():
     ap.add_argument("--no-per-workload", action="store_true",
                     help="time only the headline workload (skip the 32K, 4 x 128K and ragged lines)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--op", choices=["decode", "append", "kv_append"], default="decode",
+    ap.add_argument("--op", choices=["decode", "append", "kv_append", "prefill"], default="decode",
                     help="append: time the index-cache append instead of the decode step; "
-                         "kv_append: the KV-cache write with the index append")
+                         "kv_append: the KV-cache write with the index append; "
+                         "prefill: the prefill attention of a whole 32K prompt")
     return ap.parse_args()
 
 
@@ -547,10 +548,85 @@ def step_summary(sb, step_ms, peak, dense_ms=0.0, dense_status=0):
 OTHER_WORKLOADS = (2, 3, 5)
 
 
+def prefill_flops(T, pos, head_kind, window, sink):
+    """Multiply-add flops of a prefill chunk: 4 x 128 per attended (query,
+    key) pair (q.k and p.v), summed over heads; query t attends m + 1 keys
+    (retrieval) or its sink and window (local), m = pos + t."""
+    m = pos + np.arange(T, dtype=np.int64)
+    dense = m + 1
+    local = np.minimum(sink, m + 1) + np.maximum(0, (m + 1) - np.maximum(sink, m + 1 - window))
+    nret = int(np.sum(head_kind))
+    nloc = len(head_kind) - nret
+    return 4 * 128 * (nret * int(dense.sum()) + nloc * int(local.sum()))
+
+
+def bench_prefill(args):
+    """rtp_prefill alone: the prefill of a whole 32K prompt (B=1, 8 KV heads x
+    GQA 4, KV group 0 retrieval = 4 of 32 heads, the rest local with window
+    8192 and sink 4, the pages' prefill setting), and the same prompt with
+    every head retrieval (dense causal attention, the stand-in for the pages'
+    dense baseline).  Tensor-core bound: flops / time against the measured
+    bf16 peak.  L2 flushed before every timed call."""
+    import torch
+
+    import sparse_attention_decode_rtpurbo_b200 as rtp
+
+    dev = torch.device("cuda", 0)
+    flush_w = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    B, Hkv, G, T = 1, 8, 4, 32768 // max(1, args.scale)
+    window, sink = 8192 // max(1, args.scale), 4
+    ncap = (T + 63) // 64 * 64
+    g = torch.Generator(device=dev).manual_seed(7)
+    q = torch.randn((B, Hkv * G, T, 128), generator=g, device=dev).to(torch.bfloat16)
+    k = torch.randn((B, Hkv, ncap, 128), generator=g, device=dev).to(torch.bfloat16)
+    v = torch.randn((B, Hkv, ncap, 128), generator=g, device=dev).to(torch.bfloat16)
+    pos = torch.zeros(B, dtype=torch.int32, device=dev)
+    out = torch.empty((B, Hkv * G, T, 128), dtype=torch.bfloat16, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    dims = rtp.make_dims(B, Hkv * G, Hkv, ncap)
+    stream = torch.cuda.current_stream()
+    try:
+        peak = float(json.load(open(PEAKS_FILE))["bf16_tflops"])
+        peak_kind = "measured (MEASURED_PEAKS.json bf16_tflops, burst)"
+    except Exception:
+        peak, peak_kind = 1590.0, "fallback"
+    res = {}
+    for name, hk in (("sparse", [1] * G + [0] * (Hkv - 1) * G), ("dense", [1] * (Hkv * G))):
+        ts = []
+        for i in range(args.warmup + args.steps):
+            flush_w.zero_()
+            a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            rtp.prefill(dims, q, k, v, hk, pos, T, window, sink, out, status, stream)
+            z.record(stream)
+            z.synchronize()
+            if i >= args.warmup:
+                ts.append(a.elapsed_time(z))
+        if int(status.item()) != 0:
+            raise SystemExit(f"prefill device status {int(status.item())}")
+        t_ms = statistics.mean(ts)
+        fl = prefill_flops(T, 0, np.array(hk), window, sink)
+        tf = fl / (t_ms * 1e-3) / 1e12
+        res[name] = {"ms_per_call": t_ms, "flops": fl, "tflops": tf, "frac": tf / peak,
+                     "tokens_per_s": B * T / (t_ms * 1e-3)}
+    print(json.dumps({"metric": "prefill tokens/s (rtp_prefill, whole prompt)", "op": "prefill",
+                      "value": res["sparse"]["tokens_per_s"], "unit": "tokens/s",
+                      "config": {"batch": B, "prompt": T, "q_heads": Hkv * G, "kv_heads": Hkv, "retrieval_heads": G,
+                                 "window": window, "sink": sink, "l2": "flushed (256 MB write) before every call"},
+                      "roofline": {"bound": "tensor", "achieved": res["sparse"]["tflops"], "peak": peak,
+                                   "unit": "TFLOP/s", "frac": res["sparse"]["frac"], "peak_source": peak_kind,
+                                   "kernel": "rtp::prefill_kernel (mma.sync m16n8k16 bf16)"},
+                      "sparse": res["sparse"], "dense_all_heads_retrieval": res["dense"],
+                      "speedup_over_dense": res["dense"]["ms_per_call"] / res["sparse"]["ms_per_call"],
+                      "steps": args.steps, "warmup": args.warmup}), flush=True)
+
+
 def main():
     args = parse()
     if args.op in ("append", "kv_append"):
         return bench_append(args)
+    if args.op == "prefill":
+        return bench_prefill(args)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

@@ -379,6 +379,49 @@ rtp_status rtp_kv_append(const rtp_dims* dims, const uint16_t* k_pre, const uint
                          uint16_t* k_idx, uint16_t* k_cache, uint16_t* v_cache, uint32_t* device_status,
                          void* stream);
 
+/*
+ * rtp_prefill -- prefill attention of a chunk of num_q queries per sequence,
+ * the method's other workload: retrieval heads attend densely and causally,
+ * local heads only to their sink and sliding window.
+ *
+ * Source: review "RTPurbo" on dongryeollee1.github.io, Method: "Adaptive
+ * sparse attention" (in prefill the retrieval heads keep full attention and
+ * the local heads a sink and a sliding window); Experiments, efficiency (the
+ * prefill speedups over dense attention); aitrends.kr summary, efficiency
+ * paragraph.
+ *
+ * For every sequence b, query head h and query t < num_q, at position
+ * m = pos[b] + t (the cache already holds the keys and values of positions
+ * 0 .. pos[b] + num_q - 1, these queries' own included):
+ *   retrieval head (head_kind[h] == 1): positions [0, m];
+ *   local head     (head_kind[h] == 0): [0, min(sink, m + 1)) U
+ *                                       [max(0, m + 1 - window), m + 1);
+ *   out[b, h, t] = softmax_n(q[b, h, t] . k_n / sqrt(128)) . v_n over those
+ *   positions (the decode step's position sets at length L = m + 1).
+ *
+ *   dims      : batch, num_q_heads, num_kv_heads, head_dim 128, block_size 64,
+ *               max_seq_len and the paged fields as for rtp_decode_step
+ *               (idx_dim, workspace, debug and timing fields are not used).
+ *   q         : device bf16 [B, Hq, num_q, 128], RoPE'd queries, 16-byte aligned.
+ *   k_cache, v_cache : the decode step's caches (contiguous or paged), 16-byte aligned.
+ *   head_kind : HOST uint8 [Hq], 1 = retrieval head, 0 = local head.
+ *   pos       : device int32 [B], position of each sequence's first query.
+ *   num_q     : queries per sequence, 0 <= num_q <= max_seq_len (0: nothing is enqueued).
+ *   window, sink : the local heads' window and sink, >= 0, window + sink >= 1.
+ *   out       : device bf16 [B, Hq, num_q, 128], 16-byte aligned (round to nearest even).
+ *   device_status : optional device uint32, set to RTP_ERR_DEVICE_INPUT (if 0) for a
+ *               sequence with pos[b] < 0 or pos[b] + num_q > max_seq_len (its outputs are
+ *               not written) or a page id out of range (its outputs are unspecified), and
+ *               to RTP_ERR_TIMEOUT if a bounded wait in the kernel gave up.
+ *   stream    : the cudaStream_t the kernel is enqueued on.
+ * Cache rows no query may read are never part of the arithmetic, whatever they hold.
+ * Returns RTP_OK, or RTP_ERR_NULL / RTP_ERR_SHAPE / RTP_ERR_UNSUPPORTED before anything is
+ * enqueued, or RTP_ERR_CUDA if the tensor maps or the launch failed.
+ */
+rtp_status rtp_prefill(const rtp_dims* dims, const uint16_t* q, const uint16_t* k_cache, const uint16_t* v_cache,
+                       const uint8_t* head_kind, const int32_t* pos, int32_t num_q, int32_t window, int32_t sink,
+                       uint16_t* out, uint32_t* device_status, void* stream);
+
 /* Static string naming a status code. */
 const char* rtp_status_string(rtp_status status);
 

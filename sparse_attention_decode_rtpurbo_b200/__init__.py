@@ -15,7 +15,8 @@ from typing import Optional
 from .build import LIB as _LIB_PATH
 
 __all__ = ["RTP_OK", "RtpError", "RtpDims", "RtpDebug", "lib", "status_string", "workspace_size", "decode_step",
-           "get_status", "Step", "PHASES", "TIMING_EVENTS", "decode_step_noalloc", "NOALLOC_SCRATCH_BYTES"]
+           "get_status", "Step", "PHASES", "TIMING_EVENTS", "decode_step_noalloc", "NOALLOC_SCRATCH_BYTES",
+           "prefill"]
 
 RTP_OK = 0
 _STATUS_NAMES = {0: "RTP_OK", 1: "RTP_ERR_NULL", 2: "RTP_ERR_SHAPE", 3: "RTP_ERR_UNSUPPORTED", 4: "RTP_ERR_WORKSPACE",
@@ -90,6 +91,8 @@ def _load():
     L.rtp_kv_append.argtypes = [ctypes.POINTER(RtpDims), vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp]
     L.rtp_kv_append.restype = ctypes.c_int
     L.rtp_get_status.restype = ctypes.c_int
+    L.rtp_prefill.argtypes = [ctypes.POINTER(RtpDims), vp, vp, vp, vp, vp, i32, i32, i32, vp, vp, vp]
+    L.rtp_prefill.restype = ctypes.c_int
     L.rtp_status_string.argtypes = [ctypes.c_int]
     L.rtp_status_string.restype = ctypes.c_char_p
     return L
@@ -228,6 +231,19 @@ def kv_append(dims: RtpDims, k_pre, v_new, Wk_idx, rope_cos, rope_sin, pos, num_
                            _ptr(pos), int(num_new), _ptr(k_idx), _ptr(k_cache), _ptr(v_cache), _ptr(device_status), st)
     if rc != RTP_OK:
         raise RtpError(rc, "rtp_kv_append")
+
+
+def prefill(dims: RtpDims, q, k_cache, v_cache, head_kind, pos, num_q: int, window: int, sink: int, out,
+            device_status=None, stream=None) -> None:
+    """rtp_prefill: causal attention of num_q queries per sequence (q [B, Hq,
+    num_q, 128] bf16, RoPE'd) at positions pos[b] + t over the caches:
+    retrieval heads densely, local heads over their sink and window; out [B,
+    Hq, num_q, 128] bf16.  head_kind is a host sequence of 0/1."""
+    st = 0 if stream is None else (stream if isinstance(stream, int) else stream.cuda_stream)
+    rc = lib.rtp_prefill(ctypes.byref(dims), _ptr(q), _ptr(k_cache), _ptr(v_cache), _head_kind_buf(head_kind),
+                         _ptr(pos), int(num_q), int(window), int(sink), _ptr(out), _ptr(device_status), st)
+    if rc != RTP_OK:
+        raise RtpError(rc, "rtp_prefill")
 
 
 def get_status(dims: RtpDims, stream=None) -> int:

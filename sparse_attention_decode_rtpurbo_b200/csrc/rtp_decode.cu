@@ -17,6 +17,7 @@
 #include "../../include/rtp_decode.h"
 #include "rtp_retrieve.cuh"
 #include "rtp_append.cuh"
+#include "rtp_prefill.cuh"
 
 namespace rtp {
 
@@ -181,7 +182,7 @@ struct OccCache {
     int occ[16];
     int n = 0;
 };
-static int occupancy(const void* fn, size_t smem) {
+static int occupancy(const void* fn, size_t smem, int threads = THREADS) {
     static OccCache c;
     int dev = 0, maxs = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 0;
@@ -195,7 +196,7 @@ static int occupancy(const void* fn, size_t smem) {
     if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, maxs) != cudaSuccess) return 0;
     cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, THREADS, smem) != cudaSuccess) return 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, threads, smem) != cudaSuccess) return 0;
     const int slot = c.n < 16 ? c.n++ : 15;
     c.fn[slot] = fn;
     c.smem[slot] = smem;
@@ -673,6 +674,89 @@ extern "C" rtp_status rtp_kv_append(const rtp_dims* d, const uint16_t* k_pre, co
     if (!k_cache) return RTP_ERR_NULL;
     return append_impl(d, k_pre, v_new, Wk_idx, rope_cos, rope_sin, pos, num_new, k_idx, k_cache, v_cache,
                        device_status, stream);
+}
+
+// ---------------------------------------------------------------------------
+// prefill attention of a chunk of queries
+// ---------------------------------------------------------------------------
+extern "C" rtp_status rtp_prefill(const rtp_dims* d, const uint16_t* q, const uint16_t* k_cache,
+                                  const uint16_t* v_cache, const uint8_t* head_kind, const int32_t* pos,
+                                  int32_t num_q, int32_t window, int32_t sink, uint16_t* out,
+                                  uint32_t* device_status, void* stream) {
+    if (!d || !head_kind) return RTP_ERR_NULL;
+    if (d->head_dim != D || d->block_size != BLK) return RTP_ERR_UNSUPPORTED;
+    if (d->batch < 1 || d->num_q_heads < 1 || d->num_kv_heads < 1 || num_q < 0) return RTP_ERR_SHAPE;
+    if (d->num_q_heads % d->num_kv_heads) return RTP_ERR_SHAPE;
+    const int G = d->num_q_heads / d->num_kv_heads;
+    if (G != 1 && G != 2 && G != 4 && G != 8) return RTP_ERR_UNSUPPORTED;
+    if (d->num_q_heads > MAX_HQ || d->num_kv_heads > MAX_HKV || d->batch > MAX_B) return RTP_ERR_UNSUPPORTED;
+    if (d->max_seq_len < BLK || d->max_seq_len % BLK || num_q > d->max_seq_len) return RTP_ERR_SHAPE;
+    if (window < 0 || sink < 0 || (int64_t)window + sink < 1) return RTP_ERR_SHAPE;
+    if (d->block_table) {
+        if (d->max_blocks_per_seq < 1 || d->num_pages < 1) return RTP_ERR_SHAPE;
+        if ((int64_t)d->max_blocks_per_seq * BLK != d->max_seq_len) return RTP_ERR_SHAPE;
+        if ((int64_t)d->num_pages * d->num_kv_heads * BLK >= (1ll << 31)) return RTP_ERR_UNSUPPORTED;
+    } else if ((int64_t)d->batch * d->num_kv_heads * d->max_seq_len >= (1ll << 31)) {
+        return RTP_ERR_UNSUPPORTED;   // TMA row coordinates are 32-bit
+    }
+    if (num_q == 0) return RTP_OK;
+    if (!q || !k_cache || !v_cache || !pos || !out) return RTP_ERR_NULL;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out)) return RTP_ERR_UNSUPPORTED;
+    PrefillK K;
+    memset(&K, 0, sizeof(K));
+    PrefillParams& P = K.P;
+    P.B = d->batch;
+    P.Hq = d->num_q_heads;
+    P.Hkv = d->num_kv_heads;
+    P.G = G;
+    P.Ncap = d->max_seq_len;
+    P.mbps = d->block_table ? d->max_blocks_per_seq : 0;
+    P.num_pages = d->block_table ? d->num_pages : 0;
+    P.T = num_q;
+    P.window = window;
+    P.sink = sink;
+    P.nt16 = (num_q + 15) / 16;
+    // the (KV group, head kind) sets: retrieval heads first, then local heads, per group
+    int cta = 0;
+    for (int g = 0; g < P.Hkv; ++g)
+        for (int kind = 1; kind >= 0; --kind) {
+            int nh = 0;
+            uint8_t heads[MAX_G];
+            for (int i = 0; i < G; ++i) {
+                const uint8_t k = head_kind[g * G + i];
+                if (k > 1) return RTP_ERR_SHAPE;
+                if (k == kind) heads[nh++] = (uint8_t)i;
+            }
+            if (!nh) continue;
+            const int s = P.n_sets++;
+            P.set_g[s] = (uint8_t)g;
+            P.set_kind[s] = (uint8_t)kind;
+            P.set_nh[s] = (uint8_t)nh;
+            memcpy(P.set_heads[s], heads, nh);
+            P.set_cta0[s] = cta;
+            cta += (int)(((int64_t)nh * P.nt16 + PF_UNITS - 1) / PF_UNITS);
+        }
+    P.set_cta0[P.n_sets] = cta;
+    P.cta_per_b = cta;
+    const int64_t grid = (int64_t)P.B * cta;
+    if (grid > 0x7FFFFFFF) return RTP_ERR_UNSUPPORTED;
+    P.q = q;
+    P.pos = pos;
+    P.block_table = d->block_table;
+    P.out = out;
+    P.status = device_status;
+    const long long rows = d->block_table ? (long long)d->num_pages * P.Hkv * BLK : (long long)P.B * P.Hkv * P.Ncap;
+    if (!encode_cache_map(&K.tmk, k_cache, rows) || !encode_cache_map(&K.tmv, v_cache, rows)) {
+        report(cudaErrorInvalidValue, "prefill K/V tensor map");
+        return RTP_ERR_CUDA;
+    }
+    const size_t smem = sizeof(PfSmem);
+    if (occupancy((const void*)prefill_kernel, smem, PF_THREADS) < 1) {
+        report(cudaErrorInvalidConfiguration, "prefill kernel occupancy");
+        return RTP_ERR_CUDA;
+    }
+    prefill_kernel<<<(unsigned)grid, PF_THREADS, smem, (cudaStream_t)stream>>>(K);
+    return report(cudaGetLastError(), "prefill launch") == cudaSuccess ? RTP_OK : RTP_ERR_CUDA;
 }
 
 extern "C" const char* rtp_status_string(rtp_status status) {

@@ -196,6 +196,38 @@ def test_kv_append_host_side_checks():
     assert call(bad) == 3
 
 
+def test_prefill_host_side_checks():
+    """rtp_prefill: bad arguments are refused before any CUDA call."""
+    fake = 4096   # never dereferenced: every call below returns first
+    d = dims()
+    HK = rtp._head_kind_buf([1, 0, 0, 1, 1, 0, 0, 1][:d.num_q_heads] + [0] * max(0, d.num_q_heads - 8))
+
+    def call(dd, q=fake, kc=fake, vc=fake, hk=HK, pos=fake, n=16, window=64, sink=4, out=fake):
+        return rtp.lib.rtp_prefill(ctypes.byref(dd) if dd is not None else None, q, kc, vc, hk, pos, n, window,
+                                   sink, out, None, None)
+
+    assert call(None) == 1                           # NULL dims
+    assert call(d, hk=None) == 1                     # NULL head split
+    assert call(d, q=None) == 1
+    assert call(d, kc=None) == 1
+    assert call(d, pos=None) == 1
+    assert call(d, out=None) == 1
+    assert call(d, n=0) == 0                         # no queries: nothing to do
+    assert call(d, n=-1) == 2
+    assert call(d, n=d.max_seq_len + 1) == 2         # more queries than the capacity
+    assert call(d, window=0, sink=0) == 2            # local heads would attend to nothing
+    assert call(d, window=-1) == 2
+    assert call(d, q=fake + 8) == 3                  # 16-byte alignment
+    assert call(d, vc=fake + 2) == 3
+    assert call(d, out=fake + 4) == 3
+    bad = dims()
+    bad.head_dim = 64
+    assert call(bad) == 3
+    bad = dims()
+    bad.num_kv_heads = 3                             # Hq % Hkv != 0
+    assert call(bad) == 2
+
+
 def test_binding_refuses_host_and_strided_tensors():
     """The binding passes tensors by address: a host tensor or a strided view
     is refused before the library is called."""

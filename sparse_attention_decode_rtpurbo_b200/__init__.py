@@ -12,7 +12,12 @@ import ctypes
 import os
 from typing import Optional
 
-from .build import LIB as _LIB_PATH
+from .build import LIB as _BUILT_LIB
+
+# RTP_LIBRARY=<path>: load another build of the library (a comparison build,
+# e.g. the one whose attention tiles run on the FMA pipe); default: the
+# package's librtp.so
+_LIB_PATH = os.environ.get("RTP_LIBRARY") or _BUILT_LIB
 
 __all__ = ["RTP_OK", "RtpError", "RtpDims", "RtpDebug", "lib", "status_string", "workspace_size", "decode_step",
            "get_status", "Step", "PHASES", "TIMING_EVENTS", "decode_step_noalloc", "NOALLOC_SCRATCH_BYTES",

@@ -18,21 +18,29 @@ def _inputs():
     return files
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and os.path.exists(LIB):
+def build(force: bool = False, verbose: bool = False, defines=(), out: str = LIB) -> str:
+    """Build `out` (default: the package's librtp.so) unless it is newer than
+    every source.  `defines`: extra preprocessor names, e.g. RTP_ATTN_FMA for
+    the variant whose attention tiles run on the FMA pipe (a comparison build:
+    give it its own `out` and load it with RTP_LIBRARY=<path>)."""
+    if not force and os.path.exists(out):
         newest = max(os.path.getmtime(f) for f in _inputs())
-        if os.path.getmtime(LIB) >= newest:
-            return LIB
+        if os.path.getmtime(out) >= newest:
+            return out
     nvcc = os.environ.get("NVCC", "nvcc")
-    tmp = LIB + f".{os.getpid()}.tmp"
-    cmd = [nvcc, *NVCC_FLAGS, *[os.path.join(SRC_DIR, s) for s in SOURCES], "-o", tmp]
+    tmp = out + f".{os.getpid()}.tmp"
+    cmd = [nvcc, *NVCC_FLAGS, *[f"-D{d}" for d in defines], *[os.path.join(SRC_DIR, s) for s in SOURCES], "-o", tmp]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
         print(" ".join(cmd), file=sys.stderr)
     subprocess.check_call(cmd)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, out)
+    return out
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))
+    # python -m sparse_attention_decode_rtpurbo_b200.build [--force] [-v] [--define NAME ...] [--out PATH]
+    argv = sys.argv[1:]
+    defs = [argv[i + 1] for i, a in enumerate(argv) if a == "--define"]
+    out = argv[argv.index("--out") + 1] if "--out" in argv else LIB
+    print(build(force="--force" in argv, verbose="-v" in argv, defines=defs, out=os.path.abspath(out)))

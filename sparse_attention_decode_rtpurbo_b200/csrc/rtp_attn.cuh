@@ -19,6 +19,9 @@ struct AttnScratch {
     alignas(16) float red[4][G][D];   // per-warp unnormalised outputs
     float wm[4][G], wl[4][G];         // per-warp running max (log2 units) and sum
     float cm[G], cden[G];             // combine: max and denominator per head
+#ifdef RTP_ATTN_FMA
+    alignas(16) uint16_t qf[4][G][D];   // FmaAttn: each compute warp's copy of its group's queries (bf16)
+#endif
 };
 
 // Address of 16-byte chunk c (0..15, 8 dims each) of row `row` of a 64 x 128
@@ -44,7 +47,7 @@ struct MmaAttn {
     float m, l;          // head lane/4: running max of the scaled logits, this thread's share of the sum
     int q_tag;
 
-    __device__ __forceinline__ void init() { q_tag = -1; }
+    __device__ __forceinline__ void init(uint32_t = 0u) { q_tag = -1; }
 
     // arrive: the CTA's first segment (named barrier 4 lets the copy warp
     // issue the first tile once the query loads are on their way)
@@ -181,6 +184,151 @@ struct MmaAttn {
         }
     }
 };
+
+#ifdef RTP_ATTN_FMA
+__device__ __forceinline__ uint2 lds64(uint32_t addr) {
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+    return v;
+}
+
+// The same per-warp split attention on the FP32 FMA pipe instead of the
+// tensor cores (a build with RTP_ATTN_FMA defined), kept to compare the two
+// on the same kernels: scores with lane = (token lane % 16, half of the 128
+// dims), then P V with lane = 4 output dims of every head.  Same inputs,
+// masks, online softmax (log2 domain) and per-warp state as MmaAttn, so
+// split_emit and combine_splits serve both.
+template <int G>
+struct FmaAttn {
+    float o[G][4];   // dims 4 lane .. 4 lane + 3 of every head
+    float m[G], l[G];
+    int q_tag;
+    uint32_t qs;     // this warp's query copy in shared memory (bf16 [G][128])
+
+    __device__ __forceinline__ void init(uint32_t q_smem) {
+        q_tag = -1;
+        qs = q_smem;
+    }
+
+    __device__ __forceinline__ void begin(const Params& P, int b, int g, int lane, bool arrive = false) {
+        const int tag = b * P.Hkv + g;
+        if (tag != q_tag) {
+            q_tag = tag;
+            __syncwarp();   // (the previous segment's reads of the copy are done)
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                const uint2 v = __ldg(reinterpret_cast<const uint2*>(P.q_rope + ((int64_t)b * P.Hq + g * G + h) * D) + lane);
+                asm volatile("st.shared.v2.u32 [%0], {%1,%2};" ::"r"(qs + (uint32_t)(h * D + 4 * lane) * 2), "r"(v.x),
+                             "r"(v.y)
+                             : "memory");
+            }
+            __syncwarp();
+        }
+        if (arrive) asm volatile("bar.arrive 4, 160;" ::: "memory");
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            m[h] = -INFINITY;
+            l[h] = 0.f;
+            o[h][0] = o[h][1] = o[h][2] = o[h][3] = 0.f;
+        }
+    }
+
+    __device__ __forceinline__ bool tile(uint32_t K, uint32_t V, int warp, int lane, int n0, int nvalid,
+                                         uint32_t hmask, bool local, int s_end, int w_lo) {
+        const int r0 = warp * 16;
+        const int rl = r0 + (lane & 15), nl = n0 + rl;
+        const bool rd = rl < nvalid && (!local || nl < s_end || nl >= w_lo);
+        const uint32_t bad = ~__ballot_sync(0xffffffffu, rd) & 0xFFFFu;
+        if (bad) {
+            const int tr = lane >> 1;
+            if ((bad >> tr) & 1u) {
+                const uint32_t row = V + (uint32_t)((lane & 1) * 8192 + (r0 + tr) * 128);
+#pragma unroll
+                for (int c = 0; c < 8; ++c) sts128_zero(row + c * 16);
+            }
+            __syncwarp();
+        }
+        // partial dots over this lane's 64 dims, every head
+        const int hf = lane >> 4;
+        float acc[G];
+#pragma unroll
+        for (int h = 0; h < G; ++h) acc[h] = 0.f;
+#pragma unroll 2
+        for (int c = 0; c < 8; ++c) {
+            const uint4 kv = lds128(sw_addr(K, rl, 8 * hf + c));
+            const uint32_t ku[4] = {kv.x, kv.y, kv.z, kv.w};
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                const uint4 qv = lds128(qs + (uint32_t)(h * D + (8 * hf + c) * 8) * 2);
+                const uint32_t qu[4] = {qv.x, qv.y, qv.z, qv.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    acc[h] = fmaf(bf_lo(ku[j]), bf_lo(qu[j]), acc[h]);
+                    acc[h] = fmaf(bf_hi(ku[j]), bf_hi(qu[j]), acc[h]);
+                }
+            }
+        }
+        constexpr float SCALE = 0.08838834764831845f * 1.4426950408889634f;   // log2(e)/sqrt(128)
+        float pr[G];
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            const float sc = acc[h] + __shfl_xor_sync(0xffffffffu, acc[h], 16);
+            const float x = (rd && ((hmask >> h) & 1u)) ? sc * SCALE : -INFINITY;
+            float mt = x;
+#pragma unroll
+            for (int ofs = 8; ofs > 0; ofs >>= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, ofs));
+            const float mn = fmaxf(m[h], mt);
+            const float alpha = mn == -INFINITY ? 1.f : ex2_approx(m[h] - mn);
+            const float p = mn == -INFINITY ? 0.f : ex2_approx(x - mn);
+            float ps = p;
+#pragma unroll
+            for (int ofs = 8; ofs > 0; ofs >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, ofs);
+            l[h] = l[h] * alpha + ps;
+            m[h] = mn;
+            pr[h] = p;
+            o[h][0] *= alpha;
+            o[h][1] *= alpha;
+            o[h][2] *= alpha;
+            o[h][3] *= alpha;
+        }
+        // O += P V over the warp's 16 tokens: lane holds dims 4 lane .. 4 lane + 3
+#pragma unroll 4
+        for (int r = 0; r < 16; ++r) {
+            const uint2 vv = lds64(sw_addr(V, r0 + r, lane >> 1) + (uint32_t)(lane & 1) * 8u);
+            const float v0 = bf_lo(vv.x), v1 = bf_hi(vv.x), v2 = bf_lo(vv.y), v3 = bf_hi(vv.y);
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                const float p = __shfl_sync(0xffffffffu, pr[h], r);
+                o[h][0] = fmaf(p, v0, o[h][0]);
+                o[h][1] = fmaf(p, v1, o[h][1]);
+                o[h][2] = fmaf(p, v2, o[h][2]);
+                o[h][3] = fmaf(p, v3, o[h][3]);
+            }
+        }
+        return bad != 0;
+    }
+
+    __device__ __forceinline__ void finish(AttnScratch<G>& X, int warp, int lane) {
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            if (lane == 0) {
+                X.wm[warp][h] = m[h];
+                X.wl[warp][h] = l[h];
+            }
+            *reinterpret_cast<float4*>(&X.red[warp][h][4 * lane]) = make_float4(o[h][0], o[h][1], o[h][2], o[h][3]);
+        }
+    }
+};
+template <int G>
+using Attn = FmaAttn<G>;
+template <int G>
+__device__ __forceinline__ uint32_t attn_q_smem(AttnScratch<G>& X, int warp) { return smem_u32(&X.qf[warp][0][0]); }
+#else
+template <int G>
+using Attn = MmaAttn<G>;
+template <int G>
+__device__ __forceinline__ uint32_t attn_q_smem(AttnScratch<G>&, int) { return 0u; }
+#endif
 
 // Merge the four warps of a split (after finish + consumer_sync): each
 // consumer thread owns one of the 128 dims.  Writes the split's partial

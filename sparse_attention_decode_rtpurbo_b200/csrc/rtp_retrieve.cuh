@@ -1049,8 +1049,8 @@ __device__ __forceinline__ void r_consume_attn(const KParams& K, BSmem<G>& S, ui
     constexpr int NST = BSmem<G>::NST;
     const Params& P = K.P;
     const int warp = tid >> 5, lane = tid & 31;
-    MmaAttn<G> attn;
-    attn.init();
+    Attn<G> attn;
+    attn.init(attn_q_smem<G>(S.X, warp));
     Acct ac;
     ac.init(P, S.acct, tid == 0);
     while (true) {

@@ -769,8 +769,8 @@ __device__ __forceinline__ void a_consumers(const KParams& K, ASmem<G>& S, AWalk
     uint32_t k = 0;
     int q_tag = -1;
     QFrag qf;
-    MmaAttn<G> attn;
-    attn.init();
+    Attn<G> attn;
+    attn.init(attn_q_smem<G>(S.X, warp));
     Acct ac;
     ac.init(P, S.acct, tid == 0);
     bool first_data = true;

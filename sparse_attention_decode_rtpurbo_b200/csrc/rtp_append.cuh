@@ -7,16 +7,18 @@
 // retrieval key k^idx_n = W^K k^pre_n, a rank-16 projection kept as a bf16
 // cache); aitrends.kr summary, item 2 (low-rank retrieval routing).
 //
-// One thread per (token, 4 output rows): the 128 products of two bf16 values
-// are exact in fp64 and each row's are summed in index order, then rounded
-// once to bf16 (round to nearest even) -- the same value whichever thread or
-// launch computes it; the four rows' chains run side by side.  The work is
-// a few KB per token: bound by reading k_pre (256 B per token and KV head)
-// and the fp64 pipe, far below any tensor-core shape.
+// One thread per token and KV head, all 16 output rows: the 128 products of
+// two bf16 values are exact in fp64 and each row's are summed in index
+// order, then rounded once to bf16 (round to nearest even) -- the same value
+// whichever thread or launch computes it.  The 16 rows' chains run side by
+// side (a chain of 128 dependent fp64 fused multiply-adds is the latency
+// that bounds the kernel; 16 of them in flight per thread hide it).  The work
+// is a few KB per token: bound by reading k_pre (256 B per token and KV
+// head) and the fp64 pipe, far below any tensor-core shape.
 //
-// The KV-cache write (kv_append) runs in the same threads: the thread of
-// output rows 4q .. 4q+3 also rotates the key pairs (i, i + 64) for
-// i in [16q, 16q + 16) by the caller's angle table,
+// The KV-cache write (kv_append) runs in the same threads: for each quarter
+// q the thread rotates the key pairs (i, i + 64) for i in [16q, 16q + 16) by
+// the caller's angle table,
 //     y_i = k_i cos - k_{i+64} sin,   y_{i+64} = k_{i+64} cos + k_i sin,
 // each the fp64 fused multiply-add of one exact product onto the other
 // (a bf16 times an fp32 value is exact in fp64), rounded to bf16, and copies
@@ -49,7 +51,7 @@ struct AppendParams {
 };
 
 constexpr int APPEND_THREADS = 256;
-constexpr int APPEND_ROWS = 4;   // output rows per thread: independent fp64 chains over shared k_pre loads
+constexpr int APPEND_ROWS = R;   // output rows per thread: independent fp64 chains over shared k_pre loads
 
 // KV = false: the index-cache append alone; KV = true: with the KV-cache write.
 template <bool KV>
@@ -58,7 +60,7 @@ __global__ void __launch_bounds__(APPEND_THREADS) append_kernel(const __grid_con
     const int64_t i = (int64_t)blockIdx.x * APPEND_THREADS + threadIdx.x;
     const int64_t total = (int64_t)A.B * A.Hkv * A.T * RQ;
     if (i >= total) return;
-    const int r0 = (int)(i % RQ) * APPEND_ROWS;   // rows r0 .. r0 + 3
+    const int r0 = (int)(i % RQ) * APPEND_ROWS;   // rows r0 .. r0 + APPEND_ROWS - 1
     const int64_t tok = i / RQ;                  // (b, g, t) in row-major order
     const int t = (int)(tok % A.T);
     const int g = (int)((tok / A.T) % A.Hkv);
@@ -104,10 +106,13 @@ __global__ void __launch_bounds__(APPEND_THREADS) append_kernel(const __grid_con
     uint16_t o[APPEND_ROWS];
 #pragma unroll
     for (int q = 0; q < APPEND_ROWS; ++q) o[q] = __bfloat16_as_ushort(__double2bfloat16(acc[q]));
-    *reinterpret_cast<uint2*>(A.k_idx + row * R + r0) =
-        make_uint2((uint32_t)o[0] | ((uint32_t)o[1] << 16), (uint32_t)o[2] | ((uint32_t)o[3] << 16));
+#pragma unroll
+    for (int q = 0; q < APPEND_ROWS; q += 4)   // 8-byte stores: the cache is only 8-byte aligned
+        *reinterpret_cast<uint2*>(A.k_idx + row * R + r0 + q) =
+            make_uint2((uint32_t)o[q] | ((uint32_t)o[q + 1] << 16), (uint32_t)o[q + 2] | ((uint32_t)o[q + 3] << 16));
     if constexpr (KV) {
-        const int q = r0 / APPEND_ROWS;             // quarter: pairs 16q .. 16q+15, value bytes 64q .. 64q+63
+#pragma unroll 1
+      for (int q = 0; q < 4; ++q) {                 // quarter: pairs 16q .. 16q+15, value bytes 64q .. 64q+63
         const int64_t n16 = n * (D / 2);            // the angle table's row n (64 floats)
         const float4* cs = reinterpret_cast<const float4*>(A.rope_cos + n16) + q * 4;
         const float4* sn = reinterpret_cast<const float4*>(A.rope_sin + n16) + q * 4;
@@ -142,6 +147,7 @@ __global__ void __launch_bounds__(APPEND_THREADS) append_kernel(const __grid_con
         uint4* vd = reinterpret_cast<uint4*>(A.v_cache + row * D) + q * 4;
 #pragma unroll
         for (int c = 0; c < 4; ++c) vd[c] = __ldg(vs + c);
+      }
     }
 }
 

@@ -591,6 +591,7 @@ def bench_prefill(args):
     except Exception:
         peak, peak_kind = 1590.0, "fallback"
     res = {}
+    kernel = "tcgen05 (tensor memory)" if os.environ.get("RTP_PREFILL_TC") == "1" else "mma.sync m16n8k16 bf16"
     for name, hk in (("sparse", [1] * G + [0] * (Hkv - 1) * G), ("dense", [1] * (Hkv * G))):
         ts = []
         for i in range(args.warmup + args.steps):
@@ -615,7 +616,7 @@ def bench_prefill(args):
                                  "window": window, "sink": sink, "l2": "flushed (256 MB write) before every call"},
                       "roofline": {"bound": "tensor", "achieved": res["sparse"]["tflops"], "peak": peak,
                                    "unit": "TFLOP/s", "frac": res["sparse"]["frac"], "peak_source": peak_kind,
-                                   "kernel": "rtp::prefill_kernel (mma.sync m16n8k16 bf16)"},
+                                   "kernel": f"rtp_prefill: {kernel}"},
                       "sparse": res["sparse"], "dense_all_heads_retrieval": res["dense"],
                       "speedup_over_dense": res["dense"]["ms_per_call"] / res["sparse"]["ms_per_call"],
                       "steps": args.steps, "warmup": args.warmup}), flush=True)

@@ -18,6 +18,7 @@
 #include "rtp_retrieve.cuh"
 #include "rtp_append.cuh"
 #include "rtp_prefill.cuh"
+#include "rtp_prefill_tc.cuh"
 
 namespace rtp {
 
@@ -716,6 +717,11 @@ extern "C" rtp_status rtp_prefill(const rtp_dims* d, const uint16_t* q, const ui
     P.window = window;
     P.sink = sink;
     P.nt16 = (num_q + 15) / 16;
+    // RTP_PREFILL_TC=1 (read at every call): the tcgen05 kernel, eight units
+    // per CTA; otherwise the warp-MMA kernel, four
+    const char* tcv = getenv("RTP_PREFILL_TC");
+    const bool tc = tcv && atoi(tcv) == 1;
+    const int units = tc ? PT_UNITS : PF_UNITS;
     // the (KV group, head kind) sets: retrieval heads first, then local heads, per group
     int cta = 0;
     for (int g = 0; g < P.Hkv; ++g)
@@ -734,7 +740,7 @@ extern "C" rtp_status rtp_prefill(const rtp_dims* d, const uint16_t* q, const ui
             P.set_nh[s] = (uint8_t)nh;
             memcpy(P.set_heads[s], heads, nh);
             P.set_cta0[s] = cta;
-            cta += (int)(((int64_t)nh * P.nt16 + PF_UNITS - 1) / PF_UNITS);
+            cta += (int)(((int64_t)nh * P.nt16 + units - 1) / units);
         }
     P.set_cta0[P.n_sets] = cta;
     P.cta_per_b = cta;
@@ -749,6 +755,19 @@ extern "C" rtp_status rtp_prefill(const rtp_dims* d, const uint16_t* q, const ui
     if (!encode_cache_map(&K.tmk, k_cache, rows) || !encode_cache_map(&K.tmv, v_cache, rows)) {
         report(cudaErrorInvalidValue, "prefill K/V tensor map");
         return RTP_ERR_CUDA;
+    }
+    if (tc) {
+        PrefillTcK T;
+        T.k_cache = k_cache;
+        T.v_cache = v_cache;
+        T.P = P;
+        const size_t smem = sizeof(PtSmem);
+        if (occupancy((const void*)prefill_tc_kernel, smem, PT_THREADS) < 1) {
+            report(cudaErrorInvalidConfiguration, "prefill tcgen05 kernel occupancy");
+            return RTP_ERR_CUDA;
+        }
+        prefill_tc_kernel<<<(unsigned)grid, PT_THREADS, smem, (cudaStream_t)stream>>>(T);
+        return report(cudaGetLastError(), "prefill tcgen05 launch") == cudaSuccess ? RTP_OK : RTP_ERR_CUDA;
     }
     const size_t smem = sizeof(PfSmem);
     if (occupancy((const void*)prefill_kernel, smem, PF_THREADS) < 1) {

@@ -1,5 +1,5 @@
-"""GPU parity of the prefill attention (rtp_prefill) against the fp64 oracle's
-prefill: query t of sequence b at position pos[b] + t attends causally, densely
+"""GPU parity of the prefill attention (rtp_prefill, both of its kernels)
+against the fp64 oracle's prefill: query t of sequence b at position pos[b] + t attends causally, densely
 for retrieval heads and over the sink and window for local heads.  Outputs
 within 4e-3 + 1e-2 |ref|, element by element; cache rows at or beyond each
 sequence's length are NaN, so a stray read shows up as a non-finite output."""
@@ -18,6 +18,17 @@ if not torch.cuda.is_available():
     pytest.skip("needs a CUDA GPU", allow_module_level=True)
 
 from synth.torch_io import bf16_tensor  # noqa: E402
+
+
+@pytest.fixture(params=["warp-mma", "tcgen05"], autouse=True)
+def prefill_kernel(request, monkeypatch):
+    """Every case runs on both prefill kernels: the warp-level MMA one and the
+    tcgen05 one with its accumulators in tensor memory (RTP_PREFILL_TC=1)."""
+    if request.param == "tcgen05":
+        monkeypatch.setenv("RTP_PREFILL_TC", "1")
+    else:
+        monkeypatch.delenv("RTP_PREFILL_TC", raising=False)
+    return request.param
 
 
 def run_prefill(case, q, pos, expect_status=0):

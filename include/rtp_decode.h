@@ -415,6 +415,9 @@ rtp_status rtp_kv_append(const rtp_dims* dims, const uint16_t* k_pre, const uint
  *               to RTP_ERR_TIMEOUT if a bounded wait in the kernel gave up.
  *   stream    : the cudaStream_t the kernel is enqueued on.
  * Cache rows no query may read are never part of the arithmetic, whatever they hold.
+ * Kernel: tcgen05 MMAs with tensor-memory accumulators and TMA-fed K/V tiles;
+ * RTP_PREFILL_TC=0 in the environment (read at every call) selects the
+ * warp-level MMA kernel instead (the same results within rounding).
  * Returns RTP_OK, or RTP_ERR_NULL / RTP_ERR_SHAPE / RTP_ERR_UNSUPPORTED before anything is
  * enqueued, or RTP_ERR_CUDA if the tensor maps or the launch failed.
  */

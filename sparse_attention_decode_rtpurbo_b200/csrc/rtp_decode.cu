@@ -717,10 +717,10 @@ extern "C" rtp_status rtp_prefill(const rtp_dims* d, const uint16_t* q, const ui
     P.window = window;
     P.sink = sink;
     P.nt16 = (num_q + 15) / 16;
-    // RTP_PREFILL_TC=1 (read at every call): the tcgen05 kernel, eight units
-    // per CTA; otherwise the warp-MMA kernel, four
+    // the tcgen05 kernel, eight units per CTA; RTP_PREFILL_TC=0 (read at every
+    // call): the warp-MMA kernel, four
     const char* tcv = getenv("RTP_PREFILL_TC");
-    const bool tc = tcv && atoi(tcv) == 1;
+    const bool tc = !(tcv && atoi(tcv) == 0);
     const int units = tc ? PT_UNITS : PF_UNITS;
     // the (KV group, head kind) sets: retrieval heads first, then local heads, per group
     int cta = 0;
@@ -758,8 +758,8 @@ extern "C" rtp_status rtp_prefill(const rtp_dims* d, const uint16_t* q, const ui
     }
     if (tc) {
         PrefillTcK T;
-        T.k_cache = k_cache;
-        T.v_cache = v_cache;
+        T.tmk = K.tmk;
+        T.tmv = K.tmv;
         T.P = P;
         const size_t smem = sizeof(PtSmem);
         if (occupancy((const void*)prefill_tc_kernel, smem, PT_THREADS) < 1) {

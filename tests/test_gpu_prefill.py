@@ -22,12 +22,13 @@ from synth.torch_io import bf16_tensor  # noqa: E402
 
 @pytest.fixture(params=["warp-mma", "tcgen05"], autouse=True)
 def prefill_kernel(request, monkeypatch):
-    """Every case runs on both prefill kernels: the warp-level MMA one and the
-    tcgen05 one with its accumulators in tensor memory (RTP_PREFILL_TC=1)."""
+    """Every case runs on both prefill kernels: the tcgen05 one with its
+    accumulators in tensor memory (the default) and the warp-level MMA one
+    (RTP_PREFILL_TC=0)."""
     if request.param == "tcgen05":
-        monkeypatch.setenv("RTP_PREFILL_TC", "1")
-    else:
         monkeypatch.delenv("RTP_PREFILL_TC", raising=False)
+    else:
+        monkeypatch.setenv("RTP_PREFILL_TC", "0")
     return request.param
 
 

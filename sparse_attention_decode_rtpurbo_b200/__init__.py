@@ -42,15 +42,15 @@ class RtpDebug(ctypes.Structure):
 
 
 TRACE_EVENTS = ["start", "select_done", "local_done", "lists_ready", "retrieval_done", "end", "select_start",
-                "stream_work_start", "radix1", "radix2", "radix3", "radix4", "mark", "ret_kernel_start", "pass0_hist",
-                "attn_start"]
+                "stream_work_start", "unused_8", "unused_9", "unused_10", "unused_11", "select_units_done",
+                "ret_kernel_start", "select_bins_done", "attn_start"]
 # debug sums (slots 16..): SM cycles of one thread per CTA by category, counts,
 # and the latest %globaltimer of two events
 TRACE_SUMS = ["a_cyc_wait", "a_cyc_score", "a_cyc_attn", "a_n_score", "a_n_attn", "a_cyc_score_begin",
-              "a_first_data", "a_consumers_done", "b_cyc_bins", "b_n_pass_tiles", "b_cyc_compact",
-              "b_cyc_mark", "a_cyc_score_end", "a_cyc_local_begin", "a_cyc_local_end", "b_cyc_grid_sync",
-              "b_attn_wait", "b_attn_tile", "b_attn_end", "b_n_attn", "b_prod_wait", "b_cyc_digit", "b_cyc_local_select",
-              "b_cyc_blist", "b_cyc_res_wait", "t_unused_41", "t_unused_42", "t_decide_reduced",
+              "a_first_data", "a_consumers_done", "unused_24", "unused_25", "unused_26",
+              "unused_27", "a_cyc_score_end", "a_cyc_local_begin", "a_cyc_local_end", "b_cyc_grid_sync",
+              "b_attn_wait", "b_attn_tile", "b_attn_end", "b_n_attn", "b_prod_wait", "b_cyc_sel_bins",
+              "b_cyc_sel_units", "b_cyc_sel_finish", "unused_40", "t_unused_41", "t_unused_42", "t_decide_reduced",
               "t_decide_modes", "t_unused_45", "t_split_ticketed", "t_split_reduced"]
 # TRACE_SUMS entries that are %globaltimer maxima (events), not cycle sums
 TRACE_SUM_EVENTS = ("a_first_data", "a_consumers_done") + tuple(n for n in TRACE_SUMS if n.startswith("t_"))

@@ -53,13 +53,11 @@ struct HeadState {
 struct Sync {
     uint32_t n_radix_heads;    // heads needing the exact select (list in rlist)
     uint32_t n_radix_groups;   // (b, group) pairs holding such heads (list in rglist)
-    uint32_t any_ties;         // some radix head takes only part of its threshold ties
     uint32_t barrier;          // grid barrier arrivals of the retrieval kernel
     uint32_t exit_count;
     uint32_t kb_work;          // groups left to the retrieval kernel (a select, or blocks to attend)
-    uint32_t any_global;       // some radix head's threshold bin is too large for the in-CTA select
     uint32_t n_decided;        // (b, group) pairs decided so far (a count the single launch waits for)
-    uint32_t pad[15];
+    uint32_t pad[17];
 };
 
 // Head split (host-derived): retrieval groups (KV heads with >= 1 retrieval
@@ -102,14 +100,19 @@ struct Params {
     uint32_t* status;
     Sync* sync;
     uint32_t *rlist, *rglist;
-    uint32_t *tick_score, *tick_local, *tick_ret, *tick_sel, *tick_grp;
+    uint32_t *tick_score, *tick_local, *tick_ret;
+    uint32_t* tick_grp;   // [B * n_rg] radix heads of the group done with their select (zero between calls)
+    // the exact select's per-head global state (zero between calls): merged
+    // first-pass histogram (count, 2^-40 mass), gathered candidates, and the
+    // units that have added their bins / finished their compaction
+    uint32_t* sel_cnt;                // [B * n_ret, 256]
+    unsigned long long* sel_mass;     // [B * n_ret, 256]
+    uint32_t* sel_ncand;              // [B * n_ret]
+    uint32_t* sel_arrive;             // [B * n_ret, 2]
     HeadAgg* agg;
     HeadState* hs;
-    uint32_t* hist_cnt;
-    unsigned long long* hist_mass;
     uint32_t* tie_cnt;
     float* scores;   // [B * n_ret, sstride] fp32 index scores, written by the streaming kernel, read by the select
-    uint32_t* cand_cnt;              // [B * n_ret] candidates gathered from the threshold bin
     unsigned long long* cand;        // [B * n_ret, CAND_CAP] (key << 32 | token index)
     uint32_t* bitmap;
     uint32_t* blist;

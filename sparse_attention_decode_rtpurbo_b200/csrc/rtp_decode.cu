@@ -33,7 +33,7 @@ struct Plan {
     uint8_t lg_group[MAX_HKV], lg_mask[MAX_HKV];
     uint8_t slot_head[MAX_HQ], slot_rg[MAX_HQ];
     // workspace byte offsets; [0, zero_end) must be zero when a call starts
-    size_t o_status, o_sync, o_tick_score, o_tick_local, o_tick_ret, o_tick_sel, o_tick_grp, o_cand_cnt, o_agg, o_hist_cnt, o_hist_mass, zero_end;
+    size_t o_status, o_sync, o_tick_score, o_tick_local, o_tick_ret, o_tick_grp, o_agg, o_sel_cnt, o_sel_mass, o_sel_ncand, o_sel_arrive, zero_end;
     size_t o_rlist, o_rglist, o_hs, o_tie_cnt, o_scores, o_cand, o_bitmap, o_blist, o_bcount, o_lpart, o_rpart, total;
 };
 
@@ -117,12 +117,12 @@ static rtp_status make_plan(const rtp_dims* d, const uint8_t* head_kind, int win
     pl->o_tick_score = take(BG * 4);
     pl->o_tick_local = take(BL * 4);
     pl->o_tick_ret = take(BG * 4);
-    pl->o_tick_sel = take(BR * 4);
     pl->o_tick_grp = take(BG * 4);
-    pl->o_cand_cnt = take(BR * 4);
     pl->o_agg = take(BR * AGG_BUCKETS * sizeof(HeadAgg));
-    pl->o_hist_cnt = take(BR * 256 * 4);
-    pl->o_hist_mass = take(BR * 256 * 8);
+    pl->o_sel_cnt = take(BR * 256 * 4);
+    pl->o_sel_mass = take(BR * 256 * 8);
+    pl->o_sel_ncand = take(BR * 4);
+    pl->o_sel_arrive = take(BR * 2 * 4);
     pl->zero_end = o;
     pl->o_rlist = take(BR * 4);
     pl->o_rglist = take(BG * 4);
@@ -256,7 +256,7 @@ static cudaError_t launch(const KParams& K, const Plan& pl, cudaStream_t s, void
         // one resident wave with room for either phase's shared memory (the
         // retrieval phase's grid barriers need every CTA resident; surplus
         // CTAs take no share of the streaming phase)
-        const size_t smem = std::max(asmem_bytes<G>(pl.B), bsmem_bytes<G>(pl.B * pl.n_rg));
+        const size_t smem = std::max(asmem_bytes<G>(pl.B), bsmem_bytes<G>(pl.B * pl.n_ret));
         const int occ = occupancy((const void*)step_kernel<G>, smem);
         if (occ < 1) return report(cudaErrorInvalidConfiguration, "step kernel occupancy");
         const int grid = std::min(cap, occ * sms);
@@ -291,7 +291,7 @@ static cudaError_t launch(const KParams& K, const Plan& pl, cudaStream_t s, void
     // launched as a programmatic dependent of the streaming kernel so that
     // its launch overlaps that kernel's tail
     {
-        const size_t smem = bsmem_bytes<G>(pl.B * pl.n_rg);
+        const size_t smem = bsmem_bytes<G>(pl.B * pl.n_ret);
         const int occ = occupancy((const void*)retrieve_kernel<G>, smem);
         if (occ < 1) return report(cudaErrorInvalidConfiguration, "retrieval kernel occupancy");
         const int grid = std::min(cap, occ * sms);
@@ -422,15 +422,15 @@ static rtp_status decode_step_ws(const rtp_dims* dims, const uint16_t* q_pre, co
     P.tick_score = (uint32_t*)(ws + pl.o_tick_score);
     P.tick_local = (uint32_t*)(ws + pl.o_tick_local);
     P.tick_ret = (uint32_t*)(ws + pl.o_tick_ret);
-    P.tick_sel = (uint32_t*)(ws + pl.o_tick_sel);
     P.tick_grp = (uint32_t*)(ws + pl.o_tick_grp);
+    P.sel_cnt = (uint32_t*)(ws + pl.o_sel_cnt);
+    P.sel_mass = (unsigned long long*)(ws + pl.o_sel_mass);
+    P.sel_ncand = (uint32_t*)(ws + pl.o_sel_ncand);
+    P.sel_arrive = (uint32_t*)(ws + pl.o_sel_arrive);
     P.agg = (HeadAgg*)(ws + pl.o_agg);
     P.hs = (HeadState*)(ws + pl.o_hs);
-    P.hist_cnt = (uint32_t*)(ws + pl.o_hist_cnt);
-    P.hist_mass = (unsigned long long*)(ws + pl.o_hist_mass);
     P.tie_cnt = (uint32_t*)(ws + pl.o_tie_cnt);
     P.scores = (float*)(ws + pl.o_scores);
-    P.cand_cnt = (uint32_t*)(ws + pl.o_cand_cnt);
     P.cand = (unsigned long long*)(ws + pl.o_cand);
     P.bitmap = (uint32_t*)(ws + pl.o_bitmap);
     P.blist = (uint32_t*)(ws + pl.o_blist);

@@ -1,18 +1,20 @@
 // Retrieval kernel of the decode step (sm_100a), launched after the
 // streaming kernel (programmatic dependent launch; it waits for that grid):
 //   1. (only when some head needs it) the exact top-p select over the fp32
-//      index scores the streaming kernel stored: a first pass bins smax - s
-//      (255 bins, count and 2^-40 fixed-point softmax mass), a 256-bin search
-//      picks the bin that completes ceil(p Z), a compaction pass gathers that
-//      bin's tokens and one CTA per head selects inside them (8-bit MSD
-//      digits over the order-preserving u32 keys, ties toward the lowest
-//      index); a bin of more than 4096 tokens takes four refine passes over
-//      all scores instead.  A mark pass sets block bits, one CTA per group
-//      builds its block list.  Each CTA holds its share of the scores in
-//      shared memory when it fits.  Passes are separated by grid barriers:
-//      the grid is one resident wave and no CTA of it depends on work that
-//      is not already running (the streaming kernel it follows never waits
-//      on it).
+//      index scores the streaming kernel stored, one CTA per head, with no
+//      grid barrier between its steps: a first pass bins smax - s (255 bins,
+//      count and 2^-40 fixed-point softmax mass, in shared memory), a 256-bin
+//      search picks the bin that completes ceil(p Z), a second pass marks the
+//      blocks of the tokens above that bin and gathers the bin's tokens, and
+//      the CTA selects inside them (8-bit MSD digits over the
+//      order-preserving u32 keys, ties toward the lowest index); a bin of
+//      more than 4096 tokens takes four refine passes and a mark pass
+//      instead.  The scores stream through the stage buffers in 16 KB bulk
+//      copies.  The last head of a group (a ticket) builds the group's block
+//      list.  One grid barrier then separates the select from the attention:
+//      the grid is one resident wave (cooperative launch) and no CTA of it
+//      depends on work that is not already running (the streaming kernel it
+//      follows never waits on it).
 //   2. block-sparse attention of the retrieval heads over their groups'
 //      block lists, split evenly over the CTAs (TMA-staged K/V, tensor
 //      cores), and the log-sum-exp combine of the splits.
@@ -81,19 +83,15 @@ struct BSmem {
     alignas(16) float qi[MAX_G][R];
     unsigned long long dmass[256];
     uint32_t dcnt[256];
-    uint32_t tmask[MAX_G];
     uint32_t tcnt[MAX_G];
-    uint8_t rlist_h[MAX_G];
-    uint32_t want_mask;   // bit hx: this pass processes radix head rlist_h[hx]
-    RHead rhs[MAX_G];   // select state of the segment's radix heads (r_pass)
-    uint32_t nrad_h;
+    uint32_t hcand;   // candidates gathered by a compaction pass of this CTA alone
+    HeadState hst;    // the head's select state as this CTA's digit step computed it
     uint32_t lsel_prefix, lsel_count, lsel_neq;
     unsigned long long lsel_mass, lsel_meq;
     uint8_t tflag[SROWS];
     RDesc desc[NST];
     alignas(8) uint64_t full[NST], empty[NST];
-    alignas(8) uint64_t res_bar;   // the resident score tiles have landed
-    uint32_t resident;             // this CTA's score tiles sit in the stage buffers
+    alignas(8) uint64_t hfull[2 * STAGE_BYTES / (SROWS * 4)];   // select passes: a 4 KB score copy has landed
     uint32_t flag, gen, abort, base;
     unsigned long long acct[ACCT_SLOTS];   // debug cycle sums of thread 0
     unsigned long long sc_k[4], hit_k;     // bin_search: per-warp key sums, key sum before the hit
@@ -101,7 +99,7 @@ struct BSmem {
     int kept[MAX_G];
     uint32_t wsum[4];
     HeadTab tab;
-    int pre[2];   // really [max(B * n_rg, 1) + 1]: tiles before group i (radix groups, then all groups)
+    int pre[2];   // really [max(B * n_ret, 1) + 1]: units before radix head i, then tiles before group i
 };
 
 template <int G>
@@ -149,35 +147,6 @@ __device__ __forceinline__ bool grid_sync(const Params& P, SM& S) {
     return S.abort == 0;
 }
 
-// (b, group) of radix group i
-__device__ __forceinline__ void radix_group(const Params& P, int i, int& b, int& rg) {
-    const uint32_t e = __ldcg(P.rglist + i);
-    b = (int)(e >> 16);
-    rg = (int)(e & 0xFFFFu);
-}
-
-// ---------------------------------------------------------------------------
-// index tiles of the radix groups: a walk shared by the copy warp and the
-// compute warps (CTA c takes tiles [c*T/grid, (c+1)*T/grid))
-// ---------------------------------------------------------------------------
-struct RSeg {
-    int gi, b, rg, L, first, ntiles;
-};
-struct RWalk {
-    int t, t1, ngr;
-    __device__ __forceinline__ bool next(const Params& P, const int* pre, RSeg& s) {
-        if (t >= t1) return false;
-        s.gi = last_le(pre, ngr + 1, t);
-        radix_group(P, s.gi, s.b, s.rg);
-        s.L = __ldg(P.seq_lens + s.b);
-        const int nt = pre[s.gi + 1] - pre[s.gi];
-        s.first = t - pre[s.gi];
-        s.ntiles = min(nt - s.first, t1 - t);
-        t += s.ntiles;
-        return true;
-    }
-};
-
 __device__ __forceinline__ RHead load_rhead(const HeadState* h) {
     RHead r;
     r.prefix = __ldcg(&h->prefix);
@@ -199,355 +168,212 @@ __device__ __forceinline__ uint32_t score_bin(float s, float smax, float dr, flo
     return d < dr ? (uint32_t)min((int)(d * inv_w), 254) : 255u;
 }
 
-// What a pass does with every stored score of a radix head:
-// RP_BINS histograms the first-pass bins; RP_COMPACT gathers the tokens of
-// the threshold bin (when at most CAND_CAP) for a select inside one CTA;
-// otherwise RP_REF0..3 histogram the next 8 key bits of the scores in the
-// threshold bin that match the key prefix found so far and RP_TIES counts
-// threshold ties per tile; RP_MARK marks blocks.
+// What a pass does with every stored score of the head:
+// RP_BINS histograms the first-pass bins; RP_COMPACT marks the blocks of the
+// tokens above the threshold bin and gathers the bin's tokens (when at most
+// CAND_CAP) for the select inside the CTA; otherwise RP_REF0..3 histogram
+// the next 8 key bits of the scores in the threshold bin that match the key
+// prefix found so far, RP_TIES counts threshold ties per 1024-token tile and
+// RP_MARK marks the blocks of the kept tokens.
 enum RPass : int { RP_BINS = 0, RP_REF0, RP_REF1, RP_REF2, RP_REF3, RP_TIES, RP_MARK, RP_COMPACT };
 
-template <int G, int pass>
-__device__ __noinline__ void r_digit(const Params& P, int b, int slot, int tid);
-template <int G>
-__device__ __noinline__ void r_tie_locate(const Params& P, int b, int slot, int tid);
-template <int G>
-__device__ __noinline__ void r_blist(const Params& P, int b, int rg, int tid);
+// A head's stored scores stream through the two stage buffers as 4 KB bulk
+// copies of one 1024-token tile each (sixteen in flight, issued by consumer
+// thread 0); every pass of the select is one sweep over them, its
+// histograms in shared memory.
+constexpr int HS_CHUNK = SROWS;                               // scores per copy (4 KB)
+constexpr int HS_SLOTS = 2 * STAGE_BYTES / (HS_CHUNK * 4);    // copies in flight
+constexpr int HS_U = HS_CHUNK / CONSUMERS;                    // scores per thread and copy
+constexpr int HS_FOLD = HIST_FLUSH_TOKENS / HS_CHUNK;         // copies between folds of the 32-bit partial sums
 
-// One pass over the stored scores of this CTA's share of the radix groups'
-// 1024-token tiles (consumer threads; thread tid takes tokens n0 + tid + 128 u
-// of one radix head's tile per item; items walk (tile, head) in order).  The
-// scores come from the stage buffers when the share is resident there, else
-// from global memory.  Histogram passes fold the CTA's shared histograms into
-// the heads' global ones at the end of each run of a group's tiles (and every
-// 64 tiles); the compaction and mark passes write candidates and bitmap bits.
-// The per-head steps between passes run after a grid barrier.
-template <int G, int pass>
-__device__ __noinline__ void r_pass(const Params& P, RWalk wk, const int* pre, int tid) {
-    BSmem<G>& S = bsmem<G>();
-    constexpr int U = SROWS / CONSUMERS;
-    const int lane = tid & 31;
-    RSeg sg;
-    Acct ac;
-    ac.init(P, S.acct, tid == 0);
-    const int rp = pass - RP_REF0;
-    // key bits above the refine pass's digit (the prefix found so far); unused in pass RP_REF0
-    constexpr int psh = (pass > RP_REF0 && pass <= RP_REF3) ? 32 - 8 * (pass - RP_REF0) : 0;
-    // the parameters this loop uses, read once: through a reference into the
-    // parameter block they would be read again after every global atomic
-    const int n_ret = P.n_ret, sstride = P.sstride, words_cap = P.words_cap, ntiles_cap = P.ntiles_cap;
-    const HeadState* const hs = P.hs;
-    const float* const scores = P.scores;
-    uint32_t* const hist_cnt = P.hist_cnt;
-    unsigned long long* const hist_mass_g = P.hist_mass;
-    uint32_t* const cand_cnt = P.cand_cnt;
-    unsigned long long* const cand = P.cand;
-    uint32_t* const bitmap = P.bitmap;
-    uint32_t* const tie_cnt = P.tie_cnt;
-    const bool unit = P.topk > 0;   // static top-k: every token weighs 1 (the histograms count)
-    const bool resident = S.resident != 0;
-    if (resident) {
-        const long long tq = clock64();
-        if (!mbar_wait_bounded(&S.res_bar, 0u)) set_status(P, ST_TIMEOUT);
-        if (tid == 0 && P.dbg_trace) S.acct[40 - 16] += (unsigned long long)(clock64() - tq);
+// The histogram's 32-bit partial sums (S.H, head 0) into the 64-bit ones
+// (S.dcnt, S.dmass); every bin's partials back to zero.
+template <int G>
+__device__ __forceinline__ void h_fold(BSmem<G>& S, int tid) {
+    consumer_sync();
+    for (int d = tid; d < 256; d += CONSUMERS) {
+        S.dcnt[d] += S.H.cnt[0][d];
+        S.dmass[d] += hist_mass(S.H, 0, d);
+        S.H.cnt[0][d] = 0;
+        S.H.m[0][0][d] = 0;
+        S.H.m[1][0][d] = 0;
+        S.H.m[2][0][d] = 0;
     }
-    int sbase = 0;
-    while (wk.next(P, pre, sg)) {
-        const int nh = S.tab.rg_nh[sg.rg], slot0 = S.tab.rg_slot0[sg.rg];
-        const int64_t bs0 = (int64_t)sg.b * n_ret + slot0;
-        for (int x = tid; x < 4 * G * 256; x += CONSUMERS) (&S.H.cnt[0][0])[x] = 0;
-        if (tid < MAX_G) {
-            S.tmask[tid] = 0;
-            S.tcnt[tid] = 0;
-        }
-        // the group's radix heads (then their select state, once per run),
-        // then a flat loop over (tile, head) items
-        if (tid == 0) {
-            uint32_t n = 0, wm = 0;
-            for (int hh = 0; hh < nh; ++hh) {
-                const HeadState* h = hs + bs0 + hh;
-                if (__ldcg(&h->mode) != MODE_RADIX) continue;
-                const bool local = __ldcg(&h->n_cand) <= (uint32_t)CAND_CAP;
-                const bool want = (pass == RP_BINS || pass == RP_MARK) ? true : (pass == RP_COMPACT ? local : !local);
-                if (want) wm |= 1u << n;
-                S.rlist_h[n++] = (uint8_t)hh;
-            }
-            S.nrad_h = n;
-            S.want_mask = wm;
-        }
-        consumer_sync();
-        const int nr = (int)S.nrad_h;
-        const uint32_t wantm = S.want_mask;
-        if (tid < nr) S.rhs[tid] = load_rhead(hs + bs0 + S.rlist_h[tid]);
-        const int nitems = sg.ntiles * nr;
-        // this CTA's histograms -> the heads' global ones (at the end of the
-        // run, and every 64 tiles so that no partial sum can wrap)
-        auto flush = [&]() {
-            consumer_sync();
-            for (int x = tid; x < nh * 256; x += CONSUMERS) {
-                const int hh = x >> 8, d = x & 255;
-                const uint32_t c = S.H.cnt[hh][d];
-                if (c) {
-                    atomicAdd(hist_cnt + (bs0 + hh) * 256 + d, c);
-                    atomicAdd(hist_mass_g + (bs0 + hh) * 256 + d, hist_mass(S.H, hh, d));
-                    S.H.cnt[hh][d] = 0;
-                    S.H.m[0][hh][d] = 0;
-                    S.H.m[1][hh][d] = 0;
-                    S.H.m[2][hh][d] = 0;
-                }
-            }
-            consumer_sync();
-        };
-        // items of every radix head in (tile, head) order: resident ones from
-        // the stage buffers (slot sbase + it), else from the stored scores
-        const float* res = reinterpret_cast<const float*>(&S.stage[0][0]) + (size_t)sbase * SROWS;
-        float vn[U];
-        auto load_item = [&](int it, int tile, int hx, float* dst) {
-            const int hh = S.rlist_h[hx];
-            const int n0 = tile * SROWS, nvalid = min(SROWS, sg.L - n0);
-            const float* src = resident ? res + (size_t)it * SROWS : scores + (bs0 + hh) * sstride + n0;
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int r = tid + u * CONSUMERS;
-                dst[u] = r < nvalid ? (resident ? src[r] : __ldcg(src + r)) : 0.f;
-            }
-        };
-        if (nitems > 0) load_item(0, sg.first, 0, vn);
-        consumer_sync();   // S.rhs
-        if constexpr (pass == RP_COMPACT) {
-            if (resident) {
-                // resident scores: count the threshold-bin tokens per head,
-                // reserve each head's range with one atomic, then write (one
-                // global round trip per head and run instead of per item)
-                for (int sub = 0; sub < 2; ++sub) {
-                    int tile = sg.first - 1, hx = nr - 1;
-#pragma unroll 1
-                    for (int it = 0; it < nitems; ++it) {
-                        if (++hx == nr) {
-                            hx = 0;
-                            ++tile;
-                        }
-                        if (!((wantm >> hx) & 1u)) continue;
-                        const RHead rh = S.rhs[hx];
-                        const int n0 = tile * SROWS, nvalid = min(SROWS, sg.L - n0);
-                        const float* src = res + (size_t)it * SROWS;
-                        uint32_t bal[U], tot = 0;
-                        float v[U];
-#pragma unroll
-                        for (int u = 0; u < U; ++u) {
-                            const int r = tid + u * CONSUMERS;
-                            v[u] = src[r];
-                            bal[u] = __ballot_sync(0xffffffffu,
-                                                   r < nvalid && score_bin(v[u], rh.smax, rh.dr, rh.inv_w) == rh.bstar);
-                            tot += __popc(bal[u]);
-                        }
-                        if (sub == 0) {
-                            if (lane == 0 && tot) atomicAdd(&S.tcnt[hx], tot);
-                        } else if (tot) {
-                            uint32_t off = 0;
-                            if (lane == 0) off = atomicAdd(&S.tcnt[hx], tot);
-                            uint32_t pos = S.tmask[hx] + __shfl_sync(0xffffffffu, off, 0);
-#pragma unroll
-                            for (int u = 0; u < U; ++u) {
-                                if ((bal[u] >> lane) & 1u) {
-                                    const uint32_t pp = pos + __popc(bal[u] & ((1u << lane) - 1u));
-                                    if (pp < (uint32_t)CAND_CAP)
-                                        cand[(bs0 + S.rlist_h[hx]) * CAND_CAP + pp] =
-                                            ((unsigned long long)f2key(v[u]) << 32) | (uint32_t)(n0 + tid + u * CONSUMERS);
-                                }
-                                pos += __popc(bal[u]);
-                            }
-                        }
-                    }
-                    consumer_sync();
-                    if (sub == 0) {
-                        if (tid < nr && ((wantm >> tid) & 1u)) {
-                            S.tmask[tid] = atomicAdd(cand_cnt + bs0 + S.rlist_h[tid], S.tcnt[tid]);
-                            S.tcnt[tid] = 0;
-                        }
-                        consumer_sync();
-                    }
-                }
-                ac.mark(26);
-                sbase += nitems;
-                continue;
-            }
-        }
-        uint32_t ovf_n = 0u;
-        unsigned long long ovf_m = 0ull;
-        int cur_h = -1;
-        // item it = (tile, head hx), walked without divisions
-        int tile = sg.first - 1, hx = nr - 1;
-#pragma unroll 1
-        for (int it = 0; it < nitems; ++it) {
-            if (++hx == nr) {
-                hx = 0;
-                ++tile;
-            }
-            float v[U];
-#pragma unroll
-            for (int u = 0; u < U; ++u) v[u] = vn[u];
-            if (it + 1 < nitems) {
-                if (hx + 1 == nr) load_item(it + 1, tile + 1, 0, vn);
-                else load_item(it + 1, tile, hx + 1, vn);
-            }
-            const int hh = S.rlist_h[hx];
-            const int n0 = tile * SROWS, nvalid = min(SROWS, sg.L - n0);
-            if (pass <= RP_REF3 && hx == 0 && tile > sg.first && ((tile - sg.first) & (HIST_FLUSH_TOKENS / SROWS - 1)) == 0) {
-                // every 64 tiles: no partial sum can wrap (the overflow bin's
-                // register sums join at the head's next switch)
-                flush();
-            }
-            if (!((wantm >> hx) & 1u)) continue;   // (uniform over the CTA)
-            if (pass == RP_BINS && hh != cur_h && cur_h >= 0) {
-                // out-of-range sums of the previous head
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) {
-                    ovf_n += __shfl_xor_sync(0xffffffffu, ovf_n, o);
-                    ovf_m += __shfl_xor_sync(0xffffffffu, ovf_m, o);
-                }
-                if (lane == 0 && ovf_n) hist_add(S.H, cur_h, 255, ovf_n, ovf_m);
-                ovf_n = 0u;
-                ovf_m = 0ull;
-            }
-            cur_h = hh;
-            const RHead rh = S.rhs[hx];
-            uint32_t bits = 0u, cnt = 0u;
-            uint32_t bal[U];
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int r = tid + u * CONSUMERS;
-                const bool ok = r < nvalid;
-                const uint32_t key = f2key(v[u]);
-                if constexpr (pass == RP_BINS) {
-                    if (ok) {
-                        const uint32_t bn = score_bin(v[u], rh.smax, rh.dr, rh.inv_w);
-                        const unsigned long long ms = unit ? 1ull : fixmass(key, rh.smax);
-                        if (bn < 255u) {
-                            hist_add(S.H, hh, (int)bn, 1u, ms);
-                        } else {
-                            ovf_n += 1u;
-                            ovf_m += ms;
-                        }
-                    }
-                } else if constexpr (pass <= RP_REF3) {
-                    if (ok && score_bin(v[u], rh.smax, rh.dr, rh.inv_w) == rh.bstar &&
-                        (rp == 0 || (key >> psh) == rh.prefix)) {
-                        const uint32_t d = (key >> (24 - 8 * rp)) & 255u;
-                        hist_add(S.H, hh, (int)d, 1u, unit ? 1ull : fixmass(key, rh.smax));
-                    }
-                } else if constexpr (pass == RP_TIES) {
-                    cnt += (ok && key == rh.tau) ? 1u : 0u;
-                } else if constexpr (pass == RP_COMPACT) {
-                    // ballots only: the warp's candidates of the item go out below
-                    const bool in = ok && score_bin(v[u], rh.smax, rh.dr, rh.inv_w) == rh.bstar;
-                    bal[u] = __ballot_sync(0xffffffffu, in);
-                } else {
-                    const bool keep = ok && (key > rh.tau || (key == rh.tau && (uint32_t)(n0 + r) <= rh.tie_idx));
-                    // a warp's 32 tokens lie in one 64-token block: one vote per warp
-                    if (__any_sync(0xffffffffu, keep) && lane == 0) bits |= 1u << ((r / BLK) & 15);
-                }
-            }
-            if constexpr (pass == RP_COMPACT) {
-                // one reservation per warp and item, then the candidates in
-                // ballot order
-                uint32_t tot = 0;
-#pragma unroll
-                for (int u = 0; u < U; ++u) tot += __popc(bal[u]);
-                if (tot) {
-                    uint32_t base = 0;
-                    if (lane == 0) base = atomicAdd(cand_cnt + bs0 + hh, tot);
-                    base = __shfl_sync(0xffffffffu, base, 0);
-#pragma unroll
-                    for (int u = 0; u < U; ++u) {
-                        if ((bal[u] >> lane) & 1u) {
-                            const uint32_t pos = base + __popc(bal[u] & ((1u << lane) - 1u));
-                            if (pos < (uint32_t)CAND_CAP) {
-                                const int r = tid + u * CONSUMERS;
-                                cand[(bs0 + hh) * CAND_CAP + pos] =
-                                    ((unsigned long long)f2key(v[u]) << 32) | (uint32_t)(n0 + r);
-                            }
-                        }
-                        base += __popc(bal[u]);
-                    }
-                }
-            }
-            if constexpr (pass == RP_MARK) {
-                // the warp's blocks straight into the head's bitmap (zeroed
-                // when the group was registered for the select)
-                if (lane == 0 && bits)
-                    atomicOr(bitmap + (bs0 + hh) * words_cap + tile / 2, bits << ((tile & 1) * 16));
-            } else if constexpr (pass == RP_TIES) {
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
-                if (lane == 0 && cnt) atomicAdd(&S.tcnt[hh], cnt);
-                consumer_sync();
-                if (tid == 0) {
-                    tie_cnt[(bs0 + hh) * ntiles_cap + tile] = S.tcnt[hh];
-                    S.tcnt[hh] = 0;
-                }
-                consumer_sync();
-            }
-            ac.mark(pass == RP_COMPACT ? 26 : (pass == RP_MARK ? 27 : 24));
-            ac.count(25);
-        }
-        if (pass == RP_BINS && cur_h >= 0) {
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                ovf_n += __shfl_xor_sync(0xffffffffu, ovf_n, o);
-                ovf_m += __shfl_xor_sync(0xffffffffu, ovf_m, o);
-            }
-            if (lane == 0 && ovf_n) hist_add(S.H, cur_h, 255, ovf_n, ovf_m);
-        }
-        if constexpr (pass <= RP_REF3) flush();
-        consumer_sync();
-        sbase += nitems;
-    }
+    consumer_sync();
 }
 
-// The copy warp at the start of the select: when this CTA's share of score
-// items (every radix head of its tiles) fits the two stage buffers, all of
-// them are copied there at once (one 4 KB bulk copy per item, in the order
-// the passes walk them) and every pass then reads shared memory only.
-constexpr int RES_ITEMS = 2 * STAGE_BYTES / (SROWS * 4);
-template <int G>
-__device__ __noinline__ void r_load_scores(const Params& P, RWalk wk, const int* pre, int lane) {
+// One pass over copies [c0, c1) of the stored scores of radix head (b, slot)
+// by this CTA's consumer threads (thread tid takes scores tid + 128 u of every
+// copy, so a warp's 32 scores lie in one 64-token block).  `unit`: the CTA
+// holds one unit of a head shared by several CTAs, so the bins go to the
+// head's global histogram and the candidates are reserved in the head's
+// global count; otherwise the whole head is this CTA's.  `seq` counts the
+// copies this CTA has waited for (it picks the slot and the barrier phase).
+// A wait that gives up sets the status and S.abort; the pass then stops
+// after waiting, bounded, for the copies it has in flight.
+template <int G, int pass>
+__device__ __noinline__ void h_pass(const Params& P, int b, int slot, const RHead rh, int c0, int c1, bool unit_of_many,
+                                    uint32_t& seq, int tid) {
     BSmem<G>& S = bsmem<G>();
-    if (lane != 0) return;
-    int items = 0;
-    {
-        RWalk w2 = wk;
-        RSeg sg;
-        while (w2.next(P, pre, sg)) {
-            const int nh = S.tab.rg_nh[sg.rg], slot0 = S.tab.rg_slot0[sg.rg];
-            int nr = 0;
-            for (int hh = 0; hh < nh; ++hh)
-                nr += __ldcg(&P.hs[(int64_t)sg.b * P.n_ret + slot0 + hh].mode) == MODE_RADIX;
-            items += sg.ntiles * nr;
+    const int lane = tid & 31, warp = tid >> 5;
+    const int64_t bs = (int64_t)b * P.n_ret + slot;
+    const int L = __ldg(P.seq_lens + b);
+    const int nch = c1 - c0;
+    const float* const src = P.scores + bs * P.sstride;
+    uint8_t* const ring = &S.stage[0][0];
+    const bool unit = P.topk > 0;   // static top-k: every token weighs 1 (the histograms count)
+    constexpr int rp = pass - RP_REF0;
+    // key bits above the refine pass's digit (the prefix found so far); unused in pass RP_REF0
+    constexpr int psh = (pass > RP_REF0 && pass <= RP_REF3) ? 32 - 8 * (pass - RP_REF0) : 0;
+    uint32_t* const bmp = P.bitmap + bs * P.words_cap;
+    unsigned long long* const cand = P.cand + bs * CAND_CAP;
+    auto issue = [&](int k) {   // copy c0 + k of the pass into its slot (thread 0)
+        const uint32_t q = seq + (uint32_t)k, sl = q % HS_SLOTS;
+        const int c = c0 + k;
+        const int nv = min(HS_CHUNK, L - c * HS_CHUNK);
+        const uint32_t bytes = (uint32_t)((nv + 3) & ~3) * 4u;   // whole 16-byte units inside the row
+        mbar_expect_tx(&S.hfull[sl], bytes);
+        bulk_g2s(ring + (size_t)sl * HS_CHUNK * 4, src + (size_t)c * HS_CHUNK, bytes, &S.hfull[sl]);
+    };
+    if constexpr (pass <= RP_REF3) {
+        for (int d = tid; d < 256; d += CONSUMERS) {
+            S.dcnt[d] = 0;
+            S.dmass[d] = 0ull;
+            S.H.cnt[0][d] = 0;
+            S.H.m[0][0][d] = 0;
+            S.H.m[1][0][d] = 0;
+            S.H.m[2][0][d] = 0;
         }
     }
-    if (items == 0 || items > RES_ITEMS) {
-        S.resident = 0;
+    if (tid < MAX_G) S.tcnt[tid] = 0;
+    if (tid == 0) S.hcand = 0;
+    consumer_sync();
+    if (tid == 0)
+        for (int c = 0; c < HS_SLOTS && c < nch; ++c) issue(c);
+    uint32_t ovf_n = 0u;
+    unsigned long long ovf_m = 0ull;
+    int k = 0;
+    for (; k < nch; ++k) {
+        const uint32_t q = seq + (uint32_t)k, sl = q % HS_SLOTS;
+        if (!mbar_wait_bounded(&S.hfull[sl], (q / HS_SLOTS) & 1u)) {
+            set_status(P, ST_TIMEOUT);
+            S.abort = 1;
+        }
+        const float* x = reinterpret_cast<const float*>(ring + (size_t)sl * HS_CHUNK * 4);
+        const int c = c0 + k;
+        const int n0 = c * HS_CHUNK, nv = min(HS_CHUNK, L - n0);
+        uint32_t w0 = 0u;        // RP_COMPACT / RP_MARK: bits of blocks n0/64 + 0..15
+        uint32_t tcount = 0u;    // RP_TIES: threshold ties of this thread in the tile
+#pragma unroll
+        for (int u = 0; u < HS_U; ++u) {
+            const int r = tid + u * CONSUMERS;
+            const bool ok = r < nv;
+            const float v = x[r];
+            const uint32_t key = f2key(v);
+            if constexpr (pass == RP_BINS) {
+                if (ok) {
+                    const uint32_t bn = score_bin(v, rh.smax, rh.dr, rh.inv_w);
+                    const unsigned long long ms = unit ? 1ull : fixmass(key, rh.smax);
+                    if (bn < 255u) {
+                        hist_add(S.H, 0, (int)bn, 1u, ms);
+                    } else {
+                        ovf_n += 1u;
+                        ovf_m += ms;
+                    }
+                }
+            } else if constexpr (pass <= RP_REF3) {
+                if (ok && score_bin(v, rh.smax, rh.dr, rh.inv_w) == rh.bstar && (rp == 0 || (key >> psh) == rh.prefix))
+                    hist_add(S.H, 0, (int)((key >> (24 - 8 * rp)) & 255u), 1u, unit ? 1ull : fixmass(key, rh.smax));
+            } else if constexpr (pass == RP_TIES) {
+                tcount += (ok && key == rh.tau) ? 1u : 0u;
+            } else {
+                bool keep;
+                if constexpr (pass == RP_COMPACT) {
+                    const uint32_t bn = ok ? score_bin(v, rh.smax, rh.dr, rh.inv_w) : 256u;
+                    keep = bn < rh.bstar;
+                    // the bin's tokens, in ballot order behind one reservation per warp
+                    const uint32_t bal = __ballot_sync(0xffffffffu, bn == rh.bstar);
+                    if (bal) {
+                        uint32_t base = 0;
+                        if (lane == 0)
+                            base = unit_of_many ? atomicAdd(P.sel_ncand + bs, (uint32_t)__popc(bal))
+                                                : atomicAdd(&S.hcand, (uint32_t)__popc(bal));
+                        base = __shfl_sync(0xffffffffu, base, 0);
+                        const uint32_t pos = base + __popc(bal & ((1u << lane) - 1u));
+                        if (bn == rh.bstar && pos < (uint32_t)CAND_CAP)
+                            cand[pos] = ((unsigned long long)key << 32) | (uint32_t)(n0 + r);
+                    }
+                } else {
+                    keep = ok && (key > rh.tau || (key == rh.tau && (uint32_t)(n0 + r) <= rh.tie_idx));
+                }
+                // block of the warp's 32 scores within the tile: 2 u + warp / 2
+                if (__any_sync(0xffffffffu, keep)) w0 |= 1u << (2 * u + (warp >> 1));
+            }
+        }
+        if constexpr (pass == RP_COMPACT || pass == RP_MARK) {
+            // the blocks straight into the head's bitmap (zeroed when the
+            // group was registered for the select)
+            if (lane == 0 && w0) atomicOr(bmp + c / 2, w0 << ((c & 1) * 16));
+        } else if constexpr (pass == RP_TIES) {
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) tcount += __shfl_xor_sync(0xffffffffu, tcount, o);
+            if (lane == 0 && tcount) atomicAdd(&S.tcnt[k & 1], tcount);
+        }
+        consumer_sync();   // the slot is read (and this copy's tie counts are complete)
+        if constexpr (pass == RP_TIES) {
+            if (tid == 0) {
+                P.tie_cnt[bs * P.ntiles_cap + c] = S.tcnt[k & 1];
+                S.tcnt[k & 1] = 0;
+            }
+        }
+        if (S.abort) break;   // (set before the barrier: every thread sees it)
+        if (tid == 0 && k + HS_SLOTS < nch) issue(k + HS_SLOTS);
+        if constexpr (pass <= RP_REF3) {
+            if ((k + 1) % HS_FOLD == 0 && k + 1 < nch) h_fold(S, tid);
+        }
+    }
+    if (k < nch) {
+        // gave up: wait, bounded, for the copies still in flight, then stop
+        for (int d = k + 1; d < nch && d <= k + HS_SLOTS - 1; ++d) {
+            const uint32_t q = seq + (uint32_t)d;
+            mbar_wait_bounded(&S.hfull[q % HS_SLOTS], (q / HS_SLOTS) & 1u);
+        }
+        consumer_sync();
         return;
     }
-    S.resident = 1;
-    mbar_expect_tx(&S.res_bar, (uint32_t)items * SROWS * 4);
-    uint8_t* dst = &S.stage[0][0];
-    RSeg sg;
-    while (wk.next(P, pre, sg)) {
-        const int nh = S.tab.rg_nh[sg.rg], slot0 = S.tab.rg_slot0[sg.rg];
-        const int64_t bs0 = (int64_t)sg.b * P.n_ret + slot0;
-        for (int t = 0; t < sg.ntiles; ++t)
-            for (int hh = 0; hh < nh; ++hh) {
-                if (__ldcg(&P.hs[bs0 + hh].mode) != MODE_RADIX) continue;
-                bulk_g2s(dst, P.scores + (bs0 + hh) * P.sstride + (int64_t)(sg.first + t) * SROWS, SROWS * 4, &S.res_bar);
-                dst += SROWS * 4;
-            }
+    seq += (uint32_t)nch;
+    if constexpr (pass == RP_BINS) {
+        // tokens beyond the binned range: bin 255
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            ovf_n += __shfl_xor_sync(0xffffffffu, ovf_n, o);
+            ovf_m += __shfl_xor_sync(0xffffffffu, ovf_m, o);
+        }
+        if (lane == 0 && ovf_n) {
+            atomicAdd(&S.H.cnt[0][255], ovf_n);
+            atomicAdd(&S.dmass[255], ovf_m);
+        }
     }
+    if constexpr (pass <= RP_REF3) h_fold(S, tid);
+    if constexpr (pass == RP_BINS) {
+        if (unit_of_many) {
+            // the unit's bins into the head's global histogram
+            for (int d = tid; d < 256; d += CONSUMERS) {
+                const uint32_t n = S.dcnt[d];
+                if (n) {
+                    atomicAdd(P.sel_cnt + bs * 256 + d, n);
+                    atomicAdd(P.sel_mass + bs * 256 + d, S.dmass[d]);
+                }
+            }
+        }
+    }
+    if constexpr (pass == RP_COMPACT || pass == RP_MARK || pass == RP_BINS)
+        __threadfence();   // bitmap bits, candidates and bins before the head's and the group's tickets
+    consumer_sync();
 }
 
 // ---------------------------------------------------------------------------
-// per-head steps between the passes (one CTA per radix head)
+// steps between the passes (inside the head's CTA)
 // ---------------------------------------------------------------------------
 // Pick the digit of pass `pass` for radix head `hx`: the largest digit d whose
 // bins >= d hold at least the target mass (over the tokens above the prefix).
@@ -607,19 +433,13 @@ __device__ __forceinline__ void bin_search(BSmem<G>& S, KF key_of, AF aux_of, bo
     consumer_sync();
 }
 
+// The threshold step after a pass: `publish` writes the head's new select
+// state to the workspace (else it is only in S.hst, for this CTA).
 template <int G, int pass>
-__device__ __noinline__ void r_digit(const Params& P, int b, int slot, int tid) {
+__device__ __noinline__ void r_digit(const Params& P, int b, int slot, int tid, bool publish = true) {
     BSmem<G>& S = bsmem<G>();
     const int64_t bs = (int64_t)b * P.n_ret + slot;
-    uint32_t* gcnt = P.hist_cnt + bs * 256;
-    unsigned long long* gmass = P.hist_mass + bs * 256;
-    for (int d = tid; d < 256; d += CONSUMERS) {
-        S.dcnt[d] = __ldcg(gcnt + d);
-        S.dmass[d] = __ldcg(gmass + d);
-        gcnt[d] = 0;
-        gmass[d] = 0ull;
-    }
-    consumer_sync();
+    // (the pass's histogram is in S.dcnt / S.dmass)
     auto mass_of = [&](int d) { return S.dmass[d]; };
     auto cnt_of = [&](int d) { return S.dcnt[d]; };
     if constexpr (pass == RP_BINS) {
@@ -647,8 +467,8 @@ __device__ __noinline__ void r_digit(const Params& P, int b, int slot, int tid) 
             st.mass_above = S.hit_k;
             st.count_above = S.hit_a;
             st.prefix = 0;
-            if (st.n_cand > (uint32_t)CAND_CAP) atomicOr(&P.sync->any_global, 1u);
-            P.hs[bs] = st;
+            S.hst = st;
+            if (publish) P.hs[bs] = st;
         }
         consumer_sync();
         return;
@@ -682,7 +502,6 @@ __device__ __noinline__ void r_digit(const Params& P, int b, int slot, int tid) 
                 const int bh = b * P.Hq + S.tab.slot_head[slot];
                 if (P.dbg_tau) P.dbg_tau[bh] = key2f(st.tau_key);
                 if (P.dbg_kstar) P.dbg_kstar[bh] = (int32_t)st.kstar;
-                if (!st.all_ties) atomicOr(&P.sync->any_ties, 1u);
             }
         }
         P.hs[bs] = st;
@@ -829,7 +648,6 @@ __device__ __noinline__ void r_local_select(const Params& P, int b, int slot, in
         const int bh = b * P.Hq + S.tab.slot_head[slot];
         if (P.dbg_tau) P.dbg_tau[bh] = key2f(tau);
         if (P.dbg_kstar) P.dbg_kstar[bh] = (int32_t)(count_above + n_tie);
-        P.cand_cnt[bs] = 0;
     }
     consumer_sync();
 }
@@ -883,6 +701,68 @@ __device__ __noinline__ void r_tie_locate(const Params& P, int b, int slot, int 
             cum += c;
         }
         if (lane == 0) P.hs[bs].tie_idx = (uint32_t)(n0 + found);
+    }
+    consumer_sync();
+}
+
+// After the select inside the CTA: the blocks of the kept candidates (key
+// above tau, or tau with an index up to the largest tie kept) into the head's
+// bitmap.
+template <int G>
+__device__ __noinline__ void h_mark_cand(const Params& P, int b, int slot, int tid) {
+    const int64_t bs = (int64_t)b * P.n_ret + slot;
+    const uint32_t n = min(__ldcg(&P.hs[bs].n_cand), (uint32_t)CAND_CAP);
+    const uint32_t tau = __ldcg(&P.hs[bs].tau_key), tie = __ldcg(&P.hs[bs].tie_idx);
+    uint32_t* const bmp = P.bitmap + bs * P.words_cap;
+    for (uint32_t i = (uint32_t)tid; i < n; i += CONSUMERS) {
+        const unsigned long long c = __ldcg(P.cand + bs * CAND_CAP + i);
+        const uint32_t key = (uint32_t)(c >> 32), idx = (uint32_t)(c & 0xFFFFFFFFull);
+        if (key > tau || (key == tau && idx <= tie)) atomicOr(bmp + (idx >> 11), 1u << ((idx >> 6) & 31));
+    }
+    __threadfence();   // bitmap bits before the group ticket
+    consumer_sync();
+}
+
+// The end of the select of radix head (b, slot), by the CTA that finished the
+// head's last unit: with at most CAND_CAP tokens in the threshold bin (all
+// gathered by the units' compactions, which also marked the blocks above
+// it), the select inside the CTA and the marks of the kept candidates;
+// otherwise four refine passes, the tie location and a mark pass over the
+// whole head, in this CTA.  Then the head's global select state goes back to
+// zero for the next call.
+template <int G>
+__device__ __noinline__ void h_finish(const Params& P, int b, int slot, uint32_t& seq, int tid) {
+    BSmem<G>& S = bsmem<G>();
+    const int64_t bs = (int64_t)b * P.n_ret + slot;
+    const uint32_t ncand = __ldcg(&P.hs[bs].n_cand);
+    if (ncand <= (uint32_t)CAND_CAP) {
+        if (ncand <= 8u * CONSUMERS) r_local_select<G, 8>(P, b, slot, tid);
+        else r_local_select<G, CAND_CAP / CONSUMERS>(P, b, slot, tid);
+        h_mark_cand<G>(P, b, slot, tid);
+    } else {
+        const int nch = (__ldg(P.seq_lens + b) + HS_CHUNK - 1) / HS_CHUNK;
+        h_pass<G, RP_REF0>(P, b, slot, load_rhead(P.hs + bs), 0, nch, false, seq, tid);
+        if (!S.abort) r_digit<G, RP_REF0>(P, b, slot, tid);
+        if (!S.abort) h_pass<G, RP_REF1>(P, b, slot, load_rhead(P.hs + bs), 0, nch, false, seq, tid);
+        if (!S.abort) r_digit<G, RP_REF1>(P, b, slot, tid);
+        if (!S.abort) h_pass<G, RP_REF2>(P, b, slot, load_rhead(P.hs + bs), 0, nch, false, seq, tid);
+        if (!S.abort) r_digit<G, RP_REF2>(P, b, slot, tid);
+        if (!S.abort) h_pass<G, RP_REF3>(P, b, slot, load_rhead(P.hs + bs), 0, nch, false, seq, tid);
+        if (!S.abort) r_digit<G, RP_REF3>(P, b, slot, tid);
+        if (!S.abort && !__ldcg(&P.hs[bs].all_ties)) {
+            h_pass<G, RP_TIES>(P, b, slot, load_rhead(P.hs + bs), 0, nch, false, seq, tid);
+            if (!S.abort) r_tie_locate<G>(P, b, slot, tid);
+        }
+        if (!S.abort) h_pass<G, RP_MARK>(P, b, slot, load_rhead(P.hs + bs), 0, nch, false, seq, tid);
+    }
+    for (int d = tid; d < 256; d += CONSUMERS) {
+        P.sel_cnt[bs * 256 + d] = 0;
+        P.sel_mass[bs * 256 + d] = 0ull;
+    }
+    if (tid == 0) {
+        P.sel_ncand[bs] = 0;
+        P.sel_arrive[2 * bs] = 0;
+        P.sel_arrive[2 * bs + 1] = 0;
     }
     consumer_sync();
 }
@@ -1126,32 +1006,35 @@ __device__ __forceinline__ void r_setup(const Params& P, int tid) {
             mbar_init(&S.full[i], 1);
             mbar_init(&S.empty[i], CONSUMERS / 32);
         }
-        mbar_init(&S.res_bar, 1);
+        for (int i = 0; i < HS_SLOTS; ++i) mbar_init(&S.hfull[i], 1);
         mbar_fence_init();
         S.gen = 0;
         S.abort = 0;
         for (int i = 0; i < ACCT_SLOTS; ++i) S.acct[i] = 0ull;
-        S.resident = 0;
     }
     if (tid >= 32) copy_tab(P.tab, S.tab, tid - 32, THREADS - 32);
 }
 
 // The call's coordination words back to zero, by the last CTA out of the
-// call's last kernel (after an aborted call also the select histograms it
-// may have left).
+// call's last kernel (after an aborted call also the group tickets of the
+// select it may have left).
 __device__ __noinline__ void clear_call_words(const Params& P) {
     P.sync->n_radix_heads = 0;
     P.sync->n_radix_groups = 0;
-    P.sync->any_ties = 0;
     P.sync->barrier = 0;
     P.sync->kb_work = 0;
     if (__ldcg(P.status) != 0) {
-        for (int64_t i = 0; i < (int64_t)P.B * P.n_ret * 256; ++i) {
-            P.hist_cnt[i] = 0;
-            P.hist_mass[i] = 0ull;
+        for (int i = 0; i < P.B * P.n_rg; ++i) P.tick_grp[i] = 0;
+        for (int64_t i = 0; i < (int64_t)P.B * P.n_ret; ++i) {
+            for (int d = 0; d < 256; ++d) {
+                P.sel_cnt[i * 256 + d] = 0;
+                P.sel_mass[i * 256 + d] = 0ull;
+            }
+            P.sel_ncand[i] = 0;
+            P.sel_arrive[2 * i] = 0;
+            P.sel_arrive[2 * i + 1] = 0;
         }
     }
-    P.sync->any_global = 0;
     P.sync->n_decided = 0;
     P.sync->exit_count = 0;
     __threadfence();
@@ -1198,104 +1081,107 @@ __device__ __forceinline__ void r_body(const KParams& K, bool single) {
     bool ok = S.abort == 0;
     const uint32_t nrad = (ok && work) ? __ldcg(&P.sync->n_radix_heads) : 0u;
     if (nrad > 0) {
-        // ---- exact select of the radix heads
-        const int ngr = (int)__ldcg(&P.sync->n_radix_groups);
-        if (tid < 32)
-            warp_prefix(pre, ngr, [&](int i) {
-                int b, rg;
-                radix_group(P, i, b, rg);
-                return (__ldg(P.seq_lens + b) + SROWS - 1) / SROWS;
-            }, lane);
+        // ---- exact select.  The radix heads' 1024-token score tiles, in head
+        // order, are split into contiguous ranges, one per CTA: every range's
+        // bins go into its heads' global histograms (phase A); then, per head
+        // of the range, the threshold bin from the merged histogram as soon as
+        // all of the head's tiles have added their bins, and the range's
+        // compaction (phase B).  The CTA that completes a head's last tile (a
+        // ticket) selects inside the threshold bin, and the last head of a
+        // group (a second ticket) builds the group's block list.  CTAs wait
+        // only for tiles of the same head, all of which run on resident CTAs
+        // that wait for nothing in phase A.
+        auto head_tiles = [&](int hx) {
+            const uint32_t e = __ldcg(P.rlist + hx);
+            return (__ldg(P.seq_lens + (int)(e >> 16)) + HS_CHUNK - 1) / HS_CHUNK;
+        };
+        if (tid < 32) warp_prefix(pre, (int)nrad, head_tiles, lane);
         __syncthreads();
-        const long long T = pre[ngr];
-        RWalk wk;
-        wk.t = (int)((long long)blockIdx.x * T / gridDim.x);
-        wk.t1 = (int)((long long)(blockIdx.x + 1) * T / gridDim.x);
-        wk.ngr = ngr;
-        if (copier && tid == CONSUMERS) r_load_scores<G>(P, wk, pre, 0);
-        __syncthreads();
-        // first pass: bins; then the threshold bin's tokens are gathered and
-        // selected inside one CTA per head, or, for a bin of more than
-        // CAND_CAP tokens, refined by four more passes over all scores
-        if (!copier) r_pass<G, RP_BINS>(P, wk, pre, tid);
-        ok = gsync();
-        if (ok && !copier)
-            for (int hx = blockIdx.x; hx < (int)nrad; hx += gridDim.x) {
-                const uint32_t e = __ldcg(P.rlist + hx);
-                const long long tq = clock64();
-                r_digit<G, RP_BINS>(P, (int)(e >> 16), (int)(e & 0xFFFFu), tid);
-                if (tid == 0 && P.dbg_trace) S.acct[37 - 16] += (unsigned long long)(clock64() - tq);
+        const int NT = pre[nrad];
+        const int t0 = (int)((long long)blockIdx.x * NT / gridDim.x);
+        const int t1 = (int)((long long)(blockIdx.x + 1) * NT / gridDim.x);
+        uint32_t seq = 0;   // score copies this CTA has waited for
+        // the range's head segments: head hx, its tiles [c0, c1)
+        auto segment = [&](int t, int& hx, int& b, int& slot, int& c0, int& c1, int& nch) {
+            hx = last_le(pre, (int)nrad + 1, t);
+            const uint32_t e = __ldcg(P.rlist + hx);
+            b = (int)(e >> 16);
+            slot = (int)(e & 0xFFFFu);
+            nch = pre[hx + 1] - pre[hx];
+            c0 = t - pre[hx];
+            c1 = min(nch, t1 - pre[hx]);
+        };
+        if (!copier) {
+            const long long ta = clock64();
+            for (int t = t0; t < t1 && S.abort == 0;) {
+                int hx, b, slot, c0, c1, nch;
+                segment(t, hx, b, slot, c0, c1, nch);
+                const int64_t bs = (int64_t)b * P.n_ret + slot;
+                h_pass<G, RP_BINS>(P, b, slot, load_rhead(P.hs + bs), c0, c1, true, seq, tid);
+                if (tid == 0) atomicAdd(P.sel_arrive + 2 * bs, (uint32_t)(c1 - c0));
+                t = pre[hx] + c1;
             }
-        ok = ok && gsync();
-        if (tid == 0) trace_max(P, 14);
-        if (ok) {
-            if (!copier) r_pass<G, RP_COMPACT>(P, wk, pre, tid);
-            ok = gsync();
-        }
-        if (ok && !copier)
-            for (int hx = blockIdx.x; hx < (int)nrad; hx += gridDim.x) {
-                const uint32_t e = __ldcg(P.rlist + hx);
+            if (tid == 0 && P.dbg_trace) S.acct[37 - 16] += (unsigned long long)(clock64() - ta);
+            if (tid == 0) trace_max(P, 14);
+            for (int t = t0; t < t1 && S.abort == 0;) {
                 const long long tq = clock64();
-                const int64_t bsx = (int64_t)(e >> 16) * P.n_ret + (e & 0xFFFFu);
-                if (__ldcg(&P.hs[bsx].n_cand) <= 8u * CONSUMERS)
-                    r_local_select<G, 8>(P, (int)(e >> 16), (int)(e & 0xFFFFu), tid);
-                else
-                    r_local_select<G, CAND_CAP / CONSUMERS>(P, (int)(e >> 16), (int)(e & 0xFFFFu), tid);
+                int hx, b, slot, c0, c1, nch;
+                segment(t, hx, b, slot, c0, c1, nch);
+                t = pre[hx] + c1;
+                const int64_t bs = (int64_t)b * P.n_ret + slot;
+                // every tile of the head has added its bins
+                if (tid == 0 && !wait_counter(P.sel_arrive + 2 * bs, (uint32_t)nch)) {
+                    set_status(P, ST_TIMEOUT);
+                    S.abort = 1;
+                }
+                consumer_sync();
+                if (S.abort) break;
+                for (int d = tid; d < 256; d += CONSUMERS) {
+                    S.dcnt[d] = __ldcg(P.sel_cnt + bs * 256 + d);
+                    S.dmass[d] = __ldcg(P.sel_mass + bs * 256 + d);
+                }
+                consumer_sync();
+                // the threshold bin (every range alike; the one holding tile 0 publishes it)
+                r_digit<G, RP_BINS>(P, b, slot, tid, c0 == 0);
+                if (S.hst.n_cand <= (uint32_t)CAND_CAP) {
+                    RHead rh = load_rhead(P.hs + bs);
+                    rh.bstar = S.hst.bstar;
+                    h_pass<G, RP_COMPACT>(P, b, slot, rh, c0, c1, true, seq, tid);
+                }
+                if (tid == 0) {
+                    __threadfence();
+                    S.flag = atomicAdd(P.sel_arrive + 2 * bs + 1, (uint32_t)(c1 - c0)) + (uint32_t)(c1 - c0) ==
+                                     (uint32_t)nch ? 1u : 0u;
+                    if (S.flag) __threadfence();
+                }
+                consumer_sync();
                 if (tid == 0 && P.dbg_trace) S.acct[38 - 16] += (unsigned long long)(clock64() - tq);
+                if (!S.flag || S.abort) continue;
+                // this CTA completed the head's last tiles
+                const long long tf = clock64();
+                h_finish<G>(P, b, slot, seq, tid);
+                if (S.abort) break;
+                const int rg = S.tab.slot_rg[slot];
+                if (tid == 0) {
+                    const int slot0 = S.tab.rg_slot0[rg], nh = S.tab.rg_nh[rg];
+                    uint32_t nrh = 0;
+                    for (int hh = 0; hh < nh; ++hh)
+                        nrh += __ldcg(&P.hs[(int64_t)b * P.n_ret + slot0 + hh].mode) == MODE_RADIX ? 1u : 0u;
+                    __threadfence();
+                    const int bg = b * P.n_rg + rg;
+                    S.flag = atomicAdd(P.tick_grp + bg, 1u) + 1 == nrh ? 1u : 0u;
+                    if (S.flag) {
+                        __threadfence();
+                        P.tick_grp[bg] = 0;   // re-armed for the next call
+                    }
+                }
+                consumer_sync();
+                if (S.flag) r_blist<G>(P, b, rg, tid);
+                if (tid == 0 && P.dbg_trace) S.acct[39 - 16] += (unsigned long long)(clock64() - tf);
             }
-        if (ok) ok = gsync();
-        if (tid == 0) trace_max(P, 8);
-        const bool global = ok && __ldcg(&P.sync->any_global) != 0;
-        for (int pass = RP_REF0; global && pass <= RP_REF3 && ok; ++pass) {
-            if (!copier) {
-                if (pass == RP_REF0) r_pass<G, RP_REF0>(P, wk, pre, tid);
-                else if (pass == RP_REF1) r_pass<G, RP_REF1>(P, wk, pre, tid);
-                else if (pass == RP_REF2) r_pass<G, RP_REF2>(P, wk, pre, tid);
-                else r_pass<G, RP_REF3>(P, wk, pre, tid);
-            }
-            ok = gsync();
-            if (!ok) break;
-            if (!copier)
-                for (int hx = blockIdx.x; hx < (int)nrad; hx += gridDim.x) {
-                    const uint32_t e = __ldcg(P.rlist + hx);
-                    const int64_t bs = (int64_t)(e >> 16) * P.n_ret + (e & 0xFFFFu);
-                    if (__ldcg(&P.hs[bs].n_cand) > (uint32_t)CAND_CAP)
-                        if (pass == RP_REF0) r_digit<G, RP_REF0>(P, (int)(e >> 16), (int)(e & 0xFFFFu), tid);
-                        else if (pass == RP_REF1) r_digit<G, RP_REF1>(P, (int)(e >> 16), (int)(e & 0xFFFFu), tid);
-                        else if (pass == RP_REF2) r_digit<G, RP_REF2>(P, (int)(e >> 16), (int)(e & 0xFFFFu), tid);
-                        else r_digit<G, RP_REF3>(P, (int)(e >> 16), (int)(e & 0xFFFFu), tid);
-                }
-            ok = gsync();
-            if (tid == 0) trace_max(P, 8 + pass - RP_REF0);
         }
-        if (ok && __ldcg(&P.sync->any_ties)) {
-            if (!copier) r_pass<G, RP_TIES>(P, wk, pre, tid);
-            ok = gsync();
-            if (ok && !copier)
-                for (int hx = blockIdx.x; hx < (int)nrad; hx += gridDim.x) {
-                    const uint32_t e = __ldcg(P.rlist + hx);
-                    const int64_t bs = (int64_t)(e >> 16) * P.n_ret + (e & 0xFFFFu);
-                    if (__ldcg(&P.hs[bs].n_cand) > (uint32_t)CAND_CAP)
-                        r_tie_locate<G>(P, (int)(e >> 16), (int)(e & 0xFFFFu), tid);
-                }
-            ok = ok && gsync();
-        }
-        if (ok) {
-            if (!copier) r_pass<G, RP_MARK>(P, wk, pre, tid);
-            ok = gsync();
-            if (tid == 0) trace_max(P, 12);
-        }
-        if (ok) {
-            if (!copier)
-                for (int i = blockIdx.x; i < ngr; i += gridDim.x) {
-                    int b, rg;
-                    radix_group(P, i, b, rg);
-                    const long long tq = clock64();
-                    r_blist<G>(P, b, rg, tid);
-                    if (tid == 0 && P.dbg_trace) S.acct[39 - 16] += (unsigned long long)(clock64() - tq);
-                }
-            ok = gsync();
-        }
+        if (tid == 0) trace_max(P, 12);
+        ok = gsync();
     }
     if (tid == 0) trace_max(P, 3);
     if (ok && work) {

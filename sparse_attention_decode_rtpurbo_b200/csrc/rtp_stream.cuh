@@ -425,9 +425,6 @@ __device__ __forceinline__ void decide_group_body(const KParams& K, ASmem<G>& S,
         }
     }
     const int bg = b * P.n_rg + rg;
-    // (the exact select's histograms are zero already: they lie in the
-    // workspace region every call leaves at zero, the digit step clears each
-    // after reading it, and an aborted call clears them all)
     // bitmap words of the heads (read by the block-list builder of a group
     // with radix heads, and by the debug sink)
     if (any_radix || P.dbg_bitmap != nullptr) {

@@ -84,7 +84,8 @@ struct BSmem {
     unsigned long long dmass[256];
     uint32_t dcnt[256];
     uint32_t tcnt[MAX_G];
-    uint32_t hcand;   // candidates gathered by a compaction pass of this CTA alone
+    uint32_t hcand;   // candidates gathered by a compaction pass of this CTA alone (or by the warp finish)
+    uint32_t lw_key[32], lw_idx[32];   // the in-bin select's last bucket, finished by one warp
     HeadState hst;    // the head's select state as this CTA's digit step computed it
     uint32_t lsel_prefix, lsel_count, lsel_neq;
     unsigned long long lsel_mass, lsel_meq;
@@ -566,7 +567,10 @@ __device__ __noinline__ void r_local_select(const Params& P, int b, int slot, in
     }
     const unsigned long long target = __ldcg(&P.hs[bs].target);
     const bool unit = P.topk > 0;   // static top-k: every token weighs 1
-    for (int rp = rp0; rp < 4; ++rp) {
+    // digits resolved when a bucket of at most 32 candidates is left: one warp
+    // then finishes it (below); -1 while the digit rounds go on
+    int depth = n <= 32 ? rp0 : -1;
+    for (int rp = rp0; rp < 4 && depth < 0; ++rp) {
         for (int d = tid; d < 256; d += CONSUMERS) {
             S.H.cnt[0][d] = 0;
             S.H.m[0][0][d] = 0;
@@ -595,6 +599,78 @@ __device__ __noinline__ void r_local_select(const Params& P, int b, int slot, in
             S.lsel_meq = hist_mass(S.H, 0, dstar);
         }
         consumer_sync();
+        if (rp < 3 && S.lsel_neq <= 32u) depth = rp + 1;
+    }
+    auto publish = [&](uint32_t tau, uint32_t n_eq, uint32_t n_tie, uint32_t tie_idx, uint32_t count_above) {
+        HeadState* h = P.hs + bs;
+        h->tau_key = tau;
+        h->n_eq = n_eq;
+        h->n_tie = n_tie;
+        h->all_ties = n_tie == n_eq ? 1u : 0u;
+        h->tie_idx = tie_idx;
+        h->kstar = count_above + n_tie;
+        const int bh = b * P.Hq + S.tab.slot_head[slot];
+        if (P.dbg_tau) P.dbg_tau[bh] = key2f(tau);
+        if (P.dbg_kstar) P.dbg_kstar[bh] = (int32_t)(count_above + n_tie);
+    };
+    if (depth >= 0) {
+        // The bucket (candidates that share the `depth` leading key bytes
+        // found so far; it completes the target) in one warp: sorted by (key
+        // desc, index asc), the order the select keeps tokens in, its masses
+        // summed in that order; the first candidate that brings the mass above
+        // the bucket to the target is the last one kept.
+        const uint32_t prefix = S.lsel_prefix;
+        if (tid == 0) S.hcand = 0;
+        consumer_sync();
+#pragma unroll
+        for (int j = 0; j < CPT; ++j) {
+            if (tid + j * CONSUMERS >= n || (depth > 0 && (keys[j] >> (32 - 8 * depth)) != prefix)) continue;
+            const uint32_t pos = atomicAdd(&S.hcand, 1u);
+            if (pos < 32u) {
+                S.lw_key[pos] = keys[j];
+                S.lw_idx[pos] = idx[j];
+            }
+        }
+        consumer_sync();
+        if (tid < 32) {
+            const int lane = tid;
+            const uint32_t m = min(S.hcand, 32u);
+            bool v = (uint32_t)lane < m;
+            uint32_t k = v ? S.lw_key[lane] : 0u, x = v ? S.lw_idx[lane] : 0xFFFFFFFFu;
+            // bitonic sort over the 32 lanes; a valid entry precedes an empty one
+#pragma unroll
+            for (int kk = 2; kk <= 32; kk <<= 1) {
+#pragma unroll
+                for (int jj = kk >> 1; jj > 0; jj >>= 1) {
+                    const uint32_t ok = __shfl_xor_sync(0xffffffffu, k, jj), ox = __shfl_xor_sync(0xffffffffu, x, jj);
+                    const bool ov = __shfl_xor_sync(0xffffffffu, v ? 1 : 0, jj) != 0;
+                    const bool self_first = v && (!ov || k > ok || (k == ok && x < ox));
+                    const bool take_first = ((lane & jj) == 0) == ((lane & kk) == 0);
+                    if (take_first ? !self_first : self_first) {
+                        k = ok;
+                        x = ox;
+                        v = ov;
+                    }
+                }
+            }
+            unsigned long long inc = v ? (unit ? 1ull : fixmass(k, smax)) : 0ull;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const unsigned long long t = __shfl_up_sync(0xffffffffu, inc, o);
+                if (lane >= o) inc += t;
+            }
+            const unsigned long long base = S.lsel_mass;
+            const uint32_t hb = __ballot_sync(0xffffffffu, v && base + inc >= target);
+            const int hit = hb ? __ffs(hb) - 1 : (int)m - 1;   // (the bucket completes the target)
+            const uint32_t tau = __shfl_sync(0xffffffffu, k, hit), tie_x = __shfl_sync(0xffffffffu, x, hit);
+            const uint32_t eq = __ballot_sync(0xffffffffu, v && k == tau);
+            const uint32_t upto = hit == 31 ? 0xFFFFFFFFu : ((2u << hit) - 1u);
+            const uint32_t n_eq = __popc(eq), n_tie = __popc(eq & upto);
+            const uint32_t above = __popc(__ballot_sync(0xffffffffu, v && k > tau));
+            if (lane == 0) publish(tau, n_eq, n_tie, n_tie == n_eq ? 0xFFFFFFFFu : tie_x, S.lsel_count + above);
+        }
+        consumer_sync();
+        return;
     }
     const uint32_t tau = S.lsel_prefix, n_eq = S.lsel_neq, count_above = S.lsel_count;
     uint32_t n_tie = n_eq;
@@ -637,18 +713,7 @@ __device__ __noinline__ void r_local_select(const Params& P, int b, int slot, in
         }
         tie_idx = S.lsel_prefix;
     }
-    if (tid == 0) {
-        HeadState* h = P.hs + bs;
-        h->tau_key = tau;
-        h->n_eq = n_eq;
-        h->n_tie = n_tie;
-        h->all_ties = n_tie == n_eq ? 1u : 0u;
-        h->tie_idx = tie_idx;
-        h->kstar = count_above + n_tie;
-        const int bh = b * P.Hq + S.tab.slot_head[slot];
-        if (P.dbg_tau) P.dbg_tau[bh] = key2f(tau);
-        if (P.dbg_kstar) P.dbg_kstar[bh] = (int32_t)(count_above + n_tie);
-    }
+    if (tid == 0) publish(tau, n_eq, n_tie, tie_idx, count_above);
     consumer_sync();
 }
 

@@ -103,11 +103,13 @@ struct Params {
     uint32_t *tick_score, *tick_local, *tick_ret;
     uint32_t* tick_grp;   // [B * n_rg] radix heads of the group done with their select (zero between calls)
     // the exact select's per-head global state (zero between calls): merged
-    // first-pass histogram (count, 2^-40 mass), gathered candidates, and the
-    // units that have added their bins / finished their compaction
+    // first-pass histogram (2^-40 mass; counts only from a CTA that held the
+    // whole head), gathered candidates, and the tiles that have added their
+    // bins / finished their compaction
     uint32_t* sel_cnt;                // [B * n_ret, 256]
     unsigned long long* sel_mass;     // [B * n_ret, 256]
-    uint32_t* sel_ncand;              // [B * n_ret]
+    uint32_t* sel_ncand;              // [B * n_ret] tokens in the threshold bin (all gathered up to CAND_CAP)
+    uint32_t* sel_above;              // [B * n_ret] tokens above the threshold bin
     uint32_t* sel_arrive;             // [B * n_ret, 2]
     HeadAgg* agg;
     HeadState* hs;

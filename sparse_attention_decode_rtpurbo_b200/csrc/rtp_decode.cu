@@ -33,7 +33,7 @@ struct Plan {
     uint8_t lg_group[MAX_HKV], lg_mask[MAX_HKV];
     uint8_t slot_head[MAX_HQ], slot_rg[MAX_HQ];
     // workspace byte offsets; [0, zero_end) must be zero when a call starts
-    size_t o_status, o_sync, o_tick_score, o_tick_local, o_tick_ret, o_tick_grp, o_agg, o_sel_cnt, o_sel_mass, o_sel_ncand, o_sel_arrive, zero_end;
+    size_t o_status, o_sync, o_tick_score, o_tick_local, o_tick_ret, o_tick_grp, o_agg, o_sel_cnt, o_sel_mass, o_sel_ncand, o_sel_above, o_sel_arrive, zero_end;
     size_t o_rlist, o_rglist, o_hs, o_tie_cnt, o_scores, o_cand, o_bitmap, o_blist, o_bcount, o_lpart, o_rpart, total;
 };
 
@@ -122,6 +122,7 @@ static rtp_status make_plan(const rtp_dims* d, const uint8_t* head_kind, int win
     pl->o_sel_cnt = take(BR * 256 * 4);
     pl->o_sel_mass = take(BR * 256 * 8);
     pl->o_sel_ncand = take(BR * 4);
+    pl->o_sel_above = take(BR * 4);
     pl->o_sel_arrive = take(BR * 2 * 4);
     pl->zero_end = o;
     pl->o_rlist = take(BR * 4);
@@ -426,6 +427,7 @@ static rtp_status decode_step_ws(const rtp_dims* dims, const uint16_t* q_pre, co
     P.sel_cnt = (uint32_t*)(ws + pl.o_sel_cnt);
     P.sel_mass = (unsigned long long*)(ws + pl.o_sel_mass);
     P.sel_ncand = (uint32_t*)(ws + pl.o_sel_ncand);
+    P.sel_above = (uint32_t*)(ws + pl.o_sel_above);
     P.sel_arrive = (uint32_t*)(ws + pl.o_sel_arrive);
     P.agg = (HeadAgg*)(ws + pl.o_agg);
     P.hs = (HeadState*)(ws + pl.o_hs);

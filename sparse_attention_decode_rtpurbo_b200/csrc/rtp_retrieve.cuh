@@ -66,6 +66,14 @@ __device__ __forceinline__ void hist_add(RHist<G>& H, int h, int d, uint32_t n, 
     atomicAdd(&H.m[1][h][d], (uint32_t)((ms >> 16) & 0xFFFFull));
     atomicAdd(&H.m[2][h][d], (uint32_t)(ms >> 32));
 }
+// The mass alone (the spread first pass: its bin counts are not needed, the
+// threshold bin's size and the count above it come from the compaction).
+template <int G>
+__device__ __forceinline__ void hist_add_mass(RHist<G>& H, int h, int d, unsigned long long ms) {
+    atomicAdd(&H.m[0][h][d], (uint32_t)(ms & 0xFFFFull));
+    atomicAdd(&H.m[1][h][d], (uint32_t)((ms >> 16) & 0xFFFFull));
+    atomicAdd(&H.m[2][h][d], (uint32_t)(ms >> 32));
+}
 template <int G>
 __device__ __forceinline__ unsigned long long hist_mass(const RHist<G>& H, int h, int d) {
     return (unsigned long long)H.m[0][h][d] + ((unsigned long long)H.m[1][h][d] << 16) +
@@ -86,6 +94,7 @@ struct BSmem {
     uint32_t tcnt[MAX_G];
     uint32_t hcand;   // candidates gathered by a compaction pass of this CTA alone (or by the warp finish)
     uint32_t lw_key[32], lw_idx[32];   // the in-bin select's last bucket, finished by one warp
+    uint32_t fin_tau, fin_tie;         // the in-bin select's result: tau and the largest tie index kept
     HeadState hst;    // the head's select state as this CTA's digit step computed it
     uint32_t lsel_prefix, lsel_count, lsel_neq;
     unsigned long long lsel_mass, lsel_meq;
@@ -264,6 +273,7 @@ __device__ __noinline__ void h_pass(const Params& P, int b, int slot, const RHea
         const int c = c0 + k;
         const int n0 = c * HS_CHUNK, nv = min(HS_CHUNK, L - n0);
         uint32_t w0 = 0u;        // RP_COMPACT / RP_MARK: bits of blocks n0/64 + 0..15
+        uint32_t n_above = 0u;   // RP_COMPACT: the warp's tokens above the threshold bin (lane 0)
         uint32_t tcount = 0u;    // RP_TIES: threshold ties of this thread in the tile
 #pragma unroll
         for (int u = 0; u < HS_U; ++u) {
@@ -276,7 +286,8 @@ __device__ __noinline__ void h_pass(const Params& P, int b, int slot, const RHea
                     const uint32_t bn = score_bin(v, rh.smax, rh.dr, rh.inv_w);
                     const unsigned long long ms = unit ? 1ull : fixmass(key, rh.smax);
                     if (bn < 255u) {
-                        hist_add(S.H, 0, (int)bn, 1u, ms);
+                        if (unit_of_many) hist_add_mass(S.H, 0, (int)bn, ms);
+                        else hist_add(S.H, 0, (int)bn, 1u, ms);
                     } else {
                         ovf_n += 1u;
                         ovf_m += ms;
@@ -308,13 +319,18 @@ __device__ __noinline__ void h_pass(const Params& P, int b, int slot, const RHea
                     keep = ok && (key > rh.tau || (key == rh.tau && (uint32_t)(n0 + r) <= rh.tie_idx));
                 }
                 // block of the warp's 32 scores within the tile: 2 u + warp / 2
-                if (__any_sync(0xffffffffu, keep)) w0 |= 1u << (2 * u + (warp >> 1));
+                const uint32_t kb = __ballot_sync(0xffffffffu, keep);
+                if (kb) w0 |= 1u << (2 * u + (warp >> 1));
+                n_above += __popc(kb);
             }
         }
         if constexpr (pass == RP_COMPACT || pass == RP_MARK) {
             // the blocks straight into the head's bitmap (zeroed when the
             // group was registered for the select)
             if (lane == 0 && w0) atomicOr(bmp + c / 2, w0 << ((c & 1) * 16));
+            if constexpr (pass == RP_COMPACT) {
+                if (unit_of_many && lane == 0 && n_above) atomicAdd(P.sel_above + bs, n_above);
+            }
         } else if constexpr (pass == RP_TIES) {
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) tcount += __shfl_xor_sync(0xffffffffu, tcount, o);
@@ -361,10 +377,9 @@ __device__ __noinline__ void h_pass(const Params& P, int b, int slot, const RHea
             // the unit's bins into the head's global histogram
             for (int d = tid; d < 256; d += CONSUMERS) {
                 const uint32_t n = S.dcnt[d];
-                if (n) {
-                    atomicAdd(P.sel_cnt + bs * 256 + d, n);
-                    atomicAdd(P.sel_mass + bs * 256 + d, S.dmass[d]);
-                }
+                const unsigned long long m = S.dmass[d];
+                if (n) atomicAdd(P.sel_cnt + bs * 256 + d, n);
+                if (m) atomicAdd(P.sel_mass + bs * 256 + d, m);
             }
         }
     }
@@ -512,14 +527,16 @@ __device__ __noinline__ void r_digit(const Params& P, int b, int slot, int tid, 
 
 // Threshold of a radix head whose threshold bin holds at most CAND_CAP
 // tokens, inside one CTA: the bin's (key, index) pairs, gathered by the
-// compaction pass, go to shared memory; four 8-bit MSD passes over the keys
-// (count and fixed-point mass per digit, cumulative from the mass above the
-// bin) give tau and the number of its ties to keep, and a four-pass select
-// over the tie indices gives the largest tie index kept (ties toward the
-// lower index).  CPT candidates per thread, kept in registers: an instance
-// for at most 1024 candidates (8 per thread) and one for CAND_CAP; the
-// smaller one is a quarter of the code, which matters for code that runs
-// once per head and per step.
+// compaction, are held in registers; 8-bit MSD passes over the keys (count
+// and fixed-point mass per digit, cumulative from the mass above the bin)
+// narrow them to the digit bucket that completes the target, one warp
+// finishes a bucket of at most 32 (sorted by key desc, index asc), and only
+// more than 32 exact ties take the four-pass select over the tie indices
+// (ties toward the lower index).  The kept candidates' blocks then go into
+// the head's bitmap.  CPT candidates per thread: an instance for at most
+// 1024 candidates (8 per thread) and one for CAND_CAP; the smaller one is a
+// quarter of the code, which matters for code that runs once per head and
+// per step.
 template <int G, int CPT>
 __device__ __noinline__ void r_local_select(const Params& P, int b, int slot, int tid) {
     BSmem<G>& S = bsmem<G>();
@@ -602,6 +619,8 @@ __device__ __noinline__ void r_local_select(const Params& P, int b, int slot, in
         if (rp < 3 && S.lsel_neq <= 32u) depth = rp + 1;
     }
     auto publish = [&](uint32_t tau, uint32_t n_eq, uint32_t n_tie, uint32_t tie_idx, uint32_t count_above) {
+        S.fin_tau = tau;
+        S.fin_tie = tie_idx;
         HeadState* h = P.hs + bs;
         h->tau_key = tau;
         h->n_eq = n_eq;
@@ -612,6 +631,20 @@ __device__ __noinline__ void r_local_select(const Params& P, int b, int slot, in
         const int bh = b * P.Hq + S.tab.slot_head[slot];
         if (P.dbg_tau) P.dbg_tau[bh] = key2f(tau);
         if (P.dbg_kstar) P.dbg_kstar[bh] = (int32_t)(count_above + n_tie);
+    };
+    // the blocks of the kept candidates (key above tau, or tau with an index up
+    // to the largest tie kept) into the head's bitmap, from the registers
+    auto mark_kept = [&]() {
+        const uint32_t tau = S.fin_tau, tie = S.fin_tie;
+        uint32_t* const bmp = P.bitmap + bs * P.words_cap;
+#pragma unroll
+        for (int j = 0; j < CPT; ++j) {
+            if (tid + j * CONSUMERS >= n) continue;
+            const uint32_t key = keys[j], x = idx[j];
+            if (key > tau || (key == tau && x <= tie)) atomicOr(bmp + (x >> 11), 1u << ((x >> 6) & 31));
+        }
+        __threadfence();   // bitmap bits before the group ticket
+        consumer_sync();
     };
     if (depth >= 0) {
         // The bucket (candidates that share the `depth` leading key bytes
@@ -670,6 +703,7 @@ __device__ __noinline__ void r_local_select(const Params& P, int b, int slot, in
             if (lane == 0) publish(tau, n_eq, n_tie, n_tie == n_eq ? 0xFFFFFFFFu : tie_x, S.lsel_count + above);
         }
         consumer_sync();
+        mark_kept();
         return;
     }
     const uint32_t tau = S.lsel_prefix, n_eq = S.lsel_neq, count_above = S.lsel_count;
@@ -715,6 +749,7 @@ __device__ __noinline__ void r_local_select(const Params& P, int b, int slot, in
     }
     if (tid == 0) publish(tau, n_eq, n_tie, tie_idx, count_above);
     consumer_sync();
+    mark_kept();
 }
 
 // For a radix head that keeps only n_tie of its n_eq threshold ties: find the
@@ -770,24 +805,6 @@ __device__ __noinline__ void r_tie_locate(const Params& P, int b, int slot, int 
     consumer_sync();
 }
 
-// After the select inside the CTA: the blocks of the kept candidates (key
-// above tau, or tau with an index up to the largest tie kept) into the head's
-// bitmap.
-template <int G>
-__device__ __noinline__ void h_mark_cand(const Params& P, int b, int slot, int tid) {
-    const int64_t bs = (int64_t)b * P.n_ret + slot;
-    const uint32_t n = min(__ldcg(&P.hs[bs].n_cand), (uint32_t)CAND_CAP);
-    const uint32_t tau = __ldcg(&P.hs[bs].tau_key), tie = __ldcg(&P.hs[bs].tie_idx);
-    uint32_t* const bmp = P.bitmap + bs * P.words_cap;
-    for (uint32_t i = (uint32_t)tid; i < n; i += CONSUMERS) {
-        const unsigned long long c = __ldcg(P.cand + bs * CAND_CAP + i);
-        const uint32_t key = (uint32_t)(c >> 32), idx = (uint32_t)(c & 0xFFFFFFFFull);
-        if (key > tau || (key == tau && idx <= tie)) atomicOr(bmp + (idx >> 11), 1u << ((idx >> 6) & 31));
-    }
-    __threadfence();   // bitmap bits before the group ticket
-    consumer_sync();
-}
-
 // The end of the select of radix head (b, slot), by the CTA that finished the
 // head's last unit: with at most CAND_CAP tokens in the threshold bin (all
 // gathered by the units' compactions, which also marked the blocks above
@@ -799,11 +816,16 @@ template <int G>
 __device__ __noinline__ void h_finish(const Params& P, int b, int slot, uint32_t& seq, int tid) {
     BSmem<G>& S = bsmem<G>();
     const int64_t bs = (int64_t)b * P.n_ret + slot;
-    const uint32_t ncand = __ldcg(&P.hs[bs].n_cand);
+    // the threshold bin's size and the tokens above it, as the ranges counted them
+    const uint32_t ncand = __ldcg(P.sel_ncand + bs);
+    if (tid == 0) {
+        P.hs[bs].n_cand = ncand;
+        P.hs[bs].count_above = __ldcg(P.sel_above + bs);
+    }
+    consumer_sync();
     if (ncand <= (uint32_t)CAND_CAP) {
         if (ncand <= 8u * CONSUMERS) r_local_select<G, 8>(P, b, slot, tid);
         else r_local_select<G, CAND_CAP / CONSUMERS>(P, b, slot, tid);
-        h_mark_cand<G>(P, b, slot, tid);
     } else {
         const int nch = (__ldg(P.seq_lens + b) + HS_CHUNK - 1) / HS_CHUNK;
         h_pass<G, RP_REF0>(P, b, slot, load_rhead(P.hs + bs), 0, nch, false, seq, tid);
@@ -826,6 +848,7 @@ __device__ __noinline__ void h_finish(const Params& P, int b, int slot, uint32_t
     }
     if (tid == 0) {
         P.sel_ncand[bs] = 0;
+        P.sel_above[bs] = 0;
         P.sel_arrive[2 * bs] = 0;
         P.sel_arrive[2 * bs + 1] = 0;
     }
@@ -1096,6 +1119,7 @@ __device__ __noinline__ void clear_call_words(const Params& P) {
                 P.sel_mass[i * 256 + d] = 0ull;
             }
             P.sel_ncand[i] = 0;
+            P.sel_above[i] = 0;
             P.sel_arrive[2 * i] = 0;
             P.sel_arrive[2 * i + 1] = 0;
         }
@@ -1208,7 +1232,10 @@ __device__ __forceinline__ void r_body(const KParams& K, bool single) {
                 consumer_sync();
                 // the threshold bin (every range alike; the one holding tile 0 publishes it)
                 r_digit<G, RP_BINS>(P, b, slot, tid, c0 == 0);
-                if (S.hst.n_cand <= (uint32_t)CAND_CAP) {
+                {
+                    // every range compacts (gathering at most CAND_CAP, counting
+                    // all): the bin's size and the count above it are known only
+                    // when the head's last range is done
                     RHead rh = load_rhead(P.hs + bs);
                     rh.bstar = S.hst.bstar;
                     h_pass<G, RP_COMPACT>(P, b, slot, rh, c0, c1, true, seq, tid);

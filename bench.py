@@ -591,7 +591,8 @@ def bench_prefill(args):
     except Exception:
         peak, peak_kind = 1590.0, "fallback"
     res = {}
-    kernel = "mma.sync m16n8k16 bf16" if os.environ.get("RTP_PREFILL_TC") == "0" else "tcgen05 (tensor memory, TMA)"
+    kernel = ("mma.sync m16n8k16 bf16" if os.environ.get("RTP_PREFILL_TC") == "0"
+              else "tcgen05, 128-key tiles, two row groups per CTA (tensor memory, TMA)")
     for name, hk in (("sparse", [1] * G + [0] * (Hkv - 1) * G), ("dense", [1] * (Hkv * G))):
         ts = []
         for i in range(args.warmup + args.steps):

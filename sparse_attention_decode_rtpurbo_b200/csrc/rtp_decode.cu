@@ -719,8 +719,8 @@ extern "C" rtp_status rtp_prefill(const rtp_dims* d, const uint16_t* q, const ui
     P.window = window;
     P.sink = sink;
     P.nt16 = (num_q + 15) / 16;
-    // the tcgen05 kernel, eight units per CTA; RTP_PREFILL_TC=0 (read at every
-    // call): the warp-MMA kernel, four
+    // the tcgen05 kernel, sixteen units per CTA; RTP_PREFILL_TC=0 (read at
+    // every call): the warp-MMA kernel, four
     const char* tcv = getenv("RTP_PREFILL_TC");
     const bool tc = !(tcv && atoi(tcv) == 0);
     const int units = tc ? PT_UNITS : PF_UNITS;

@@ -1,58 +1,43 @@
-// Prefill attention on the 5th-generation tensor cores (sm_100a): the same
-// operation as prefill_kernel (rtp_prefill.cuh: retrieval heads dense and
-// causal, local heads sink + window; review "RTPurbo" on
-// dongryeollee1.github.io, Method: "Adaptive sparse attention", the prefill
-// paragraph), with the two contractions on tcgen05 and their accumulators
-// in tensor memory.
+// Prefill attention on the 5th-generation tensor cores (sm_100a), with
+// 128-key tiles and two row groups per CTA: the same operation as
+// prefill_kernel (rtp_prefill.cuh: retrieval heads dense and causal, local
+// heads sink + window; review "RTPurbo" on dongryeollee1.github.io, Method:
+// "Adaptive sparse attention", the prefill paragraph), with both
+// contractions on tcgen05 and their accumulators in tensor memory.
 //
-// A CTA takes eight (head, 16-position) units of one (KV group, head kind)
-// set: M = 128 query rows that all read the same KV head.  Per 64-key tile:
-//   S = Q K^T       tcgen05.mma M128 N64, K = 128 in eight K16 steps, S in
-//                   tensor memory (64 columns)
-//   softmax         four warps, thread i owns row i: tcgen05.ld of its 64
-//                   scores, mask, max, exp2, row sum in registers; P (bf16)
-//                   to shared memory as the A operand of the next MMA
-//   O += P V        tcgen05.mma M128 N128, K = 64 in four K16 steps, O in
-//                   tensor memory (128 columns)
-// (Build option RTP_PT_P_TMEM: P goes back to tensor memory and the P V MMA
-// reads its A operand from there; correct, and measured slower on the 32K
-// prompt, 393 against 420 TFLOP/s.)
-// K and V tiles arrive by TMA, each as two 64 x 64 boxes with the 128-byte
-// swizzle, and are read in place: K as the K-major B operand of Q K^T, V as
-// the MN-major B operand of P V (head dimension contiguous), so V needs no
-// transpose.  Q (cp.async, once per CTA) and P are unswizzled K-major core
-// matrices (8 rows x 16 bytes).  Pipeline per tile k: S_{k+1} is issued
-// before the softmax of tile k, and the TMA loads of K_{k+2} and V_{k+1}
-// (two buffers each) run meanwhile; one thread issues the loads and the
-// MMAs, and two CTAs per SM overlap the rest.
-// The online softmax keeps a reference maximum per row and rescales O in
-// tensor memory only when a tile's maximum exceeds it by more than 2^8
-// (P <= 256 then): the normalised result does not depend on the reference.
+// A CTA takes sixteen (head, 16-position) units of one (KV group, head kind)
+// set: two row groups of M = 128 query rows that read the same KV head, so a
+// 128-key K/V tile is loaded once for 256 rows.  One CTA per SM (192 KB of
+// shared memory, all 512 tensor-memory columns).  Warp roles:
+//   warps 0-7  softmax, row group rg = warp / 4, thread i of the group owns
+//              row i (tensor-memory lane i)
+//   warp 8     one lane issues every TMA load and every MMA
+// Per tile k and row group g, in tensor memory: S_g (128 fp32 columns), then
+// P_g (bf16 pairs) written over the first 64 of them, and O_g (128 columns).
+//   S_g = Q_g K^T   tcgen05.mma M128 N128, eight K16 steps over the head dim
+//   O_g += P_g V    tcgen05.mma M128 N128, eight K16 steps over the 128 keys,
+//                   A = P_g from tensor memory, B = V (MN-major)
+// The issuing lane orders, per tile: P V of tile k for group 0, S of tile
+// k + 1 for group 0 (it may overwrite P_0 only after that P V, and the tensor
+// cores run one lane's MMAs in order), then the same for group 1; so the
+// tensor cores compute one group's products while the other group's softmax
+// runs.  A group meets the issuing lane at two mbarriers per tile: S full
+// (commit; it also means the group's previous P V is done, so O_g may be
+// rescaled) and P full (the group's 128 threads).
+// K and V tiles arrive by TMA, two 64-key blocks per tile, each as two 64 x
+// 64 boxes with the 128-byte swizzle: box (head-dim half h, block b) at
+// h * 16384 + b * 8192, so each half holds 128 consecutive key rows.  A block
+// past the CTA's last query position is not loaded.
+// Per tile a softmax thread makes two passes over its 128 scores, 64 at a
+// time (the maximum, then 2^(s - m) into P), so its registers hold 64 scores.
 #pragma once
 #include "rtp_prefill.cuh"
 #include "rtp_tc.cuh"
 
 namespace rtp {
 
-constexpr int PT_UNITS = 8;                  // (head, 16 positions) units per CTA: M = 128 rows
-constexpr int PT_THREADS = 128;              // warp w owns rows (tensor-memory lanes) 32w .. 32w+31
 constexpr float PT_RESCALE = 8.f;            // log2 of the largest P before O is rescaled
-// tensor-memory columns: S, P (bf16 pairs), O
-constexpr uint32_t PT_TM_S = 0, PT_TM_P = 64, PT_TM_O = 128, PT_TM_COLS = 256;
 
-struct PtSmem {
-    alignas(1024) uint8_t q[128 * 128 * 2];      // Q: chunk (row r, dims 8c..) at c*2048 + r*16
-    // K / V tiles: box b (dims 64b..64b+63) at b*8192, key r at r*128, 16-byte
-    // chunk c of the row at ((c ^ r) % 8)*16 (the TMA's 128-byte swizzle)
-    alignas(1024) uint8_t k[2][64 * 128 * 2];
-    alignas(1024) uint8_t v[2][64 * 128 * 2];
-#ifndef RTP_PT_P_TMEM
-    alignas(1024) uint8_t p[128 * 64 * 2];      // P: chunk (row r, keys 8c..) at c*2048 + r*16
-#endif
-    alignas(8) uint64_t s_bar, o_bar;            // S = Q K^T / O += P V complete
-    alignas(8) uint64_t kfull[2], vfull[2];      // a K / V buffer's TMA loads have landed
-    uint32_t tmem_base;
-};
 
 __device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
     asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
@@ -121,7 +106,42 @@ __device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, u
         : "memory");
 }
 
-// The CTA's set, units and key tiles: as pf_cta, with PT_UNITS units.
+// bits [lo, hi) of a 64-bit word, the bounds clamped to [0, 64]
+__device__ __forceinline__ uint64_t pt_bits(int lo, int hi) {
+    lo = max(lo, 0);
+    hi = min(hi, 64);
+    if (hi <= lo) return 0ull;
+    const uint64_t below_hi = hi >= 64 ? ~0ull : ((1ull << hi) - 1ull);
+    return below_hi & ~((1ull << lo) - 1ull);
+}
+
+struct PrefillTcK {
+    CUtensorMap tmk, tmv;   // K / V caches as [rows][128] bf16, 64 x 64 boxes, 128-byte swizzle
+    PrefillParams P;
+};
+
+constexpr int PT_UNITS = 16;                 // (head, 16 positions) units per CTA: two groups of 128 rows
+constexpr int PT_SOFT = 256;                 // softmax threads (warps 0-7)
+constexpr int PT_THREADS = PT_SOFT + 32;     // + the TMA / MMA warp
+constexpr int PT_TK = 2 * BLK;               // keys per tile
+constexpr uint32_t PT_TM_COLS = 512;         // S_g / P_g at 128 g, O_g at 256 + 128 g
+
+struct PtSmem {
+    alignas(1024) uint8_t q[2][128 * 128 * 2];   // Q of group g: chunk (row r, dims 8c..) at c*2048 + r*16
+    alignas(1024) uint8_t k[2][PT_TK * 128 * 2];   // K tiles (two stages), layout above
+    alignas(1024) uint8_t v[2][PT_TK * 128 * 2];   // V tiles (two stages)
+    alignas(8) uint64_t q_full;                  // Q copied (every softmax thread)
+    uint64_t kfull[2], vfull[2];                 // TMA landed
+    uint64_t kempty[2], vempty[2];               // the MMAs reading the stage are done (commit)
+    uint64_t s_full[2];                          // [group] S computed, and the group's previous P V done
+    uint64_t p_full[2];                          // [group] P written and O rescaled (the group's threads)
+    uint64_t o_done[2];                          // [group] P V done (commit; its last phase gives the output)
+    uint32_t tmem_base;
+    volatile uint32_t abort;                     // a bounded wait gave up: every role leaves its loop
+};
+
+// The CTA's set, units and 128-key tiles (as pf_cta, with PT_UNITS units and
+// tiles of PT_TK keys).
 __device__ __forceinline__ PfCta pt_cta(const PrefillParams& P) {
     PfCta c;
     const int x = (int)blockIdx.x;
@@ -149,14 +169,14 @@ __device__ __forceinline__ PfCta pt_cta(const PrefillParams& P) {
     c.w_lo = max(0, c.m_lo + 1 - P.window);
     if (c.kind == 1) {
         c.j0a = 0;
-        c.j1a = c.m_hi / BLK + 1;
+        c.j1a = c.m_hi / PT_TK + 1;
         c.j0b = c.j1b = c.j1a;
     } else {
         c.j0a = 0;
-        c.j1a = (c.s_end + BLK - 1) / BLK;
+        c.j1a = (c.s_end + PT_TK - 1) / PT_TK;
         if (P.window > 0) {
-            c.j0b = max(c.j1a, c.w_lo / BLK);
-            c.j1b = max(c.j0b, c.m_hi / BLK + 1);
+            c.j0b = max(c.j1a, c.w_lo / PT_TK);
+            c.j1b = max(c.j0b, c.m_hi / PT_TK + 1);
         } else {
             c.j0b = c.j1b = c.j1a;
         }
@@ -164,30 +184,31 @@ __device__ __forceinline__ PfCta pt_cta(const PrefillParams& P) {
     return c;
 }
 
-// Global address of cache row `row` (from pf_row) of the K or V cache.
-__device__ __forceinline__ const uint8_t* pt_cache_row(const uint16_t* cache, int row) {
-    return reinterpret_cast<const uint8_t*>(cache) + (int64_t)row * (D * 2);
+// Bounded mbarrier wait shared by all roles: false once this or another
+// thread gave up (the CTA's abort flag), or after about two seconds (this
+// thread then raises the flag and reports the timeout).
+__device__ __forceinline__ bool pt_wait(uint64_t* bar, uint32_t parity, volatile uint32_t* abort,
+                                        const PrefillParams& P) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 31u) == 0) {
+            if (*abort) return false;
+            if (global_ns() - t0 > 2000000000ull) {
+                *abort = 1u;
+                pf_status(P, ST_TIMEOUT);
+                return false;
+            }
+        }
+    }
 }
 
-// bits [lo, hi) of a 64-bit word, the bounds clamped to [0, 64]
-__device__ __forceinline__ uint64_t pt_bits(int lo, int hi) {
-    lo = max(lo, 0);
-    hi = min(hi, 64);
-    if (hi <= lo) return 0ull;
-    const uint64_t below_hi = hi >= 64 ? ~0ull : ((1ull << hi) - 1ull);
-    return below_hi & ~((1ull << lo) - 1ull);
-}
-
-struct PrefillTcK {
-    CUtensorMap tmk, tmv;   // K / V caches as [rows][128] bf16, 64 x 64 boxes, 128-byte swizzle
-    PrefillParams P;
-};
-
-__global__ void __launch_bounds__(PT_THREADS, 2) prefill_tc_kernel(const __grid_constant__ PrefillTcK K) {
+__global__ void __launch_bounds__(PT_THREADS, 1) prefill_tc_kernel(const __grid_constant__ PrefillTcK K) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     PtSmem& S = *reinterpret_cast<PtSmem*>(smem_raw);
     const PrefillParams& P = K.P;
-    const int tid = threadIdx.x, warp = tid >> 5;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (smem_u32(smem_raw) & 1023u) {
         if (tid == 0) pf_status(P, 5u);
         return;
@@ -197,17 +218,19 @@ __global__ void __launch_bounds__(PT_THREADS, 2) prefill_tc_kernel(const __grid_
         if (tid == 0) pf_status(P, ST_DEVICE_INPUT);   // this sequence's outputs are not written
         return;
     }
-    const uint32_t qs = smem_u32(S.q);
-    const uint32_t kbuf[2] = {smem_u32(S.k[0]), smem_u32(S.k[1])};
-    const uint32_t vbuf[2] = {smem_u32(S.v[0]), smem_u32(S.v[1])};
     if (tid == 0) {
-        mbar_init(&S.s_bar, 1);
-        mbar_init(&S.o_bar, 1);
+        mbar_init(&S.q_full, PT_SOFT);
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
             mbar_init(&S.kfull[i], 1);
             mbar_init(&S.vfull[i], 1);
+            mbar_init(&S.kempty[i], 1);
+            mbar_init(&S.vempty[i], 1);
+            mbar_init(&S.s_full[i], 1);
+            mbar_init(&S.p_full[i], 128);
+            mbar_init(&S.o_done[i], 1);
         }
+        S.abort = 0u;
         mbar_fence_init();
     }
     if (warp == 0) tmem_alloc(&S.tmem_base, PT_TM_COLS);
@@ -215,221 +238,248 @@ __global__ void __launch_bounds__(PT_THREADS, 2) prefill_tc_kernel(const __grid_
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = S.tmem_base;
-    const uint32_t t_lane = tbase + ((uint32_t)(32 * warp) << 16);   // this warp's lanes
     const int nt = c.ntiles();
-
-    // ---- this thread's row: unit u0 + row / 16, position t
-    const int row = tid;
-    const int u = c.u0 + row / 16;
-    const int t = u < c.units ? 16 * (P.nt16 - 1 - u / c.nh) + (row & 15) : P.T;
-    const bool valid = u < c.units && t < P.T;
-    const int h = c.g * P.G + P.set_heads[c.set][valid ? u % c.nh : 0];
-    const int m = c.pos_b + t;
     const bool retr = c.kind == 1;
     const int window = P.window, sink = P.sink;
-    // this thread's row of a V tile to zero on an edge tile: key zr, box zb
-    const int zr = tid >> 1, zb = tid & 1;
 
-    constexpr float SCALE = 0.08838834764831845f * 1.4426950408889634f;   // log2(e)/sqrt(128)
-    constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 64);
-    constexpr uint32_t IDESC_O = idesc_bf16_f32(128, 128) | (1u << 16);   // B (V) MN-major
-    // a tile with every key visible to every row of the CTA needs no mask; an
-    // edge tile holds keys no row reads
-    auto interior = [&](int n0) {
-        return n0 + BLK - 1 <= c.m_lo && (retr || n0 + BLK - 1 < sink || n0 > c.m_hi - window);
-    };
-    auto edge = [&](int n0) { return n0 + BLK - 1 > c.m_hi || (!retr && n0 + BLK > c.s_end && n0 < c.w_lo); };
-    // TMA load of tile kt's K or V (two boxes) into buffer `dst` (thread 0)
-    auto load_tile = [&](const CUtensorMap* map, uint8_t* dst, uint64_t* bar, int kt) {
-        const int r0 = pf_row(P, c.b, c.g, c.tile(kt));
-        mbar_expect_tx(bar, 64 * 128 * 2);
-        tma_load_2d(dst, map, 0, r0, bar);
-        tma_load_2d(dst + 8192, map, 64, r0, bar);
-    };
-    // a bounded wait that gave up marks this thread; the CTA leaves the tile
-    // loop together at the next barrier that ORs the marks (__syncthreads_or)
-    bool bad = false;
-    auto wait_or_abort = [&](uint64_t* bar, uint32_t parity) {
-        if (!mbar_wait_bounded(bar, parity)) {
-            pf_status(P, ST_TIMEOUT);
-            bad = true;
-        }
-    };
-    auto issue_s = [&](uint32_t kb) {   // S = Q K^T
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-            umma_bf16(tbase + PT_TM_S, smem_desc(qs + kk * 4096, 2048, 128),
-                      smem_desc_sw128(kb + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), IDESC_S, kk > 0);
-        umma_commit(&S.s_bar);
-    };
-
-    // ---- prologue: tiles 0 and 1 and Q in flight; S_0
-    if (tid == 0)
-        for (int i = 0; i < 2 && i < nt; ++i) {
-            load_tile(&K.tmk, S.k[i], &S.kfull[i], i);
-            load_tile(&K.tmv, S.v[i], &S.vfull[i], i);
-        }
-    {
-        const uint8_t* qrow = reinterpret_cast<const uint8_t*>(P.q + (((int64_t)c.b * P.Hq + h) * P.T + t) * D);
-#pragma unroll
-        for (int ch = 0; ch < 16; ++ch) {
-            const uint32_t dst = qs + (uint32_t)(ch * 2048 + row * 16);
-            if (valid) cp_async16(dst, qrow + ch * 16);
-            else sts128(dst, 0u, 0u, 0u, 0u);
-        }
-    }
-    cp_async_wait_all();
-    fence_proxy_async();
-    tc_fence_before();
-    bool aborted = __syncthreads_or(bad) != 0;
-    if (nt > 0 && !aborted && tid == 0) {
-        wait_or_abort(&S.kfull[0], 0u);
-        if (!bad) issue_s(kbuf[0]);
-    }
-
-    float m_ref = -INFINITY, l = 0.f;
-    for (int k = 0; k < nt && !aborted; ++k) {
-        const int n0 = c.tile(k) * BLK;
-        // (1) S_k; its K buffer is free again: K_{k+2} goes there
-        wait_or_abort(&S.s_bar, (uint32_t)k & 1u);
-        tc_fence_after();
-        float s[64];
-        tmem_ld64(t_lane + PT_TM_S, s);
-        if (k + 2 < nt && tid == 0) load_tile(&K.tmk, S.k[k & 1], &S.kfull[k & 1], k + 2);
-        // (2) S_{k+1} on the tensor cores while this tile's softmax runs
-        if (k + 1 < nt) {
-            tc_fence_before();
-            if ((aborted = __syncthreads_or(bad) != 0)) break;   // every S_k is in registers
-            if (tid == 0) {
-                wait_or_abort(&S.kfull[(k + 1) & 1], (uint32_t)((k + 1) >> 1) & 1u);
-                if (!bad) issue_s(kbuf[(k + 1) & 1]);
+    if (warp == 8) {
+        // ================= TMA and MMA issue (lane 0; the warp zeroes unread value rows)
+        constexpr uint32_t IDESC = idesc_bf16_f32(128, 128);
+        constexpr uint32_t IDESC_O = IDESC | (1u << 16);   // B (V) MN-major
+        const bool leader = lane == 0;
+        // TMA of tile kt's K or V: its blocks up to the CTA's last query position
+        auto load_tile = [&](const CUtensorMap* map, uint8_t* dst, uint64_t* bar, int kt) {
+            const int j0 = 2 * c.tile(kt);
+            const int nb = (j0 + 1) * BLK <= c.m_hi ? 2 : 1;
+            mbar_expect_tx(bar, (uint32_t)nb * BLK * 128 * 2);
+            for (int bb = 0; bb < nb; ++bb) {
+                const int r0 = pf_row(P, c.b, c.g, j0 + bb);
+                tma_load_2d(dst + bb * 8192, map, 0, r0, bar);
+                tma_load_2d(dst + 16384 + bb * 8192, map, 64, r0, bar);
             }
-        }
-        // (3) mask, row maximum (of the unscaled scores); a reference that
-        // moves only in steps above 2^8
-        if (!(valid && interior(n0))) {
-            uint64_t keep = 0ull;
-            if (valid) {
-                keep = pt_bits(0, m - n0 + 1);
-                if (!retr) keep &= pt_bits(0, sink - n0) | pt_bits(m - window + 1 - n0, 64);
-            }
-#pragma unroll
-            for (int i = 0; i < 64; ++i)
-                if (!((keep >> i) & 1ull)) s[i] = -INFINITY;
-        }
-        float mx;
-        {
-            float a[22];
-#pragma unroll
-            for (int i = 0; i < 21; ++i) a[i] = fmax3(s[3 * i], s[3 * i + 1], s[3 * i + 2]);
-            a[21] = s[63];
-            float b[8];
-#pragma unroll
-            for (int i = 0; i < 7; ++i) b[i] = fmax3(a[3 * i], a[3 * i + 1], a[3 * i + 2]);
-            b[7] = a[21];
-            mx = fmax3(fmax3(b[0], b[1], b[2]), fmax3(b[3], b[4], b[5]), fmaxf(b[6], b[7])) * SCALE;
-        }
-        float alpha = 1.f;
-        if (mx > m_ref + PT_RESCALE) {
-            alpha = m_ref == -INFINITY ? 1.f : ex2_approx(m_ref - mx);
-            m_ref = mx;
-        }
-        // (4) P V of the previous tile done: P's columns and V_{k-1}'s buffer
-        // are free, O is rescaled if needed; V_{k+1} on its way
-        if (k > 0) {
-            wait_or_abort(&S.o_bar, (uint32_t)(k - 1) & 1u);
+        };
+        auto issue_s = [&](int g, int st) {   // S_g = Q_g K^T of the tile in K stage st
             tc_fence_after();
-            if (__any_sync(0xffffffffu, alpha != 1.f)) {
+            const uint32_t qs = smem_u32(S.q[g]), kb = smem_u32(S.k[st]);
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    float o[64];
-                    tmem_ld64(t_lane + PT_TM_O + 64 * half, o);
+            for (int kk = 0; kk < 8; ++kk)
+                umma_bf16(tbase + 128u * (uint32_t)g, smem_desc(qs + kk * 4096, 2048, 128),
+                          smem_desc_sw128(kb + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024), IDESC, kk > 0);
+            umma_commit(&S.s_full[g]);
+        };
+        bool ok = true;
+        if (leader) {
+            for (int j = 0; j < 2 && j < nt; ++j) {
+                load_tile(&K.tmk, S.k[j], &S.kfull[j], j);
+                load_tile(&K.tmv, S.v[j], &S.vfull[j], j);
+            }
+            ok = pt_wait(&S.q_full, 0u, &S.abort, P);
+            if (ok && nt > 0) ok = pt_wait(&S.kfull[0], 0u, &S.abort, P);
+            if (ok && nt > 0) {
+                issue_s(0, 0);
+                issue_s(1, 0);
+                umma_commit(&S.kempty[0]);
+            }
+        }
+        for (int k = 0; k < nt; ++k) {
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            if (!ok) break;
+            const int st = k & 1, st1 = (k + 1) & 1;
+            // V of tile k + 1 into the stage tile k - 1 used, once its P V are done
+            if (leader && k >= 1 && k + 1 < nt) {
+                ok = pt_wait(&S.vempty[st1], (uint32_t)((k - 1) >> 1) & 1u, &S.abort, P);
+                if (ok) load_tile(&K.tmv, S.v[st1], &S.vfull[st1], k + 1);
+            }
+            // V of tile k landed; on an edge tile the value rows no row of the CTA
+            // may read are zeroed (a cache row may hold anything, and 0 x NaN
+            // would reach O through P = 0)
+            const int n0 = c.tile(k) * PT_TK;
+            const bool edge = n0 + PT_TK - 1 > c.m_hi || (!retr && n0 + PT_TK > c.s_end && n0 < c.w_lo);
+            if (edge) {
+                const bool landed = pt_wait(&S.vfull[st], (uint32_t)(k >> 1) & 1u, &S.abort, P);
+                if (landed) {
+                    const uint32_t vb = smem_u32(S.v[st]);
+                    for (int x = lane; x < 2 * PT_TK; x += 32) {   // (key x / 2, head-dim half x % 2)
+                        if (c.needed(n0 + (x >> 1), window)) continue;
+                        const uint32_t rowa = vb + (uint32_t)((x & 1) * 16384 + (x >> 1) * 128);
 #pragma unroll
-                    for (int i = 0; i < 64; ++i) o[i] *= alpha;
-                    tmem_st64(t_lane + PT_TM_O + 64 * half, o);
+                        for (int i = 0; i < 8; ++i) sts128(rowa + 16 * i, 0u, 0u, 0u, 0u);
+                    }
+                    fence_proxy_async();
+                }
+                __syncwarp();
+                if (!__all_sync(0xffffffffu, landed)) break;
+            }
+            if (leader) {
+                if (!edge && ok) ok = pt_wait(&S.vfull[st], (uint32_t)(k >> 1) & 1u, &S.abort, P);
+                // K of tile k + 1 landed
+                if (ok && k + 1 < nt) ok = pt_wait(&S.kfull[st1], (uint32_t)((k + 1) >> 1) & 1u, &S.abort, P);
+                const uint32_t vb = smem_u32(S.v[st]);
+                for (int g = 0; g < 2 && ok; ++g) {
+                    // O_g += P_g V once the group has written P_g ...
+                    ok = pt_wait(&S.p_full[g], (uint32_t)k & 1u, &S.abort, P);
+                    if (!ok) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        umma_bf16_ts(tbase + 256u + 128u * (uint32_t)g, tbase + 128u * (uint32_t)g + 8u * (uint32_t)kk,
+                                     smem_desc_sw128(vb + kk * 2048, 16384, 1024), IDESC_O, (k > 0 || kk > 0) ? 1u : 0u);
+                    umma_commit(&S.o_done[g]);
+                    // ... then S_g of tile k + 1 over the same columns
+                    if (k + 1 < nt) issue_s(g, st1);
+                }
+                if (ok) {
+                    umma_commit(&S.vempty[st]);
+                    if (k + 1 < nt) umma_commit(&S.kempty[st1]);
+                }
+                // K of tile k + 2 into the stage tile k used (its S MMAs were issued
+                // one tile ago)
+                if (ok && k + 2 < nt) {
+                    ok = pt_wait(&S.kempty[st], (uint32_t)(k >> 1) & 1u, &S.abort, P);
+                    if (ok) load_tile(&K.tmk, S.k[st], &S.kfull[st], k + 2);
                 }
             }
-            if (k + 1 < nt && tid == 0) load_tile(&K.tmv, S.v[(k + 1) & 1], &S.vfull[(k + 1) & 1], k + 1);
         }
-        // (5) P = 2^(s * SCALE - m_ref) as bf16 into tensor memory, row sum
-        // in fp32 (a row with nothing visible yet has m_ref = -inf: P = 0)
+        // never leave with copies or MMAs of this CTA in flight: the softmax
+        // threads wait for the last P V; the copies were all waited for
+    } else {
+        // ================= softmax: row group rg, row `row` (tensor-memory lane)
+        const int rg = warp >> 2, row = tid & 127;
+        const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
+        const uint32_t t_s = tbase + lane_off + 128u * (uint32_t)rg;          // S_g; P_g in its first 64 columns
+        const uint32_t t_o = tbase + lane_off + 256u + 128u * (uint32_t)rg;   // O_g
+        const int u = c.u0 + 8 * rg + row / 16;
+        const int t = u < c.units ? 16 * (P.nt16 - 1 - u / c.nh) + (row & 15) : P.T;
+        const bool valid = u < c.units && t < P.T;
+        const int h = c.g * P.G + P.set_heads[c.set][valid ? u % c.nh : 0];
+        const int m = c.pos_b + t;
+        // Q: this row's 16 chunks (zeros for a row past the units), made
+        // visible to the tensor cores' proxy before the arrival
         {
+            const uint32_t qs = smem_u32(S.q[rg]);
+            if (valid) {
+                const uint8_t* qrow = reinterpret_cast<const uint8_t*>(P.q + (((int64_t)c.b * P.Hq + h) * P.T + t) * D);
+#pragma unroll
+                for (int ch = 0; ch < 16; ++ch) cp_async16(qs + (uint32_t)(ch * 2048 + row * 16), qrow + ch * 16);
+                cp_async_wait_all();
+            } else {
+#pragma unroll
+                for (int ch = 0; ch < 16; ++ch) sts128(qs + (uint32_t)(ch * 2048 + row * 16), 0u, 0u, 0u, 0u);
+            }
+            fence_proxy_async();
+            mbar_arrive(&S.q_full);
+        }
+        constexpr float SCALE = 0.08838834764831845f * 1.4426950408889634f;   // log2(e)/sqrt(128)
+        // a tile with every key visible to every row of the CTA needs no mask
+        auto interior = [&](int n0) {
+            return n0 + PT_TK - 1 <= c.m_lo && (retr || n0 + PT_TK - 1 < sink || n0 > c.m_hi - window);
+        };
+        // the keys n0 + 64 half + i (i < 64) this row may read
+        auto keep_bits = [&](int nh0) -> uint64_t {
+            if (!valid) return 0ull;
+            uint64_t keep = pt_bits(0, m - nh0 + 1);
+            if (!retr) keep &= pt_bits(0, sink - nh0) | pt_bits(m - window + 1 - nh0, 64);
+            return keep;
+        };
+        float m_ref = -INFINITY, l = 0.f;
+        bool ok = true;
+        for (int k = 0; k < nt; ++k) {
+            const int n0 = c.tile(k) * PT_TK;
+            const bool full = valid && interior(n0);
+            // (1) S_k (and the group's previous P V) done
+            if (!(ok = pt_wait(&S.s_full[rg], (uint32_t)k & 1u, &S.abort, P))) break;
+            tc_fence_after();
+            // (2) the row maximum of the unscaled scores, 64 at a time
+            float mx = -INFINITY;
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                float s[64];
+                tmem_ld64(t_s + 64u * (uint32_t)hf, s);
+                if (!full) {
+                    const uint64_t keep = keep_bits(n0 + 64 * hf);
+#pragma unroll
+                    for (int i = 0; i < 64; ++i)
+                        if (!((keep >> i) & 1ull)) s[i] = -INFINITY;
+                }
+                float a[22];
+#pragma unroll
+                for (int i = 0; i < 21; ++i) a[i] = fmax3(s[3 * i], s[3 * i + 1], s[3 * i + 2]);
+                a[21] = s[63];
+                float b[8];
+#pragma unroll
+                for (int i = 0; i < 7; ++i) b[i] = fmax3(a[3 * i], a[3 * i + 1], a[3 * i + 2]);
+                b[7] = a[21];
+                mx = fmax3(mx, fmax3(fmax3(b[0], b[1], b[2]), fmax3(b[3], b[4], b[5]), fmaxf(b[6], b[7])), -INFINITY);
+            }
+            mx *= SCALE;
+            float alpha = 1.f;
+            if (mx > m_ref + PT_RESCALE) {
+                alpha = m_ref == -INFINITY ? 1.f : ex2_approx(m_ref - mx);
+                m_ref = mx;
+            }
+            // (3) O rescaled if the reference moved (the group's previous P V is done)
+            if (k > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll 1
+                for (int half = 0; half < 2; ++half) {
+                    float o[64];
+                    tmem_ld64(t_o + 64 * half, o);
+#pragma unroll
+                    for (int i = 0; i < 64; ++i) o[i] *= alpha;
+                    tmem_st64(t_o + 64 * half, o);
+                }
+            }
+            // (4) P = 2^(s * SCALE - m_ref) as bf16 over the first 64 columns of S,
+            // row sum in fp32 (a row with nothing visible yet has m_ref = -inf: P = 0)
             const float nb = m_ref == -INFINITY ? 0.f : -m_ref;
             const uint64_t sc2 = f2pack(SCALE, SCALE), nb2 = f2pack(nb, nb);
             uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
-            uint32_t w[32];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                float x0, x1;
-                f2unpack(ffma2(f2pack(s[2 * i], s[2 * i + 1]), sc2, nb2), x0, x1);
-                const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-                acc[i & 3] = fadd2(acc[i & 3], f2pack(p0, p1));
-                w[i] = bf16x2(p0, p1);
+            for (int hf = 0; hf < 2; ++hf) {
+                float s[64];
+                tmem_ld64(t_s + 64u * (uint32_t)hf, s);
+                if (!full) {
+                    const uint64_t keep = keep_bits(n0 + 64 * hf);
+#pragma unroll
+                    for (int i = 0; i < 64; ++i)
+                        if (!((keep >> i) & 1ull)) s[i] = -INFINITY;
+                }
+                uint32_t w[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    float x0, x1;
+                    f2unpack(ffma2(f2pack(s[2 * i], s[2 * i + 1]), sc2, nb2), x0, x1);
+                    const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+                    acc[i & 3] = fadd2(acc[i & 3], f2pack(p0, p1));
+                    w[i] = bf16x2(p0, p1);
+                }
+                tmem_st32(t_s + 32u * (uint32_t)hf, w);
             }
             float a0, a1, a2, a3;
             f2unpack(fadd2(acc[0], acc[1]), a0, a1);
             f2unpack(fadd2(acc[2], acc[3]), a2, a3);
             l = l * alpha + ((a0 + a2) + (a1 + a3));
-#ifndef RTP_PT_P_TMEM
-#pragma unroll
-            for (int ch = 0; ch < 8; ++ch)
-                sts128(smem_u32(S.p) + (uint32_t)(ch * 2048 + row * 16), w[4 * ch], w[4 * ch + 1], w[4 * ch + 2], w[4 * ch + 3]);
-#else
-            tmem_st32(t_lane + PT_TM_P, w);
-#endif
+            tc_fence_before();
+            mbar_arrive(&S.p_full[rg]);
         }
-        // (6) O += P V once V_k has landed; on an edge tile the value rows
-        // no row of the CTA may read are zeroed first (a cache row may hold
-        // anything, and 0 x NaN would reach O through P = 0)
-        const bool zero_rows = edge(n0);
-        if (zero_rows) {
-            wait_or_abort(&S.vfull[k & 1], (uint32_t)(k >> 1) & 1u);
-            if (!c.needed(n0 + zr, window)) {
-                const uint32_t rowa = vbuf[k & 1] + (uint32_t)(zb * 8192 + zr * 128);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) sts128(rowa + 16 * i, 0u, 0u, 0u, 0u);
-            }
-        }
-        fence_proxy_async();
-        tc_fence_before();
-        if ((aborted = __syncthreads_or(bad) != 0)) break;
-        if (tid == 0) {
-            if (!zero_rows) wait_or_abort(&S.vfull[k & 1], (uint32_t)(k >> 1) & 1u);
+        // ---- the output of this row, once the group's last P V is done
+        if (ok && nt > 0) {
+            ok = pt_wait(&S.o_done[rg], (uint32_t)(nt - 1) & 1u, &S.abort, P);
             tc_fence_after();
-            const uint32_t vb = vbuf[k & 1];
-#pragma unroll
-            for (int kk = 0; kk < 4 && !bad; ++kk)
-#ifndef RTP_PT_P_TMEM
-                umma_bf16(tbase + PT_TM_O, smem_desc(smem_u32(S.p) + kk * 4096, 2048, 128),
-                          smem_desc_sw128(vb + kk * 2048, 8192, 1024), IDESC_O, (k > 0 || kk > 0) ? 1u : 0u);
-#else
-                umma_bf16_ts(tbase + PT_TM_O, tbase + PT_TM_P + 8 * kk, smem_desc_sw128(vb + kk * 2048, 8192, 1024),
-                             IDESC_O, (k > 0 || kk > 0) ? 1u : 0u);
-#endif
-            umma_commit(&S.o_bar);
         }
-    }
-    cp_async_wait_all();
-    // ---- the output of this thread's row, once the last P V is done
-    if (!aborted && nt > 0) {
-        wait_or_abort(&S.o_bar, (uint32_t)(nt - 1) & 1u);
-        tc_fence_after();
-    }
-    const bool ok = !__syncthreads_or(bad) && !aborted && nt > 0;
-    if (ok) {
-        uint4* orow = reinterpret_cast<uint4*>(P.out + (((int64_t)c.b * P.Hq + h) * P.T + t) * D);
-        const float inv = l > 0.f ? 1.f / l : 0.f;
+        if (ok && nt > 0 && !S.abort) {
+            uint4* orow = reinterpret_cast<uint4*>(P.out + (((int64_t)c.b * P.Hq + h) * P.T + t) * D);
+            const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll 1
+            for (int half = 0; half < 2; ++half) {
+                float o[64];
+                tmem_ld64(t_o + 64 * half, o);
+                if (valid && l > 0.f) {
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            float o[64];
-            tmem_ld64(t_lane + PT_TM_O + 64 * half, o);
-            if (valid && l > 0.f) {
-#pragma unroll
-                for (int i = 0; i < 8; ++i)
-                    orow[8 * half + i] = make_uint4(
-                        bf16x2(o[8 * i] * inv, o[8 * i + 1] * inv), bf16x2(o[8 * i + 2] * inv, o[8 * i + 3] * inv),
-                        bf16x2(o[8 * i + 4] * inv, o[8 * i + 5] * inv), bf16x2(o[8 * i + 6] * inv, o[8 * i + 7] * inv));
+                    for (int i = 0; i < 8; ++i)
+                        orow[8 * half + i] = make_uint4(
+                            bf16x2(o[8 * i] * inv, o[8 * i + 1] * inv), bf16x2(o[8 * i + 2] * inv, o[8 * i + 3] * inv),
+                            bf16x2(o[8 * i + 4] * inv, o[8 * i + 5] * inv), bf16x2(o[8 * i + 6] * inv, o[8 * i + 7] * inv));
+                }
             }
         }
     }

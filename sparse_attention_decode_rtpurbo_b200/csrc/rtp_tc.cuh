@@ -104,17 +104,11 @@ __device__ __forceinline__ void tmem_st64(uint32_t taddr, const float* v) {
         : "memory");
 }
 
-// 16-byte asynchronous copy global -> shared (cp.async, L2 only) and its waits.
+// 16-byte asynchronous copy global -> shared (cp.async, L2 only) and the wait
+// for all of this thread's copies.
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
-// The mbarrier receives this thread's arrival once every cp.async it issued
-// before has landed (no increment of the pending count: the barrier is
-// initialised with one arrival per participating thread).
-__device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
-    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
 
 }  // namespace rtp

@@ -46,16 +46,16 @@ struct RHead {
     float smax, dr, inv_w;
 };
 
-// Per-bin histograms of the select passes in shared memory: a count and the
-// 2^-40 fixed-point mass held as three partial sums, of bits 0-15, 16-31 and
-// 32 up of every token's mass (mass = m[0] + m[1] 2^16 + m[2] 2^32).  All
-// four are 32-bit atomics, which the shared-memory units resolve without
-// retries even when a warp's lanes collide; a partial sum cannot wrap while a
-// bin gathers at most 65536 tokens between flushes.
+// Per-bin histogram of a select pass in shared memory (one head at a time): a
+// count and the 2^-40 fixed-point mass held as three partial sums, of bits
+// 0-15, 16-31 and 32 up of every token's mass (mass = m[0] + m[1] 2^16 +
+// m[2] 2^32).  All four are 32-bit atomics, which the shared-memory units
+// resolve without retries even when a warp's lanes collide; a partial sum
+// cannot wrap while a bin gathers at most 65536 tokens between flushes.
 template <int G>
 struct RHist {
-    uint32_t cnt[G][256];
-    uint32_t m[3][G][256];
+    uint32_t cnt[1][256];   // (one head at a time)
+    uint32_t m[3][1][256];
 };
 constexpr int HIST_FLUSH_TOKENS = 65536;
 
@@ -82,7 +82,7 @@ __device__ __forceinline__ unsigned long long hist_mass(const RHist<G>& H, int h
 
 template <int G>
 struct BSmem {
-    static constexpr int NST = 2;
+    static constexpr int NST = 2;   // attention ring stages of 32 KB (a third measured no faster)
     alignas(1024) uint8_t stage[NST][STAGE_BYTES];
     union {
         AttnScratch<G> X;   // attention phase

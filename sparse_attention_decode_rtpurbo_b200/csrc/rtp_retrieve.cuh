@@ -1129,16 +1129,19 @@ __device__ __noinline__ void clear_call_words(const Params& P) {
     __threadfence();
 }
 
-// The stored scores are dead once the select is done (or was not needed):
-// drop their L2 lines without writing them back (each CTA a slice of every
-// retrieval head's used range).
+// The stored scores, dead when every group was settled in the streaming
+// kernel: drop their L2 lines without writing them back (each CTA a slice of
+// every retrieval head's used range).
 __device__ __forceinline__ void drop_scores(const Params& P, int tid) {
     for (int bs = 0; bs < P.B * P.n_ret; ++bs) {
         const int L = __ldg(P.seq_lens + bs / P.n_ret);
         if (!seq_ok(P, L)) continue;
         const char* base = reinterpret_cast<const char*>(P.scores + (int64_t)bs * P.sstride);
         const int nlines = (L * 4 + 127) / 128;
-        for (int x = blockIdx.x * THREADS + tid; x < nlines; x += gridDim.x * THREADS)
+        // the CTAs in a rotated order per head, so a head shorter than the grid's
+        // threads does not always fall to the same first CTAs
+        const int rb = (int)(((long long)blockIdx.x + (long long)bs * 37) % gridDim.x);
+        for (int x = rb * THREADS + tid; x < nlines; x += gridDim.x * THREADS)
             asm volatile("discard.global.L2 [%0], 128;" ::"l"(base + (int64_t)x * 128) : "memory");
     }
 }
@@ -1276,6 +1279,13 @@ __device__ __forceinline__ void r_body(const KParams& K, bool single) {
         ok = gsync();
     }
     if (tid == 0) trace_max(P, 3);
+    // The stored scores are dead from here on.  Without attention work they
+    // are dropped from L2 (no write-back of lines that are still there).  With
+    // attention work they are left: its K/V loads evict them anyway, and the
+    // drop measured 11-18 us on the step's critical path at 4 x 128K, wherever
+    // it was put (the discards block their thread), against ~5 us of
+    // write-back bandwidth for those 32 MB during the attention.
+    if (!work) drop_scores(P, tid);
     if (ok && work) {
         // ---- block-sparse attention over every group's block list
         const int ngroups = P.B * P.n_rg;
@@ -1296,7 +1306,6 @@ __device__ __forceinline__ void r_body(const KParams& K, bool single) {
         if (tid == 0) trace_max(P, 4);
     }
     if (tid == 0) acct_flush(P, S.acct);
-    if (ok || !work) drop_scores(P, tid);
     // the last CTA out clears the call's coordination words (none was set
     // when every group was settled in the streaming kernel: no count then,
     // except for the single launch's transition barrier)

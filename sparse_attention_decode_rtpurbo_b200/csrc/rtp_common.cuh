@@ -52,12 +52,11 @@ struct HeadState {
 // Coordination words of one call (workspace; zero between calls).
 struct Sync {
     uint32_t n_radix_heads;    // heads needing the exact select (list in rlist)
-    uint32_t n_radix_groups;   // (b, group) pairs holding such heads (list in rglist)
     uint32_t barrier;          // grid barrier arrivals of the retrieval kernel
     uint32_t exit_count;
     uint32_t kb_work;          // groups left to the retrieval kernel (a select, or blocks to attend)
     uint32_t n_decided;        // (b, group) pairs decided so far (a count the single launch waits for)
-    uint32_t pad[17];
+    uint32_t pad[18];
 };
 
 // Head split (host-derived): retrieval groups (KV heads with >= 1 retrieval
@@ -99,7 +98,7 @@ struct Params {
     // workspace
     uint32_t* status;
     Sync* sync;
-    uint32_t *rlist, *rglist;
+    uint32_t* rlist;
     uint32_t *tick_score, *tick_local, *tick_ret;
     uint32_t* tick_grp;   // [B * n_rg] radix heads of the group done with their select (zero between calls)
     // the exact select's per-head global state (zero between calls): merged

@@ -34,7 +34,7 @@ struct Plan {
     uint8_t slot_head[MAX_HQ], slot_rg[MAX_HQ];
     // workspace byte offsets; [0, zero_end) must be zero when a call starts
     size_t o_status, o_sync, o_tick_score, o_tick_local, o_tick_ret, o_tick_grp, o_agg, o_sel_cnt, o_sel_mass, o_sel_ncand, o_sel_above, o_sel_arrive, zero_end;
-    size_t o_rlist, o_rglist, o_hs, o_tie_cnt, o_scores, o_cand, o_bitmap, o_blist, o_bcount, o_lpart, o_rpart, total;
+    size_t o_rlist, o_hs, o_tie_cnt, o_scores, o_cand, o_bitmap, o_blist, o_bcount, o_lpart, o_rpart, total;
 };
 
 static size_t align_up(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -126,7 +126,6 @@ static rtp_status make_plan(const rtp_dims* d, const uint8_t* head_kind, int win
     pl->o_sel_arrive = take(BR * 2 * 4);
     pl->zero_end = o;
     pl->o_rlist = take(BR * 4);
-    pl->o_rglist = take(BG * 4);
     pl->o_hs = take(BR * sizeof(HeadState));
     pl->o_tie_cnt = take(BR * pl->ntiles_cap * 4);
     pl->o_scores = take(BR * (size_t)pl->ntiles_cap * SROWS * 4);
@@ -419,7 +418,6 @@ static rtp_status decode_step_ws(const rtp_dims* dims, const uint16_t* q_pre, co
     P.status = (uint32_t*)(ws + pl.o_status);
     P.sync = (Sync*)(ws + pl.o_sync);
     P.rlist = (uint32_t*)(ws + pl.o_rlist);
-    P.rglist = (uint32_t*)(ws + pl.o_rglist);
     P.tick_score = (uint32_t*)(ws + pl.o_tick_score);
     P.tick_local = (uint32_t*)(ws + pl.o_tick_local);
     P.tick_ret = (uint32_t*)(ws + pl.o_tick_ret);

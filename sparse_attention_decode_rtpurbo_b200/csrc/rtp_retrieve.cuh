@@ -1108,7 +1108,6 @@ __device__ __forceinline__ void r_setup(const Params& P, int tid) {
 // select it may have left).
 __device__ __noinline__ void clear_call_words(const Params& P) {
     P.sync->n_radix_heads = 0;
-    P.sync->n_radix_groups = 0;
     P.sync->barrier = 0;
     P.sync->kb_work = 0;
     if (__ldcg(P.status) != 0) {

@@ -455,8 +455,6 @@ __device__ __forceinline__ void decide_group_body(const KParams& K, ASmem<G>& S,
                     const uint32_t kx = atomicAdd(&P.sync->n_radix_heads, 1u);
                     P.rlist[kx] = ((uint32_t)b << 16) | (uint32_t)(slot0 + hh);
                 }
-            const uint32_t gi = atomicAdd(&P.sync->n_radix_groups, 1u);
-            P.rglist[gi] = ((uint32_t)b << 16) | (uint32_t)rg;
             atomicAdd(&P.sync->kb_work, 1u);
         }
         return;

@@ -421,7 +421,7 @@ __device__ __noinline__ void combine_splits(AttnScratch<G>& X, const float* part
     }
     consumer_sync();
     if (in_smem) {
-        constexpr int U = G >= 8 ? 4 : 8;   // parts per batch (registers)
+        constexpr int U = G >= 8 ? 8 : 16;   // parts per batch: 64 loads in flight per thread
         float acc[G];
 #pragma unroll
         for (int h = 0; h < G; ++h) acc[h] = 0.f;

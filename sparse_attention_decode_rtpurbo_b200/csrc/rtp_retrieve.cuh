@@ -275,11 +275,17 @@ __device__ __noinline__ void h_pass(const Params& P, int b, int slot, const RHea
         uint32_t w0 = 0u;        // RP_COMPACT / RP_MARK: bits of blocks n0/64 + 0..15
         uint32_t n_above = 0u;   // RP_COMPACT: the warp's tokens above the threshold bin (lane 0)
         uint32_t tcount = 0u;    // RP_TIES: threshold ties of this thread in the tile
+        uint32_t in_bin[HS_U];   // RP_COMPACT: the warp's ballots of tokens in the threshold bin
+        // the thread's scores of the copy into registers first: the loads then
+        // overlap, where the shared-memory atomics below would keep them in order
+        float xv[HS_U];
+#pragma unroll
+        for (int u = 0; u < HS_U; ++u) xv[u] = x[tid + u * CONSUMERS];
 #pragma unroll
         for (int u = 0; u < HS_U; ++u) {
             const int r = tid + u * CONSUMERS;
             const bool ok = r < nv;
-            const float v = x[r];
+            const float v = xv[u];
             const uint32_t key = f2key(v);
             if constexpr (pass == RP_BINS) {
                 if (ok) {
@@ -303,18 +309,7 @@ __device__ __noinline__ void h_pass(const Params& P, int b, int slot, const RHea
                 if constexpr (pass == RP_COMPACT) {
                     const uint32_t bn = ok ? score_bin(v, rh.smax, rh.dr, rh.inv_w) : 256u;
                     keep = bn < rh.bstar;
-                    // the bin's tokens, in ballot order behind one reservation per warp
-                    const uint32_t bal = __ballot_sync(0xffffffffu, bn == rh.bstar);
-                    if (bal) {
-                        uint32_t base = 0;
-                        if (lane == 0)
-                            base = unit_of_many ? atomicAdd(P.sel_ncand + bs, (uint32_t)__popc(bal))
-                                                : atomicAdd(&S.hcand, (uint32_t)__popc(bal));
-                        base = __shfl_sync(0xffffffffu, base, 0);
-                        const uint32_t pos = base + __popc(bal & ((1u << lane) - 1u));
-                        if (bn == rh.bstar && pos < (uint32_t)CAND_CAP)
-                            cand[pos] = ((unsigned long long)key << 32) | (uint32_t)(n0 + r);
-                    }
+                    in_bin[u] = __ballot_sync(0xffffffffu, bn == rh.bstar);
                 } else {
                     keep = ok && (key > rh.tau || (key == rh.tau && (uint32_t)(n0 + r) <= rh.tie_idx));
                 }
@@ -322,6 +317,29 @@ __device__ __noinline__ void h_pass(const Params& P, int b, int slot, const RHea
                 const uint32_t kb = __ballot_sync(0xffffffffu, keep);
                 if (kb) w0 |= 1u << (2 * u + (warp >> 1));
                 n_above += __popc(kb);
+            }
+        }
+        if constexpr (pass == RP_COMPACT) {
+            // the bin's tokens of the copy, in ballot order behind one
+            // reservation per warp (a returning global atomic per 32 tokens
+            // would put its round trip on the loop's path HS_U times)
+            uint32_t tot = 0u;
+#pragma unroll
+            for (int u = 0; u < HS_U; ++u) tot += (uint32_t)__popc(in_bin[u]);
+            if (tot) {
+                uint32_t base = 0;
+                if (lane == 0)
+                    base = unit_of_many ? atomicAdd(P.sel_ncand + bs, tot) : atomicAdd(&S.hcand, tot);
+                base = __shfl_sync(0xffffffffu, base, 0);
+#pragma unroll
+                for (int u = 0; u < HS_U; ++u) {
+                    const uint32_t pos = base + (uint32_t)__popc(in_bin[u] & ((1u << lane) - 1u));
+                    if (((in_bin[u] >> lane) & 1u) && pos < (uint32_t)CAND_CAP) {
+                        const int r = tid + u * CONSUMERS;
+                        cand[pos] = ((unsigned long long)f2key(xv[u]) << 32) | (uint32_t)(n0 + r);
+                    }
+                    base += (uint32_t)__popc(in_bin[u]);
+                }
             }
         }
         if constexpr (pass == RP_COMPACT || pass == RP_MARK) {
